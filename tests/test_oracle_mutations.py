@@ -1,0 +1,95 @@
+"""Planted mistakes: each test patches a plausible bug into the oracle (on the CPU
+only) and checks that one of the pins catches it. This shows the pins cover every
+part of the oracle."""
+
+import json
+import os
+
+import numpy as np
+import pytest
+
+from oracle import nvfp4 as F
+from oracle import verify as V
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _hand_blocks_pass():
+    with open(os.path.join(GOLDEN, "hand_blocks.json")) as f:
+        g = json.load(f)
+    W = np.array(g["W"], dtype=np.float32)
+    for case in g["cases"]:
+        q, sf, ts = F.quantize_nvfp4(W, case["tensor_scale_in"])
+        if float(ts) != case["ts"] or sf.tolist() != case["sf"] or q.tolist() != case["q"]:
+            return False
+    return True
+
+
+def test_baseline_passes():
+    assert _hand_blocks_pass()
+
+
+def test_swapped_nibbles_caught(monkeypatch):
+    monkeypatch.setattr(F, "pack_codes", lambda c: (np.asarray(c)[:, 1::2] & 0xF) | ((np.asarray(c)[:, 0::2] & 0xF) << 4))
+    assert not _hand_blocks_pass()
+
+
+def test_ties_away_from_zero_caught(monkeypatch):
+    def bad(a):
+        a = np.minimum(np.asarray(a, dtype=np.float64), 6.0)
+        _, ex = np.frexp(a)
+        e = np.maximum(ex - 1, 0) - 1
+        return np.minimum(np.ldexp(np.floor(np.ldexp(a, -e) + 0.5), e), 6.0)
+    monkeypatch.setattr(F, "e2m1_round_magnitude", bad)
+    assert not _hand_blocks_pass()
+
+
+def test_unrounded_block_scale_caught(monkeypatch):
+    orig = F.e4m3_encode
+    # plant: use the unrounded quotient for the element codes by rounding the scale toward zero
+    def bad(v):
+        v = np.asarray(v, dtype=np.float64)
+        c = orig(v)
+        down = np.maximum(c.astype(np.int32) - 1, 0).astype(np.uint8)
+        return np.where(F.E4M3_VALUES[c] > v, down, c)
+    monkeypatch.setattr(F, "e4m3_encode", bad)
+    assert not _hand_blocks_pass()
+
+
+def test_absolute_block_scale_reading_caught(monkeypatch):
+    """The literal reading S = amax/6 (ignoring ts) gives different scale bytes."""
+    orig = F.quantize_codes
+    def bad(W, tensor_scale_in=None):
+        codes, sf, ts = orig(W, tensor_scale_in)
+        amax_b = np.abs(np.asarray(W, np.float64)).reshape(W.shape[0], -1, 16).max(axis=2)
+        return codes, F.e4m3_encode(amax_b / 6.0), ts
+    monkeypatch.setattr(F, "quantize_codes", bad)
+    assert not _hand_blocks_pass()
+
+
+def test_dropped_sign_caught(monkeypatch):
+    orig = F.e2m1_encode
+    monkeypatch.setattr(F, "e2m1_encode", lambda r: orig(np.abs(r)))
+    assert not _hand_blocks_pass()
+
+
+def test_dropped_tensor_scale_in_dequant_caught():
+    q, sf, ts = F.quantize_nvfp4(np.array([[6.0] + [1.0] * 15], np.float32), 2.0 ** -4)
+    good = F.dequantize_nvfp4(q, sf, ts)
+    bad = F.dequantize_nvfp4(q, sf, 1.0)
+    assert not np.array_equal(good, bad)
+    assert good[0, 0] == 6.0                           # the round-trip pin holds only with ts applied
+
+
+def test_accept_off_by_one_caught():
+    t = np.array([1, 2, 3])
+    d = np.array([[1, 9]])
+    assert V.accept_ref(t, d, 2).tolist() == [1]
+    bad = lambda t, d, D: np.array([min(D, V.accept_ref(t, d, D)[0] + 1)])
+    assert bad(t, d, 2).tolist() != [1]
+
+
+def test_last_index_argmax_caught():
+    y = np.array([[1.0, 3.0, 3.0]])
+    last = y.shape[1] - 1 - np.argmax(y[:, ::-1], axis=1)
+    assert last.tolist() != V.argmax_ref(y).tolist()
