@@ -1,0 +1,453 @@
+#!/usr/bin/env python3
+"""Benchmark: weight GB/s and % of the B200 HBM roofline for one 27B weight pass.
+
+Step = one pass of the whole hot path over resident synthetic weights:
+  64 layers x {gate+up 5120->34816, down 17408->5120, qkv 5120->10240} NVFP4 GEMMs
+  followed by the fused lm_head verify (5120->248,320 rows, argmax + accept length).
+The headline is M = 17 (16 drafted tokens + 1). M = 1 (plain decode) and M = 68
+(4 sequences x 17 sharing one read) are reported in ``per_m``. Each pass is
+captured as two CUDA graphs (the 192 GEMMs, then the verify) and replayed; CUDA
+events on the launching stream bracket both. The weight stack (11.5 GB) is far
+larger than L2, so no flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With --gpus N > 1 (under torchrun) every rank runs its own replica of the pass
+on its own GPU. There is no data-path collective, ``scaling`` is weak, and value
+is the sum over ranks, taken over the max-over-ranks time.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic as S  # noqa: E402
+
+BYTES_PER_WEIGHT = 0.5 + 1.0 / 16.0          # E2M1 nibble + E4M3 scale per 16
+METRIC = "weight GB/s and % of B200 HBM roofline per 27B weight pass at M=1/17/68"
+WORKLOAD = ("27B weight pass: 64 x {gate_up 5120->34816, down 17408->5120, qkv 5120->10240} NVFP4 GEMMs "
+            "+ lm_head verify 5120->248320 (argmax + accept)")
+
+
+def weight_bytes(N: int, K: int) -> int:
+    return N * K // 2 + N * K // 16
+
+
+def stack_weight_bytes() -> int:
+    return S.N_LAYERS * sum(weight_bytes(N, K) for (K, N) in (S.LAYER_SHAPES[n] for n in S.LAYER_ORDER))
+
+
+def lmhead_weight_bytes() -> int:
+    return weight_bytes(S.VOCAB, S.LMHEAD_K)
+
+
+def gemm_alg_bytes(M: int) -> int:
+    """Algorithmic bytes of the 192 GEMMs of one pass: W + scales + X (bf16) + Y (fp32)."""
+    total = 0
+    for name in S.LAYER_ORDER:
+        K, N = S.LAYER_SHAPES[name]
+        total += weight_bytes(N, K) + M * K * 2 + M * N * 4
+    return S.N_LAYERS * total
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines: list[str] = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def build_pass(nv, torch, dev, M_list, rank: int):
+    """Pack the 192-matrix stack and the lm_head on the GPU; make inputs for every M."""
+    stack = []
+    for layer in range(S.N_LAYERS):
+        for j, name in enumerate(S.LAYER_ORDER):
+            K, N = S.LAYER_SHAPES[name]
+            g = torch.Generator(device=dev)
+            g.manual_seed(1000 * layer + j + 1_000_003 * rank)
+            W = torch.randn(N, K, generator=g, device=dev, dtype=torch.float32).mul_(S.W_STD)
+            q, sf, ts = nv.pack(W)
+            del W
+            stack.append((name, K, N, q, sf, ts))
+    g = torch.Generator(device=dev)
+    g.manual_seed(S.LMHEAD_W_SEED + 1_000_003 * rank)
+    W = torch.randn(S.VOCAB, S.LMHEAD_K, generator=g, device=dev, dtype=torch.float32).mul_(S.W_STD)
+    lm = nv.pack(W)
+    del W
+    torch.cuda.synchronize()
+    return stack, lm
+
+
+class Pass:
+    """One M: per-layer X, outputs, workspaces, drafts, and the two captured graphs."""
+
+    def __init__(self, nv, torch, dev, stack, lm, M: int, rank: int):
+        self.M = M
+        self.torch = torch
+        self.B = max(1, M // (S.DRAFT_LEN + 1)) if M >= S.DRAFT_LEN + 1 else 1
+        self.D = M // self.B - 1
+        assert self.B * (self.D + 1) == M
+        g = torch.Generator(device=dev)
+        g.manual_seed(7 + M + 1_000_003 * rank)
+        # one device buffer holds every per-layer X (plus the lm_head X) so one copy refreshes them all
+        sizes = [M * K for (_, K, _, _, _, _) in stack] + [M * S.LMHEAD_K]
+        self.x_all = torch.randn(sum(sizes), generator=g, device=dev).to(torch.bfloat16)
+        self.xs, off = [], 0
+        for n in sizes:
+            self.xs.append(self.x_all[off: off + n])
+            off += n
+        self.ys = [torch.empty((M, N), dtype=torch.float32, device=dev) for (_, _, N, _, _, _) in stack]
+        wsb = max(nv.gemm_workspace_bytes(M, N, K) for (_, K, N, _, _, _) in stack)
+        self.gws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
+        self.vws = torch.empty(max(nv.verify_workspace_bytes(M, S.VOCAB, S.LMHEAD_K), 16), dtype=torch.uint8,
+                               device=dev)
+        self.argmax = torch.empty(M, dtype=torch.int32, device=dev)
+        self.accept = torch.empty(self.B, dtype=torch.int32, device=dev)
+        self.vmax = torch.empty(M, dtype=torch.float32, device=dev)
+        self.stack, self.lm, self.nv = stack, lm, nv
+        # drafts: the target's own greedy tokens for a prefix L* ~ U{0..D}, then random ids
+        self.drafts = torch.zeros((self.B, self.D), dtype=torch.int32, device=dev)
+        self.verify_call()
+        torch.cuda.synchronize()
+        t = self.argmax.cpu().numpy()
+        Lstar = np.random.default_rng(S.LMHEAD_L_SEED + M).integers(0, self.D + 1, size=self.B)
+        d = S.drafts_with_prefix(t, Lstar, self.D, S.VOCAB)
+        self.drafts.copy_(torch.from_numpy(d))
+        self.Lstar = Lstar
+
+    def gemm_calls(self):
+        nv, M = self.nv, self.M
+        for i, (name, K, N, q, sf, ts) in enumerate(self.stack):
+            X = self.xs[i].view(M, K)
+            nv.gemm(X, q, sf, ts, out=self.ys[i], workspace=self.gws)
+
+    def verify_call(self):
+        q, sf, ts = self.lm
+        X = self.xs[-1].view(self.M, S.LMHEAD_K)
+        self.nv.verify(X, q, sf, ts, self.drafts, workspace=self.vws, out=(self.argmax, self.accept, self.vmax))
+
+    def capture(self):
+        torch = self.torch
+        lib = self.nv.lib()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):           # warm both paths outside capture
+            self.gemm_calls()
+            self.verify_call()
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        n0 = lib.nvfp4ws_kernel_launches()
+        self.g_gemm = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.g_gemm):
+            self.gemm_calls()
+        n1 = lib.nvfp4ws_kernel_launches()
+        self.g_verify = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.g_verify):
+            self.verify_call()
+        n2 = lib.nvfp4ws_kernel_launches()
+        self.launches_gemm, self.launches_verify = n1 - n0, n2 - n1
+        torch.cuda.synchronize()
+
+    def run_timed(self, steps: int):
+        torch = self.torch
+        st = torch.cuda.current_stream()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        for k in range(steps):
+            ev[k][0].record(st)
+            self.g_gemm.replay()
+            ev[k][1].record(st)
+            self.g_verify.replay()
+            ev[k][2].record(st)
+        torch.cuda.synchronize()
+        gemm_ms = np.array([ev[k][0].elapsed_time(ev[k][1]) for k in range(steps)])
+        ver_ms = np.array([ev[k][1].elapsed_time(ev[k][2]) for k in range(steps)])
+        total_ms = ev[0][0].elapsed_time(ev[-1][2])
+        return total_ms, gemm_ms, ver_ms
+
+    def run_e2e(self, steps: int, x_host, out_host):
+        """Host buffers: copy every input in (pinned -> device) and the verify result out, each step."""
+        torch = self.torch
+        st = torch.cuda.current_stream()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        for _ in range(steps):
+            self.x_all.copy_(x_host, non_blocking=True)
+            self.g_gemm.replay()
+            self.g_verify.replay()
+            out_host[0][: self.M].copy_(self.argmax, non_blocking=True)
+            out_host[1][: self.B].copy_(self.accept, non_blocking=True)
+        e1.record(st)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1)
+
+
+def cpu_baseline(seconds: float = 12.0):
+    """The oracle, as it stands, on a bounded sample: dequant + float64 GEMM of the
+    qkv matrix (5120->10240) at M=17, repeated until ``seconds`` have passed."""
+    from oracle import gemm as G
+    from oracle import nvfp4 as F
+    W, x = S.layer("qkv", M=17)
+    q, sf, ts = F.quantize_nvfp4(W)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        G.gemm_ref(x, q, sf, ts)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    K, N = S.LAYER_SHAPES["qkv"]
+    gbs = reps * weight_bytes(N, K) / el / 1e9
+    try:
+        from threadpoolctl import threadpool_info
+        blas = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        blas = None
+    cores = len(os.sched_getaffinity(0))
+    return {"value": gbs, "unit": "GB/s", "cores": blas or cores, "kind": "oracle",
+            "sample": f"{reps} x (dequantise + float64 GEMM) of qkv 5120->10240 at M=17, {el:.1f} s; "
+                      f"host has {cores} cores, BLAS threads {blas}"}
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import nvfp4_weight_streaming_gemm_b200 as nv
+    from nvfp4_weight_streaming_gemm_b200 import build as nvbuild
+    nvbuild.build()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    M_list = [int(m) for m in args.ms.split(",")]
+    stack, lm = build_pass(nv, torch, dev, M_list, rank)
+    passes = {M: Pass(nv, torch, dev, stack, lm, M, rank) for M in M_list}
+    for p in passes.values():
+        p.capture()
+        for _ in range(args.warmup):
+            p.g_gemm.replay()
+            p.g_verify.replay()
+    torch.cuda.synchronize()
+
+    wbytes = stack_weight_bytes() + lmhead_weight_bytes()
+    peak, peak_kind = measured_peaks()
+    results, clocks = {}, None
+    head = 17 if 17 in passes else M_list[0]
+    for M, p in passes.items():
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        sampler = ClockSampler(local_rank) if (M == head and rank == 0) else None
+        if sampler:
+            sampler.start()
+        total_ms, gemm_ms, ver_ms = p.run_timed(args.steps)
+        if sampler:
+            clocks = sampler.stop()
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        if dist:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+        ms = total_ms / args.steps
+        gemm_avg = float(gemm_ms.mean())
+        results[M] = {
+            "ms_per_pass": ms,
+            "weight_gbs": world * wbytes / (ms * 1e-3) / 1e9,
+            "pct_of_8tbs": 100.0 * wbytes / (ms * 1e-3) / 8e12,
+            "passes_per_s": world * 1e3 / ms,
+            "gemm_ms": gemm_avg,
+            "gemm_gbs_alg": gemm_alg_bytes(M) / (gemm_avg * 1e-3) / 1e9,
+            "gemm_weight_gbs": stack_weight_bytes() / (gemm_avg * 1e-3) / 1e9,
+            "verify_ms": float(ver_ms.mean()),
+            "verify_weight_gbs": lmhead_weight_bytes() / (float(ver_ms.mean()) * 1e-3) / 1e9,
+            "launches_per_pass": p.launches_gemm + p.launches_verify,
+            "B": p.B, "D": p.D,
+        }
+
+    # end to end through the public API with host buffers (headline M)
+    p = passes[head]
+    x_host = torch.empty(p.x_all.numel(), dtype=torch.bfloat16, pin_memory=True)
+    x_host.copy_(p.x_all.cpu())
+    out_host = (torch.empty(p.M, dtype=torch.int32, pin_memory=True),
+                torch.empty(p.B, dtype=torch.int32, pin_memory=True))
+    for _ in range(args.warmup):
+        p.run_e2e(1, x_host, out_host)
+    if dist:
+        dist.barrier()
+    e2e_ms = p.run_e2e(args.steps, x_host, out_host)
+    t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if dist:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_ms = float(t.item()) / args.steps
+    h2d = p.x_all.numel() * 2
+    d2h = p.M * 4 + p.B * 4
+
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    r = results[head]
+    line = {
+        "metric": METRIC,
+        "value": r["weight_gbs"],
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": r["ms_per_pass"],
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e2m1*e4m3 weights x f16 activations -> f32 accumulate",
+        "data": "synthetic (seeded N(0,0.02) weights packed on the GPU, N(0,1) bf16 activations)",
+        "config": {"workload": WORKLOAD, "M": head, "B": r["B"], "D": r["D"], "layers": S.N_LAYERS,
+                   "weight_bytes_per_pass": wbytes, "l2": "inputs larger than L2 (11.5 GB weight stack, no flush)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "pct_of_8tbs": r["pct_of_8tbs"],
+        "passes_per_s": r["passes_per_s"],
+        "decode_steps_per_s": r["passes_per_s"],
+        "per_m": {str(M): {k: (round(v, 4) if isinstance(v, float) else v) for k, v in res.items()}
+                  for M, res in results.items()},
+        "roofline": {"bound": "hbm", "kernel": "GEMM launches of the pass (192 per pass)",
+                     "achieved": r["gemm_gbs_alg"], "peak": peak, "unit": "GB/s",
+                     "frac": r["gemm_gbs_alg"] / peak, "peak_kind": peak_kind, "traffic": args.traffic},
+        "e2e": {"value": world * wbytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": r["launches_per_pass"] * args.steps,
+        "clocks": clocks,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args, rank, world):
+    """The CPU oracle timed as it stands: each step dequantises and multiplies one qkv
+    matrix (5120->10240) in float64 at M=17. That is a bounded sample of the pass, in
+    the same unit (weight GB/s)."""
+    if rank != 0:
+        return
+    from oracle import gemm as G
+    from oracle import nvfp4 as F
+    W, x = S.layer("qkv", M=17)
+    q, sf, ts = F.quantize_nvfp4(W)
+    for _ in range(args.warmup):
+        G.gemm_ref(x, q, sf, ts)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        G.gemm_ref(x, q, sf, ts)
+    el = time.perf_counter() - t0
+    K, N = S.LAYER_SHAPES["qkv"]
+    gbs = args.steps * weight_bytes(N, K) / el / 1e9
+    cores = len(os.sched_getaffinity(0))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD + " -- sampled: one qkv matrix per step", "M": 17},
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": "one qkv 5120->10240 dequant + float64 GEMM at M=17 per step"},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--ms", default="17,1,68", help="comma list of M; the first 17 (else the first) is the headline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="DRAM bytes per GEMM pass from an ncu capture (reported as roofline.traffic)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

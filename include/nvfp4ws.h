@@ -1,0 +1,210 @@
+/*
+ * nvfp4ws.h -- C ABI of libnvfp4ws.so: NVFP4 weight-streaming skinny GEMM and
+ * fused greedy verify for NVIDIA B200 (sm_100a).
+ *
+ * The operation comes from these web pages, cited by title and section:
+ *   - "Qwen3.8 on DGX Spark (GB10)", "The seven targets, and switching between
+ *     them": the weights are NVFP4 group-16.
+ *   - The same page, introduction: the target verifies drafted tokens over the
+ *     full 248,320-row vocabulary; the draft head may be a 65,536-row slice.
+ *   - "TandemLLM", introduction: accept drafted tokens up to the first one the
+ *     target disagrees with, then emit the target's own token (greedy verify).
+ *     The same paragraph gives the one-ulp near-tie caveat.
+ *   - "TandemLLM", "How it works": one decode step reads every weight once.
+ *   - "ling-engine", introduction: 16 drafted tokens per step, and 2-4 sequences
+ *     that share one weight read.
+ *
+ * Conventions common to every entry point
+ *   - Pointers. All tensor pointers are DEVICE pointers unless a comment says
+ *     otherwise. The caller owns every buffer. The library never allocates
+ *     device or host memory.
+ *   - Layouts. All layouts are row-major and dense (leading dimension = row
+ *     length).
+ *   - Asynchrony. Work is enqueued on `stream` (NULL = the legacy default
+ *     stream) and runs asynchronously. The call returns once it is enqueued.
+ *   - Validation. Argument checks are synchronous, on the host, and enqueue
+ *     nothing when they fail. The return value is an nvfp4ws_status; the last
+ *     error text of the calling thread is available from nvfp4ws_last_error().
+ *   - Errors. A launch failure returns NVFP4WS_ERR_CUDA. No C++ exception
+ *     crosses this interface.
+ *   - Device errors. Kernels that wait for other CTAs give up after a bounded
+ *     number of polls and record a code in a device error word. The
+ *     next call of nvfp4ws_check() reports it.
+ *   - Threads. The entry points are reentrant. Concurrent calls must not share
+ *     a workspace.
+ */
+#ifndef NVFP4WS_H_
+#define NVFP4WS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream (cudaStream_t / CUstream). Kept opaque so this header needs no CUDA header. */
+typedef void* nvfp4ws_stream_t;
+
+typedef enum {
+  NVFP4WS_OK = 0,
+  NVFP4WS_ERR_INVALID_ARG = 1,    /* null pointer, bad size or bad enum value */
+  NVFP4WS_ERR_UNSUPPORTED = 2,    /* shape outside what the kernels support (e.g. K % 32 != 0, M > 256) */
+  NVFP4WS_ERR_MISALIGNED = 3,     /* a pointer does not have the alignment the call requires */
+  NVFP4WS_ERR_WORKSPACE = 4,      /* workspace missing or smaller than the *_workspace_bytes query */
+  NVFP4WS_ERR_CUDA = 5,           /* a CUDA runtime call or kernel launch failed */
+  NVFP4WS_ERR_DEVICE_TIMEOUT = 6  /* a bounded device-side wait gave up (see nvfp4ws_check) */
+} nvfp4ws_status;
+
+/* Output element type of nvfp4_gemm_skinny. */
+typedef enum { NVFP4WS_Y_F32 = 0, NVFP4WS_Y_BF16 = 1 } nvfp4ws_ydtype;
+
+/* Kernel path of the GEMM. AUTO picks by M (the tuned crossover). The others force a path. */
+typedef enum {
+  NVFP4WS_PATH_AUTO = 0,
+  NVFP4WS_PATH_GEMV = 1,          /* CUDA-core streaming GEMV: dequantises in registers */
+  NVFP4WS_PATH_MMA = 2            /* tcgen05 tensor-core path: TMA-staged, TMEM accumulators */
+} nvfp4ws_path;
+
+/* Human-readable name of a status code. Never NULL. Static storage. */
+const char* nvfp4ws_status_string(int status);
+
+/* Detail text of the last failing call on this host thread ("" if none). Thread-local storage. */
+const char* nvfp4ws_last_error(void);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int nvfp4ws_version(void);
+
+/* Largest M (rows of X) accepted by the GEMM and verify entry points. */
+#define NVFP4WS_MAX_M 256
+
+/*
+ * nvfp4_pack -- quantise an fp32 weight to NVFP4 (two-level scaling) and pack it.
+ *
+ * Passage: "Qwen3.8 on DGX Spark (GB10)", "The seven targets ...": NVFP4
+ * group-16. The pages give no bit-level definition. This library reads it as:
+ *   ts   = fp32( amax(|W|) / (6 * 448) )                    per tensor
+ *   S    = E4M3_rne_satfinite( amax(|block|) / (6 * ts) )    per 16 consecutive k
+ *   code = E2M1_rne_satfinite( w / (S * ts) )                per element; sign kept
+ * Both quotients are formed in float64 and rounded once (ties to even). If
+ * ts == 0 or S == 0, the affected codes are +0.
+ *
+ * Arguments
+ *   W               fp32 [N, K] row-major, device, 16-byte aligned. Read only.
+ *   N, K            N >= 1, K >= 16, K % 16 == 0.
+ *   q               out: uint8 [N, K/2], device. Byte (n, j) holds code(n, 2j) in
+ *                   bits 0..3 and code(n, 2j+1) in bits 4..7.
+ *   sf              out: uint8 [N, K/16], device. E4M3 bits of each block scale.
+ *   tensor_scale    out: fp32 [1], device. The ts used.
+ *   tensor_scale_in in: fp32 [1], device, or NULL. When non-NULL, this ts is used
+ *                   instead of amax/2688, and copied to tensor_scale.
+ * Returns NVFP4WS_OK, or INVALID_ARG / MISALIGNED / CUDA.
+ */
+int nvfp4_pack(const float* W, int64_t N, int64_t K, uint8_t* q, uint8_t* sf,
+               float* tensor_scale, const float* tensor_scale_in, nvfp4ws_stream_t stream);
+
+/*
+ * nvfp4_gemm_workspace_bytes -- device workspace needed by nvfp4_gemm_skinny for
+ * this shape (0 when none is needed). Pass at least this many bytes.
+ */
+size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/*
+ * nvfp4_gemm_skinny -- Y[M, N] = X[M, K] . dequant(W)[N, K]^T.
+ *
+ * Passage: "TandemLLM", "How it works" (each step reads every weight once, at
+ * NVFP4), and the veloGB10 page, "Unique aspects: Engineered to the roofline"
+ * (the pass is weight-bandwidth bound). M = 1 is plain decode, 17 is 16 drafts
+ * + 1, and 68 is four sequences sharing one read.
+ *
+ * Arithmetic: each product x * (e2m1 * S) is exact. Sums are fp32. The result is
+ * multiplied by ts once, in fp32. X is converted to f16 for the products; that
+ * is exact for |x| in [2^-14, 65504]. Smaller magnitudes round to f16
+ * subnormals (absolute error below 2^-25). Larger ones saturate to 65504.
+ *
+ * Arguments
+ *   X       bf16 [M, K] row-major, device, 16-byte aligned.
+ *   q, sf   packed NVFP4 weight as produced by nvfp4_pack, device, 16-byte aligned.
+ *   tensor_scale  fp32 [1], device.
+ *   M       1 <= M <= NVFP4WS_MAX_M.   N >= 1.   K >= 32, K % 32 == 0.
+ *   Y       out: [M, N] row-major, device, 16-byte aligned; fp32 or bf16 per y_dtype.
+ *   workspace, workspace_bytes  device scratch of at least
+ *           nvfp4_gemm_workspace_bytes(M, N, K) bytes (may be NULL when that is 0).
+ *           Contents on entry do not matter.
+ * Returns NVFP4WS_OK, or INVALID_ARG / UNSUPPORTED / MISALIGNED / WORKSPACE / CUDA.
+ */
+int nvfp4_gemm_skinny(const void* X, const uint8_t* q, const uint8_t* sf, const float* tensor_scale,
+                      int64_t M, int64_t N, int64_t K, void* Y, int y_dtype,
+                      void* workspace, size_t workspace_bytes, nvfp4ws_stream_t stream);
+
+/* As nvfp4_gemm_skinny, with an explicit kernel path (nvfp4ws_path). Used by the M sweep and the tests. */
+int nvfp4_gemm_skinny_path(const void* X, const uint8_t* q, const uint8_t* sf, const float* tensor_scale,
+                           int64_t M, int64_t N, int64_t K, void* Y, int y_dtype,
+                           void* workspace, size_t workspace_bytes, int path, nvfp4ws_stream_t stream);
+
+/* Workspace needed by lmhead_verify_argmax_accept for this shape. */
+size_t lmhead_verify_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/*
+ * lmhead_verify_argmax_accept -- lm_head GEMM with fused greedy verify.
+ *
+ * Passages: "TandemLLM", introduction (accept drafts up to the first
+ * disagreement, then the target's token) and "How it works" (keep the longest
+ * agreeing path). "Qwen3.8 on DGX Spark (GB10)", introduction (verify over the
+ * whole vocabulary).
+ *
+ * The logits y = X . dequant(W)^T are computed exactly as in nvfp4_gemm_skinny
+ * but never written to memory. Per row m:
+ *   argmax[m] = the smallest n with y[m, n] == max_n y[m, n]
+ * Rows are grouped per sequence: M = B * (D + 1), and row b*(D+1)+i is the
+ * target's prediction for draft slot i of sequence b. Then:
+ *   accept_len[b] = min{ i in [0, D) : drafts[b, i] != argmax[b*(D+1) + i] }, or D
+ * The committed tokens of sequence b are argmax[b*(D+1) .. b*(D+1) + accept_len[b]]:
+ * the accepted drafts followed by the target's correction (or bonus) token.
+ *
+ * Arguments
+ *   X, q, sf, tensor_scale, N, K   as in nvfp4_gemm_skinny (N = vocabulary rows).
+ *   M           must equal B * (D + 1); 1 <= M <= NVFP4WS_MAX_M.
+ *   drafts      int32 [B, D] row-major, device (may be NULL when D == 0).
+ *   B, D        B >= 1, D >= 0.
+ *   argmax      out: int32 [M], device.
+ *   accept_len  out: int32 [B], device.
+ *   max_logit   out: fp32 [M], device, or NULL to skip (the winning logit, for tie diagnostics).
+ *   workspace   device scratch of at least lmhead_verify_workspace_bytes(M, N, K) bytes.
+ *               Contents on entry do not matter.
+ * Returns NVFP4WS_OK, or INVALID_ARG / UNSUPPORTED / MISALIGNED / WORKSPACE / CUDA.
+ * Logits that are NaN make argmax undefined.
+ */
+int lmhead_verify_argmax_accept(const void* X, const uint8_t* q, const uint8_t* sf,
+                                const float* tensor_scale, int64_t M, int64_t N, int64_t K,
+                                const int32_t* drafts, int32_t B, int32_t D,
+                                int32_t* argmax, int32_t* accept_len, float* max_logit,
+                                void* workspace, size_t workspace_bytes, nvfp4ws_stream_t stream);
+
+/* As lmhead_verify_argmax_accept, with an explicit kernel path (nvfp4ws_path). */
+int lmhead_verify_argmax_accept_path(const void* X, const uint8_t* q, const uint8_t* sf,
+                                     const float* tensor_scale, int64_t M, int64_t N, int64_t K,
+                                     const int32_t* drafts, int32_t B, int32_t D,
+                                     int32_t* argmax, int32_t* accept_len, float* max_logit,
+                                     void* workspace, size_t workspace_bytes, int path,
+                                     nvfp4ws_stream_t stream);
+
+/*
+ * nvfp4ws_check -- synchronise `stream`, then read and clear the device error word
+ * of the current device. Returns NVFP4WS_OK, NVFP4WS_ERR_DEVICE_TIMEOUT (a bounded
+ * wait gave up; the detail is in nvfp4ws_last_error) or NVFP4WS_ERR_CUDA.
+ */
+int nvfp4ws_check(nvfp4ws_stream_t stream);
+
+/* Number of SMs the kernels size their grids for (the current device's count). -1 on error. */
+int nvfp4ws_sm_count(void);
+
+/* Kernels (and memset nodes) this process has enqueued through the library so far, all
+   devices and threads together. During CUDA-graph capture this counts what the graph holds. */
+unsigned long long nvfp4ws_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4WS_H_ */

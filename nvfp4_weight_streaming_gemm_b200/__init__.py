@@ -1,0 +1,144 @@
+"""NVFP4 weight-streaming skinny GEMM and fused greedy verify for B200 (sm_100a).
+
+A thin binding over the C ABI of ``libnvfp4ws.so`` (declared in
+``include/nvfp4ws.h``). Every step of the computation runs in the library's CUDA
+kernels. This module only checks tensor properties, allocates outputs with
+torch, and passes raw device pointers and the current CUDA stream.
+
+    q, sf, ts = pack(W)                        # fp32 [N, K] -> NVFP4
+    Y = gemm(X, q, sf, ts)                     # bf16 [M, K] -> fp32 [M, N]
+    t, L, vmax = verify(X, q, sf, ts, drafts)  # fused lm_head argmax + accept length
+"""
+
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+
+PATHS = {"auto": 0, "gemv": 1, "mma": 2}
+STATUS_OK = 0
+
+
+class NVFP4WSError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        lib = _lib.load()
+        name = lib.nvfp4ws_status_string(status).decode()
+        detail = lib.nvfp4ws_last_error().decode()
+        super().__init__(f"{where}: {name}: {detail}")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    return _lib.load()
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _check(status: int, where: str):
+    if status != STATUS_OK:
+        raise NVFP4WSError(status, where)
+
+
+def _need_cuda(t, name, dtype=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def pack(W: torch.Tensor, tensor_scale_in: torch.Tensor | None = None, stream=None, out=None):
+    """Quantise fp32 W [N, K] to NVFP4. Returns ``(q uint8 [N, K/2], sf uint8 [N, K/16], ts fp32 [1])``."""
+    _need_cuda(W, "W", torch.float32)
+    N, K = W.shape
+    if out is None:
+        q = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device)
+        sf = torch.empty((N, K // 16), dtype=torch.uint8, device=W.device)
+        ts = torch.empty(1, dtype=torch.float32, device=W.device)
+    else:
+        q, sf, ts = out
+    if tensor_scale_in is not None:
+        _need_cuda(tensor_scale_in, "tensor_scale_in", torch.float32)
+    _check(lib().nvfp4_pack(_ptr(W), N, K, _ptr(q), _ptr(sf), _ptr(ts), _ptr(tensor_scale_in), _stream(stream)),
+           "nvfp4_pack")
+    return q, sf, ts
+
+
+def gemm_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib().nvfp4_gemm_workspace_bytes(M, N, K))
+
+
+def verify_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib().lmhead_verify_workspace_bytes(M, N, K))
+
+
+def _workspace(nbytes: int, device, workspace):
+    if nbytes == 0:
+        return None
+    if workspace is not None and workspace.numel() * workspace.element_size() >= nbytes:
+        return workspace
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def gemm(X: torch.Tensor, q: torch.Tensor, sf: torch.Tensor, ts: torch.Tensor, out: torch.Tensor | None = None,
+         y_dtype: torch.dtype = torch.float32, workspace: torch.Tensor | None = None, path: str = "auto",
+         stream=None) -> torch.Tensor:
+    """Y[M, N] = X[M, K] . dequant(W)^T with X bf16; Y fp32 (default) or bf16."""
+    _need_cuda(X, "X", torch.bfloat16)
+    _need_cuda(q, "q", torch.uint8)
+    _need_cuda(sf, "sf", torch.uint8)
+    M, K = X.shape
+    N = q.shape[0]
+    if q.shape[1] * 2 != K or sf.shape != (N, K // 16):
+        raise ValueError("q / sf shapes do not match X")
+    if out is None:
+        out = torch.empty((M, N), dtype=y_dtype, device=X.device)
+    yd = {torch.float32: 0, torch.bfloat16: 1}[out.dtype]
+    ws = _workspace(gemm_workspace_bytes(M, N, K), X.device, workspace)
+    nbytes = 0 if ws is None else ws.numel()
+    _check(lib().nvfp4_gemm_skinny_path(_ptr(X), _ptr(q), _ptr(sf), _ptr(ts), M, N, K, _ptr(out), yd, _ptr(ws),
+                                        nbytes, PATHS[path], _stream(stream)), "nvfp4_gemm_skinny")
+    return out
+
+
+def verify(X: torch.Tensor, q: torch.Tensor, sf: torch.Tensor, ts: torch.Tensor, drafts: torch.Tensor,
+           workspace: torch.Tensor | None = None, with_max_logit: bool = True, path: str = "auto", stream=None,
+           out=None):
+    """Fused lm_head greedy verify. ``drafts`` int32 [B, D]; X has M = B*(D+1) rows.
+
+    Returns ``(argmax int32 [M], accept_len int32 [B], max_logit fp32 [M] or None)``.
+    """
+    _need_cuda(X, "X", torch.bfloat16)
+    _need_cuda(drafts, "drafts", torch.int32)
+    M, K = X.shape
+    N = q.shape[0]
+    B, D = drafts.shape
+    if out is None:
+        amax = torch.empty(M, dtype=torch.int32, device=X.device)
+        acc = torch.empty(B, dtype=torch.int32, device=X.device)
+        vmax = torch.empty(M, dtype=torch.float32, device=X.device) if with_max_logit else None
+    else:
+        amax, acc, vmax = out
+    ws = _workspace(verify_workspace_bytes(M, N, K), X.device, workspace)
+    nbytes = 0 if ws is None else ws.numel()
+    dptr = _ptr(drafts) if drafts.numel() else None
+    _check(lib().lmhead_verify_argmax_accept_path(_ptr(X), _ptr(q), _ptr(sf), _ptr(ts), M, N, K, dptr, B, D,
+                                                  _ptr(amax), _ptr(acc), _ptr(vmax), _ptr(ws), nbytes, PATHS[path],
+                                                  _stream(stream)), "lmhead_verify_argmax_accept")
+    return amax, acc, vmax
+
+
+def check(stream=None):
+    """Synchronise and report a device-side bounded-wait failure, if any."""
+    _check(lib().nvfp4ws_check(_stream(stream)), "nvfp4ws_check")

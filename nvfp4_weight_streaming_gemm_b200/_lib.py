@@ -1,0 +1,53 @@
+"""ctypes loader of libnvfp4ws.so (the C ABI declared in include/nvfp4ws.h).
+
+There is no fallback. If the library is missing or does not load, importing the
+binding raises. Build it with ``python -m nvfp4_weight_streaming_gemm_b200.build``.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libnvfp4ws.so")
+
+c_i64, c_i32, c_p, c_sz = ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t
+
+# name -> (restype, argtypes)
+SIGNATURES = {
+    "nvfp4ws_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "nvfp4ws_last_error": (ctypes.c_char_p, []),
+    "nvfp4ws_version": (ctypes.c_int, []),
+    "nvfp4ws_sm_count": (ctypes.c_int, []),
+    "nvfp4_pack": (ctypes.c_int, [c_p, c_i64, c_i64, c_p, c_p, c_p, c_p, c_p]),
+    "nvfp4_gemm_workspace_bytes": (c_sz, [c_i64, c_i64, c_i64]),
+    "nvfp4_gemm_skinny": (ctypes.c_int, [c_p, c_p, c_p, c_p, c_i64, c_i64, c_i64, c_p, ctypes.c_int, c_p, c_sz, c_p]),
+    "nvfp4_gemm_skinny_path": (ctypes.c_int, [c_p, c_p, c_p, c_p, c_i64, c_i64, c_i64, c_p, ctypes.c_int, c_p, c_sz,
+                                              ctypes.c_int, c_p]),
+    "lmhead_verify_workspace_bytes": (c_sz, [c_i64, c_i64, c_i64]),
+    "lmhead_verify_argmax_accept": (ctypes.c_int, [c_p, c_p, c_p, c_p, c_i64, c_i64, c_i64, c_p, c_i32, c_i32, c_p,
+                                                   c_p, c_p, c_p, c_sz, c_p]),
+    "lmhead_verify_argmax_accept_path": (ctypes.c_int, [c_p, c_p, c_p, c_p, c_i64, c_i64, c_i64, c_p, c_i32, c_i32,
+                                                        c_p, c_p, c_p, c_p, c_sz, ctypes.c_int, c_p]),
+    "nvfp4ws_check": (ctypes.c_int, [c_p]),
+    "nvfp4ws_kernel_launches": (ctypes.c_ulonglong, []),
+}
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load the library once and declare every signature. Raises OSError if it is absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise OSError(f"{LIB_PATH} is missing: build it with `python -m nvfp4_weight_streaming_gemm_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib

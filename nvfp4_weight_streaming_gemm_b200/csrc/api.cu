@@ -1,0 +1,241 @@
+// The C ABI of libnvfp4ws (include/nvfp4ws.h): argument validation, workspace
+// sizing, kernel-path dispatch and error reporting. Every check runs on the host
+// before anything is enqueued.
+#include "common.cuh"
+#include "kernels.h"
+#include "mma.h"
+
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+namespace nvfp4ws {
+
+static thread_local char g_last_error[512] = "";
+__device__ unsigned int g_device_error = 0u;
+
+int set_error(int status, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return status;
+}
+
+static std::atomic<unsigned long long> g_launches{0};
+
+int check_launch(const char* what) {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(NVFP4WS_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return NVFP4WS_OK;
+}
+
+unsigned int* device_error_word() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+  return static_cast<unsigned int*>(p);
+}
+
+int device_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  return n;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Shared validation of the GEMM-shaped calls.
+static int validate_gemm(const void* X, const uint8_t* q, const uint8_t* sf, const float* ts, int64_t M,
+                         int64_t N, int64_t K, const char* who) {
+  if (!X || !q || !sf || !ts) return set_error(NVFP4WS_ERR_INVALID_ARG, "%s: null input pointer", who);
+  if (M < 1 || N < 1 || K < 1) return set_error(NVFP4WS_ERR_INVALID_ARG, "%s: M, N, K must be >= 1", who);
+  if (M > NVFP4WS_MAX_M)
+    return set_error(NVFP4WS_ERR_UNSUPPORTED, "%s: M=%lld exceeds %d", who, (long long)M, NVFP4WS_MAX_M);
+  if (K % 32 != 0) return set_error(NVFP4WS_ERR_UNSUPPORTED, "%s: K=%lld is not a multiple of 32", who, (long long)K);
+  if (N > (int64_t)0x7fffffff || K > ((int64_t)1 << 24))
+    return set_error(NVFP4WS_ERR_UNSUPPORTED, "%s: N or K too large", who);
+  if (!aligned16(X) || !aligned16(q) || !aligned16(sf))
+    return set_error(NVFP4WS_ERR_MISALIGNED, "%s: X, q and sf must be 16-byte aligned", who);
+  return NVFP4WS_OK;
+}
+
+static int resolve_path(int path, int64_t M, int64_t K) {
+  if (path == NVFP4WS_PATH_AUTO) {
+    if (mma_supported(M, K) && M >= mma_min_m()) return NVFP4WS_PATH_MMA;
+    return NVFP4WS_PATH_GEMV;
+  }
+  return path;
+}
+
+}  // namespace nvfp4ws
+
+using namespace nvfp4ws;
+
+extern "C" {
+
+const char* nvfp4ws_status_string(int status) {
+  switch (status) {
+    case NVFP4WS_OK: return "NVFP4WS_OK";
+    case NVFP4WS_ERR_INVALID_ARG: return "NVFP4WS_ERR_INVALID_ARG";
+    case NVFP4WS_ERR_UNSUPPORTED: return "NVFP4WS_ERR_UNSUPPORTED";
+    case NVFP4WS_ERR_MISALIGNED: return "NVFP4WS_ERR_MISALIGNED";
+    case NVFP4WS_ERR_WORKSPACE: return "NVFP4WS_ERR_WORKSPACE";
+    case NVFP4WS_ERR_CUDA: return "NVFP4WS_ERR_CUDA";
+    case NVFP4WS_ERR_DEVICE_TIMEOUT: return "NVFP4WS_ERR_DEVICE_TIMEOUT";
+    default: return "NVFP4WS_UNKNOWN_STATUS";
+  }
+}
+
+const char* nvfp4ws_last_error(void) { return g_last_error; }
+
+int nvfp4ws_version(void) { return 100; }
+
+int nvfp4ws_sm_count(void) { return device_sm_count(); }
+
+unsigned long long nvfp4ws_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int nvfp4_pack(const float* W, int64_t N, int64_t K, uint8_t* q, uint8_t* sf, float* tensor_scale,
+               const float* tensor_scale_in, nvfp4ws_stream_t stream) {
+  g_last_error[0] = 0;
+  if (!W || !q || !sf || !tensor_scale) return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_pack: null pointer");
+  if (N < 1 || K < 16 || K % 16 != 0)
+    return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_pack: need N >= 1 and K a positive multiple of 16");
+  if (!aligned16(W) || !aligned16(q))
+    return set_error(NVFP4WS_ERR_MISALIGNED, "nvfp4_pack: W and q must be 16-byte aligned");
+  if (((uintptr_t)tensor_scale & 3u) || ((uintptr_t)tensor_scale_in & 3u))
+    return set_error(NVFP4WS_ERR_MISALIGNED, "nvfp4_pack: tensor scales must be 4-byte aligned");
+  return launch_pack(W, N, K, q, sf, tensor_scale, tensor_scale_in, (cudaStream_t)stream);
+}
+
+size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M < 1 || N < 1 || K < 32) return 0;
+  int path = resolve_path(NVFP4WS_PATH_AUTO, M, K);
+  if (path == NVFP4WS_PATH_MMA) return mma_gemm_workspace_bytes(M, N, K);
+  return 0;
+}
+
+int nvfp4_gemm_skinny_path(const void* X, const uint8_t* q, const uint8_t* sf, const float* tensor_scale,
+                           int64_t M, int64_t N, int64_t K, void* Y, int y_dtype, void* workspace,
+                           size_t workspace_bytes, int path, nvfp4ws_stream_t stream) {
+  g_last_error[0] = 0;
+  if (int e = validate_gemm(X, q, sf, tensor_scale, M, N, K, "nvfp4_gemm_skinny")) return e;
+  if (!Y) return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_gemm_skinny: Y is null");
+  if (!aligned16(Y)) return set_error(NVFP4WS_ERR_MISALIGNED, "nvfp4_gemm_skinny: Y must be 16-byte aligned");
+  if (y_dtype != NVFP4WS_Y_F32 && y_dtype != NVFP4WS_Y_BF16)
+    return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_gemm_skinny: bad y_dtype %d", y_dtype);
+  if (path < NVFP4WS_PATH_AUTO || path > NVFP4WS_PATH_MMA)
+    return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_gemm_skinny: bad path %d", path);
+  path = resolve_path(path, M, K);
+  cudaStream_t s = (cudaStream_t)stream;
+  if (path == NVFP4WS_PATH_MMA) {
+    if (!mma_supported(M, K))
+      return set_error(NVFP4WS_ERR_UNSUPPORTED, "nvfp4_gemm_skinny: MMA path does not support M=%lld K=%lld",
+                       (long long)M, (long long)K);
+    size_t need = mma_gemm_workspace_bytes(M, N, K);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need))
+      return set_error(NVFP4WS_ERR_WORKSPACE, "nvfp4_gemm_skinny: workspace needs %zu bytes", need);
+    if (need > 0 && !aligned16(workspace))
+      return set_error(NVFP4WS_ERR_MISALIGNED, "nvfp4_gemm_skinny: workspace must be 16-byte aligned");
+    return launch_mma_gemm(static_cast<const uint16_t*>(X), q, sf, tensor_scale, M, N, K, Y, y_dtype,
+                           workspace, workspace_bytes, s);
+  }
+  if (!gemv_supported(K))
+    return set_error(NVFP4WS_ERR_UNSUPPORTED, "nvfp4_gemm_skinny: GEMV path supports K <= 65536");
+  GemvArgs a{};
+  a.X = static_cast<const uint16_t*>(X);
+  a.q = q; a.sf = sf; a.ts = tensor_scale;
+  a.M = M; a.N = N; a.K = K;
+  a.Y = Y; a.y_bf16 = (y_dtype == NVFP4WS_Y_BF16);
+  return launch_gemv(a, false, s);
+}
+
+int nvfp4_gemm_skinny(const void* X, const uint8_t* q, const uint8_t* sf, const float* tensor_scale, int64_t M,
+                      int64_t N, int64_t K, void* Y, int y_dtype, void* workspace, size_t workspace_bytes,
+                      nvfp4ws_stream_t stream) {
+  return nvfp4_gemm_skinny_path(X, q, sf, tensor_scale, M, N, K, Y, y_dtype, workspace, workspace_bytes,
+                                NVFP4WS_PATH_AUTO, stream);
+}
+
+static size_t gemv_verify_workspace(int64_t M, int64_t N, int64_t K) {
+  GemvPlan p = gemv_plan(M, N, K);
+  return 2 * align_up((size_t)p.grid * (size_t)M * 4, 256);
+}
+
+size_t lmhead_verify_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M < 1 || N < 1 || K < 32) return 0;
+  size_t w = gemv_verify_workspace(M, N, K);
+  size_t m = mma_supported(M, K) ? mma_verify_workspace_bytes(M, N, K) : 0;
+  return w > m ? w : m;
+}
+
+int lmhead_verify_argmax_accept_path(const void* X, const uint8_t* q, const uint8_t* sf, const float* tensor_scale,
+                                     int64_t M, int64_t N, int64_t K, const int32_t* drafts, int32_t B, int32_t D,
+                                     int32_t* argmax, int32_t* accept_len, float* max_logit, void* workspace,
+                                     size_t workspace_bytes, int path, nvfp4ws_stream_t stream) {
+  g_last_error[0] = 0;
+  if (int e = validate_gemm(X, q, sf, tensor_scale, M, N, K, "lmhead_verify")) return e;
+  if (B < 1 || D < 0) return set_error(NVFP4WS_ERR_INVALID_ARG, "lmhead_verify: need B >= 1 and D >= 0");
+  if ((int64_t)B * (D + 1) != M)
+    return set_error(NVFP4WS_ERR_INVALID_ARG, "lmhead_verify: M=%lld must equal B*(D+1)=%lld", (long long)M,
+                     (long long)B * (D + 1));
+  if (D > 0 && !drafts) return set_error(NVFP4WS_ERR_INVALID_ARG, "lmhead_verify: drafts is null");
+  if (!argmax || !accept_len) return set_error(NVFP4WS_ERR_INVALID_ARG, "lmhead_verify: null output pointer");
+  if (path < NVFP4WS_PATH_AUTO || path > NVFP4WS_PATH_MMA)
+    return set_error(NVFP4WS_ERR_INVALID_ARG, "lmhead_verify: bad path %d", path);
+  path = resolve_path(path, M, K);
+  cudaStream_t s = (cudaStream_t)stream;
+  if (path == NVFP4WS_PATH_MMA) {
+    if (!mma_supported(M, K))
+      return set_error(NVFP4WS_ERR_UNSUPPORTED, "lmhead_verify: MMA path does not support M=%lld K=%lld",
+                       (long long)M, (long long)K);
+    size_t need = mma_verify_workspace_bytes(M, N, K);
+    if (workspace == nullptr || workspace_bytes < need)
+      return set_error(NVFP4WS_ERR_WORKSPACE, "lmhead_verify: workspace needs %zu bytes", need);
+    if (!aligned16(workspace)) return set_error(NVFP4WS_ERR_MISALIGNED, "lmhead_verify: workspace must be 16-byte aligned");
+    return launch_mma_verify(static_cast<const uint16_t*>(X), q, sf, tensor_scale, M, N, K, drafts, B, D, argmax,
+                             accept_len, max_logit, workspace, s);
+  }
+  if (!gemv_supported(K)) return set_error(NVFP4WS_ERR_UNSUPPORTED, "lmhead_verify: GEMV path supports K <= 65536");
+  size_t need = gemv_verify_workspace(M, N, K);
+  if (workspace == nullptr || workspace_bytes < need)
+    return set_error(NVFP4WS_ERR_WORKSPACE, "lmhead_verify: workspace needs %zu bytes", need);
+  if (!aligned16(workspace)) return set_error(NVFP4WS_ERR_MISALIGNED, "lmhead_verify: workspace must be 16-byte aligned");
+  GemvPlan p = gemv_plan(M, N, K);
+  GemvArgs a{};
+  a.X = static_cast<const uint16_t*>(X);
+  a.q = q; a.sf = sf; a.ts = tensor_scale;
+  a.M = M; a.N = N; a.K = K;
+  a.part_val = static_cast<float*>(workspace);
+  a.part_idx = reinterpret_cast<int*>(static_cast<char*>(workspace) + align_up((size_t)p.grid * M * 4, 256));
+  if (int e = launch_gemv(a, true, s)) return e;
+  return launch_verify_stage2(a.part_val, a.part_idx, p.grid, (int)M, drafts, B, D, argmax, accept_len, max_logit, s);
+}
+
+int lmhead_verify_argmax_accept(const void* X, const uint8_t* q, const uint8_t* sf, const float* tensor_scale,
+                                int64_t M, int64_t N, int64_t K, const int32_t* drafts, int32_t B, int32_t D,
+                                int32_t* argmax, int32_t* accept_len, float* max_logit, void* workspace,
+                                size_t workspace_bytes, nvfp4ws_stream_t stream) {
+  return lmhead_verify_argmax_accept_path(X, q, sf, tensor_scale, M, N, K, drafts, B, D, argmax, accept_len,
+                                          max_logit, workspace, workspace_bytes, NVFP4WS_PATH_AUTO, stream);
+}
+
+int nvfp4ws_check(nvfp4ws_stream_t stream) {
+  g_last_error[0] = 0;
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return set_error(NVFP4WS_ERR_CUDA, "nvfp4ws_check: %s", cudaGetErrorString(e));
+  unsigned int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v));
+  if (e != cudaSuccess) return set_error(NVFP4WS_ERR_CUDA, "nvfp4ws_check: %s", cudaGetErrorString(e));
+  if (v != 0) {
+    unsigned int zero = 0;
+    cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
+    return set_error(NVFP4WS_ERR_DEVICE_TIMEOUT, "a bounded device wait gave up (code 0x%x)", v);
+  }
+  return NVFP4WS_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,254 @@
+// CUDA-core streaming GEMV for small M:
+//   y[m, n] = ts * sum_b S[n, b] * sum_{k in block b} x[m, k] * e2m1(code[n, k])
+//
+// Why this shape. At M = 1 a weight pass streams ~0.56 bytes per element and does
+// 2 flops per element: it is HBM-bound by a factor of ~500 ("veloGB10",
+// "Unique aspects: Engineered to the roofline": "~94% GEMM and
+// weight-bandwidth-bound"). The only arithmetic that matters is keeping the
+// dequantisation ahead of HBM. On B200 the cheapest exact form measured was a
+// hardware E2M1x2 -> f16x2 conversion followed by mixed f16 x f16 -> f32 FMAs.
+//
+// Mapping. The threads of a CTA span K. Thread t owns the 32-element chunks
+// c = t + j*T (j < CPT, T = blockDim.x). Its slice of X stays in registers as
+// f16x2 for the whole kernel. A CTA walks row groups of R rows, grid-stride. For
+// each row it loads one 16-byte nibble word per chunk
+// (ld.global.nc.L1::no_allocate) and one 2-byte scale pair. The next group is
+// prefetched into registers while the current one is computed. Per-row partial
+// sums are reduced with warp shuffles, then across warps through shared memory,
+// in a fixed order. The result is deterministic and uses no atomics.
+//
+// In verify mode the reducing thread of each token keeps a running (max, lowest
+// index) over the rows the CTA visits, and writes one partial per CTA. Logits
+// never reach HBM.
+#include "common.cuh"
+#include "kernels.h"
+
+#include <algorithm>
+#include <climits>
+#include <cmath>
+
+namespace nvfp4ws {
+
+template <int MT, int CPT, int R, bool VERIFY>
+__global__ void __launch_bounds__(512) gemv_kernel(GemvArgs a) {
+  const int T = blockDim.x;
+  const int t = threadIdx.x;
+  const int lane = t & 31, warp = t >> 5, nwarps = T >> 5;
+  const int C = a.K >> 5;                       // 32-element chunks per row
+  const long long rowq = a.K >> 1;              // bytes of q per row
+  const long long rows = a.K >> 4;              // bytes of sf per row
+
+  // X slice -> registers (f16x2), zero outside [0, C) and beyond M
+  uint32_t xr[MT][CPT][16];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) {
+      const int c = t + j * T;
+      const int mm = a.m0 + m;
+      if (c < C && mm < a.M) {
+        const uint4* src = reinterpret_cast<const uint4*>(a.X + (long long)mm * a.K + (long long)c * 32);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          uint4 b = src[v];
+          xr[m][j][4 * v + 0] = bf16x2_to_f16x2_sat(b.x);
+          xr[m][j][4 * v + 1] = bf16x2_to_f16x2_sat(b.y);
+          xr[m][j][4 * v + 2] = bf16x2_to_f16x2_sat(b.z);
+          xr[m][j][4 * v + 3] = bf16x2_to_f16x2_sat(b.w);
+        }
+      } else {
+#pragma unroll
+        for (int v = 0; v < 16; ++v) xr[m][j][v] = 0u;
+      }
+    }
+  }
+
+  extern __shared__ float red[];                // [2][nwarps][R][MT]
+  const float ts = *a.ts;
+  const int ngroups = (int)((a.N + R - 1) / R);
+
+  float bestv = -INFINITY;
+  int besti = INT_MAX;
+
+  uint4 cur[R][CPT];
+  uint32_t curs[R][CPT];
+
+  auto load_group = [&](int g, uint4 (&qv)[R][CPT], uint32_t (&sv)[R][CPT]) {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const long long n = (long long)g * R + r;
+#pragma unroll
+      for (int j = 0; j < CPT; ++j) {
+        const int c = t + j * T;
+        if (n < a.N && c < C) {
+          qv[r][j] = ld_stream_v4(a.q + n * rowq + (long long)c * 16);
+          sv[r][j] = ld_stream_u16(a.sf + n * rows + (long long)c * 2);
+        } else {
+          qv[r][j] = make_uint4(0, 0, 0, 0);
+          sv[r][j] = 0u;
+        }
+      }
+    }
+  };
+
+  int g = blockIdx.x;
+  if (g < ngroups) load_group(g, cur, curs);
+  int buf = 0;
+  for (; g < ngroups; g += gridDim.x) {
+    uint4 nxt[R][CPT];
+    uint32_t nxts[R][CPT];
+    const int gn = g + gridDim.x;
+    if (gn < ngroups) load_group(gn, nxt, nxts);
+
+    float acc[R][MT];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int m = 0; m < MT; ++m) acc[r][m] = 0.0f;
+
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+#pragma unroll
+      for (int j = 0; j < CPT; ++j) {
+        const uint32_t s2 = e4m3x2_to_f16x2(curs[r][j]);
+        const float S0 = f16lo_to_f32(s2), S1 = f16hi_to_f32(s2);
+        const uint32_t w[4] = {cur[r][j].x, cur[r][j].y, cur[r][j].z, cur[r][j].w};
+        uint32_t h[16];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int b = 0; b < 4; ++b) h[4 * i + b] = e2m1x2_to_f16x2(w[i] >> (8 * b));
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) dot2_f16_f32(p0, p1, h[e], xr[m][j][e]);
+#pragma unroll
+          for (int e = 8; e < 16; ++e) dot2_f16_f32(p2, p3, h[e], xr[m][j][e]);
+          acc[r][m] = fmaf(S0, p0 + p1, acc[r][m]);
+          acc[r][m] = fmaf(S1, p2 + p3, acc[r][m]);
+        }
+      }
+    }
+
+    // reduce over the CTA: shuffles within each warp, then warps in order
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        float v = acc[r][m];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0) red[((buf * nwarps + warp) * R + r) * MT + m] = v;
+      }
+    __syncthreads();
+    if constexpr (!VERIFY) {
+      if (t < R * MT) {
+        const int r = t / MT, m = t - r * MT;
+        const long long n = (long long)g * R + r;
+        const int mm = a.m0 + m;
+        if (n < a.N && mm < a.M) {
+          float s = 0.f;
+          for (int w = 0; w < nwarps; ++w) s += red[((buf * nwarps + w) * R + r) * MT + m];
+          const float y = s * ts;
+          if (a.y_bf16)
+            reinterpret_cast<uint16_t*>(a.Y)[(long long)mm * a.N + n] = f32_to_bf16_rn(y);
+          else
+            reinterpret_cast<float*>(a.Y)[(long long)mm * a.N + n] = y;
+        }
+      }
+    } else {
+      if (t < MT) {
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const long long n = (long long)g * R + r;
+          if (n < a.N) {
+            float s = 0.f;
+            for (int w = 0; w < nwarps; ++w) s += red[((buf * nwarps + w) * R + r) * MT + t];
+            const float y = s * ts;
+            if (argmax_better(y, (int)n, bestv, besti)) { bestv = y; besti = (int)n; }
+          }
+        }
+      }
+    }
+    buf ^= 1;
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int j = 0; j < CPT; ++j) { cur[r][j] = nxt[r][j]; curs[r][j] = nxts[r][j]; }
+  }
+  if constexpr (VERIFY) {
+    if (t < MT && a.m0 + t < a.M) {
+      a.part_val[(long long)blockIdx.x * a.M + a.m0 + t] = bestv;
+      a.part_idx[(long long)blockIdx.x * a.M + a.m0 + t] = besti;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side: pick (MT, CPT, R, T) and the grid
+// ---------------------------------------------------------------------------
+
+template <int MT, int CPT, int R, bool VERIFY>
+static int launch_one(const GemvArgs& a, int T, int grid, cudaStream_t s) {
+  const int nwarps = T / 32;
+  const size_t smem = sizeof(float) * 2 * nwarps * R * MT;
+  gemv_kernel<MT, CPT, R, VERIFY><<<grid, T, smem, s>>>(a);
+  return check_launch("gemv_kernel");
+}
+
+template <int MT, int CPT, int R, bool VERIFY>
+static int occupancy_of(int T) {
+  const int nwarps = T / 32;
+  const size_t smem = sizeof(float) * 2 * nwarps * R * MT;
+  int nb = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, gemv_kernel<MT, CPT, R, VERIFY>, T, smem) != cudaSuccess)
+    return 1;
+  return std::max(nb, 1);
+}
+
+GemvPlan gemv_plan(long long M, long long N, long long K) {
+  GemvPlan p{};
+  const int C = (int)(K / 32);
+  p.cpt = C <= 512 ? 1 : (C <= 1024 ? 2 : 4);
+  int per = (C + p.cpt - 1) / p.cpt;
+  p.threads = std::max(32, ((per + 31) / 32) * 32);
+  p.mt = (M >= 4 && p.cpt == 1) ? 4 : (M >= 2 && p.cpt <= 2 ? 2 : 1);
+  p.rows = p.cpt == 1 ? 4 : (p.cpt == 2 ? 2 : 1);
+  int occ = 1;
+#define OCC(MT_, CPT_, R_) if (p.mt == MT_ && p.cpt == CPT_) occ = occupancy_of<MT_, CPT_, R_, true>(p.threads);
+  OCC(1, 1, 4) OCC(1, 2, 2) OCC(1, 4, 1) OCC(2, 1, 4) OCC(2, 2, 2) OCC(4, 1, 4)
+#undef OCC
+  const long long ngroups = (N + p.rows - 1) / p.rows;
+  const int sms = device_sm_count();
+  p.grid = (int)std::max<long long>(1, std::min<long long>(ngroups, (long long)sms * occ));
+  return p;
+}
+
+bool gemv_supported(long long K) { return K % 32 == 0 && K / 32 <= 2048; }
+
+int launch_gemv(const GemvArgs& base, bool verify, cudaStream_t s) {
+  const GemvPlan p = gemv_plan(base.M, base.N, base.K);
+  for (long long m0 = 0; m0 < base.M;) {
+    GemvArgs a = base;
+    a.m0 = (int)m0;
+    const long long left = base.M - m0;
+    int mt = p.mt;
+    while (mt > 1 && mt > left) mt >>= 1;
+    int e = 0;
+#define L(MT_, CPT_, R_)                                                              \
+  if (mt == MT_ && p.cpt == CPT_) {                                                   \
+    e = verify ? launch_one<MT_, CPT_, R_, true>(a, p.threads, p.grid, s)             \
+               : launch_one<MT_, CPT_, R_, false>(a, p.threads, p.grid, s);           \
+  } else
+    L(1, 1, 4) L(1, 2, 2) L(1, 4, 1) L(2, 1, 4) L(2, 2, 2) L(4, 1, 4) {
+      return set_error(NVFP4WS_ERR_UNSUPPORTED, "no GEMV variant for mt=%d cpt=%d", mt, p.cpt);
+    }
+#undef L
+    if (e) return e;
+    m0 += mt;
+  }
+  return NVFP4WS_OK;
+}
+
+}  // namespace nvfp4ws

@@ -1,0 +1,39 @@
+// Internal launch interfaces of libnvfp4ws (not part of the C ABI).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace nvfp4ws {
+
+struct GemvArgs {
+  const uint16_t* X;        // bf16 [M, K]
+  const uint8_t* q;         // [N, K/2]
+  const uint8_t* sf;        // [N, K/16]
+  const float* ts;          // [1]
+  long long M, N, K;
+  int m0;                   // first token of this launch
+  void* Y;                  // [M, N] (GEMM mode)
+  int y_bf16;
+  float* part_val;          // [grid, M] (verify mode)
+  int* part_idx;            // [grid, M]
+};
+
+struct GemvPlan {
+  int mt, cpt, rows, threads, grid;
+};
+
+GemvPlan gemv_plan(long long M, long long N, long long K);
+bool gemv_supported(long long K);
+int launch_gemv(const GemvArgs& a, bool verify, cudaStream_t s);
+
+int launch_pack(const float* W, long long N, long long K, uint8_t* q, uint8_t* sf, float* ts,
+                const float* ts_in, cudaStream_t s);
+
+// Stage 2 of the verify: reduce per-CTA (max, index) partials to argmax[M], then
+// the accept length of every sequence.
+int launch_verify_stage2(const float* part_val, const int* part_idx, int nparts, int M,
+                         const int32_t* drafts, int B, int D, int32_t* argmax, int32_t* accept_len,
+                         float* max_logit, cudaStream_t s);
+
+}  // namespace nvfp4ws

@@ -1,0 +1,20 @@
+// Internal interface of the tcgen05 tensor-core path (not part of the C ABI).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace nvfp4ws {
+
+bool mma_supported(long long M, long long K);
+int mma_min_m();
+size_t mma_gemm_workspace_bytes(long long M, long long N, long long K);
+size_t mma_verify_workspace_bytes(long long M, long long N, long long K);
+int launch_mma_gemm(const uint16_t* X, const uint8_t* q, const uint8_t* sf, const float* ts, long long M, long long N,
+                    long long K, void* Y, int y_dtype, void* workspace, size_t workspace_bytes, cudaStream_t s);
+int launch_mma_verify(const uint16_t* X, const uint8_t* q, const uint8_t* sf, const float* ts, long long M,
+                      long long N, long long K, const int32_t* drafts, int B, int D, int32_t* argmax,
+                      int32_t* accept_len, float* max_logit, void* workspace, cudaStream_t s);
+
+}  // namespace nvfp4ws

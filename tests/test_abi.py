@@ -1,0 +1,95 @@
+"""CPU checks of the C ABI: the library loads, exports every function that
+include/nvfp4ws.h declares, and rejects bad arguments on the host before
+touching the GPU. No compute call is made here."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "nvfp4ws.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from nvfp4_weight_streaming_gemm_b200 import build, _lib
+    build.build()
+    return _lib.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = "\n".join(l for l in text.splitlines() if not l.lstrip().startswith("#"))
+    names = []
+    for decl in text.split(";"):
+        if "(" not in decl or "typedef" in decl or "{" in decl.split("(")[0]:
+            continue
+        m = re.search(r"([A-Za-z_][A-Za-z0-9_]*)\s*\($", decl.split("(")[0] + "(")
+        if m:
+            names.append(m.group(1))
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("nvfp4_pack", "nvfp4_gemm_skinny", "lmhead_verify_argmax_accept",
+                     "nvfp4_gemm_workspace_bytes", "lmhead_verify_workspace_bytes", "nvfp4ws_status_string",
+                     "nvfp4ws_last_error", "nvfp4ws_check"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert missing == []
+
+
+def test_binding_covers_header(lib):
+    from nvfp4_weight_streaming_gemm_b200 import _lib
+    assert sorted(_lib.SIGNATURES) == declared_functions()
+
+
+def test_status_strings(lib):
+    assert lib.nvfp4ws_status_string(0) == b"NVFP4WS_OK"
+    assert lib.nvfp4ws_status_string(6) == b"NVFP4WS_ERR_DEVICE_TIMEOUT"
+    assert lib.nvfp4ws_status_string(99) == b"NVFP4WS_UNKNOWN_STATUS"
+    assert lib.nvfp4ws_version() >= 100
+
+
+FAKE = 0x1000000        # 16-byte aligned, never dereferenced: validation fails first
+
+
+def test_gemm_rejects_null_and_bad_shapes(lib):
+    f = lib.nvfp4_gemm_skinny
+    assert f(None, FAKE, FAKE, FAKE, 1, 16, 64, FAKE, 0, None, 0, None) == 1
+    assert f(FAKE, FAKE, FAKE, FAKE, 0, 16, 64, FAKE, 0, None, 0, None) == 1
+    assert f(FAKE, FAKE, FAKE, FAKE, 1, 16, 48, FAKE, 0, None, 0, None) == 2      # K % 32
+    assert f(FAKE, FAKE, FAKE, FAKE, 257, 16, 64, FAKE, 0, None, 0, None) == 2    # M > 256
+    assert f(FAKE + 8, FAKE, FAKE, FAKE, 1, 16, 64, FAKE, 0, None, 0, None) == 3  # misaligned X
+    assert f(FAKE, FAKE, FAKE, FAKE, 1, 16, 64, FAKE + 4, 0, None, 0, None) == 3  # misaligned Y
+    assert f(FAKE, FAKE, FAKE, FAKE, 1, 16, 64, FAKE, 7, None, 0, None) == 1      # bad y dtype
+    assert b"K=48" in lib.nvfp4ws_last_error() or lib.nvfp4ws_last_error() != b""
+
+
+def test_gemm_rejects_bad_path(lib):
+    assert lib.nvfp4_gemm_skinny_path(FAKE, FAKE, FAKE, FAKE, 1, 16, 64, FAKE, 0, None, 0, 9, None) == 1
+
+
+def test_pack_rejects(lib):
+    f = lib.nvfp4_pack
+    assert f(None, 4, 32, FAKE, FAKE, FAKE, None, None) == 1
+    assert f(FAKE, 4, 24, FAKE, FAKE, FAKE, None, None) == 1                      # K % 16
+    assert f(FAKE + 4, 4, 32, FAKE, FAKE, FAKE, None, None) == 3
+
+
+def test_verify_rejects(lib):
+    f = lib.lmhead_verify_argmax_accept
+    # M != B*(D+1)
+    assert f(FAKE, FAKE, FAKE, FAKE, 17, 100, 64, FAKE, 2, 16, FAKE, FAKE, None, FAKE, 1 << 20, None) == 1
+    # drafts missing with D > 0
+    assert f(FAKE, FAKE, FAKE, FAKE, 17, 100, 64, None, 1, 16, FAKE, FAKE, None, FAKE, 1 << 20, None) == 1
+    # null outputs
+    assert f(FAKE, FAKE, FAKE, FAKE, 17, 100, 64, FAKE, 1, 16, None, FAKE, None, FAKE, 1 << 20, None) == 1
+    assert f(FAKE, FAKE, FAKE, FAKE, 1, 100, 64, None, 0, 0, FAKE, FAKE, None, FAKE, 1 << 20, None) == 1  # B < 1
