@@ -168,8 +168,8 @@ class Pass:
             off += n
         self.ys = [torch.empty((M, N), dtype=torch.float32, device=dev) for (_, _, N, _, _, _) in stack]
         wsb = max(nv.gemm_workspace_bytes(M, N, K) for (_, K, N, _, _, _) in stack)
-        self.gws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
-        self.vws = torch.empty(max(nv.verify_workspace_bytes(M, S.VOCAB, S.LMHEAD_K), 16), dtype=torch.uint8,
+        self.gws = torch.zeros(max(wsb, 16), dtype=torch.uint8, device=dev)
+        self.vws = torch.zeros(max(nv.verify_workspace_bytes(M, S.VOCAB, S.LMHEAD_K), 16), dtype=torch.uint8,
                                device=dev)
         self.argmax = torch.empty(M, dtype=torch.int32, device=dev)
         self.accept = torch.empty(self.B, dtype=torch.int32, device=dev)
@@ -393,6 +393,55 @@ def run_ours(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- per-shape sweep
+
+def run_sweep(args):
+    """One matrix shape at several M (and paths), rotating through ``--copies``
+    distinct packed copies of the weight so that every launch reads from HBM
+    (copies x weight bytes > L2). Prints one JSON line per (M, path). This is the
+    M sweep on the gate+up shape, and the small case ncu captures are taken on."""
+    import torch
+    import nvfp4_weight_streaming_gemm_b200 as nv
+    from nvfp4_weight_streaming_gemm_b200 import build as nvbuild
+    nvbuild.build()
+    dev = torch.device("cuda", 0)
+    K, N = S.LAYER_SHAPES[args.shape] if args.shape in S.LAYER_SHAPES else (S.LMHEAD_K, S.VOCAB)
+    copies = []
+    for i in range(args.copies):
+        g = torch.Generator(device=dev)
+        g.manual_seed(500 + i)
+        W = torch.randn(N, K, generator=g, device=dev).mul_(S.W_STD)
+        copies.append(nv.pack(W))
+        del W
+    peak, peak_kind = measured_peaks()
+    for M in [int(m) for m in args.ms.split(",")]:
+        X = torch.randn(M, K, device=dev).to(torch.bfloat16)
+        Y = torch.empty(M, N, device=dev)
+        ws = torch.zeros(max(16, nv.gemm_workspace_bytes(M, N, K)), dtype=torch.uint8, device=dev)
+        for path in args.paths.split(","):
+            try:
+                for i in range(args.warmup):
+                    q, sf, ts = copies[i % len(copies)]
+                    nv.gemm(X, q, sf, ts, out=Y, workspace=ws, path=path)
+            except Exception as e:  # a forced path that does not support this shape
+                print(json.dumps({"shape": args.shape, "M": M, "path": path, "skipped": str(e)}), flush=True)
+                continue
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for i in range(args.steps):
+                q, sf, ts = copies[i % len(copies)]
+                nv.gemm(X, q, sf, ts, out=Y, workspace=ws, path=path)
+            e1.record()
+            torch.cuda.synchronize()
+            us = 1e3 * e0.elapsed_time(e1) / args.steps
+            alg = weight_bytes(N, K) + M * K * 2 + M * N * 4
+            print(json.dumps({"shape": args.shape, "N": N, "K": K, "M": M, "path": path, "us_per_launch": us,
+                              "weight_gbs": weight_bytes(N, K) / us / 1e3, "alg_gbs": alg / us / 1e3,
+                              "frac_of_peak": alg / us / 1e3 / peak, "peak_kind": peak_kind,
+                              "copies": args.copies}), flush=True)
+
+
 # ----------------------------------------------------------------------------- reference arm
 
 def run_reference(args, rank, world):
@@ -437,13 +486,19 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per GEMM pass from an ncu capture (reported as roofline.traffic)")
+    ap.add_argument("--sweep", action="store_true", help="time one matrix shape per M and path (no pass)")
+    ap.add_argument("--shape", default="gate_up", help="sweep shape: gate_up, down, qkv or lm_head")
+    ap.add_argument("--paths", default="auto,gemv,mma")
+    ap.add_argument("--copies", type=int, default=4)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.impl == "reference":
+    if args.sweep:
+        run_sweep(args)
+    elif args.impl == "reference":
         run_reference(args, rank, world)
     else:
         run_ours(args, rank, world, local_rank)

@@ -104,8 +104,8 @@ int nvfp4_pack(const float* W, int64_t N, int64_t K, uint8_t* q, uint8_t* sf,
                float* tensor_scale, const float* tensor_scale_in, nvfp4ws_stream_t stream);
 
 /*
- * nvfp4_gemm_workspace_bytes -- device workspace needed by nvfp4_gemm_skinny for
- * this shape (0 when none is needed). Pass at least this many bytes.
+ * nvfp4_gemm_workspace_bytes -- device workspace needed by nvfp4_gemm_skinny (any
+ * path) for this shape; 0 when none is needed. Pass at least this many bytes.
  */
 size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
@@ -129,8 +129,10 @@ size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
  *   M       1 <= M <= NVFP4WS_MAX_M.   N >= 1.   K >= 32, K % 32 == 0.
  *   Y       out: [M, N] row-major, device, 16-byte aligned; fp32 or bf16 per y_dtype.
  *   workspace, workspace_bytes  device scratch of at least
- *           nvfp4_gemm_workspace_bytes(M, N, K) bytes (may be NULL when that is 0).
- *           Contents on entry do not matter.
+ *           nvfp4_gemm_workspace_bytes(M, N, K) bytes, 16-byte aligned (may be NULL
+ *           when that is 0). It must be zero-filled before its first use. Every
+ *           completed call leaves the part that needs it zero again, so a buffer
+ *           can be reused across calls and shapes without clearing.
  * Returns NVFP4WS_OK, or INVALID_ARG / UNSUPPORTED / MISALIGNED / WORKSPACE / CUDA.
  */
 int nvfp4_gemm_skinny(const void* X, const uint8_t* q, const uint8_t* sf, const float* tensor_scale,
@@ -170,8 +172,8 @@ size_t lmhead_verify_workspace_bytes(int64_t M, int64_t N, int64_t K);
  *   argmax      out: int32 [M], device.
  *   accept_len  out: int32 [B], device.
  *   max_logit   out: fp32 [M], device, or NULL to skip (the winning logit, for tie diagnostics).
- *   workspace   device scratch of at least lmhead_verify_workspace_bytes(M, N, K) bytes.
- *               Contents on entry do not matter.
+ *   workspace   device scratch of at least lmhead_verify_workspace_bytes(M, N, K) bytes,
+ *               16-byte aligned, zero-filled before its first use (as for the GEMM).
  * Returns NVFP4WS_OK, or INVALID_ARG / UNSUPPORTED / MISALIGNED / WORKSPACE / CUDA.
  * Logits that are NaN make argmax undefined.
  */

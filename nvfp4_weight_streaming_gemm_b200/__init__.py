@@ -88,7 +88,7 @@ def _workspace(nbytes: int, device, workspace):
         return None
     if workspace is not None and workspace.numel() * workspace.element_size() >= nbytes:
         return workspace
-    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device)   # the library needs it zeroed once
 
 
 def gemm(X: torch.Tensor, q: torch.Tensor, sf: torch.Tensor, ts: torch.Tensor, out: torch.Tensor | None = None,

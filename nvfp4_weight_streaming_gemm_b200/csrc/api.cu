@@ -113,9 +113,8 @@ int nvfp4_pack(const float* W, int64_t N, int64_t K, uint8_t* q, uint8_t* sf, fl
 
 size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   if (M < 1 || N < 1 || K < 32) return 0;
-  int path = resolve_path(NVFP4WS_PATH_AUTO, M, K);
-  if (path == NVFP4WS_PATH_MMA) return mma_gemm_workspace_bytes(M, N, K);
-  return 0;
+  // enough for every path that supports the shape, so a forced path works too
+  return mma_supported(M, K) ? mma_gemm_workspace_bytes(M, N, K) : 0;
 }
 
 int nvfp4_gemm_skinny_path(const void* X, const uint8_t* q, const uint8_t* sf, const float* tensor_scale,
