@@ -62,8 +62,10 @@ typedef enum { NVFP4WS_Y_F32 = 0, NVFP4WS_Y_BF16 = 1 } nvfp4ws_ydtype;
 /* Kernel path of the GEMM. AUTO picks by M (the tuned crossover). The others force a path. */
 typedef enum {
   NVFP4WS_PATH_AUTO = 0,
-  NVFP4WS_PATH_GEMV = 1,          /* CUDA-core streaming GEMV: dequantises in registers */
-  NVFP4WS_PATH_MMA = 2            /* tcgen05 tensor-core path: TMA-staged, TMEM accumulators */
+  NVFP4WS_PATH_GEMV = 1,          /* CUDA-core streaming GEMV: dequantises in registers; rows staged by
+                                     cp.async.bulk when K % 256 == 0, else register prefetch */
+  NVFP4WS_PATH_MMA = 2,           /* tcgen05 tensor-core path: TMA-staged, TMEM accumulators */
+  NVFP4WS_PATH_GEMV_REGS = 3      /* the register-prefetch GEMV variant at any K (for comparisons) */
 } nvfp4ws_path;
 
 /* Human-readable name of a status code. Never NULL. Static storage. */

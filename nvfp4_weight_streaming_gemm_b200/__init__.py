@@ -18,7 +18,7 @@ import torch
 
 from . import _lib
 
-PATHS = {"auto": 0, "gemv": 1, "mma": 2}
+PATHS = {"auto": 0, "gemv": 1, "mma": 2, "gemv_regs": 3}
 STATUS_OK = 0
 
 

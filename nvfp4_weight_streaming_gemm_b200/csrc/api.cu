@@ -126,7 +126,7 @@ int nvfp4_gemm_skinny_path(const void* X, const uint8_t* q, const uint8_t* sf, c
   if (!aligned16(Y)) return set_error(NVFP4WS_ERR_MISALIGNED, "nvfp4_gemm_skinny: Y must be 16-byte aligned");
   if (y_dtype != NVFP4WS_Y_F32 && y_dtype != NVFP4WS_Y_BF16)
     return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_gemm_skinny: bad y_dtype %d", y_dtype);
-  if (path < NVFP4WS_PATH_AUTO || path > NVFP4WS_PATH_MMA)
+  if (path < NVFP4WS_PATH_AUTO || path > NVFP4WS_PATH_GEMV_REGS)
     return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_gemm_skinny: bad path %d", path);
   path = resolve_path(path, M, K);
   cudaStream_t s = (cudaStream_t)stream;
@@ -149,7 +149,7 @@ int nvfp4_gemm_skinny_path(const void* X, const uint8_t* q, const uint8_t* sf, c
   a.q = q; a.sf = sf; a.ts = tensor_scale;
   a.M = M; a.N = N; a.K = K;
   a.Y = Y; a.y_bf16 = (y_dtype == NVFP4WS_Y_BF16);
-  return launch_gemv(a, false, s);
+  return launch_gemv(a, false, path == NVFP4WS_PATH_GEMV_REGS, s);
 }
 
 int nvfp4_gemm_skinny(const void* X, const uint8_t* q, const uint8_t* sf, const float* tensor_scale, int64_t M,
@@ -159,9 +159,14 @@ int nvfp4_gemm_skinny(const void* X, const uint8_t* q, const uint8_t* sf, const 
                                 NVFP4WS_PATH_AUTO, stream);
 }
 
+// Largest partial-argmax grid of the two GEMV variants, so either fits the workspace.
+static int gemv_verify_grid(int64_t M, int64_t N, int64_t K) {
+  GemvPlan a = gemv_plan(M, N, K, false), b = gemv_plan(M, N, K, true);
+  return a.grid > b.grid ? a.grid : b.grid;
+}
+
 static size_t gemv_verify_workspace(int64_t M, int64_t N, int64_t K) {
-  GemvPlan p = gemv_plan(M, N, K);
-  return 2 * align_up((size_t)p.grid * (size_t)M * 4, 256);
+  return 2 * align_up((size_t)gemv_verify_grid(M, N, K) * (size_t)M * 4, 256);
 }
 
 size_t lmhead_verify_workspace_bytes(int64_t M, int64_t N, int64_t K) {
@@ -183,7 +188,7 @@ int lmhead_verify_argmax_accept_path(const void* X, const uint8_t* q, const uint
                      (long long)B * (D + 1));
   if (D > 0 && !drafts) return set_error(NVFP4WS_ERR_INVALID_ARG, "lmhead_verify: drafts is null");
   if (!argmax || !accept_len) return set_error(NVFP4WS_ERR_INVALID_ARG, "lmhead_verify: null output pointer");
-  if (path < NVFP4WS_PATH_AUTO || path > NVFP4WS_PATH_MMA)
+  if (path < NVFP4WS_PATH_AUTO || path > NVFP4WS_PATH_GEMV_REGS)
     return set_error(NVFP4WS_ERR_INVALID_ARG, "lmhead_verify: bad path %d", path);
   path = resolve_path(path, M, K);
   cudaStream_t s = (cudaStream_t)stream;
@@ -203,14 +208,16 @@ int lmhead_verify_argmax_accept_path(const void* X, const uint8_t* q, const uint
   if (workspace == nullptr || workspace_bytes < need)
     return set_error(NVFP4WS_ERR_WORKSPACE, "lmhead_verify: workspace needs %zu bytes", need);
   if (!aligned16(workspace)) return set_error(NVFP4WS_ERR_MISALIGNED, "lmhead_verify: workspace must be 16-byte aligned");
-  GemvPlan p = gemv_plan(M, N, K);
+  const bool regs_only = (path == NVFP4WS_PATH_GEMV_REGS);
+  GemvPlan p = gemv_plan(M, N, K, regs_only);
+  const int pgrid = gemv_verify_grid(M, N, K);
   GemvArgs a{};
   a.X = static_cast<const uint16_t*>(X);
   a.q = q; a.sf = sf; a.ts = tensor_scale;
   a.M = M; a.N = N; a.K = K;
   a.part_val = static_cast<float*>(workspace);
-  a.part_idx = reinterpret_cast<int*>(static_cast<char*>(workspace) + align_up((size_t)p.grid * M * 4, 256));
-  if (int e = launch_gemv(a, true, s)) return e;
+  a.part_idx = reinterpret_cast<int*>(static_cast<char*>(workspace) + align_up((size_t)pgrid * M * 4, 256));
+  if (int e = launch_gemv(a, true, regs_only, s)) return e;
   return launch_verify_stage2(a.part_val, a.part_idx, p.grid, (int)M, drafts, B, D, argmax, accept_len, max_logit, s);
 }
 

@@ -17,15 +17,21 @@ struct GemvArgs {
   int y_bf16;
   float* part_val;          // [grid, M] (verify mode)
   int* part_idx;            // [grid, M]
+  int verify;               // staged kernel: write argmax partials instead of Y
+  unsigned int* err;        // device error word (bounded waits)
 };
 
 struct GemvPlan {
   int mt, cpt, rows, threads, grid;
+  int staged;               // 1: bulk-copy-staged kernel (threads includes the producer warp)
+  int stages;
+  unsigned int stage_bytes;
+  size_t smem;
 };
 
-GemvPlan gemv_plan(long long M, long long N, long long K);
+GemvPlan gemv_plan(long long M, long long N, long long K, bool regs_only);
 bool gemv_supported(long long K);
-int launch_gemv(const GemvArgs& a, bool verify, cudaStream_t s);
+int launch_gemv(const GemvArgs& a, bool verify, bool regs_only, cudaStream_t s);
 
 int launch_pack(const float* W, long long N, long long K, uint8_t* q, uint8_t* sf, float* ts,
                 const float* ts_in, cudaStream_t s);

@@ -133,7 +133,7 @@ def test_gemm_tiny(nv):
     assert_rowwise(Y.cpu().numpy(), y_ref)
 
 
-@pytest.mark.parametrize("path", ["gemv", "auto"])
+@pytest.mark.parametrize("path", ["gemv", "gemv_regs", "auto"])
 @pytest.mark.parametrize("M,N,K", [(1, 1, 32), (1, 37, 96), (2, 100, 1024), (3, 1000, 64), (4, 513, 256),
                                    (5, 77, 17408), (7, 130, 5120), (17, 300, 512), (1, 64, 33 * 1024)])
 def test_gemm_ragged(nv, M, N, K, path):
@@ -327,3 +327,12 @@ def test_verify_mma_small_vocab(nv, B, D):
 def test_verify_mma_lmhead_slice(nv):
     W, x, Lstar = S.lmhead_inputs(N=S.VOCAB_SLICE, B=1)
     run_verify(nv, W, x, Lstar, S.DRAFT_LEN, path="mma")
+
+
+@pytest.mark.parametrize("path", ["gemv", "gemv_regs"])
+@pytest.mark.parametrize("B,D", [(1, 0), (1, 16), (2, 1)])
+def test_verify_gemv_variants(nv, path, B, D):
+    N, K = 2500, 1024
+    W, x = S.random_case(B * 13 + D, B * (D + 1), N, K, w_std=0.05)
+    Lstar = np.random.default_rng(B * 5 + D).integers(0, D + 1, size=B)
+    run_verify(nv, W, x, Lstar, D, path=path)
