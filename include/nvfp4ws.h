@@ -194,6 +194,31 @@ int lmhead_verify_argmax_accept_path(const void* X, const uint8_t* q, const uint
                                      nvfp4ws_stream_t stream);
 
 /*
+ * nvfp4_gemm_skinny_noalloc -- the tensor-core GEMM of nvfp4_gemm_skinny for callers
+ * that cannot allocate device memory and so cannot pass a workspace. Examples are a
+ * host that fixes its device-memory plan at start-up and forbids later allocation,
+ * code running under another framework's pooling allocator, and a plugin interface
+ * that provides no scratch buffer. (The pages have no counterpart: this is a
+ * packaging choice of this library.)
+ *
+ * Scratch comes from one built-in device array of 16 MiB. Every GPU that loads the
+ * library holds it until the process exits. The first call on a device looks up the
+ * array's address (cudaGetSymbolAddress), so make that first call before any
+ * stream capture. Every call shares the array and leaves its last contents in it.
+ * Each call clears the part that must start at zero (cudaMemsetAsync on `stream`).
+ * Calls whose work overlaps on the GPU race on the array.
+ * Nothing is allocated: no cudaMalloc, no cudaFree, no allocating library routine.
+ *
+ * Arguments and result are as for nvfp4_gemm_skinny, restricted to the tensor-core
+ * path: 1 <= M <= 128, K a positive multiple of 256, N >= 1.
+ * Returns NVFP4WS_ERR_UNSUPPORTED for a shape outside that range, or whose scratch
+ * (nvfp4_gemm_workspace_bytes) exceeds the 16 MiB array; otherwise as nvfp4_gemm_skinny.
+ */
+int nvfp4_gemm_skinny_noalloc(const void* X, const uint8_t* q, const uint8_t* sf,
+                              const float* tensor_scale, int64_t M, int64_t N, int64_t K,
+                              void* Y, int y_dtype, nvfp4ws_stream_t stream);
+
+/*
  * nvfp4ws_check -- synchronise `stream`, then read and clear the device error word
  * of the current device. Returns NVFP4WS_OK, NVFP4WS_ERR_DEVICE_TIMEOUT (a bounded
  * wait gave up; the detail is in nvfp4ws_last_error) or NVFP4WS_ERR_CUDA.

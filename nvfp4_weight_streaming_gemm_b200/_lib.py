@@ -31,6 +31,7 @@ SIGNATURES = {
     "lmhead_verify_argmax_accept_path": (ctypes.c_int, [c_p, c_p, c_p, c_p, c_i64, c_i64, c_i64, c_p, c_i32, c_i32,
                                                         c_p, c_p, c_p, c_p, c_sz, ctypes.c_int, c_p]),
     "nvfp4ws_check": (ctypes.c_int, [c_p]),
+    "nvfp4_gemm_skinny_noalloc": (ctypes.c_int, [c_p, c_p, c_p, c_p, c_i64, c_i64, c_i64, c_p, ctypes.c_int, c_p]),
     "nvfp4ws_kernel_launches": (ctypes.c_ulonglong, []),
 }
 

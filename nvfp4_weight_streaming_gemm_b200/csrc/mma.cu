@@ -556,6 +556,11 @@ size_t mma_gemm_workspace_bytes(long long M, long long N, long long K) {
   return align256((size_t)pl.tiles * 4) + align256((size_t)2 * pl.grid * M * kTileRows * 4);
 }
 
+size_t mma_gemm_counter_bytes(long long M, long long N, long long K) {
+  if (!mma_supported(M, K)) return 0;
+  return align256((size_t)plan_of(M, N, K).tiles * 4);
+}
+
 size_t mma_verify_workspace_bytes(long long M, long long N, long long K) {
   if (!mma_supported(M, K)) return 0;
   MmaPlan pl = plan_of(M, N, K);

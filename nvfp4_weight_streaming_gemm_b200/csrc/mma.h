@@ -10,6 +10,8 @@ namespace nvfp4ws {
 bool mma_supported(long long M, long long K);
 int mma_min_m();
 size_t mma_gemm_workspace_bytes(long long M, long long N, long long K);
+// Bytes of ticket counters at the start of the GEMM workspace (must be zero on entry).
+size_t mma_gemm_counter_bytes(long long M, long long N, long long K);
 size_t mma_verify_workspace_bytes(long long M, long long N, long long K);
 int launch_mma_gemm(const uint16_t* X, const uint8_t* q, const uint8_t* sf, const float* ts, long long M, long long N,
                     long long K, void* Y, int y_dtype, void* workspace, size_t workspace_bytes, cudaStream_t s);
