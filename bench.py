@@ -427,13 +427,21 @@ def run_sweep(args):
                 print(json.dumps({"shape": args.shape, "M": M, "path": path, "skipped": str(e)}), flush=True)
                 continue
             torch.cuda.synchronize()
+            # capture the launches in a CUDA graph: the replay times the GPU work and the
+            # launch gaps a graph-captured pass has, without host-side launch overhead
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for i in range(args.steps):
+                    q, sf, ts = copies[i % len(copies)]
+                    nv.gemm(X, q, sf, ts, out=Y, workspace=ws, path=path)
+            g.replay()
+            torch.cuda.synchronize()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
-            for i in range(args.steps):
-                q, sf, ts = copies[i % len(copies)]
-                nv.gemm(X, q, sf, ts, out=Y, workspace=ws, path=path)
+            g.replay()
             e1.record()
             torch.cuda.synchronize()
+            del g
             us = 1e3 * e0.elapsed_time(e1) / args.steps
             alg = weight_bytes(N, K) + M * K * 2 + M * N * 4
             print(json.dumps({"shape": args.shape, "N": N, "K": K, "M": M, "path": path, "us_per_launch": us,

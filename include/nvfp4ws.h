@@ -64,8 +64,11 @@ typedef enum {
   NVFP4WS_PATH_AUTO = 0,
   NVFP4WS_PATH_GEMV = 1,          /* CUDA-core streaming GEMV: dequantises in registers; rows staged by
                                      cp.async.bulk when K % 256 == 0, else register prefetch */
-  NVFP4WS_PATH_MMA = 2,           /* tcgen05 tensor-core path: TMA-staged, TMEM accumulators */
-  NVFP4WS_PATH_GEMV_REGS = 3      /* the register-prefetch GEMV variant at any K (for comparisons) */
+  NVFP4WS_PATH_MMA = 2,           /* tcgen05 tensor-core path: block-scaled kind::mxf4nvf4 on the packed
+                                     weights when M*5 <= 352 (activations as 5 residual NVFP4 terms),
+                                     else the f16 kernel below */
+  NVFP4WS_PATH_GEMV_REGS = 3,     /* the register-prefetch GEMV variant at any K (for comparisons) */
+  NVFP4WS_PATH_MMA_F16 = 4        /* tcgen05 kind::f16 on weights dequantised exactly to f16 in TMEM */
 } nvfp4ws_path;
 
 /* Human-readable name of a status code. Never NULL. Static storage. */
@@ -119,10 +122,16 @@ size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
  * (the pass is weight-bandwidth bound). M = 1 is plain decode, 17 is 16 drafts
  * + 1, and 68 is four sequences sharing one read.
  *
- * Arithmetic: each product x * (e2m1 * S) is exact. Sums are fp32. The result is
- * multiplied by ts once, in fp32. X is converted to f16 for the products; that
- * is exact for |x| in [2^-14, 65504]. Smaller magnitudes round to f16
- * subnormals (absolute error below 2^-25). Larger ones saturate to 65504.
+ * Arithmetic of the GEMV and f16 tensor-core paths: each product x * (e2m1 * S) is
+ * exact, sums are fp32, and the result is multiplied by ts once, in fp32. X is
+ * converted to f16 for the products; that is exact for |x| in [2^-14, 65504].
+ * Smaller magnitudes round to f16 subnormals (absolute error below 2^-25); larger
+ * ones saturate to 65504.
+ * Arithmetic of the block-scaled path (the default for 2 <= M <= 70 when K % 256 == 0):
+ * X is first written as 5 residual NVFP4 terms. Each is a per-row fp32 scale, an
+ * E4M3 scale per 16 and E2M1 codes; each term quantises what the previous ones left.
+ * The tensor core then multiplies the packed weights by those terms exactly, with
+ * fp32 accumulation. Measured error against the exact product is ~1e-5 of max|y|.
  *
  * Arguments
  *   X       bf16 [M, K] row-major, device, 16-byte aligned.

@@ -18,7 +18,7 @@ import torch
 
 from . import _lib
 
-PATHS = {"auto": 0, "gemv": 1, "mma": 2, "gemv_regs": 3}
+PATHS = {"auto": 0, "gemv": 1, "mma": 2, "gemv_regs": 3, "mma_f16": 4}
 STATUS_OK = 0
 
 

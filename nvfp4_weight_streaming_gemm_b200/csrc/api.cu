@@ -63,12 +63,31 @@ static int validate_gemm(const void* X, const uint8_t* q, const uint8_t* sf, con
   return NVFP4WS_OK;
 }
 
+// Kernel actually used for a request: MMA means the block-scaled kernel when the
+// shape allows it, else the f16 tensor-core kernel.
+enum { KPATH_GEMV = 1, KPATH_MXF4 = 2, KPATH_GEMV_REGS = 3, KPATH_MMA_F16 = 4, KPATH_NONE = 0 };
+
 static int resolve_path(int path, int64_t M, int64_t K) {
-  if (path == NVFP4WS_PATH_AUTO) {
-    if (mma_supported(M, K) && M >= mma_min_m()) return NVFP4WS_PATH_MMA;
-    return NVFP4WS_PATH_GEMV;
+  switch (path) {
+    case NVFP4WS_PATH_AUTO:
+      if (M >= mma_min_m() && mxf4_supported(M, K)) return KPATH_MXF4;
+      if (M >= mma_min_m() && mma_supported(M, K)) return KPATH_MMA_F16;
+      return KPATH_GEMV;
+    case NVFP4WS_PATH_GEMV: return KPATH_GEMV;
+    case NVFP4WS_PATH_GEMV_REGS: return KPATH_GEMV_REGS;
+    case NVFP4WS_PATH_MMA:
+      if (mxf4_supported(M, K)) return KPATH_MXF4;
+      return mma_supported(M, K) ? KPATH_MMA_F16 : KPATH_NONE;
+    case NVFP4WS_PATH_MMA_F16: return mma_supported(M, K) ? KPATH_MMA_F16 : KPATH_NONE;
+    default: return KPATH_NONE;
   }
-  return path;
+}
+
+// Workspace that serves every path supporting the shape.
+static size_t gemm_ws_any(int64_t M, int64_t N, int64_t K) {
+  size_t a = mma_supported(M, K) ? mma_gemm_workspace_bytes(M, N, K) : 0;
+  size_t b = mxf4_supported(M, K) ? mxf4_workspace_bytes(M, N, K) : 0;
+  return a > b ? a : b;
 }
 
 }  // namespace nvfp4ws
@@ -113,8 +132,7 @@ int nvfp4_pack(const float* W, int64_t N, int64_t K, uint8_t* q, uint8_t* sf, fl
 
 size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   if (M < 1 || N < 1 || K < 32) return 0;
-  // enough for every path that supports the shape, so a forced path works too
-  return mma_supported(M, K) ? mma_gemm_workspace_bytes(M, N, K) : 0;
+  return gemm_ws_any(M, N, K);   // enough for every path that supports the shape, so a forced path works too
 }
 
 int nvfp4_gemm_skinny_path(const void* X, const uint8_t* q, const uint8_t* sf, const float* tensor_scale,
@@ -126,14 +144,22 @@ int nvfp4_gemm_skinny_path(const void* X, const uint8_t* q, const uint8_t* sf, c
   if (!aligned16(Y)) return set_error(NVFP4WS_ERR_MISALIGNED, "nvfp4_gemm_skinny: Y must be 16-byte aligned");
   if (y_dtype != NVFP4WS_Y_F32 && y_dtype != NVFP4WS_Y_BF16)
     return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_gemm_skinny: bad y_dtype %d", y_dtype);
-  if (path < NVFP4WS_PATH_AUTO || path > NVFP4WS_PATH_GEMV_REGS)
+  if (path < NVFP4WS_PATH_AUTO || path > NVFP4WS_PATH_MMA_F16)
     return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_gemm_skinny: bad path %d", path);
-  path = resolve_path(path, M, K);
+  const int kp = resolve_path(path, M, K);
   cudaStream_t s = (cudaStream_t)stream;
-  if (path == NVFP4WS_PATH_MMA) {
-    if (!mma_supported(M, K))
-      return set_error(NVFP4WS_ERR_UNSUPPORTED, "nvfp4_gemm_skinny: MMA path does not support M=%lld K=%lld",
-                       (long long)M, (long long)K);
+  if (kp == KPATH_NONE)
+    return set_error(NVFP4WS_ERR_UNSUPPORTED, "nvfp4_gemm_skinny: the tensor-core paths need K %% 256 == 0 and "
+                     "M <= 128 (M=%lld K=%lld)", (long long)M, (long long)K);
+  if (kp == KPATH_MXF4) {
+    size_t need = mxf4_workspace_bytes(M, N, K);
+    if (workspace == nullptr || workspace_bytes < need)
+      return set_error(NVFP4WS_ERR_WORKSPACE, "nvfp4_gemm_skinny: workspace needs %zu bytes", need);
+    if (!aligned16(workspace))
+      return set_error(NVFP4WS_ERR_MISALIGNED, "nvfp4_gemm_skinny: workspace must be 16-byte aligned");
+    return launch_mxf4_gemm(static_cast<const uint16_t*>(X), q, sf, tensor_scale, M, N, K, Y, y_dtype, workspace, s);
+  }
+  if (kp == KPATH_MMA_F16) {
     size_t need = mma_gemm_workspace_bytes(M, N, K);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need))
       return set_error(NVFP4WS_ERR_WORKSPACE, "nvfp4_gemm_skinny: workspace needs %zu bytes", need);
@@ -149,7 +175,7 @@ int nvfp4_gemm_skinny_path(const void* X, const uint8_t* q, const uint8_t* sf, c
   a.q = q; a.sf = sf; a.ts = tensor_scale;
   a.M = M; a.N = N; a.K = K;
   a.Y = Y; a.y_bf16 = (y_dtype == NVFP4WS_Y_BF16);
-  return launch_gemv(a, false, path == NVFP4WS_PATH_GEMV_REGS, s);
+  return launch_gemv(a, false, kp == KPATH_GEMV_REGS, s);
 }
 
 int nvfp4_gemm_skinny(const void* X, const uint8_t* q, const uint8_t* sf, const float* tensor_scale, int64_t M,
@@ -173,7 +199,9 @@ size_t lmhead_verify_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   if (M < 1 || N < 1 || K < 32) return 0;
   size_t w = gemv_verify_workspace(M, N, K);
   size_t m = mma_supported(M, K) ? mma_verify_workspace_bytes(M, N, K) : 0;
-  return w > m ? w : m;
+  size_t x = mxf4_supported(M, K) ? mxf4_workspace_bytes(M, N, K) : 0;
+  if (m > w) w = m;
+  return x > w ? x : w;
 }
 
 int lmhead_verify_argmax_accept_path(const void* X, const uint8_t* q, const uint8_t* sf, const float* tensor_scale,
@@ -188,14 +216,22 @@ int lmhead_verify_argmax_accept_path(const void* X, const uint8_t* q, const uint
                      (long long)B * (D + 1));
   if (D > 0 && !drafts) return set_error(NVFP4WS_ERR_INVALID_ARG, "lmhead_verify: drafts is null");
   if (!argmax || !accept_len) return set_error(NVFP4WS_ERR_INVALID_ARG, "lmhead_verify: null output pointer");
-  if (path < NVFP4WS_PATH_AUTO || path > NVFP4WS_PATH_GEMV_REGS)
+  if (path < NVFP4WS_PATH_AUTO || path > NVFP4WS_PATH_MMA_F16)
     return set_error(NVFP4WS_ERR_INVALID_ARG, "lmhead_verify: bad path %d", path);
-  path = resolve_path(path, M, K);
+  const int kp = resolve_path(path, M, K);
   cudaStream_t s = (cudaStream_t)stream;
-  if (path == NVFP4WS_PATH_MMA) {
-    if (!mma_supported(M, K))
-      return set_error(NVFP4WS_ERR_UNSUPPORTED, "lmhead_verify: MMA path does not support M=%lld K=%lld",
-                       (long long)M, (long long)K);
+  if (kp == KPATH_NONE)
+    return set_error(NVFP4WS_ERR_UNSUPPORTED, "lmhead_verify: the tensor-core paths need K %% 256 == 0 and "
+                     "M <= 128 (M=%lld K=%lld)", (long long)M, (long long)K);
+  if (kp == KPATH_MXF4) {
+    size_t need = mxf4_workspace_bytes(M, N, K);
+    if (workspace == nullptr || workspace_bytes < need)
+      return set_error(NVFP4WS_ERR_WORKSPACE, "lmhead_verify: workspace needs %zu bytes", need);
+    if (!aligned16(workspace)) return set_error(NVFP4WS_ERR_MISALIGNED, "lmhead_verify: workspace must be 16-byte aligned");
+    return launch_mxf4_verify(static_cast<const uint16_t*>(X), q, sf, tensor_scale, M, N, K, drafts, B, D, argmax,
+                              accept_len, max_logit, workspace, s);
+  }
+  if (kp == KPATH_MMA_F16) {
     size_t need = mma_verify_workspace_bytes(M, N, K);
     if (workspace == nullptr || workspace_bytes < need)
       return set_error(NVFP4WS_ERR_WORKSPACE, "lmhead_verify: workspace needs %zu bytes", need);
@@ -208,7 +244,7 @@ int lmhead_verify_argmax_accept_path(const void* X, const uint8_t* q, const uint
   if (workspace == nullptr || workspace_bytes < need)
     return set_error(NVFP4WS_ERR_WORKSPACE, "lmhead_verify: workspace needs %zu bytes", need);
   if (!aligned16(workspace)) return set_error(NVFP4WS_ERR_MISALIGNED, "lmhead_verify: workspace must be 16-byte aligned");
-  const bool regs_only = (path == NVFP4WS_PATH_GEMV_REGS);
+  const bool regs_only = (kp == KPATH_GEMV_REGS);
   GemvPlan p = gemv_plan(M, N, K, regs_only);
   const int pgrid = gemv_verify_grid(M, N, K);
   GemvArgs a{};

@@ -255,12 +255,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t pol_w = policy_evict_first(), pol_x = policy_evict_last();
       const uint32_t tx = kNibBytes + kSfBytes + (uint32_t)npad * 512u;
       int issued = 0;
+      int s = 0, tile = (int)(u_begin / p.kch), kc = (int)(u_begin % p.kch);   // advanced incrementally below
+      uint32_t ph = 0;
       for (int i = 0; i < nunits; ++i) {
-        const int s = i % S;
-        const uint32_t ph = (uint32_t)(i / S) & 1u;
         if (!mbar_wait(bar_empty(s), ph ^ 1u, s_abort, p.err)) break;
-        const long long u = u_begin + i;
-        const int tile = (int)(u / p.kch), kc = (int)(u % p.kch);
         uint8_t* st = smem + (size_t)s * p.stage_bytes;
         mbar_arrive_expect_tx(bar_full(s), tx);
         tma_load_2d(smem_u32(st), &tm_q, kc * (kKC / 2), tile * kTileRows, bar_full(s), pol_w);
@@ -270,6 +268,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int a = 0; a < 4; ++a)
           tma_load_2d(smem_u32(st + kNibBytes + a * npad * 128), &tm_x, kc * kKC + a * 64, 0, bar_full(s), pol_x);
         issued = i + 1;
+        if (++kc == p.kch) { kc = 0; ++tile; }
+        if (++s == S) { s = 0; ph ^= 1u; }
       }
       if (*s_abort) {       // drain: wait (bounded) for every copy this thread issued
         for (int i = (issued > S ? issued - S : 0); i < issued; ++i) {
@@ -284,18 +284,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc = (1u << 4) | ((uint32_t)(npad >> 3) << 17) | ((uint32_t)(kTileRows >> 4) << 24);
       int seg = 0;
       bool ok = true;
+      int s = 0, kc = (int)(u_begin % p.kch);
+      uint32_t ph = 0;
       for (int i = 0; i < nunits && ok; ++i) {
-        const int s = i % S, g = i & 1;
-        const long long u = u_begin + i;
-        const int tile = (int)(u / p.kch);
-        const bool seg_first = (i == 0) || ((u - 1) / p.kch != tile);
-        const bool seg_last = (i == nunits - 1) || ((u + 1) / p.kch != tile);
+        const int g = i & 1;
+        const bool seg_first = (i == 0) || (kc == 0);
+        const bool seg_last = (i == nunits - 1) || (kc == p.kch - 1);
         const int ab = seg & 1;
         if (seg_first) {
           ok = mbar_wait(bar_accempty(ab), ((uint32_t)(seg >> 1) & 1u) ^ 1u, s_abort, p.err);
           if (!ok) break;
         }
-        ok = mbar_wait(bar_full(s), (uint32_t)(i / S) & 1u, s_abort, p.err) &&
+        ok = mbar_wait(bar_full(s), ph, s_abort, p.err) &&
              mbar_wait(bar_afull(g), (uint32_t)(i >> 1) & 1u, s_abort, p.err);
         if (!ok) break;
         tc_fence_after();
@@ -310,6 +310,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_commit(bar_empty(s));       // stage reusable once these MMAs retire
         tc_commit(bar_aempty(g));      // A buffer reusable
         if (seg_last) { tc_commit(bar_accfull(ab)); ++seg; }
+        if (++kc == p.kch) kc = 0;
+        if (++s == S) { s = 0; ph ^= 1u; }
       }
       tc_commit(bar_drain);            // completes when every MMA issued above has retired
       const unsigned long long t0 = globaltimer();
@@ -321,9 +323,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;                          // TMEM lane quarter
     const int r = q * 32 + lane;                     // row within the tile
     const int tg = threadIdx.x - (4 + 4 * g) * 32;   // 0..127 within the warpgroup
+    int s = g % S;
+    uint32_t ph = (uint32_t)(g / S) & 1u;
     for (int i = g; i < nunits; i += 2) {
-      const int s = i % S;
-      if (!mbar_wait(bar_full(s), (uint32_t)(i / S) & 1u, s_abort, p.err)) break;
+      if (i != g) {                                   // advance the ring position by two units
+        s += 2;
+        if (s >= S) { s -= S; ph ^= 1u; }
+      }
+      if (!mbar_wait(bar_full(s), ph, s_abort, p.err)) break;
       if (!mbar_wait(bar_aempty(g), ((uint32_t)(i >> 1) & 1u) ^ 1u, s_abort, p.err)) break;
       tc_fence_after();
       uint8_t* st = smem + (size_t)s * p.stage_bytes;
@@ -376,10 +383,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int et = threadIdx.x - 12 * 32;            // 0..127
     const float ts = *p.ts;
     int seg = 0;
+    int tile_it = (int)(u_begin / p.kch), kc_it = (int)(u_begin % p.kch);
     for (int i = 0; i < nunits; ++i) {
       const long long u = u_begin + i;
-      const int tile = (int)(u / p.kch);
-      const bool seg_last = (i == nunits - 1) || ((u + 1) / p.kch != tile);
+      const int tile = tile_it;
+      const bool seg_last = (i == nunits - 1) || (kc_it == p.kch - 1);
+      if (++kc_it == p.kch) { kc_it = 0; ++tile_it; }
       if (!seg_last) continue;
       // this segment covers units [seg_u0, u] of `tile`
       const long long tile_u0 = (long long)tile * p.kch, tile_u1 = tile_u0 + p.kch;
@@ -453,9 +462,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (b1 <= b0) continue;
             const int sl = (b0 >= tile_u0) ? 2 * cc : 2 * cc + 1;
             const float* src = p.partials + ((long long)sl * p.M) * kTileRows;
+            float v[16];   // all loads of the chunk first: one L2 round trip per contributor
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-              if (m0 + j < p.M) y[j] += __ldcg(src + (long long)(m0 + j) * kTileRows + row.rowl);
+              v[j] = (m0 + j < p.M) ? __ldcg(src + (long long)(m0 + j) * kTileRows + row.rowl) : 0.f;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) y[j] += v[j];
           }
 #pragma unroll
           for (int j = 0; j < 16; ++j) y[j] *= ts;

@@ -19,4 +19,15 @@ int launch_mma_verify(const uint16_t* X, const uint8_t* q, const uint8_t* sf, co
                       long long N, long long K, const int32_t* drafts, int B, int D, int32_t* argmax,
                       int32_t* accept_len, float* max_logit, void* workspace, cudaStream_t s);
 
+// Block-scaled (kind::mxf4nvf4) path: activations as kMxf4Terms residual NVFP4 terms.
+constexpr int kMxf4Terms = 5;
+bool mxf4_supported(long long M, long long K);
+size_t mxf4_workspace_bytes(long long M, long long N, long long K);
+size_t mxf4_counter_bytes(long long M, long long N, long long K);
+int launch_mxf4_gemm(const uint16_t* X, const uint8_t* q, const uint8_t* sf, const float* ts, long long M,
+                     long long N, long long K, void* Y, int y_dtype, void* workspace, cudaStream_t s);
+int launch_mxf4_verify(const uint16_t* X, const uint8_t* q, const uint8_t* sf, const float* ts, long long M,
+                       long long N, long long K, const int32_t* drafts, int B, int D, int32_t* argmax,
+                       int32_t* accept_len, float* max_logit, void* workspace, cudaStream_t s);
+
 }  // namespace nvfp4ws

@@ -37,15 +37,41 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait that lets the hardware suspend the thread until the phase completes, for
+// at most `hint_ns`. A waiting warp then issues no instructions, so it takes no
+// issue slots from the warps doing the work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ int ld_shared_volatile(const volatile int* p) {
+  int v;
+  asm volatile("ld.volatile.shared.b32 %0, [%1];" : "=r"(v) : "r"(smem_u32((const void*)p)));
+  return v;
+}
+
 // Bounded wait. Returns false (and records the error) when the limit passes or
-// another role of this CTA has already given up.
+// another role of this CTA has already given up. The thread sleeps inside
+// try_wait between checks.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           unsigned int* err) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait(bar, parity)) return true;          // fast path: the phase is usually complete
   const unsigned long long t0 = globaltimer();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
+#ifndef NVFP4WS_WAIT_HINT_NS
+#define NVFP4WS_WAIT_HINT_NS 0u
+#endif
+    if (NVFP4WS_WAIT_HINT_NS == 0u ? mbar_try_wait(bar, parity) : mbar_try_wait_sleep(bar, parity, NVFP4WS_WAIT_HINT_NS))
+      return true;
+    if (ld_shared_volatile(abort_flag)) return false;
     if (globaltimer() - t0 > kWaitLimitNs) {
       atomicOr(err, kDevErrWaitTimeout);
       *abort_flag = 1;

@@ -275,6 +275,7 @@ def test_verify_workspace_too_small(nv):
 
 # ------------------------------------------------------------------ tcgen05 MMA path
 
+@pytest.mark.parametrize("path", ["mma", "mma_f16"])
 @pytest.mark.parametrize("M,N,K", [
     (1, 128, 256),        # one tile, one chunk
     (2, 100, 1024),       # ragged N inside one tile
@@ -286,47 +287,53 @@ def test_verify_workspace_too_small(nv):
     (100, 513, 768),      # npad 112
     (128, 300, 1280),     # npad 128
 ])
-def test_gemm_mma(nv, M, N, K):
+def test_gemm_mma(nv, M, N, K, path):
+    """mma: block-scaled kind::mxf4nvf4 where M*5 <= 352, else f16; mma_f16: the exact f16 kernel."""
     W, x = S.random_case(M * 31 + N + K, M, N, K)
-    Y, y_ref = run_gemm(nv, W, x, path="mma")
+    Y, y_ref = run_gemm(nv, W, x, path=path)
     assert_rowwise(Y.cpu().numpy(), y_ref)
 
 
-def test_gemm_mma_bf16_and_deterministic(nv):
+@pytest.mark.parametrize("path", ["mma", "mma_f16"])
+def test_gemm_mma_bf16_and_deterministic(nv, path):
     W, x = S.random_case(61, 17, 2000, 4096)
     Wd = torch.from_numpy(W).cuda()
     q, sf, ts = nv.pack(Wd)
     X = to_dev_bf16(x)
     ws = torch.zeros(nv.gemm_workspace_bytes(17, 2000, 4096), dtype=torch.uint8, device="cuda")
-    Y1 = nv.gemm(X, q, sf, ts, workspace=ws, path="mma")
-    Y2 = nv.gemm(X, q, sf, ts, workspace=ws, path="mma")      # the workspace counters must be zero again
-    Yb = nv.gemm(X, q, sf, ts, workspace=ws, path="mma", y_dtype=torch.bfloat16)
+    Y1 = nv.gemm(X, q, sf, ts, workspace=ws, path=path)
+    Y2 = nv.gemm(X, q, sf, ts, workspace=ws, path=path)      # the workspace counters must be zero again
+    Yb = nv.gemm(X, q, sf, ts, workspace=ws, path=path, y_dtype=torch.bfloat16)
     torch.cuda.synchronize()
     assert torch.equal(Y1, Y2)
     assert torch.equal(Yb, Y1.to(torch.bfloat16))
     nv.check()
 
 
+@pytest.mark.parametrize("path", ["mma", "mma_f16"])
 @pytest.mark.parametrize("name", S.LAYER_ORDER)
 @pytest.mark.parametrize("M", [17, 68])
-def test_gemm_layer_shapes_mma(nv, name, M):
+def test_gemm_layer_shapes_mma(nv, name, M, path):
     """The M=17 and M=68 launch configurations of the bench at the 27B layer shapes."""
     W, x = S.layer(name, M=M)
-    Y, y_ref = run_gemm(nv, W, x, path="mma")
+    Y, y_ref = run_gemm(nv, W, x, path=path)
     assert_rowwise(Y.cpu().numpy(), y_ref)
 
 
+@pytest.mark.parametrize("path", ["mma", "mma_f16"])
 @pytest.mark.parametrize("B,D", [(1, 16), (4, 16), (2, 3)])
-def test_verify_mma_small_vocab(nv, B, D):
+def test_verify_mma_small_vocab(nv, B, D, path):
     N, K = 3000, 512
     W, x = S.random_case(B * 7 + D, B * (D + 1), N, K, w_std=0.05)
     Lstar = np.random.default_rng(B * 3 + D).integers(0, D + 1, size=B)
-    run_verify(nv, W, x, Lstar, D, path="mma")
+    run_verify(nv, W, x, Lstar, D, path=path)
 
 
-def test_verify_mma_lmhead_slice(nv):
-    W, x, Lstar = S.lmhead_inputs(N=S.VOCAB_SLICE, B=1)
-    run_verify(nv, W, x, Lstar, S.DRAFT_LEN, path="mma")
+@pytest.mark.parametrize("path", ["mma", "mma_f16"])
+@pytest.mark.parametrize("B", [1, 4])
+def test_verify_mma_lmhead_slice(nv, path, B):
+    W, x, Lstar = S.lmhead_inputs(N=S.VOCAB_SLICE, B=B)
+    run_verify(nv, W, x, Lstar, S.DRAFT_LEN, path=path)
 
 
 @pytest.mark.parametrize("path", ["gemv", "gemv_regs"])
