@@ -44,21 +44,23 @@ def weight_bytes(N: int, K: int) -> int:
     return N * K // 2 + N * K // 16
 
 
-def stack_weight_bytes() -> int:
-    return S.N_LAYERS * sum(weight_bytes(N, K) for (K, N) in (S.LAYER_SHAPES[n] for n in S.LAYER_ORDER))
+def stack_weight_bytes(layers: int = S.N_LAYERS) -> int:
+    return layers * sum(weight_bytes(N, K) for (K, N) in (S.LAYER_SHAPES[n] for n in S.LAYER_ORDER))
 
 
 def lmhead_weight_bytes() -> int:
     return weight_bytes(S.VOCAB, S.LMHEAD_K)
 
 
-def gemm_alg_bytes(M: int) -> int:
-    """Algorithmic bytes of the 192 GEMMs of one pass: W + scales + X (bf16) + Y (fp32)."""
+def pass_alg_bytes(M: int, layers: int = S.N_LAYERS) -> int:
+    """Algorithmic bytes of one pass: every weight and scale read once, every
+    activation row read once (bf16), every GEMM output written once (fp32), and the
+    lm_head's weights and activations (its logits never leave the chip)."""
     total = 0
     for name in S.LAYER_ORDER:
         K, N = S.LAYER_SHAPES[name]
         total += weight_bytes(N, K) + M * K * 2 + M * N * 4
-    return S.N_LAYERS * total
+    return layers * total + lmhead_weight_bytes() + M * S.LMHEAD_K * 2
 
 
 def measured_peaks():
@@ -127,10 +129,10 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- our arm
 
-def build_pass(nv, torch, dev, M_list, rank: int):
-    """Pack the 192-matrix stack and the lm_head on the GPU; make inputs for every M."""
+def build_pass(nv, torch, dev, M_list, rank: int, layers: int):
+    """Pack the layer stack and the lm_head on the GPU; make inputs for every M."""
     stack = []
-    for layer in range(S.N_LAYERS):
+    for layer in range(layers):
         for j, name in enumerate(S.LAYER_ORDER):
             K, N = S.LAYER_SHAPES[name]
             g = torch.Generator(device=dev)
@@ -149,9 +151,11 @@ def build_pass(nv, torch, dev, M_list, rank: int):
 
 
 class Pass:
-    """One M: per-layer X, outputs, workspaces, drafts, and the two captured graphs."""
+    """One M: per-layer X and Y, drafts, the weight pass (one persistent launch over the
+    192 GEMMs with the lm_head verify as its last problem), and, for comparison, the
+    chained per-GEMM launch sequence, each captured in a CUDA graph."""
 
-    def __init__(self, nv, torch, dev, stack, lm, M: int, rank: int):
+    def __init__(self, nv, torch, dev, stack, lm, M: int, rank: int, chain: bool):
         self.M = M
         self.torch = torch
         self.B = max(1, M // (S.DRAFT_LEN + 1)) if M >= S.DRAFT_LEN + 1 else 1
@@ -167,17 +171,22 @@ class Pass:
             self.xs.append(self.x_all[off: off + n])
             off += n
         self.ys = [torch.empty((M, N), dtype=torch.float32, device=dev) for (_, _, N, _, _, _) in stack]
-        wsb = max(nv.gemm_workspace_bytes(M, N, K) for (_, K, N, _, _, _) in stack)
-        self.gws = torch.zeros(max(wsb, 16), dtype=torch.uint8, device=dev)
-        self.vws = torch.zeros(max(nv.verify_workspace_bytes(M, S.VOCAB, S.LMHEAD_K), 16), dtype=torch.uint8,
-                               device=dev)
         self.argmax = torch.empty(M, dtype=torch.int32, device=dev)
         self.accept = torch.empty(self.B, dtype=torch.int32, device=dev)
         self.vmax = torch.empty(M, dtype=torch.float32, device=dev)
-        self.stack, self.lm, self.nv = stack, lm, nv
-        # drafts: the target's own greedy tokens for a prefix L* ~ U{0..D}, then random ids
         self.drafts = torch.zeros((self.B, self.D), dtype=torch.int32, device=dev)
-        self.verify_call()
+        self.stack, self.lm, self.nv, self.chain = stack, lm, nv, chain
+        problems = [(self.xs[i].view(M, K), q, sf, ts, self.ys[i]) for i, (_, K, _, q, sf, ts) in enumerate(stack)]
+        ql, sfl, tsl = lm
+        problems.append((self.xs[-1].view(M, S.LMHEAD_K), ql, sfl, tsl, None))
+        self.wp = nv.WeightPass(problems, M, verify=(self.drafts, self.argmax, self.accept, self.vmax))
+        if chain:
+            wsb = max(nv.gemm_workspace_bytes(M, N, K) for (_, K, N, _, _, _) in stack)
+            self.gws = torch.zeros(max(wsb, 16), dtype=torch.uint8, device=dev)
+            self.vws = torch.zeros(max(nv.verify_workspace_bytes(M, S.VOCAB, S.LMHEAD_K), 16), dtype=torch.uint8,
+                                   device=dev)
+        # drafts: the target's own greedy tokens for a prefix L* ~ U{0..D}, then random ids
+        self.wp.run()
         torch.cuda.synchronize()
         t = self.argmax.cpu().numpy()
         Lstar = np.random.default_rng(S.LMHEAD_L_SEED + M).integers(0, self.D + 1, size=self.B)
@@ -185,13 +194,13 @@ class Pass:
         self.drafts.copy_(torch.from_numpy(d))
         self.Lstar = Lstar
 
-    def gemm_calls(self):
+    def chain_gemm_calls(self):
         nv, M = self.nv, self.M
         for i, (name, K, N, q, sf, ts) in enumerate(self.stack):
             X = self.xs[i].view(M, K)
             nv.gemm(X, q, sf, ts, out=self.ys[i], workspace=self.gws)
 
-    def verify_call(self):
+    def chain_verify_call(self):
         q, sf, ts = self.lm
         X = self.xs[-1].view(self.M, S.LMHEAD_K)
         self.nv.verify(X, q, sf, ts, self.drafts, workspace=self.vws, out=(self.argmax, self.accept, self.vmax))
@@ -201,38 +210,37 @@ class Pass:
         lib = self.nv.lib()
         s = torch.cuda.Stream()
         s.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(s):           # warm both paths outside capture
-            self.gemm_calls()
-            self.verify_call()
+        with torch.cuda.stream(s):           # warm every path outside capture
+            self.wp.run()
+            if self.chain:
+                self.chain_gemm_calls()
+                self.chain_verify_call()
         torch.cuda.current_stream().wait_stream(s)
         torch.cuda.synchronize()
         n0 = lib.nvfp4ws_kernel_launches()
-        self.g_gemm = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(self.g_gemm):
-            self.gemm_calls()
-        n1 = lib.nvfp4ws_kernel_launches()
-        self.g_verify = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(self.g_verify):
-            self.verify_call()
-        n2 = lib.nvfp4ws_kernel_launches()
-        self.launches_gemm, self.launches_verify = n1 - n0, n2 - n1
+        self.g_pass = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.g_pass):
+            self.wp.run()
+        self.launches_pass = lib.nvfp4ws_kernel_launches() - n0
+        if self.chain:
+            self.g_chain = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(self.g_chain):
+                self.chain_gemm_calls()
+                self.chain_verify_call()
         torch.cuda.synchronize()
 
-    def run_timed(self, steps: int):
+    def run_timed(self, steps: int, graph=None):
         torch = self.torch
+        graph = graph or self.g_pass
         st = torch.cuda.current_stream()
-        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+        ev[0].record(st)
         for k in range(steps):
-            ev[k][0].record(st)
-            self.g_gemm.replay()
-            ev[k][1].record(st)
-            self.g_verify.replay()
-            ev[k][2].record(st)
+            graph.replay()
+            ev[k + 1].record(st)
         torch.cuda.synchronize()
-        gemm_ms = np.array([ev[k][0].elapsed_time(ev[k][1]) for k in range(steps)])
-        ver_ms = np.array([ev[k][1].elapsed_time(ev[k][2]) for k in range(steps)])
-        total_ms = ev[0][0].elapsed_time(ev[-1][2])
-        return total_ms, gemm_ms, ver_ms
+        per = np.array([ev[k].elapsed_time(ev[k + 1]) for k in range(steps)])
+        return ev[0].elapsed_time(ev[-1]), per
 
     def run_e2e(self, steps: int, x_host, out_host):
         """Host buffers: copy every input in (pinned -> device) and the verify result out, each step."""
@@ -242,8 +250,7 @@ class Pass:
         e0.record(st)
         for _ in range(steps):
             self.x_all.copy_(x_host, non_blocking=True)
-            self.g_gemm.replay()
-            self.g_verify.replay()
+            self.g_pass.replay()
             out_host[0][: self.M].copy_(self.argmax, non_blocking=True)
             out_host[1][: self.B].copy_(self.accept, non_blocking=True)
         e1.record(st)
@@ -292,19 +299,20 @@ def run_ours(args, rank, world, local_rank):
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
 
     M_list = [int(m) for m in args.ms.split(",")]
-    stack, lm = build_pass(nv, torch, dev, M_list, rank)
-    passes = {M: Pass(nv, torch, dev, stack, lm, M, rank) for M in M_list}
+    stack, lm = build_pass(nv, torch, dev, M_list, rank, args.layers)
+    head = 17 if 17 in M_list else M_list[0]
+    passes = {M: Pass(nv, torch, dev, stack, lm, M, rank, chain=not args.no_chain) for M in M_list}
     for p in passes.values():
         p.capture()
         for _ in range(args.warmup):
-            p.g_gemm.replay()
-            p.g_verify.replay()
+            p.g_pass.replay()
+            if p.chain:
+                p.g_chain.replay()
     torch.cuda.synchronize()
 
-    wbytes = stack_weight_bytes() + lmhead_weight_bytes()
+    wbytes = stack_weight_bytes(args.layers) + lmhead_weight_bytes()
     peak, peak_kind = measured_peaks()
     results, clocks = {}, None
-    head = 17 if 17 in passes else M_list[0]
     for M, p in passes.items():
         if dist:
             dist.barrier()
@@ -312,7 +320,7 @@ def run_ours(args, rank, world, local_rank):
         sampler = ClockSampler(local_rank) if (M == head and rank == 0) else None
         if sampler:
             sampler.start()
-        total_ms, gemm_ms, ver_ms = p.run_timed(args.steps)
+        total_ms, per = p.run_timed(args.steps)
         if sampler:
             clocks = sampler.stop()
         t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
@@ -320,20 +328,29 @@ def run_ours(args, rank, world, local_rank):
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total_ms = float(t.item())
         ms = total_ms / args.steps
-        gemm_avg = float(gemm_ms.mean())
-        results[M] = {
+        res = {
             "ms_per_pass": ms,
             "weight_gbs": world * wbytes / (ms * 1e-3) / 1e9,
             "pct_of_8tbs": 100.0 * wbytes / (ms * 1e-3) / 8e12,
             "passes_per_s": world * 1e3 / ms,
-            "gemm_ms": gemm_avg,
-            "gemm_gbs_alg": gemm_alg_bytes(M) / (gemm_avg * 1e-3) / 1e9,
-            "gemm_weight_gbs": stack_weight_bytes() / (gemm_avg * 1e-3) / 1e9,
-            "verify_ms": float(ver_ms.mean()),
-            "verify_weight_gbs": lmhead_weight_bytes() / (float(ver_ms.mean()) * 1e-3) / 1e9,
-            "launches_per_pass": p.launches_gemm + p.launches_verify,
+            "alg_gbs": pass_alg_bytes(M, args.layers) / (ms * 1e-3) / 1e9,
+            "ms_min": float(per.min()),
+            "ms_max": float(per.max()),
+            "launches_per_pass": p.launches_pass,
             "B": p.B, "D": p.D,
         }
+        if p.chain:
+            # the same work as 193 chained launches: each GEMM's activations are read only
+            # after the previous GEMM has finished, as a decode step's layer order requires
+            if dist:
+                dist.barrier()
+            chain_total, _ = p.run_timed(max(3, args.steps // 4), p.g_chain)
+            t = torch.tensor([chain_total / max(3, args.steps // 4)], dtype=torch.float64, device=dev)
+            if dist:
+                dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            res["chained_ms_per_pass"] = float(t.item())
+            res["chained_weight_gbs"] = world * wbytes / (float(t.item()) * 1e-3) / 1e9
+        results[M] = res
 
     # end to end through the public API with host buffers (headline M)
     p = passes[head]
@@ -370,9 +387,11 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "e2m1*e4m3 weights x f16 activations -> f32 accumulate",
+        "dtype": "e2m1*e4m3 weights x bf16 activations (as 5 residual e2m1*e4m3 terms) -> f32 accumulate",
         "data": "synthetic (seeded N(0,0.02) weights packed on the GPU, N(0,1) bf16 activations)",
-        "config": {"workload": WORKLOAD, "M": head, "B": r["B"], "D": r["D"], "layers": S.N_LAYERS,
+        "config": {"workload": WORKLOAD if args.layers == S.N_LAYERS else
+                   WORKLOAD.replace("64 x", f"{args.layers} x") + " (reduced stack: not the benchmark workload)",
+                   "M": head, "B": r["B"], "D": r["D"], "layers": args.layers,
                    "weight_bytes_per_pass": wbytes, "l2": "inputs larger than L2 (11.5 GB weight stack, no flush)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "pct_of_8tbs": r["pct_of_8tbs"],
@@ -380,9 +399,11 @@ def run_ours(args, rank, world, local_rank):
         "decode_steps_per_s": r["passes_per_s"],
         "per_m": {str(M): {k: (round(v, 4) if isinstance(v, float) else v) for k, v in res.items()}
                   for M, res in results.items()},
-        "roofline": {"bound": "hbm", "kernel": "GEMM launches of the pass (192 per pass)",
-                     "achieved": r["gemm_gbs_alg"], "peak": peak, "unit": "GB/s",
-                     "frac": r["gemm_gbs_alg"] / peak, "peak_kind": peak_kind, "traffic": args.traffic},
+        "roofline": {"bound": "hbm", "kernel": "pass_kernel (one launch per pass; the prep and verify-stage-2 "
+                                                 "launches are inside the timed step too)",
+                     "achieved": r["alg_gbs"], "peak": peak, "unit": "GB/s",
+                     "frac": r["alg_gbs"] / peak, "peak_kind": peak_kind, "traffic": args.traffic,
+                     "algorithmic_bytes_per_launch": pass_alg_bytes(head, args.layers)},
         "e2e": {"value": world * wbytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": r["launches_per_pass"] * args.steps,
@@ -491,6 +512,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--ms", default="17,1,68", help="comma list of M; the first 17 (else the first) is the headline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-chain", action="store_true", help="skip the chained per-GEMM comparison")
+    ap.add_argument("--layers", type=int, default=S.N_LAYERS,
+                    help="layers in the stack (the default is the 27B model's; fewer only for small profiling cases)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per GEMM pass from an ncu capture (reported as roofline.traffic)")

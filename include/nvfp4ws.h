@@ -203,6 +203,80 @@ int lmhead_verify_argmax_accept_path(const void* X, const uint8_t* q, const uint
                                      nvfp4ws_stream_t stream);
 
 /*
+ * Weight passes -- a list of independent GEMMs that share M, run by ONE persistent
+ * launch, optionally ending with the fused lm_head verify.
+ *
+ * Passage: "TandemLLM", "How it works" (one decode step reads every weight once)
+ * and the veloGB10 page, "Unique aspects: Engineered to the roofline" (the pass is
+ * bound by weight bandwidth). On B200 a single GEMM of a 27B layer streams for
+ * only 5-15 us, about as long as launching, filling and draining a persistent
+ * kernel. A pass therefore streams the whole list as one sequence of (problem,
+ * 128-row tile, 256-wide K-chunk) units, split evenly across the SMs: each SM's
+ * weight stream runs from its first unit to its last without a drain.
+ *
+ * Each problem computes Y_i[M, N_i] = X_i[M, K_i] . dequant(W_i)^T exactly as
+ * nvfp4_gemm_skinny's block-scaled path does (same arithmetic and error). The
+ * problems run concurrently in no particular order: no problem's X may be another
+ * problem's Y. With `verify` non-NULL the LAST problem is the lm_head: its Y is
+ * ignored and the step ends with the argmax over its N rows and the accept lengths,
+ * as lmhead_verify_argmax_accept computes them.
+ *
+ * nvfp4_pass_workspace_bytes -- device workspace for this list (verify_last != 0
+ *   when the last problem is the verify problem); 0 when the list is invalid.
+ * nvfp4_pass_init -- validates the list, lays out the workspace and writes the
+ *   problems' descriptors into it with a SYNCHRONOUS copy: call it at set-up, not
+ *   while a stream is being captured, and not while a run on this workspace is in
+ *   flight. The workspace must be zero-filled before the first run; every run
+ *   leaves the part that needs it zero again. The pointers given (X, W, Y, verify
+ *   buffers, workspace) are baked into the pass: later runs read and write the
+ *   same buffers, so refill X in place between runs.
+ * nvfp4_pass_run -- enqueues the pass on `stream` (3 kernels with verify, else 2).
+ *   It can be captured in a CUDA graph.
+ *
+ * Arguments
+ *   problems[i]   X: bf16 [M, K], device, 16-byte aligned.  q, sf, tensor_scale: as
+ *                 produced by nvfp4_pack.  N >= 1.  K a multiple of 256, 256 <= K <=
+ *                 32768.  Y: [M, N] fp32 or bf16 per y_dtype (ignored for the verify
+ *                 problem).
+ *   count         >= 1.
+ *   M             1 <= M <= 70 (the block-scaled path's limit).
+ *   verify        NULL, or the verify buffers: M must equal B * (D + 1); drafts int32
+ *                 [B, D] (may be NULL when D == 0); argmax int32 [M]; accept_len int32
+ *                 [B]; max_logit fp32 [M] or NULL.
+ *   pass          caller-owned host state, filled by nvfp4_pass_init.
+ * Returns NVFP4WS_OK, or INVALID_ARG / UNSUPPORTED / MISALIGNED / WORKSPACE / CUDA.
+ */
+typedef struct nvfp4_gemm_problem {
+  const void* X;
+  const uint8_t* q;
+  const uint8_t* sf;
+  const float* tensor_scale;
+  int64_t N;
+  int64_t K;
+  void* Y;
+  int32_t y_dtype;
+} nvfp4_gemm_problem;
+
+typedef struct nvfp4_verify_spec {
+  const int32_t* drafts;
+  int32_t B;
+  int32_t D;
+  int32_t* argmax;
+  int32_t* accept_len;
+  float* max_logit;
+} nvfp4_verify_spec;
+
+typedef struct nvfp4_pass {
+  uint64_t opaque[32];
+} nvfp4_pass;
+
+size_t nvfp4_pass_workspace_bytes(const nvfp4_gemm_problem* problems, int32_t count, int64_t M,
+                                  int32_t verify_last);
+int nvfp4_pass_init(nvfp4_pass* pass, const nvfp4_gemm_problem* problems, int32_t count, int64_t M,
+                    const nvfp4_verify_spec* verify, void* workspace, size_t workspace_bytes);
+int nvfp4_pass_run(const nvfp4_pass* pass, nvfp4ws_stream_t stream);
+
+/*
  * nvfp4_gemm_skinny_noalloc -- the tensor-core GEMM of nvfp4_gemm_skinny for callers
  * that cannot allocate device memory and so cannot pass a workspace. Examples are a
  * host that fixes its device-memory plan at start-up and forbids later allocation,

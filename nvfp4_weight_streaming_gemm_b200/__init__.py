@@ -8,6 +8,8 @@ torch, and passes raw device pointers and the current CUDA stream.
     q, sf, ts = pack(W)                        # fp32 [N, K] -> NVFP4
     Y = gemm(X, q, sf, ts)                     # bf16 [M, K] -> fp32 [M, N]
     t, L, vmax = verify(X, q, sf, ts, drafts)  # fused lm_head argmax + accept length
+    p = WeightPass([(X_i, q_i, sf_i, ts_i, Y_i), ...], M, verify=...)   # a whole list, one launch
+    p.run()
 """
 
 from __future__ import annotations
@@ -142,3 +144,60 @@ def verify(X: torch.Tensor, q: torch.Tensor, sf: torch.Tensor, ts: torch.Tensor,
 def check(stream=None):
     """Synchronise and report a device-side bounded-wait failure, if any."""
     _check(lib().nvfp4ws_check(_stream(stream)), "nvfp4ws_check")
+
+
+class WeightPass:
+    """A list of independent GEMMs sharing M, run by one persistent launch (``nvfp4_pass_*``).
+
+    ``problems`` is a list of ``(X, q, sf, ts, Y)``: X bf16 [M, K], the packed weight,
+    and Y fp32 or bf16 [M, N]. With ``verify=(drafts, argmax, accept_len, max_logit)``
+    the last problem is the lm_head: its Y may be None, and each run ends with the
+    argmax over its rows and the accept lengths. Every tensor is referenced by address:
+    keep them alive and refill X in place between runs.
+    """
+
+    def __init__(self, problems, M: int, verify=None, workspace: torch.Tensor | None = None):
+        L = _lib
+        n = len(problems)
+        self._keep = []
+        arr = (L.GemmProblem * n)()
+        for i, (X, q, sf, ts, Y) in enumerate(problems):
+            _need_cuda(X, "X", torch.bfloat16)
+            _need_cuda(q, "q", torch.uint8)
+            _need_cuda(sf, "sf", torch.uint8)
+            if X.shape[0] != M:
+                raise ValueError(f"problem {i}: X has {X.shape[0]} rows, expected M={M}")
+            K = X.shape[1]
+            N = q.shape[0]
+            if q.shape[1] * 2 != K or sf.shape != (N, K // 16):
+                raise ValueError(f"problem {i}: q / sf shapes do not match X")
+            yd = 0
+            if Y is not None:
+                _need_cuda(Y, "Y")
+                if Y.shape != (M, N):
+                    raise ValueError(f"problem {i}: Y must be [{M}, {N}]")
+                yd = {torch.float32: 0, torch.bfloat16: 1}[Y.dtype]
+            arr[i] = L.GemmProblem(_ptr(X), _ptr(q), _ptr(sf), _ptr(ts), N, K, _ptr(Y), yd)
+            self._keep.extend([X, q, sf, ts, Y])
+        vs = None
+        if verify is not None:
+            drafts, amax, acc, vmax = verify
+            _need_cuda(drafts, "drafts", torch.int32)
+            B, D = drafts.shape
+            vs = L.VerifySpec(_ptr(drafts) if drafts.numel() else None, B, D, _ptr(amax), _ptr(acc), _ptr(vmax))
+            self._keep.extend([drafts, amax, acc, vmax])
+        nbytes = int(lib().nvfp4_pass_workspace_bytes(arr, n, M, 1 if verify is not None else 0))
+        if nbytes == 0:
+            raise NVFP4WSError(1, "nvfp4_pass_workspace_bytes")
+        dev = problems[0][0].device
+        self.workspace = _workspace(nbytes, dev, workspace)
+        self.workspace_bytes = nbytes
+        self.state = L.PassState()
+        _check(lib().nvfp4_pass_init(ctypes.byref(self.state), arr, n, M,
+                                     ctypes.byref(vs) if vs is not None else None, _ptr(self.workspace), nbytes),
+               "nvfp4_pass_init")
+        self.M = M
+        self.count = n
+
+    def run(self, stream=None):
+        _check(lib().nvfp4_pass_run(ctypes.byref(self.state), _stream(stream)), "nvfp4_pass_run")

@@ -14,6 +14,24 @@ LIB_PATH = os.path.join(HERE, "libnvfp4ws.so")
 
 c_i64, c_i32, c_p, c_sz = ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t
 
+
+class GemmProblem(ctypes.Structure):
+    """nvfp4_gemm_problem: one GEMM of a weight pass."""
+    _fields_ = [("X", c_p), ("q", c_p), ("sf", c_p), ("tensor_scale", c_p), ("N", c_i64), ("K", c_i64),
+                ("Y", c_p), ("y_dtype", c_i32)]
+
+
+class VerifySpec(ctypes.Structure):
+    """nvfp4_verify_spec: the verify buffers of a pass whose last problem is the lm_head."""
+    _fields_ = [("drafts", c_p), ("B", c_i32), ("D", c_i32), ("argmax", c_p), ("accept_len", c_p),
+                ("max_logit", c_p)]
+
+
+class PassState(ctypes.Structure):
+    """nvfp4_pass: caller-owned host state of an initialised pass."""
+    _fields_ = [("opaque", ctypes.c_uint64 * 32)]
+
+
 # name -> (restype, argtypes)
 SIGNATURES = {
     "nvfp4ws_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -33,6 +51,10 @@ SIGNATURES = {
     "nvfp4ws_check": (ctypes.c_int, [c_p]),
     "nvfp4_gemm_skinny_noalloc": (ctypes.c_int, [c_p, c_p, c_p, c_p, c_i64, c_i64, c_i64, c_p, ctypes.c_int, c_p]),
     "nvfp4ws_kernel_launches": (ctypes.c_ulonglong, []),
+    "nvfp4_pass_workspace_bytes": (c_sz, [ctypes.POINTER(GemmProblem), c_i32, c_i64, c_i32]),
+    "nvfp4_pass_init": (ctypes.c_int, [ctypes.POINTER(PassState), ctypes.POINTER(GemmProblem), c_i32, c_i64,
+                                       ctypes.POINTER(VerifySpec), c_p, c_sz]),
+    "nvfp4_pass_run": (ctypes.c_int, [ctypes.POINTER(PassState), c_p]),
 }
 
 _lib = None

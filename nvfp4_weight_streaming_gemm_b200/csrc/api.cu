@@ -9,6 +9,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <vector>
 
 namespace nvfp4ws {
 
@@ -263,6 +264,71 @@ int lmhead_verify_argmax_accept(const void* X, const uint8_t* q, const uint8_t* 
                                 size_t workspace_bytes, nvfp4ws_stream_t stream) {
   return lmhead_verify_argmax_accept_path(X, q, sf, tensor_scale, M, N, K, drafts, B, D, argmax, accept_len,
                                           max_logit, workspace, workspace_bytes, NVFP4WS_PATH_AUTO, stream);
+}
+
+// ------------------------------------------------------------------ weight passes
+
+static int to_host_problems(const nvfp4_gemm_problem* problems, int32_t count, int64_t M, int verify_last,
+                            std::vector<MxHostProblem>* out, const char* who) {
+  if (!problems || count < 1) return set_error(NVFP4WS_ERR_INVALID_ARG, "%s: need count >= 1 problems", who);
+  if (M < 1 || !mxf4_supported(M, 256))
+    return set_error(NVFP4WS_ERR_UNSUPPORTED, "%s: M=%lld outside 1..%d", who, (long long)M, 352 / kMxf4Terms);
+  out->clear();
+  for (int32_t i = 0; i < count; ++i) {
+    const nvfp4_gemm_problem& p = problems[i];
+    const bool v = verify_last && i == count - 1;
+    if (int e = validate_gemm(p.X, p.q, p.sf, p.tensor_scale, M, p.N, p.K, who)) return e;
+    if (!mxf4_supported(M, p.K))
+      return set_error(NVFP4WS_ERR_UNSUPPORTED, "%s: problem %d: K=%lld must be a multiple of 256 in [256, 32768]",
+                       who, i, (long long)p.K);
+    if (!v) {
+      if (!p.Y) return set_error(NVFP4WS_ERR_INVALID_ARG, "%s: problem %d: Y is null", who, i);
+      if (!aligned16(p.Y)) return set_error(NVFP4WS_ERR_MISALIGNED, "%s: problem %d: Y must be 16-byte aligned", who, i);
+      if (p.y_dtype != NVFP4WS_Y_F32 && p.y_dtype != NVFP4WS_Y_BF16)
+        return set_error(NVFP4WS_ERR_INVALID_ARG, "%s: problem %d: bad y_dtype %d", who, i, p.y_dtype);
+    }
+    MxHostProblem h{static_cast<const uint16_t*>(p.X), p.q, p.sf, p.tensor_scale, p.N, p.K,
+                    v ? nullptr : p.Y, (!v && p.y_dtype == NVFP4WS_Y_BF16) ? 1 : 0, v ? 1 : 0};
+    out->push_back(h);
+  }
+  return NVFP4WS_OK;
+}
+
+size_t nvfp4_pass_workspace_bytes(const nvfp4_gemm_problem* problems, int32_t count, int64_t M, int32_t verify_last) {
+  std::vector<MxHostProblem> hp;
+  if (to_host_problems(problems, count, M, verify_last, &hp, "nvfp4_pass_workspace_bytes") != NVFP4WS_OK) return 0;
+  return mxf4_pass_workspace_bytes(hp.data(), count, M);
+}
+
+int nvfp4_pass_init(nvfp4_pass* pass, const nvfp4_gemm_problem* problems, int32_t count, int64_t M,
+                    const nvfp4_verify_spec* verify, void* workspace, size_t workspace_bytes) {
+  g_last_error[0] = 0;
+  static_assert(sizeof(nvfp4_pass) >= kMxPassStateBytes, "nvfp4_pass is too small for the pass state");
+  if (!pass) return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_pass_init: pass is null");
+  std::memset(pass, 0, sizeof(nvfp4_pass));
+  std::vector<MxHostProblem> hp;
+  if (int e = to_host_problems(problems, count, M, verify != nullptr, &hp, "nvfp4_pass_init")) return e;
+  MxVerifySpec vs{};
+  if (verify) {
+    if (verify->B < 1 || verify->D < 0)
+      return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_pass_init: verify needs B >= 1 and D >= 0");
+    if ((int64_t)verify->B * (verify->D + 1) != M)
+      return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_pass_init: M=%lld must equal B*(D+1)=%lld", (long long)M,
+                       (long long)verify->B * (verify->D + 1));
+    if (verify->D > 0 && !verify->drafts) return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_pass_init: drafts is null");
+    if (!verify->argmax || !verify->accept_len)
+      return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_pass_init: null verify output pointer");
+    vs = MxVerifySpec{verify->drafts, verify->B, verify->D, verify->argmax, verify->accept_len, verify->max_logit};
+  }
+  if (!workspace) return set_error(NVFP4WS_ERR_WORKSPACE, "nvfp4_pass_init: workspace is null");
+  if (!aligned16(workspace)) return set_error(NVFP4WS_ERR_MISALIGNED, "nvfp4_pass_init: workspace must be 16-byte aligned");
+  return mxf4_pass_init(pass->opaque, hp.data(), count, M, verify ? &vs : nullptr, workspace, workspace_bytes);
+}
+
+int nvfp4_pass_run(const nvfp4_pass* pass, nvfp4ws_stream_t stream) {
+  g_last_error[0] = 0;
+  if (!pass) return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_pass_run: pass is null");
+  return mxf4_pass_run(pass->opaque, (cudaStream_t)stream);
 }
 
 int nvfp4ws_check(nvfp4ws_stream_t stream) {

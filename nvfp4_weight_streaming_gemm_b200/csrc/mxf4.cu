@@ -1,4 +1,5 @@
-// Block-scaled tensor-core path: tcgen05.mma kind::mxf4nvf4 on packed NVFP4 weights.
+// Block-scaled tensor-core path: tcgen05.mma kind::mxf4nvf4 on packed NVFP4 weights,
+// for one GEMM or for a whole list of them (a weight pass) in one persistent launch.
 //
 // Why. On B200 a tcgen05.mma kind::f16 instruction (M=128, K=16) costs ~70-96 SM
 // cycles for every N up to 128 (measured). So a path that dequantises W to f16
@@ -8,36 +9,42 @@
 // instruction, with no per-element work on the CUDA cores at all.
 //
 // The catch is that both operands must be NVFP4. The activations are bf16, so
-// they are represented as T residual NVFP4 terms:
-//   r_0 = x;  for t < T:  g_t = amax|r_t| / 2688,  S_t = E4M3(amax_block(r_t) / (6 g_t)),
-//                          c_t = E2M1(r_t / (S_t g_t)),  r_{t+1} = r_t - c_t S_t g_t
-// so x = sum_t g_t S_t c_t + r_T. Every term is an ordinary two-level NVFP4
-// quantisation of the residual left by the previous ones. Each term cuts the
-// error about 10x. With T = 5 the GEMM matches the exact float64 result to ~1e-5
-// relative, and logits to ~4e-5 absolute. The terms are extra B columns (token m,
-// term t -> column m*T + t). The epilogue folds them: y[m] = ts * sum_t g_t acc[m*T+t].
+// they are represented as T residual NVFP4 terms with one row amax:
+//   g_0 = amax|x| / 2688,  g_t = g_0 / 4^t,  r_0 = x,  for t < T:
+//       S_t = E4M3(amax_block(r_t) / (6 g_t)),  c_t = E2M1(r_t / (S_t g_t)),  r_{t+1} = r_t - c_t S_t g_t
+// so x = sum_t g_t S_t c_t + r_T. One E2M1 code with its E4M3 block scale leaves
+// at most ~0.18 of the block magnitude behind, so r_t stays below 6 * 448 * g_t
+// and every S_t fits E4M3. Each term cuts the error about 10x; with T = 5 the
+// GEMM matches the exact float64 result to ~1e-5 relative and logits to ~5e-5
+// absolute. The terms are extra B rows (token m, term t -> row m*T + t). The
+// epilogue folds them: y[m] = ts * sum_t g_t acc[m*T+t].
 //
 // Kernels.
-//   x_prep_kernel   one CTA per activation row: the T-term decomposition into the
-//                   workspace (codes [M*T, K/2], scales [M*T, K/16], g [M, T]). It
-//                   triggers dependent launch at once, so the GEMM's prologue and
-//                   first weight loads overlap it.
-//   mxf4_kernel     one persistent CTA per SM, 12 warps:
-//     warp 0        TMA producer: the W tile (128 rows x 128 B nibbles, SW128; 128 x 16 B
-//                   scales) and the X-term tile (codes SW128, scales) per 256-wide
-//                   K-chunk. The first stages' weight loads are issued before waiting
-//                   on x_prep.
+//   x_prep_kernel   one CTA per (activation row, problem): the T-term decomposition,
+//                   written as per-K-chunk images that are byte-for-byte the shared
+//                   memory operand (128-byte-swizzled code rows, then 16 scale bytes
+//                   per row). The GEMM fetches each with ONE contiguous bulk copy:
+//                   measured on B200, a 2D tensor box gathering R rows of 128 B from
+//                   L2 cuts the concurrent HBM weight stream by 11% (R=16) to 50%
+//                   (R=352); a contiguous bulk copy of the same bytes costs ~3%.
+//   pass_kernel     one persistent CTA per SM, 12 warps, over the concatenated
+//                   (problem, 128-row tile, 256-wide K-chunk) units of all problems,
+//                   split evenly across CTAs (stream-K). Tiles split between CTAs
+//                   occur only at the G-1 CTA range boundaries of the whole list.
+//     warp 0        TMA producer: the W tile (128 rows x 128 B nibbles, SW128) and its
+//                   128 x 16 B scales (2D tensor loads), then the activation image
+//                   (1D bulk). The first stages' weight loads are issued before waiting
+//                   on the prep kernel.
 //     warp 1        TMEM allocator and MMA issuer: 4 K-steps x B-tiles of
-//                   tcgen05.mma kind::mxf4nvf4.block_scale.block16 per chunk.
-//     warps 4-7     scale-factor warpgroup: copies the chunk's W and X block scales
+//                   tcgen05.mma kind::mxf4nvf4.block_scale.block16 per unit.
+//     warps 4-7     scale-factor warpgroup: copies the unit's W and X block scales
 //                   from shared memory into TMEM in the layout the MMA reads (the 4
 //                   scales of row m0 + 32*j in column j of lane m0, replicated over the
 //                   four lane quarters).
 //     warps 8-11    epilogue: tcgen05.ld of the accumulators, fold of the terms,
-//                   x ts, then Y or the per-tile argmax. Split tiles are finished as on
-//                   the f16 path.
-// Scheduling (stream-K over (tile, chunk) units, last-arriver fixed-order split-tile
-// reduction) and bounded waits are the same as on the f16 path.
+//                   x ts, then Y or the per-tile argmax of a verify problem. The last
+//                   CTA to finish a split tile sums the partials in CTA order.
+// Every wait is bounded (see sync.cuh); a timeout sets the device error word.
 #include "common.cuh"
 #include "kernels.h"
 #include "mma.h"
@@ -49,16 +56,18 @@
 #include <algorithm>
 #include <climits>
 #include <cmath>
+#include <cstring>
+#include <vector>
 
 namespace nvfp4ws {
 namespace mxk {
 
-// Optional per-unit timeline of CTA 0 (clock64 at each hand-off), for pipeline
-// analysis. Compiled out unless NVFP4WS_TRACE is defined; it changes no work.
+// Optional timelines for pipeline analysis, compiled out unless NVFP4WS_TRACE is
+// defined; they change no work. g_trace: clock64 per unit of CTA 0 at each hand-off.
+// g_cta_trace: per-CTA global-timer events (ns): [cta][event].
 #ifdef NVFP4WS_TRACE
 __device__ unsigned long long g_trace[16 * 64];
 #define MX_TRACE(f, i) do { if (blockIdx.x == 0 && (i) < 64) g_trace[(f) * 64 + (i)] = clock64(); } while (0)
-// per-CTA events on the global timer (ns): [cta][event]
 __device__ unsigned long long g_cta_trace[256 * 16];
 #define MX_CTA(e) do { if (blockIdx.x < 256) g_cta_trace[blockIdx.x * 16 + (e)] = globaltimer(); } while (0)
 #else
@@ -68,24 +77,65 @@ __device__ unsigned long long g_cta_trace[256 * 16];
 
 constexpr int kThreads = 384;
 constexpr int kTileRows = 128;
-constexpr int kKC = 256;
-constexpr int kNibBytes = kTileRows * kKC / 2;     // 16 KB
-constexpr int kSfBytes = kTileRows * kKC / 16;     // 2 KB
+constexpr int kKC = 256;                           // one K-chunk; a unit is 1 or 2 chunks (Geom::ku)
+constexpr int kNibBytes = kTileRows * kKC / 2;     // 16 KB of W codes per chunk (one SW128 block)
+constexpr int kSfBytes = kTileRows * kKC / 16;     // 2 KB of W scales per chunk
+constexpr uint32_t kWChunk = kNibBytes + kSfBytes; // weight bytes per chunk (1024-aligned)
+constexpr int kMaxStages = 12;
 constexpr int kMaxB = 352;                         // B rows (tokens x terms) the TMEM budget allows
 constexpr size_t kTailBytes = 8192;
+constexpr int kPrepThreads = 512;                  // K <= 512 * 4 * 16 = 32768 with 4 blocks per thread
+constexpr int kMaxSfBufs = 8;
 
-// ------------------------------------------------------------------ activation decomposition
-
-struct XPrepArgs {
-  const uint16_t* X;
-  int M, T;
-  long long K;
-  uint8_t* xq;     // [M*T, K/2]
-  uint8_t* xs;     // [M*T, K/16]
-  float* xg;       // [M, T]
+// One GEMM of a launch. Lives in device memory (a pass) or in the kernel's parameter
+// space (a single GEMM); the tensor maps are read by TMA from wherever it lives.
+struct alignas(64) Problem {
+  CUtensorMap tm_q;        // W codes [N, K/2] u8, box 128 B x 128 rows, 128-byte swizzle
+  CUtensorMap tm_sf;       // W scales [N, K/16] u8, box 16 B x 128 rows
+  const uint16_t* X;       // [M, K] bf16
+  uint8_t* ximg;           // [K/256][img_stride] activation-term images, one per 256-wide chunk
+  float* xg;               // [M*T] per-term global scales
+  const float* ts;         // W tensor scale (device)
+  void* Y;                 // [M, N] f32 or bf16 (unused by a verify problem)
+  float* part_val;         // verify problem: per-tile row maxima [tiles][M]
+  int* part_idx;           //                 and their indices
+  long long N;
+  unsigned int unit0;      // first unit of this problem in the launch's unit numbering
+  int K, kch, tiles, y_bf16, verify;
 };
 
-constexpr int kPrepThreads = 512;                 // K <= 512 * 4 * 16 = 32768 with 4 blocks per thread
+// What depends on M alone, shared by every problem of a launch.
+struct Geom {
+  int M, T, nb, nbt, nb_tile, nsfb;
+  int ku;                  // 256-wide K-chunks per unit (1 or 2)
+  uint32_t img_bytes;      // one chunk's image: nbt*nb_tile rows x (128 B codes + 16 B scales)
+  uint32_t img_stride;     // images are 1024-byte aligned (the MMA operand's swizzle atom)
+  uint32_t img_xs_off;     // offset of the scale rows in an image
+  uint32_t wbytes;         // weight bytes of a unit: ku x (codes + scales)
+};
+
+struct PassParams {
+  Geom g;
+  const Problem* probs;    // device array, or nullptr: the single problem passed by value
+  int nprob;
+  // Waves: consecutive problems whose activation images fit L2 together. Units of wave w
+  // are [wave_u0[w], wave_u0[w+1]); each is split evenly across the CTAs (stream-K), so
+  // at any time every CTA works on the same few problems. nullptr: one wave of `units`.
+  const uint32_t* wave_u0; // [nwave + 1]
+  const int* cta_prob;     // [nwave][grid] problem holding each CTA's first unit of a wave
+  const int* cta_units;    // [grid] units of each CTA over all waves
+  int nwave;
+  unsigned int units;
+  int grid, stages;
+  uint32_t stage_bytes;    // one stage: W codes (ku blocks), W scales, then ku activation images
+  int acc_bufs, sf_bufs;
+  uint32_t sf_cols, acc_col0, acc_stride;
+  unsigned int* counters;  // [nwave][grid] split-tile tickets, zero on entry and on exit
+  float* partials;         // [nwave][2*grid][M][128] split-tile partial sums
+  unsigned int* err;
+};
+
+// ------------------------------------------------------------------ activation decomposition
 
 __device__ __forceinline__ float block_amax16(const float (&v)[16]) {
   float a = 0.f;
@@ -94,22 +144,32 @@ __device__ __forceinline__ float block_amax16(const float (&v)[16]) {
   return a;
 }
 
+// Grid (M, problems). Repeated multiplication by 0.25 is exact unless g underflows;
+// the decomposition and the stored g follow the same sequence.
 template <int BPT>
-__global__ void __launch_bounds__(kPrepThreads) x_prep_kernel(XPrepArgs a) {
+__global__ void __launch_bounds__(kPrepThreads) x_prep_kernel(const __grid_constant__ Problem single,
+                                                               const Problem* probs, const Geom g) {
   asm volatile("griddepcontrol.launch_dependents;");
+  // X may come from the previous kernel of the stream, and the previous GEMM may still
+  // read this workspace: nothing is read or written before that kernel has finished.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const Problem* pr = probs ? probs + blockIdx.y : &single;
 #ifdef NVFP4WS_TRACE
-  if (threadIdx.x == 0 && blockIdx.x < 56) g_cta_trace[(200 + blockIdx.x) * 16 + 0] = globaltimer();
+  if (threadIdx.x == 0 && blockIdx.x < 56 && blockIdx.y == 0) g_cta_trace[(200 + blockIdx.x) * 16 + 0] = globaltimer();
 #endif
   const int m = blockIdx.x;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const int nblk = (int)(a.K / 16);
+  const long long K = pr->K;
+  const int nblk = (int)(K / 16);
+  const uint16_t* X = pr->X + (long long)m * K;
+  uint8_t* img = pr->ximg;
   __shared__ float s_red[kPrepThreads / 32];
   float r[BPT][16];
 #pragma unroll
   for (int j = 0; j < BPT; ++j) {
     const int b = t + j * kPrepThreads;
     if (b < nblk) {
-      const uint4* src = reinterpret_cast<const uint4*>(a.X + (long long)m * a.K + (long long)b * 16);
+      const uint4* src = reinterpret_cast<const uint4*>(X + (long long)b * 16);
       const uint4 u0 = src[0], u1 = src[1];
       const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
 #pragma unroll
@@ -122,34 +182,36 @@ __global__ void __launch_bounds__(kPrepThreads) x_prep_kernel(XPrepArgs a) {
       for (int i = 0; i < 16; ++i) r[j][i] = 0.f;
     }
   }
-  for (int term = 0; term < a.T; ++term) {
-    float amax = 0.f;
+  float amax = 0.f;
 #pragma unroll
-    for (int j = 0; j < BPT; ++j) amax = fmaxf(amax, block_amax16(r[j]));
+  for (int j = 0; j < BPT; ++j) amax = fmaxf(amax, block_amax16(r[j]));
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    if (lane == 0) s_red[warp] = amax;
-    __syncthreads();
-    float row_amax = 0.f;
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if (lane == 0) s_red[warp] = amax;
+  __syncthreads();
+  float row_amax = 0.f;
 #pragma unroll
-    for (int w = 0; w < kPrepThreads / 32; ++w) row_amax = fmaxf(row_amax, s_red[w]);
-    __syncthreads();
-    const float g = row_amax / 2688.0f;
-    if (t == 0) a.xg[m * a.T + term] = g;
-    const long long brow = (long long)m * a.T + term;
+  for (int w = 0; w < kPrepThreads / 32; ++w) row_amax = fmaxf(row_amax, s_red[w]);
+  const float g0 = row_amax / 2688.0f;
+  if (t == 0) {
+    float gt = g0;
+    for (int term = 0; term < g.T; ++term, gt *= 0.25f) pr->xg[m * g.T + term] = gt;
+  }
 #pragma unroll
-    for (int j = 0; j < BPT; ++j) {
-      const int b = t + j * kPrepThreads;
-      if (b >= nblk) continue;
+  for (int j = 0; j < BPT; ++j) {
+    const int b = t + j * kPrepThreads;
+    if (b >= nblk) continue;
+    const int kc = b >> 4, bi = b & 15;           // K-chunk and block within it
+    uint8_t* base = img + (size_t)kc * g.img_stride;
+    float gt = g0;
+    for (int term = 0; term < g.T; ++term, gt *= 0.25f) {
       uint32_t sbits = 0, lo = 0, hi = 0;
-      if (g > 0.f) {
-        const float want = block_amax16(r[j]) / (6.0f * g);
+      if (gt > 0.f) {
+        const float want = block_amax16(r[j]) / (6.0f * gt);
         uint16_t s2;
         asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(s2) : "f"(0.0f), "f"(want));
         sbits = s2 & 0xFFu;
-        const uint32_t sh = e4m3x2_to_f16x2(sbits);
-        const float S = f16lo_to_f32(sh);
-        const float den = S * g;
+        const float den = f16lo_to_f32(e4m3x2_to_f16x2(sbits)) * gt;
         if (den > 0.f) {
           const float inv = 1.0f / den;
 #pragma unroll
@@ -165,42 +227,21 @@ __global__ void __launch_bounds__(kPrepThreads) x_prep_kernel(XPrepArgs a) {
           }
         }
       }
-      *reinterpret_cast<uint2*>(a.xq + brow * (a.K / 2) + (long long)b * 8) = make_uint2(lo, hi);
-      a.xs[brow * (a.K / 16) + b] = (uint8_t)sbits;
+      // B row of (token m, term): its 128 code bytes for this chunk, with the 16-byte
+      // pieces permuted by the 128-byte swizzle (piece p of row r at p ^ (r & 7)).
+      const int row = m * g.T + term;
+      const uint32_t off = (uint32_t)row * 128u + ((uint32_t)((bi >> 1) ^ (row & 7)) << 4) + ((uint32_t)(bi & 1) << 3);
+      *reinterpret_cast<uint2*>(base + off) = make_uint2(lo, hi);
+      base[g.img_xs_off + (uint32_t)row * 16u + (uint32_t)bi] = (uint8_t)sbits;
     }
   }
 #ifdef NVFP4WS_TRACE
   __syncthreads();
-  if (threadIdx.x == 0 && blockIdx.x < 56) g_cta_trace[(200 + blockIdx.x) * 16 + 1] = globaltimer();
+  if (threadIdx.x == 0 && blockIdx.x < 56 && blockIdx.y == 0) g_cta_trace[(200 + blockIdx.x) * 16 + 1] = globaltimer();
 #endif
 }
 
 // ------------------------------------------------------------------ GEMM
-
-struct Params {
-  float* Y;
-  int y_bf16;
-  const float* ts;
-  const float* xg;          // [M, T]
-  int M, T, nb;             // nb = M*T B rows
-  int nbt, nb_tile;         // B tiles per MMA K-step and rows per B tile (multiple of 8)
-  int nsfb;                 // TMEM columns of B scales per (K-step, B tile): 4 (<=128 rows) or 8
-  long long N, K;
-  int tiles, kch;
-  long long units;
-  int grid, stages;
-  uint32_t stage_bytes, xq_off, sfw_off, xs_off;
-  int acc_bufs;             // 1 or 2 accumulator buffers
-  int sf_bufs;              // scale-factor TMEM buffers (2..stages); unit i uses buffer i % sf_bufs
-  uint32_t sf_cols;         // TMEM columns per scale-factor buffer
-  uint32_t acc_col0, acc_stride;
-  unsigned int* counters;
-  float* partials;
-  int verify;
-  float* part_val;
-  int* part_idx;
-  unsigned int* err;
-};
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -229,7 +270,12 @@ __device__ __forceinline__ void tc_st_x8(uint32_t taddr, const uint32_t (&v)[8])
                "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
                : "memory");
 }
-__device__ __forceinline__ void tc_ld_x16(uint32_t taddr, uint32_t (&v)[16]) {
+__device__ __forceinline__ void tc_st_x4(uint32_t taddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+__device__ __forceinline__ void tc_ld_x16(uint32_t taddr, uint32_t* v) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
       "%15}, [%16];"
@@ -258,27 +304,76 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
   return d;
 }
 
-__device__ __forceinline__ long long unit_begin(long long c, long long U, int G) { return c * U / G; }
-__device__ __forceinline__ int cta_of_unit(long long u, long long U, int G) {
-  int c = (int)(u * G / U);
-  while (c + 1 < G && unit_begin(c + 1, U, G) <= u) ++c;
-  while (c > 0 && unit_begin(c, U, G) > u) --c;
-  return c;
-}
+// Stream-K partition: CTA c owns units [floor(c*U/G), floor((c+1)*U/G)). The host keeps
+// G <= U (every CTA owns at least one unit) and U * G < 2^32, so 32-bit arithmetic is exact.
+__device__ __forceinline__ uint32_t unit_begin(uint32_t c, uint32_t U, uint32_t G) { return c * U / G; }
+// The CTA owning unit u: the largest c with floor(c*U/G) <= u.
+__device__ __forceinline__ uint32_t cta_of_unit(uint32_t u, uint32_t U, uint32_t G) { return ((u + 1) * G - 1) / U; }
 
-template <int NBT>
+// Position of a unit: problem, tile, K-chunk. Advances without divisions; a problem's
+// sizes are read once when the walk enters it.
+struct Cursor {
+  int pi, tile, kc, kch, tiles;
+  __device__ __forceinline__ void init(const Problem* probs, int p0, uint32_t u) {
+    pi = p0;
+    kch = probs[pi].kch;
+    tiles = probs[pi].tiles;
+    const uint32_t rel = u - probs[pi].unit0;
+    tile = (int)(rel / (uint32_t)kch);
+    kc = (int)(rel - (uint32_t)tile * (uint32_t)kch);
+  }
+  __device__ __forceinline__ void advance(const Problem* probs, int nprob) {
+    if (++kc < kch) return;
+    kc = 0;
+    if (++tile < tiles) return;
+    tile = 0;
+    if (++pi < nprob) { kch = probs[pi].kch; tiles = probs[pi].tiles; }
+  }
+};
+
+// The units one CTA processes, wave by wave: in wave w of Uw units starting at w0,
+// CTA c owns [w0 + floor(c*Uw/G), w0 + floor((c+1)*Uw/G)) (at least one unit: the host
+// makes every wave at least G units long).
+struct Walk {
+  int w;                   // current wave
+  uint32_t w0, Uw;         // its first unit and size
+  uint32_t r0, r1;         // this CTA's range in it
+  uint32_t u;              // current unit
+  Cursor cu;
+  __device__ __forceinline__ void start(const PassParams& p, const Problem* probs, int c, int w_) {
+    w = w_;
+    w0 = p.wave_u0 ? p.wave_u0[w] : 0u;
+    Uw = (p.wave_u0 ? p.wave_u0[w + 1] : p.units) - w0;
+    r0 = w0 + unit_begin((uint32_t)c, Uw, (uint32_t)p.grid);
+    r1 = w0 + unit_begin((uint32_t)c + 1u, Uw, (uint32_t)p.grid);
+    u = r0;
+    cu.init(probs, p.cta_prob ? p.cta_prob[w * p.grid + c] : 0, u);
+  }
+  // Advance one unit; at the end of a wave's range jump to the next wave (callers stop
+  // after the CTA's unit count, so no wave past the last is started).
+  __device__ __forceinline__ void next(const PassParams& p, const Problem* probs, int c) {
+    if (++u < r1) { cu.advance(probs, p.nprob); return; }
+    if (w + 1 < p.nwave) start(p, probs, c, w + 1);
+  }
+  __device__ __forceinline__ bool first() const { return u == r0; }
+  __device__ __forceinline__ bool last() const { return u + 1 == r1; }
+};
+
+template <int NBT, int KU>
 __global__ void __launch_bounds__(kThreads, 1)
-    mxf4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_sf,
-                const __grid_constant__ CUtensorMap tm_xq, const __grid_constant__ CUtensorMap tm_xs,
-                const Params p) {
+    pass_kernel(const __grid_constant__ Problem single, const PassParams p) {
+  // The next kernel of the stream may launch as soon as SMs free up: the library's prep
+  // kernel waits for this grid to finish before touching the workspace or its input.
+  asm volatile("griddepcontrol.launch_dependents;");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const int S = p.stages;
+  const Geom& g = p.g;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)S * p.stage_bytes);
-  // [0,S) full  [S,2S) mma_done (one commit per unit: frees the stage and the unit's scale buffer)
-  // 2S+{0,1} acc_full  2S+{2,3} acc_empty  2S+4 drain  2S+5+{0..7} sf_full
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 2 * S + 13);
+  // [0,S) full  [S,2S) empty (one MMA commit per unit frees the stage and the unit's scale
+  // buffer)  2S+{0,1} acc_full  2S+{2,3} acc_empty  2S+4 drain  2S+5+{0..7} sf_full
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 2 * S + 5 + kMaxSfBufs);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   int* s_last = reinterpret_cast<int*>(s_tmem + 2);
   float* s_val = reinterpret_cast<float*>(s_tmem + 4);                 // [4][72]
@@ -292,11 +387,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bar_drain = smem_u32(bars + 2 * S + 4);
   auto bar_sffull = [&](int b) { return smem_u32(bars + 2 * S + 5 + b); };
 
+  const Problem* probs = p.probs ? p.probs : &single;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c = blockIdx.x;
-  const long long U = p.units;
-  const long long u_begin = unit_begin(c, U, p.grid), u_end = unit_begin(c + 1, U, p.grid);
-  const int nunits = (int)(u_end - u_begin);
+  const uint32_t G = (uint32_t)p.grid;
+  const int nunits = p.cta_units ? p.cta_units[c]
+                                 : (int)(unit_begin((uint32_t)c + 1u, p.units, G) - unit_begin((uint32_t)c, p.units, G));
 
   if (threadIdx.x == 0) MX_CTA(0);
   if (threadIdx.x == 0) {
@@ -317,62 +413,51 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   if (threadIdx.x == 0) MX_CTA(1);
   const uint32_t tmem = *s_tmem;
-  const uint32_t bytes_x = (uint32_t)(p.nbt * p.nb_tile) * (128u + 16u);
-  const uint32_t tx = kNibBytes + kSfBytes + bytes_x;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       const uint64_t pol_w = policy_evict_first(), pol_x = policy_evict_last();
+      const uint32_t xbytes = (uint32_t)g.ku * g.img_stride;
+      const uint32_t tx = g.wbytes + xbytes;
       int issued = 0;
-      // (tile, kc) of unit u_begin + i advance incrementally: no 64-bit divisions in the loop
-      const int tile0 = (int)(u_begin / p.kch), kc0 = (int)(u_begin % p.kch);
-      auto load_w = [&](int s, int tile, int kc) {
+      auto load_w = [&](int s, const Cursor& cu) {
         const uint32_t st = sbase + (uint32_t)s * p.stage_bytes;
+        const Problem* pr = probs + cu.pi;
         mbar_arrive_expect_tx(bar_full(s), tx);
-        tma_load_2d(st, &tm_q, kc * (kKC / 2), tile * kTileRows, bar_full(s), pol_w);
-        tma_load_2d(st + p.sfw_off, &tm_sf, kc * (kKC / 16), tile * kTileRows, bar_full(s), pol_w);
+        for (int h = 0; h < g.ku; ++h)
+          tma_load_2d(st + (uint32_t)h * kNibBytes, &pr->tm_q, (cu.kc * g.ku + h) * (kKC / 2), cu.tile * kTileRows,
+                      bar_full(s), pol_w);
+        tma_load_2d(st + (uint32_t)g.ku * kNibBytes, &pr->tm_sf, cu.kc * g.ku * (kKC / 16), cu.tile * kTileRows,
+                    bar_full(s), pol_w);
       };
-      auto load_x = [&](int s, int kc) {
-        const uint32_t st = sbase + (uint32_t)s * p.stage_bytes;
-        for (int bt = 0; bt < p.nbt; ++bt) {
-          tma_load_2d(st + p.xq_off + bt * p.nb_tile * 128, &tm_xq, kc * (kKC / 2), bt * p.nb_tile, bar_full(s), pol_x);
-          tma_load_2d(st + p.xs_off + bt * p.nb_tile * 16, &tm_xs, kc * (kKC / 16), bt * p.nb_tile, bar_full(s), pol_x);
-        }
+      auto load_x = [&](int s, const Cursor& cu) {
+        bulk_load(sbase + (uint32_t)s * p.stage_bytes + g.wbytes, probs[cu.pi].ximg + (size_t)cu.kc * xbytes, xbytes,
+                  bar_full(s), pol_x);
       };
       // weights of the first stages do not depend on the activation prep: load them first
       const int pre = nunits < S ? nunits : S;
-      {
-        int tile = tile0, kc = kc0;
-        for (int i = 0; i < pre; ++i) {
-          load_w(i, tile, kc);
-          issued = i + 1;
-          if (++kc == p.kch) { kc = 0; ++tile; }
-        }
-      }
+      Walk wk;
+      wk.start(p, probs, c, 0);
+      for (int i = 0; i < pre; ++i) { load_w(i, wk.cu); issued = i + 1; wk.next(p, probs, c); }
       asm volatile("griddepcontrol.wait;" ::: "memory");
       {
-        int kc = kc0;
-        for (int i = 0; i < pre; ++i) {
-          load_x(i, kc);
-          if (++kc == p.kch) kc = 0;
-        }
+        Walk wx;
+        wx.start(p, probs, c, 0);
+        for (int i = 0; i < pre; ++i) { load_x(i, wx.cu); wx.next(p, probs, c); }
       }
-      {
-        int tile = tile0 + (kc0 + pre) / p.kch, kc = (kc0 + pre) % p.kch;
-        int s = pre % S;
-        uint32_t ph = (uint32_t)(pre / S) & 1u;
-        for (int i = pre; i < nunits; ++i) {
-          if (!mbar_wait(bar_empty(s), ph ^ 1u, s_abort, p.err)) break;
-          MX_TRACE(0, i);
-          load_w(s, tile, kc);
-          load_x(s, kc);
-          issued = i + 1;
-          if (++kc == p.kch) { kc = 0; ++tile; }
-          if (++s == S) { s = 0; ph ^= 1u; }
-        }
+      int s = pre % S;
+      uint32_t ph = (uint32_t)(pre / S) & 1u;
+      for (int i = pre; i < nunits; ++i) {
+        if (!mbar_wait(bar_empty(s), ph ^ 1u, s_abort, p.err)) break;
+        MX_TRACE(0, i);
+        load_w(s, wk.cu);
+        load_x(s, wk.cu);
+        issued = i + 1;
+        wk.next(p, probs, c);
+        if (++s == S) { s = 0; ph ^= 1u; }
       }
-      if (*s_abort) {
+      if (*s_abort) {   // let the copies in flight land before the CTA exits
         for (int i = (issued > S ? issued - S : 0); i < issued; ++i) {
           const unsigned long long t0 = globaltimer();
           while (!mbar_try_wait(bar_full(i % S), (uint32_t)(i / S) & 1u) && globaltimer() - t0 < kWaitLimitNs) {}
@@ -381,43 +466,48 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // The single issuing thread is latency-bound, so its loop is kept minimal: it waits
+    // only for the unit's scale buffer. The scale warps arrive on it after observing the
+    // stage's TMA completion, and that arrive/wait pair (release/acquire) orders the
+    // landed operands before the MMAs. Descriptors are precomputed and advanced by adds.
     if (lane == 0) {
       int seg = 0;
       bool ok = true;
-      int s = 0, kc = (int)(u_begin % p.kch);
-      uint32_t ph = 0;
-      const uint32_t idesc = (1u << 7) | (1u << 10) | ((uint32_t)(p.nb_tile >> 3) << 17) |
+      int s = 0;
+      Walk wk;
+      wk.start(p, probs, c, 0);
+      const uint32_t idesc = (1u << 7) | (1u << 10) | ((uint32_t)(g.nb_tile >> 3) << 17) |
                              ((uint32_t)(kTileRows >> 4) << 24);
-      // Everything an MMA needs is precomputed: the single issuing thread is
-      // latency-bound on scalar work between MMAs, so the loop does adds only.
-      const uint64_t adesc_base = sw128_desc(sbase);
-      const uint64_t bdesc_base = sw128_desc(sbase + p.xq_off);
-      const uint64_t stage_step = (uint64_t)(p.stage_bytes >> 4);
+      const uint64_t adesc_base = sw128_desc(sbase), bdesc_base = sw128_desc(sbase + g.wbytes);
+      const uint64_t step = (uint64_t)(p.stage_bytes >> 4);
       uint64_t adesc = adesc_base, bdesc = bdesc_base;
-      uint32_t boff[NBT], doff[NBT], sfboff[4][NBT];
+      // K-step kk of chunk h: A at block h, B in image h, scales in columns laid out as the
+      // scale warps store them (W: 4 per K-step; X: nsfb per K-step and B tile).
+      uint32_t boff[KU][NBT], doff[NBT], sfboff[KU][4][NBT];
 #pragma unroll
       for (int bt = 0; bt < NBT; ++bt) {
-        boff[bt] = (uint32_t)(bt * p.nb_tile * 8);
-        doff[bt] = (uint32_t)(bt * p.nb_tile);
+        doff[bt] = (uint32_t)(bt * g.nb_tile);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) sfboff[kk][bt] = 16u + (uint32_t)((kk * NBT + bt) * p.nsfb);
+        for (int h = 0; h < KU; ++h) {
+          boff[h][bt] = (h * g.img_stride >> 4) + (uint32_t)(bt * g.nb_tile * 8);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            sfboff[h][kk][bt] = 16u * KU + (uint32_t)(((h * 4 + kk) * NBT + bt) * g.nsfb);
+        }
       }
       int fb = 0;                                     // scale-factor buffer of unit i
       uint32_t fph = 0;
       const uint32_t acc0 = tmem + p.acc_col0, acc1 = tmem + p.acc_col0 + p.acc_stride;
       for (int i = 0; i < nunits && ok; ++i) {
-        const bool seg_first = (i == 0) || (kc == 0);
-        const bool seg_last = (i == nunits - 1) || (kc == p.kch - 1);
+        const bool seg_first = wk.first() || (wk.cu.kc == 0);
+        const bool seg_last = wk.last() || (wk.cu.kc == wk.cu.kch - 1);
         const int ab = (p.acc_bufs == 2) ? (seg & 1) : 0;
         if (seg_first) {
           const uint32_t acc_use = (p.acc_bufs == 2) ? (uint32_t)(seg >> 1) : (uint32_t)seg;
           ok = mbar_wait(bar_accempty(ab), (acc_use & 1u) ^ 1u, s_abort, p.err);
           if (!ok) break;
         }
-        MX_TRACE(11, i);
-        ok = mbar_wait(bar_full(s), ph, s_abort, p.err);
-        MX_TRACE(1, i);
-        ok = ok && mbar_wait(bar_sffull(fb), fph, s_abort, p.err);
+        ok = mbar_wait(bar_sffull(fb), fph, s_abort, p.err);
         if (!ok) break;
         MX_TRACE(2, i);
         if (i == 0) MX_CTA(2);
@@ -426,20 +516,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t d0 = ab ? acc1 : acc0;
         const uint32_t first = seg_first ? 0u : 1u;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
+        for (int h = 0; h < KU; ++h) {
 #pragma unroll
-          for (int bt = 0; bt < NBT; ++bt)
-            tc_mma_mxf4(d0 + doff[bt], adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(boff[bt] + kk * 2), idesc,
-                        sf + (uint32_t)(kk * 4), sf + sfboff[kk][bt], kk == 0 ? first : 1u);
+          for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+            for (int bt = 0; bt < NBT; ++bt)
+              tc_mma_mxf4(d0 + doff[bt], adesc + (uint64_t)(h * (kNibBytes >> 4) + kk * 2),
+                          bdesc + (uint64_t)(boff[h][bt] + kk * 2), idesc, sf + (uint32_t)((h * 4 + kk) * 4),
+                          sf + sfboff[h][kk][bt], (h == 0 && kk == 0) ? first : 1u);
+          }
         }
         MX_TRACE(3, i);
         tc_commit(bar_empty(s));                      // stage s and scale buffer fb are free once these retire
         if (seg_last) { tc_commit(bar_accfull(ab)); ++seg; }
-        MX_TRACE(4, i);
-        if (++kc == p.kch) kc = 0;
+        wk.next(p, probs, c);
         if (++fb == p.sf_bufs) { fb = 0; fph ^= 1u; }
-        if (++s == S) { s = 0; ph ^= 1u; adesc = adesc_base; bdesc = bdesc_base; }
-        else { adesc += stage_step; bdesc += stage_step; }
+        if (++s == S) { s = 0; adesc = adesc_base; bdesc = bdesc_base; }
+        else { adesc += step; bdesc += step; }
       }
       MX_CTA(3);
       tc_commit(bar_drain);
@@ -452,61 +545,71 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int m0 = lane;
     int s = 0;
     uint32_t ph = 0;
-    const int NF = p.sf_bufs;
-    int s2 = S - NF;                // ring position of unit i - NF (valid once i >= NF)
+    const int NF = p.sf_bufs;               // <= S
+    int s2 = S - NF;                        // ring position of unit i - NF (valid once i >= NF)
     uint32_t ph2 = 1u;
     int fb = 0;
-    uint32_t fph = 0;
+    const uint32_t wsf_off = (uint32_t)g.ku * kNibBytes;       // W scales: row m has 16*ku bytes
+    const uint32_t wsf_row = 16u * (uint32_t)g.ku;
     for (int i = 0; i < nunits; ++i) {
       if (!mbar_wait(bar_full(s), ph, s_abort, p.err)) break;
       if (lane == 0 && warp == 4) MX_TRACE(5, i);
       // scale buffer fb was last read by the MMAs of unit i - NF
       if (i >= NF && !mbar_wait(bar_empty(s2), ph2, s_abort, p.err)) break;
-      if (lane == 0 && warp == 4) MX_TRACE(6, i);
       tc_fence_after();
       const uint32_t st = sbase + (uint32_t)s * p.stage_bytes;
       const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)fb * p.sf_cols;
-      {   // W scales: column 4*kk + j of lane m0 = the 4 block scales (K-step kk) of tile row m0 + 32*j
-        uint4 R[4];
+      for (int h = 0; h < g.ku; ++h) {
+        {   // W scales: column 4*(4h+kk) + j of lane m0 = the 4 block scales (K-step kk of chunk h) of row m0 + 32*j
+          uint4 R[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) R[j] = lds128(st + p.sfw_off + (uint32_t)((m0 + 32 * j) * 16));
-        uint32_t out[16];
+          for (int j = 0; j < 4; ++j) R[j] = lds128(st + wsf_off + (uint32_t)(m0 + 32 * j) * wsf_row + (uint32_t)h * 16u);
+          uint32_t out[16];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          out[0 + j] = R[j].x; out[4 + j] = R[j].y; out[8 + j] = R[j].z; out[12 + j] = R[j].w;
+          for (int j = 0; j < 4; ++j) {
+            out[0 + j] = R[j].x; out[4 + j] = R[j].y; out[8 + j] = R[j].z; out[12 + j] = R[j].w;
+          }
+          tc_st_x16(lane_base + (uint32_t)h * 16u, out);
         }
-        tc_st_x16(lane_base, out);
-      }
-      for (int bt = 0; bt < p.nbt; ++bt) {   // X-term scales, per B tile: nsfb columns per K-step
-        uint4 R[8];
+        const uint32_t xs = st + g.wbytes + (uint32_t)h * g.img_stride + g.img_xs_off;
+        if (g.nbt == 1 && g.nsfb == 4) {
+          // one B tile of <= 128 rows: the chunk's 4 K-steps x 4 columns are contiguous, so
+          // column 4*kk + j of lane m0 (B row m0 + 32*j, K-step kk) goes in one x16 store
+          uint4 R[4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int row = m0 + 32 * j;
-          R[j] = (j < p.nsfb && row < p.nb_tile) ? lds128(st + p.xs_off + (uint32_t)((bt * p.nb_tile + row) * 16))
-                                                 : make_uint4(0, 0, 0, 0);
+          for (int j = 0; j < 4; ++j)
+            R[j] = (m0 + 32 * j < g.nb_tile) ? lds128(xs + (uint32_t)((m0 + 32 * j) * 16)) : make_uint4(0, 0, 0, 0);
+          uint32_t out[16];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            out[0 + j] = R[j].x; out[4 + j] = R[j].y; out[8 + j] = R[j].z; out[12 + j] = R[j].w;
+          }
+          tc_st_x16(lane_base + 16u * (uint32_t)g.ku + (uint32_t)h * 16u, out);
+          continue;
         }
-        for (int kk = 0; kk < 4; ++kk) {
-          uint32_t out[8];
+        for (int bt = 0; bt < g.nbt; ++bt) {   // X-term scales, per B tile: nsfb columns per K-step
+          uint4 R[8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) out[j] = kk == 0 ? R[j].x : kk == 1 ? R[j].y : kk == 2 ? R[j].z : R[j].w;
-          const uint32_t col = 16u + (uint32_t)((kk * p.nbt + bt) * p.nsfb);
-          if (p.nsfb == 8) {
-            tc_st_x8(lane_base + col, out);
-          } else {
-            uint32_t o4[8] = {out[0], out[1], out[2], out[3], 0, 0, 0, 0};
-            asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(lane_base + col),
-                         "r"(o4[0]), "r"(o4[1]), "r"(o4[2]), "r"(o4[3])
-                         : "memory");
+          for (int j = 0; j < 8; ++j) {
+            const int row = m0 + 32 * j;
+            R[j] = (j < g.nsfb && row < g.nb_tile) ? lds128(xs + (uint32_t)((bt * g.nb_tile + row) * 16))
+                                                   : make_uint4(0, 0, 0, 0);
+          }
+          for (int kk = 0; kk < 4; ++kk) {
+            uint32_t out[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) out[j] = kk == 0 ? R[j].x : kk == 1 ? R[j].y : kk == 2 ? R[j].z : R[j].w;
+            const uint32_t col = 16u * (uint32_t)g.ku + (uint32_t)(((h * 4 + kk) * g.nbt + bt) * g.nsfb);
+            if (g.nsfb == 8) tc_st_x8(lane_base + col, out);
+            else tc_st_x4(lane_base + col, out[0], out[1], out[2], out[3]);
           }
         }
       }
       tc_wait_st();
       tc_fence_before();
       if (lane == 0 && warp == 4) MX_TRACE(7, i);
-      if (lane == 0 && warp == 7) MX_TRACE(8, i);
       mbar_arrive(bar_sffull(fb));
-      (void)fph;
-      if (++fb == NF) { fb = 0; fph ^= 1u; }
+      if (++fb == NF) fb = 0;
       if (++s == S) { s = 0; ph ^= 1u; }
       if (++s2 == S) { s2 = 0; ph2 ^= 1u; }
     }
@@ -516,160 +619,154 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;
     const int rowl = q * 32 + lane;
     const int et = threadIdx.x - 8 * 32;
-    for (int j = et; j < p.nb; j += 128) s_g[j] = p.xg[j];
-    named_bar(1, 128);
-    const float ts = *p.ts;
+    const int M = g.M;
+    int gprob = -1;                         // problem whose term scales are in s_g
     int seg = 0;
-    int tile = (int)(u_begin / p.kch), kc = (int)(u_begin % p.kch);
+    Walk wk;
+    wk.start(p, probs, c, 0);
     for (int i = 0; i < nunits; ++i) {
-      const long long u = u_begin + i;
-      const bool seg_last = (i == nunits - 1) || (kc == p.kch - 1);
-      const int cur_tile = tile;
-      if (++kc == p.kch) { kc = 0; ++tile; }
+      const uint32_t u = wk.u, r0 = wk.r0, w0 = wk.w0, Uw = wk.Uw;
+      const int wave = wk.w;
+      const bool seg_last = wk.last() || (wk.cu.kc == wk.cu.kch - 1);
+      const int pi = wk.cu.pi, cur_tile = wk.cu.tile, kch = wk.cu.kch;
+      wk.next(p, probs, c);
       if (!seg_last) continue;
-      const long long tile_u0 = (long long)cur_tile * p.kch, tile_u1 = tile_u0 + p.kch;
-      const long long seg_u0 = u_begin > tile_u0 ? u_begin : tile_u0;
+      const Problem* pr = probs + pi;
+      const uint32_t tile_u0 = pr->unit0 + (uint32_t)cur_tile * (uint32_t)kch, tile_u1 = tile_u0 + (uint32_t)kch;
+      const uint32_t seg_u0 = r0 > tile_u0 ? r0 : tile_u0;
       const bool complete = (seg_u0 == tile_u0) && (u + 1 == tile_u1);
+      if (pi != gprob) {
+        named_bar(1, 128);
+        for (int j = et; j < g.nb; j += 128) s_g[j] = pr->xg[j];
+        named_bar(1, 128);
+        gprob = pi;
+      }
+      const float ts = *pr->ts;
+      const long long N = pr->N;
+      const int verify = pr->verify, y_bf16 = pr->y_bf16;
+      float* Yf = static_cast<float*>(pr->Y);
       const int ab = (p.acc_bufs == 2) ? (seg & 1) : 0;
       const uint32_t acc_use = (p.acc_bufs == 2) ? (uint32_t)(seg >> 1) : (uint32_t)seg;
       if (!mbar_wait(bar_accfull(ab), acc_use & 1u, s_abort, p.err)) break;
-      if (et == 0) MX_TRACE(9, seg);
       if (et == 0 && seg < 2) MX_CTA(8 + 4 * seg);
       tc_fence_after();
       const long long n = (long long)cur_tile * kTileRows + rowl;
       const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + p.acc_col0 + (uint32_t)ab * p.acc_stride;
-      const int slot = (seg_u0 == u_begin) ? 2 * c : 2 * c + 1;
-      float* dst = p.partials + ((long long)slot * p.M) * kTileRows;
+      float* wave_part = p.partials + (long long)wave * 2 * G * M * kTileRows;
+      const int slot = (seg_u0 == r0) ? 2 * c : 2 * c + 1;
+      float* dst = wave_part + ((long long)slot * M) * kTileRows;
+      auto emit = [&](int m, float y) {   // a finished output: Y, or this row's argmax candidate
+        if (verify) {
+          float bv = (n < N) ? y : -INFINITY;
+          int bi = (n < N) ? (int)n : INT_MAX;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (argmax_better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+          }
+          if (lane == 0) { s_val[q * 72 + m] = bv; s_idx[q * 72 + m] = bi; }
+        } else if (n < N) {
+          if (y_bf16) reinterpret_cast<uint16_t*>(Yf)[(long long)m * N + n] = f32_to_bf16_rn(y);
+          else Yf[(long long)m * N + n] = y;
+        }
+      };
+      auto tile_argmax = [&]() {          // combine the 4 warps' candidates of each row
+        named_bar(1, 128);
+        if (et < M) {
+          float bv = s_val[et];
+          int bi = s_idx[et];
+          for (int w = 1; w < 4; ++w)
+            if (argmax_better(s_val[w * 72 + et], s_idx[w * 72 + et], bv, bi)) { bv = s_val[w * 72 + et]; bi = s_idx[w * 72 + et]; }
+          pr->part_val[(long long)cur_tile * M + et] = bv;
+          pr->part_idx[(long long)cur_tile * M + et] = bi;
+        }
+        named_bar(1, 128);
+      };
       // Fold the T terms of each token: y[m] = sum_t g[m,t] * acc[m*T + t]. Accumulator
-      // column c holds B row c, so token m's terms are columns m*T .. m*T+T-1. Tokens are
+      // column j holds B row j, so token m's terms are columns m*T .. m*T+T-1. Tokens are
       // taken 16 at a time: up to 5 TMEM loads of 16 columns are issued back to back and
       // waited for once, and the fold uses the compile-time term count.
       static_assert(kMxf4Terms == 5, "the fold below is written for 5 terms");
-      const int nb16 = (p.nb + 15) & ~15;                 // columns that exist in the accumulator
-      for (int mc = 0; mc < p.M; mc += 16) {
+      const int nb16 = (g.nb + 15) & ~15;                 // columns that exist in the accumulator
+      for (int mc = 0; mc < M; mc += 16) {
         const int col0 = mc * kMxf4Terms;                 // multiple of 80
         const int nld = (nb16 - col0) / 16 < 5 ? (nb16 - col0) / 16 : 5;
         uint32_t v[80];
-        tc_ld_x16(taddr + (uint32_t)col0, *reinterpret_cast<uint32_t(*)[16]>(v));
-        if (nld > 1) tc_ld_x16(taddr + (uint32_t)(col0 + 16), *reinterpret_cast<uint32_t(*)[16]>(v + 16));
-        if (nld > 2) tc_ld_x16(taddr + (uint32_t)(col0 + 32), *reinterpret_cast<uint32_t(*)[16]>(v + 32));
-        if (nld > 3) tc_ld_x16(taddr + (uint32_t)(col0 + 48), *reinterpret_cast<uint32_t(*)[16]>(v + 48));
-        if (nld > 4) tc_ld_x16(taddr + (uint32_t)(col0 + 64), *reinterpret_cast<uint32_t(*)[16]>(v + 64));
+        tc_ld_x16(taddr + (uint32_t)col0, v);
+        if (nld > 1) tc_ld_x16(taddr + (uint32_t)(col0 + 16), v + 16);
+        if (nld > 2) tc_ld_x16(taddr + (uint32_t)(col0 + 32), v + 32);
+        if (nld > 3) tc_ld_x16(taddr + (uint32_t)(col0 + 48), v + 48);
+        if (nld > 4) tc_ld_x16(taddr + (uint32_t)(col0 + 64), v + 64);
         tc_wait_ld();
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const int m = mc + j;
-          if (m >= p.M) break;
+          if (m >= M) break;
           float ym = 0.f;
 #pragma unroll
           for (int t = 0; t < kMxf4Terms; ++t)
             ym = fmaf(s_g[m * kMxf4Terms + t], __uint_as_float(v[j * kMxf4Terms + t]), ym);
-          if (complete) {
-            const float y = ym * ts;
-            if (p.verify) {
-              float bv = (n < p.N) ? y : -INFINITY;
-              int bi = (n < p.N) ? (int)n : INT_MAX;
-#pragma unroll
-              for (int o = 16; o > 0; o >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                if (argmax_better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
-              }
-              if (lane == 0) { s_val[q * 72 + m] = bv; s_idx[q * 72 + m] = bi; }
-            } else if (n < p.N) {
-              if (p.y_bf16) reinterpret_cast<uint16_t*>(p.Y)[(long long)m * p.N + n] = f32_to_bf16_rn(y);
-              else p.Y[(long long)m * p.N + n] = y;
-            }
-          } else {
-            dst[(long long)m * kTileRows + rowl] = ym;
-          }
+          if (complete) emit(m, ym * ts);
+          else dst[(long long)m * kTileRows + rowl] = ym;
         }
       }
       tc_fence_before();
-      if (et == 0) MX_TRACE(10, seg);
       if (et == 0 && seg < 2) MX_CTA(9 + 4 * seg);
       mbar_arrive(bar_accempty(ab));
       ++seg;
       if (complete) {
-        if (p.verify) {
-          named_bar(1, 128);
-          if (et < p.M) {
-            float bv = s_val[et];
-            int bi = s_idx[et];
-            for (int w = 1; w < 4; ++w)
-              if (argmax_better(s_val[w * 72 + et], s_idx[w * 72 + et], bv, bi)) { bv = s_val[w * 72 + et]; bi = s_idx[w * 72 + et]; }
-            p.part_val[(long long)cur_tile * p.M + et] = bv;
-            p.part_idx[(long long)cur_tile * p.M + et] = bi;
-          }
-          named_bar(1, 128);
-        }
+        if (verify) tile_argmax();
         continue;
       }
-      __threadfence();
-      if (et == 0 && seg <= 2) MX_CTA(10 + 4 * (seg - 1));
+      // Split tile: count this CTA's arrival. The barrier orders every epilogue thread's
+      // partial stores before thread 0's release; the acquire side of the same atomic
+      // orders the last arriver's loads of the other contributors' partials after it.
+      // The ticket of a split tile is indexed by its first contributing CTA, which has
+      // at most one split tile starting in its range.
+      const int c0 = (int)cta_of_unit(tile_u0 - w0, Uw, G), c1 = (int)cta_of_unit(tile_u1 - 1u - w0, Uw, G);
+      unsigned int* ticket = p.counters + (long long)wave * G + c0;
       named_bar(1, 128);
       if (et == 0) {
-        const int c0 = cta_of_unit(tile_u0, U, p.grid), c1 = cta_of_unit(tile_u1 - 1, U, p.grid);
-        int expected = 0;
-        for (int cc = c0; cc <= c1; ++cc)
-          if (unit_begin(cc + 1, U, p.grid) > unit_begin(cc, U, p.grid)) ++expected;
-        const unsigned int prev = atomicAdd(p.counters + cur_tile, 1u);
-        *s_last = (prev + 1 == (unsigned int)expected) ? 1 : 0;
+        unsigned int prev;
+        asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(prev) : "l"(ticket) : "memory");
+        *s_last = (prev + 1 == (unsigned int)(c1 - c0 + 1)) ? 1 : 0;   // every CTA owns >= 1 unit
       }
       named_bar(1, 128);
+      if (et == 0 && seg <= 2) MX_CTA(10 + 4 * (seg - 1));
       if (*s_last) {
-        __threadfence();
-        const int c0 = cta_of_unit(tile_u0, U, p.grid), c1 = cta_of_unit(tile_u1 - 1, U, p.grid);
-        // 16 tokens at a time: issue all partial loads of a chunk before summing them, so
-        // the fix-up costs one L2 round trip per (chunk, contributor), not one per token.
-        for (int mc = 0; mc < p.M; mc += 16) {
+        // Sum the contributors' partials in CTA order (deterministic), two contributors'
+        // loads in flight at a time, 16 tokens per pass.
+        for (int mc = 0; mc < M; mc += 16) {
           float acc[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) acc[j] = 0.f;
-          for (int cc = c0; cc <= c1; ++cc) {
-            const long long b0 = unit_begin(cc, U, p.grid), b1 = unit_begin(cc + 1, U, p.grid);
-            if (b1 <= b0) continue;
-            const int sl = (b0 >= tile_u0) ? 2 * cc : 2 * cc + 1;
-            const float* src = p.partials + ((long long)sl * p.M) * kTileRows + rowl;
-            float v[16];
+          for (int cc = c0; cc <= c1; cc += 2) {
+            const bool two = cc + 1 <= c1;
+            const int sl0 = (w0 + unit_begin((uint32_t)cc, Uw, G) >= tile_u0) ? 2 * cc : 2 * cc + 1;
+            const int sl1 = two ? ((w0 + unit_begin((uint32_t)cc + 1u, Uw, G) >= tile_u0) ? 2 * cc + 2 : 2 * cc + 3) : sl0;
+            const float* src0 = wave_part + ((long long)sl0 * M + mc) * kTileRows + rowl;
+            const float* src1 = wave_part + ((long long)sl1 * M + mc) * kTileRows + rowl;
+            float v0[16], v1[16];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] = (mc + j < p.M) ? __ldcg(src + (long long)(mc + j) * kTileRows) : 0.f;
+            for (int j = 0; j < 16; ++j) {
+              v0[j] = (mc + j < M) ? __ldcg(src0 + j * kTileRows) : 0.f;
+              v1[j] = (two && mc + j < M) ? __ldcg(src1 + j * kTileRows) : 0.f;
+            }
 #pragma unroll
-            for (int j = 0; j < 16; ++j) acc[j] += v[j];
+            for (int j = 0; j < 16; ++j) {
+              acc[j] += v0[j];
+              if (two) acc[j] += v1[j];
+            }
           }
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const int m = mc + j;
-            if (m >= p.M) break;
-            const float y = acc[j] * ts;
-            if (p.verify) {
-              float bv = (n < p.N) ? y : -INFINITY;
-              int bi = (n < p.N) ? (int)n : INT_MAX;
-#pragma unroll
-              for (int o = 16; o > 0; o >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                if (argmax_better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
-              }
-              if (lane == 0) { s_val[q * 72 + m] = bv; s_idx[q * 72 + m] = bi; }
-            } else if (n < p.N) {
-              if (p.y_bf16) reinterpret_cast<uint16_t*>(p.Y)[(long long)m * p.N + n] = f32_to_bf16_rn(y);
-              else p.Y[(long long)m * p.N + n] = y;
-            }
+            if (mc + j >= M) break;
+            emit(mc + j, acc[j] * ts);
           }
         }
-        if (p.verify) {
-          named_bar(1, 128);
-          if (et < p.M) {
-            float bv = s_val[et];
-            int bi = s_idx[et];
-            for (int w = 1; w < 4; ++w)
-              if (argmax_better(s_val[w * 72 + et], s_idx[w * 72 + et], bv, bi)) { bv = s_val[w * 72 + et]; bi = s_idx[w * 72 + et]; }
-            p.part_val[(long long)cur_tile * p.M + et] = bv;
-            p.part_idx[(long long)cur_tile * p.M + et] = bi;
-          }
-        }
-        if (et == 0) p.counters[cur_tile] = 0u;
+        if (verify) tile_argmax();
+        if (et == 0) *ticket = 0u;           // ready for the next launch
       }
       named_bar(1, 128);
       if (et == 0 && seg <= 2) MX_CTA(11 + 4 * (seg - 1));
@@ -717,132 +814,241 @@ static bool map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t ou
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+static size_t al256(size_t v) { return (v + 255) / 256 * 256; }
+
+// Launch geometry: depends on M, and on whether every K of the launch is a multiple of
+// 512 (then a unit may span two 256-wide chunks).
 struct MxPlan {
-  int T, nb, nbt, nb_tile, nsfb, tiles, kch, grid, stages, acc_bufs, sf_bufs;
-  long long units;
-  uint32_t stage_bytes, xq_off, sfw_off, xs_off, sf_cols, acc_col0, acc_stride;
+  Geom g;
+  int stages, acc_bufs, sf_bufs;
+  uint32_t stage_bytes, sf_cols, acc_col0, acc_stride;
   size_t smem;
 };
 
-static size_t al256(size_t v) { return (v + 255) / 256 * 256; }
-
-static MxPlan mx_plan(long long M, long long N, long long K) {
+static MxPlan mx_plan_ku(long long M, int ku) {
   MxPlan pl{};
-  pl.T = kMxf4Terms;
-  pl.nb = (int)M * pl.T;
-  pl.nbt = (pl.nb + 255) / 256;
-  pl.nb_tile = ((pl.nb + pl.nbt - 1) / pl.nbt + 15) / 16 * 16;   // MMA N; a multiple of 16 keeps x16 loads inside the tile
-  pl.nsfb = pl.nb_tile <= 128 ? 4 : 8;
-  pl.sf_cols = 16u + 4u * (uint32_t)(pl.nbt * pl.nsfb);
-  pl.acc_stride = (uint32_t)(pl.nbt * pl.nb_tile);
+  Geom& g = pl.g;
+  g.M = (int)M;
+  g.T = kMxf4Terms;
+  g.nb = (int)M * g.T;
+  g.nbt = (g.nb + 255) / 256;
+  g.nb_tile = ((g.nb + g.nbt - 1) / g.nbt + 15) / 16 * 16;   // MMA N; a multiple of 16 keeps x16 loads inside the tile
+  g.nsfb = g.nb_tile <= 128 ? 4 : 8;
+  g.ku = ku;
+  g.img_xs_off = (uint32_t)(g.nbt * g.nb_tile) * 128u;
+  g.img_bytes = (uint32_t)(g.nbt * g.nb_tile) * 144u;
+  g.img_stride = (g.img_bytes + 1023) / 1024 * 1024;
+  g.wbytes = (uint32_t)ku * kWChunk;
+  pl.sf_cols = 16u * (uint32_t)ku + 4u * (uint32_t)(ku * g.nbt * g.nsfb);
+  pl.acc_stride = (uint32_t)(g.nbt * g.nb_tile);
   pl.acc_bufs = (2 * pl.sf_cols + 2 * pl.acc_stride <= 512) ? 2 : 1;
-  pl.tiles = (int)((N + kTileRows - 1) / kTileRows);
-  pl.kch = (int)(K / kKC);
-  pl.units = (long long)pl.tiles * pl.kch;
-  const int sms = std::max(1, device_sm_count());
-  pl.grid = (int)std::min<long long>(sms, pl.units);
-  const uint32_t xq = (uint32_t)(pl.nbt * pl.nb_tile) * 128u;
-  const uint32_t xs = (uint32_t)(pl.nbt * pl.nb_tile) * 16u;
-  pl.xq_off = kNibBytes;
-  pl.sfw_off = (pl.xq_off + xq + 1023) / 1024 * 1024;
-  pl.xs_off = pl.sfw_off + kSfBytes;
-  pl.stage_bytes = (pl.xs_off + xs + 1023) / 1024 * 1024;
+  // One ring: a stage holds a unit's weight tile, its scales and its activation images.
+  // Measured: under a saturated weight stream the L2-resident images arrive with about the
+  // weights' latency, so they need the same prefetch depth.
+  pl.stage_bytes = g.wbytes + (uint32_t)ku * g.img_stride;
   const size_t budget = 227 * 1024 - 1024 - kTailBytes;
-  pl.stages = (int)std::min<size_t>(8, budget / pl.stage_bytes);
+  pl.stages = (int)std::min<size_t>(kMaxStages, budget / pl.stage_bytes);
   pl.smem = 1024 + (size_t)pl.stages * pl.stage_bytes + kTailBytes;
-  // scale-factor buffers: one per ring stage when TMEM allows (the scale copy then runs ahead like TMA)
+  // scale-factor buffers: one per stage when TMEM allows (the scale copy then runs ahead like TMA)
   const uint32_t acc_cols = (uint32_t)pl.acc_bufs * pl.acc_stride;
-  pl.sf_bufs = (int)std::min<uint32_t>((uint32_t)pl.stages, (512u - acc_cols) / pl.sf_cols);
+  pl.sf_bufs = (int)std::min<uint32_t>((uint32_t)std::min(pl.stages, kMaxSfBufs), (512u - acc_cols) / pl.sf_cols);
   if (pl.sf_bufs < 2) pl.sf_bufs = 2;
   pl.acc_col0 = (uint32_t)pl.sf_bufs * pl.sf_cols;
   return pl;
+}
+
+// Two-chunk units halve the issuing thread's per-unit work (its waits, commit and loop
+// bookkeeping are per unit, the MMAs per K-step). They are used when every K allows it,
+// the activations fit one B tile and the accumulator stays double-buffered.
+static MxPlan mx_plan(long long M, bool k512) {
+  if (k512) {
+    const MxPlan two = mx_plan_ku(M, 2);
+    if (two.g.nbt == 1 && two.acc_bufs == 2 && two.stages >= 3) return two;
+  }
+  return mx_plan_ku(M, 1);
 }
 
 bool mxf4_supported(long long M, long long K) {
   return M >= 1 && M * kMxf4Terms <= kMaxB && K % kKC == 0 && K >= kKC && K <= 32768;
 }
 
-// workspace: counters | partials [2*grid][M][128] | xq [nb][K/2] | xs [nb][K/16] | xg [M][T] | (verify) part val/idx
-static void mx_ws_layout(long long M, long long N, long long K, size_t* off_part, size_t* off_xq, size_t* off_xs,
-                         size_t* off_xg, size_t* off_pv, size_t* off_pi, size_t* total) {
-  MxPlan pl = mx_plan(M, N, K);
-  size_t o = al256((size_t)pl.tiles * 4);
-  *off_part = o; o += al256((size_t)2 * pl.grid * M * kTileRows * 4);
-  *off_xq = o; o += al256((size_t)pl.nb * (K / 2));
-  *off_xs = o; o += al256((size_t)pl.nb * (K / 16));
-  *off_xg = o; o += al256((size_t)pl.nb * 4);
-  *off_pv = o; o += al256((size_t)pl.tiles * M * 4);
-  *off_pi = o; o += al256((size_t)pl.tiles * M * 4);
-  *total = o;
+// Activation-image bytes a wave may hold: small enough that a wave's images stay in L2
+// while the weight stream passes through it.
+constexpr size_t kWaveImageBudget = size_t(24) << 20;
+
+// Workspace: counters [nwave][grid] | partials [nwave][2*grid][M][128] | (a pass) problem
+// descriptors, wave starts, per-(wave, CTA) first problems, per-CTA unit counts | per
+// problem: images, term scales, and (verify) the per-tile row maxima and indices.
+struct WsLayout {
+  int grid, nwave;
+  unsigned long long units;
+  std::vector<int> wave_first;              // first problem of each wave, plus n
+  size_t off_part, off_desc, off_wave, off_cta, off_cunits, total;
+  std::vector<size_t> off_img, off_xg, off_pv, off_pi;
+};
+
+static unsigned long long problem_units(const MxHostProblem& h, int ku) {
+  return (unsigned long long)((h.N + kTileRows - 1) / kTileRows) * (unsigned long long)(h.K / (kKC * ku));
 }
 
-size_t mxf4_workspace_bytes(long long M, long long N, long long K) {
-  if (!mxf4_supported(M, K)) return 0;
-  size_t a, b, c, d, e, f, t;
-  mx_ws_layout(M, N, K, &a, &b, &c, &d, &e, &f, &t);
-  return t;
+static bool all_k512(const MxHostProblem* hp, int n) {
+  for (int i = 0; i < n; ++i)
+    if (hp[i].K % (2 * kKC) != 0) return false;
+  return true;
 }
 
-size_t mxf4_counter_bytes(long long M, long long N, long long K) {
-  return mxf4_supported(M, K) ? al256((size_t)mx_plan(M, N, K).tiles * 4) : 0;
+// with_desc: a pass keeps its descriptors and wave tables in the workspace.
+static WsLayout mx_layout(const MxHostProblem* hp, int n, long long M, bool with_desc) {
+  const MxPlan pl = mx_plan(M, all_k512(hp, n));
+  const int ku = pl.g.ku;
+  WsLayout L;
+  L.units = 0;
+  for (int i = 0; i < n; ++i) L.units += problem_units(hp[i], ku);
+  const int sms = std::max(1, device_sm_count());
+  L.grid = (int)std::max<unsigned long long>(1ull, std::min<unsigned long long>((unsigned long long)sms, L.units));
+  // waves: greedy over the list; a wave closes when the next problem's images would pass
+  // the budget and it already has >= grid units (so every CTA owns a unit of it)
+  L.wave_first.push_back(0);
+  size_t img = 0;
+  unsigned long long wu = 0;
+  for (int i = 0; i < n; ++i) {
+    const size_t pimg = (size_t)(hp[i].K / kKC) * pl.g.img_stride;
+    if (i > 0 && wu >= (unsigned long long)L.grid && img + pimg > kWaveImageBudget) {
+      L.wave_first.push_back(i);
+      img = 0;
+      wu = 0;
+    }
+    img += pimg;
+    wu += problem_units(hp[i], ku);
+  }
+  if (L.wave_first.size() > 1 && wu < (unsigned long long)L.grid) L.wave_first.pop_back();   // merge a short tail
+  L.wave_first.push_back(n);
+  L.nwave = (int)L.wave_first.size() - 1;
+  size_t o = al256((size_t)L.nwave * L.grid * 4);
+  L.off_part = o;
+  o += al256((size_t)L.nwave * 2 * L.grid * M * kTileRows * 4);
+  L.off_desc = L.off_wave = L.off_cta = L.off_cunits = 0;
+  if (with_desc) {
+    L.off_desc = o; o += al256(sizeof(Problem) * (size_t)n);
+    L.off_wave = o; o += al256(sizeof(uint32_t) * (size_t)(L.nwave + 1));
+    L.off_cta = o; o += al256(sizeof(int) * (size_t)L.nwave * L.grid);
+    L.off_cunits = o; o += al256(sizeof(int) * (size_t)L.grid);
+  }
+  for (int i = 0; i < n; ++i) {
+    const long long tiles = (hp[i].N + kTileRows - 1) / kTileRows;
+    L.off_img.push_back(o); o += al256((size_t)(hp[i].K / kKC) * pl.g.img_stride);
+    L.off_xg.push_back(o); o += al256((size_t)pl.g.nb * 4);
+    if (hp[i].verify) {
+      L.off_pv.push_back(o); o += al256((size_t)tiles * M * 4);
+      L.off_pi.push_back(o); o += al256((size_t)tiles * M * 4);
+    } else {
+      L.off_pv.push_back(0);
+      L.off_pi.push_back(0);
+    }
+  }
+  L.total = o;
+  return L;
 }
 
-static int launch_mxf4(const uint16_t* X, const uint8_t* q, const uint8_t* sf, const float* ts, long long M,
-                       long long N, long long K, void* Y, int y_dtype, void* workspace, bool verify, float** pv_out,
-                       int** pi_out, int* nparts_out, cudaStream_t s) {
-  MxPlan pl = mx_plan(M, N, K);
-  size_t off_part, off_xq, off_xs, off_xg, off_pv, off_pi, total;
-  mx_ws_layout(M, N, K, &off_part, &off_xq, &off_xs, &off_xg, &off_pv, &off_pi, &total);
-  char* ws = static_cast<char*>(workspace);
+static int fill_problem(Problem* P, const MxHostProblem& h, const WsLayout& L, int i, unsigned long long unit0,
+                        char* ws, int ku) {
+  std::memset(static_cast<void*>(P), 0, sizeof(Problem));
+  if (!map_u8(&P->tm_q, h.q, h.K / 2, h.N, kKC / 2, kTileRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map_u8(&P->tm_sf, h.sf, h.K / 16, h.N, (uint32_t)(ku * kKC / 16), kTileRows, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return set_error(NVFP4WS_ERR_CUDA, "cuTensorMapEncodeTiled failed (block-scaled path)");
+  P->X = h.X;
+  P->ximg = reinterpret_cast<uint8_t*>(ws + L.off_img[i]);
+  P->xg = reinterpret_cast<float*>(ws + L.off_xg[i]);
+  P->ts = h.ts;
+  P->Y = h.Y;
+  P->part_val = h.verify ? reinterpret_cast<float*>(ws + L.off_pv[i]) : nullptr;
+  P->part_idx = h.verify ? reinterpret_cast<int*>(ws + L.off_pi[i]) : nullptr;
+  P->N = h.N;
+  P->unit0 = (unsigned int)unit0;
+  P->K = (int)h.K;
+  P->kch = (int)(h.K / (kKC * ku));
+  P->tiles = (int)((h.N + kTileRows - 1) / kTileRows);
+  P->y_bf16 = h.y_bf16;
+  P->verify = h.verify;
+  return NVFP4WS_OK;
+}
 
-  // 1) activation decomposition
-  XPrepArgs xa{};
-  xa.X = X; xa.M = (int)M; xa.T = pl.T; xa.K = K;
-  xa.xq = reinterpret_cast<uint8_t*>(ws + off_xq);
-  xa.xs = reinterpret_cast<uint8_t*>(ws + off_xs);
-  xa.xg = reinterpret_cast<float*>(ws + off_xg);
-  const int bpt = (int)((K / 16 + kPrepThreads - 1) / kPrepThreads);
-  if (bpt <= 1) x_prep_kernel<1><<<(int)M, kPrepThreads, 0, s>>>(xa);
-  else if (bpt == 2) x_prep_kernel<2><<<(int)M, kPrepThreads, 0, s>>>(xa);
-  else if (bpt == 3) x_prep_kernel<3><<<(int)M, kPrepThreads, 0, s>>>(xa);
-  else x_prep_kernel<4><<<(int)M, kPrepThreads, 0, s>>>(xa);
-  if (int e = check_launch("x_prep_kernel")) return e;
-
-  // 2) the GEMM, launched as a programmatic dependent of the prep kernel
-  alignas(64) CUtensorMap tq, tsf, txq, txs;
-  if (!map_u8(&tq, q, K / 2, N, kKC / 2, kTileRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !map_u8(&tsf, sf, K / 16, N, kKC / 16, kTileRows, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !map_u8(&txq, ws + off_xq, K / 2, pl.nb, kKC / 2, pl.nb_tile, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !map_u8(&txs, ws + off_xs, K / 16, pl.nb, kKC / 16, pl.nb_tile, CU_TENSOR_MAP_SWIZZLE_NONE))
-    return set_error(NVFP4WS_ERR_CUDA, "cuTensorMapEncodeTiled failed (mxf4 path)");
-  Params p{};
-  p.Y = static_cast<float*>(Y);
-  p.y_bf16 = (y_dtype == NVFP4WS_Y_BF16);
-  p.ts = ts;
-  p.xg = reinterpret_cast<const float*>(ws + off_xg);
-  p.M = (int)M; p.T = pl.T; p.nb = pl.nb; p.nbt = pl.nbt; p.nb_tile = pl.nb_tile; p.nsfb = pl.nsfb;
-  p.N = N; p.K = K; p.tiles = pl.tiles; p.kch = pl.kch; p.units = pl.units; p.grid = pl.grid; p.stages = pl.stages;
-  p.stage_bytes = pl.stage_bytes; p.xq_off = pl.xq_off; p.sfw_off = pl.sfw_off; p.xs_off = pl.xs_off;
-  p.acc_bufs = pl.acc_bufs; p.sf_bufs = pl.sf_bufs; p.sf_cols = pl.sf_cols; p.acc_col0 = pl.acc_col0; p.acc_stride = pl.acc_stride;
-  p.counters = reinterpret_cast<unsigned int*>(ws);
-  p.partials = reinterpret_cast<float*>(ws + off_part);
-  p.verify = verify ? 1 : 0;
-  p.part_val = reinterpret_cast<float*>(ws + off_pv);
-  p.part_idx = reinterpret_cast<int*>(ws + off_pi);
-  if (verify) { *pv_out = p.part_val; *pi_out = p.part_idx; *nparts_out = pl.tiles; }
-  p.err = device_error_word();
-  if (!p.err) return set_error(NVFP4WS_ERR_CUDA, "cannot resolve the device error word");
+static int ensure_attrs() {
   static bool attr_set[64] = {};
   int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(mxf4_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess ||
-        cudaFuncSetAttribute(mxf4_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
-      return check_launch("cudaFuncSetAttribute(mxf4_kernel)");
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+    return set_error(NVFP4WS_ERR_CUDA, "cannot get the current device");
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(pass_kernel<1, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess ||
+        cudaFuncSetAttribute(pass_kernel<1, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess ||
+        cudaFuncSetAttribute(pass_kernel<2, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
+      return check_launch("cudaFuncSetAttribute(pass_kernel)");
     attr_set[dev] = true;
   }
+  return NVFP4WS_OK;
+}
+
+// Enqueue prep + GEMM. `single` is used when `probs_dev` is null (one problem).
+struct PassTables {           // device wave tables of a pass (all null for one GEMM)
+  const uint32_t* wave_u0;
+  const int* cta_prob;
+  const int* cta_units;
+  int nwave;
+};
+
+static int launch_pass(const Problem& single, const Problem* probs_dev, const PassTables& tb, int nprob,
+                       const MxPlan& pl, int grid, unsigned long long units, size_t off_part, long long max_k,
+                       char* ws, cudaStream_t s) {
+  if (units * (unsigned long long)grid >= (1ull << 32))
+    return set_error(NVFP4WS_ERR_UNSUPPORTED, "block-scaled path: too many units for the stream-K partition");
+  if (int e = ensure_attrs()) return e;
+
+  // 1) activation decomposition (programmatic dependent launch: it may start while the
+  //    previous kernel of the stream finishes, and waits for it before any access)
+  {
+    const int bpt = (int)((max_k / 16 + kPrepThreads - 1) / kPrepThreads);
+    cudaLaunchConfig_t pc = {};
+    pc.gridDim = dim3((unsigned)pl.g.M, (unsigned)nprob);
+    pc.blockDim = dim3(kPrepThreads);
+    pc.stream = s;
+    cudaLaunchAttribute pa[1];
+    pa[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pa[0].val.programmaticStreamSerializationAllowed = 1;
+    pc.attrs = pa;
+    pc.numAttrs = 1;
+    const Geom g = pl.g;
+    cudaError_t pe = (bpt <= 1) ? cudaLaunchKernelEx(&pc, x_prep_kernel<1>, single, probs_dev, g)
+                     : (bpt == 2) ? cudaLaunchKernelEx(&pc, x_prep_kernel<2>, single, probs_dev, g)
+                     : (bpt == 3) ? cudaLaunchKernelEx(&pc, x_prep_kernel<3>, single, probs_dev, g)
+                                  : cudaLaunchKernelEx(&pc, x_prep_kernel<4>, single, probs_dev, g);
+    if (pe != cudaSuccess) return set_error(NVFP4WS_ERR_CUDA, "x_prep_kernel launch: %s", cudaGetErrorString(pe));
+    if (int e = check_launch("x_prep_kernel")) return e;
+  }
+
+  // 2) the GEMM, a programmatic dependent of the prep kernel
+  PassParams p{};
+  p.g = pl.g;
+  p.probs = probs_dev;
+  p.nprob = nprob;
+  p.wave_u0 = tb.wave_u0;
+  p.cta_prob = tb.cta_prob;
+  p.cta_units = tb.cta_units;
+  p.nwave = tb.nwave;
+  p.units = (unsigned int)units;
+  p.grid = grid;
+  p.stages = pl.stages;
+  p.stage_bytes = pl.stage_bytes;
+  p.acc_bufs = pl.acc_bufs;
+  p.sf_bufs = pl.sf_bufs;
+  p.sf_cols = pl.sf_cols;
+  p.acc_col0 = pl.acc_col0;
+  p.acc_stride = pl.acc_stride;
+  p.counters = reinterpret_cast<unsigned int*>(ws);
+  p.partials = reinterpret_cast<float*>(ws + off_part);
+  p.err = device_error_word();
+  if (!p.err) return set_error(NVFP4WS_ERR_CUDA, "cannot resolve the device error word");
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(pl.grid);
+  cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = pl.smem;
   cfg.stream = s;
@@ -851,25 +1057,148 @@ static int launch_mxf4(const uint16_t* X, const uint8_t* q, const uint8_t* sf, c
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = (pl.nbt == 1) ? cudaLaunchKernelEx(&cfg, mxf4_kernel<1>, tq, tsf, txq, txs, p)
-                                 : cudaLaunchKernelEx(&cfg, mxf4_kernel<2>, tq, tsf, txq, txs, p);
-  if (e != cudaSuccess) return set_error(NVFP4WS_ERR_CUDA, "mxf4_kernel launch: %s", cudaGetErrorString(e));
-  return check_launch("mxf4_kernel");
+  cudaError_t e = (pl.g.nbt == 2)  ? cudaLaunchKernelEx(&cfg, pass_kernel<2, 1>, single, p)
+                  : (pl.g.ku == 2) ? cudaLaunchKernelEx(&cfg, pass_kernel<1, 2>, single, p)
+                                   : cudaLaunchKernelEx(&cfg, pass_kernel<1, 1>, single, p);
+  if (e != cudaSuccess) return set_error(NVFP4WS_ERR_CUDA, "pass_kernel launch: %s", cudaGetErrorString(e));
+  return check_launch("pass_kernel");
+}
+
+size_t mxf4_workspace_bytes(long long M, long long N, long long K) {
+  if (!mxf4_supported(M, K)) return 0;
+  MxHostProblem h{nullptr, nullptr, nullptr, nullptr, N, K, nullptr, 0, 1};   // sized with the verify tail
+  return mx_layout(&h, 1, M, false).total;
+}
+
+static int launch_single(const MxHostProblem& h, long long M, void* workspace, cudaStream_t s, Problem* out) {
+  const MxPlan pl = mx_plan(M, all_k512(&h, 1));
+  const WsLayout L = mx_layout(&h, 1, M, false);
+  char* ws = static_cast<char*>(workspace);
+  if (int e = fill_problem(out, h, L, 0, 0, ws, pl.g.ku)) return e;
+  const PassTables none{nullptr, nullptr, nullptr, 1};
+  return launch_pass(*out, nullptr, none, 1, pl, L.grid, L.units, L.off_part, h.K, ws, s);
 }
 
 int launch_mxf4_gemm(const uint16_t* X, const uint8_t* q, const uint8_t* sf, const float* ts, long long M,
                      long long N, long long K, void* Y, int y_dtype, void* workspace, cudaStream_t s) {
-  return launch_mxf4(X, q, sf, ts, M, N, K, Y, y_dtype, workspace, false, nullptr, nullptr, nullptr, s);
+  MxHostProblem h{X, q, sf, ts, N, K, Y, y_dtype == NVFP4WS_Y_BF16 ? 1 : 0, 0};
+  Problem P;
+  return launch_single(h, M, workspace, s, &P);
 }
 
 int launch_mxf4_verify(const uint16_t* X, const uint8_t* q, const uint8_t* sf, const float* ts, long long M,
                        long long N, long long K, const int32_t* drafts, int B, int D, int32_t* argmax,
                        int32_t* accept_len, float* max_logit, void* workspace, cudaStream_t s) {
-  float* pv = nullptr;
-  int* pi = nullptr;
-  int nparts = 0;
-  if (int e = launch_mxf4(X, q, sf, ts, M, N, K, nullptr, 0, workspace, true, &pv, &pi, &nparts, s)) return e;
-  return launch_verify_stage2(pv, pi, nparts, (int)M, drafts, B, D, argmax, accept_len, max_logit, s);
+  MxHostProblem h{X, q, sf, ts, N, K, nullptr, 0, 1};
+  Problem P;
+  if (int e = launch_single(h, M, workspace, s, &P)) return e;
+  return launch_verify_stage2(P.part_val, P.part_idx, P.tiles, (int)M, drafts, B, D, argmax, accept_len, max_logit, s);
+}
+
+// ------------------------------------------------------------------ multi-problem passes
+
+// Host state of a pass: plain data in caller-owned memory (no allocation).
+struct MxPassState {
+  uint32_t magic;
+  int nprob, grid, verify, vtiles, k512;
+  long long M, max_k;
+  unsigned long long units;
+  size_t off_part;
+  char* ws;
+  Problem* probs_dev;
+  PassTables tb;
+  float* pv;
+  int* pi;
+  MxVerifySpec vs;
+};
+static_assert(sizeof(MxPassState) <= kMxPassStateBytes, "pass state does not fit the caller's handle");
+constexpr uint32_t kPassMagic = 0x4e565053u;
+
+size_t mxf4_pass_workspace_bytes(const MxHostProblem* hp, int n, long long M) {
+  return mx_layout(hp, n, M, true).total;
+}
+
+int mxf4_pass_init(void* state, const MxHostProblem* hp, int n, long long M, const MxVerifySpec* vs, void* workspace,
+                   size_t workspace_bytes) {
+  MxPassState* P = static_cast<MxPassState*>(state);
+  std::memset(static_cast<void*>(P), 0, sizeof(MxPassState));
+  const WsLayout L = mx_layout(hp, n, M, true);
+  const int ku = mx_plan(M, all_k512(hp, n)).g.ku;
+  if (workspace_bytes < L.total)
+    return set_error(NVFP4WS_ERR_WORKSPACE, "nvfp4_pass_init: workspace %zu bytes < required %zu", workspace_bytes,
+                     L.total);
+  char* ws = static_cast<char*>(workspace);
+  std::vector<Problem> host(n);
+  std::vector<unsigned long long> first(n);
+  unsigned long long unit0 = 0;
+  long long max_k = 0;
+  for (int i = 0; i < n; ++i) {
+    first[i] = unit0;
+    if (int e = fill_problem(&host[i], hp[i], L, i, unit0, ws, ku)) return e;
+    unit0 += (unsigned long long)host[i].tiles * (unsigned long long)host[i].kch;
+    max_k = std::max(max_k, hp[i].K);
+  }
+  // wave tables: wave starts, each CTA's first problem in each wave, each CTA's unit count
+  std::vector<uint32_t> wave_u0(L.nwave + 1);
+  std::vector<int> cta_prob((size_t)L.nwave * L.grid), cta_units(L.grid, 0);
+  for (int w = 0; w < L.nwave; ++w) {
+    const unsigned long long w0 = first[L.wave_first[w]];
+    const unsigned long long w1 = (L.wave_first[w + 1] < n) ? first[L.wave_first[w + 1]] : unit0;
+    wave_u0[w] = (uint32_t)w0;
+    const unsigned long long Uw = w1 - w0;
+    if (Uw < (unsigned long long)L.grid)
+      return set_error(NVFP4WS_ERR_UNSUPPORTED, "nvfp4_pass_init: internal wave plan has a wave of %llu < %d units",
+                       Uw, L.grid);
+    for (int c = 0, i = L.wave_first[w]; c < L.grid; ++c) {
+      const unsigned long long b = w0 + (unsigned long long)c * Uw / (unsigned long long)L.grid;
+      const unsigned long long e = w0 + (unsigned long long)(c + 1) * Uw / (unsigned long long)L.grid;
+      while (i + 1 < n && first[i + 1] <= b) ++i;
+      cta_prob[(size_t)w * L.grid + c] = i;
+      cta_units[c] += (int)(e - b);
+    }
+  }
+  wave_u0[L.nwave] = (uint32_t)unit0;
+  Problem* probs_dev = reinterpret_cast<Problem*>(ws + L.off_desc);
+  uint32_t* wave_dev = reinterpret_cast<uint32_t*>(ws + L.off_wave);
+  int* cta_dev = reinterpret_cast<int*>(ws + L.off_cta);
+  int* cunits_dev = reinterpret_cast<int*>(ws + L.off_cunits);
+  if (cudaMemcpy(probs_dev, host.data(), sizeof(Problem) * (size_t)n, cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(wave_dev, wave_u0.data(), sizeof(uint32_t) * wave_u0.size(), cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(cta_dev, cta_prob.data(), sizeof(int) * cta_prob.size(), cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(cunits_dev, cta_units.data(), sizeof(int) * cta_units.size(), cudaMemcpyHostToDevice) != cudaSuccess)
+    return check_launch("nvfp4_pass_init: descriptor upload");
+  P->nprob = n;
+  P->k512 = all_k512(hp, n) ? 1 : 0;
+  P->grid = L.grid;
+  P->units = L.units;
+  P->off_part = L.off_part;
+  P->M = M;
+  P->max_k = max_k;
+  P->ws = ws;
+  P->probs_dev = probs_dev;
+  P->tb = PassTables{wave_dev, cta_dev, cunits_dev, L.nwave};
+  P->verify = vs != nullptr;
+  if (vs) {
+    P->vs = *vs;
+    P->pv = host[n - 1].part_val;
+    P->pi = host[n - 1].part_idx;
+    P->vtiles = host[n - 1].tiles;
+  }
+  P->magic = kPassMagic;
+  return NVFP4WS_OK;
+}
+
+int mxf4_pass_run(const void* state, cudaStream_t s) {
+  const MxPassState* P = static_cast<const MxPassState*>(state);
+  if (P->magic != kPassMagic) return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_pass_run: pass not initialised");
+  static const Problem kNoProblem{};   // the kernels' by-value problem slot, unused by a pass
+  const MxPlan pl = mx_plan(P->M, P->k512 != 0);
+  if (int e = launch_pass(kNoProblem, P->probs_dev, P->tb, P->nprob, pl, P->grid, P->units, P->off_part,
+                          P->max_k, P->ws, s))
+    return e;
+  if (!P->verify) return NVFP4WS_OK;
+  return launch_verify_stage2(P->pv, P->pi, P->vtiles, (int)P->M, P->vs.drafts, P->vs.B, P->vs.D, P->vs.argmax,
+                              P->vs.accept_len, P->vs.max_logit, s);
 }
 
 }  // namespace nvfp4ws
@@ -880,7 +1209,7 @@ extern "C" int nvfp4ws_trace_read(unsigned long long* host, int n) {
   if (n > 16 * 64) n = 16 * 64;
   return cudaMemcpyFromSymbol(host, nvfp4ws::mxk::g_trace, sizeof(unsigned long long) * n) == cudaSuccess ? 0 : 5;
 }
-// Per-CTA global-timer events: [256][8] (GEMM CTAs 0..147; prep kernel rows at 200+m).
+// Per-CTA global-timer events: [256][16] (GEMM CTAs 0..147; prep kernel rows at 200+m).
 extern "C" int nvfp4ws_trace_cta_read(unsigned long long* host) {
   return cudaMemcpyFromSymbol(host, nvfp4ws::mxk::g_cta_trace, sizeof(unsigned long long) * 256 * 16) == cudaSuccess ? 0 : 5;
 }

@@ -66,8 +66,11 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   if (mbar_try_wait(bar, parity)) return true;          // fast path: the phase is usually complete
   const unsigned long long t0 = globaltimer();
   while (true) {
+// Waiting warps let try_wait suspend them (up to this long per try) instead of spinning:
+// measured on B200, spinning warps take issue slots from the single MMA-issuing thread that
+// shares their SM sub-partition.
 #ifndef NVFP4WS_WAIT_HINT_NS
-#define NVFP4WS_WAIT_HINT_NS 0u
+#define NVFP4WS_WAIT_HINT_NS 20000u
 #endif
     if (NVFP4WS_WAIT_HINT_NS == 0u ? mbar_try_wait(bar, parity) : mbar_try_wait_sleep(bar, parity, NVFP4WS_WAIT_HINT_NS))
       return true;

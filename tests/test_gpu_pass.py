@@ -1,0 +1,214 @@
+"""GPU parity of weight passes (nvfp4_pass_*): lists of GEMMs sharing M, run by one
+persistent launch, against the CPU oracle on the same seeded inputs.
+
+A pass splits the concatenated (problem, tile, K-chunk) units of the whole list
+evenly across the SMs. So besides ragged shapes these cases cover: a list with
+fewer units than SMs (one unit per CTA, so nearly every tile is split), CTA ranges
+that cross several problems, tiles split three or more ways, mixed K, M up to the
+two-B-tile layout (M=68), a verify problem at the end, run-to-run determinism, and
+the full-size layer shapes on sampled outputs.
+
+Bars as in the other parity tests: GEMM rows within 2e-3 of max|y_ref|; argmax and
+accept lengths bit-exact away from near ties (top-2 gap < 1e-3).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import synthetic as S
+from oracle import gemm as G
+from oracle import nvfp4 as F
+from oracle import verify as V
+
+pytestmark = pytest.mark.gpu
+REL_TOL = 2e-3
+
+
+@pytest.fixture(scope="module")
+def nv():
+    import nvfp4_weight_streaming_gemm_b200 as nv
+    from nvfp4_weight_streaming_gemm_b200 import build
+    build.build()
+    return nv
+
+
+def to_dev_bf16(x_bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(x_bits.view(np.int16).copy()).view(torch.bfloat16).cuda()
+
+
+def assert_rowwise(y: np.ndarray, y_ref: np.ndarray, rel=REL_TOL):
+    err = np.abs(y.astype(np.float64) - y_ref).max(axis=1)
+    scale = np.abs(y_ref).max(axis=1)
+    worst = (err / np.maximum(scale, 1e-300)).max()
+    assert (err <= rel * scale).all(), f"rowwise error {worst:.3e} > {rel}"
+
+
+def make_problems(nv, shapes, M, seed, y_dtype=torch.float32):
+    probs, refs = [], []
+    for i, (N, K) in enumerate(shapes):
+        W, x = S.random_case(seed + 31 * i, M, N, K)
+        q, sf, ts = nv.pack(torch.from_numpy(W).cuda())
+        Y = torch.full((M, N), float("nan"), dtype=y_dtype, device="cuda")
+        probs.append((to_dev_bf16(x), q, sf, ts, Y))
+        refs.append((W, x))
+    return probs, refs
+
+
+def oracle_y(W, x):
+    q, sf, ts = F.quantize_nvfp4(W)
+    return G.gemm_ref(x, q, sf, ts)
+
+
+def units(shapes):
+    return sum(((N + 127) // 128) * (K // 256) for N, K in shapes)
+
+
+@pytest.mark.parametrize("M", [1, 2, 17, 68])
+def test_pass_fewer_units_than_sms(nv, M):
+    """84 units over at most 148 SMs: one unit per CTA, nearly every tile split."""
+    shapes = [(300, 512), (1000, 1024), (130, 768), (4096, 256), (77, 2048)]
+    assert units(shapes) < nv.lib().nvfp4ws_sm_count()
+    probs, refs = make_problems(nv, shapes, M, 500 + M)
+    p = nv.WeightPass(probs, M)
+    p.run()
+    torch.cuda.synchronize()
+    nv.check()
+    for (_, _, _, _, Y), (W, x) in zip(probs, refs):
+        assert_rowwise(Y.cpu().numpy(), oracle_y(W, x))
+
+
+@pytest.mark.parametrize("M", [1, 17, 68])
+def test_pass_many_problems(nv, M):
+    """24 problems, mixed K: CTA ranges cross problem boundaries and split tiles."""
+    rng = np.random.default_rng(40 + M)
+    shapes = [(int(rng.integers(100, 3000)), int(rng.choice([256, 512, 1280, 2560]))) for _ in range(24)]
+    assert units(shapes) > 2 * nv.lib().nvfp4ws_sm_count()
+    probs, refs = make_problems(nv, shapes, M, 900 + M)
+    p = nv.WeightPass(probs, M)
+    p.run()
+    torch.cuda.synchronize()
+    nv.check()
+    for (_, _, _, _, Y), (W, x) in zip(probs, refs):
+        assert_rowwise(Y.cpu().numpy(), oracle_y(W, x))
+
+
+def test_pass_deterministic_bf16_and_repeat(nv):
+    """Runs reuse the workspace (tickets reset themselves) and give identical bits;
+    bf16 Y is the fp32 result rounded once."""
+    M = 17
+    shapes = [(2000, 1024), (640, 2560), (3000, 512)]
+    probs, refs = make_problems(nv, shapes, M, 77)
+    p = nv.WeightPass(probs, M)
+    p.run()
+    torch.cuda.synchronize()
+    first = [pr[4].clone() for pr in probs]
+    for _ in range(3):
+        for pr in probs:
+            pr[4].fill_(float("nan"))
+        p.run()
+    torch.cuda.synchronize()
+    nv.check()
+    for pr, y0 in zip(probs, first):
+        assert torch.equal(pr[4], y0)
+    probs16 = [(X, q, sf, ts, torch.empty(Y.shape, dtype=torch.bfloat16, device="cuda")) for X, q, sf, ts, Y in probs]
+    p16 = nv.WeightPass(probs16, M)
+    p16.run()
+    torch.cuda.synchronize()
+    for pr16, y0 in zip(probs16, first):
+        assert torch.equal(pr16[4], y0.to(torch.bfloat16))
+
+
+def test_pass_agrees_with_single_gemm(nv):
+    """The same problem through the pass and through nvfp4_gemm_skinny's block-scaled
+    path: both within the bar of the oracle (their split points differ)."""
+    M = 17
+    shapes = [(5000, 1280)]
+    probs, refs = make_problems(nv, shapes, M, 123)
+    nv.WeightPass(probs, M).run()
+    X, q, sf, ts, Y = probs[0]
+    Y1 = nv.gemm(X, q, sf, ts, path="mma")
+    torch.cuda.synchronize()
+    y_ref = oracle_y(*refs[0])
+    assert_rowwise(Y.cpu().numpy(), y_ref)
+    assert_rowwise(Y1.cpu().numpy(), y_ref)
+
+
+@pytest.mark.parametrize("B,D", [(1, 16), (4, 16), (2, 0)])
+def test_pass_with_verify_tail(nv, B, D):
+    """Two GEMMs, then the lm_head as the verify problem of the same launch."""
+    M = B * (D + 1)
+    probs, refs = make_problems(nv, [(1500, 512), (700, 1280)], M, 300 + B + D)
+    N, K = 20000, 1024
+    W, x = S.random_case(600 + B + D, M, N, K, w_std=0.05)
+    y_ref = oracle_y(W, x)
+    t_ref = V.argmax_fast(y_ref)
+    Lstar = np.random.default_rng(B * 7 + D).integers(0, D + 1, size=B)
+    drafts = S.drafts_with_prefix(t_ref, Lstar, D, N)
+    L_ref = V.accept_ref(t_ref, drafts, D)
+    q, sf, ts = nv.pack(torch.from_numpy(W).cuda())
+    probs.append((to_dev_bf16(x), q, sf, ts, None))
+    t = torch.full((M,), -1, dtype=torch.int32, device="cuda")
+    L = torch.full((B,), -1, dtype=torch.int32, device="cuda")
+    vmax = torch.empty(M, dtype=torch.float32, device="cuda")
+    p = nv.WeightPass(probs, M, verify=(torch.from_numpy(drafts).cuda(), t, L, vmax))
+    p.run()
+    torch.cuda.synchronize()
+    nv.check()
+    for (_, _, _, _, Y), (Wi, xi) in zip(probs[:2], refs):
+        assert_rowwise(Y.cpu().numpy(), oracle_y(Wi, xi))
+    t, L, vmax = t.cpu().numpy(), L.cpu().numpy(), vmax.cpu().numpy()
+    gap = V.top2_gap(y_ref)
+    rows = V.comparable_rows(gap)
+    seqs = V.comparable_sequences(gap, L_ref, D)
+    assert np.array_equal(t[rows], t_ref[rows])
+    assert np.array_equal(L[seqs], L_ref[seqs])
+    ymax = y_ref[np.arange(M), t]
+    assert (np.abs(vmax - ymax) <= REL_TOL * np.abs(y_ref).max(axis=1)).all()
+    assert (y_ref.max(axis=1) - ymax <= V.NEAR_TIE).all()
+
+
+def test_pass_layer_shapes_sampled(nv):
+    """The 27B layer shapes at M=17 in one pass with the full 248,320-row lm_head as
+    its verify tail: sampled outputs against the oracle, computed element by element
+    from the oracle's quantisation of the sampled weight rows."""
+    M, D = 17, S.DRAFT_LEN
+    probs, sampled = [], []
+    rng = np.random.default_rng(2024)
+    for name in S.LAYER_ORDER:
+        W, x = S.layer(name, M=M)
+        q, sf, ts = nv.pack(torch.from_numpy(W).cuda())
+        Y = torch.full((M, W.shape[0]), float("nan"), dtype=torch.float32, device="cuda")
+        probs.append((to_dev_bf16(x), q, sf, ts, Y))
+        rows = rng.choice(W.shape[0], 256, replace=False)
+        sampled.append((W[rows].copy(), rows, x, F.tensor_scale(W)))
+        del W
+    Wl, xl, _ = S.lmhead_inputs(N=S.VOCAB, B=1)
+    ql, sfl, tsl = nv.pack(torch.from_numpy(Wl).cuda())
+    drafts = np.random.default_rng(11).integers(0, S.VOCAB, size=(1, D)).astype(np.int32)
+    probs.append((to_dev_bf16(xl), ql, sfl, tsl, None))
+    t = torch.empty(M, dtype=torch.int32, device="cuda")
+    L = torch.empty(1, dtype=torch.int32, device="cuda")
+    vmax = torch.empty(M, dtype=torch.float32, device="cuda")
+    p = nv.WeightPass(probs, M, verify=(torch.from_numpy(drafts).cuda(), t, L, vmax))
+    p.run()
+    torch.cuda.synchronize()
+    nv.check()
+    for (_, _, _, _, Y), (Wr, rows, x, ts_ref) in zip(probs, sampled):
+        q_r, sf_r, _ = F.quantize_nvfp4(Wr, ts_ref)
+        y_s = G.gemm_ref(x, q_r, sf_r, ts_ref)             # oracle at the sampled rows, all tokens
+        y_full = Y.cpu().numpy()
+        assert np.isfinite(y_full).all()
+        scale = np.abs(y_s).max(axis=1)                    # the sampled rows' magnitude stands in for max|y|
+        assert (np.abs(y_full[:, rows] - y_s).max(axis=1) <= REL_TOL * scale).all()
+    t, L, vmax = t.cpu().numpy(), L.cpu().numpy(), vmax.cpu().numpy()
+    rows = np.unique(np.concatenate([t, np.random.default_rng(12).choice(S.VOCAB, 3000, replace=False)]))
+    ts_l = F.tensor_scale(Wl)
+    q_r, sf_r, _ = F.quantize_nvfp4(Wl[rows], ts_l)
+    y_s = G.gemm_ref(xl, q_r, sf_r, ts_l)
+    col = {int(r): i for i, r in enumerate(rows)}
+    for m in range(M):
+        y_t = y_s[m, col[int(t[m])]]
+        assert abs(vmax[m] - y_t) <= 1e-4 * max(1.0, abs(y_t))
+        assert (y_s[m] <= y_t + V.NEAR_TIE).all()
+    assert np.array_equal(L, V.accept_ref(t, drafts, D))
