@@ -5,10 +5,13 @@ Step = one pass of the whole hot path over resident synthetic weights:
   64 layers x {gate+up 5120->34816, down 17408->5120, qkv 5120->10240} NVFP4 GEMMs
   followed by the fused lm_head verify (5120->248,320 rows, argmax + accept length).
 The headline is M = 17 (16 drafted tokens + 1). M = 1 (plain decode) and M = 68
-(4 sequences x 17 sharing one read) are reported in ``per_m``. Each pass is
-captured as two CUDA graphs (the 192 GEMMs, then the verify) and replayed; CUDA
-events on the launching stream bracket both. The weight stack (11.5 GB) is far
-larger than L2, so no flush is needed between steps.
+(4 sequences x 17 sharing one read) are reported in ``per_m``. Each pass is one
+weight pass of the library (activation prep, the persistent pass kernel over all
+193 GEMMs with the lm_head as its verify problem, verify stage 2), captured in a
+CUDA graph and replayed; CUDA events on the launching stream bracket every step.
+Beside it, ``chained_ms_per_pass`` times the same work as 193 per-GEMM launches in
+layer order. The weight stack (11.5 GB) is far larger than L2, so no flush is
+needed between steps.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 

@@ -84,7 +84,6 @@ constexpr uint32_t kWChunk = kNibBytes + kSfBytes; // weight bytes per chunk (10
 constexpr int kMaxStages = 12;
 constexpr int kMaxB = 352;                         // B rows (tokens x terms) the TMEM budget allows
 constexpr size_t kTailBytes = 8192;
-constexpr int kPrepThreads = 512;                  // K <= 512 * 4 * 16 = 32768 with 4 blocks per thread
 constexpr int kMaxSfBufs = 8;
 
 // One GEMM of a launch. Lives in device memory (a pass) or in the kernel's parameter
@@ -144,101 +143,113 @@ __device__ __forceinline__ float block_amax16(const float (&v)[16]) {
   return a;
 }
 
-// Grid (M, problems). Repeated multiplication by 0.25 is exact unless g underflows;
-// the decomposition and the stored g follow the same sequence.
-template <int BPT>
-__global__ void __launch_bounds__(kPrepThreads) x_prep_kernel(const __grid_constant__ Problem single,
-                                                               const Problem* probs, const Geom g) {
+// One CTA per (activation row, problem). A first sweep over the row finds amax|x|
+// (one CTA reduction), a second re-reads it (from L2) and writes the T terms of each
+// 16-element block. Per-thread state is small, so several CTAs fit an SM and the many
+// short rows of a pass are prepared at once. Repeated
+// multiplication by 0.25 is exact unless g underflows; the decomposition and the stored
+// g follow the same sequence. The code and scale choices only need to be consistent
+// with the residual they leave (which is exact), so they use reciprocal multiplies.
+constexpr int kPrepThreads = 256;
+
+__device__ __forceinline__ void load_block16(const uint16_t* X, int b, float (&r)[16]) {
+  const uint4* src = reinterpret_cast<const uint4*>(X + (long long)b * 16);
+  const uint4 u0 = __ldg(src), u1 = __ldg(src + 1);
+  const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    r[2 * i] = __uint_as_float(w[i] << 16);
+    r[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// The T terms of block b (16 values in r) into the chunk images; gt0 = g_0, inv6 = 1/(6 g_t).
+template <int T>
+__device__ __forceinline__ void quantise_block(float (&r)[16], int b, int m, float gt0, const float (&inv6)[T],
+                                               const Geom& g, uint8_t* img) {
+  const int kc = b >> 4, bi = b & 15;           // K-chunk and block within it
+  uint8_t* base = img + (size_t)kc * g.img_stride;
+  float gt = gt0;
+#pragma unroll
+  for (int term = 0; term < T; ++term, gt *= 0.25f) {
+    uint32_t sbits = 0, lo = 0, hi = 0;
+    if (gt > 0.f) {
+      uint16_t s2;
+      asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(s2) : "f"(0.0f), "f"(block_amax16(r) * inv6[term]));
+      sbits = s2 & 0xFFu;
+      const float den = f16lo_to_f32(e4m3x2_to_f16x2(sbits)) * gt;
+      if (den > 0.f) {
+        const float inv = rcp_approx(den);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          uint16_t c2;
+          asm("{ .reg .b8 b; cvt.rn.satfinite.e2m1x2.f32 b, %1, %2; cvt.u16.u8 %0, b; }"
+              : "=h"(c2) : "f"(r[2 * i + 1] * inv), "f"(r[2 * i] * inv));
+          const uint32_t h = e2m1x2_to_f16x2(c2);
+          r[2 * i] = fmaf(-f16lo_to_f32(h), den, r[2 * i]);
+          r[2 * i + 1] = fmaf(-f16hi_to_f32(h), den, r[2 * i + 1]);
+          if (i < 4) lo |= (uint32_t)(c2 & 0xFF) << (8 * i);
+          else hi |= (uint32_t)(c2 & 0xFF) << (8 * (i - 4));
+        }
+      }
+    }
+    // B row of (token m, term): its 128 code bytes for this chunk, with the 16-byte
+    // pieces permuted by the 128-byte swizzle (piece p of row r at p ^ (r & 7)).
+    const int row = m * T + term;
+    const uint32_t off = (uint32_t)row * 128u + ((uint32_t)((bi >> 1) ^ (row & 7)) << 4) + ((uint32_t)(bi & 1) << 3);
+    *reinterpret_cast<uint2*>(base + off) = make_uint2(lo, hi);
+    base[g.img_xs_off + (uint32_t)row * 16u + (uint32_t)bi] = (uint8_t)sbits;
+  }
+}
+
+__global__ void __launch_bounds__(kPrepThreads, 6) x_prep_kernel(const __grid_constant__ Problem single,
+                                                                  const Problem* probs, const Geom g) {
   asm volatile("griddepcontrol.launch_dependents;");
   // X may come from the previous kernel of the stream, and the previous GEMM may still
   // read this workspace: nothing is read or written before that kernel has finished.
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const Problem* pr = probs ? probs + blockIdx.y : &single;
-#ifdef NVFP4WS_TRACE
-  if (threadIdx.x == 0 && blockIdx.x < 56 && blockIdx.y == 0) g_cta_trace[(200 + blockIdx.x) * 16 + 0] = globaltimer();
-#endif
-  const int m = blockIdx.x;
+  constexpr int T = kMxf4Terms;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const long long K = pr->K;
-  const int nblk = (int)(K / 16);
-  const uint16_t* X = pr->X + (long long)m * K;
+  const int m = blockIdx.x % g.M;
+  const Problem* pr = probs ? probs + blockIdx.x / g.M : &single;
+  const int nblk = pr->K / 16;
+  const uint16_t* X = pr->X + (long long)m * pr->K;
   uint8_t* img = pr->ximg;
   __shared__ float s_red[kPrepThreads / 32];
-  float r[BPT][16];
-#pragma unroll
-  for (int j = 0; j < BPT; ++j) {
-    const int b = t + j * kPrepThreads;
-    if (b < nblk) {
-      const uint4* src = reinterpret_cast<const uint4*>(X + (long long)b * 16);
-      const uint4 u0 = src[0], u1 = src[1];
-      const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        r[j][2 * i] = __uint_as_float(w[i] << 16);
-        r[j][2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) r[j][i] = 0.f;
-    }
-  }
   float amax = 0.f;
-#pragma unroll
-  for (int j = 0; j < BPT; ++j) amax = fmaxf(amax, block_amax16(r[j]));
+  for (int b = t; b < nblk; b += kPrepThreads) {
+    float r[16];
+    load_block16(X, b, r);
+    amax = fmaxf(amax, block_amax16(r));
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   if (lane == 0) s_red[warp] = amax;
   __syncthreads();
-  float row_amax = 0.f;
+  amax = 0.f;
 #pragma unroll
-  for (int w = 0; w < kPrepThreads / 32; ++w) row_amax = fmaxf(row_amax, s_red[w]);
-  const float g0 = row_amax / 2688.0f;
-  if (t == 0) {
+  for (int w = 0; w < kPrepThreads / 32; ++w) amax = fmaxf(amax, s_red[w]);
+  const float g0 = amax / 2688.0f;
+  float inv6[T];
+  {
     float gt = g0;
-    for (int term = 0; term < g.T; ++term, gt *= 0.25f) pr->xg[m * g.T + term] = gt;
-  }
 #pragma unroll
-  for (int j = 0; j < BPT; ++j) {
-    const int b = t + j * kPrepThreads;
-    if (b >= nblk) continue;
-    const int kc = b >> 4, bi = b & 15;           // K-chunk and block within it
-    uint8_t* base = img + (size_t)kc * g.img_stride;
-    float gt = g0;
-    for (int term = 0; term < g.T; ++term, gt *= 0.25f) {
-      uint32_t sbits = 0, lo = 0, hi = 0;
-      if (gt > 0.f) {
-        const float want = block_amax16(r[j]) / (6.0f * gt);
-        uint16_t s2;
-        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(s2) : "f"(0.0f), "f"(want));
-        sbits = s2 & 0xFFu;
-        const float den = f16lo_to_f32(e4m3x2_to_f16x2(sbits)) * gt;
-        if (den > 0.f) {
-          const float inv = 1.0f / den;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            uint16_t c2;
-            asm("{ .reg .b8 b; cvt.rn.satfinite.e2m1x2.f32 b, %1, %2; cvt.u16.u8 %0, b; }"
-                : "=h"(c2) : "f"(r[j][2 * i + 1] * inv), "f"(r[j][2 * i] * inv));
-            const uint32_t h = e2m1x2_to_f16x2(c2);
-            r[j][2 * i] = fmaf(-f16lo_to_f32(h), den, r[j][2 * i]);
-            r[j][2 * i + 1] = fmaf(-f16hi_to_f32(h), den, r[j][2 * i + 1]);
-            if (i < 4) lo |= (uint32_t)(c2 & 0xFF) << (8 * i);
-            else hi |= (uint32_t)(c2 & 0xFF) << (8 * (i - 4));
-          }
-        }
-      }
-      // B row of (token m, term): its 128 code bytes for this chunk, with the 16-byte
-      // pieces permuted by the 128-byte swizzle (piece p of row r at p ^ (r & 7)).
-      const int row = m * g.T + term;
-      const uint32_t off = (uint32_t)row * 128u + ((uint32_t)((bi >> 1) ^ (row & 7)) << 4) + ((uint32_t)(bi & 1) << 3);
-      *reinterpret_cast<uint2*>(base + off) = make_uint2(lo, hi);
-      base[g.img_xs_off + (uint32_t)row * 16u + (uint32_t)bi] = (uint8_t)sbits;
+    for (int term = 0; term < T; ++term, gt *= 0.25f) {
+      inv6[term] = gt > 0.f ? 1.0f / (6.0f * gt) : 0.f;
+      if (t == 0) pr->xg[m * T + term] = gt;
     }
   }
-#ifdef NVFP4WS_TRACE
-  __syncthreads();
-  if (threadIdx.x == 0 && blockIdx.x < 56 && blockIdx.y == 0) g_cta_trace[(200 + blockIdx.x) * 16 + 1] = globaltimer();
-#endif
+  for (int b = t; b < nblk; b += kPrepThreads) {
+    float r[16];
+    load_block16(X, b, r);
+    quantise_block<T>(r, b, m, g0, inv6, g, img);
+  }
 }
 
 // ------------------------------------------------------------------ GEMM
@@ -1006,9 +1017,8 @@ static int launch_pass(const Problem& single, const Problem* probs_dev, const Pa
   // 1) activation decomposition (programmatic dependent launch: it may start while the
   //    previous kernel of the stream finishes, and waits for it before any access)
   {
-    const int bpt = (int)((max_k / 16 + kPrepThreads - 1) / kPrepThreads);
     cudaLaunchConfig_t pc = {};
-    pc.gridDim = dim3((unsigned)pl.g.M, (unsigned)nprob);
+    pc.gridDim = dim3((unsigned)(pl.g.M * nprob));
     pc.blockDim = dim3(kPrepThreads);
     pc.stream = s;
     cudaLaunchAttribute pa[1];
@@ -1017,10 +1027,7 @@ static int launch_pass(const Problem& single, const Problem* probs_dev, const Pa
     pc.attrs = pa;
     pc.numAttrs = 1;
     const Geom g = pl.g;
-    cudaError_t pe = (bpt <= 1) ? cudaLaunchKernelEx(&pc, x_prep_kernel<1>, single, probs_dev, g)
-                     : (bpt == 2) ? cudaLaunchKernelEx(&pc, x_prep_kernel<2>, single, probs_dev, g)
-                     : (bpt == 3) ? cudaLaunchKernelEx(&pc, x_prep_kernel<3>, single, probs_dev, g)
-                                  : cudaLaunchKernelEx(&pc, x_prep_kernel<4>, single, probs_dev, g);
+    cudaError_t pe = cudaLaunchKernelEx(&pc, x_prep_kernel, single, probs_dev, g);
     if (pe != cudaSuccess) return set_error(NVFP4WS_ERR_CUDA, "x_prep_kernel launch: %s", cudaGetErrorString(pe));
     if (int e = check_launch("x_prep_kernel")) return e;
   }

@@ -6,8 +6,10 @@
 // M = B*(D+1) rows, row b*(D+1)+i holds the target's token for draft slot i of
 // sequence b:
 //   accept_len[b] = min{ i < D : drafts[b, i] != argmax[b*(D+1) + i] }, else D.
-// One CTA: a fixed-order reduction of the per-CTA (max, lowest index) partials
-// for every row, then one thread per sequence for the accept length.
+// One CTA per sequence b: it reduces the per-tile (max, lowest index) partials of its
+// D+1 rows, 16 rows at a time, each thread reading every row of a partial together
+// (they are contiguous), then computes that sequence's accept length. The (value,
+// lowest index) order is total, so the result does not depend on reduction order.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -16,45 +18,66 @@
 
 namespace nvfp4ws {
 
-__global__ void __launch_bounds__(256) verify_stage2_kernel(const float* __restrict__ pv,
-                                                            const int* __restrict__ pi, int nparts, int M,
-                                                            const int32_t* __restrict__ drafts, int B, int D,
-                                                            int32_t* __restrict__ argmax,
-                                                            int32_t* __restrict__ accept_len,
-                                                            float* __restrict__ max_logit) {
+constexpr int kS2Threads = 512;
+constexpr int kS2Rows = 16;
+
+__global__ void __launch_bounds__(kS2Threads) verify_stage2_kernel(const float* __restrict__ pv,
+                                                                   const int* __restrict__ pi, int nparts, int M,
+                                                                   const int32_t* __restrict__ drafts, int B, int D,
+                                                                   int32_t* __restrict__ argmax,
+                                                                   int32_t* __restrict__ accept_len,
+                                                                   float* __restrict__ max_logit) {
+  // Launched as a programmatic dependent of the GEMM that wrote the partials.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  __shared__ float s_v[kS2Threads / 32][kS2Rows];
+  __shared__ int s_i[kS2Threads / 32][kS2Rows];
   __shared__ int s_arg[NVFP4WS_MAX_M];
-  __shared__ float s_v[8];
-  __shared__ int s_i[8];
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  for (int m = 0; m < M; ++m) {
-    float bv = -INFINITY;
-    int bi = INT_MAX;
-    for (int p = t; p < nparts; p += blockDim.x) {
-      const float v = pv[(long long)p * M + m];
-      const int i = pi[(long long)p * M + m];
-      if (argmax_better(v, i, bv, bi)) { bv = v; bi = i; }
+  const int b = blockIdx.x, R = D + 1, row0 = b * R;
+  for (int r0 = 0; r0 < R; r0 += kS2Rows) {
+    const int nr = (R - r0) < kS2Rows ? (R - r0) : kS2Rows;
+    float bv[kS2Rows];
+    int bi[kS2Rows];
+#pragma unroll
+    for (int j = 0; j < kS2Rows; ++j) { bv[j] = -INFINITY; bi[j] = INT_MAX; }
+    for (int p = t; p < nparts; p += kS2Threads) {
+      const float* v = pv + (long long)p * M + row0 + r0;
+      const int* ix = pi + (long long)p * M + row0 + r0;
+#pragma unroll
+      for (int j = 0; j < kS2Rows; ++j) {
+        if (j < nr) {
+          const float vv = v[j];
+          const int ii = ix[j];
+          if (argmax_better(vv, ii, bv[j], bi[j])) { bv[j] = vv; bi[j] = ii; }
+        }
+      }
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float v = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int i = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (argmax_better(v, i, bv, bi)) { bv = v; bi = i; }
+    for (int j = 0; j < kS2Rows; ++j) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float v = __shfl_xor_sync(0xffffffffu, bv[j], o);
+        const int i = __shfl_xor_sync(0xffffffffu, bi[j], o);
+        if (argmax_better(v, i, bv[j], bi[j])) { bv[j] = v; bi[j] = i; }
+      }
+      if (lane == 0) { s_v[warp][j] = bv[j]; s_i[warp][j] = bi[j]; }
     }
-    if (lane == 0) { s_v[warp] = bv; s_i[warp] = bi; }
     __syncthreads();
-    if (t == 0) {
-      for (int w = 1; w < (int)(blockDim.x >> 5); ++w)
-        if (argmax_better(s_v[w], s_i[w], bv, bi)) { bv = s_v[w]; bi = s_i[w]; }
-      argmax[m] = bi;
-      s_arg[m] = bi;
-      if (max_logit) max_logit[m] = bv;
+    if (t < nr) {
+      float v = s_v[0][t];
+      int i = s_i[0][t];
+      for (int w = 1; w < kS2Threads / 32; ++w)
+        if (argmax_better(s_v[w][t], s_i[w][t], v, i)) { v = s_v[w][t]; i = s_i[w][t]; }
+      argmax[row0 + r0 + t] = i;
+      s_arg[r0 + t] = i;
+      if (max_logit) max_logit[row0 + r0 + t] = v;
     }
     __syncthreads();
   }
-  for (int b = t; b < B; b += blockDim.x) {
+  if (t == 0) {
     int L = D;
     for (int i = 0; i < D; ++i) {
-      if (drafts[(long long)b * D + i] != s_arg[b * (D + 1) + i]) { L = i; break; }
+      if (drafts[(long long)b * D + i] != s_arg[i]) { L = i; break; }
     }
     accept_len[b] = L;
   }
@@ -63,8 +86,18 @@ __global__ void __launch_bounds__(256) verify_stage2_kernel(const float* __restr
 int launch_verify_stage2(const float* part_val, const int* part_idx, int nparts, int M,
                          const int32_t* drafts, int B, int D, int32_t* argmax, int32_t* accept_len,
                          float* max_logit, cudaStream_t s) {
-  verify_stage2_kernel<<<1, 256, 0, s>>>(part_val, part_idx, nparts, M, drafts, B, D, argmax, accept_len,
-                                         max_logit);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)B);
+  cfg.blockDim = dim3(kS2Threads);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, verify_stage2_kernel, part_val, part_idx, nparts, M, drafts, B, D, argmax,
+                                     accept_len, max_logit);
+  if (e != cudaSuccess) return set_error(NVFP4WS_ERR_CUDA, "verify_stage2_kernel launch: %s", cudaGetErrorString(e));
   return check_launch("verify_stage2_kernel");
 }
 
