@@ -101,16 +101,18 @@ struct alignas(64) Problem {
   long long N;
   unsigned int unit0;      // first unit of this problem in the launch's unit numbering
   int K, kch, tiles, y_bf16, verify;
+  int groups;              // groups of tpu tiles: units are (group, K-chunk)
 };
 
 // What depends on M alone, shared by every problem of a launch.
 struct Geom {
   int M, T, nb, nbt, nb_tile, nsfb;
   int ku;                  // 256-wide K-chunks per unit (1 or 2)
+  int tpu;                 // 128-row weight tiles per unit (1 or 2); they share the unit's activation images
   uint32_t img_bytes;      // one chunk's image: nbt*nb_tile rows x (128 B codes + 16 B scales)
   uint32_t img_stride;     // images are 1024-byte aligned (the MMA operand's swizzle atom)
   uint32_t img_xs_off;     // offset of the scale rows in an image
-  uint32_t wbytes;         // weight bytes of a unit: ku x (codes + scales)
+  uint32_t wbytes;         // weight bytes of a unit: tpu x ku x (codes + scales)
 };
 
 struct PassParams {
@@ -126,11 +128,11 @@ struct PassParams {
   int nwave;
   unsigned int units;
   int grid, stages;
-  uint32_t stage_bytes;    // one stage: W codes (ku blocks), W scales, then ku activation images
+  uint32_t stage_bytes;    // one stage: W codes (tpu x ku blocks), W scales (tpu tiles), then ku activation images
   int acc_bufs, sf_bufs;
   uint32_t sf_cols, acc_col0, acc_stride;
   unsigned int* counters;  // [nwave][grid] split-tile tickets, zero on entry and on exit
-  float* partials;         // [nwave][2*grid][M][128] split-tile partial sums
+  float* partials;         // [nwave][2*grid][tpu][128 rows][Mp] split-tile partial sums, Mp = M rounded up to 4
   unsigned int* err;
 };
 
@@ -321,14 +323,14 @@ __device__ __forceinline__ uint32_t unit_begin(uint32_t c, uint32_t U, uint32_t 
 // The CTA owning unit u: the largest c with floor(c*U/G) <= u.
 __device__ __forceinline__ uint32_t cta_of_unit(uint32_t u, uint32_t U, uint32_t G) { return ((u + 1) * G - 1) / U; }
 
-// Position of a unit: problem, tile, K-chunk. Advances without divisions; a problem's
-// sizes are read once when the walk enters it.
+// Position of a unit: problem, tile group, K-chunk. Advances without divisions; a
+// problem's sizes are read once when the walk enters it.
 struct Cursor {
-  int pi, tile, kc, kch, tiles;
+  int pi, tile, kc, kch, tiles;   // tile: the tile group; tiles: groups in the problem
   __device__ __forceinline__ void init(const Problem* probs, int p0, uint32_t u) {
     pi = p0;
     kch = probs[pi].kch;
-    tiles = probs[pi].tiles;
+    tiles = probs[pi].groups;
     const uint32_t rel = u - probs[pi].unit0;
     tile = (int)(rel / (uint32_t)kch);
     kc = (int)(rel - (uint32_t)tile * (uint32_t)kch);
@@ -338,7 +340,7 @@ struct Cursor {
     kc = 0;
     if (++tile < tiles) return;
     tile = 0;
-    if (++pi < nprob) { kch = probs[pi].kch; tiles = probs[pi].tiles; }
+    if (++pi < nprob) { kch = probs[pi].kch; tiles = probs[pi].groups; }
   }
 };
 
@@ -368,9 +370,26 @@ struct Walk {
   }
   __device__ __forceinline__ bool first() const { return u == r0; }
   __device__ __forceinline__ bool last() const { return u + 1 == r1; }
+  // Units left in the current segment: to the end of the tile or of this wave's range.
+  __device__ __forceinline__ int seg_units() const {
+    const uint32_t to_tile = (uint32_t)(cu.kch - cu.kc), to_range = r1 - u;
+    return (int)(to_tile < to_range ? to_tile : to_range);
+  }
+  // Skip the n units that finish the current segment (n == seg_units()).
+  __device__ __forceinline__ void skip_segment(const PassParams& p, const Problem* probs, int c, int n) {
+    u += (uint32_t)n;
+    if (u == r1) {
+      if (w + 1 < p.nwave) start(p, probs, c, w + 1);
+      return;
+    }
+    cu.kc = 0;
+    if (++cu.tile < cu.tiles) return;
+    cu.tile = 0;
+    if (++cu.pi < p.nprob) { cu.kch = probs[cu.pi].kch; cu.tiles = probs[cu.pi].groups; }
+  }
 };
 
-template <int NBT, int KU>
+template <int NBT, int KU, int TPU>
 __global__ void __launch_bounds__(kThreads, 1)
     pass_kernel(const __grid_constant__ Problem single, const PassParams p) {
   // The next kernel of the stream may launch as soon as SMs free up: the library's prep
@@ -389,7 +408,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* s_last = reinterpret_cast<int*>(s_tmem + 2);
   float* s_val = reinterpret_cast<float*>(s_tmem + 4);                 // [4][72]
   int* s_idx = reinterpret_cast<int*>(s_val + 4 * 72);                 // [4][72]
-  float* s_g = reinterpret_cast<float*>(s_idx + 4 * 72);               // [kMaxB]
+  // g_0 of each token of the current problem, 16-byte aligned for float4 reads [80]
+  float* s_g0 = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(s_idx + 4 * 72) + 15) & ~uintptr_t(15));
 
   auto bar_full = [&](int s) { return smem_u32(bars + s); };
   auto bar_empty = [&](int s) { return smem_u32(bars + S + s); };
@@ -436,11 +456,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t st = sbase + (uint32_t)s * p.stage_bytes;
         const Problem* pr = probs + cu.pi;
         mbar_arrive_expect_tx(bar_full(s), tx);
-        for (int h = 0; h < g.ku; ++h)
-          tma_load_2d(st + (uint32_t)h * kNibBytes, &pr->tm_q, (cu.kc * g.ku + h) * (kKC / 2), cu.tile * kTileRows,
-                      bar_full(s), pol_w);
-        tma_load_2d(st + (uint32_t)g.ku * kNibBytes, &pr->tm_sf, cu.kc * g.ku * (kKC / 16), cu.tile * kTileRows,
-                    bar_full(s), pol_w);
+        for (int j = 0; j < g.tpu; ++j) {
+          const int row = (cu.tile * g.tpu + j) * kTileRows;   // rows past N read as zeros
+          for (int h = 0; h < g.ku; ++h)
+            tma_load_2d(st + (uint32_t)(j * g.ku + h) * kNibBytes, &pr->tm_q, (cu.kc * g.ku + h) * (kKC / 2), row,
+                        bar_full(s), pol_w);
+          tma_load_2d(st + (uint32_t)(g.tpu * g.ku) * kNibBytes + (uint32_t)j * (kTileRows * 16u * g.ku), &pr->tm_sf,
+                      cu.kc * g.ku * (kKC / 16), row, bar_full(s), pol_w);
+        }
       };
       auto load_x = [&](int s, const Cursor& cu) {
         bulk_load(sbase + (uint32_t)s * p.stage_bytes + g.wbytes, probs[cu.pi].ximg + (size_t)cu.kc * xbytes, xbytes,
@@ -492,29 +515,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t adesc_base = sw128_desc(sbase), bdesc_base = sw128_desc(sbase + g.wbytes);
       const uint64_t step = (uint64_t)(p.stage_bytes >> 4);
       uint64_t adesc = adesc_base, bdesc = bdesc_base;
-      // K-step kk of chunk h: A at block h, B in image h, scales in columns laid out as the
-      // scale warps store them (W: 4 per K-step; X: nsfb per K-step and B tile).
-      uint32_t boff[KU][NBT], doff[NBT], sfboff[KU][4][NBT];
+      // K-step kk of chunk h: A (tile j) at block j*KU + h, B in image h, scales in columns
+      // laid out as the scale warps store them (W: 4 per K-step and tile, tile-major; then X:
+      // nsfb per K-step and B tile). Tile j accumulates at column j*NBT*nb_tile.
+      uint32_t boff[KU][NBT], doff[TPU][NBT], sfboff[KU][4][NBT];
 #pragma unroll
       for (int bt = 0; bt < NBT; ++bt) {
-        doff[bt] = (uint32_t)(bt * g.nb_tile);
+#pragma unroll
+        for (int j = 0; j < TPU; ++j) doff[j][bt] = (uint32_t)((j * NBT + bt) * g.nb_tile);
 #pragma unroll
         for (int h = 0; h < KU; ++h) {
           boff[h][bt] = (h * g.img_stride >> 4) + (uint32_t)(bt * g.nb_tile * 8);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            sfboff[h][kk][bt] = 16u * KU + (uint32_t)(((h * 4 + kk) * NBT + bt) * g.nsfb);
+            sfboff[h][kk][bt] = 16u * KU * TPU + (uint32_t)(((h * 4 + kk) * NBT + bt) * g.nsfb);
         }
       }
       int fb = 0;                                     // scale-factor buffer of unit i
       uint32_t fph = 0;
       const uint32_t acc0 = tmem + p.acc_col0, acc1 = tmem + p.acc_col0 + p.acc_stride;
+      // Segment bookkeeping is a countdown: the walk is consulted once per segment.
+      int seg_len = 0, seg_left = 0;
+      const bool two_acc = p.acc_bufs == 2;
       for (int i = 0; i < nunits && ok; ++i) {
-        const bool seg_first = wk.first() || (wk.cu.kc == 0);
-        const bool seg_last = wk.last() || (wk.cu.kc == wk.cu.kch - 1);
-        const int ab = (p.acc_bufs == 2) ? (seg & 1) : 0;
+        const bool seg_first = seg_left == 0;
+        const int ab = two_acc ? (seg & 1) : 0;
         if (seg_first) {
-          const uint32_t acc_use = (p.acc_bufs == 2) ? (uint32_t)(seg >> 1) : (uint32_t)seg;
+          seg_len = seg_left = wk.seg_units();
+          const uint32_t acc_use = two_acc ? (uint32_t)(seg >> 1) : (uint32_t)seg;
           ok = mbar_wait(bar_accempty(ab), (acc_use & 1u) ^ 1u, s_abort, p.err);
           if (!ok) break;
         }
@@ -531,16 +559,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
 #pragma unroll
-            for (int bt = 0; bt < NBT; ++bt)
-              tc_mma_mxf4(d0 + doff[bt], adesc + (uint64_t)(h * (kNibBytes >> 4) + kk * 2),
-                          bdesc + (uint64_t)(boff[h][bt] + kk * 2), idesc, sf + (uint32_t)((h * 4 + kk) * 4),
-                          sf + sfboff[h][kk][bt], (h == 0 && kk == 0) ? first : 1u);
+            for (int j = 0; j < TPU; ++j) {
+#pragma unroll
+              for (int bt = 0; bt < NBT; ++bt)
+                tc_mma_mxf4(d0 + doff[j][bt], adesc + (uint64_t)((j * KU + h) * (kNibBytes >> 4) + kk * 2),
+                            bdesc + (uint64_t)(boff[h][bt] + kk * 2), idesc,
+                            sf + (uint32_t)((j * 4 * KU + h * 4 + kk) * 4), sf + sfboff[h][kk][bt],
+                            (h == 0 && kk == 0) ? first : 1u);
+            }
           }
         }
         MX_TRACE(3, i);
         tc_commit(bar_empty(s));                      // stage s and scale buffer fb are free once these retire
-        if (seg_last) { tc_commit(bar_accfull(ab)); ++seg; }
-        wk.next(p, probs, c);
+        if (--seg_left == 0) {
+          tc_commit(bar_accfull(ab));
+          ++seg;
+          wk.skip_segment(p, probs, c, seg_len);
+        }
         if (++fb == p.sf_bufs) { fb = 0; fph ^= 1u; }
         if (++s == S) { s = 0; adesc = adesc_base; bdesc = bdesc_base; }
         else { adesc += step; bdesc += step; }
@@ -560,8 +595,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int s2 = S - NF;                        // ring position of unit i - NF (valid once i >= NF)
     uint32_t ph2 = 1u;
     int fb = 0;
-    const uint32_t wsf_off = (uint32_t)g.ku * kNibBytes;       // W scales: row m has 16*ku bytes
-    const uint32_t wsf_row = 16u * (uint32_t)g.ku;
+    const uint32_t wsf_row = 16u * (uint32_t)g.ku;                          // W scales: row m has 16*ku bytes
+    const uint32_t wsf_off = (uint32_t)(g.tpu * g.ku) * kNibBytes;          // tile j's scales at + j*128*wsf_row
+    const uint32_t xsf_col = 16u * (uint32_t)(g.ku * g.tpu);                // X scale columns follow the W ones
     for (int i = 0; i < nunits; ++i) {
       if (!mbar_wait(bar_full(s), ph, s_abort, p.err)) break;
       if (lane == 0 && warp == 4) MX_TRACE(5, i);
@@ -571,16 +607,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t st = sbase + (uint32_t)s * p.stage_bytes;
       const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)fb * p.sf_cols;
       for (int h = 0; h < g.ku; ++h) {
-        {   // W scales: column 4*(4h+kk) + j of lane m0 = the 4 block scales (K-step kk of chunk h) of row m0 + 32*j
+        // W scales of tile t: column 16*(t*ku + h) + 4*kk + j of lane m0 = the 4 block scales
+        // (K-step kk of chunk h) of row m0 + 32*j
+        for (int t = 0; t < g.tpu; ++t) {
+          const uint32_t wsf = st + wsf_off + (uint32_t)t * (kTileRows * wsf_row);
           uint4 R[4];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) R[j] = lds128(st + wsf_off + (uint32_t)(m0 + 32 * j) * wsf_row + (uint32_t)h * 16u);
+          for (int j = 0; j < 4; ++j) R[j] = lds128(wsf + (uint32_t)(m0 + 32 * j) * wsf_row + (uint32_t)h * 16u);
           uint32_t out[16];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             out[0 + j] = R[j].x; out[4 + j] = R[j].y; out[8 + j] = R[j].z; out[12 + j] = R[j].w;
           }
-          tc_st_x16(lane_base + (uint32_t)h * 16u, out);
+          tc_st_x16(lane_base + (uint32_t)(t * g.ku + h) * 16u, out);
         }
         const uint32_t xs = st + g.wbytes + (uint32_t)h * g.img_stride + g.img_xs_off;
         if (g.nbt == 1 && g.nsfb == 4) {
@@ -595,7 +634,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < 4; ++j) {
             out[0 + j] = R[j].x; out[4 + j] = R[j].y; out[8 + j] = R[j].z; out[12 + j] = R[j].w;
           }
-          tc_st_x16(lane_base + 16u * (uint32_t)g.ku + (uint32_t)h * 16u, out);
+          tc_st_x16(lane_base + xsf_col + (uint32_t)h * 16u, out);
           continue;
         }
         for (int bt = 0; bt < g.nbt; ++bt) {   // X-term scales, per B tile: nsfb columns per K-step
@@ -610,7 +649,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t out[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) out[j] = kk == 0 ? R[j].x : kk == 1 ? R[j].y : kk == 2 ? R[j].z : R[j].w;
-            const uint32_t col = 16u * (uint32_t)g.ku + (uint32_t)(((h * 4 + kk) * g.nbt + bt) * g.nsfb);
+            const uint32_t col = xsf_col + (uint32_t)(((h * 4 + kk) * g.nbt + bt) * g.nsfb);
             if (g.nsfb == 8) tc_st_x8(lane_base + col, out);
             else tc_st_x4(lane_base + col, out[0], out[1], out[2], out[3]);
           }
@@ -635,106 +674,144 @@ __global__ void __launch_bounds__(kThreads, 1)
     int seg = 0;
     Walk wk;
     wk.start(p, probs, c, 0);
-    for (int i = 0; i < nunits; ++i) {
-      const uint32_t u = wk.u, r0 = wk.r0, w0 = wk.w0, Uw = wk.Uw;
+    for (int done = 0; done < nunits;) {   // one iteration per segment
+      const int n_seg = wk.seg_units();
+      const uint32_t u = wk.u + (uint32_t)(n_seg - 1), r0 = wk.r0, w0 = wk.w0, Uw = wk.Uw;   // u: the segment's last unit
       const int wave = wk.w;
-      const bool seg_last = wk.last() || (wk.cu.kc == wk.cu.kch - 1);
-      const int pi = wk.cu.pi, cur_tile = wk.cu.tile, kch = wk.cu.kch;
-      wk.next(p, probs, c);
-      if (!seg_last) continue;
+      const int pi = wk.cu.pi, group = wk.cu.tile, kch = wk.cu.kch;
+      wk.skip_segment(p, probs, c, n_seg);
+      done += n_seg;
       const Problem* pr = probs + pi;
-      const uint32_t tile_u0 = pr->unit0 + (uint32_t)cur_tile * (uint32_t)kch, tile_u1 = tile_u0 + (uint32_t)kch;
+      const uint32_t tile_u0 = pr->unit0 + (uint32_t)group * (uint32_t)kch, tile_u1 = tile_u0 + (uint32_t)kch;
       const uint32_t seg_u0 = r0 > tile_u0 ? r0 : tile_u0;
       const bool complete = (seg_u0 == tile_u0) && (u + 1 == tile_u1);
       if (pi != gprob) {
         named_bar(1, 128);
-        for (int j = et; j < g.nb; j += 128) s_g[j] = pr->xg[j];
+        for (int j = et; j < M; j += 128) s_g0[j] = pr->xg[j * kMxf4Terms];
         named_bar(1, 128);
         gprob = pi;
       }
       const float ts = *pr->ts;
       const long long N = pr->N;
-      const int verify = pr->verify, y_bf16 = pr->y_bf16;
+      const int verify = pr->verify, y_bf16 = pr->y_bf16, tiles = pr->tiles;
       float* Yf = static_cast<float*>(pr->Y);
       const int ab = (p.acc_bufs == 2) ? (seg & 1) : 0;
       const uint32_t acc_use = (p.acc_bufs == 2) ? (uint32_t)(seg >> 1) : (uint32_t)seg;
       if (!mbar_wait(bar_accfull(ab), acc_use & 1u, s_abort, p.err)) break;
       if (et == 0 && seg < 2) MX_CTA(8 + 4 * seg);
       tc_fence_after();
-      const long long n = (long long)cur_tile * kTileRows + rowl;
-      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + p.acc_col0 + (uint32_t)ab * p.acc_stride;
-      float* wave_part = p.partials + (long long)wave * 2 * G * M * kTileRows;
+      const uint32_t taddr0 = tmem + ((uint32_t)(q * 32) << 16) + p.acc_col0 + (uint32_t)ab * p.acc_stride;
+      const int Mp = (M + 3) & ~3;
+      float* wave_part = p.partials + (long long)wave * 2 * G * g.tpu * kTileRows * Mp;
       const int slot = (seg_u0 == r0) ? 2 * c : 2 * c + 1;
-      float* dst = wave_part + ((long long)slot * M) * kTileRows;
-      auto emit = [&](int m, float y) {   // a finished output: Y, or this row's argmax candidate
+      // Finished outputs of row n for tokens mc .. mc+15 (y[j], already x ts).
+      // Verify problem: each token's argmax candidate of the 4 warps' rows. Otherwise Y,
+      // one token per warp-wide 128-byte store (measured: a 4x4 shuffle transpose into
+      // 16-byte stores was slower here, Y rows being N floats apart).
+      auto emit16 = [&](long long n, int mc, const float (&y)[16]) {
         if (verify) {
-          float bv = (n < N) ? y : -INFINITY;
-          int bi = (n < N) ? (int)n : INT_MAX;
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (argmax_better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+          for (int j = 0; j < 16; ++j) {
+            const int m = mc + j;
+            if (m >= M) break;
+            float bv = (n < N) ? y[j] : -INFINITY;
+            int bi = (n < N) ? (int)n : INT_MAX;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+              const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+              const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+              if (argmax_better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+            }
+            if (lane == 0) { s_val[q * 72 + m] = bv; s_idx[q * 72 + m] = bi; }
           }
-          if (lane == 0) { s_val[q * 72 + m] = bv; s_idx[q * 72 + m] = bi; }
-        } else if (n < N) {
-          if (y_bf16) reinterpret_cast<uint16_t*>(Yf)[(long long)m * N + n] = f32_to_bf16_rn(y);
-          else Yf[(long long)m * N + n] = y;
+          return;
+        }
+        if (n < N) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int m = mc + j;
+            if (m >= M) break;
+            if (y_bf16) reinterpret_cast<uint16_t*>(Yf)[(long long)m * N + n] = f32_to_bf16_rn(y[j]);
+            else Yf[(long long)m * N + n] = y[j];
+          }
         }
       };
-      auto tile_argmax = [&]() {          // combine the 4 warps' candidates of each row
+      auto tile_argmax = [&](int tile) {  // combine the 4 warps' candidates of each row
         named_bar(1, 128);
         if (et < M) {
           float bv = s_val[et];
           int bi = s_idx[et];
           for (int w = 1; w < 4; ++w)
             if (argmax_better(s_val[w * 72 + et], s_idx[w * 72 + et], bv, bi)) { bv = s_val[w * 72 + et]; bi = s_idx[w * 72 + et]; }
-          pr->part_val[(long long)cur_tile * M + et] = bv;
-          pr->part_idx[(long long)cur_tile * M + et] = bi;
+          pr->part_val[(long long)tile * M + et] = bv;
+          pr->part_idx[(long long)tile * M + et] = bi;
         }
         named_bar(1, 128);
       };
-      // Fold the T terms of each token: y[m] = sum_t g[m,t] * acc[m*T + t]. Accumulator
-      // column j holds B row j, so token m's terms are columns m*T .. m*T+T-1. Tokens are
-      // taken 16 at a time: up to 5 TMEM loads of 16 columns are issued back to back and
-      // waited for once, and the fold uses the compile-time term count.
+      // Fold the T terms of each token: y[m] = sum_t g_t acc[m*T + t] with g_t = g_0 / 4^t,
+      // i.e. g_0 * (acc_0 + (acc_1 + (acc_2 + (acc_3 + acc_4/4)/4)/4)/4) (the multiplications
+      // by 1/4 are exact; the prep kernel's g_t are the same sequence unless it underflows).
+      // Accumulator column j holds B row j, so token m's terms are columns m*T .. m*T+T-1.
+      // Tokens are taken 16 at a time: up to 5 TMEM loads of 16 columns are issued back to
+      // back and waited for once, and the 16 g_0 arrive as four 16-byte shared loads.
+      // Measured: with one epilogue warp per sub-partition the fold is latency-bound, and
+      // a per-term scale load ahead of every FMA made it 4x slower.
       static_assert(kMxf4Terms == 5, "the fold below is written for 5 terms");
       const int nb16 = (g.nb + 15) & ~15;                 // columns that exist in the accumulator
-      for (int mc = 0; mc < M; mc += 16) {
-        const int col0 = mc * kMxf4Terms;                 // multiple of 80
-        const int nld = (nb16 - col0) / 16 < 5 ? (nb16 - col0) / 16 : 5;
-        uint32_t v[80];
-        tc_ld_x16(taddr + (uint32_t)col0, v);
-        if (nld > 1) tc_ld_x16(taddr + (uint32_t)(col0 + 16), v + 16);
-        if (nld > 2) tc_ld_x16(taddr + (uint32_t)(col0 + 32), v + 32);
-        if (nld > 3) tc_ld_x16(taddr + (uint32_t)(col0 + 48), v + 48);
-        if (nld > 4) tc_ld_x16(taddr + (uint32_t)(col0 + 64), v + 64);
-        tc_wait_ld();
+      for (int tj = 0; tj < g.tpu; ++tj) {
+        const int tile = group * g.tpu + tj;
+        const long long n = (long long)tile * kTileRows + rowl;
+        const uint32_t taddr = taddr0 + (uint32_t)(tj * g.nbt * g.nb_tile);
+        float* dst = wave_part + ((long long)(slot * g.tpu + tj) * kTileRows + rowl) * Mp;   // this row's partials
+        for (int mc = 0; mc < M; mc += 16) {
+          const int col0 = mc * kMxf4Terms;                 // multiple of 80
+          const int nld = (nb16 - col0) / 16 < 5 ? (nb16 - col0) / 16 : 5;
+          uint32_t v[80];
+          tc_ld_x16(taddr + (uint32_t)col0, v);
+          if (nld > 1) tc_ld_x16(taddr + (uint32_t)(col0 + 16), v + 16);
+          if (nld > 2) tc_ld_x16(taddr + (uint32_t)(col0 + 32), v + 32);
+          if (nld > 3) tc_ld_x16(taddr + (uint32_t)(col0 + 48), v + 48);
+          if (nld > 4) tc_ld_x16(taddr + (uint32_t)(col0 + 64), v + 64);
+          float g0[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int m = mc + j;
-          if (m >= M) break;
-          float ym = 0.f;
+          for (int k = 0; k < 4; ++k) {
+            const float4 t4 = reinterpret_cast<const float4*>(s_g0 + mc)[k];
+            g0[4 * k] = t4.x; g0[4 * k + 1] = t4.y; g0[4 * k + 2] = t4.z; g0[4 * k + 3] = t4.w;
+          }
+          tc_wait_ld();
+          float yv[16];
 #pragma unroll
-          for (int t = 0; t < kMxf4Terms; ++t)
-            ym = fmaf(s_g[m * kMxf4Terms + t], __uint_as_float(v[j * kMxf4Terms + t]), ym);
-          if (complete) emit(m, ym * ts);
-          else dst[(long long)m * kTileRows + rowl] = ym;
+          for (int j = 0; j < 16; ++j) {
+            float a = __uint_as_float(v[j * kMxf4Terms + 4]);
+            a = fmaf(a, 0.25f, __uint_as_float(v[j * kMxf4Terms + 3]));
+            a = fmaf(a, 0.25f, __uint_as_float(v[j * kMxf4Terms + 2]));
+            a = fmaf(a, 0.25f, __uint_as_float(v[j * kMxf4Terms + 1]));
+            a = fmaf(a, 0.25f, __uint_as_float(v[j * kMxf4Terms + 0]));
+            yv[j] = (mc + j < M) ? a * g0[j] : 0.f;   // columns past the tokens are never loaded
+          }
+          if (complete) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) yv[j] *= ts;
+            emit16(n, mc, yv);
+          } else {
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+              if (mc + 4 * b < Mp)
+                *reinterpret_cast<float4*>(dst + mc + 4 * b) = make_float4(yv[4 * b], yv[4 * b + 1], yv[4 * b + 2], yv[4 * b + 3]);
+          }
         }
+        if (complete && verify && tile < tiles) tile_argmax(tile);
       }
       tc_fence_before();
       if (et == 0 && seg < 2) MX_CTA(9 + 4 * seg);
       mbar_arrive(bar_accempty(ab));
       ++seg;
-      if (complete) {
-        if (verify) tile_argmax();
-        continue;
-      }
-      // Split tile: count this CTA's arrival. The barrier orders every epilogue thread's
-      // partial stores before thread 0's release; the acquire side of the same atomic
-      // orders the last arriver's loads of the other contributors' partials after it.
-      // The ticket of a split tile is indexed by its first contributing CTA, which has
-      // at most one split tile starting in its range.
+      if (complete) continue;
+      // Split tile group: count this CTA's arrival. The barrier orders every epilogue
+      // thread's partial stores before thread 0's release; the acquire side of the same
+      // atomic orders the last arriver's loads of the other contributors' partials after
+      // it. The ticket of a split group is indexed by its first contributing CTA, which
+      // has at most one split group starting in its range.
       const int c0 = (int)cta_of_unit(tile_u0 - w0, Uw, G), c1 = (int)cta_of_unit(tile_u1 - 1u - w0, Uw, G);
       unsigned int* ticket = p.counters + (long long)wave * G + c0;
       named_bar(1, 128);
@@ -748,35 +825,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (*s_last) {
         // Sum the contributors' partials in CTA order (deterministic), two contributors'
         // loads in flight at a time, 16 tokens per pass.
-        for (int mc = 0; mc < M; mc += 16) {
-          float acc[16];
+        for (int tj = 0; tj < g.tpu; ++tj) {
+          const int tile = group * g.tpu + tj;
+          const long long n = (long long)tile * kTileRows + rowl;
+          for (int mc = 0; mc < M; mc += 16) {
+            float acc[16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) acc[j] = 0.f;
-          for (int cc = c0; cc <= c1; cc += 2) {
-            const bool two = cc + 1 <= c1;
-            const int sl0 = (w0 + unit_begin((uint32_t)cc, Uw, G) >= tile_u0) ? 2 * cc : 2 * cc + 1;
-            const int sl1 = two ? ((w0 + unit_begin((uint32_t)cc + 1u, Uw, G) >= tile_u0) ? 2 * cc + 2 : 2 * cc + 3) : sl0;
-            const float* src0 = wave_part + ((long long)sl0 * M + mc) * kTileRows + rowl;
-            const float* src1 = wave_part + ((long long)sl1 * M + mc) * kTileRows + rowl;
-            float v0[16], v1[16];
+            for (int j = 0; j < 16; ++j) acc[j] = 0.f;
+            for (int cc = c0; cc <= c1; cc += 2) {
+              const bool two = cc + 1 <= c1;
+              const int sl0 = (w0 + unit_begin((uint32_t)cc, Uw, G) >= tile_u0) ? 2 * cc : 2 * cc + 1;
+              const int sl1 = two ? ((w0 + unit_begin((uint32_t)cc + 1u, Uw, G) >= tile_u0) ? 2 * cc + 2 : 2 * cc + 3) : sl0;
+              const float4* src0 =
+                  reinterpret_cast<const float4*>(wave_part + ((long long)(sl0 * g.tpu + tj) * kTileRows + rowl) * Mp + mc);
+              const float4* src1 =
+                  reinterpret_cast<const float4*>(wave_part + ((long long)(sl1 * g.tpu + tj) * kTileRows + rowl) * Mp + mc);
+              float4 v0[4], v1[4];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              v0[j] = (mc + j < M) ? __ldcg(src0 + j * kTileRows) : 0.f;
-              v1[j] = (two && mc + j < M) ? __ldcg(src1 + j * kTileRows) : 0.f;
+              for (int b = 0; b < 4; ++b) {
+                v0[b] = (mc + 4 * b < Mp) ? __ldcg(src0 + b) : make_float4(0.f, 0.f, 0.f, 0.f);
+                v1[b] = (two && mc + 4 * b < Mp) ? __ldcg(src1 + b) : make_float4(0.f, 0.f, 0.f, 0.f);
+              }
+#pragma unroll
+              for (int b = 0; b < 4; ++b) {
+                acc[4 * b] += v0[b].x; acc[4 * b + 1] += v0[b].y; acc[4 * b + 2] += v0[b].z; acc[4 * b + 3] += v0[b].w;
+                if (two) {
+                  acc[4 * b] += v1[b].x; acc[4 * b + 1] += v1[b].y; acc[4 * b + 2] += v1[b].z; acc[4 * b + 3] += v1[b].w;
+                }
+              }
             }
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              acc[j] += v0[j];
-              if (two) acc[j] += v1[j];
-            }
+            for (int j = 0; j < 16; ++j) acc[j] = (mc + j < M) ? acc[j] * ts : 0.f;
+            emit16(n, mc, acc);
           }
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            if (mc + j >= M) break;
-            emit(mc + j, acc[j] * ts);
-          }
+          if (verify && tile < tiles) tile_argmax(tile);
         }
-        if (verify) tile_argmax();
         if (et == 0) *ticket = 0u;           // ready for the next launch
       }
       named_bar(1, 128);
@@ -836,7 +919,7 @@ struct MxPlan {
   size_t smem;
 };
 
-static MxPlan mx_plan_ku(long long M, int ku) {
+static MxPlan mx_plan_ku(long long M, int ku, int tpu) {
   MxPlan pl{};
   Geom& g = pl.g;
   g.M = (int)M;
@@ -846,12 +929,13 @@ static MxPlan mx_plan_ku(long long M, int ku) {
   g.nb_tile = ((g.nb + g.nbt - 1) / g.nbt + 15) / 16 * 16;   // MMA N; a multiple of 16 keeps x16 loads inside the tile
   g.nsfb = g.nb_tile <= 128 ? 4 : 8;
   g.ku = ku;
+  g.tpu = tpu;
   g.img_xs_off = (uint32_t)(g.nbt * g.nb_tile) * 128u;
   g.img_bytes = (uint32_t)(g.nbt * g.nb_tile) * 144u;
   g.img_stride = (g.img_bytes + 1023) / 1024 * 1024;
-  g.wbytes = (uint32_t)ku * kWChunk;
-  pl.sf_cols = 16u * (uint32_t)ku + 4u * (uint32_t)(ku * g.nbt * g.nsfb);
-  pl.acc_stride = (uint32_t)(g.nbt * g.nb_tile);
+  g.wbytes = (uint32_t)(tpu * ku) * kWChunk;
+  pl.sf_cols = 16u * (uint32_t)(ku * tpu) + 4u * (uint32_t)(ku * g.nbt * g.nsfb);
+  pl.acc_stride = (uint32_t)(tpu * g.nbt * g.nb_tile);
   pl.acc_bufs = (2 * pl.sf_cols + 2 * pl.acc_stride <= 512) ? 2 : 1;
   // One ring: a stage holds a unit's weight tile, its scales and its activation images.
   // Measured: under a saturated weight stream the L2-resident images arrive with about the
@@ -868,15 +952,27 @@ static MxPlan mx_plan_ku(long long M, int ku) {
   return pl;
 }
 
-// Two-chunk units halve the issuing thread's per-unit work (its waits, commit and loop
-// bookkeeping are per unit, the MMAs per K-step). They are used when every K allows it,
-// the activations fit one B tile and the accumulator stays double-buffered.
+// Units of two K-chunks or two weight tiles halve the issuing thread's per-unit work (its
+// waits, commit and loop bookkeeping are per unit, the MMAs per K-step and tile). Measured
+// on the 27B pass: two chunks of one tile stream best while the ring keeps >= 4 stages
+// (M <= 12); past that, two tiles sharing one chunk's activation images carry half the
+// image bytes per weight byte, so more weight bytes fit in flight (M=17: 4 stages instead
+// of 3). Either needs one B tile and a double-buffered accumulator.
 static MxPlan mx_plan(long long M, bool k512) {
+  auto ok = [](const MxPlan& x, int min_stages) {
+    return x.g.nbt == 1 && x.acc_bufs == 2 && x.stages >= min_stages;
+  };
   if (k512) {
-    const MxPlan two = mx_plan_ku(M, 2);
-    if (two.g.nbt == 1 && two.acc_bufs == 2 && two.stages >= 3) return two;
+    const MxPlan two = mx_plan_ku(M, 2, 1);
+    if (ok(two, 4)) return two;
   }
-  return mx_plan_ku(M, 1);
+  const MxPlan pair = mx_plan_ku(M, 1, 2);
+  if (ok(pair, 3)) return pair;
+  if (k512) {
+    const MxPlan two = mx_plan_ku(M, 2, 1);
+    if (ok(two, 3)) return two;
+  }
+  return mx_plan_ku(M, 1, 1);
 }
 
 bool mxf4_supported(long long M, long long K) {
@@ -898,8 +994,13 @@ struct WsLayout {
   std::vector<size_t> off_img, off_xg, off_pv, off_pi;
 };
 
-static unsigned long long problem_units(const MxHostProblem& h, int ku) {
-  return (unsigned long long)((h.N + kTileRows - 1) / kTileRows) * (unsigned long long)(h.K / (kKC * ku));
+static long long problem_groups(const MxHostProblem& h, int tpu) {
+  const long long tiles = (h.N + kTileRows - 1) / kTileRows;
+  return (tiles + tpu - 1) / tpu;
+}
+
+static unsigned long long problem_units(const MxHostProblem& h, int ku, int tpu) {
+  return (unsigned long long)problem_groups(h, tpu) * (unsigned long long)(h.K / (kKC * ku));
 }
 
 static bool all_k512(const MxHostProblem* hp, int n) {
@@ -911,10 +1012,10 @@ static bool all_k512(const MxHostProblem* hp, int n) {
 // with_desc: a pass keeps its descriptors and wave tables in the workspace.
 static WsLayout mx_layout(const MxHostProblem* hp, int n, long long M, bool with_desc) {
   const MxPlan pl = mx_plan(M, all_k512(hp, n));
-  const int ku = pl.g.ku;
+  const int ku = pl.g.ku, tpu = pl.g.tpu;
   WsLayout L;
   L.units = 0;
-  for (int i = 0; i < n; ++i) L.units += problem_units(hp[i], ku);
+  for (int i = 0; i < n; ++i) L.units += problem_units(hp[i], ku, tpu);
   const int sms = std::max(1, device_sm_count());
   L.grid = (int)std::max<unsigned long long>(1ull, std::min<unsigned long long>((unsigned long long)sms, L.units));
   // waves: greedy over the list; a wave closes when the next problem's images would pass
@@ -930,14 +1031,14 @@ static WsLayout mx_layout(const MxHostProblem* hp, int n, long long M, bool with
       wu = 0;
     }
     img += pimg;
-    wu += problem_units(hp[i], ku);
+    wu += problem_units(hp[i], ku, tpu);
   }
   if (L.wave_first.size() > 1 && wu < (unsigned long long)L.grid) L.wave_first.pop_back();   // merge a short tail
   L.wave_first.push_back(n);
   L.nwave = (int)L.wave_first.size() - 1;
   size_t o = al256((size_t)L.nwave * L.grid * 4);
   L.off_part = o;
-  o += al256((size_t)L.nwave * 2 * L.grid * M * kTileRows * 4);
+  o += al256((size_t)L.nwave * 2 * L.grid * tpu * kTileRows * (size_t)((M + 3) & ~3LL) * 4);
   L.off_desc = L.off_wave = L.off_cta = L.off_cunits = 0;
   if (with_desc) {
     L.off_desc = o; o += al256(sizeof(Problem) * (size_t)n);
@@ -962,7 +1063,7 @@ static WsLayout mx_layout(const MxHostProblem* hp, int n, long long M, bool with
 }
 
 static int fill_problem(Problem* P, const MxHostProblem& h, const WsLayout& L, int i, unsigned long long unit0,
-                        char* ws, int ku) {
+                        char* ws, int ku, int tpu) {
   std::memset(static_cast<void*>(P), 0, sizeof(Problem));
   if (!map_u8(&P->tm_q, h.q, h.K / 2, h.N, kKC / 2, kTileRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !map_u8(&P->tm_sf, h.sf, h.K / 16, h.N, (uint32_t)(ku * kKC / 16), kTileRows, CU_TENSOR_MAP_SWIZZLE_NONE))
@@ -978,6 +1079,7 @@ static int fill_problem(Problem* P, const MxHostProblem& h, const WsLayout& L, i
   P->unit0 = (unsigned int)unit0;
   P->K = (int)h.K;
   P->kch = (int)(h.K / (kKC * ku));
+  P->groups = (int)problem_groups(h, tpu);
   P->tiles = (int)((h.N + kTileRows - 1) / kTileRows);
   P->y_bf16 = h.y_bf16;
   P->verify = h.verify;
@@ -990,9 +1092,10 @@ static int ensure_attrs() {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
     return set_error(NVFP4WS_ERR_CUDA, "cannot get the current device");
   if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(pass_kernel<1, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess ||
-        cudaFuncSetAttribute(pass_kernel<1, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess ||
-        cudaFuncSetAttribute(pass_kernel<2, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
+    if (cudaFuncSetAttribute(pass_kernel<1, 1, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess ||
+        cudaFuncSetAttribute(pass_kernel<1, 2, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess ||
+        cudaFuncSetAttribute(pass_kernel<1, 1, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess ||
+        cudaFuncSetAttribute(pass_kernel<2, 1, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
       return check_launch("cudaFuncSetAttribute(pass_kernel)");
     attr_set[dev] = true;
   }
@@ -1064,9 +1167,10 @@ static int launch_pass(const Problem& single, const Problem* probs_dev, const Pa
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = (pl.g.nbt == 2)  ? cudaLaunchKernelEx(&cfg, pass_kernel<2, 1>, single, p)
-                  : (pl.g.ku == 2) ? cudaLaunchKernelEx(&cfg, pass_kernel<1, 2>, single, p)
-                                   : cudaLaunchKernelEx(&cfg, pass_kernel<1, 1>, single, p);
+  cudaError_t e = (pl.g.nbt == 2)   ? cudaLaunchKernelEx(&cfg, pass_kernel<2, 1, 1>, single, p)
+                  : (pl.g.tpu == 2) ? cudaLaunchKernelEx(&cfg, pass_kernel<1, 1, 2>, single, p)
+                  : (pl.g.ku == 2)  ? cudaLaunchKernelEx(&cfg, pass_kernel<1, 2, 1>, single, p)
+                                    : cudaLaunchKernelEx(&cfg, pass_kernel<1, 1, 1>, single, p);
   if (e != cudaSuccess) return set_error(NVFP4WS_ERR_CUDA, "pass_kernel launch: %s", cudaGetErrorString(e));
   return check_launch("pass_kernel");
 }
@@ -1081,7 +1185,7 @@ static int launch_single(const MxHostProblem& h, long long M, void* workspace, c
   const MxPlan pl = mx_plan(M, all_k512(&h, 1));
   const WsLayout L = mx_layout(&h, 1, M, false);
   char* ws = static_cast<char*>(workspace);
-  if (int e = fill_problem(out, h, L, 0, 0, ws, pl.g.ku)) return e;
+  if (int e = fill_problem(out, h, L, 0, 0, ws, pl.g.ku, pl.g.tpu)) return e;
   const PassTables none{nullptr, nullptr, nullptr, 1};
   return launch_pass(*out, nullptr, none, 1, pl, L.grid, L.units, L.off_part, h.K, ws, s);
 }
@@ -1130,7 +1234,8 @@ int mxf4_pass_init(void* state, const MxHostProblem* hp, int n, long long M, con
   MxPassState* P = static_cast<MxPassState*>(state);
   std::memset(static_cast<void*>(P), 0, sizeof(MxPassState));
   const WsLayout L = mx_layout(hp, n, M, true);
-  const int ku = mx_plan(M, all_k512(hp, n)).g.ku;
+  const MxPlan plan = mx_plan(M, all_k512(hp, n));
+  const int ku = plan.g.ku, tpu = plan.g.tpu;
   if (workspace_bytes < L.total)
     return set_error(NVFP4WS_ERR_WORKSPACE, "nvfp4_pass_init: workspace %zu bytes < required %zu", workspace_bytes,
                      L.total);
@@ -1141,8 +1246,8 @@ int mxf4_pass_init(void* state, const MxHostProblem* hp, int n, long long M, con
   long long max_k = 0;
   for (int i = 0; i < n; ++i) {
     first[i] = unit0;
-    if (int e = fill_problem(&host[i], hp[i], L, i, unit0, ws, ku)) return e;
-    unit0 += (unsigned long long)host[i].tiles * (unsigned long long)host[i].kch;
+    if (int e = fill_problem(&host[i], hp[i], L, i, unit0, ws, ku, tpu)) return e;
+    unit0 += (unsigned long long)host[i].groups * (unsigned long long)host[i].kch;
     max_k = std::max(max_k, hp[i].K);
   }
   // wave tables: wave starts, each CTA's first problem in each wave, each CTA's unit count
