@@ -448,7 +448,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      const uint64_t pol_w = policy_evict_first(), pol_x = policy_evict_last();
+      // Weight codes stream through L2 once (evict-first). A row's 128-byte scale line
+      // serves eight consecutive K-chunks, and every CTA of a problem reads the same
+      // activation images, so both stay (evict-last).
+      const uint64_t pol_w = policy_evict_first(), pol_sf = policy_evict_last(), pol_x = policy_evict_last();
       const uint32_t xbytes = (uint32_t)g.ku * g.img_stride;
       const uint32_t tx = g.wbytes + xbytes;
       int issued = 0;
@@ -462,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_2d(st + (uint32_t)(j * g.ku + h) * kNibBytes, &pr->tm_q, (cu.kc * g.ku + h) * (kKC / 2), row,
                         bar_full(s), pol_w);
           tma_load_2d(st + (uint32_t)(g.tpu * g.ku) * kNibBytes + (uint32_t)j * (kTileRows * 16u * g.ku), &pr->tm_sf,
-                      cu.kc * g.ku * (kKC / 16), row, bar_full(s), pol_w);
+                      cu.kc * g.ku * (kKC / 16), row, bar_full(s), pol_sf);
         }
       };
       auto load_x = [&](int s, const Cursor& cu) {
