@@ -297,6 +297,12 @@ __device__ __forceinline__ void tc_ld_x16(uint32_t taddr, uint32_t* v) {
       : "r"(taddr)
       : "memory");
 }
+__device__ __forceinline__ void tc_ld_x8(uint32_t taddr, uint32_t* v) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+               : "r"(taddr)
+               : "memory");
+}
 __device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
@@ -389,6 +395,11 @@ struct Walk {
   }
 };
 
+// Most tokens a kernel instance folds in registers: two B tiles hold M*T <= 352 rows
+// (M <= 70); one B tile M*T <= 256 (M <= 51); a tile pair needs a double-buffered
+// accumulator, which leaves N <= 104 per tile (M <= 20).
+__host__ __device__ constexpr int pass_max_tokens(int nbt, int tpu) { return tpu == 2 ? 24 : (nbt == 2 ? 72 : 56); }
+
 template <int NBT, int KU, int TPU>
 __global__ void __launch_bounds__(kThreads, 1)
     pass_kernel(const __grid_constant__ Problem single, const PassParams p) {
@@ -418,6 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bar_drain = smem_u32(bars + 2 * S + 4);
   auto bar_sffull = [&](int b) { return smem_u32(bars + 2 * S + 5 + b); };
 
+  constexpr int MT = pass_max_tokens(NBT, TPU);
   const Problem* probs = p.probs ? p.probs : &single;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c = blockIdx.x;
@@ -755,59 +767,76 @@ __global__ void __launch_bounds__(kThreads, 1)
       // i.e. g_0 * (acc_0 + (acc_1 + (acc_2 + (acc_3 + acc_4/4)/4)/4)/4) (the multiplications
       // by 1/4 are exact; the prep kernel's g_t are the same sequence unless it underflows).
       // Accumulator column j holds B row j, so token m's terms are columns m*T .. m*T+T-1.
-      // Tokens are taken 16 at a time: up to 5 TMEM loads of 16 columns are issued back to
-      // back and waited for once, and the 16 g_0 arrive as four 16-byte shared loads.
-      // Measured: with one epilogue warp per sub-partition the fold is latency-bound, and
-      // a per-term scale load ahead of every FMA made it 4x slower.
+      // Tokens are taken 8 at a time: five TMEM loads of 8 columns are issued back to back
+      // and waited for once. The folded row (at most MT tokens) stays in registers, so the
+      // accumulator is handed back to the MMA thread before any global store: with one
+      // accumulator buffer (M=68) the stores of a tile then overlap the next tile's MMAs
+      // (measured: holding the buffer through the stores stalled the MMA thread ~15 us per
+      // tile under full HBM load).
       static_assert(kMxf4Terms == 5, "the fold below is written for 5 terms");
       const int nb16 = (g.nb + 15) & ~15;                 // columns that exist in the accumulator
-      for (int tj = 0; tj < g.tpu; ++tj) {
-        const int tile = group * g.tpu + tj;
-        const long long n = (long long)tile * kTileRows + rowl;
-        const uint32_t taddr = taddr0 + (uint32_t)(tj * g.nbt * g.nb_tile);
-        float* dst = wave_part + ((long long)(slot * g.tpu + tj) * kTileRows + rowl) * Mp;   // this row's partials
-        for (int mc = 0; mc < M; mc += 16) {
-          const int col0 = mc * kMxf4Terms;                 // multiple of 80
-          const int nld = (nb16 - col0) / 16 < 5 ? (nb16 - col0) / 16 : 5;
-          uint32_t v[80];
-          tc_ld_x16(taddr + (uint32_t)col0, v);
-          if (nld > 1) tc_ld_x16(taddr + (uint32_t)(col0 + 16), v + 16);
-          if (nld > 2) tc_ld_x16(taddr + (uint32_t)(col0 + 32), v + 32);
-          if (nld > 3) tc_ld_x16(taddr + (uint32_t)(col0 + 48), v + 48);
-          if (nld > 4) tc_ld_x16(taddr + (uint32_t)(col0 + 64), v + 64);
-          float g0[16];
+      float yr[TPU][MT];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float4 t4 = reinterpret_cast<const float4*>(s_g0 + mc)[k];
-            g0[4 * k] = t4.x; g0[4 * k + 1] = t4.y; g0[4 * k + 2] = t4.z; g0[4 * k + 3] = t4.w;
-          }
-          tc_wait_ld();
-          float yv[16];
+      for (int tj = 0; tj < TPU; ++tj) {
+        const uint32_t taddr = taddr0 + (uint32_t)(tj * NBT * g.nb_tile);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            float a = __uint_as_float(v[j * kMxf4Terms + 4]);
-            a = fmaf(a, 0.25f, __uint_as_float(v[j * kMxf4Terms + 3]));
-            a = fmaf(a, 0.25f, __uint_as_float(v[j * kMxf4Terms + 2]));
-            a = fmaf(a, 0.25f, __uint_as_float(v[j * kMxf4Terms + 1]));
-            a = fmaf(a, 0.25f, __uint_as_float(v[j * kMxf4Terms + 0]));
-            yv[j] = (mc + j < M) ? a * g0[j] : 0.f;   // columns past the tokens are never loaded
-          }
-          if (complete) {
+        for (int mc = 0; mc < MT; mc += 8) {
+          if (mc < M) {
+            const int col0 = mc * kMxf4Terms;               // multiple of 40
+            const int n8 = (nb16 - col0) >> 3;              // >= 1: loads stay inside the accumulator
+            uint32_t v[40];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) yv[j] *= ts;
-            emit16(n, mc, yv);
+            for (int k = 0; k < 5; ++k)
+              if (k < n8) tc_ld_x8(taddr + (uint32_t)(col0 + 8 * k), v + 8 * k);
+            const float4 ga = reinterpret_cast<const float4*>(s_g0 + mc)[0];
+            const float4 gb = reinterpret_cast<const float4*>(s_g0 + mc)[1];
+            const float g0[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+            tc_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              float a = __uint_as_float(v[j * kMxf4Terms + 4]);
+              a = fmaf(a, 0.25f, __uint_as_float(v[j * kMxf4Terms + 3]));
+              a = fmaf(a, 0.25f, __uint_as_float(v[j * kMxf4Terms + 2]));
+              a = fmaf(a, 0.25f, __uint_as_float(v[j * kMxf4Terms + 1]));
+              a = fmaf(a, 0.25f, __uint_as_float(v[j * kMxf4Terms + 0]));
+              yr[tj][mc + j] = (mc + j < M) ? a * g0[j] : 0.f;   // columns past the tokens are never loaded
+            }
           } else {
 #pragma unroll
-            for (int b = 0; b < 4; ++b)
-              if (mc + 4 * b < Mp)
-                *reinterpret_cast<float4*>(dst + mc + 4 * b) = make_float4(yv[4 * b], yv[4 * b + 1], yv[4 * b + 2], yv[4 * b + 3]);
+            for (int j = 0; j < 8; ++j) yr[tj][mc + j] = 0.f;
           }
         }
-        if (complete && verify && tile < tiles) tile_argmax(tile);
       }
       tc_fence_before();
       if (et == 0 && seg < 2) MX_CTA(9 + 4 * seg);
       mbar_arrive(bar_accempty(ab));
+#pragma unroll
+      for (int tj = 0; tj < TPU; ++tj) {
+        const int tile = group * TPU + tj;
+        const long long n = (long long)tile * kTileRows + rowl;
+        if (complete) {
+#pragma unroll
+          for (int mc = 0; mc < MT; mc += 16) {
+            if (mc < M) {
+              float y16[16];
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                const int m = mc + j < MT ? mc + j : MT - 1;    // static index; tokens >= M are zeros
+                y16[j] = (mc + j < MT) ? yr[tj][m] * ts : 0.f;
+              }
+              emit16(n, mc, y16);
+            }
+          }
+          if (verify && tile < tiles) tile_argmax(tile);
+        } else {
+          float* dst = wave_part + ((long long)(slot * TPU + tj) * kTileRows + rowl) * Mp;   // this row's partials
+#pragma unroll
+          for (int b = 0; b < MT / 4; ++b)
+            if (4 * b < Mp)
+              *reinterpret_cast<float4*>(dst + 4 * b) =
+                  make_float4(yr[tj][4 * b], yr[tj][4 * b + 1], yr[tj][4 * b + 2], yr[tj][4 * b + 3]);
+        }
+      }
       ++seg;
       if (complete) continue;
       // Split tile group: count this CTA's arrival. The barrier orders every epilogue
@@ -1170,6 +1199,7 @@ static int launch_pass(const Problem& single, const Problem* probs_dev, const Pa
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (pl.g.M > pass_max_tokens(pl.g.nbt, pl.g.tpu)) return cudaErrorInvalidValue;
   cudaError_t e = (pl.g.nbt == 2)   ? cudaLaunchKernelEx(&cfg, pass_kernel<2, 1, 1>, single, p)
                   : (pl.g.tpu == 2) ? cudaLaunchKernelEx(&cfg, pass_kernel<1, 1, 2>, single, p)
                   : (pl.g.ku == 2)  ? cudaLaunchKernelEx(&cfg, pass_kernel<1, 2, 1>, single, p)
