@@ -621,50 +621,59 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t st = sbase + (uint32_t)s * p.stage_bytes;
       const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)fb * p.sf_cols;
-      for (int h = 0; h < g.ku; ++h) {
+      // All of a chunk's shared loads are issued before its first TMEM store: under a
+      // saturated ring one round trip to shared memory costs ~250 cycles, and three
+      // dependent rounds (W, then each B tile) made this copy the slowest hand-off at M=68.
+#pragma unroll
+      for (int h = 0; h < KU; ++h) {
+        uint4 RW[TPU][4], RX[NBT][8];
+        const uint32_t xs = st + g.wbytes + (uint32_t)h * g.img_stride + g.img_xs_off;
+#pragma unroll
+        for (int t = 0; t < TPU; ++t) {
+          const uint32_t wsf = st + wsf_off + (uint32_t)t * (kTileRows * wsf_row);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) RW[t][j] = lds128(wsf + (uint32_t)(m0 + 32 * j) * wsf_row + (uint32_t)h * 16u);
+        }
+#pragma unroll
+        for (int bt = 0; bt < NBT; ++bt) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int row = m0 + 32 * j;
+            RX[bt][j] = (j < g.nsfb && row < g.nb_tile) ? lds128(xs + (uint32_t)((bt * g.nb_tile + row) * 16))
+                                                        : make_uint4(0, 0, 0, 0);
+          }
+        }
         // W scales of tile t: column 16*(t*ku + h) + 4*kk + j of lane m0 = the 4 block scales
         // (K-step kk of chunk h) of row m0 + 32*j
-        for (int t = 0; t < g.tpu; ++t) {
-          const uint32_t wsf = st + wsf_off + (uint32_t)t * (kTileRows * wsf_row);
-          uint4 R[4];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) R[j] = lds128(wsf + (uint32_t)(m0 + 32 * j) * wsf_row + (uint32_t)h * 16u);
+        for (int t = 0; t < TPU; ++t) {
           uint32_t out[16];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            out[0 + j] = R[j].x; out[4 + j] = R[j].y; out[8 + j] = R[j].z; out[12 + j] = R[j].w;
+            out[0 + j] = RW[t][j].x; out[4 + j] = RW[t][j].y; out[8 + j] = RW[t][j].z; out[12 + j] = RW[t][j].w;
           }
-          tc_st_x16(lane_base + (uint32_t)(t * g.ku + h) * 16u, out);
+          tc_st_x16(lane_base + (uint32_t)(t * KU + h) * 16u, out);
         }
-        const uint32_t xs = st + g.wbytes + (uint32_t)h * g.img_stride + g.img_xs_off;
-        if (g.nbt == 1 && g.nsfb == 4) {
+        if (NBT == 1 && g.nsfb == 4) {
           // one B tile of <= 128 rows: the chunk's 4 K-steps x 4 columns are contiguous, so
           // column 4*kk + j of lane m0 (B row m0 + 32*j, K-step kk) goes in one x16 store
-          uint4 R[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            R[j] = (m0 + 32 * j < g.nb_tile) ? lds128(xs + (uint32_t)((m0 + 32 * j) * 16)) : make_uint4(0, 0, 0, 0);
           uint32_t out[16];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            out[0 + j] = R[j].x; out[4 + j] = R[j].y; out[8 + j] = R[j].z; out[12 + j] = R[j].w;
+            out[0 + j] = RX[0][j].x; out[4 + j] = RX[0][j].y; out[8 + j] = RX[0][j].z; out[12 + j] = RX[0][j].w;
           }
           tc_st_x16(lane_base + xsf_col + (uint32_t)h * 16u, out);
           continue;
         }
-        for (int bt = 0; bt < g.nbt; ++bt) {   // X-term scales, per B tile: nsfb columns per K-step
-          uint4 R[8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int row = m0 + 32 * j;
-            R[j] = (j < g.nsfb && row < g.nb_tile) ? lds128(xs + (uint32_t)((bt * g.nb_tile + row) * 16))
-                                                   : make_uint4(0, 0, 0, 0);
-          }
+        for (int bt = 0; bt < NBT; ++bt) {   // X-term scales, per B tile: nsfb columns per K-step
+#pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             uint32_t out[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) out[j] = kk == 0 ? R[j].x : kk == 1 ? R[j].y : kk == 2 ? R[j].z : R[j].w;
-            const uint32_t col = xsf_col + (uint32_t)(((h * 4 + kk) * g.nbt + bt) * g.nsfb);
+            for (int j = 0; j < 8; ++j)
+              out[j] = kk == 0 ? RX[bt][j].x : kk == 1 ? RX[bt][j].y : kk == 2 ? RX[bt][j].z : RX[bt][j].w;
+            const uint32_t col = xsf_col + (uint32_t)(((h * 4 + kk) * NBT + bt) * g.nsfb);
             if (g.nsfb == 8) tc_st_x8(lane_base + col, out);
             else tc_st_x4(lane_base + col, out[0], out[1], out[2], out[3]);
           }
