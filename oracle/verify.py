@@ -23,6 +23,16 @@ Readings where the pages are silent:
 * The accept length is ``L = min{i in [0, D) : d[b, i] != t[b(D+1) + i]}``, or D if
   there is no mismatch. The committed tokens are ``t[b(D+1) .. b(D+1) + L]``:
   the L accepted drafts followed by the target's own token at position L.
+* Tree verify ("How it works": the drafters propose a tree, the target verifies the
+  whole tree in one pass, and the longest path it agrees with is kept). A sequence
+  has nodes 0..D: node 0 is the committed context, node k >= 1 holds draft token
+  ``d[b, k-1]`` and has parent ``p[b, k-1]`` in ``[0, k-1]``. Row ``b(D+1) + k`` is
+  the target's prediction after the root-to-k path. Node k is accepted when its
+  parent is accepted and ``d[b, k-1] == t[b(D+1) + p[b, k-1]]`` (the root always is).
+  The kept path ends at the accepted node of greatest depth, the lowest node index
+  among equals; the accept length is its depth, and the committed tokens are the
+  drafts on the path followed by the target's token at its end node. With
+  ``p[b, k-1] = k-1`` (a chain) this is the accept rule above.
 * Near ties. A row whose two largest logits differ by less than ``1e-3`` (in
   logit units) is excluded from exact argmax comparison. That is the pages'
   one-ulp caveat. A sequence is excluded from the exact accept-length comparison
@@ -122,3 +132,60 @@ def comparable_sequences(gap: np.ndarray, L: np.ndarray, D: int, tol: float = NE
         rows = ok[b * (D + 1): b * (D + 1) + int(L[b]) + 1]
         out[b] = bool(rows.all())
     return out
+
+
+def accept_tree_ref(t: np.ndarray, drafts: np.ndarray, parents: np.ndarray, D: int):
+    """Tree verify: returns ``(L [B], node [B])``, the depth and index of the kept path's end.
+
+    Nodes are visited in index order; a parent always precedes its child, so one pass
+    settles every node. A parent index outside ``[0, k-1]`` raises.
+    """
+    drafts = np.asarray(drafts, dtype=np.int64)
+    parents = np.asarray(parents, dtype=np.int64)
+    t = np.asarray(t, dtype=np.int64)
+    B = drafts.shape[0] if drafts.ndim == 2 else 0
+    if t.shape[0] != B * (D + 1) or (D > 0 and parents.shape != (B, D)):
+        raise ValueError("t must have B*(D+1) rows and parents must be [B, D]")
+    L = np.zeros(B, dtype=np.int64)
+    node = np.zeros(B, dtype=np.int64)
+    for b in range(B):
+        base = b * (D + 1)
+        accepted = [True] + [False] * D
+        depth = [0] * (D + 1)
+        for k in range(1, D + 1):
+            p = int(parents[b, k - 1])
+            if not 0 <= p < k:
+                raise ValueError(f"parent of node {k} must be in [0, {k - 1}], got {p}")
+            depth[k] = depth[p] + 1
+            accepted[k] = accepted[p] and drafts[b, k - 1] == t[base + p]
+            if accepted[k] and depth[k] > L[b]:
+                L[b], node[b] = depth[k], k
+    return L, node
+
+
+def tree_path(parents: np.ndarray, b: int, node: int):
+    """Nodes on the root-to-``node`` path of sequence b, root excluded, in path order."""
+    path = []
+    while node != 0:
+        path.append(node)
+        node = int(parents[b, node - 1])
+    return path[::-1]
+
+
+def committed_tree_ref(t: np.ndarray, drafts: np.ndarray, parents: np.ndarray, node: np.ndarray, D: int):
+    """Committed tokens per sequence: the drafts on the kept path, then the target's token at its end."""
+    t = np.asarray(t, dtype=np.int64)
+    out = []
+    for b in range(len(node)):
+        path = tree_path(parents, b, int(node[b]))
+        toks = [int(drafts[b, k - 1]) for k in path] + [int(t[b * (D + 1) + int(node[b])])]
+        out.append(np.asarray(toks, dtype=np.int64))
+    return out
+
+
+def comparable_tree_sequences(gap: np.ndarray, parents: np.ndarray, D: int, tol: float = NEAR_TIE) -> np.ndarray:
+    """Sequences whose tree verify must match exactly: every row of the sequence has a
+    top-2 gap of at least ``tol`` (any row can decide a node's acceptance in a tree)."""
+    ok = comparable_rows(gap, tol)
+    B = len(ok) // (D + 1)
+    return np.array([bool(ok[b * (D + 1): (b + 1) * (D + 1)].all()) for b in range(B)], dtype=bool)

@@ -119,3 +119,37 @@ def drafts_with_prefix(t: np.ndarray, Lstar: np.ndarray, D: int, vocab: int, see
             while d[b, Ls] == t[base + Ls]:
                 d[b, Ls] = rng.integers(0, vocab)
     return d.astype(np.int32)
+
+
+def random_tree(B: int, D: int, seed: int = 209, chain_bias: float = 0.5) -> np.ndarray:
+    """Parent arrays of B draft trees with nodes 1..D: int32 [B, D], the parent of node
+    k in [0, k-1]. With probability ``chain_bias`` a node hangs under node k-1 (deep
+    branches), else under a uniform earlier node (wide trees)."""
+    rng = np.random.default_rng(seed)
+    p = np.zeros((B, D), dtype=np.int64)
+    for b in range(B):
+        for k in range(1, D + 1):
+            p[b, k - 1] = k - 1 if rng.random() < chain_bias else rng.integers(0, k)
+    return p.astype(np.int32)
+
+
+def tree_drafts(t: np.ndarray, parents: np.ndarray, D: int, vocab: int, agree: float = 0.7,
+                seed: int = 210) -> np.ndarray:
+    """Draft tokens for the trees in ``parents``: node k copies the target token ``t`` at
+    its parent's row with probability ``agree``, else a different uniform id."""
+    t = np.asarray(t, dtype=np.int64)
+    parents = np.asarray(parents, dtype=np.int64)
+    B = parents.shape[0]
+    rng = np.random.default_rng(seed)
+    d = np.zeros((B, D), dtype=np.int64)
+    for b in range(B):
+        for k in range(1, D + 1):
+            want = t[b * (D + 1) + parents[b, k - 1]]
+            if rng.random() < agree:
+                d[b, k - 1] = want
+            else:
+                x = rng.integers(0, vocab)
+                while x == want:
+                    x = rng.integers(0, vocab)
+                d[b, k - 1] = x
+    return d.astype(np.int32)

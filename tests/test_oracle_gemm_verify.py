@@ -158,3 +158,91 @@ def test_comparable_sequences():
     assert V.comparable_sequences(gap, L, 2).tolist() == [True, True]
     L = np.array([1, 2])
     assert V.comparable_sequences(gap, L, 2).tolist() == [False, True]
+
+
+# ----------------------------------------------------------------------------- tree verify
+
+def _golden_trees():
+    import json
+    import os
+    with open(os.path.join(os.path.dirname(__file__), "golden", "tree_verify.json")) as f:
+        return json.load(f)["cases"]
+
+
+@pytest.mark.parametrize("case", _golden_trees(), ids=lambda c: c["name"])
+def test_tree_verify_hand_worked(case):
+    p = np.array([case["parents"]])
+    d = np.array([case["drafts"]])
+    t = np.array(case["t"])
+    D = p.shape[1]
+    L, node = V.accept_tree_ref(t, d, p, D)
+    assert (L.tolist(), node.tolist()) == ([case["accept_len"]], [case["accept_node"]])
+    assert V.committed_tree_ref(t, d, p, node, D)[0].tolist() == case["committed"]
+
+
+def _brute_tree(t, d, p, D):
+    """Every root-to-node path spelled out; a path is kept when each of its drafts equals the
+    target token at the row of the node before it. Longest kept path, lowest end node."""
+    best_len, best_node = 0, 0
+    for end in range(1, D + 1):
+        path = []
+        k = end
+        while k != 0:
+            path.append(k)
+            k = int(p[k - 1])
+        path.reverse()
+        prev, ok = 0, True
+        for k in path:
+            ok = ok and d[k - 1] == t[prev]
+            prev = k
+        if ok and len(path) > best_len:
+            best_len, best_node = len(path), end
+    return best_len, best_node
+
+
+def test_tree_verify_brute_force_random():
+    rng = np.random.default_rng(31)
+    for _ in range(400):
+        D = int(rng.integers(0, 9))
+        p = np.array([[int(rng.integers(0, k)) for k in range(1, D + 1)]], dtype=np.int64).reshape(1, D)
+        t = rng.integers(0, 3, size=D + 1)
+        d = rng.integers(0, 3, size=(1, D))
+        L, node = V.accept_tree_ref(t, d, p, D)
+        assert (int(L[0]), int(node[0])) == _brute_tree(t, d[0], p[0], D)
+
+
+def test_tree_verify_chain_is_the_accept_rule():
+    rng = np.random.default_rng(32)
+    B, D, vocab = 30, 16, 3
+    t = rng.integers(0, vocab, size=B * (D + 1))
+    d = rng.integers(0, vocab, size=(B, D))
+    chain = np.tile(np.arange(D), (B, 1))
+    L, node = V.accept_tree_ref(t, d, chain, D)
+    assert np.array_equal(L, V.accept_ref(t, d, D))
+    assert np.array_equal(node, L)
+
+
+def test_tree_verify_invariants_and_generators():
+    rng = np.random.default_rng(33)
+    B, D, vocab = 40, 24, 7
+    t = rng.integers(0, vocab, size=B * (D + 1))
+    p = S.random_tree(B, D, seed=5)
+    assert all(0 <= p[b, k - 1] < k for b in range(B) for k in range(1, D + 1))
+    d = S.tree_drafts(t, p, D, vocab, agree=0.8, seed=6)
+    L, node = V.accept_tree_ref(t, d, p, D)
+    for b, toks in enumerate(V.committed_tree_ref(t, d, p, node, D)):
+        path = V.tree_path(p, b, int(node[b]))
+        assert len(path) == L[b] and len(toks) == L[b] + 1
+        rows = [0] + path                        # committed tokens are the target's greedy tokens along the path
+        assert toks.tolist() == [int(t[b * (D + 1) + r]) for r in rows]
+    assert (L > 0).any() and (L < D).all()
+
+
+def test_tree_verify_rejects_bad_parent():
+    with pytest.raises(ValueError):
+        V.accept_tree_ref(np.array([1, 2, 3]), np.array([[1, 2]]), np.array([[0, 2]]), 2)
+
+
+def test_comparable_tree_sequences():
+    gap = np.array([1.0, 1.0, 1e-4, 1.0, 1.0, 1.0])   # B = 2, D = 2
+    assert V.comparable_tree_sequences(gap, None, 2).tolist() == [False, True]

@@ -93,3 +93,25 @@ def test_last_index_argmax_caught():
     y = np.array([[1.0, 3.0, 3.0]])
     last = y.shape[1] - 1 - np.argmax(y[:, ::-1], axis=1)
     assert last.tolist() != V.argmax_ref(y).tolist()
+
+
+def test_tree_child_row_instead_of_parent_row_caught():
+    """Checking a node's draft against its own row (not its parent's) breaks the hand-worked tree."""
+    with open(os.path.join(GOLDEN, "tree_verify.json")) as f:
+        case = json.load(f)["cases"][0]
+    p, d, t = np.array([case["parents"]]), np.array([case["drafts"]]), np.array(case["t"])
+    D = p.shape[1]
+
+    def wrong(t, d, p, D):
+        L, node, acc, depth = 0, 0, [True] + [False] * D, [0] * (D + 1)
+        for k in range(1, D + 1):
+            q = int(p[0, k - 1])
+            depth[k] = depth[q] + 1
+            acc[k] = acc[q] and d[0, k - 1] == t[k]
+            if acc[k] and depth[k] > L:
+                L, node = depth[k], k
+        return L, node
+
+    assert wrong(t, d, p, D) != (case["accept_len"], case["accept_node"])
+    L, node = V.accept_tree_ref(t, d, p, D)
+    assert (int(L[0]), int(node[0])) == (case["accept_len"], case["accept_node"])
