@@ -187,8 +187,9 @@ class Pass:
     192 GEMMs with the lm_head verify as its last problem), and, for comparison, the
     chained per-GEMM launch sequence, each captured in a CUDA graph."""
 
-    def __init__(self, nv, torch, dev, stack, lm, M: int, rank: int, chain: bool):
+    def __init__(self, nv, torch, dev, stack, lm, M: int, rank: int, chain: bool, tree: bool = False):
         self.M = M
+        self.tree = tree
         self.torch = torch
         self.B = max(1, M // (S.DRAFT_LEN + 1)) if M >= S.DRAFT_LEN + 1 else 1
         self.D = M // self.B - 1
@@ -211,7 +212,12 @@ class Pass:
         problems = [(self.xs[i].view(M, K), q, sf, ts, self.ys[i]) for i, (_, K, _, q, sf, ts) in enumerate(stack)]
         ql, sfl, tsl = lm
         problems.append((self.xs[-1].view(M, S.LMHEAD_K), ql, sfl, tsl, None))
-        self.wp = nv.WeightPass(problems, M, verify=(self.drafts, self.argmax, self.accept, self.vmax))
+        verify = (self.drafts, self.argmax, self.accept, self.vmax)
+        if tree:   # draft trees of D nodes per sequence instead of chains
+            self.parents = torch.from_numpy(S.random_tree(self.B, self.D, seed=S.LMHEAD_L_SEED + M)).to(dev)
+            self.node = torch.empty(self.B, dtype=torch.int32, device=dev)
+            verify = verify + (self.parents, self.node)
+        self.wp = nv.WeightPass(problems, M, verify=verify)
         if chain:
             wsb = max(nv.gemm_workspace_bytes(M, N, K) for (_, K, N, _, _, _) in stack)
             self.gws = torch.zeros(max(wsb, 16), dtype=torch.uint8, device=dev)
@@ -222,7 +228,10 @@ class Pass:
         torch.cuda.synchronize()
         t = self.argmax.cpu().numpy()
         Lstar = np.random.default_rng(S.LMHEAD_L_SEED + M).integers(0, self.D + 1, size=self.B)
-        d = S.drafts_with_prefix(t, Lstar, self.D, S.VOCAB)
+        if tree:
+            d = S.tree_drafts(t, self.parents.cpu().numpy(), self.D, S.VOCAB, agree=0.8, seed=S.LMHEAD_L_SEED + M)
+        else:
+            d = S.drafts_with_prefix(t, Lstar, self.D, S.VOCAB)
         self.drafts.copy_(torch.from_numpy(d))
         self.Lstar = Lstar
 
@@ -235,7 +244,11 @@ class Pass:
     def chain_verify_call(self):
         q, sf, ts = self.lm
         X = self.xs[-1].view(self.M, S.LMHEAD_K)
-        self.nv.verify(X, q, sf, ts, self.drafts, workspace=self.vws, out=(self.argmax, self.accept, self.vmax))
+        if self.tree:
+            self.nv.verify_tree(X, q, sf, ts, self.drafts, self.parents, workspace=self.vws,
+                                out=(self.argmax, self.accept, self.node, self.vmax))
+        else:
+            self.nv.verify(X, q, sf, ts, self.drafts, workspace=self.vws, out=(self.argmax, self.accept, self.vmax))
 
     def capture(self):
         torch = self.torch
@@ -333,7 +346,7 @@ def run_ours(args, rank, world, local_rank):
     M_list = [int(m) for m in args.ms.split(",")]
     stack, lm = build_pass(nv, torch, dev, M_list, rank, args.layers)
     head = 17 if 17 in M_list else M_list[0]
-    passes = {M: Pass(nv, torch, dev, stack, lm, M, rank, chain=not args.no_chain) for M in M_list}
+    passes = {M: Pass(nv, torch, dev, stack, lm, M, rank, chain=not args.no_chain, tree=args.tree) for M in M_list}
     for p in passes.values():
         p.capture()
         for _ in range(args.warmup):
@@ -369,7 +382,7 @@ def run_ours(args, rank, world, local_rank):
             "ms_min": float(per.min()),
             "ms_max": float(per.max()),
             "launches_per_pass": p.launches_pass,
-            "B": p.B, "D": p.D,
+            "B": p.B, "D": p.D, "verify": "tree" if p.tree else "chain",
         }
         if p.chain:
             # the same work as 193 chained launches: each GEMM's activations are read only
@@ -552,6 +565,8 @@ def main():
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per pass_kernel launch (default: the stored ncu capture in profiles/, "
                          "when the kernel sources still match it)")
+    ap.add_argument("--tree", action="store_true",
+                    help="verify draft trees of D nodes per sequence (seeded random parents) instead of chains")
     ap.add_argument("--sweep", action="store_true", help="time one matrix shape per M and path (no pass)")
     ap.add_argument("--shape", default="gate_up", help="sweep shape: gate_up, down, qkv or lm_head")
     ap.add_argument("--paths", default="auto,gemv,mma")

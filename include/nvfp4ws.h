@@ -194,6 +194,35 @@ int lmhead_verify_argmax_accept(const void* X, const uint8_t* q, const uint8_t* 
                                 int32_t* argmax, int32_t* accept_len, float* max_logit,
                                 void* workspace, size_t workspace_bytes, nvfp4ws_stream_t stream);
 
+/*
+ * lmhead_verify_tree -- lm_head GEMM with fused greedy verify of a draft TREE.
+ *
+ * Passage: "TandemLLM", "How it works" (the drafters propose a tree, the target
+ * verifies the whole tree in one pass, and the longest path it agrees with is kept).
+ *
+ * Each sequence b has nodes 0..D. Node 0 is the committed context. Node k >= 1 holds
+ * the draft token drafts[b, k-1] and hangs under node parents[b, k-1], which must lie
+ * in [0, k-1] (a parent precedes its children). Row b*(D+1)+k of X is the target's
+ * input after the root-to-k path, so argmax[b*(D+1)+k] is its greedy next token there.
+ * Node k is accepted when its parent is accepted and
+ *   drafts[b, k-1] == argmax[b*(D+1) + parents[b, k-1]]      (node 0 always is).
+ * The kept path ends at the accepted node of greatest depth (the lowest node index
+ * among equals): accept_node[b] is that node and accept_len[b] its depth. The
+ * committed tokens are the drafts on the root-to-accept_node path, in path order,
+ * followed by argmax[b*(D+1) + accept_node[b]]. With parents[b, k-1] = k-1 for every
+ * k (a chain) the result is lmhead_verify_argmax_accept's.
+ *
+ * Arguments as lmhead_verify_argmax_accept, plus
+ *   parents      int32 [B, D] row-major, device (may be NULL when D == 0).
+ *   accept_node  out: int32 [B], device, or NULL to skip.
+ * A parent outside [0, k-1] rejects its node and sets the device error word, which the
+ * next nvfp4ws_check reports as NVFP4WS_ERR_INVALID_ARG.
+ */
+int lmhead_verify_tree(const void* X, const uint8_t* q, const uint8_t* sf, const float* tensor_scale,
+                       int64_t M, int64_t N, int64_t K, const int32_t* drafts, const int32_t* parents,
+                       int32_t B, int32_t D, int32_t* argmax, int32_t* accept_len, int32_t* accept_node,
+                       float* max_logit, void* workspace, size_t workspace_bytes, nvfp4ws_stream_t stream);
+
 /* As lmhead_verify_argmax_accept, with an explicit kernel path (nvfp4ws_path). */
 int lmhead_verify_argmax_accept_path(const void* X, const uint8_t* q, const uint8_t* sf,
                                      const float* tensor_scale, int64_t M, int64_t N, int64_t K,
@@ -242,7 +271,9 @@ int lmhead_verify_argmax_accept_path(const void* X, const uint8_t* q, const uint
  *   M             1 <= M <= 70 (the block-scaled path's limit).
  *   verify        NULL, or the verify buffers: M must equal B * (D + 1); drafts int32
  *                 [B, D] (may be NULL when D == 0); argmax int32 [M]; accept_len int32
- *                 [B]; max_logit fp32 [M] or NULL.
+ *                 [B]; max_logit fp32 [M] or NULL; parents int32 [B, D] for a tree
+ *                 verify as lmhead_verify_tree computes it, or NULL for the chain rule;
+ *                 accept_node int32 [B] or NULL (the kept path's end node).
  *   pass          caller-owned host state, filled by nvfp4_pass_init.
  * Returns NVFP4WS_OK, or INVALID_ARG / UNSUPPORTED / MISALIGNED / WORKSPACE / CUDA.
  */
@@ -264,6 +295,8 @@ typedef struct nvfp4_verify_spec {
   int32_t* argmax;
   int32_t* accept_len;
   float* max_logit;
+  const int32_t* parents;
+  int32_t* accept_node;
 } nvfp4_verify_spec;
 
 typedef struct nvfp4_pass {

@@ -8,6 +8,7 @@ torch, and passes raw device pointers and the current CUDA stream.
     q, sf, ts = pack(W)                        # fp32 [N, K] -> NVFP4
     Y = gemm(X, q, sf, ts)                     # bf16 [M, K] -> fp32 [M, N]
     t, L, vmax = verify(X, q, sf, ts, drafts)  # fused lm_head argmax + accept length
+    t, L, node, vmax = verify_tree(X, q, sf, ts, drafts, parents)   # the same over a draft tree
     p = WeightPass([(X_i, q_i, sf_i, ts_i, Y_i), ...], M, verify=...)   # a whole list, one launch
     p.run()
 """
@@ -141,6 +142,39 @@ def verify(X: torch.Tensor, q: torch.Tensor, sf: torch.Tensor, ts: torch.Tensor,
     return amax, acc, vmax
 
 
+def verify_tree(X: torch.Tensor, q: torch.Tensor, sf: torch.Tensor, ts: torch.Tensor, drafts: torch.Tensor,
+                parents: torch.Tensor, workspace: torch.Tensor | None = None, with_max_logit: bool = True,
+                stream=None, out=None):
+    """Fused lm_head greedy verify of draft trees (``lmhead_verify_tree``). ``drafts`` and
+    ``parents`` int32 [B, D]: node k >= 1 holds ``drafts[b, k-1]`` under node ``parents[b, k-1]``.
+
+    Returns ``(argmax int32 [M], accept_len int32 [B], accept_node int32 [B], max_logit fp32 [M] or None)``.
+    """
+    _need_cuda(X, "X", torch.bfloat16)
+    _need_cuda(drafts, "drafts", torch.int32)
+    _need_cuda(parents, "parents", torch.int32)
+    M, K = X.shape
+    N = q.shape[0]
+    B, D = drafts.shape
+    if parents.shape != (B, D):
+        raise ValueError("parents must have the shape of drafts")
+    if out is None:
+        amax = torch.empty(M, dtype=torch.int32, device=X.device)
+        acc = torch.empty(B, dtype=torch.int32, device=X.device)
+        node = torch.empty(B, dtype=torch.int32, device=X.device)
+        vmax = torch.empty(M, dtype=torch.float32, device=X.device) if with_max_logit else None
+    else:
+        amax, acc, node, vmax = out
+    ws = _workspace(verify_workspace_bytes(M, N, K), X.device, workspace)
+    nbytes = 0 if ws is None else ws.numel()
+    dptr = _ptr(drafts) if drafts.numel() else None
+    pptr = _ptr(parents) if parents.numel() else None
+    _check(lib().lmhead_verify_tree(_ptr(X), _ptr(q), _ptr(sf), _ptr(ts), M, N, K, dptr, pptr, B, D, _ptr(amax),
+                                    _ptr(acc), _ptr(node), _ptr(vmax), _ptr(ws), nbytes, _stream(stream)),
+           "lmhead_verify_tree")
+    return amax, acc, node, vmax
+
+
 def check(stream=None):
     """Synchronise and report a device-side bounded-wait failure, if any."""
     _check(lib().nvfp4ws_check(_stream(stream)), "nvfp4ws_check")
@@ -152,8 +186,9 @@ class WeightPass:
     ``problems`` is a list of ``(X, q, sf, ts, Y)``: X bf16 [M, K], the packed weight,
     and Y fp32 or bf16 [M, N]. With ``verify=(drafts, argmax, accept_len, max_logit)``
     the last problem is the lm_head: its Y may be None, and each run ends with the
-    argmax over its rows and the accept lengths. Every tensor is referenced by address:
-    keep them alive and refill X in place between runs.
+    argmax over its rows and the accept lengths. ``verify`` may add ``(parents,
+    accept_node)`` for a tree verify (``accept_node`` may be None). Every tensor is
+    referenced by address: keep them alive and refill X in place between runs.
     """
 
     def __init__(self, problems, M: int, verify=None, workspace: torch.Tensor | None = None):
@@ -181,11 +216,17 @@ class WeightPass:
             self._keep.extend([X, q, sf, ts, Y])
         vs = None
         if verify is not None:
-            drafts, amax, acc, vmax = verify
+            drafts, amax, acc, vmax = verify[:4]
+            parents, node = (tuple(verify[4:]) + (None, None))[:2]
             _need_cuda(drafts, "drafts", torch.int32)
             B, D = drafts.shape
-            vs = L.VerifySpec(_ptr(drafts) if drafts.numel() else None, B, D, _ptr(amax), _ptr(acc), _ptr(vmax))
-            self._keep.extend([drafts, amax, acc, vmax])
+            if parents is not None:
+                _need_cuda(parents, "parents", torch.int32)
+                if parents.shape != (B, D):
+                    raise ValueError("parents must have the shape of drafts")
+            vs = L.VerifySpec(_ptr(drafts) if drafts.numel() else None, B, D, _ptr(amax), _ptr(acc), _ptr(vmax),
+                              _ptr(parents) if parents is not None and parents.numel() else None, _ptr(node))
+            self._keep.extend([drafts, amax, acc, vmax, parents, node])
         nbytes = int(lib().nvfp4_pass_workspace_bytes(arr, n, M, 1 if verify is not None else 0))
         if nbytes == 0:
             raise NVFP4WSError(1, "nvfp4_pass_workspace_bytes")

@@ -24,7 +24,7 @@ class GemmProblem(ctypes.Structure):
 class VerifySpec(ctypes.Structure):
     """nvfp4_verify_spec: the verify buffers of a pass whose last problem is the lm_head."""
     _fields_ = [("drafts", c_p), ("B", c_i32), ("D", c_i32), ("argmax", c_p), ("accept_len", c_p),
-                ("max_logit", c_p)]
+                ("max_logit", c_p), ("parents", c_p), ("accept_node", c_p)]
 
 
 class PassState(ctypes.Structure):
@@ -48,6 +48,8 @@ SIGNATURES = {
                                                    c_p, c_p, c_p, c_sz, c_p]),
     "lmhead_verify_argmax_accept_path": (ctypes.c_int, [c_p, c_p, c_p, c_p, c_i64, c_i64, c_i64, c_p, c_i32, c_i32,
                                                         c_p, c_p, c_p, c_p, c_sz, ctypes.c_int, c_p]),
+    "lmhead_verify_tree": (ctypes.c_int, [c_p, c_p, c_p, c_p, c_i64, c_i64, c_i64, c_p, c_p, c_i32, c_i32, c_p, c_p,
+                                          c_p, c_p, c_p, c_sz, c_p]),
     "nvfp4ws_check": (ctypes.c_int, [c_p]),
     "nvfp4_gemm_skinny_noalloc": (ctypes.c_int, [c_p, c_p, c_p, c_p, c_i64, c_i64, c_i64, c_p, ctypes.c_int, c_p]),
     "nvfp4ws_kernel_launches": (ctypes.c_ulonglong, []),

@@ -205,11 +205,15 @@ size_t lmhead_verify_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   return x > w ? x : w;
 }
 
-int lmhead_verify_argmax_accept_path(const void* X, const uint8_t* q, const uint8_t* sf, const float* tensor_scale,
-                                     int64_t M, int64_t N, int64_t K, const int32_t* drafts, int32_t B, int32_t D,
-                                     int32_t* argmax, int32_t* accept_len, float* max_logit, void* workspace,
-                                     size_t workspace_bytes, int path, nvfp4ws_stream_t stream) {
-  g_last_error[0] = 0;
+}  // extern "C"
+
+// The lm_head GEMM and its fused verify, chain (v.parents == null) or tree.
+static int verify_impl(const void* X, const uint8_t* q, const uint8_t* sf, const float* tensor_scale, int64_t M,
+                       int64_t N, int64_t K, const VerifyRule& v, void* workspace, size_t workspace_bytes, int path,
+                       cudaStream_t s) {
+  const int32_t* drafts = v.drafts;
+  const int32_t B = v.B, D = v.D;
+  int32_t *argmax = v.argmax, *accept_len = v.accept_len;
   if (int e = validate_gemm(X, q, sf, tensor_scale, M, N, K, "lmhead_verify")) return e;
   if (B < 1 || D < 0) return set_error(NVFP4WS_ERR_INVALID_ARG, "lmhead_verify: need B >= 1 and D >= 0");
   if ((int64_t)B * (D + 1) != M)
@@ -220,7 +224,6 @@ int lmhead_verify_argmax_accept_path(const void* X, const uint8_t* q, const uint
   if (path < NVFP4WS_PATH_AUTO || path > NVFP4WS_PATH_MMA_F16)
     return set_error(NVFP4WS_ERR_INVALID_ARG, "lmhead_verify: bad path %d", path);
   const int kp = resolve_path(path, M, K);
-  cudaStream_t s = (cudaStream_t)stream;
   if (kp == KPATH_NONE)
     return set_error(NVFP4WS_ERR_UNSUPPORTED, "lmhead_verify: the tensor-core paths need K %% 256 == 0 and "
                      "M <= 128 (M=%lld K=%lld)", (long long)M, (long long)K);
@@ -229,16 +232,14 @@ int lmhead_verify_argmax_accept_path(const void* X, const uint8_t* q, const uint
     if (workspace == nullptr || workspace_bytes < need)
       return set_error(NVFP4WS_ERR_WORKSPACE, "lmhead_verify: workspace needs %zu bytes", need);
     if (!aligned16(workspace)) return set_error(NVFP4WS_ERR_MISALIGNED, "lmhead_verify: workspace must be 16-byte aligned");
-    return launch_mxf4_verify(static_cast<const uint16_t*>(X), q, sf, tensor_scale, M, N, K, drafts, B, D, argmax,
-                              accept_len, max_logit, workspace, s);
+    return launch_mxf4_verify(static_cast<const uint16_t*>(X), q, sf, tensor_scale, M, N, K, v, workspace, s);
   }
   if (kp == KPATH_MMA_F16) {
     size_t need = mma_verify_workspace_bytes(M, N, K);
     if (workspace == nullptr || workspace_bytes < need)
       return set_error(NVFP4WS_ERR_WORKSPACE, "lmhead_verify: workspace needs %zu bytes", need);
     if (!aligned16(workspace)) return set_error(NVFP4WS_ERR_MISALIGNED, "lmhead_verify: workspace must be 16-byte aligned");
-    return launch_mma_verify(static_cast<const uint16_t*>(X), q, sf, tensor_scale, M, N, K, drafts, B, D, argmax,
-                             accept_len, max_logit, workspace, s);
+    return launch_mma_verify(static_cast<const uint16_t*>(X), q, sf, tensor_scale, M, N, K, v, workspace, s);
   }
   if (!gemv_supported(K)) return set_error(NVFP4WS_ERR_UNSUPPORTED, "lmhead_verify: GEMV path supports K <= 65536");
   size_t need = gemv_verify_workspace(M, N, K);
@@ -255,7 +256,29 @@ int lmhead_verify_argmax_accept_path(const void* X, const uint8_t* q, const uint
   a.part_val = static_cast<float*>(workspace);
   a.part_idx = reinterpret_cast<int*>(static_cast<char*>(workspace) + align_up((size_t)pgrid * M * 4, 256));
   if (int e = launch_gemv(a, true, regs_only, s)) return e;
-  return launch_verify_stage2(a.part_val, a.part_idx, p.grid, (int)M, drafts, B, D, argmax, accept_len, max_logit, s);
+  return launch_verify_stage2(a.part_val, a.part_idx, p.grid, (int)M, v, s);
+}
+
+extern "C" {
+
+int lmhead_verify_argmax_accept_path(const void* X, const uint8_t* q, const uint8_t* sf, const float* tensor_scale,
+                                     int64_t M, int64_t N, int64_t K, const int32_t* drafts, int32_t B, int32_t D,
+                                     int32_t* argmax, int32_t* accept_len, float* max_logit, void* workspace,
+                                     size_t workspace_bytes, int path, nvfp4ws_stream_t stream) {
+  g_last_error[0] = 0;
+  const VerifyRule v{drafts, nullptr, B, D, argmax, accept_len, nullptr, max_logit};
+  return verify_impl(X, q, sf, tensor_scale, M, N, K, v, workspace, workspace_bytes, path, (cudaStream_t)stream);
+}
+
+int lmhead_verify_tree(const void* X, const uint8_t* q, const uint8_t* sf, const float* tensor_scale, int64_t M,
+                       int64_t N, int64_t K, const int32_t* drafts, const int32_t* parents, int32_t B, int32_t D,
+                       int32_t* argmax, int32_t* accept_len, int32_t* accept_node, float* max_logit, void* workspace,
+                       size_t workspace_bytes, nvfp4ws_stream_t stream) {
+  g_last_error[0] = 0;
+  if (D > 0 && !parents) return set_error(NVFP4WS_ERR_INVALID_ARG, "lmhead_verify_tree: parents is null");
+  const VerifyRule v{drafts, D > 0 ? parents : nullptr, B, D, argmax, accept_len, accept_node, max_logit};
+  return verify_impl(X, q, sf, tensor_scale, M, N, K, v, workspace, workspace_bytes, NVFP4WS_PATH_AUTO,
+                     (cudaStream_t)stream);
 }
 
 int lmhead_verify_argmax_accept(const void* X, const uint8_t* q, const uint8_t* sf, const float* tensor_scale,
@@ -308,7 +331,7 @@ int nvfp4_pass_init(nvfp4_pass* pass, const nvfp4_gemm_problem* problems, int32_
   std::memset(pass, 0, sizeof(nvfp4_pass));
   std::vector<MxHostProblem> hp;
   if (int e = to_host_problems(problems, count, M, verify != nullptr, &hp, "nvfp4_pass_init")) return e;
-  MxVerifySpec vs{};
+  VerifyRule vs{};
   if (verify) {
     if (verify->B < 1 || verify->D < 0)
       return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_pass_init: verify needs B >= 1 and D >= 0");
@@ -318,7 +341,8 @@ int nvfp4_pass_init(nvfp4_pass* pass, const nvfp4_gemm_problem* problems, int32_
     if (verify->D > 0 && !verify->drafts) return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_pass_init: drafts is null");
     if (!verify->argmax || !verify->accept_len)
       return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_pass_init: null verify output pointer");
-    vs = MxVerifySpec{verify->drafts, verify->B, verify->D, verify->argmax, verify->accept_len, verify->max_logit};
+    vs = VerifyRule{verify->drafts, verify->parents, verify->B, verify->D, verify->argmax, verify->accept_len,
+                    verify->accept_node, verify->max_logit};
   }
   if (!workspace) return set_error(NVFP4WS_ERR_WORKSPACE, "nvfp4_pass_init: workspace is null");
   if (!aligned16(workspace)) return set_error(NVFP4WS_ERR_MISALIGNED, "nvfp4_pass_init: workspace must be 16-byte aligned");
@@ -341,7 +365,9 @@ int nvfp4ws_check(nvfp4ws_stream_t stream) {
   if (v != 0) {
     unsigned int zero = 0;
     cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
-    return set_error(NVFP4WS_ERR_DEVICE_TIMEOUT, "a bounded device wait gave up (code 0x%x)", v);
+    if (v & kDevErrWaitTimeout)
+      return set_error(NVFP4WS_ERR_DEVICE_TIMEOUT, "a bounded device wait gave up (code 0x%x)", v);
+    return set_error(NVFP4WS_ERR_INVALID_ARG, "a draft tree had a parent outside [0, k-1] (code 0x%x)", v);
   }
   return NVFP4WS_OK;
 }

@@ -20,6 +20,7 @@ int check_launch(const char* what);
 // read and cleared by nvfp4ws_check().
 unsigned int* device_error_word();
 constexpr unsigned int kDevErrWaitTimeout = 1u;
+constexpr unsigned int kDevErrBadTree = 2u;       // a draft tree's parent outside [0, k-1]
 
 // ----------------------------------------------------------------------------
 // Loads

@@ -36,10 +36,23 @@ int launch_gemv(const GemvArgs& a, bool verify, bool regs_only, cudaStream_t s);
 int launch_pack(const float* W, long long N, long long K, uint8_t* q, uint8_t* sf, float* ts,
                 const float* ts_in, cudaStream_t s);
 
+// The verify's inputs and outputs: drafts [B, D]; parents [B, D] (node k >= 1 hangs
+// under parents[b, k-1]) or null for a chain; argmax [M], accept_len [B], and the
+// kept path's end node accept_node [B] and the winning logits max_logit [M] (both
+// optional, null to skip).
+struct VerifyRule {
+  const int32_t* drafts;
+  const int32_t* parents;
+  int B, D;
+  int32_t* argmax;
+  int32_t* accept_len;
+  int32_t* accept_node;
+  float* max_logit;
+};
+
 // Stage 2 of the verify: reduce per-CTA (max, index) partials to argmax[M], then
-// the accept length of every sequence.
-int launch_verify_stage2(const float* part_val, const int* part_idx, int nparts, int M,
-                         const int32_t* drafts, int B, int D, int32_t* argmax, int32_t* accept_len,
-                         float* max_logit, cudaStream_t s);
+// the accept length (and end node) of every sequence.
+int launch_verify_stage2(const float* part_val, const int* part_idx, int nparts, int M, const VerifyRule& v,
+                         cudaStream_t s);
 
 }  // namespace nvfp4ws

@@ -637,13 +637,12 @@ int launch_mma_gemm(const uint16_t* X, const uint8_t* q, const uint8_t* sf, cons
 }
 
 int launch_mma_verify(const uint16_t* X, const uint8_t* q, const uint8_t* sf, const float* ts, long long M,
-                      long long N, long long K, const int32_t* drafts, int B, int D, int32_t* argmax,
-                      int32_t* accept_len, float* max_logit, void* workspace, cudaStream_t s) {
+                      long long N, long long K, const VerifyRule& v, void* workspace, cudaStream_t s) {
   float* pv = nullptr;
   int* pi = nullptr;
   int nparts = 0;
   if (int e = launch_mma(X, q, sf, ts, M, N, K, nullptr, 0, workspace, true, &pv, &pi, &nparts, s)) return e;
-  return launch_verify_stage2(pv, pi, nparts, (int)M, drafts, B, D, argmax, accept_len, max_logit, s);
+  return launch_verify_stage2(pv, pi, nparts, (int)M, v, s);
 }
 
 }  // namespace nvfp4ws

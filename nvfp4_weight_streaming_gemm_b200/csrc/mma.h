@@ -5,6 +5,8 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "kernels.h"
+
 namespace nvfp4ws {
 
 bool mma_supported(long long M, long long K);
@@ -16,8 +18,7 @@ size_t mma_verify_workspace_bytes(long long M, long long N, long long K);
 int launch_mma_gemm(const uint16_t* X, const uint8_t* q, const uint8_t* sf, const float* ts, long long M, long long N,
                     long long K, void* Y, int y_dtype, void* workspace, size_t workspace_bytes, cudaStream_t s);
 int launch_mma_verify(const uint16_t* X, const uint8_t* q, const uint8_t* sf, const float* ts, long long M,
-                      long long N, long long K, const int32_t* drafts, int B, int D, int32_t* argmax,
-                      int32_t* accept_len, float* max_logit, void* workspace, cudaStream_t s);
+                      long long N, long long K, const VerifyRule& v, void* workspace, cudaStream_t s);
 
 // Block-scaled (kind::mxf4nvf4) path: activations as kMxf4Terms residual NVFP4 terms.
 constexpr int kMxf4Terms = 5;
@@ -26,8 +27,7 @@ size_t mxf4_workspace_bytes(long long M, long long N, long long K);
 int launch_mxf4_gemm(const uint16_t* X, const uint8_t* q, const uint8_t* sf, const float* ts, long long M,
                      long long N, long long K, void* Y, int y_dtype, void* workspace, cudaStream_t s);
 int launch_mxf4_verify(const uint16_t* X, const uint8_t* q, const uint8_t* sf, const float* ts, long long M,
-                       long long N, long long K, const int32_t* drafts, int B, int D, int32_t* argmax,
-                       int32_t* accept_len, float* max_logit, void* workspace, cudaStream_t s);
+                       long long N, long long K, const VerifyRule& v, void* workspace, cudaStream_t s);
 
 // A list of GEMMs sharing M, run by one persistent launch (a weight pass).
 struct MxHostProblem {
@@ -39,17 +39,10 @@ struct MxHostProblem {
   void* Y;
   int y_bf16, verify;
 };
-struct MxVerifySpec {
-  const int32_t* drafts;
-  int B, D;
-  int32_t* argmax;
-  int32_t* accept_len;
-  float* max_logit;
-};
 // Host state of an initialised pass lives in a caller-owned buffer of this many bytes.
 constexpr size_t kMxPassStateBytes = 256;
 size_t mxf4_pass_workspace_bytes(const MxHostProblem* hp, int n, long long M);
-int mxf4_pass_init(void* state, const MxHostProblem* hp, int n, long long M, const MxVerifySpec* vs, void* workspace,
+int mxf4_pass_init(void* state, const MxHostProblem* hp, int n, long long M, const VerifyRule* vs, void* workspace,
                    size_t workspace_bytes);
 int mxf4_pass_run(const void* state, cudaStream_t s);
 

@@ -1240,12 +1240,11 @@ int launch_mxf4_gemm(const uint16_t* X, const uint8_t* q, const uint8_t* sf, con
 }
 
 int launch_mxf4_verify(const uint16_t* X, const uint8_t* q, const uint8_t* sf, const float* ts, long long M,
-                       long long N, long long K, const int32_t* drafts, int B, int D, int32_t* argmax,
-                       int32_t* accept_len, float* max_logit, void* workspace, cudaStream_t s) {
+                       long long N, long long K, const VerifyRule& v, void* workspace, cudaStream_t s) {
   MxHostProblem h{X, q, sf, ts, N, K, nullptr, 0, 1};
   Problem P;
   if (int e = launch_single(h, M, workspace, s, &P)) return e;
-  return launch_verify_stage2(P.part_val, P.part_idx, P.tiles, (int)M, drafts, B, D, argmax, accept_len, max_logit, s);
+  return launch_verify_stage2(P.part_val, P.part_idx, P.tiles, (int)M, v, s);
 }
 
 // ------------------------------------------------------------------ multi-problem passes
@@ -1262,7 +1261,7 @@ struct MxPassState {
   PassTables tb;
   float* pv;
   int* pi;
-  MxVerifySpec vs;
+  VerifyRule vs;
 };
 static_assert(sizeof(MxPassState) <= kMxPassStateBytes, "pass state does not fit the caller's handle");
 constexpr uint32_t kPassMagic = 0x4e565053u;
@@ -1271,7 +1270,7 @@ size_t mxf4_pass_workspace_bytes(const MxHostProblem* hp, int n, long long M) {
   return mx_layout(hp, n, M, true).total;
 }
 
-int mxf4_pass_init(void* state, const MxHostProblem* hp, int n, long long M, const MxVerifySpec* vs, void* workspace,
+int mxf4_pass_init(void* state, const MxHostProblem* hp, int n, long long M, const VerifyRule* vs, void* workspace,
                    size_t workspace_bytes) {
   MxPassState* P = static_cast<MxPassState*>(state);
   std::memset(static_cast<void*>(P), 0, sizeof(MxPassState));
@@ -1351,8 +1350,7 @@ int mxf4_pass_run(const void* state, cudaStream_t s) {
                           P->max_k, P->ws, s))
     return e;
   if (!P->verify) return NVFP4WS_OK;
-  return launch_verify_stage2(P->pv, P->pi, P->vtiles, (int)P->M, P->vs.drafts, P->vs.B, P->vs.D, P->vs.argmax,
-                              P->vs.accept_len, P->vs.max_logit, s);
+  return launch_verify_stage2(P->pv, P->pi, P->vtiles, (int)P->M, P->vs, s);
 }
 
 }  // namespace nvfp4ws
