@@ -187,7 +187,8 @@ class Pass:
     192 GEMMs with the lm_head verify as its last problem), and, for comparison, the
     chained per-GEMM launch sequence, each captured in a CUDA graph."""
 
-    def __init__(self, nv, torch, dev, stack, lm, M: int, rank: int, chain: bool, tree: bool = False):
+    def __init__(self, nv, torch, dev, stack, lm, M: int, rank: int, chain: bool, tree: bool = False,
+                 binv: bool = False):
         self.M = M
         self.tree = tree
         self.torch = torch
@@ -217,7 +218,8 @@ class Pass:
             self.parents = torch.from_numpy(S.random_tree(self.B, self.D, seed=S.LMHEAD_L_SEED + M)).to(dev)
             self.node = torch.empty(self.B, dtype=torch.int32, device=dev)
             verify = verify + (self.parents, self.node)
-        self.wp = nv.WeightPass(problems, M, verify=verify)
+        self.binv = binv
+        self.wp = nv.WeightPass(problems, M, verify=verify, batch_invariant=binv)
         if chain:
             wsb = max(nv.gemm_workspace_bytes(M, N, K) for (_, K, N, _, _, _) in stack)
             self.gws = torch.zeros(max(wsb, 16), dtype=torch.uint8, device=dev)
@@ -346,7 +348,8 @@ def run_ours(args, rank, world, local_rank):
     M_list = [int(m) for m in args.ms.split(",")]
     stack, lm = build_pass(nv, torch, dev, M_list, rank, args.layers)
     head = 17 if 17 in M_list else M_list[0]
-    passes = {M: Pass(nv, torch, dev, stack, lm, M, rank, chain=not args.no_chain, tree=args.tree) for M in M_list}
+    passes = {M: Pass(nv, torch, dev, stack, lm, M, rank, chain=not args.no_chain, tree=args.tree, binv=args.binv)
+              for M in M_list}
     for p in passes.values():
         p.capture()
         for _ in range(args.warmup):
@@ -382,7 +385,7 @@ def run_ours(args, rank, world, local_rank):
             "ms_min": float(per.min()),
             "ms_max": float(per.max()),
             "launches_per_pass": p.launches_pass,
-            "B": p.B, "D": p.D, "verify": "tree" if p.tree else "chain",
+            "B": p.B, "D": p.D, "verify": "tree" if p.tree else "chain", "batch_invariant": p.binv,
         }
         if p.chain:
             # the same work as 193 chained launches: each GEMM's activations are read only
@@ -567,6 +570,7 @@ def main():
                          "when the kernel sources still match it)")
     ap.add_argument("--tree", action="store_true",
                     help="verify draft trees of D nodes per sequence (seeded random parents) instead of chains")
+    ap.add_argument("--binv", action="store_true", help="batch-invariant passes (same row bits for every M)")
     ap.add_argument("--sweep", action="store_true", help="time one matrix shape per M and path (no pass)")
     ap.add_argument("--shape", default="gate_up", help="sweep shape: gate_up, down, qkv or lm_head")
     ap.add_argument("--paths", default="auto,gemv,mma")

@@ -307,6 +307,27 @@ size_t nvfp4_pass_workspace_bytes(const nvfp4_gemm_problem* problems, int32_t co
                                   int32_t verify_last);
 int nvfp4_pass_init(nvfp4_pass* pass, const nvfp4_gemm_problem* problems, int32_t count, int64_t M,
                     const nvfp4_verify_spec* verify, void* workspace, size_t workspace_bytes);
+
+/*
+ * Batch-invariant passes.
+ *
+ * Passage: "TandemLLM", "The parts" (the projection kernels give a row the same bits
+ * whatever other rows share the batch) and its feature list ("--probe-binv (batch
+ * invariance)"). With NVFP4WS_PASS_BATCH_INVARIANT a pass gives every row of Y (and of
+ * the verify's logits) the same bits for any M in [1, 70] with the same problem list:
+ * the work is split into the same units at the same points, summed in the same order,
+ * whatever M is. (A row's activation terms depend on that row alone.) It costs
+ * bandwidth at small M, where the default plan uses larger units.
+ *
+ * nvfp4_pass_workspace_bytes_ex / nvfp4_pass_init_ex -- as the calls above, with
+ *   `flags` (0 or NVFP4WS_PASS_BATCH_INVARIANT; other bits are INVALID_ARG, and the
+ *   workspace query returns 0). Pass the same flags to both.
+ */
+#define NVFP4WS_PASS_BATCH_INVARIANT 1u
+size_t nvfp4_pass_workspace_bytes_ex(const nvfp4_gemm_problem* problems, int32_t count, int64_t M,
+                                     int32_t verify_last, uint32_t flags);
+int nvfp4_pass_init_ex(nvfp4_pass* pass, const nvfp4_gemm_problem* problems, int32_t count, int64_t M,
+                       const nvfp4_verify_spec* verify, uint32_t flags, void* workspace, size_t workspace_bytes);
 int nvfp4_pass_run(const nvfp4_pass* pass, nvfp4ws_stream_t stream);
 
 /*

@@ -22,6 +22,7 @@ import torch
 from . import _lib
 
 PATHS = {"auto": 0, "gemv": 1, "mma": 2, "gemv_regs": 3, "mma_f16": 4}
+PASS_BATCH_INVARIANT = 1
 STATUS_OK = 0
 
 
@@ -187,11 +188,14 @@ class WeightPass:
     and Y fp32 or bf16 [M, N]. With ``verify=(drafts, argmax, accept_len, max_logit)``
     the last problem is the lm_head: its Y may be None, and each run ends with the
     argmax over its rows and the accept lengths. ``verify`` may add ``(parents,
-    accept_node)`` for a tree verify (``accept_node`` may be None). Every tensor is
-    referenced by address: keep them alive and refill X in place between runs.
+    accept_node)`` for a tree verify (``accept_node`` may be None). With
+    ``batch_invariant`` every row gets the same bits for any M (``nvfp4_pass_init_ex``).
+    Every tensor is referenced by address: keep them alive and refill X in place
+    between runs.
     """
 
-    def __init__(self, problems, M: int, verify=None, workspace: torch.Tensor | None = None):
+    def __init__(self, problems, M: int, verify=None, workspace: torch.Tensor | None = None,
+                 batch_invariant: bool = False):
         L = _lib
         n = len(problems)
         self._keep = []
@@ -227,16 +231,17 @@ class WeightPass:
             vs = L.VerifySpec(_ptr(drafts) if drafts.numel() else None, B, D, _ptr(amax), _ptr(acc), _ptr(vmax),
                               _ptr(parents) if parents is not None and parents.numel() else None, _ptr(node))
             self._keep.extend([drafts, amax, acc, vmax, parents, node])
-        nbytes = int(lib().nvfp4_pass_workspace_bytes(arr, n, M, 1 if verify is not None else 0))
+        flags = PASS_BATCH_INVARIANT if batch_invariant else 0
+        nbytes = int(lib().nvfp4_pass_workspace_bytes_ex(arr, n, M, 1 if verify is not None else 0, flags))
         if nbytes == 0:
             raise NVFP4WSError(1, "nvfp4_pass_workspace_bytes")
         dev = problems[0][0].device
         self.workspace = _workspace(nbytes, dev, workspace)
         self.workspace_bytes = nbytes
         self.state = L.PassState()
-        _check(lib().nvfp4_pass_init(ctypes.byref(self.state), arr, n, M,
-                                     ctypes.byref(vs) if vs is not None else None, _ptr(self.workspace), nbytes),
-               "nvfp4_pass_init")
+        _check(lib().nvfp4_pass_init_ex(ctypes.byref(self.state), arr, n, M,
+                                        ctypes.byref(vs) if vs is not None else None, flags,
+                                        _ptr(self.workspace), nbytes), "nvfp4_pass_init")
         self.M = M
         self.count = n
 

@@ -57,6 +57,9 @@ SIGNATURES = {
     "nvfp4_pass_init": (ctypes.c_int, [ctypes.POINTER(PassState), ctypes.POINTER(GemmProblem), c_i32, c_i64,
                                        ctypes.POINTER(VerifySpec), c_p, c_sz]),
     "nvfp4_pass_run": (ctypes.c_int, [ctypes.POINTER(PassState), c_p]),
+    "nvfp4_pass_workspace_bytes_ex": (c_sz, [ctypes.POINTER(GemmProblem), c_i32, c_i64, c_i32, ctypes.c_uint32]),
+    "nvfp4_pass_init_ex": (ctypes.c_int, [ctypes.POINTER(PassState), ctypes.POINTER(GemmProblem), c_i32, c_i64,
+                                          ctypes.POINTER(VerifySpec), ctypes.c_uint32, c_p, c_sz]),
 }
 
 _lib = None

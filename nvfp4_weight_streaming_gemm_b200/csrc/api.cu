@@ -317,15 +317,28 @@ static int to_host_problems(const nvfp4_gemm_problem* problems, int32_t count, i
   return NVFP4WS_OK;
 }
 
-size_t nvfp4_pass_workspace_bytes(const nvfp4_gemm_problem* problems, int32_t count, int64_t M, int32_t verify_last) {
+size_t nvfp4_pass_workspace_bytes_ex(const nvfp4_gemm_problem* problems, int32_t count, int64_t M,
+                                     int32_t verify_last, uint32_t flags) {
   std::vector<MxHostProblem> hp;
+  if ((flags & ~(uint32_t)NVFP4WS_PASS_BATCH_INVARIANT) != 0) return 0;
   if (to_host_problems(problems, count, M, verify_last, &hp, "nvfp4_pass_workspace_bytes") != NVFP4WS_OK) return 0;
-  return mxf4_pass_workspace_bytes(hp.data(), count, M);
+  return mxf4_pass_workspace_bytes(hp.data(), count, M, (flags & NVFP4WS_PASS_BATCH_INVARIANT) != 0);
+}
+
+size_t nvfp4_pass_workspace_bytes(const nvfp4_gemm_problem* problems, int32_t count, int64_t M, int32_t verify_last) {
+  return nvfp4_pass_workspace_bytes_ex(problems, count, M, verify_last, 0u);
 }
 
 int nvfp4_pass_init(nvfp4_pass* pass, const nvfp4_gemm_problem* problems, int32_t count, int64_t M,
                     const nvfp4_verify_spec* verify, void* workspace, size_t workspace_bytes) {
+  return nvfp4_pass_init_ex(pass, problems, count, M, verify, 0u, workspace, workspace_bytes);
+}
+
+int nvfp4_pass_init_ex(nvfp4_pass* pass, const nvfp4_gemm_problem* problems, int32_t count, int64_t M,
+                       const nvfp4_verify_spec* verify, uint32_t flags, void* workspace, size_t workspace_bytes) {
   g_last_error[0] = 0;
+  if ((flags & ~(uint32_t)NVFP4WS_PASS_BATCH_INVARIANT) != 0)
+    return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_pass_init: unknown flags 0x%x", flags);
   static_assert(sizeof(nvfp4_pass) >= kMxPassStateBytes, "nvfp4_pass is too small for the pass state");
   if (!pass) return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_pass_init: pass is null");
   std::memset(pass, 0, sizeof(nvfp4_pass));
@@ -346,7 +359,8 @@ int nvfp4_pass_init(nvfp4_pass* pass, const nvfp4_gemm_problem* problems, int32_
   }
   if (!workspace) return set_error(NVFP4WS_ERR_WORKSPACE, "nvfp4_pass_init: workspace is null");
   if (!aligned16(workspace)) return set_error(NVFP4WS_ERR_MISALIGNED, "nvfp4_pass_init: workspace must be 16-byte aligned");
-  return mxf4_pass_init(pass->opaque, hp.data(), count, M, verify ? &vs : nullptr, workspace, workspace_bytes);
+  return mxf4_pass_init(pass->opaque, hp.data(), count, M, verify ? &vs : nullptr,
+                        (flags & NVFP4WS_PASS_BATCH_INVARIANT) != 0, workspace, workspace_bytes);
 }
 
 int nvfp4_pass_run(const nvfp4_pass* pass, nvfp4ws_stream_t stream) {

@@ -41,9 +41,10 @@ struct MxHostProblem {
 };
 // Host state of an initialised pass lives in a caller-owned buffer of this many bytes.
 constexpr size_t kMxPassStateBytes = 256;
-size_t mxf4_pass_workspace_bytes(const MxHostProblem* hp, int n, long long M);
-int mxf4_pass_init(void* state, const MxHostProblem* hp, int n, long long M, const VerifyRule* vs, void* workspace,
-                   size_t workspace_bytes);
+// binv: a batch-invariant pass (one unit shape for every M).
+size_t mxf4_pass_workspace_bytes(const MxHostProblem* hp, int n, long long M, bool binv);
+int mxf4_pass_init(void* state, const MxHostProblem* hp, int n, long long M, const VerifyRule* vs, bool binv,
+                   void* workspace, size_t workspace_bytes);
 int mxf4_pass_run(const void* state, cudaStream_t s);
 
 }  // namespace nvfp4ws

@@ -999,10 +999,13 @@ static MxPlan mx_plan_ku(long long M, int ku, int tpu) {
 // (M <= 12); past that, two tiles sharing one chunk's activation images carry half the
 // image bytes per weight byte, so more weight bytes fit in flight (M=17: 4 stages instead
 // of 3). Either needs one B tile and a double-buffered accumulator.
-static MxPlan mx_plan(long long M, bool k512) {
+// Batch-invariant passes (binv) use one unit shape for every M, so that a row's units,
+// split points and summation order do not depend on how many rows share the pass.
+static MxPlan mx_plan(long long M, bool k512, bool binv = false) {
   auto ok = [](const MxPlan& x, int min_stages) {
     return x.g.nbt == 1 && x.acc_bufs == 2 && x.stages >= min_stages;
   };
+  if (binv) return mx_plan_ku(M, 1, 1);
   if (k512) {
     const MxPlan two = mx_plan_ku(M, 2, 1);
     if (ok(two, 4)) return two;
@@ -1051,8 +1054,10 @@ static bool all_k512(const MxHostProblem* hp, int n) {
 }
 
 // with_desc: a pass keeps its descriptors and wave tables in the workspace.
-static WsLayout mx_layout(const MxHostProblem* hp, int n, long long M, bool with_desc) {
-  const MxPlan pl = mx_plan(M, all_k512(hp, n));
+static WsLayout mx_layout(const MxHostProblem* hp, int n, long long M, bool with_desc, bool binv = false) {
+  const MxPlan pl = mx_plan(M, all_k512(hp, n), binv);
+  // waves are cut by image bytes; a batch-invariant pass cuts them as the largest M would
+  const uint32_t wave_img_stride = binv ? mx_plan_ku(kMaxB / kMxf4Terms, 1, 1).g.img_stride : pl.g.img_stride;
   const int ku = pl.g.ku, tpu = pl.g.tpu;
   WsLayout L;
   L.units = 0;
@@ -1065,7 +1070,7 @@ static WsLayout mx_layout(const MxHostProblem* hp, int n, long long M, bool with
   size_t img = 0;
   unsigned long long wu = 0;
   for (int i = 0; i < n; ++i) {
-    const size_t pimg = (size_t)(hp[i].K / kKC) * pl.g.img_stride;
+    const size_t pimg = (size_t)(hp[i].K / kKC) * wave_img_stride;
     if (i > 0 && wu >= (unsigned long long)L.grid && img + pimg > kWaveImageBudget) {
       L.wave_first.push_back(i);
       img = 0;
@@ -1252,7 +1257,7 @@ int launch_mxf4_verify(const uint16_t* X, const uint8_t* q, const uint8_t* sf, c
 // Host state of a pass: plain data in caller-owned memory (no allocation).
 struct MxPassState {
   uint32_t magic;
-  int nprob, grid, verify, vtiles, k512;
+  int nprob, grid, verify, vtiles, k512, binv;
   long long M, max_k;
   unsigned long long units;
   size_t off_part;
@@ -1266,16 +1271,16 @@ struct MxPassState {
 static_assert(sizeof(MxPassState) <= kMxPassStateBytes, "pass state does not fit the caller's handle");
 constexpr uint32_t kPassMagic = 0x4e565053u;
 
-size_t mxf4_pass_workspace_bytes(const MxHostProblem* hp, int n, long long M) {
-  return mx_layout(hp, n, M, true).total;
+size_t mxf4_pass_workspace_bytes(const MxHostProblem* hp, int n, long long M, bool binv) {
+  return mx_layout(hp, n, M, true, binv).total;
 }
 
-int mxf4_pass_init(void* state, const MxHostProblem* hp, int n, long long M, const VerifyRule* vs, void* workspace,
-                   size_t workspace_bytes) {
+int mxf4_pass_init(void* state, const MxHostProblem* hp, int n, long long M, const VerifyRule* vs, bool binv,
+                   void* workspace, size_t workspace_bytes) {
   MxPassState* P = static_cast<MxPassState*>(state);
   std::memset(static_cast<void*>(P), 0, sizeof(MxPassState));
-  const WsLayout L = mx_layout(hp, n, M, true);
-  const MxPlan plan = mx_plan(M, all_k512(hp, n));
+  const WsLayout L = mx_layout(hp, n, M, true, binv);
+  const MxPlan plan = mx_plan(M, all_k512(hp, n), binv);
   const int ku = plan.g.ku, tpu = plan.g.tpu;
   if (workspace_bytes < L.total)
     return set_error(NVFP4WS_ERR_WORKSPACE, "nvfp4_pass_init: workspace %zu bytes < required %zu", workspace_bytes,
@@ -1322,6 +1327,7 @@ int mxf4_pass_init(void* state, const MxHostProblem* hp, int n, long long M, con
     return check_launch("nvfp4_pass_init: descriptor upload");
   P->nprob = n;
   P->k512 = all_k512(hp, n) ? 1 : 0;
+  P->binv = binv ? 1 : 0;
   P->grid = L.grid;
   P->units = L.units;
   P->off_part = L.off_part;
@@ -1345,7 +1351,7 @@ int mxf4_pass_run(const void* state, cudaStream_t s) {
   const MxPassState* P = static_cast<const MxPassState*>(state);
   if (P->magic != kPassMagic) return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_pass_run: pass not initialised");
   static const Problem kNoProblem{};   // the kernels' by-value problem slot, unused by a pass
-  const MxPlan pl = mx_plan(P->M, P->k512 != 0);
+  const MxPlan pl = mx_plan(P->M, P->k512 != 0, P->binv != 0);
   if (int e = launch_pass(kNoProblem, P->probs_dev, P->tb, P->nprob, pl, P->grid, P->units, P->off_part,
                           P->max_k, P->ws, s))
     return e;
