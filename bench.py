@@ -332,6 +332,20 @@ def cpu_baseline(seconds: float = 12.0):
                       f"host has {cores} cores, BLAS threads {blas}"}
 
 
+def max_over_ranks(dist, torch, value: float, dev) -> float:
+    """The largest of each rank's device-timed value: the slowest replica sets the step
+    time of the whole job. ``dist`` is None on one GPU."""
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_gbs(world: int, nbytes: int, ms: float) -> float:
+    """Whole-job throughput of ``world`` replicas that each stream ``nbytes`` per step."""
+    return world * nbytes / (ms * 1e-3) / 1e9
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import nvfp4_weight_streaming_gemm_b200 as nv
@@ -371,14 +385,11 @@ def run_ours(args, rank, world, local_rank):
         total_ms, per = p.run_timed(args.steps)
         if sampler:
             clocks = sampler.stop()
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        if dist:
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+        total_ms = max_over_ranks(dist, torch, total_ms, dev)
         ms = total_ms / args.steps
         res = {
             "ms_per_pass": ms,
-            "weight_gbs": world * wbytes / (ms * 1e-3) / 1e9,
+            "weight_gbs": job_gbs(world, wbytes, ms),
             "pct_of_8tbs": 100.0 * wbytes / (ms * 1e-3) / 8e12,
             "passes_per_s": world * 1e3 / ms,
             "alg_gbs": pass_alg_bytes(M, args.layers) / (ms * 1e-3) / 1e9,
@@ -393,11 +404,9 @@ def run_ours(args, rank, world, local_rank):
             if dist:
                 dist.barrier()
             chain_total, _ = p.run_timed(max(3, args.steps // 4), p.g_chain)
-            t = torch.tensor([chain_total / max(3, args.steps // 4)], dtype=torch.float64, device=dev)
-            if dist:
-                dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            res["chained_ms_per_pass"] = float(t.item())
-            res["chained_weight_gbs"] = world * wbytes / (float(t.item()) * 1e-3) / 1e9
+            chain_ms = max_over_ranks(dist, torch, chain_total / max(3, args.steps // 4), dev)
+            res["chained_ms_per_pass"] = chain_ms
+            res["chained_weight_gbs"] = job_gbs(world, wbytes, chain_ms)
         results[M] = res
 
     # end to end through the public API with host buffers (headline M)
@@ -410,11 +419,7 @@ def run_ours(args, rank, world, local_rank):
         p.run_e2e(1, x_host, out_host)
     if dist:
         dist.barrier()
-    e2e_ms = p.run_e2e(args.steps, x_host, out_host)
-    t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if dist:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_ms = float(t.item()) / args.steps
+    e2e_ms = max_over_ranks(dist, torch, p.run_e2e(args.steps, x_host, out_host), dev) / args.steps
     h2d = p.x_all.numel() * 2
     d2h = p.M * 4 + p.B * 4
 
@@ -453,7 +458,7 @@ def run_ours(args, rank, world, local_rank):
                      "frac": r["alg_gbs"] / peak, "peak_kind": peak_kind,
                      "traffic": args.traffic if args.traffic is not None else measured_traffic(head, args.layers),
                      "algorithmic_bytes_per_launch": pass_alg_bytes(head, args.layers)},
-        "e2e": {"value": world * wbytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": e2e_ms,
+        "e2e": {"value": job_gbs(world, wbytes, e2e_ms), "unit": "GB/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": r["launches_per_pass"] * args.steps,
         "clocks": clocks,
