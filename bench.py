@@ -527,6 +527,65 @@ def run_sweep(args):
 
 # ----------------------------------------------------------------------------- reference arm
 
+def run_w4a4(args):
+    """The W4A4 weight pass at prefill-sized M (SURVEY-style "next" row): the 192 GEMMs of
+    the 27B stack with their activations quantised to NVFP4, one persistent launch, timed
+    as a CUDA graph. One JSON line per M with the weight GB/s against the HBM roofline and
+    the tensor TFLOP/s against the fp4 peak (measured bf16 x 4, the nominal fp4/bf16
+    ratio)."""
+    import torch
+    import nvfp4_weight_streaming_gemm_b200 as nv
+    from nvfp4_weight_streaming_gemm_b200 import build as nvbuild
+    nvbuild.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    M_list = [int(m) for m in args.ms.split(",")]
+    stack, _ = build_pass(nv, torch, dev, M_list, 0, args.layers)
+    wbytes = stack_weight_bytes(args.layers)
+    flop_per_m = 2.0 * sum(N * K for (_, K, N, _, _, _) in stack)
+    hbm, hbm_kind = measured_peaks()
+    bf16, pk = 1590.0, os.path.join(ROOT, "MEASURED_PEAKS.json")     # the recipe's fallback when absent
+    if os.path.exists(pk):
+        with open(pk) as f:
+            bf16 = float(json.load(f).get("bf16_tflops", bf16))
+    fp4_peak = 4.0 * bf16
+    for M in M_list:
+        g = torch.Generator(device=dev)
+        g.manual_seed(11 + M)
+        probs = [(torch.randn(M, K, generator=g, device=dev).to(torch.bfloat16), q, sf, ts,
+                  torch.empty((M, N), dtype=torch.bfloat16, device=dev)) for (_, K, N, q, sf, ts) in stack]
+        wp = nv.WeightPass(probs, M, w4a4=True)
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            wp.run(s)
+        torch.cuda.current_stream().wait_stream(s)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            wp.run()
+        for _ in range(args.warmup):
+            graph.replay()
+        torch.cuda.synchronize()
+        st = torch.cuda.current_stream()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+        ev[0].record(st)
+        for k in range(args.steps):
+            graph.replay()
+            ev[k + 1].record(st)
+        torch.cuda.synchronize()
+        per = np.array([ev[k].elapsed_time(ev[k + 1]) for k in range(args.steps)])
+        ms = ev[0].elapsed_time(ev[-1]) / args.steps
+        tflops = flop_per_m * M / (ms * 1e-3) / 1e12
+        print(json.dumps({
+            "metric": "W4A4 27B weight pass (NVFP4 activations, prefill-sized M)", "M": M, "layers": args.layers,
+            "ms_per_pass": ms, "ms_min": float(per.min()), "weight_gbs": wbytes / (ms * 1e-3) / 1e9,
+            "hbm_frac": wbytes / (ms * 1e-3) / 1e9 / hbm, "hbm_peak_kind": hbm_kind,
+            "tflops": tflops, "fp4_peak_tflops": fp4_peak, "tensor_frac": tflops / fp4_peak,
+            "y_dtype": "bf16", "steps": args.steps, "warmup": args.warmup}), flush=True)
+        del graph, wp, probs
+        torch.cuda.synchronize()
+
+
 def run_reference(args, rank, world):
     """The CPU oracle timed as it stands: each step dequantises and multiplies one qkv
     matrix (5120->10240) in float64 at M=17. That is a bounded sample of the pass, in
@@ -576,6 +635,8 @@ def main():
     ap.add_argument("--tree", action="store_true",
                     help="verify draft trees of D nodes per sequence (seeded random parents) instead of chains")
     ap.add_argument("--binv", action="store_true", help="batch-invariant passes (same row bits for every M)")
+    ap.add_argument("--w4a4", action="store_true",
+                    help="time W4A4 passes (NVFP4 activations) over the stack at the --ms values, e.g. 128,256")
     ap.add_argument("--sweep", action="store_true", help="time one matrix shape per M and path (no pass)")
     ap.add_argument("--shape", default="gate_up", help="sweep shape: gate_up, down, qkv or lm_head")
     ap.add_argument("--paths", default="auto,gemv,mma")
@@ -588,6 +649,8 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.sweep:
         run_sweep(args)
+    elif args.w4a4:
+        run_w4a4(args)
     elif args.impl == "reference":
         run_reference(args, rank, world)
     else:

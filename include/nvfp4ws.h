@@ -155,6 +155,30 @@ int nvfp4_gemm_skinny_path(const void* X, const uint8_t* q, const uint8_t* sf, c
                            int64_t M, int64_t N, int64_t K, void* Y, int y_dtype,
                            void* workspace, size_t workspace_bytes, int path, nvfp4ws_stream_t stream);
 
+/*
+ * nvfp4_gemm_w4a4 -- the W4A4 product for prefill-sized M: X is quantised to NVFP4 too,
+ * and both operands go through the block-scaled tensor cores.
+ *
+ * Passages: "Qwen3.8 on DGX Spark (GB10)", introduction (NVFP4 on the block-scaled
+ * tensor cores) and "TandemLLM", "The parts" (4-bit projections). The pages give no
+ * activation recipe; this library applies the weights' two-level NVFP4 scheme to each
+ * row of X, with the row's amax in place of the tensor's, every decision in fp32:
+ *   g[m]   = fp32(amax_k |x[m,k]| / 2688)
+ *   S      = E4M3_rne_satfinite(fp32(amax_block * fp32(1 / fp32(6 g[m]))))   per 16 elements
+ *   c      = E2M1_rne_satfinite(fp32(x / fp32(S g[m])))                     (0 where S g = 0)
+ *   Y[m,n] = sum_k (e2m1(c)·S·g[m])[m,k] · dequant(W)[n,k], accumulated in fp32.
+ * This is not the exact bf16 product nvfp4_gemm_skinny computes: each activation
+ * carries up to half an E2M1 step of quantisation error.
+ *
+ * Arguments as nvfp4_gemm_skinny; 1 <= M <= NVFP4WS_MAX_M; K a multiple of 256 in
+ * [256, 32768]; workspace of at least nvfp4_gemm_w4a4_workspace_bytes(M, N, K) bytes,
+ * zero-filled before its first use.
+ */
+size_t nvfp4_gemm_w4a4_workspace_bytes(int64_t M, int64_t N, int64_t K);
+int nvfp4_gemm_w4a4(const void* X, const uint8_t* q, const uint8_t* sf, const float* tensor_scale,
+                    int64_t M, int64_t N, int64_t K, void* Y, int y_dtype,
+                    void* workspace, size_t workspace_bytes, nvfp4ws_stream_t stream);
+
 /* Workspace needed by lmhead_verify_argmax_accept for this shape. */
 size_t lmhead_verify_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
@@ -320,10 +344,13 @@ int nvfp4_pass_init(nvfp4_pass* pass, const nvfp4_gemm_problem* problems, int32_
  * bandwidth at small M, where the default plan uses larger units.
  *
  * nvfp4_pass_workspace_bytes_ex / nvfp4_pass_init_ex -- as the calls above, with
- *   `flags` (0 or NVFP4WS_PASS_BATCH_INVARIANT; other bits are INVALID_ARG, and the
- *   workspace query returns 0). Pass the same flags to both.
+ *   `flags`, an OR of NVFP4WS_PASS_BATCH_INVARIANT and NVFP4WS_PASS_W4A4 (other bits
+ *   are INVALID_ARG, and the workspace query returns 0). Pass the same flags to both.
  */
 #define NVFP4WS_PASS_BATCH_INVARIANT 1u
+/* A W4A4 pass: every problem as nvfp4_gemm_w4a4 computes it (M up to NVFP4WS_MAX_M, no
+ * verify problem). */
+#define NVFP4WS_PASS_W4A4 2u
 size_t nvfp4_pass_workspace_bytes_ex(const nvfp4_gemm_problem* problems, int32_t count, int64_t M,
                                      int32_t verify_last, uint32_t flags);
 int nvfp4_pass_init_ex(nvfp4_pass* pass, const nvfp4_gemm_problem* problems, int32_t count, int64_t M,

@@ -23,6 +23,7 @@ from . import _lib
 
 PATHS = {"auto": 0, "gemv": 1, "mma": 2, "gemv_regs": 3, "mma_f16": 4}
 PASS_BATCH_INVARIANT = 1
+PASS_W4A4 = 2
 STATUS_OK = 0
 
 
@@ -176,6 +177,22 @@ def verify_tree(X: torch.Tensor, q: torch.Tensor, sf: torch.Tensor, ts: torch.Te
     return amax, acc, node, vmax
 
 
+def gemm_w4a4(X: torch.Tensor, q: torch.Tensor, sf: torch.Tensor, ts: torch.Tensor, out: torch.Tensor | None = None,
+              y_dtype=torch.float32, workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """W4A4 product (``nvfp4_gemm_w4a4``): X bf16 [M, K] is quantised to NVFP4 per row, then
+    multiplied by the packed weight on the block-scaled tensor cores. Returns Y [M, N]."""
+    _need_cuda(X, "X", torch.bfloat16)
+    M, K = X.shape
+    N = q.shape[0]
+    Y = out if out is not None else torch.empty((M, N), dtype=y_dtype, device=X.device)
+    yd = {torch.float32: 0, torch.bfloat16: 1}[Y.dtype]
+    ws = _workspace(int(lib().nvfp4_gemm_w4a4_workspace_bytes(M, N, K)), X.device, workspace)
+    nbytes = 0 if ws is None else ws.numel()
+    _check(lib().nvfp4_gemm_w4a4(_ptr(X), _ptr(q), _ptr(sf), _ptr(ts), M, N, K, _ptr(Y), yd, _ptr(ws), nbytes,
+                                 _stream(stream)), "nvfp4_gemm_w4a4")
+    return Y
+
+
 def check(stream=None):
     """Synchronise and report a device-side bounded-wait failure, if any."""
     _check(lib().nvfp4ws_check(_stream(stream)), "nvfp4ws_check")
@@ -189,13 +206,14 @@ class WeightPass:
     the last problem is the lm_head: its Y may be None, and each run ends with the
     argmax over its rows and the accept lengths. ``verify`` may add ``(parents,
     accept_node)`` for a tree verify (``accept_node`` may be None). With
-    ``batch_invariant`` every row gets the same bits for any M (``nvfp4_pass_init_ex``).
+    ``batch_invariant`` every row gets the same bits for any M; with ``w4a4`` every
+    problem is the W4A4 product of :func:`gemm_w4a4` (no verify; ``nvfp4_pass_init_ex``).
     Every tensor is referenced by address: keep them alive and refill X in place
     between runs.
     """
 
     def __init__(self, problems, M: int, verify=None, workspace: torch.Tensor | None = None,
-                 batch_invariant: bool = False):
+                 batch_invariant: bool = False, w4a4: bool = False):
         L = _lib
         n = len(problems)
         self._keep = []
@@ -231,7 +249,7 @@ class WeightPass:
             vs = L.VerifySpec(_ptr(drafts) if drafts.numel() else None, B, D, _ptr(amax), _ptr(acc), _ptr(vmax),
                               _ptr(parents) if parents is not None and parents.numel() else None, _ptr(node))
             self._keep.extend([drafts, amax, acc, vmax, parents, node])
-        flags = PASS_BATCH_INVARIANT if batch_invariant else 0
+        flags = (PASS_BATCH_INVARIANT if batch_invariant else 0) | (PASS_W4A4 if w4a4 else 0)
         nbytes = int(lib().nvfp4_pass_workspace_bytes_ex(arr, n, M, 1 if verify is not None else 0, flags))
         if nbytes == 0:
             raise NVFP4WSError(1, "nvfp4_pass_workspace_bytes")

@@ -50,6 +50,8 @@ SIGNATURES = {
                                                         c_p, c_p, c_p, c_p, c_sz, ctypes.c_int, c_p]),
     "lmhead_verify_tree": (ctypes.c_int, [c_p, c_p, c_p, c_p, c_i64, c_i64, c_i64, c_p, c_p, c_i32, c_i32, c_p, c_p,
                                           c_p, c_p, c_p, c_sz, c_p]),
+    "nvfp4_gemm_w4a4_workspace_bytes": (c_sz, [c_i64, c_i64, c_i64]),
+    "nvfp4_gemm_w4a4": (ctypes.c_int, [c_p, c_p, c_p, c_p, c_i64, c_i64, c_i64, c_p, ctypes.c_int, c_p, c_sz, c_p]),
     "nvfp4ws_check": (ctypes.c_int, [c_p]),
     "nvfp4_gemm_skinny_noalloc": (ctypes.c_int, [c_p, c_p, c_p, c_p, c_i64, c_i64, c_i64, c_p, ctypes.c_int, c_p]),
     "nvfp4ws_kernel_launches": (ctypes.c_ulonglong, []),

@@ -5,6 +5,7 @@
 #include "kernels.h"
 #include "mma.h"
 
+#include <algorithm>
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
@@ -186,6 +187,31 @@ int nvfp4_gemm_skinny(const void* X, const uint8_t* q, const uint8_t* sf, const 
                                 NVFP4WS_PATH_AUTO, stream);
 }
 
+size_t nvfp4_gemm_w4a4_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M < 1 || M > NVFP4WS_MAX_M || N < 1) return 0;
+  return mxf4_workspace_bytes(M, N, K, 1);
+}
+
+int nvfp4_gemm_w4a4(const void* X, const uint8_t* q, const uint8_t* sf, const float* tensor_scale, int64_t M,
+                    int64_t N, int64_t K, void* Y, int y_dtype, void* workspace, size_t workspace_bytes,
+                    nvfp4ws_stream_t stream) {
+  g_last_error[0] = 0;
+  if (int e = validate_gemm(X, q, sf, tensor_scale, M, N, K, "nvfp4_gemm_w4a4")) return e;
+  if (!Y) return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_gemm_w4a4: Y is null");
+  if (!aligned16(Y)) return set_error(NVFP4WS_ERR_MISALIGNED, "nvfp4_gemm_w4a4: Y must be 16-byte aligned");
+  if (y_dtype != NVFP4WS_Y_F32 && y_dtype != NVFP4WS_Y_BF16)
+    return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_gemm_w4a4: bad y_dtype %d", y_dtype);
+  if (!mxf4_supported(M, K, 1))
+    return set_error(NVFP4WS_ERR_UNSUPPORTED, "nvfp4_gemm_w4a4: needs K %% 256 == 0, 256 <= K <= 32768 (K=%lld)",
+                     (long long)K);
+  const size_t need = mxf4_workspace_bytes(M, N, K, 1);
+  if (workspace == nullptr || workspace_bytes < need)
+    return set_error(NVFP4WS_ERR_WORKSPACE, "nvfp4_gemm_w4a4: workspace needs %zu bytes", need);
+  if (!aligned16(workspace)) return set_error(NVFP4WS_ERR_MISALIGNED, "nvfp4_gemm_w4a4: workspace must be 16-byte aligned");
+  return launch_mxf4_gemm(static_cast<const uint16_t*>(X), q, sf, tensor_scale, M, N, K, Y, y_dtype, workspace,
+                          (cudaStream_t)stream, 1);
+}
+
 // Largest partial-argmax grid of the two GEMV variants, so either fits the workspace.
 static int gemv_verify_grid(int64_t M, int64_t N, int64_t K) {
   GemvPlan a = gemv_plan(M, N, K, false), b = gemv_plan(M, N, K, true);
@@ -292,16 +318,17 @@ int lmhead_verify_argmax_accept(const void* X, const uint8_t* q, const uint8_t* 
 // ------------------------------------------------------------------ weight passes
 
 static int to_host_problems(const nvfp4_gemm_problem* problems, int32_t count, int64_t M, int verify_last,
-                            std::vector<MxHostProblem>* out, const char* who) {
+                            std::vector<MxHostProblem>* out, const char* who, int terms = kMxf4Terms) {
   if (!problems || count < 1) return set_error(NVFP4WS_ERR_INVALID_ARG, "%s: need count >= 1 problems", who);
-  if (M < 1 || !mxf4_supported(M, 256))
-    return set_error(NVFP4WS_ERR_UNSUPPORTED, "%s: M=%lld outside 1..%d", who, (long long)M, 352 / kMxf4Terms);
+  const int max_m = std::min(352 / terms, NVFP4WS_MAX_M);
+  if (M < 1 || M > max_m || !mxf4_supported(M, 256, terms))
+    return set_error(NVFP4WS_ERR_UNSUPPORTED, "%s: M=%lld outside 1..%d", who, (long long)M, max_m);
   out->clear();
   for (int32_t i = 0; i < count; ++i) {
     const nvfp4_gemm_problem& p = problems[i];
     const bool v = verify_last && i == count - 1;
     if (int e = validate_gemm(p.X, p.q, p.sf, p.tensor_scale, M, p.N, p.K, who)) return e;
-    if (!mxf4_supported(M, p.K))
+    if (!mxf4_supported(M, p.K, terms))
       return set_error(NVFP4WS_ERR_UNSUPPORTED, "%s: problem %d: K=%lld must be a multiple of 256 in [256, 32768]",
                        who, i, (long long)p.K);
     if (!v) {
@@ -317,12 +344,18 @@ static int to_host_problems(const nvfp4_gemm_problem* problems, int32_t count, i
   return NVFP4WS_OK;
 }
 
+static constexpr uint32_t kPassFlags = NVFP4WS_PASS_BATCH_INVARIANT | NVFP4WS_PASS_W4A4;
+static int pass_terms(uint32_t flags) { return (flags & NVFP4WS_PASS_W4A4) ? 1 : kMxf4Terms; }
+
 size_t nvfp4_pass_workspace_bytes_ex(const nvfp4_gemm_problem* problems, int32_t count, int64_t M,
                                      int32_t verify_last, uint32_t flags) {
   std::vector<MxHostProblem> hp;
-  if ((flags & ~(uint32_t)NVFP4WS_PASS_BATCH_INVARIANT) != 0) return 0;
-  if (to_host_problems(problems, count, M, verify_last, &hp, "nvfp4_pass_workspace_bytes") != NVFP4WS_OK) return 0;
-  return mxf4_pass_workspace_bytes(hp.data(), count, M, (flags & NVFP4WS_PASS_BATCH_INVARIANT) != 0);
+  if ((flags & ~kPassFlags) != 0 || ((flags & NVFP4WS_PASS_W4A4) && verify_last)) return 0;
+  if (to_host_problems(problems, count, M, verify_last, &hp, "nvfp4_pass_workspace_bytes", pass_terms(flags)) !=
+      NVFP4WS_OK)
+    return 0;
+  return mxf4_pass_workspace_bytes(hp.data(), count, M, (flags & NVFP4WS_PASS_BATCH_INVARIANT) != 0,
+                                   pass_terms(flags));
 }
 
 size_t nvfp4_pass_workspace_bytes(const nvfp4_gemm_problem* problems, int32_t count, int64_t M, int32_t verify_last) {
@@ -337,13 +370,16 @@ int nvfp4_pass_init(nvfp4_pass* pass, const nvfp4_gemm_problem* problems, int32_
 int nvfp4_pass_init_ex(nvfp4_pass* pass, const nvfp4_gemm_problem* problems, int32_t count, int64_t M,
                        const nvfp4_verify_spec* verify, uint32_t flags, void* workspace, size_t workspace_bytes) {
   g_last_error[0] = 0;
-  if ((flags & ~(uint32_t)NVFP4WS_PASS_BATCH_INVARIANT) != 0)
+  if ((flags & ~kPassFlags) != 0)
     return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_pass_init: unknown flags 0x%x", flags);
+  if ((flags & NVFP4WS_PASS_W4A4) && verify)
+    return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_pass_init: a W4A4 pass runs no verify");
   static_assert(sizeof(nvfp4_pass) >= kMxPassStateBytes, "nvfp4_pass is too small for the pass state");
   if (!pass) return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_pass_init: pass is null");
   std::memset(pass, 0, sizeof(nvfp4_pass));
   std::vector<MxHostProblem> hp;
-  if (int e = to_host_problems(problems, count, M, verify != nullptr, &hp, "nvfp4_pass_init")) return e;
+  if (int e = to_host_problems(problems, count, M, verify != nullptr, &hp, "nvfp4_pass_init", pass_terms(flags)))
+    return e;
   VerifyRule vs{};
   if (verify) {
     if (verify->B < 1 || verify->D < 0)
@@ -360,7 +396,7 @@ int nvfp4_pass_init_ex(nvfp4_pass* pass, const nvfp4_gemm_problem* problems, int
   if (!workspace) return set_error(NVFP4WS_ERR_WORKSPACE, "nvfp4_pass_init: workspace is null");
   if (!aligned16(workspace)) return set_error(NVFP4WS_ERR_MISALIGNED, "nvfp4_pass_init: workspace must be 16-byte aligned");
   return mxf4_pass_init(pass->opaque, hp.data(), count, M, verify ? &vs : nullptr,
-                        (flags & NVFP4WS_PASS_BATCH_INVARIANT) != 0, workspace, workspace_bytes);
+                        (flags & NVFP4WS_PASS_BATCH_INVARIANT) != 0, pass_terms(flags), workspace, workspace_bytes);
 }
 
 int nvfp4_pass_run(const nvfp4_pass* pass, nvfp4ws_stream_t stream) {

@@ -191,8 +191,12 @@ __device__ __forceinline__ void quantise_block(float (&r)[16], int b, int m, flo
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           uint16_t c2;
+          // One term (W4A4): the code is the rounding of the correctly rounded fp32 quotient,
+          // a decision a reader can redo exactly. Several terms: the residual corrects it.
+          const float q1 = T == 1 ? __fdiv_rn(r[2 * i + 1], den) : r[2 * i + 1] * inv;
+          const float q0 = T == 1 ? __fdiv_rn(r[2 * i], den) : r[2 * i] * inv;
           asm("{ .reg .b8 b; cvt.rn.satfinite.e2m1x2.f32 b, %1, %2; cvt.u16.u8 %0, b; }"
-              : "=h"(c2) : "f"(r[2 * i + 1] * inv), "f"(r[2 * i] * inv));
+              : "=h"(c2) : "f"(q1), "f"(q0));
           const uint32_t h = e2m1x2_to_f16x2(c2);
           r[2 * i] = fmaf(-f16lo_to_f32(h), den, r[2 * i]);
           r[2 * i + 1] = fmaf(-f16hi_to_f32(h), den, r[2 * i + 1]);
@@ -210,13 +214,13 @@ __device__ __forceinline__ void quantise_block(float (&r)[16], int b, int m, flo
   }
 }
 
+template <int T>
 __global__ void __launch_bounds__(kPrepThreads, 6) x_prep_kernel(const __grid_constant__ Problem single,
                                                                   const Problem* probs, const Geom g) {
   asm volatile("griddepcontrol.launch_dependents;");
   // X may come from the previous kernel of the stream, and the previous GEMM may still
   // read this workspace: nothing is read or written before that kernel has finished.
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  constexpr int T = kMxf4Terms;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int m = blockIdx.x % g.M;
   const Problem* pr = probs ? probs + blockIdx.x / g.M : &single;
@@ -395,12 +399,16 @@ struct Walk {
   }
 };
 
-// Most tokens a kernel instance folds in registers: two B tiles hold M*T <= 352 rows
-// (M <= 70); one B tile M*T <= 256 (M <= 51); a tile pair needs a double-buffered
-// accumulator, which leaves N <= 104 per tile (M <= 20).
-__host__ __device__ constexpr int pass_max_tokens(int nbt, int tpu) { return tpu == 2 ? 24 : (nbt == 2 ? 72 : 56); }
+// Most tokens a kernel instance serves. Five terms: the row is folded in registers; two
+// B tiles hold M*T <= 352 rows (M <= 70), one B tile M*T <= 256 (M <= 51), and a tile
+// pair needs a double-buffered accumulator, which leaves N <= 104 per tile (M <= 20).
+// One term (W4A4): the row is streamed from TMEM, so only the B rows bound M (352).
+__host__ __device__ constexpr int pass_max_tokens(int nbt, int tpu, int terms) {
+  return terms == 1 ? kMaxB : (tpu == 2 ? 24 : (nbt == 2 ? 72 : 56));
+}
 
-template <int NBT, int KU, int TPU>
+// T: activation terms (kMxf4Terms residual terms, or 1 for NVFP4 activations).
+template <int NBT, int KU, int TPU, int T>
 __global__ void __launch_bounds__(kThreads, 1)
     pass_kernel(const __grid_constant__ Problem single, const PassParams p) {
   // The next kernel of the stream may launch as soon as SMs free up: the library's prep
@@ -419,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* s_last = reinterpret_cast<int*>(s_tmem + 2);
   float* s_val = reinterpret_cast<float*>(s_tmem + 4);                 // [4][72]
   int* s_idx = reinterpret_cast<int*>(s_val + 4 * 72);                 // [4][72]
-  // g_0 of each token of the current problem, 16-byte aligned for float4 reads [80]
+  // g_0 of each token of the current problem, 16-byte aligned for float4 reads [kMaxB]
   float* s_g0 = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(s_idx + 4 * 72) + 15) & ~uintptr_t(15));
 
   auto bar_full = [&](int s) { return smem_u32(bars + s); };
@@ -429,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bar_drain = smem_u32(bars + 2 * S + 4);
   auto bar_sffull = [&](int b) { return smem_u32(bars + 2 * S + 5 + b); };
 
-  constexpr int MT = pass_max_tokens(NBT, TPU);
+  constexpr int MT = pass_max_tokens(NBT, TPU, T);
   const Problem* probs = p.probs ? p.probs : &single;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c = blockIdx.x;
@@ -711,7 +719,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool complete = (seg_u0 == tile_u0) && (u + 1 == tile_u1);
       if (pi != gprob) {
         named_bar(1, 128);
-        for (int j = et; j < M; j += 128) s_g0[j] = pr->xg[j * kMxf4Terms];
+        for (int j = et; j < M; j += 128) s_g0[j] = pr->xg[j * T];
         named_bar(1, 128);
         gprob = pi;
       }
@@ -782,68 +790,111 @@ __global__ void __launch_bounds__(kThreads, 1)
       // accumulator buffer (M=68) the stores of a tile then overlap the next tile's MMAs
       // (measured: holding the buffer through the stores stalled the MMA thread ~15 us per
       // tile under full HBM load).
-      static_assert(kMxf4Terms == 5, "the fold below is written for 5 terms");
-      const int nb16 = (g.nb + 15) & ~15;                 // columns that exist in the accumulator
-      float yr[TPU][MT];
+      if constexpr (T == kMxf4Terms) {
+        static_assert(kMxf4Terms == 5, "the fold below is written for 5 terms");
+        const int nb16 = (g.nb + 15) & ~15;                 // columns that exist in the accumulator
+        float yr[TPU][MT];
 #pragma unroll
-      for (int tj = 0; tj < TPU; ++tj) {
-        const uint32_t taddr = taddr0 + (uint32_t)(tj * NBT * g.nb_tile);
+        for (int tj = 0; tj < TPU; ++tj) {
+          const uint32_t taddr = taddr0 + (uint32_t)(tj * NBT * g.nb_tile);
 #pragma unroll
-        for (int mc = 0; mc < MT; mc += 8) {
-          if (mc < M) {
-            const int col0 = mc * kMxf4Terms;               // multiple of 40
-            const int n8 = (nb16 - col0) >> 3;              // >= 1: loads stay inside the accumulator
-            uint32_t v[40];
+          for (int mc = 0; mc < MT; mc += 8) {
+            if (mc < M) {
+              const int col0 = mc * kMxf4Terms;               // multiple of 40
+              const int n8 = (nb16 - col0) >> 3;              // >= 1: loads stay inside the accumulator
+              uint32_t v[40];
 #pragma unroll
-            for (int k = 0; k < 5; ++k)
-              if (k < n8) tc_ld_x8(taddr + (uint32_t)(col0 + 8 * k), v + 8 * k);
-            const float4 ga = reinterpret_cast<const float4*>(s_g0 + mc)[0];
-            const float4 gb = reinterpret_cast<const float4*>(s_g0 + mc)[1];
-            const float g0[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
-            tc_wait_ld();
+              for (int k = 0; k < 5; ++k)
+                if (k < n8) tc_ld_x8(taddr + (uint32_t)(col0 + 8 * k), v + 8 * k);
+              const float4 ga = reinterpret_cast<const float4*>(s_g0 + mc)[0];
+              const float4 gb = reinterpret_cast<const float4*>(s_g0 + mc)[1];
+              const float g0[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+              tc_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              float a = __uint_as_float(v[j * kMxf4Terms + 4]);
-              a = fmaf(a, 0.25f, __uint_as_float(v[j * kMxf4Terms + 3]));
-              a = fmaf(a, 0.25f, __uint_as_float(v[j * kMxf4Terms + 2]));
-              a = fmaf(a, 0.25f, __uint_as_float(v[j * kMxf4Terms + 1]));
-              a = fmaf(a, 0.25f, __uint_as_float(v[j * kMxf4Terms + 0]));
-              yr[tj][mc + j] = (mc + j < M) ? a * g0[j] : 0.f;   // columns past the tokens are never loaded
+              for (int j = 0; j < 8; ++j) {
+                float a = __uint_as_float(v[j * kMxf4Terms + 4]);
+                a = fmaf(a, 0.25f, __uint_as_float(v[j * kMxf4Terms + 3]));
+                a = fmaf(a, 0.25f, __uint_as_float(v[j * kMxf4Terms + 2]));
+                a = fmaf(a, 0.25f, __uint_as_float(v[j * kMxf4Terms + 1]));
+                a = fmaf(a, 0.25f, __uint_as_float(v[j * kMxf4Terms + 0]));
+                yr[tj][mc + j] = (mc + j < M) ? a * g0[j] : 0.f;   // columns past the tokens are never loaded
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 8; ++j) yr[tj][mc + j] = 0.f;
             }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) yr[tj][mc + j] = 0.f;
           }
         }
-      }
-      tc_fence_before();
-      if (et == 0 && seg < 2) MX_CTA(9 + 4 * seg);
-      mbar_arrive(bar_accempty(ab));
+        tc_fence_before();
+        if (et == 0 && seg < 2) MX_CTA(9 + 4 * seg);
+        mbar_arrive(bar_accempty(ab));
 #pragma unroll
-      for (int tj = 0; tj < TPU; ++tj) {
-        const int tile = group * TPU + tj;
-        const long long n = (long long)tile * kTileRows + rowl;
-        if (complete) {
+        for (int tj = 0; tj < TPU; ++tj) {
+          const int tile = group * TPU + tj;
+          const long long n = (long long)tile * kTileRows + rowl;
+          if (complete) {
 #pragma unroll
-          for (int mc = 0; mc < MT; mc += 16) {
-            if (mc < M) {
-              float y16[16];
+            for (int mc = 0; mc < MT; mc += 16) {
+              if (mc < M) {
+                float y16[16];
 #pragma unroll
-              for (int j = 0; j < 16; ++j) {
-                const int m = mc + j < MT ? mc + j : MT - 1;    // static index; tokens >= M are zeros
-                y16[j] = (mc + j < MT) ? yr[tj][m] * ts : 0.f;
+                for (int j = 0; j < 16; ++j) {
+                  const int m = mc + j < MT ? mc + j : MT - 1;    // static index; tokens >= M are zeros
+                  y16[j] = (mc + j < MT) ? yr[tj][m] * ts : 0.f;
+                }
+                emit16(n, mc, y16);
               }
+            }
+            if (verify && tile < tiles) tile_argmax(tile);
+          } else {
+            float* dst = wave_part + ((long long)(slot * TPU + tj) * kTileRows + rowl) * Mp;   // this row's partials
+#pragma unroll
+            for (int b = 0; b < MT / 4; ++b)
+              if (4 * b < Mp)
+                *reinterpret_cast<float4*>(dst + 4 * b) =
+                    make_float4(yr[tj][4 * b], yr[tj][4 * b + 1], yr[tj][4 * b + 2], yr[tj][4 * b + 3]);
+          }
+        }
+      } else {
+        // One term (W4A4): accumulator column j is token j, so there is nothing to fold.
+        // Up to 352 tokens do not fit in registers: the row is scaled and stored 16 tokens
+        // at a time while the accumulator is held, and handed back after the last load.
+        // (The host runs no verify problem here: its candidates are kept for <= 72 rows.)
+        static_assert(T == 1, "one or kMxf4Terms activation terms");
+        for (int tj = 0; tj < TPU; ++tj) {
+          const uint32_t taddr = taddr0 + (uint32_t)(tj * NBT * g.nb_tile);
+          const int tile = group * TPU + tj;
+          const long long n = (long long)tile * kTileRows + rowl;
+          float* dst = wave_part + ((long long)(slot * TPU + tj) * kTileRows + rowl) * Mp;   // this row's partials
+          for (int mc = 0; mc < M; mc += 16) {
+            uint32_t v[16];
+            tc_ld_x16(taddr + (uint32_t)mc, v);            // mc + 16 <= (M + 15) & ~15 <= NBT * nb_tile
+            float g0[16];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float4 t4 = reinterpret_cast<const float4*>(s_g0 + mc)[k];
+              g0[4 * k] = t4.x; g0[4 * k + 1] = t4.y; g0[4 * k + 2] = t4.z; g0[4 * k + 3] = t4.w;
+            }
+            tc_wait_ld();
+            if (tj + 1 == TPU && mc + 16 >= M) {             // last load of the buffer: release it
+              tc_fence_before();
+              mbar_arrive(bar_accempty(ab));
+            }
+            float y16[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) y16[j] = (mc + j < M) ? __uint_as_float(v[j]) * g0[j] : 0.f;
+            if (complete) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) y16[j] *= ts;
               emit16(n, mc, y16);
+            } else {
+#pragma unroll
+              for (int b = 0; b < 4; ++b)
+                if (mc + 4 * b < Mp)
+                  *reinterpret_cast<float4*>(dst + mc + 4 * b) =
+                      make_float4(y16[4 * b], y16[4 * b + 1], y16[4 * b + 2], y16[4 * b + 3]);
             }
           }
-          if (verify && tile < tiles) tile_argmax(tile);
-        } else {
-          float* dst = wave_part + ((long long)(slot * TPU + tj) * kTileRows + rowl) * Mp;   // this row's partials
-#pragma unroll
-          for (int b = 0; b < MT / 4; ++b)
-            if (4 * b < Mp)
-              *reinterpret_cast<float4*>(dst + 4 * b) =
-                  make_float4(yr[tj][4 * b], yr[tj][4 * b + 1], yr[tj][4 * b + 2], yr[tj][4 * b + 3]);
         }
       }
       ++seg;
@@ -960,11 +1011,11 @@ struct MxPlan {
   size_t smem;
 };
 
-static MxPlan mx_plan_ku(long long M, int ku, int tpu) {
+static MxPlan mx_plan_ku(long long M, int ku, int tpu, int terms = kMxf4Terms) {
   MxPlan pl{};
   Geom& g = pl.g;
   g.M = (int)M;
-  g.T = kMxf4Terms;
+  g.T = terms;
   g.nb = (int)M * g.T;
   g.nbt = (g.nb + 255) / 256;
   g.nb_tile = ((g.nb + g.nbt - 1) / g.nbt + 15) / 16 * 16;   // MMA N; a multiple of 16 keeps x16 loads inside the tile
@@ -1001,26 +1052,26 @@ static MxPlan mx_plan_ku(long long M, int ku, int tpu) {
 // of 3). Either needs one B tile and a double-buffered accumulator.
 // Batch-invariant passes (binv) use one unit shape for every M, so that a row's units,
 // split points and summation order do not depend on how many rows share the pass.
-static MxPlan mx_plan(long long M, bool k512, bool binv = false) {
+static MxPlan mx_plan(long long M, bool k512, bool binv = false, int terms = kMxf4Terms) {
   auto ok = [](const MxPlan& x, int min_stages) {
     return x.g.nbt == 1 && x.acc_bufs == 2 && x.stages >= min_stages;
   };
-  if (binv) return mx_plan_ku(M, 1, 1);
+  if (binv) return mx_plan_ku(M, 1, 1, terms);
   if (k512) {
-    const MxPlan two = mx_plan_ku(M, 2, 1);
+    const MxPlan two = mx_plan_ku(M, 2, 1, terms);
     if (ok(two, 4)) return two;
   }
-  const MxPlan pair = mx_plan_ku(M, 1, 2);
-  if (ok(pair, 3)) return pair;
+  const MxPlan pair = mx_plan_ku(M, 1, 2, terms);
+  if (ok(pair, 3) && M <= pass_max_tokens(1, 2, terms)) return pair;
   if (k512) {
-    const MxPlan two = mx_plan_ku(M, 2, 1);
+    const MxPlan two = mx_plan_ku(M, 2, 1, terms);
     if (ok(two, 3)) return two;
   }
-  return mx_plan_ku(M, 1, 1);
+  return mx_plan_ku(M, 1, 1, terms);
 }
 
-bool mxf4_supported(long long M, long long K) {
-  return M >= 1 && M * kMxf4Terms <= kMaxB && K % kKC == 0 && K >= kKC && K <= 32768;
+bool mxf4_supported(long long M, long long K, int terms) {
+  return M >= 1 && M * terms <= kMaxB && K % kKC == 0 && K >= kKC && K <= 32768;
 }
 
 // Activation-image bytes a wave may hold: small enough that a wave's images stay in L2
@@ -1054,10 +1105,12 @@ static bool all_k512(const MxHostProblem* hp, int n) {
 }
 
 // with_desc: a pass keeps its descriptors and wave tables in the workspace.
-static WsLayout mx_layout(const MxHostProblem* hp, int n, long long M, bool with_desc, bool binv = false) {
-  const MxPlan pl = mx_plan(M, all_k512(hp, n), binv);
+static WsLayout mx_layout(const MxHostProblem* hp, int n, long long M, bool with_desc, bool binv = false,
+                          int terms = kMxf4Terms) {
+  const MxPlan pl = mx_plan(M, all_k512(hp, n), binv, terms);
   // waves are cut by image bytes; a batch-invariant pass cuts them as the largest M would
-  const uint32_t wave_img_stride = binv ? mx_plan_ku(kMaxB / kMxf4Terms, 1, 1).g.img_stride : pl.g.img_stride;
+  const uint32_t wave_img_stride =
+      binv ? mx_plan_ku(kMaxB / terms, 1, 1, terms).g.img_stride : pl.g.img_stride;
   const int ku = pl.g.ku, tpu = pl.g.tpu;
   WsLayout L;
   L.units = 0;
@@ -1132,17 +1185,31 @@ static int fill_problem(Problem* P, const MxHostProblem& h, const WsLayout& L, i
   return NVFP4WS_OK;
 }
 
+template <int NBT, int KU, int TPU, int T>
+static const void* pass_fn() { return reinterpret_cast<const void*>(&pass_kernel<NBT, KU, TPU, T>); }
+
+// The kernel instance of a plan: B tiles, unit shape and activation terms.
+template <int T>
+static const void* pass_instance_t(const Geom& g) {
+  return g.nbt == 2 ? pass_fn<2, 1, 1, T>() : g.tpu == 2 ? pass_fn<1, 1, 2, T>() : g.ku == 2 ? pass_fn<1, 2, 1, T>()
+                                                                                          : pass_fn<1, 1, 1, T>();
+}
+static const void* pass_instance(const Geom& g) {
+  static_assert(kMxf4Terms == 5, "pass kernel instances are built for 5 terms and 1");
+  return g.T == 1 ? pass_instance_t<1>(g) : pass_instance_t<5>(g);
+}
+
 static int ensure_attrs() {
   static bool attr_set[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
     return set_error(NVFP4WS_ERR_CUDA, "cannot get the current device");
   if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(pass_kernel<1, 1, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess ||
-        cudaFuncSetAttribute(pass_kernel<1, 2, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess ||
-        cudaFuncSetAttribute(pass_kernel<1, 1, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess ||
-        cudaFuncSetAttribute(pass_kernel<2, 1, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
-      return check_launch("cudaFuncSetAttribute(pass_kernel)");
+    const void* fns[] = {pass_fn<1, 1, 1, 5>(), pass_fn<1, 2, 1, 5>(), pass_fn<1, 1, 2, 5>(), pass_fn<2, 1, 1, 5>(),
+                         pass_fn<1, 1, 1, 1>(), pass_fn<1, 2, 1, 1>(), pass_fn<1, 1, 2, 1>(), pass_fn<2, 1, 1, 1>()};
+    for (const void* f : fns)
+      if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
+        return check_launch("cudaFuncSetAttribute(pass_kernel)");
     attr_set[dev] = true;
   }
   return NVFP4WS_OK;
@@ -1176,7 +1243,8 @@ static int launch_pass(const Problem& single, const Problem* probs_dev, const Pa
     pc.attrs = pa;
     pc.numAttrs = 1;
     const Geom g = pl.g;
-    cudaError_t pe = cudaLaunchKernelEx(&pc, x_prep_kernel, single, probs_dev, g);
+    cudaError_t pe = g.T == 1 ? cudaLaunchKernelEx(&pc, x_prep_kernel<1>, single, probs_dev, g)
+                              : cudaLaunchKernelEx(&pc, x_prep_kernel<kMxf4Terms>, single, probs_dev, g);
     if (pe != cudaSuccess) return set_error(NVFP4WS_ERR_CUDA, "x_prep_kernel launch: %s", cudaGetErrorString(pe));
     if (int e = check_launch("x_prep_kernel")) return e;
   }
@@ -1213,24 +1281,24 @@ static int launch_pass(const Problem& single, const Problem* probs_dev, const Pa
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (pl.g.M > pass_max_tokens(pl.g.nbt, pl.g.tpu)) return cudaErrorInvalidValue;
-  cudaError_t e = (pl.g.nbt == 2)   ? cudaLaunchKernelEx(&cfg, pass_kernel<2, 1, 1>, single, p)
-                  : (pl.g.tpu == 2) ? cudaLaunchKernelEx(&cfg, pass_kernel<1, 1, 2>, single, p)
-                  : (pl.g.ku == 2)  ? cudaLaunchKernelEx(&cfg, pass_kernel<1, 2, 1>, single, p)
-                                    : cudaLaunchKernelEx(&cfg, pass_kernel<1, 1, 1>, single, p);
+  if (pl.g.M > pass_max_tokens(pl.g.nbt, pl.g.tpu, pl.g.T))
+    return set_error(NVFP4WS_ERR_UNSUPPORTED, "block-scaled path: M=%d exceeds the kernel's token capacity", pl.g.M);
+  void* args[] = {const_cast<Problem*>(&single), &p};
+  cudaError_t e = cudaLaunchKernelExC(&cfg, pass_instance(pl.g), args);
   if (e != cudaSuccess) return set_error(NVFP4WS_ERR_CUDA, "pass_kernel launch: %s", cudaGetErrorString(e));
   return check_launch("pass_kernel");
 }
 
-size_t mxf4_workspace_bytes(long long M, long long N, long long K) {
-  if (!mxf4_supported(M, K)) return 0;
+size_t mxf4_workspace_bytes(long long M, long long N, long long K, int terms) {
+  if (!mxf4_supported(M, K, terms)) return 0;
   MxHostProblem h{nullptr, nullptr, nullptr, nullptr, N, K, nullptr, 0, 1};   // sized with the verify tail
-  return mx_layout(&h, 1, M, false).total;
+  return mx_layout(&h, 1, M, false, false, terms).total;
 }
 
-static int launch_single(const MxHostProblem& h, long long M, void* workspace, cudaStream_t s, Problem* out) {
-  const MxPlan pl = mx_plan(M, all_k512(&h, 1));
-  const WsLayout L = mx_layout(&h, 1, M, false);
+static int launch_single(const MxHostProblem& h, long long M, void* workspace, cudaStream_t s, Problem* out,
+                         int terms = kMxf4Terms) {
+  const MxPlan pl = mx_plan(M, all_k512(&h, 1), false, terms);
+  const WsLayout L = mx_layout(&h, 1, M, false, false, terms);
   char* ws = static_cast<char*>(workspace);
   if (int e = fill_problem(out, h, L, 0, 0, ws, pl.g.ku, pl.g.tpu)) return e;
   const PassTables none{nullptr, nullptr, nullptr, 1};
@@ -1238,10 +1306,10 @@ static int launch_single(const MxHostProblem& h, long long M, void* workspace, c
 }
 
 int launch_mxf4_gemm(const uint16_t* X, const uint8_t* q, const uint8_t* sf, const float* ts, long long M,
-                     long long N, long long K, void* Y, int y_dtype, void* workspace, cudaStream_t s) {
+                     long long N, long long K, void* Y, int y_dtype, void* workspace, cudaStream_t s, int terms) {
   MxHostProblem h{X, q, sf, ts, N, K, Y, y_dtype == NVFP4WS_Y_BF16 ? 1 : 0, 0};
   Problem P;
-  return launch_single(h, M, workspace, s, &P);
+  return launch_single(h, M, workspace, s, &P, terms);
 }
 
 int launch_mxf4_verify(const uint16_t* X, const uint8_t* q, const uint8_t* sf, const float* ts, long long M,
@@ -1257,7 +1325,7 @@ int launch_mxf4_verify(const uint16_t* X, const uint8_t* q, const uint8_t* sf, c
 // Host state of a pass: plain data in caller-owned memory (no allocation).
 struct MxPassState {
   uint32_t magic;
-  int nprob, grid, verify, vtiles, k512, binv;
+  int nprob, grid, verify, vtiles, k512, binv, terms;
   long long M, max_k;
   unsigned long long units;
   size_t off_part;
@@ -1271,16 +1339,16 @@ struct MxPassState {
 static_assert(sizeof(MxPassState) <= kMxPassStateBytes, "pass state does not fit the caller's handle");
 constexpr uint32_t kPassMagic = 0x4e565053u;
 
-size_t mxf4_pass_workspace_bytes(const MxHostProblem* hp, int n, long long M, bool binv) {
-  return mx_layout(hp, n, M, true, binv).total;
+size_t mxf4_pass_workspace_bytes(const MxHostProblem* hp, int n, long long M, bool binv, int terms) {
+  return mx_layout(hp, n, M, true, binv, terms).total;
 }
 
 int mxf4_pass_init(void* state, const MxHostProblem* hp, int n, long long M, const VerifyRule* vs, bool binv,
-                   void* workspace, size_t workspace_bytes) {
+                   int terms, void* workspace, size_t workspace_bytes) {
   MxPassState* P = static_cast<MxPassState*>(state);
   std::memset(static_cast<void*>(P), 0, sizeof(MxPassState));
-  const WsLayout L = mx_layout(hp, n, M, true, binv);
-  const MxPlan plan = mx_plan(M, all_k512(hp, n), binv);
+  const WsLayout L = mx_layout(hp, n, M, true, binv, terms);
+  const MxPlan plan = mx_plan(M, all_k512(hp, n), binv, terms);
   const int ku = plan.g.ku, tpu = plan.g.tpu;
   if (workspace_bytes < L.total)
     return set_error(NVFP4WS_ERR_WORKSPACE, "nvfp4_pass_init: workspace %zu bytes < required %zu", workspace_bytes,
@@ -1328,6 +1396,7 @@ int mxf4_pass_init(void* state, const MxHostProblem* hp, int n, long long M, con
   P->nprob = n;
   P->k512 = all_k512(hp, n) ? 1 : 0;
   P->binv = binv ? 1 : 0;
+  P->terms = terms;
   P->grid = L.grid;
   P->units = L.units;
   P->off_part = L.off_part;
@@ -1351,7 +1420,7 @@ int mxf4_pass_run(const void* state, cudaStream_t s) {
   const MxPassState* P = static_cast<const MxPassState*>(state);
   if (P->magic != kPassMagic) return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_pass_run: pass not initialised");
   static const Problem kNoProblem{};   // the kernels' by-value problem slot, unused by a pass
-  const MxPlan pl = mx_plan(P->M, P->k512 != 0, P->binv != 0);
+  const MxPlan pl = mx_plan(P->M, P->k512 != 0, P->binv != 0, P->terms);
   if (int e = launch_pass(kNoProblem, P->probs_dev, P->tb, P->nprob, pl, P->grid, P->units, P->off_part,
                           P->max_k, P->ws, s))
     return e;
