@@ -528,7 +528,7 @@ def run_sweep(args):
 # ----------------------------------------------------------------------------- reference arm
 
 def run_w4a4(args):
-    """The W4A4 weight pass at prefill-sized M (SURVEY-style "next" row): the 192 GEMMs of
+    """The W4A4 weight pass at prefill-sized M: the 192 GEMMs of
     the 27B stack with their activations quantised to NVFP4, one persistent launch, timed
     as a CUDA graph. One JSON line per M with the weight GB/s against the HBM roofline and
     the tensor TFLOP/s against the fp4 peak (measured bf16 x 4, the nominal fp4/bf16
