@@ -93,3 +93,32 @@ def test_verify_rejects(lib):
     # null outputs
     assert f(FAKE, FAKE, FAKE, FAKE, 17, 100, 64, FAKE, 1, 16, None, FAKE, None, FAKE, 1 << 20, None) == 1
     assert f(FAKE, FAKE, FAKE, FAKE, 1, 100, 64, None, 0, 0, FAKE, FAKE, None, FAKE, 1 << 20, None) == 1  # B < 1
+
+
+def test_w4a4_rejects_on_the_host(lib):
+    f = lib.nvfp4_gemm_w4a4
+    assert f(None, FAKE, FAKE, FAKE, 1, 16, 256, FAKE, 0, None, 0, None) == 1          # null X
+    assert f(FAKE, FAKE, FAKE, FAKE, 257, 16, 256, FAKE, 0, None, 0, None) == 2        # M > 256
+    assert f(FAKE, FAKE, FAKE, FAKE, 4, 16, 256, FAKE, 3, None, 0, None) == 1          # bad y dtype
+    assert f(FAKE, FAKE, FAKE, FAKE, 4, 16, 96, FAKE, 0, None, 0, None) == 2           # K % 256
+    assert f(FAKE, FAKE, FAKE, FAKE, 4, 16, 256, FAKE + 4, 0, None, 0, None) == 3      # misaligned Y
+    assert lib.nvfp4_gemm_w4a4_workspace_bytes(0, 16, 256) == 0
+    assert lib.nvfp4_gemm_w4a4_workspace_bytes(257, 16, 256) == 0
+
+
+def test_tree_verify_needs_parents(lib):
+    f = lib.lmhead_verify_tree
+    # D = 3 drafts but no parent array: refused before anything is launched
+    assert f(FAKE, FAKE, FAKE, FAKE, 4, 100, 256, FAKE, None, 1, 3, FAKE, FAKE, None, None, None, 0, None) == 1
+    assert b"parents" in lib.nvfp4ws_last_error()
+
+
+def test_pass_flags_are_checked_first(lib):
+    from nvfp4_weight_streaming_gemm_b200 import _lib as L
+    arr = (L.GemmProblem * 1)()
+    arr[0] = L.GemmProblem(FAKE, FAKE, FAKE, FAKE, 128, 256, FAKE, 0)
+    assert lib.nvfp4_pass_workspace_bytes_ex(arr, 1, 17, 0, 4) == 0        # unknown flag
+    assert lib.nvfp4_pass_workspace_bytes_ex(arr, 1, 17, 1, 2) == 0        # W4A4 with a verify problem
+    st = L.PassState()
+    assert lib.nvfp4_pass_init_ex(ctypes.byref(st), arr, 1, 17, None, 8, FAKE, 1 << 20) == 1
+    assert b"flags" in lib.nvfp4ws_last_error()
