@@ -312,6 +312,8 @@ typedef struct nvfp4_gemm_problem {
   int32_t y_dtype;
 } nvfp4_gemm_problem;
 
+/* parents and accept_node were appended in ABI version 101 (nvfp4ws_version()): code
+ * built against an older header passes a shorter struct and must be rebuilt. */
 typedef struct nvfp4_verify_spec {
   const int32_t* drafts;
   int32_t B;

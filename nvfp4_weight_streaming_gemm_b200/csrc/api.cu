@@ -113,7 +113,7 @@ const char* nvfp4ws_status_string(int status) {
 
 const char* nvfp4ws_last_error(void) { return g_last_error; }
 
-int nvfp4ws_version(void) { return 100; }
+int nvfp4ws_version(void) { return 101; }
 
 int nvfp4ws_sm_count(void) { return device_sm_count(); }
 
