@@ -73,11 +73,17 @@ TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "pass_kernel_dram_traffic.json"
 
 
 def pass_kernel_source_hash() -> str:
+    """Hash of the pass kernel's sources with comments and whitespace removed: a change
+    of the code invalidates a stored capture, a change of its comments does not."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for rel in PASS_KERNEL_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel)) as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()
 
 
