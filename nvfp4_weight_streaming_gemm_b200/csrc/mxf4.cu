@@ -17,7 +17,9 @@
 // and every S_t fits E4M3. Each term cuts the error about 10x; with T = 5 the
 // GEMM matches the exact float64 result to ~1e-5 relative and logits to ~5e-5
 // absolute. The terms are extra B rows (token m, term t -> row m*T + t). The
-// epilogue folds them: y[m] = ts * sum_t g_t acc[m*T+t].
+// epilogue folds them: y[m] = ts * sum_t g_t acc[m*T+t]. With T = 1 (the W4A4
+// product) the single term is the NVFP4 quantisation of the row, its code taken
+// from a correctly rounded fp32 quotient.
 //
 // Kernels.
 //   x_prep_kernel   one CTA per (activation row, problem): the T-term decomposition,
@@ -27,23 +29,28 @@
 //                   measured on B200, a 2D tensor box gathering R rows of 128 B from
 //                   L2 cuts the concurrent HBM weight stream by 11% (R=16) to 50%
 //                   (R=352); a contiguous bulk copy of the same bytes costs ~3%.
-//   pass_kernel     one persistent CTA per SM, 12 warps, over the concatenated
-//                   (problem, 128-row tile, 256-wide K-chunk) units of all problems,
-//                   split evenly across CTAs (stream-K). Tiles split between CTAs
-//                   occur only at the G-1 CTA range boundaries of the whole list.
-//     warp 0        TMA producer: the W tile (128 rows x 128 B nibbles, SW128) and its
-//                   128 x 16 B scales (2D tensor loads), then the activation image
-//                   (1D bulk). The first stages' weight loads are issued before waiting
-//                   on the prep kernel.
-//     warp 1        TMEM allocator and MMA issuer: 4 K-steps x B-tiles of
-//                   tcgen05.mma kind::mxf4nvf4.block_scale.block16 per unit.
+//   pass_kernel     one persistent CTA per SM, 12 warps, over the concatenated units
+//                   of all problems: a group of 1-2 128-row tiles x 1-2 256-wide
+//                   K-chunks. Consecutive problems whose images fit L2 together form a
+//                   wave, and each wave's units are split evenly across the CTAs
+//                   (stream-K), so a tile is split between CTAs only at the G-1 range
+//                   boundaries of a wave.
+//     warp 0        TMA producer: the W tiles (128 rows x 128 B nibbles, SW128) and
+//                   their 128 x 16 B scales (2D tensor loads), then the activation
+//                   images (1D bulk). Codes stream evict-first; scale lines and images,
+//                   which are read again, evict-last. The first stages' weight loads
+//                   are issued before waiting on the prep kernel.
+//     warp 1        TMEM allocator and MMA issuer: 4 K-steps x B-tiles x tiles of
+//                   tcgen05.mma kind::mxf4nvf4.block_scale.block16 per K-chunk.
 //     warps 4-7     scale-factor warpgroup: copies the unit's W and X block scales
 //                   from shared memory into TMEM in the layout the MMA reads (the 4
 //                   scales of row m0 + 32*j in column j of lane m0, replicated over the
-//                   four lane quarters).
-//     warps 8-11    epilogue: tcgen05.ld of the accumulators, fold of the terms,
-//                   x ts, then Y or the per-tile argmax of a verify problem. The last
-//                   CTA to finish a split tile sums the partials in CTA order.
+//                   four lane quarters), all of a chunk's shared loads first.
+//     warps 8-11    epilogue: tcgen05.ld of the accumulators; five terms are folded
+//                   into registers and the accumulator is released before any store,
+//                   one term is streamed 16 tokens at a time; then x ts and Y, the
+//                   per-tile argmax of a verify problem, or a split tile's partials,
+//                   which the last CTA to finish the tile sums in CTA order.
 // Every wait is bounded (see sync.cuh); a timeout sets the device error word.
 #include "common.cuh"
 #include "kernels.h"
