@@ -360,6 +360,51 @@ int nvfp4_pass_init_ex(nvfp4_pass* pass, const nvfp4_gemm_problem* problems, int
 int nvfp4_pass_run(const nvfp4_pass* pass, nvfp4ws_stream_t stream);
 
 /*
+ * FP8 weights -- E4M3 codes with one fp32 scale per 128 x 128 block (rows x K).
+ *
+ * Passages: "TandemLLM", "The parts" (an FP8 e4m3 output head, loaded over the vendor's
+ * FP8 checkpoint) and "Qwen3.8 on DGX Spark (GB10)" (FP8 block-scaled projections). The
+ * pages give neither the block shape nor the scale rule. This library reads them as
+ *   s[i, j] = fp32( amax|W[128i .. 128i+127, 128j .. 128j+127]| / 448 )   0 for a zero block
+ *   code    = E4M3_rne_satfinite( w / s ), sign kept                   +0 where s = 0
+ * with the quotient formed in float64 and rounded once. Blocks at the right and bottom
+ * edges cover what remains of W.
+ *
+ * fp8_pack -- quantise an fp32 weight.
+ *   W        fp32 [N, K] row-major, device, 16-byte aligned. Read only.
+ *   N, K     N >= 1; K >= 16, K % 16 == 0, K <= 8388480.
+ *   q        out: uint8 [N, K] row-major, device, 16-byte aligned: E4M3 bits per element.
+ *   scales   out: fp32 [ceil(N/128), ceil(K/128)] row-major, device, 4-byte aligned.
+ * Returns NVFP4WS_OK, or INVALID_ARG / MISALIGNED / CUDA.
+ *
+ * fp8_gemm_skinny -- Y[M, N] = X[M, K] . dequant(W)^T, with
+ *   dequant(W)[n, k] = e4m3(q[n, k]) * scales[n / 128, k / 128].
+ *   X is converted to f16 as in nvfp4_gemm_skinny, so each product x * e4m3(q) is exact;
+ *   each block's 128 products are summed in fp32, multiplied by the block's scale and
+ *   added to the row's sum in K order, in fp32.
+ *   X        bf16 [M, K], device, 16-byte aligned.   1 <= M <= 128.
+ *   q, scales  as written by fp8_pack.   N >= 1.   K a positive multiple of 128.
+ *   Y        out: [M, N], device, 16-byte aligned; fp32 or bf16 per y_dtype.
+ *   workspace  at least fp8_gemm_workspace_bytes(M, N, K) bytes, 16-byte aligned, zero-filled
+ *            before its first use; every completed call leaves it reusable.
+ * Returns NVFP4WS_OK, or INVALID_ARG / UNSUPPORTED / MISALIGNED / WORKSPACE / CUDA.
+ *
+ * fp8_lmhead_verify -- the FP8 lm_head with the fused greedy verify. The logits are
+ *   fp8_gemm_skinny's and are never written to memory. `verify` gives the rule and its
+ *   buffers as for a weight pass: the chain rule of lmhead_verify_argmax_accept when
+ *   verify->parents is NULL, else the tree rule of lmhead_verify_tree. M must equal
+ *   verify->B * (verify->D + 1). Workspace: fp8_lmhead_verify_workspace_bytes(M, N, K).
+ */
+int fp8_pack(const float* W, int64_t N, int64_t K, uint8_t* q, float* scales, nvfp4ws_stream_t stream);
+size_t fp8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+int fp8_gemm_skinny(const void* X, const uint8_t* q, const float* scales, int64_t M, int64_t N, int64_t K,
+                    void* Y, int y_dtype, void* workspace, size_t workspace_bytes, nvfp4ws_stream_t stream);
+size_t fp8_lmhead_verify_workspace_bytes(int64_t M, int64_t N, int64_t K);
+int fp8_lmhead_verify(const void* X, const uint8_t* q, const float* scales, int64_t M, int64_t N, int64_t K,
+                      const nvfp4_verify_spec* verify, void* workspace, size_t workspace_bytes,
+                      nvfp4ws_stream_t stream);
+
+/*
  * nvfp4_gemm_skinny_noalloc -- the tensor-core GEMM of nvfp4_gemm_skinny for callers
  * that cannot allocate device memory and so cannot pass a workspace. Examples are a
  * host that fixes its device-memory plan at start-up and forbids later allocation,

@@ -11,6 +11,8 @@ torch, and passes raw device pointers and the current CUDA stream.
     t, L, node, vmax = verify_tree(X, q, sf, ts, drafts, parents)   # the same over a draft tree
     p = WeightPass([(X_i, q_i, sf_i, ts_i, Y_i), ...], M, verify=...)   # a whole list, one launch
     p.run()
+    q8, s8 = fp8_pack(W)                       # fp32 [N, K] -> E4M3 + fp32 per 128 x 128 block
+    Y = fp8_gemm(X, q8, s8)                    # and its verify: fp8_verify(X, q8, s8, drafts[, parents])
 """
 
 from __future__ import annotations
@@ -191,6 +193,71 @@ def gemm_w4a4(X: torch.Tensor, q: torch.Tensor, sf: torch.Tensor, ts: torch.Tens
     _check(lib().nvfp4_gemm_w4a4(_ptr(X), _ptr(q), _ptr(sf), _ptr(ts), M, N, K, _ptr(Y), yd, _ptr(ws), nbytes,
                                  _stream(stream)), "nvfp4_gemm_w4a4")
     return Y
+
+
+def fp8_pack(W: torch.Tensor, stream=None, out=None):
+    """Quantise fp32 W [N, K] to FP8 E4M3 with one fp32 scale per 128 x 128 block (``fp8_pack``).
+
+    Returns ``(q uint8 [N, K], scales fp32 [ceil(N/128), ceil(K/128)])``.
+    """
+    _need_cuda(W, "W", torch.float32)
+    N, K = W.shape
+    if out is None:
+        q = torch.empty((N, K), dtype=torch.uint8, device=W.device)
+        scales = torch.empty(((N + 127) // 128, (K + 127) // 128), dtype=torch.float32, device=W.device)
+    else:
+        q, scales = out
+    _check(lib().fp8_pack(_ptr(W), N, K, _ptr(q), _ptr(scales), _stream(stream)), "fp8_pack")
+    return q, scales
+
+
+def fp8_gemm(X: torch.Tensor, q: torch.Tensor, scales: torch.Tensor, out: torch.Tensor | None = None,
+             y_dtype: torch.dtype = torch.float32, workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Y[M, N] = X[M, K] . dequant(W)^T for FP8 block-scaled W (``fp8_gemm_skinny``); X bf16."""
+    _need_cuda(X, "X", torch.bfloat16)
+    _need_cuda(q, "q", torch.uint8)
+    _need_cuda(scales, "scales", torch.float32)
+    M, K = X.shape
+    N = q.shape[0]
+    if q.shape[1] != K or scales.shape != ((N + 127) // 128, (K + 127) // 128):
+        raise ValueError("q / scales shapes do not match X")
+    Y = out if out is not None else torch.empty((M, N), dtype=y_dtype, device=X.device)
+    yd = {torch.float32: 0, torch.bfloat16: 1}[Y.dtype]
+    ws = _workspace(int(lib().fp8_gemm_workspace_bytes(M, N, K)), X.device, workspace)
+    nbytes = 0 if ws is None else ws.numel()
+    _check(lib().fp8_gemm_skinny(_ptr(X), _ptr(q), _ptr(scales), M, N, K, _ptr(Y), yd, _ptr(ws), nbytes,
+                                 _stream(stream)), "fp8_gemm_skinny")
+    return Y
+
+
+def fp8_verify(X: torch.Tensor, q: torch.Tensor, scales: torch.Tensor, drafts: torch.Tensor,
+               parents: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+               with_max_logit: bool = True, stream=None):
+    """Fused greedy verify over an FP8 lm_head (``fp8_lmhead_verify``): the chain rule, or the
+    tree rule when ``parents`` is given.
+
+    Returns ``(argmax int32 [M], accept_len int32 [B], accept_node int32 [B], max_logit fp32 [M] or None)``.
+    """
+    _need_cuda(X, "X", torch.bfloat16)
+    _need_cuda(drafts, "drafts", torch.int32)
+    M, K = X.shape
+    N = q.shape[0]
+    B, D = drafts.shape
+    if parents is not None:
+        _need_cuda(parents, "parents", torch.int32)
+        if parents.shape != (B, D):
+            raise ValueError("parents must have the shape of drafts")
+    amax = torch.empty(M, dtype=torch.int32, device=X.device)
+    acc = torch.empty(B, dtype=torch.int32, device=X.device)
+    node = torch.empty(B, dtype=torch.int32, device=X.device)
+    vmax = torch.empty(M, dtype=torch.float32, device=X.device) if with_max_logit else None
+    spec = _lib.VerifySpec(_ptr(drafts) if drafts.numel() else None, B, D, _ptr(amax), _ptr(acc), _ptr(vmax),
+                           _ptr(parents) if parents is not None and parents.numel() else None, _ptr(node))
+    ws = _workspace(int(lib().fp8_lmhead_verify_workspace_bytes(M, N, K)), X.device, workspace)
+    nbytes = 0 if ws is None else ws.numel()
+    _check(lib().fp8_lmhead_verify(_ptr(X), _ptr(q), _ptr(scales), M, N, K, ctypes.byref(spec), _ptr(ws), nbytes,
+                                   _stream(stream)), "fp8_lmhead_verify")
+    return amax, acc, node, vmax
 
 
 def check(stream=None):

@@ -62,6 +62,12 @@ SIGNATURES = {
     "nvfp4_pass_workspace_bytes_ex": (c_sz, [ctypes.POINTER(GemmProblem), c_i32, c_i64, c_i32, ctypes.c_uint32]),
     "nvfp4_pass_init_ex": (ctypes.c_int, [ctypes.POINTER(PassState), ctypes.POINTER(GemmProblem), c_i32, c_i64,
                                           ctypes.POINTER(VerifySpec), ctypes.c_uint32, c_p, c_sz]),
+    "fp8_pack": (ctypes.c_int, [c_p, c_i64, c_i64, c_p, c_p, c_p]),
+    "fp8_gemm_workspace_bytes": (c_sz, [c_i64, c_i64, c_i64]),
+    "fp8_gemm_skinny": (ctypes.c_int, [c_p, c_p, c_p, c_i64, c_i64, c_i64, c_p, ctypes.c_int, c_p, c_sz, c_p]),
+    "fp8_lmhead_verify_workspace_bytes": (c_sz, [c_i64, c_i64, c_i64]),
+    "fp8_lmhead_verify": (ctypes.c_int, [c_p, c_p, c_p, c_i64, c_i64, c_i64, ctypes.POINTER(VerifySpec), c_p, c_sz,
+                                         c_p]),
 }
 
 _lib = None

@@ -2,6 +2,7 @@
 // sizing, kernel-path dispatch and error reporting. Every check runs on the host
 // before anything is enqueued.
 #include "common.cuh"
+#include "fp8.h"
 #include "kernels.h"
 #include "mma.h"
 
@@ -113,7 +114,7 @@ const char* nvfp4ws_status_string(int status) {
 
 const char* nvfp4ws_last_error(void) { return g_last_error; }
 
-int nvfp4ws_version(void) { return 101; }
+int nvfp4ws_version(void) { return 102; }
 
 int nvfp4ws_sm_count(void) { return device_sm_count(); }
 
@@ -403,6 +404,75 @@ int nvfp4_pass_run(const nvfp4_pass* pass, nvfp4ws_stream_t stream) {
   g_last_error[0] = 0;
   if (!pass) return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_pass_run: pass is null");
   return mxf4_pass_run(pass->opaque, (cudaStream_t)stream);
+}
+
+// ------------------------------------------------------------------ FP8 weights
+
+int fp8_pack(const float* W, int64_t N, int64_t K, uint8_t* q, float* scales, nvfp4ws_stream_t stream) {
+  g_last_error[0] = 0;
+  if (!W || !q || !scales) return set_error(NVFP4WS_ERR_INVALID_ARG, "fp8_pack: null pointer");
+  if (N < 1 || K < 16 || K % 16 != 0 || K > (int64_t)65535 * kFp8Block || N > (int64_t)0x7fffffff * kFp8Block)
+    return set_error(NVFP4WS_ERR_INVALID_ARG, "fp8_pack: need N >= 1 and K a multiple of 16 in [16, 8388480]");
+  if (!aligned16(W) || !aligned16(q)) return set_error(NVFP4WS_ERR_MISALIGNED, "fp8_pack: W and q must be 16-byte aligned");
+  if ((uintptr_t)scales & 3u) return set_error(NVFP4WS_ERR_MISALIGNED, "fp8_pack: scales must be 4-byte aligned");
+  return launch_fp8_pack(W, N, K, q, scales, (cudaStream_t)stream);
+}
+
+size_t fp8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) { return fp8_gemm_workspace_bytes_int(M, N, K); }
+
+size_t fp8_lmhead_verify_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  return fp8_verify_workspace_bytes_int(M, N, K);
+}
+
+static int validate_fp8(const void* X, const uint8_t* q, const float* scales, int64_t M, int64_t N, int64_t K,
+                        void* workspace, size_t workspace_bytes, size_t need, const char* who) {
+  if (!X || !q || !scales) return set_error(NVFP4WS_ERR_INVALID_ARG, "%s: null input pointer", who);
+  if (M < 1 || N < 1 || K < 1) return set_error(NVFP4WS_ERR_INVALID_ARG, "%s: M, N, K must be >= 1", who);
+  if (N > (int64_t)0x7fffffff) return set_error(NVFP4WS_ERR_UNSUPPORTED, "%s: N too large", who);
+  if (!fp8_supported(M, K))
+    return set_error(NVFP4WS_ERR_UNSUPPORTED, "%s: needs 1 <= M <= 128 and K a positive multiple of 128 (M=%lld K=%lld)",
+                     who, (long long)M, (long long)K);
+  if (!aligned16(X) || !aligned16(q)) return set_error(NVFP4WS_ERR_MISALIGNED, "%s: X and q must be 16-byte aligned", who);
+  if ((uintptr_t)scales & 3u) return set_error(NVFP4WS_ERR_MISALIGNED, "%s: scales must be 4-byte aligned", who);
+  if (workspace == nullptr || workspace_bytes < need)
+    return set_error(NVFP4WS_ERR_WORKSPACE, "%s: workspace needs %zu bytes", who, need);
+  if (!aligned16(workspace)) return set_error(NVFP4WS_ERR_MISALIGNED, "%s: workspace must be 16-byte aligned", who);
+  return NVFP4WS_OK;
+}
+
+int fp8_gemm_skinny(const void* X, const uint8_t* q, const float* scales, int64_t M, int64_t N, int64_t K, void* Y,
+                    int y_dtype, void* workspace, size_t workspace_bytes, nvfp4ws_stream_t stream) {
+  g_last_error[0] = 0;
+  if (!Y) return set_error(NVFP4WS_ERR_INVALID_ARG, "fp8_gemm_skinny: Y is null");
+  if (y_dtype != NVFP4WS_Y_F32 && y_dtype != NVFP4WS_Y_BF16)
+    return set_error(NVFP4WS_ERR_INVALID_ARG, "fp8_gemm_skinny: bad y_dtype %d", y_dtype);
+  if (int e = validate_fp8(X, q, scales, M, N, K, workspace, workspace_bytes, fp8_gemm_workspace_bytes_int(M, N, K),
+                           "fp8_gemm_skinny"))
+    return e;
+  if (!aligned16(Y)) return set_error(NVFP4WS_ERR_MISALIGNED, "fp8_gemm_skinny: Y must be 16-byte aligned");
+  return launch_fp8_gemm(static_cast<const uint16_t*>(X), q, scales, M, N, K, Y, y_dtype, workspace,
+                         (cudaStream_t)stream);
+}
+
+int fp8_lmhead_verify(const void* X, const uint8_t* q, const float* scales, int64_t M, int64_t N, int64_t K,
+                      const nvfp4_verify_spec* verify, void* workspace, size_t workspace_bytes,
+                      nvfp4ws_stream_t stream) {
+  g_last_error[0] = 0;
+  if (!verify) return set_error(NVFP4WS_ERR_INVALID_ARG, "fp8_lmhead_verify: verify is null");
+  const int32_t B = verify->B, D = verify->D;
+  if (B < 1 || D < 0) return set_error(NVFP4WS_ERR_INVALID_ARG, "fp8_lmhead_verify: need B >= 1 and D >= 0");
+  if ((int64_t)B * (D + 1) != M)
+    return set_error(NVFP4WS_ERR_INVALID_ARG, "fp8_lmhead_verify: M=%lld must equal B*(D+1)=%lld", (long long)M,
+                     (long long)B * (D + 1));
+  if (D > 0 && !verify->drafts) return set_error(NVFP4WS_ERR_INVALID_ARG, "fp8_lmhead_verify: drafts is null");
+  if (!verify->argmax || !verify->accept_len)
+    return set_error(NVFP4WS_ERR_INVALID_ARG, "fp8_lmhead_verify: null output pointer");
+  if (int e = validate_fp8(X, q, scales, M, N, K, workspace, workspace_bytes, fp8_verify_workspace_bytes_int(M, N, K),
+                           "fp8_lmhead_verify"))
+    return e;
+  const VerifyRule v{verify->drafts, D > 0 ? verify->parents : nullptr, B, D, verify->argmax, verify->accept_len,
+                     verify->accept_node, verify->max_logit};
+  return launch_fp8_verify(static_cast<const uint16_t*>(X), q, scales, M, N, K, v, workspace, (cudaStream_t)stream);
 }
 
 int nvfp4ws_check(nvfp4ws_stream_t stream) {

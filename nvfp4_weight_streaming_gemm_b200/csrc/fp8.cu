@@ -1,0 +1,623 @@
+// FP8 (E4M3) block-scaled weight GEMM and fused verify on the tcgen05 tensor cores (sm_100a).
+//
+//   Y[m, n] = sum_kb s[n / 128, kb] * sum_{k in block kb} x16[m, k] * e4m3(code[n, k])
+//
+// The weight format is one E4M3 code per element and one fp32 scale per 128 x 128 block
+// (rows x K), s = fp32(amax_block / 448) ("TandemLLM", "The parts": an FP8 e4m3 output head;
+// "Qwen3.8 on DGX Spark (GB10)", the model list: FP8 block-scaled projections). The pages
+// name no block shape; 128 x 128 is the reading taken here.
+//
+// Exactness. An E4M3 value has at most 4 significant bits and lies in [2^-9, 448], so it is
+// exact in f16, as is the activation for |x| in [2^-14, 65504] (bf16 -> f16, nearest,
+// saturating). Every product is then exact in the fp32 accumulator. The block scale is an
+// arbitrary fp32 and would round if folded into either f16 operand, so a unit of work is one
+// 128 x 128 block: the tensor core sums the block's 128 products per (row, token) into a fresh
+// TMEM buffer P, and the epilogue promotes it into a running sum R = s * P, then R += s * P,
+// in fp32 (R also lives in TMEM).
+//
+// Roles per CTA (one persistent CTA per SM, 16 warps):
+//   warp 0        TMA producer: the 16 KB code tile (128 rows x 128 B, 128-byte swizzle) and
+//                 the unit's bf16 X slice (two 64-wide swizzled atoms) into a ring of stages.
+//                 No multicast.
+//   warp 1        TMEM allocator and the single MMA-issuing thread: 8 x kind::f16 (K = 16)
+//                 per unit, A from TMEM, B from shared memory, into one of np rotating P
+//                 buffers.
+//   warps 4-7,    two dequantisation warpgroups taking alternate units. Each thread owns one
+//   warps 8-11    weight row (its TMEM lane): E4M3 pairs -> f16 pairs (cvt.rn.f16x2.e4m3x2)
+//                 written into TMEM as the A operand. The same threads convert the unit's X
+//                 rows from bf16 to f16 in place.
+//   warps 12-15   promotion and epilogue: at the end of a tile's K range, Y (or the tile's
+//                 per-token argmax in verify mode, or a split-K partial).
+//
+// TMEM columns (512, one CTA per SM): [0, 64) and [64, 128) the two A buffers (64 f16 pairs
+// per row), [128, 128 + npad) R, then np P buffers of npad columns.
+//
+// Scheduling is stream-K: the (tile, K-block) units are cut into equal contiguous ranges, one
+// per CTA. A tile whose K range spans several CTAs is finished by the last to arrive: each
+// publishes its fp32 partial, takes a ticket, and the holder of the last ticket sums the
+// partials in K order, so results are deterministic and no CTA waits for another. Every
+// mbarrier wait is bounded; on expiry the thread records kDevErrWaitTimeout and the CTA
+// winds down (drains its copies and MMAs, frees its TMEM).
+#include "common.cuh"
+#include "fp8.h"
+#include "kernels.h"
+#include "sync.cuh"
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <climits>
+#include <cmath>
+
+namespace nvfp4ws {
+namespace fp8k {
+
+constexpr int kThreads = 512;
+constexpr int kTileRows = 128;
+constexpr int kKB = kFp8Block;                       // K elements per unit = one scale block
+constexpr uint32_t kWBytes = kTileRows * kKB;        // 16 KB of codes per unit
+constexpr int kMaxNpad = 128;
+constexpr int kACols = kKB / 2;                      // f16 pairs per row = TMEM columns per A buffer
+constexpr uint32_t kRCol = 2 * kACols;               // running sums after the two A buffers
+constexpr int kMaxP = 4;
+constexpr int kMaxStages = 8;
+constexpr size_t kTailBytes = 8192;
+
+struct Params {
+  float* Y;                // fp32 or bf16 (y_bf16)
+  int y_bf16;
+  const float* scales;     // [tiles][kbs]
+  int M, npad, np;
+  long long N, K;
+  int tiles, kbs;
+  long long units;
+  int grid;
+  int stages;
+  uint32_t stage_bytes;
+  unsigned int* counters;  // [tiles], zero between calls
+  float* partials;         // [2 * grid][M][128]
+  int verify;
+  float* part_val;         // [tiles][M]
+  int* part_idx;
+  unsigned int* err;
+};
+
+// ---------------------------------------------------------------- PTX helpers
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+
+// D[128 x N] (+)= A[128 x 16] (TMEM, f16) * B[16 x N] (shared memory, f16), fp32 accumulation.
+__device__ __forceinline__ void tc_mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{ .reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p; }" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_st_x32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
+      "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+      "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_st_x16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_ld_x16(uint32_t taddr, uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
+        "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups 1024 B apart.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFF) >> 4);          // start address
+  d |= (uint64_t)1 << 16;                           // leading byte offset (unused for swizzled K-major)
+  d |= (uint64_t)(1024 >> 4) << 32;                 // stride byte offset
+  d |= (uint64_t)1 << 46;                           // descriptor version (sm_100)
+  d |= (uint64_t)2 << 61;                           // SWIZZLE_128B
+  return d;
+}
+
+// ---------------------------------------------------------------- schedule helpers
+
+__device__ __forceinline__ long long unit_begin(long long c, long long U, int G) { return c * U / G; }
+
+__device__ __forceinline__ int cta_of_unit(long long u, long long U, int G) {
+  int c = (int)(u * G / U);
+  while (c + 1 < G && unit_begin(c + 1, U, G) <= u) ++c;
+  while (c > 0 && unit_begin(c, U, G) > u) --c;
+  return c;
+}
+
+// ---------------------------------------------------------------- epilogue pieces
+
+// Writes y for tokens [m0, m0+16) of weight row n.
+__device__ __forceinline__ void write_y(const Params& p, long long n, int m0, const float (&y)[16]) {
+  if (n >= p.N) return;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const int m = m0 + j;
+    if (m < p.M) {
+      if (p.y_bf16)
+        reinterpret_cast<uint16_t*>(p.Y)[(long long)m * p.N + n] = f32_to_bf16_rn(y[j]);
+      else
+        p.Y[(long long)m * p.N + n] = y[j];
+    }
+  }
+}
+
+// Per-token argmax over the 32 rows of this warp; lane 0 stages the warp's winner.
+__device__ __forceinline__ void warp_argmax(const Params& p, long long n, int m0, const float (&y)[16], float* s_val,
+                                            int* s_idx, int q, int lane) {
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    float v = (n < p.N) ? y[j] : -INFINITY;
+    int i = (n < p.N) ? (int)n : INT_MAX;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, v, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, i, o);
+      if (argmax_better(ov, oi, v, i)) { v = ov; i = oi; }
+    }
+    if (lane == 0) { s_val[q * kMaxNpad + m0 + j] = v; s_idx[q * kMaxNpad + m0 + j] = i; }
+  }
+}
+
+// Combines the 4 warps' staged winners into the tile's partial (one thread per token).
+__device__ __forceinline__ void tile_argmax_out(const Params& p, int tile, int et, const float* s_val,
+                                                const int* s_idx) {
+  if (et >= p.M) return;
+  float bv = s_val[et];
+  int bi = s_idx[et];
+  for (int w = 1; w < 4; ++w)
+    if (argmax_better(s_val[w * kMaxNpad + et], s_idx[w * kMaxNpad + et], bv, bi)) {
+      bv = s_val[w * kMaxNpad + et];
+      bi = s_idx[w * kMaxNpad + et];
+    }
+  p.part_val[(long long)tile * p.M + et] = bv;
+  p.part_idx[(long long)tile * p.M + et] = bi;
+}
+
+// ---------------------------------------------------------------- the kernel
+
+__global__ void __launch_bounds__(kThreads, 1)
+    fp8_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x, const Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int S = p.stages, NP = p.np;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)S * p.stage_bytes);
+  // [0,S) full, [S,2S) empty, 2S+{0,1} a_full, 2S+{2,3} a_empty, 2S+4+b p_full, 2S+4+kMaxP+b p_empty,
+  // 2S+4+2kMaxP drain
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 2 * S + 5 + 2 * kMaxP);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+  int* s_last = reinterpret_cast<int*>(s_tmem + 2);
+  float* s_val = reinterpret_cast<float*>(s_tmem + 4);                  // [4][kMaxNpad]
+  int* s_idx = reinterpret_cast<int*>(s_val + 4 * kMaxNpad);            // [4][kMaxNpad]
+
+  auto bar_full = [&](int s) { return smem_u32(bars + s); };
+  auto bar_empty = [&](int s) { return smem_u32(bars + S + s); };
+  auto bar_afull = [&](int g) { return smem_u32(bars + 2 * S + g); };
+  auto bar_aempty = [&](int g) { return smem_u32(bars + 2 * S + 2 + g); };
+  auto bar_pfull = [&](int b) { return smem_u32(bars + 2 * S + 4 + b); };
+  auto bar_pempty = [&](int b) { return smem_u32(bars + 2 * S + 4 + kMaxP + b); };
+  const uint32_t bar_drain = smem_u32(bars + 2 * S + 4 + 2 * kMaxP);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = blockIdx.x;
+  const long long U = p.units;
+  const long long u_begin = unit_begin(c, U, p.grid), u_end = unit_begin(c + 1, U, p.grid);
+  const int nunits = (int)(u_end - u_begin);
+  const int npad = p.npad, kbs = p.kbs;
+  const uint32_t pcol0 = kRCol + (uint32_t)npad;   // first P buffer
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) { mbar_init(bar_full(s), 1); mbar_init(bar_empty(s), 1); }
+    for (int g = 0; g < 2; ++g) { mbar_init(bar_afull(g), 128); mbar_init(bar_aempty(g), 1); }
+    for (int b = 0; b < kMaxP; ++b) { mbar_init(bar_pfull(b), 1); mbar_init(bar_pempty(b), 128); }
+    mbar_init(bar_drain, 1);
+    *s_abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {   // whole warp allocates all 512 TMEM columns (one CTA per SM)
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(s_tmem)),
+                 "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first(), pol_x = policy_evict_last();
+      const uint32_t tx = kWBytes + (uint32_t)npad * 256u;
+      int issued = 0;
+      long long tile = u_begin / kbs;
+      int kb = (int)(u_begin % kbs);
+      int s = 0;
+      uint32_t ph = 0;
+      for (int i = 0; i < nunits; ++i) {
+        if (!mbar_wait(bar_empty(s), ph ^ 1u, s_abort, p.err)) break;
+        uint8_t* st = smem + (size_t)s * p.stage_bytes;
+        mbar_arrive_expect_tx(bar_full(s), tx);
+        tma_load_2d(smem_u32(st), &tm_w, kb * kKB, (int)(tile * kTileRows), bar_full(s), pol_w);
+#pragma unroll
+        for (int a = 0; a < 2; ++a)
+          tma_load_2d(smem_u32(st + kWBytes + a * npad * 128), &tm_x, kb * kKB + a * 64, 0, bar_full(s), pol_x);
+        issued = i + 1;
+        if (++kb == kbs) { kb = 0; ++tile; }
+        if (++s == S) { s = 0; ph ^= 1u; }
+      }
+      if (*s_abort) {       // drain: wait (bounded) for every copy this thread issued
+        for (int i = (issued > S ? issued - S : 0); i < issued; ++i) {
+          const unsigned long long t0 = globaltimer();
+          while (!mbar_try_wait(bar_full(i % S), (uint32_t)(i / S) & 1u) && globaltimer() - t0 < kWaitLimitNs) {}
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      // kind::f16: f32 accumulator, A and B f16, both K-major, N = npad, M = 128
+      const uint32_t idesc = (1u << 4) | ((uint32_t)(npad >> 3) << 17) | ((uint32_t)(kTileRows >> 4) << 24);
+      int s = 0;
+      uint32_t ph = 0;
+      for (int i = 0; i < nunits; ++i) {
+        const int g = i & 1, b = i % NP, k = i / NP;
+        const bool ok = mbar_wait(bar_pempty(b), ((uint32_t)k & 1u) ^ 1u, s_abort, p.err) &&
+                        mbar_wait(bar_full(s), ph, s_abort, p.err) &&
+                        mbar_wait(bar_afull(g), (uint32_t)(i >> 1) & 1u, s_abort, p.err);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t xbase = smem_u32(smem + (size_t)s * p.stage_bytes + kWBytes);
+        const uint32_t d_tmem = tmem + pcol0 + (uint32_t)(b * npad);
+        const uint32_t a_tmem = tmem + (uint32_t)(g * kACols);
+#pragma unroll
+        for (int kk = 0; kk < kKB / 16; ++kk) {
+          const uint64_t bdesc = sw128_desc(xbase + (kk >> 2) * npad * 128 + (kk & 3) * 32);
+          tc_mma_f16_ts(d_tmem, a_tmem + kk * 8, bdesc, idesc, kk == 0 ? 0u : 1u);
+        }
+        tc_commit(bar_empty(s));       // stage reusable once these MMAs retire
+        tc_commit(bar_aempty(g));      // A buffer reusable
+        tc_commit(bar_pfull(b));       // the block's sums are ready for promotion
+        if (++s == S) { s = 0; ph ^= 1u; }
+      }
+      tc_commit(bar_drain);            // completes when every MMA issued above has retired
+      const unsigned long long t0 = globaltimer();
+      while (!mbar_try_wait(bar_drain, 0) && globaltimer() - t0 < kWaitLimitNs) {}
+    }
+  } else if (warp >= 4 && warp < 12) {
+    // ------------------------------------------------------------ dequantisation warpgroups
+    const int g = (warp - 4) >> 2;                   // warpgroup 0 or 1
+    const int q = warp & 3;                          // TMEM lane quarter
+    const int r = q * 32 + lane;                     // row within the tile
+    const int tg = threadIdx.x - (4 + 4 * g) * 32;   // 0..127 within the warpgroup
+    int s = g % S;
+    uint32_t ph = (uint32_t)(g / S) & 1u;
+    for (int i = g; i < nunits; i += 2) {
+      if (i != g) {                                   // advance the ring position by two units
+        s += 2;
+        if (s >= S) { s -= S; ph ^= 1u; }
+      }
+      if (!mbar_wait(bar_full(s), ph, s_abort, p.err)) break;
+      if (!mbar_wait(bar_aempty(g), ((uint32_t)(i >> 1) & 1u) ^ 1u, s_abort, p.err)) break;
+      tc_fence_after();
+      uint8_t* st = smem + (size_t)s * p.stage_bytes;
+      // X slice: bf16 -> f16 in place (rows < M; TMA zero-filled the rest)
+      {
+        uint8_t* xs = st + kWBytes;
+        const int words = 2 * p.M * 8;               // 16-byte words: 2 atoms x M rows x 8
+        for (int w = tg; w < words; w += 128) {
+          const int a = w / (p.M * 8), rem = w - a * (p.M * 8);
+          uint4* ptr = reinterpret_cast<uint4*>(xs + a * npad * 128 + (rem >> 3) * 128 + (rem & 7) * 16);
+          uint4 v = *ptr;
+          v.x = bf16x2_to_f16x2_sat(v.x); v.y = bf16x2_to_f16x2_sat(v.y);
+          v.z = bf16x2_to_f16x2_sat(v.z); v.w = bf16x2_to_f16x2_sat(v.w);
+          *ptr = v;
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      }
+      // weight row r: 128 codes in eight swizzled 16-byte chunks -> 64 f16 pairs in TMEM
+      const uint8_t* row = st + r * 128;
+      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(g * kACols);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t out[32];
+#pragma unroll
+        for (int j2 = 0; j2 < 4; ++j2) {
+          const int j = half * 4 + j2;                // logical chunk: elements 16j .. 16j+15
+          const uint4 w = *reinterpret_cast<const uint4*>(row + ((j ^ (r & 7)) << 4));
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int e = 0; e < 8; ++e) out[j2 * 8 + e] = e4m3x2_to_f16x2(ww[e >> 1] >> ((e & 1) * 16));
+        }
+        tc_st_x32(taddr + half * 32, out);
+      }
+      tc_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar_afull(g));
+    }
+  } else if (warp >= 12) {
+    // ------------------------------------------------------------ promotion and epilogue warpgroup
+    const int q = warp & 3;
+    const int rowl = q * 32 + lane;
+    const int et = threadIdx.x - 12 * 32;            // 0..127
+    const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
+    long long tile_it = u_begin / kbs;
+    int kb_it = (int)(u_begin % kbs);
+    for (int i = 0; i < nunits; ++i) {
+      const long long u = u_begin + i;
+      const long long tile = tile_it;
+      const int kb = kb_it;
+      const bool seg_first = (i == 0) || (kb == 0);
+      const bool seg_last = (i == nunits - 1) || (kb == kbs - 1);
+      if (++kb_it == kbs) { kb_it = 0; ++tile_it; }
+      const int b = i % NP, k = i / NP;
+      const float sc = __ldg(p.scales + tile * kbs + kb);
+      // Every thread reaches the barrier, so a give-up seen by any of them ends the loop for all.
+      mbar_wait(bar_pfull(b), (uint32_t)k & 1u, s_abort, p.err);
+      named_bar(1, 128);
+      if (ld_shared_volatile(s_abort)) break;
+      tc_fence_after();
+      const long long n = tile * kTileRows + rowl;
+      const long long tile_u0 = tile * kbs, tile_u1 = tile_u0 + kbs;
+      const long long seg_u0 = u_begin > tile_u0 ? u_begin : tile_u0;
+      const bool complete = (seg_u0 == tile_u0) && (u + 1 == tile_u1);
+      const int slot = (seg_u0 == u_begin) ? 2 * c : 2 * c + 1;
+      const uint32_t pcol = pcol0 + (uint32_t)(b * npad);
+      for (int m0 = 0; m0 < p.M; m0 += 16) {
+        uint32_t pv[16], rv[16];
+        tc_ld_x16(lane_base + pcol + m0, pv);
+        if (!seg_first) tc_ld_x16(lane_base + kRCol + m0, rv);
+        tc_wait_ld();
+        float y[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          y[j] = seg_first ? sc * __uint_as_float(pv[j]) : fmaf(sc, __uint_as_float(pv[j]), __uint_as_float(rv[j]));
+        if (!seg_last) {
+          uint32_t o[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(y[j]);
+          tc_st_x16(lane_base + kRCol + m0, o);
+        } else if (complete) {
+          if (p.verify) warp_argmax(p, n, m0, y, s_val, s_idx, q, lane);
+          else write_y(p, n, m0, y);
+        } else {
+          float* dst = p.partials + ((long long)slot * p.M) * kTileRows;
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (m0 + j < p.M) dst[(long long)(m0 + j) * kTileRows + rowl] = y[j];
+        }
+      }
+      if (!seg_last) tc_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar_pempty(b));
+      if (!seg_last) continue;
+      if (complete) {
+        if (p.verify) {
+          named_bar(1, 128);
+          tile_argmax_out(p, (int)tile, et, s_val, s_idx);
+          named_bar(1, 128);
+        }
+        continue;
+      }
+      // split tile: publish the partial, take a ticket; the last arrival finishes the tile
+      __threadfence();
+      named_bar(1, 128);
+      if (et == 0) {
+        const int c0 = cta_of_unit(tile_u0, U, p.grid), c1 = cta_of_unit(tile_u1 - 1, U, p.grid);
+        int expected = 0;
+        for (int cc = c0; cc <= c1; ++cc)
+          if (unit_begin(cc + 1, U, p.grid) > unit_begin(cc, U, p.grid)) ++expected;
+        const unsigned int prev = atomicAdd(p.counters + tile, 1u);
+        *s_last = (prev + 1 == (unsigned int)expected) ? 1 : 0;
+      }
+      named_bar(1, 128);
+      if (*s_last) {
+        __threadfence();
+        const int c0 = cta_of_unit(tile_u0, U, p.grid), c1 = cta_of_unit(tile_u1 - 1, U, p.grid);
+        for (int m0 = 0; m0 < p.M; m0 += 16) {
+          float y[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) y[j] = 0.0f;
+          for (int cc = c0; cc <= c1; ++cc) {
+            const long long b0 = unit_begin(cc, U, p.grid), b1 = unit_begin(cc + 1, U, p.grid);
+            if (b1 <= b0) continue;
+            const int sl = (b0 >= tile_u0) ? 2 * cc : 2 * cc + 1;
+            const float* src = p.partials + ((long long)sl * p.M) * kTileRows;
+            float v[16];   // all loads of the chunk first: one L2 round trip per contributor
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              v[j] = (m0 + j < p.M) ? __ldcg(src + (long long)(m0 + j) * kTileRows + rowl) : 0.f;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) y[j] += v[j];
+          }
+          if (p.verify) warp_argmax(p, n, m0, y, s_val, s_idx, q, lane);
+          else write_y(p, n, m0, y);
+        }
+        if (p.verify) {
+          named_bar(1, 128);
+          tile_argmax_out(p, (int)tile, et, s_val, s_idx);
+        }
+        if (et == 0) p.counters[tile] = 0u;          // ready for the next call
+      }
+      named_bar(1, 128);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+  }
+}
+
+}  // namespace fp8k
+
+// ============================================================================ host side
+
+using namespace fp8k;
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn_fp8() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* f = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  return fn;
+}
+
+static bool make_map_fp8(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+                         uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  auto fn = encode_fn_fp8();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool fp8_supported(long long M, long long K) {
+  return M >= 1 && M <= kMaxNpad && K >= kKB && K % kKB == 0 && K / kKB <= (1ll << 24);
+}
+
+struct Fp8Plan {
+  int npad, np, tiles, kbs, grid, stages;
+  long long units;
+  uint32_t stage_bytes;
+  size_t smem;
+};
+
+static Fp8Plan fp8_plan(long long M, long long N, long long K) {
+  Fp8Plan pl{};
+  pl.npad = (int)std::max<long long>(16, (M + 15) / 16 * 16);
+  pl.np = std::min(kMaxP, (int)((512 - kRCol - pl.npad) / pl.npad));
+  pl.tiles = (int)((N + kTileRows - 1) / kTileRows);
+  pl.kbs = (int)(K / kKB);
+  pl.units = (long long)pl.tiles * pl.kbs;
+  const int sms = std::max(1, device_sm_count());
+  pl.grid = (int)std::min<long long>(sms, pl.units);
+  pl.stage_bytes = kWBytes + (uint32_t)pl.npad * 256u;
+  const size_t budget = 227 * 1024 - 1024 - kTailBytes;
+  pl.stages = (int)std::min<size_t>(kMaxStages, budget / pl.stage_bytes);
+  pl.smem = 1024 + (size_t)pl.stages * pl.stage_bytes + kTailBytes;
+  return pl;
+}
+
+static size_t al256_fp8(size_t v) { return (v + 255) / 256 * 256; }
+
+size_t fp8_gemm_workspace_bytes_int(long long M, long long N, long long K) {
+  if (!fp8_supported(M, K) || N < 1) return 0;
+  const Fp8Plan pl = fp8_plan(M, N, K);
+  return al256_fp8((size_t)pl.tiles * 4) + al256_fp8((size_t)2 * pl.grid * M * kTileRows * 4);
+}
+
+size_t fp8_verify_workspace_bytes_int(long long M, long long N, long long K) {
+  if (!fp8_supported(M, K) || N < 1) return 0;
+  const Fp8Plan pl = fp8_plan(M, N, K);
+  return fp8_gemm_workspace_bytes_int(M, N, K) + 2 * al256_fp8((size_t)pl.tiles * M * 4);
+}
+
+static int launch_fp8(const uint16_t* X, const uint8_t* q, const float* scales, long long M, long long N,
+                      long long K, void* Y, int y_dtype, void* workspace, bool verify, float** pv_out, int** pi_out,
+                      int* nparts_out, cudaStream_t s) {
+  const Fp8Plan pl = fp8_plan(M, N, K);
+  alignas(64) CUtensorMap tw, tx;
+  if (!make_map_fp8(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, K, N, K, kKB, kTileRows) ||
+      !make_map_fp8(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, pl.npad))
+    return set_error(NVFP4WS_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  Params p{};
+  p.Y = static_cast<float*>(Y);
+  p.y_bf16 = (y_dtype == NVFP4WS_Y_BF16);
+  p.scales = scales;
+  p.M = (int)M;
+  p.npad = pl.npad;
+  p.np = pl.np;
+  p.N = N;
+  p.K = K;
+  p.tiles = pl.tiles;
+  p.kbs = pl.kbs;
+  p.units = pl.units;
+  p.grid = pl.grid;
+  p.stages = pl.stages;
+  p.stage_bytes = pl.stage_bytes;
+  char* ws = static_cast<char*>(workspace);
+  p.counters = reinterpret_cast<unsigned int*>(ws);
+  p.partials = reinterpret_cast<float*>(ws + al256_fp8((size_t)pl.tiles * 4));
+  p.verify = verify ? 1 : 0;
+  if (verify) {
+    char* v = ws + fp8_gemm_workspace_bytes_int(M, N, K);
+    p.part_val = reinterpret_cast<float*>(v);
+    p.part_idx = reinterpret_cast<int*>(v + al256_fp8((size_t)pl.tiles * M * 4));
+    *pv_out = p.part_val;
+    *pi_out = p.part_idx;
+    *nparts_out = pl.tiles;
+  }
+  p.err = device_error_word();
+  if (!p.err) return set_error(NVFP4WS_ERR_CUDA, "cannot resolve the device error word");
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    if (cudaFuncSetAttribute(fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
+      return check_launch("cudaFuncSetAttribute(fp8_kernel)");
+    attr_set[dev] = true;
+  }
+  fp8_kernel<<<pl.grid, kThreads, pl.smem, s>>>(tw, tx, p);
+  return check_launch("fp8_kernel");
+}
+
+int launch_fp8_gemm(const uint16_t* X, const uint8_t* q, const float* scales, long long M, long long N, long long K,
+                    void* Y, int y_dtype, void* workspace, cudaStream_t s) {
+  return launch_fp8(X, q, scales, M, N, K, Y, y_dtype, workspace, false, nullptr, nullptr, nullptr, s);
+}
+
+int launch_fp8_verify(const uint16_t* X, const uint8_t* q, const float* scales, long long M, long long N,
+                      long long K, const VerifyRule& v, void* workspace, cudaStream_t s) {
+  float* pv = nullptr;
+  int* pi = nullptr;
+  int nparts = 0;
+  if (int e = launch_fp8(X, q, scales, M, N, K, nullptr, 0, workspace, true, &pv, &pi, &nparts, s)) return e;
+  return launch_verify_stage2(pv, pi, nparts, (int)M, v, s);
+}
+
+}  // namespace nvfp4ws

@@ -1,0 +1,27 @@
+// Internal interface of the FP8 (E4M3, 128 x 128 block-scaled) weight path (not part of the C ABI).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "kernels.h"
+
+namespace nvfp4ws {
+
+// Rows and K elements covered by one fp32 block scale.
+constexpr int kFp8Block = 128;
+
+// The tensor-core kernel's shape limits: 1 <= M <= 128, K a positive multiple of 128.
+bool fp8_supported(long long M, long long K);
+size_t fp8_gemm_workspace_bytes_int(long long M, long long N, long long K);
+size_t fp8_verify_workspace_bytes_int(long long M, long long N, long long K);
+int launch_fp8_gemm(const uint16_t* X, const uint8_t* q, const float* scales, long long M, long long N, long long K,
+                    void* Y, int y_dtype, void* workspace, cudaStream_t s);
+int launch_fp8_verify(const uint16_t* X, const uint8_t* q, const float* scales, long long M, long long N,
+                      long long K, const VerifyRule& v, void* workspace, cudaStream_t s);
+
+// fp32 W [N, K] -> E4M3 codes [N, K] and fp32 scales [ceil(N/128), ceil(K/128)].
+int launch_fp8_pack(const float* W, long long N, long long K, uint8_t* q, float* scales, cudaStream_t s);
+
+}  // namespace nvfp4ws

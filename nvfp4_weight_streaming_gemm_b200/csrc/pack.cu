@@ -11,6 +11,7 @@
 // Three launches: an amax reduction (atomicMax on the bit pattern, exact and
 // order-free), a one-thread finalisation of ts, and one thread per 16-element block.
 #include "common.cuh"
+#include "fp8.h"
 
 #include <algorithm>
 #include <cmath>
@@ -135,6 +136,77 @@ __global__ void __launch_bounds__(256) pack_kernel(const float* __restrict__ W, 
     *reinterpret_cast<uint2*>(q + n * (K / 2) + b * 8) = make_uint2(lo, hi);
     sf[t] = (uint8_t)sbits;
   }
+}
+
+// ---------------------------------------------------------------------------- FP8 block scaling
+//
+// One CTA per 128 x 128 block (rows x K) of W, 256 threads, two per row, 64 elements each:
+//   s    = fp32( amax_block / 448 )                     0 for an all-zero block
+//   code = E4M3_rne_satfinite( w / s ), sign kept       +0 where s = 0
+// The quotient is formed in double precision and rounded once, as for the NVFP4 codes.
+// Blocks at the right and bottom edges hold what remains of W.
+
+__device__ __forceinline__ uint32_t e4m3_code_signed(double r) {
+  const uint32_t sign = signbit(r) ? 0x80u : 0u;
+  return sign | e4m3_bits(e4m3_round(fabs(r)));
+}
+
+__global__ void __launch_bounds__(256) fp8_pack_kernel(const float* __restrict__ W, long long N, long long K,
+                                                       uint8_t* __restrict__ q, float* __restrict__ scales, int kbs) {
+  const long long nb = blockIdx.x;
+  const int kb = blockIdx.y;
+  const int r = threadIdx.x >> 1, h = threadIdx.x & 1;
+  const long long n = nb * 128 + r;
+  const long long k0 = (long long)kb * 128 + h * 64;
+  const bool row_ok = n < N;
+  float amax = 0.0f;
+  if (row_ok) {
+    for (int c = 0; c < 4; ++c) {
+      const long long k = k0 + 16 * c;
+      if (k >= K) break;
+      const float4* src = reinterpret_cast<const float4*>(W + n * K + k);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 v = src[i];
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+      }
+    }
+  }
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  __shared__ float red[8];
+  __shared__ float s_scale;
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float b = 0.0f;
+    for (int w = 0; w < 8; ++w) b = fmaxf(b, red[w]);
+    s_scale = (float)((double)b / 448.0);
+    scales[nb * kbs + kb] = s_scale;
+  }
+  __syncthreads();
+  const double s = (double)s_scale;
+  if (!row_ok) return;
+  for (int c = 0; c < 4; ++c) {
+    const long long k = k0 + 16 * c;
+    if (k >= K) break;
+    const float4* src = reinterpret_cast<const float4*>(W + n * K + k);
+    uint32_t wd[4] = {0u, 0u, 0u, 0u};
+    if (s > 0.0) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 v = src[i];
+        wd[i] = e4m3_code_signed((double)v.x / s) | (e4m3_code_signed((double)v.y / s) << 8) |
+                (e4m3_code_signed((double)v.z / s) << 16) | (e4m3_code_signed((double)v.w / s) << 24);
+      }
+    }
+    *reinterpret_cast<uint4*>(q + n * K + k) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+  }
+}
+
+int launch_fp8_pack(const float* W, long long N, long long K, uint8_t* q, float* scales, cudaStream_t s) {
+  const long long nbs = (N + 127) / 128, kbs = (K + 127) / 128;
+  fp8_pack_kernel<<<dim3((unsigned)nbs, (unsigned)kbs), 256, 0, s>>>(W, N, K, q, scales, (int)kbs);
+  return check_launch("fp8_pack_kernel");
 }
 
 int launch_pack(const float* W, long long N, long long K, uint8_t* q, uint8_t* sf, float* ts,

@@ -88,6 +88,18 @@ def random_case(seed: int, M: int, N: int, K: int, w_std: float = W_STD):
     return normal_weight(rng, N, K, w_std), normal_x_bits(rng, M, K)
 
 
+def block_varied_case(seed: int, M: int, N: int, K: int, block: int = 128, spread: int = 4):
+    """Like ``random_case``, with each ``block x block`` tile of W multiplied by its own power
+    of two 2^e, e ~ U{-spread..spread}: per-block scales then differ by up to 2^(2 spread), so
+    a scale applied to the wrong block is visible in Y."""
+    rng = np.random.default_rng(seed)
+    W = normal_weight(rng, N, K)
+    e = rng.integers(-spread, spread + 1, size=(-(-N // block), -(-K // block)))
+    f = np.repeat(np.repeat(np.ldexp(1.0, e), block, axis=0), block, axis=1)[:N, :K]
+    W = (W * f).astype(np.float32)
+    return W, normal_x_bits(rng, M, K)
+
+
 def lmhead_inputs(N: int = VOCAB, B: int = 1, D: int = DRAFT_LEN, K: int = LMHEAD_K):
     """lm_head weight, hidden states and prefix lengths.
 

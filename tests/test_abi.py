@@ -122,3 +122,27 @@ def test_pass_flags_are_checked_first(lib):
     st = L.PassState()
     assert lib.nvfp4_pass_init_ex(ctypes.byref(st), arr, 1, 17, None, 8, FAKE, 1 << 20) == 1
     assert b"flags" in lib.nvfp4ws_last_error()
+
+
+def test_fp8_rejects_on_the_host(lib):
+    from nvfp4_weight_streaming_gemm_b200 import _lib as L
+    p = lib.fp8_pack
+    assert p(None, 4, 128, FAKE, FAKE, None) == 1
+    assert p(FAKE, 4, 24, FAKE, FAKE, None) == 1                                     # K % 16
+    assert p(FAKE + 4, 4, 128, FAKE, FAKE, None) == 3                                # misaligned W
+    assert p(FAKE, 4, 128, FAKE, FAKE + 2, None) == 3                                # misaligned scales
+    g = lib.fp8_gemm_skinny
+    assert g(None, FAKE, FAKE, 1, 16, 128, FAKE, 0, FAKE, 1 << 30, None) == 1
+    assert g(FAKE, FAKE, FAKE, 129, 16, 128, FAKE, 0, FAKE, 1 << 30, None) == 2      # M > 128
+    assert g(FAKE, FAKE, FAKE, 4, 16, 192, FAKE, 0, FAKE, 1 << 30, None) == 2        # K % 128
+    assert g(FAKE, FAKE, FAKE, 4, 16, 128, FAKE, 2, FAKE, 1 << 30, None) == 1        # bad y dtype
+    assert g(FAKE, FAKE, FAKE, 4, 16, 128, FAKE + 4, 0, FAKE, 1 << 30, None) == 3    # misaligned Y
+    assert g(FAKE, FAKE, FAKE, 4, 16, 128, FAKE, 0, None, 0, None) == 4              # no workspace
+    assert lib.fp8_gemm_workspace_bytes(129, 16, 128) == 0
+    assert lib.fp8_gemm_workspace_bytes(4, 16, 128) > 0
+    v = lib.fp8_lmhead_verify
+    spec = L.VerifySpec(FAKE, 2, 16, FAKE, FAKE, None, None, None)
+    assert v(FAKE, FAKE, FAKE, 17, 100, 128, ctypes.byref(spec), FAKE, 1 << 30, None) == 1   # M != B*(D+1)
+    assert v(FAKE, FAKE, FAKE, 17, 100, 128, None, FAKE, 1 << 30, None) == 1                 # no rule
+    spec = L.VerifySpec(None, 1, 16, FAKE, FAKE, None, None, None)
+    assert v(FAKE, FAKE, FAKE, 17, 100, 128, ctypes.byref(spec), FAKE, 1 << 30, None) == 1   # drafts missing

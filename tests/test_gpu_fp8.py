@@ -1,0 +1,122 @@
+"""GPU parity of the FP8 (E4M3, 128 x 128 block-scaled) weight path against the oracle
+on the same seeded inputs.
+
+Bars:
+* fp8_pack: codes and scales bit-exact (both sides form the quotient in float64 and
+  round once, ties to even).
+* fp8_gemm_skinny: per row max |y - y_ref| <= 1e-5 * max |y_ref|. Each product
+  x * e4m3 is exact in fp32 (both exact in f16); what remains is the fp32 sum inside a
+  block, one rounding for the scale product and the fp32 sum over blocks. bf16 Y is the
+  fp32 result rounded once.
+* fp8_lmhead_verify: argmax bit-exact on rows whose oracle top-2 gap is >= 1e-3; accept
+  length (and end node for a tree) bit-exact on sequences with no near-tie row that can
+  decide them.
+The weights vary by up to 2^16 between blocks, so a scale applied to the wrong block
+misses the bar by orders of magnitude.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import synthetic as S
+from oracle import fp8 as P
+from oracle import verify as V
+
+pytestmark = pytest.mark.gpu
+TOL = 1e-5
+
+
+@pytest.fixture(scope="module")
+def nv():
+    import nvfp4_weight_streaming_gemm_b200 as nv
+    from nvfp4_weight_streaming_gemm_b200 import build
+    build.build()
+    return nv
+
+
+def to_dev_bf16(x_bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(x_bits.view(np.int16).copy()).view(torch.bfloat16).cuda()
+
+
+def rowwise_err(y, y_ref):
+    return (np.abs(y.astype(np.float64) - y_ref).max(axis=1) / np.abs(y_ref).max(axis=1)).max()
+
+
+def packed(nv, W):
+    """Packs on the GPU and checks the bytes against the oracle; returns device and oracle copies."""
+    q, s = nv.fp8_pack(torch.from_numpy(W).cuda())
+    codes_ref, scales_ref = P.quantize_fp8_blocks(W)
+    assert np.array_equal(q.cpu().numpy(), codes_ref)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), scales_ref.view(np.uint32))
+    return q, s, codes_ref, scales_ref
+
+
+@pytest.mark.parametrize("N,K", [(1000, 256), (130, 80), (3, 16), (257, 400)])
+def test_fp8_pack_bit_exact(nv, N, K):
+    W, _ = S.block_varied_case(900 + N, 1, N, K)
+    if N >= 128 and K >= 128:
+        W[:128, :128] = 0.0                                   # an all-zero block: s = 0, codes +0
+    W[-1, :8] = [448.0, -224.0, 8.5, -0.0, 216.0, 1e-30, -1e-30, 0.0]   # saturating, tie, signed-zero cases
+    packed(nv, W)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 1000, 256), (17, 3000, 1024), (68, 777, 768), (128, 4096, 5120),
+                                   (5, 130, 128), (17, 640, 5120), (17, 128, 16384)])
+def test_fp8_gemm(nv, M, N, K):
+    W, x = S.block_varied_case(1000 + M + N, M, N, K)
+    q, s, codes_ref, scales_ref = packed(nv, W)
+    Y = nv.fp8_gemm(to_dev_bf16(x), q, s)
+    nv.check()
+    y_ref = P.gemm_fp8_ref(x, codes_ref, scales_ref)
+    assert rowwise_err(Y.cpu().numpy(), y_ref) <= TOL
+
+
+def test_fp8_gemm_bf16_and_repeat(nv):
+    M, N, K = 17, 2500, 2048
+    W, x = S.block_varied_case(1100, M, N, K)
+    q, s, _, _ = packed(nv, W)
+    X = to_dev_bf16(x)
+    Y1 = nv.fp8_gemm(X, q, s)
+    Y2 = nv.fp8_gemm(X, q, s)
+    Yb = nv.fp8_gemm(X, q, s, y_dtype=torch.bfloat16)
+    nv.check()
+    assert torch.equal(Y1, Y2)                                # fixed sum order: deterministic
+    assert torch.equal(Yb, Y1.to(torch.bfloat16))
+
+
+def test_fp8_verify_chain(nv):
+    B, D, N, K = 1, 16, 20077, 2048
+    W, x = S.random_case(1200, B * (D + 1), N, K, w_std=0.2)
+    q, s, codes_ref, scales_ref = packed(nv, W)
+    y_ref = P.gemm_fp8_ref(x, codes_ref, scales_ref)
+    t_ref = V.argmax_fast(y_ref)
+    Lstar = np.array([9])
+    drafts = S.drafts_with_prefix(t_ref, Lstar, D, N)
+    t, L, _, vmax = nv.fp8_verify(to_dev_bf16(x), q, s, torch.from_numpy(drafts).cuda())
+    nv.check()
+    t, L = t.cpu().numpy(), L.cpu().numpy()
+    gap = V.top2_gap(y_ref)
+    rows = V.comparable_rows(gap)
+    assert rows.all()                                          # no near tie for this seed (oracle-checked)
+    assert np.array_equal(t, t_ref)
+    assert L.tolist() == V.accept_ref(t_ref, drafts, D).tolist() == [9]
+    np.testing.assert_allclose(vmax.cpu().numpy(), y_ref.max(axis=1), rtol=TOL, atol=0)
+
+
+def test_fp8_verify_tree(nv):
+    B, D, N, K = 4, 16, 9000, 1024
+    W, x = S.random_case(1300, B * (D + 1), N, K, w_std=0.2)
+    q, s, codes_ref, scales_ref = packed(nv, W)
+    y_ref = P.gemm_fp8_ref(x, codes_ref, scales_ref)
+    t_ref = V.argmax_fast(y_ref)
+    parents = S.random_tree(B, D, seed=31, chain_bias=0.5)
+    drafts = S.tree_drafts(t_ref, parents, D, N, agree=0.75, seed=32)
+    t, L, node, _ = nv.fp8_verify(to_dev_bf16(x), q, s, torch.from_numpy(drafts).cuda(),
+                                  torch.from_numpy(parents).cuda())
+    nv.check()
+    L_ref, node_ref = V.accept_tree_ref(t_ref, drafts, parents, D)
+    gap = V.top2_gap(y_ref)
+    assert V.comparable_tree_sequences(gap, parents, D).all()  # no near tie for this seed (oracle-checked)
+    assert np.array_equal(t.cpu().numpy(), t_ref)
+    assert np.array_equal(L.cpu().numpy(), L_ref) and np.array_equal(node.cpu().numpy(), node_ref)
