@@ -592,6 +592,62 @@ def run_w4a4(args):
         torch.cuda.synchronize()
 
 
+def run_fp8(args):
+    """The FP8 output head: E4M3 codes with one fp32 scale per 128 x 128 block over the
+    full 248,320 x 5120 vocabulary (1.27 GB, ten times L2), packed on the GPU from a seeded
+    N(0, 0.02) weight. Per M, the fused verify (M a multiple of 17: B sequences of 16 drafts
+    + 1) and the plain GEMM, each timed by CUDA events over `steps` calls after `warmup`.
+    One JSON line per (call, M) with the weight GB/s against the HBM roofline."""
+    import torch
+    import nvfp4_weight_streaming_gemm_b200 as nv
+    from nvfp4_weight_streaming_gemm_b200 import build as nvbuild
+    nvbuild.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    N, K = S.VOCAB, S.LMHEAD_K
+    g = torch.Generator(device=dev)
+    g.manual_seed(S.LMHEAD_W_SEED)
+    W = torch.randn(N, K, generator=g, device=dev) * S.W_STD
+    q, sc = nv.fp8_pack(W)
+    del W
+    wbytes = N * K + sc.numel() * 4
+    hbm, hbm_kind = measured_peaks()
+    st = torch.cuda.current_stream()
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+        ev[0].record(st)
+        for k in range(args.steps):
+            fn()
+            ev[k + 1].record(st)
+        torch.cuda.synchronize()
+        nv.check()
+        per = np.array([ev[k].elapsed_time(ev[k + 1]) for k in range(args.steps)])
+        return ev[0].elapsed_time(ev[-1]) / args.steps, float(per.min())
+
+    for M in [int(m) for m in args.ms.split(",")]:
+        X = torch.randn(M, K, generator=g, device=dev).to(torch.bfloat16)
+        calls = []
+        if M % (S.DRAFT_LEN + 1) == 0:
+            B = M // (S.DRAFT_LEN + 1)
+            drafts = torch.zeros((B, S.DRAFT_LEN), dtype=torch.int32, device=dev)
+            wsv = torch.zeros(int(nv.lib().fp8_lmhead_verify_workspace_bytes(M, N, K)), dtype=torch.uint8, device=dev)
+            calls.append(("verify", lambda: nv.fp8_verify(X, q, sc, drafts, workspace=wsv)))
+        Y = torch.empty((M, N), dtype=torch.float32, device=dev)
+        wsg = torch.zeros(int(nv.lib().fp8_gemm_workspace_bytes(M, N, K)), dtype=torch.uint8, device=dev)
+        calls.append(("gemm", lambda: nv.fp8_gemm(X, q, sc, out=Y, workspace=wsg)))
+        for name, fn in calls:
+            ms, ms_min = timed(fn)
+            gbs = wbytes / (ms * 1e-3) / 1e9
+            print(json.dumps({
+                "metric": f"FP8 lm_head {name} (E4M3, 128x128 fp32 block scales)", "M": M, "N": N, "K": K,
+                "ms": ms, "ms_min": ms_min, "weight_gbs": gbs, "hbm_frac": gbs / hbm, "hbm_peak_kind": hbm_kind,
+                "steps": args.steps, "warmup": args.warmup}), flush=True)
+
+
 def run_reference(args, rank, world):
     """The CPU oracle timed as it stands: each step dequantises and multiplies one qkv
     matrix (5120->10240) in float64 at M=17. That is a bounded sample of the pass, in
@@ -643,6 +699,8 @@ def main():
     ap.add_argument("--binv", action="store_true", help="batch-invariant passes (same row bits for every M)")
     ap.add_argument("--w4a4", action="store_true",
                     help="time W4A4 passes (NVFP4 activations) over the stack at the --ms values, e.g. 128,256")
+    ap.add_argument("--fp8", action="store_true",
+                    help="the FP8 (E4M3, 128x128 block-scaled) output head: verify and GEMM per M")
     ap.add_argument("--sweep", action="store_true", help="time one matrix shape per M and path (no pass)")
     ap.add_argument("--shape", default="gate_up", help="sweep shape: gate_up, down, qkv or lm_head")
     ap.add_argument("--paths", default="auto,gemv,mma")
@@ -657,6 +715,8 @@ def main():
         run_sweep(args)
     elif args.w4a4:
         run_w4a4(args)
+    elif args.fp8:
+        run_fp8(args)
     elif args.impl == "reference":
         run_reference(args, rank, world)
     else:

@@ -10,6 +10,9 @@
 //   code = E2M1_rne_satfinite( w / (S * ts) ), sign of w kept
 // Three launches: an amax reduction (atomicMax on the bit pattern, exact and
 // order-free), a one-thread finalisation of ts, and one thread per 16-element block.
+//
+// The file also holds the FP8 pack (E4M3 codes, one fp32 scale per 128 x 128 block),
+// which shares the double-precision E4M3 rounding.
 #include "common.cuh"
 #include "fp8.h"
 
