@@ -338,6 +338,26 @@ def cpu_baseline(seconds: float = 12.0):
                       f"host has {cores} cores, BLAS threads {blas}"}
 
 
+def cpu_baseline_fp8(seconds: float = 12.0, rows: int = 4096):
+    """The FP8 oracle, as it stands, on a bounded sample of the FP8 head: dequantise + float64
+    GEMM of its first ``rows`` rows (K = 5120) at M=17, repeated until ``seconds`` have passed."""
+    from oracle import fp8 as P8
+    W, x = S.random_case(S.LMHEAD_W_SEED, S.DRAFT_LEN + 1, rows, S.LMHEAD_K)
+    codes, scales = P8.quantize_fp8_blocks(W)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        P8.gemm_fp8_ref(x, codes, scales)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    gbs = reps * (rows * S.LMHEAD_K + scales.size * 4) / el / 1e9
+    cores = len(os.sched_getaffinity(0))
+    return {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{reps} x (dequantise + float64 GEMM) of a {rows} x {S.LMHEAD_K} FP8 head slice at M=17, "
+                      f"{el:.1f} s"}
+
+
 def max_over_ranks(dist, torch, value: float, dev) -> float:
     """The largest of each rank's device-timed value: the slowest replica sets the step
     time of the whole job. ``dist`` is None on one GPU."""
@@ -613,6 +633,7 @@ def run_fp8(args):
     wbytes = N * K + sc.numel() * 4
     hbm, hbm_kind = measured_peaks()
     st = torch.cuda.current_stream()
+    cpu = None if args.no_cpu_baseline else cpu_baseline_fp8(args.cpu_seconds)
 
     def timed(fn):
         for _ in range(args.warmup):
@@ -645,7 +666,7 @@ def run_fp8(args):
             print(json.dumps({
                 "metric": f"FP8 lm_head {name} (E4M3, 128x128 fp32 block scales)", "M": M, "N": N, "K": K,
                 "ms": ms, "ms_min": ms_min, "weight_gbs": gbs, "hbm_frac": gbs / hbm, "hbm_peak_kind": hbm_kind,
-                "steps": args.steps, "warmup": args.warmup}), flush=True)
+                "steps": args.steps, "warmup": args.warmup, "cpu_baseline": cpu}), flush=True)
 
 
 def run_reference(args, rank, world):

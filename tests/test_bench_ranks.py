@@ -81,3 +81,10 @@ def test_reference_arm_prints_on_rank_zero_only():
     with contextlib.redirect_stdout(out):
         b.run_reference(Args(), rank=1, world=2)
     assert out.getvalue() == ""
+
+
+def test_fp8_cpu_baseline_runs_the_oracle():
+    b = _bench()
+    r = b.cpu_baseline_fp8(seconds=0.01, rows=256)
+    assert r["kind"] == "oracle" and r["unit"] == "GB/s" and r["value"] > 0 and r["cores"] >= 1
+    assert "FP8 head slice" in r["sample"]
