@@ -115,3 +115,80 @@ def test_tree_child_row_instead_of_parent_row_caught():
     assert wrong(t, d, p, D) != (case["accept_len"], case["accept_node"])
     L, node = V.accept_tree_ref(t, d, p, D)
     assert (int(L[0]), int(node[0])) == (case["accept_len"], case["accept_node"])
+
+
+# ------------------------------------------------------------------ FP8 block-scaled weights
+
+def _fp8_pins_pass():
+    """The FP8 pins: the hand-worked blocks (scales, codes, dequantised values) and a
+    brute-force GEMM over non-square blocks."""
+    import synthetic as S
+    from oracle import fp8 as P8
+    from oracle import gemm as G
+    with open(os.path.join(GOLDEN, "fp8_blocks.json")) as f:
+        cases = json.load(f)["cases"]
+    for case in cases:
+        W = np.array(case["W"], dtype=np.float32)
+        block = tuple(case["block"])
+        codes, scales = P8.quantize_fp8_blocks(W, block)
+        if scales.tolist() != case["scales"] or codes.tolist() != case["codes"]:
+            return False
+        if P8.dequantize_fp8_blocks(codes, scales, block).tolist() != case["dequant"]:
+            return False
+    W, x = S.random_case(85, 2, 5, 40)
+    codes, scales = P8.quantize_fp8_blocks(W, (2, 8))
+    y = P8.gemm_fp8_ref(x, codes, scales, (2, 8))
+    xf = G.bf16_bits_to_float64(x)
+    for m in range(2):
+        for n in range(5):
+            acc = sum(xf[m, k] * F.E4M3_VALUES[codes[n, k]] * float(scales[n // 2, k // 8]) for k in range(40))
+            if abs(y[m, n] - acc) > 1e-12 * max(1e-30, abs(acc)):
+                return False
+    return True
+
+
+def test_fp8_baseline_passes():
+    assert _fp8_pins_pass()
+
+
+def test_fp8_nvfp4_scale_rule_caught(monkeypatch):
+    """s = amax/6 (the NVFP4 rule) in place of amax/448."""
+    from oracle import fp8 as P8
+    monkeypatch.setattr(P8, "E4M3_MAX", 6.0)
+    assert not _fp8_pins_pass()
+
+
+def test_fp8_ties_away_from_zero_caught(monkeypatch):
+    from oracle import fp8 as P8
+    orig = P8.e4m3_encode
+    monkeypatch.setattr(P8, "e4m3_encode", lambda v: orig(np.asarray(v, np.float64) * (1.0 + 2.0 ** -30)))
+    assert not _fp8_pins_pass()
+
+
+def test_fp8_dropped_sign_caught(monkeypatch):
+    from oracle import fp8 as P8
+    orig = P8.e4m3_encode
+    monkeypatch.setattr(P8, "e4m3_encode", lambda v: orig(np.abs(np.asarray(v, np.float64))))
+    assert not _fp8_pins_pass()
+
+
+def test_fp8_transposed_block_index_caught(monkeypatch):
+    """The scale of block (k // bc, n // br) instead of (n // br, k // bc)."""
+    from oracle import fp8 as P8
+
+    def bad(codes, scales, block=P8.BLOCK):
+        codes = np.asarray(codes, dtype=np.uint8)
+        N, K = codes.shape
+        br, bc = block
+        s = np.asarray(scales, dtype=np.float64)
+        flat = s.reshape(-1)
+        idx = (np.arange(K)[None, :] // bc) * s.shape[1] + (np.arange(N)[:, None] // br)
+        return F.E4M3_VALUES[codes] * flat[np.minimum(idx, flat.size - 1)]
+    monkeypatch.setattr(P8, "dequantize_fp8_blocks", bad)
+    assert not _fp8_pins_pass()
+
+
+def test_fp8_unsigned_dequant_caught(monkeypatch):
+    from oracle import fp8 as P8
+    monkeypatch.setattr(P8, "E4M3_VALUES", np.abs(F.E4M3_VALUES))
+    assert not _fp8_pins_pass()
