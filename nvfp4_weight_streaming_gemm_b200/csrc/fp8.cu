@@ -47,6 +47,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <climits>
 #include <cmath>
 
@@ -491,15 +492,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 using namespace fp8k;
 
+// Looked up once per process; a function-local static is initialised exactly once even
+// when several host threads make their first call together.
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn_fp8() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
     cudaDriverEntryPointQueryResult q;
     void* f = nullptr;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-  }
+      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    return nullptr;
+  }();
   return fn;
 }
 
@@ -594,13 +597,13 @@ static int launch_fp8(const uint16_t* X, const uint8_t* q, const float* scales, 
   }
   p.err = device_error_word();
   if (!p.err) return set_error(NVFP4WS_ERR_CUDA, "cannot resolve the device error word");
-  static bool attr_set[64] = {};
+  static std::atomic<bool> attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
+  if (dev < 64 && !attr_set[dev].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
       return check_launch("cudaFuncSetAttribute(fp8_kernel)");
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
   fp8_kernel<<<pl.grid, kThreads, pl.smem, s>>>(tw, tx, p);
   return check_launch("fp8_kernel");

@@ -25,6 +25,7 @@
 #include "sync.cuh"
 
 #include <algorithm>
+#include <atomic>
 #include <climits>
 #include <cmath>
 
@@ -377,14 +378,14 @@ static int occupancy_of(int T) {
 
 template <int MT, int CPT, int RG>
 static int launch_staged(const GemvArgs& a, const GemvPlan& p, cudaStream_t s) {
-  static bool attr[64] = {};
+  static std::atomic<bool> attr[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 64 && !attr[dev]) {
+  if (dev < 64 && !attr[dev].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(gemv_staged_kernel<MT, CPT, RG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              227 * 1024) != cudaSuccess)
       return check_launch("cudaFuncSetAttribute(gemv_staged_kernel)");
-    attr[dev] = true;
+    attr[dev].store(true, std::memory_order_release);
   }
   gemv_staged_kernel<MT, CPT, RG><<<p.grid, p.threads, p.smem, s>>>(a, p.stages, p.stage_bytes);
   return check_launch("gemv_staged_kernel");

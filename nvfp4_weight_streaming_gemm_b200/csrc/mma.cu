@@ -46,6 +46,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <climits>
 #include <cmath>
 
@@ -507,15 +508,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 using namespace mmak;
 
+// Looked up once per process; a function-local static is initialised exactly once even
+// when several host threads make their first call together.
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
     cudaDriverEntryPointQueryResult q;
     void* f = nullptr;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-  }
+      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    return nullptr;
+  }();
   return fn;
 }
 
@@ -619,13 +622,13 @@ static int launch_mma(const uint16_t* X, const uint8_t* q, const uint8_t* sf, co
   }
   p.err = device_error_word();
   if (!p.err) return set_error(NVFP4WS_ERR_CUDA, "cannot resolve the device error word");
-  static bool attr_set[64] = {};
+  static std::atomic<bool> attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
+  if (dev < 64 && !attr_set[dev].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
       return check_launch("cudaFuncSetAttribute(mma_kernel)");
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
   mma_kernel<<<pl.grid, kThreads, pl.smem, s>>>(tq, tsf, tx, p);
   return check_launch("mma_kernel");
