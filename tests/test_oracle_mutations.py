@@ -192,3 +192,69 @@ def test_fp8_unsigned_dequant_caught(monkeypatch):
     from oracle import fp8 as P8
     monkeypatch.setattr(P8, "E4M3_VALUES", np.abs(F.E4M3_VALUES))
     assert not _fp8_pins_pass()
+
+
+# ------------------------------------------------------------------ W4A4 activation rows
+
+def _w4a4_pins_pass():
+    """The W4A4 pins: the hand-worked rows (row scales, block scales, codes) and a brute-force
+    product over the dequantised rows."""
+    import synthetic as S
+    from oracle import gemm as G
+    with open(os.path.join(GOLDEN, "w4a4_rows.json")) as f:
+        g = json.load(f)
+    rows = np.asarray(g["rows"], dtype=np.float32)
+    bits = (rows.view(np.uint32) >> 16).astype(np.uint16)
+    codes, sf, gs = G.quantize_x_rows(bits)
+    if gs.tolist() != g["g"] or sf.tolist() != g["sf"] or codes.tolist() != g["codes"]:
+        return False
+    W, x = S.random_case(9, 2, 3, 48)
+    q, wsf, ts = F.quantize_nvfp4(W)
+    y = G.gemm_w4a4_ref(x, q, wsf, ts)
+    xc, xs, xg = G.quantize_x_rows(x)
+    wc = F.unpack_codes(q)
+    for m in range(2):
+        for n in range(3):
+            acc = sum(F.E2M1_VALUES[xc[m, k]] * F.E4M3_VALUES[xs[m, k // 16]] * float(xg[m]) *
+                      F.E2M1_VALUES[wc[n, k]] * F.E4M3_VALUES[wsf[n, k // 16]] * float(ts) for k in range(48))
+            if abs(y[m, n] - acc) > 1e-12 * max(1e-30, abs(acc)):
+                return False
+    return True
+
+
+def test_w4a4_baseline_passes():
+    assert _w4a4_pins_pass()
+
+
+def test_w4a4_fp8_style_row_scale_caught(monkeypatch):
+    """g = amax/448 (an FP8 rule) in place of amax/2688."""
+    from oracle import gemm as G
+    monkeypatch.setattr(G, "TENSOR_SCALE_DIVISOR", 448.0)
+    assert not _w4a4_pins_pass()
+
+
+def test_w4a4_dropped_sign_caught(monkeypatch):
+    from oracle import gemm as G
+    orig = G.e2m1_encode
+    monkeypatch.setattr(G, "e2m1_encode", lambda r: orig(np.abs(np.asarray(r, np.float64))))
+    assert not _w4a4_pins_pass()
+
+
+def test_w4a4_ties_away_from_zero_caught(monkeypatch):
+    from oracle import gemm as G
+    orig = G.e2m1_encode
+    monkeypatch.setattr(G, "e2m1_encode", lambda r: orig(np.asarray(r, np.float64) * (1.0 + 2.0 ** -30)))
+    assert not _w4a4_pins_pass()
+
+
+def test_w4a4_block_scale_of_the_wrong_block_caught(monkeypatch):
+    """Dequantisation with the scale of block k // 8 instead of k // 16."""
+    from oracle import gemm as G
+
+    def bad(codes, sf, g):
+        codes = np.asarray(codes)
+        K = codes.shape[1]
+        idx = np.minimum(np.arange(K) // 8, sf.shape[1] - 1)
+        return F.E2M1_VALUES[codes] * F.E4M3_VALUES[sf][:, idx] * np.asarray(g, np.float64)[:, None]
+    monkeypatch.setattr(G, "dequantize_x_rows", bad)
+    assert not _w4a4_pins_pass()
