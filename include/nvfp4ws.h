@@ -362,8 +362,8 @@ int nvfp4_pass_run(const nvfp4_pass* pass, nvfp4ws_stream_t stream);
 /*
  * FP8 weights -- E4M3 codes with one fp32 scale per 128 x 128 block (rows x K).
  *
- * Passages: "TandemLLM", "The parts" (an FP8 e4m3 output head, loaded over the vendor's
- * FP8 checkpoint) and "Qwen3.8 on DGX Spark (GB10)" (FP8 block-scaled projections). The
+ * Passages: "TandemLLM", "The parts" (the lm_head is kept in FP8 E4M3, as the vendor's
+ * checkpoint ships it) and "Qwen3.8 on DGX Spark (GB10)" (block-scaled FP8 projections). The
  * pages give neither the block shape nor the scale rule. This library reads them as
  *   s[i, j] = fp32( amax|W[128i .. 128i+127, 128j .. 128j+127]| / 448 )   0 for a zero block
  *   code    = E4M3_rne_satfinite( w / s ), sign kept                   +0 where s = 0

@@ -3,7 +3,7 @@
 //   Y[m, n] = sum_kb s[n / 128, kb] * sum_{k in block kb} x16[m, k] * e4m3(code[n, k])
 //
 // The weight format is one E4M3 code per element and one fp32 scale per 128 x 128 block
-// (rows x K), s = fp32(amax_block / 448) ("TandemLLM", "The parts": an FP8 e4m3 output head;
+// (rows x K), s = fp32(amax_block / 448) ("TandemLLM", "The parts": the lm_head in FP8 E4M3;
 // "Qwen3.8 on DGX Spark (GB10)", the model list: FP8 block-scaled projections). The pages
 // name no block shape; 128 x 128 is the reading taken here.
 //

@@ -2,14 +2,14 @@
 infrastructure only).
 
 What the pages fix: the output head (and, in the vendor's export, the attention
-projections) are FP8 E4M3 ("TandemLLM", "The parts": "an FP8 (e4m3) output head,
-loaded over the vendor's FP8 checkpoint"; "Qwen3.8 on DGX Spark (GB10)", the flash
-lane's description: "FP8 block-scaled" experts; the 27B export's map: "FP8 on all 48
-linear-attention and 16 self-attention projections").
+projections) are FP8 E4M3. "TandemLLM", "The parts", loads its output head in FP8
+(e4m3) from the vendor's FP8 checkpoint; "Qwen3.8 on DGX Spark (GB10)" describes a
+lane whose experts use block-scaled FP8, and its 27B export keeps every linear-
+and self-attention projection (48 and 16 of them) in FP8.
 
 What the pages leave open, with the reading taken here:
 
-* Scale granularity. "Block-scaled" with no block shape. Reading: one FP32 scale per
+* Scale granularity. Block scaling is named without a block shape. Reading: one FP32 scale per
   block of ``br x bc`` weights (rows x K), 128 x 128 by default, the block shape the
   vendor's FP8 checkpoints use. The block shape is a parameter so that small blocks
   can be worked by hand.

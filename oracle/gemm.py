@@ -2,9 +2,9 @@
 
 The operation is ``Y[M, N] = X[M, K] . dequant(W)[N, K]^T``. X is bf16, W is NVFP4
 and the accumulation is at least fp32. The pages frame this as the weight pass
-that every decode or verify step makes: "TandemLLM", "How it works" ("a decode
-step of a 27B model reads every weight once"), and the veloGB10 page, section
-"Unique aspects: Engineered to the roofline".
+that every decode or verify step makes: "TandemLLM", "How it works" (each decode
+step of the 27B model streams all of its weights once), and the veloGB10 page,
+section "Unique aspects: Engineered to the roofline".
 
 Here both operands are exact in float64: a bf16 value has 8 significant bits and
 a dequantised weight at most 6. The only rounding is in the float64 sums, so the

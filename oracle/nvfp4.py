@@ -1,7 +1,7 @@
 """NVFP4 format, quantiser and dequantiser in plain float64 (oracle; test infrastructure only).
 
-What the pages fix: the weights are "NVFP4 group-16" ("Qwen3.8 on DGX Spark (GB10)",
-section "The seven targets, and switching between them"). That is 4-bit E2M1
+What the pages fix: the weights are NVFP4 with groups of 16 ("Qwen3.8 on DGX Spark
+(GB10)", section "The seven targets, and switching between them"). That is 4-bit E2M1
 values, one FP8 E4M3 scale for every 16 consecutive elements along K, and one
 FP32 scale per tensor.
 
