@@ -77,7 +77,8 @@ const char* nvfp4ws_status_string(int status);
 /* Detail text of the last failing call on this host thread ("" if none). Thread-local storage. */
 const char* nvfp4ws_last_error(void);
 
-/* Library version as major*10000 + minor*100 + patch. */
+/* Library version as major*10000 + minor*100 + patch. 200 added struct_size to
+ * nvfp4_gemm_problem and nvfp4_verify_spec. */
 int nvfp4ws_version(void);
 
 /* Largest M (rows of X) accepted by the GEMM and verify entry points. */
@@ -122,11 +123,12 @@ size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
  * (the pass is weight-bandwidth bound). M = 1 is plain decode, 17 is 16 drafts
  * + 1, and 68 is four sequences sharing one read.
  *
- * Arithmetic of the GEMV and f16 tensor-core paths: each product x * (e2m1 * S) is
- * exact, sums are fp32, and the result is multiplied by ts once, in fp32. X is
- * converted to f16 for the products; that is exact for |x| in [2^-14, 65504].
- * Smaller magnitudes round to f16 subnormals (absolute error below 2^-25); larger
- * ones saturate to 65504.
+ * Arithmetic of the GEMV and f16 tensor-core paths: each row of X is multiplied by a
+ * power of two 2^-e, with e chosen from the row's amax so that amax * 2^-e lies in
+ * [2^14, 2^15), and converted to f16. That is exact for every value above 2^-25 * amax
+ * (smaller ones round to f16 subnormals), and nothing saturates. Each product
+ * x * (e2m1 * S) is then exact, sums are fp32, and the result is multiplied by ts and
+ * by 2^e, in fp32.
  * Arithmetic of the block-scaled path (the default for 2 <= M <= 70 when K % 256 == 0):
  * X is first written as 5 residual NVFP4 terms. Each is a per-row fp32 scale, an
  * E4M3 scale per 16 and E2M1 codes; each term quantises what the previous ones left.
@@ -301,7 +303,13 @@ int lmhead_verify_argmax_accept_path(const void* X, const uint8_t* q, const uint
  *   pass          caller-owned host state, filled by nvfp4_pass_init.
  * Returns NVFP4WS_OK, or INVALID_ARG / UNSUPPORTED / MISALIGNED / WORKSPACE / CUDA.
  */
+/* Both structs below open with struct_size, which the caller sets to the struct's size as
+ * compiled (NVFP4WS_GEMM_PROBLEM_SIZE, NVFP4WS_VERIFY_SPEC_SIZE). A call that gets any other
+ * value returns NVFP4WS_ERR_INVALID_ARG before it reads a further member, so code built
+ * against another version of this header is refused on the host instead of having its
+ * struct read past its end. */
 typedef struct nvfp4_gemm_problem {
+  uint32_t struct_size;    /* = NVFP4WS_GEMM_PROBLEM_SIZE */
   const void* X;
   const uint8_t* q;
   const uint8_t* sf;
@@ -312,9 +320,8 @@ typedef struct nvfp4_gemm_problem {
   int32_t y_dtype;
 } nvfp4_gemm_problem;
 
-/* parents and accept_node were appended in ABI version 101 (nvfp4ws_version()): code
- * built against an older header passes a shorter struct and must be rebuilt. */
 typedef struct nvfp4_verify_spec {
+  uint32_t struct_size;    /* = NVFP4WS_VERIFY_SPEC_SIZE */
   const int32_t* drafts;
   int32_t B;
   int32_t D;
@@ -324,6 +331,9 @@ typedef struct nvfp4_verify_spec {
   const int32_t* parents;
   int32_t* accept_node;
 } nvfp4_verify_spec;
+
+#define NVFP4WS_GEMM_PROBLEM_SIZE ((uint32_t)sizeof(nvfp4_gemm_problem))
+#define NVFP4WS_VERIFY_SPEC_SIZE ((uint32_t)sizeof(nvfp4_verify_spec))
 
 typedef struct nvfp4_pass {
   uint64_t opaque[32];
@@ -420,8 +430,10 @@ int fp8_lmhead_verify(const void* X, const uint8_t* q, const float* scales, int6
  * Calls whose work overlaps on the GPU race on the array.
  * Nothing is allocated: no cudaMalloc, no cudaFree, no allocating library routine.
  *
- * Arguments and result are as for nvfp4_gemm_skinny, restricted to the tensor-core
- * path: 1 <= M <= 128, K a positive multiple of 256, N >= 1.
+ * It always runs the f16 tensor-core kernel (NVFP4WS_PATH_MMA_F16), whatever M is, with
+ * that kernel's arithmetic as nvfp4_gemm_skinny describes it (rows of X shifted by a power
+ * of two, exact f16 products, fp32 sums). Arguments and result are as for
+ * nvfp4_gemm_skinny on that path: 1 <= M <= 128, K a positive multiple of 256, N >= 1.
  * Returns NVFP4WS_ERR_UNSUPPORTED for a shape outside that range, or whose scratch
  * (nvfp4_gemm_workspace_bytes) exceeds the 16 MiB array; otherwise as nvfp4_gemm_skinny.
  */

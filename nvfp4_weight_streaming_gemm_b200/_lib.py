@@ -16,15 +16,23 @@ c_i64, c_i32, c_p, c_sz = ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p, ctype
 
 
 class GemmProblem(ctypes.Structure):
-    """nvfp4_gemm_problem: one GEMM of a weight pass."""
-    _fields_ = [("X", c_p), ("q", c_p), ("sf", c_p), ("tensor_scale", c_p), ("N", c_i64), ("K", c_i64),
-                ("Y", c_p), ("y_dtype", c_i32)]
+    """nvfp4_gemm_problem: one GEMM of a weight pass. ``struct_size`` is filled in by the
+    constructor (the library refuses any other value)."""
+    _fields_ = [("struct_size", ctypes.c_uint32), ("X", c_p), ("q", c_p), ("sf", c_p), ("tensor_scale", c_p),
+                ("N", c_i64), ("K", c_i64), ("Y", c_p), ("y_dtype", c_i32)]
+
+    def __init__(self, *args, **kw):
+        super().__init__(ctypes.sizeof(GemmProblem), *args, **kw)
 
 
 class VerifySpec(ctypes.Structure):
-    """nvfp4_verify_spec: the verify buffers of a pass whose last problem is the lm_head."""
-    _fields_ = [("drafts", c_p), ("B", c_i32), ("D", c_i32), ("argmax", c_p), ("accept_len", c_p),
-                ("max_logit", c_p), ("parents", c_p), ("accept_node", c_p)]
+    """nvfp4_verify_spec: the verify buffers of a pass whose last problem is the lm_head.
+    ``struct_size`` is filled in by the constructor."""
+    _fields_ = [("struct_size", ctypes.c_uint32), ("drafts", c_p), ("B", c_i32), ("D", c_i32), ("argmax", c_p),
+                ("accept_len", c_p), ("max_logit", c_p), ("parents", c_p), ("accept_node", c_p)]
+
+    def __init__(self, *args, **kw):
+        super().__init__(ctypes.sizeof(VerifySpec), *args, **kw)
 
 
 class PassState(ctypes.Structure):

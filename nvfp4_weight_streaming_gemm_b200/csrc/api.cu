@@ -26,6 +26,8 @@ int set_error(int status, const char* fmt, ...) {
   return status;
 }
 
+void clear_error() { g_last_error[0] = 0; }
+
 static std::atomic<unsigned long long> g_launches{0};
 
 int check_launch(const char* what) {
@@ -114,7 +116,7 @@ const char* nvfp4ws_status_string(int status) {
 
 const char* nvfp4ws_last_error(void) { return g_last_error; }
 
-int nvfp4ws_version(void) { return 102; }
+int nvfp4ws_version(void) { return 200; }
 
 int nvfp4ws_sm_count(void) { return device_sm_count(); }
 
@@ -318,9 +320,27 @@ int lmhead_verify_argmax_accept(const void* X, const uint8_t* q, const uint8_t* 
 
 // ------------------------------------------------------------------ weight passes
 
+// A caller built against another version of the header passes structs of another size: refuse
+// them before reading any member past struct_size.
+static int check_problem_sizes(const nvfp4_gemm_problem* problems, int32_t count, const char* who) {
+  for (int32_t i = 0; i < count; ++i)
+    if (problems[i].struct_size != NVFP4WS_GEMM_PROBLEM_SIZE)
+      return set_error(NVFP4WS_ERR_INVALID_ARG, "%s: problem %d: struct_size %u, this library expects %u (rebuild "
+                       "against this nvfp4ws.h)", who, i, problems[i].struct_size, NVFP4WS_GEMM_PROBLEM_SIZE);
+  return NVFP4WS_OK;
+}
+
+static int check_verify_size(const nvfp4_verify_spec* v, const char* who) {
+  if (v->struct_size != NVFP4WS_VERIFY_SPEC_SIZE)
+    return set_error(NVFP4WS_ERR_INVALID_ARG, "%s: verify struct_size %u, this library expects %u (rebuild against "
+                     "this nvfp4ws.h)", who, v->struct_size, NVFP4WS_VERIFY_SPEC_SIZE);
+  return NVFP4WS_OK;
+}
+
 static int to_host_problems(const nvfp4_gemm_problem* problems, int32_t count, int64_t M, int verify_last,
                             std::vector<MxHostProblem>* out, const char* who, int terms = kMxf4Terms) {
   if (!problems || count < 1) return set_error(NVFP4WS_ERR_INVALID_ARG, "%s: need count >= 1 problems", who);
+  if (int e = check_problem_sizes(problems, count, who)) return e;
   const int max_m = std::min(352 / terms, NVFP4WS_MAX_M);
   if (M < 1 || M > max_m || !mxf4_supported(M, 256, terms))
     return set_error(NVFP4WS_ERR_UNSUPPORTED, "%s: M=%lld outside 1..%d", who, (long long)M, max_m);
@@ -378,6 +398,8 @@ int nvfp4_pass_init_ex(nvfp4_pass* pass, const nvfp4_gemm_problem* problems, int
   static_assert(sizeof(nvfp4_pass) >= kMxPassStateBytes, "nvfp4_pass is too small for the pass state");
   if (!pass) return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_pass_init: pass is null");
   std::memset(pass, 0, sizeof(nvfp4_pass));
+  if (verify)
+    if (int e = check_verify_size(verify, "nvfp4_pass_init")) return e;
   std::vector<MxHostProblem> hp;
   if (int e = to_host_problems(problems, count, M, verify != nullptr, &hp, "nvfp4_pass_init", pass_terms(flags)))
     return e;
@@ -459,6 +481,7 @@ int fp8_lmhead_verify(const void* X, const uint8_t* q, const float* scales, int6
                       nvfp4ws_stream_t stream) {
   g_last_error[0] = 0;
   if (!verify) return set_error(NVFP4WS_ERR_INVALID_ARG, "fp8_lmhead_verify: verify is null");
+  if (int e = check_verify_size(verify, "fp8_lmhead_verify")) return e;
   const int32_t B = verify->B, D = verify->D;
   if (B < 1 || D < 0) return set_error(NVFP4WS_ERR_INVALID_ARG, "fp8_lmhead_verify: need B >= 1 and D >= 0");
   if ((int64_t)B * (D + 1) != M)

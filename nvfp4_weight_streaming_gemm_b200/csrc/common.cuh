@@ -13,6 +13,7 @@ namespace nvfp4ws {
 // Host-side error reporting (thread-local detail text)
 // ----------------------------------------------------------------------------
 int set_error(int status, const char* fmt, ...);
+void clear_error();       // every entry point starts with an empty detail text
 int check_launch(const char* what);
 
 // Device error word (one per device, in api.cu). Kernels with bounded waits get
@@ -77,6 +78,49 @@ __device__ __forceinline__ float f16hi_to_f32(uint32_t h2) {
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2_sat(uint32_t b2) {
   float lo = __uint_as_float(b2 << 16);
   float hi = __uint_as_float(b2 & 0xFFFF0000u);
+  uint32_t r;
+  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// ----------------------------------------------------------------------------
+// Per-row power-of-two shift of the activations (the f16 paths)
+// ----------------------------------------------------------------------------
+// A bf16 row is converted to f16 as x * 2^-e, with e chosen from the row's amax so that
+// amax * 2^-e lies in [2^14, 2^15). Every bf16 value (8 significant bits) of the row then
+// converts exactly, nothing saturates, and only values below 2^-25 of the row's amax lose
+// bits (f16 subnormals). Products and fp32 sums of the shifted row are the unshifted ones
+// times 2^-e exactly (barring fp32 underflow), and the epilogue multiplies by 2^e.
+
+// floor(log2(a)) for a finite a > 0, subnormals included.
+__device__ __forceinline__ int floor_log2_pos(float a) {
+  const uint32_t u = __float_as_uint(a);
+  const int ex = (int)((u >> 23) & 0xFFu);
+  if (ex != 0) return ex - 127;
+  return (31 - __clz((int)(u & 0x7FFFFFu))) - 149;          // a = m * 2^-149
+}
+
+// The shift e of a row whose largest magnitude is amax (0 for a zero or non-finite amax).
+__device__ __forceinline__ int row_shift_of_amax(float amax) {
+  return (amax > 0.f && amax <= 3.402823466e38f) ? floor_log2_pos(amax) - 14 : 0;
+}
+
+// v * 2^k for k in [-252, 254], by at most two multiplications by exact powers of two:
+// exact unless the result leaves the normal fp32 range.
+__device__ __forceinline__ float mul_pow2(float v, int k) {
+  if (k > 127) { v *= __uint_as_float(254u << 23); k -= 127; }
+  else if (k < -126) { v *= __uint_as_float(1u << 23); k += 126; }
+  return v * __uint_as_float((uint32_t)(k + 127) << 23);
+}
+
+__device__ __forceinline__ float bf16x2_absmax(uint32_t b2) {
+  return fmaxf(fabsf(__uint_as_float(b2 << 16)), fabsf(__uint_as_float(b2 & 0xFFFF0000u)));
+}
+
+// Two bf16 times 2^-e -> f16x2 (nearest); exact for a row shifted by row_shift_of_amax.
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2_shifted(uint32_t b2, int e) {
+  const float lo = mul_pow2(__uint_as_float(b2 << 16), -e);
+  const float hi = mul_pow2(__uint_as_float(b2 & 0xFFFF0000u), -e);
   uint32_t r;
   asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;

@@ -31,17 +31,9 @@
 
 namespace nvfp4ws {
 
-template <int MT, int CPT, int R, bool VERIFY>
-__global__ void __launch_bounds__(512) gemv_kernel(GemvArgs a) {
-  const int T = blockDim.x;
-  const int t = threadIdx.x;
-  const int lane = t & 31, warp = t >> 5, nwarps = T >> 5;
-  const int C = a.K >> 5;                       // 32-element chunks per row
-  const long long rowq = a.K >> 1;              // bytes of q per row
-  const long long rows = a.K >> 4;              // bytes of sf per row
-
-  // X slice -> registers (f16x2), zero outside [0, C) and beyond M
-  uint32_t xr[MT][CPT][16];
+// x[m][k] as raw bf16 pairs: thread t owns the 32-element chunks t + j*T of rows m0..m0+MT-1.
+template <int MT, int CPT>
+__device__ __forceinline__ void load_x_rows(const GemvArgs& a, int t, int T, int C, uint32_t (&xr)[MT][CPT][16]) {
 #pragma unroll
   for (int m = 0; m < MT; ++m) {
 #pragma unroll
@@ -52,11 +44,11 @@ __global__ void __launch_bounds__(512) gemv_kernel(GemvArgs a) {
         const uint4* src = reinterpret_cast<const uint4*>(a.X + (long long)mm * a.K + (long long)c * 32);
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
-          uint4 b = src[v];
-          xr[m][j][4 * v + 0] = bf16x2_to_f16x2_sat(b.x);
-          xr[m][j][4 * v + 1] = bf16x2_to_f16x2_sat(b.y);
-          xr[m][j][4 * v + 2] = bf16x2_to_f16x2_sat(b.z);
-          xr[m][j][4 * v + 3] = bf16x2_to_f16x2_sat(b.w);
+          const uint4 b = src[v];
+          xr[m][j][4 * v + 0] = b.x;
+          xr[m][j][4 * v + 1] = b.y;
+          xr[m][j][4 * v + 2] = b.z;
+          xr[m][j][4 * v + 3] = b.w;
         }
       } else {
 #pragma unroll
@@ -64,8 +56,70 @@ __global__ void __launch_bounds__(512) gemv_kernel(GemvArgs a) {
       }
     }
   }
+}
 
+// Each row's power-of-two shift (row_shift_of_amax) from the amax over the threads that hold
+// it: warp shuffles, then one value per warp in `red` between two barriers (`sync`).
+template <int MT, int CPT, typename Sync>
+__device__ __forceinline__ void row_shifts(const uint32_t (&xr)[MT][CPT][16], float* red, int lane, int warp,
+                                           int nwarps, int (&xe)[MT], Sync sync) {
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    float v = 0.f;
+#pragma unroll
+    for (int j = 0; j < CPT; ++j)
+#pragma unroll
+      for (int e = 0; e < 16; ++e) v = fmaxf(v, bf16x2_absmax(xr[m][j][e]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if (lane == 0) red[warp * MT + m] = v;
+  }
+  sync();
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    float v = 0.f;
+    for (int w = 0; w < nwarps; ++w) v = fmaxf(v, red[w * MT + m]);
+    xe[m] = row_shift_of_amax(v);
+  }
+  sync();                                        // `red` is reused by the caller
+}
+
+template <int MT, int CPT>
+__device__ __forceinline__ void convert_x_rows(uint32_t (&xr)[MT][CPT][16], const int (&xe)[MT]) {
+#pragma unroll
+  for (int m = 0; m < MT; ++m)
+#pragma unroll
+    for (int j = 0; j < CPT; ++j)
+#pragma unroll
+      for (int v = 0; v < 16; ++v) xr[m][j][v] = bf16x2_to_f16x2_shifted(xr[m][j][v], xe[m]);
+}
+
+// xe[m] for a run-time m < MT without dynamic register indexing.
+template <int MT>
+__device__ __forceinline__ int pick(const int (&xe)[MT], int m) {
+  int r = xe[0];
+#pragma unroll
+  for (int k = 1; k < MT; ++k) r = (m == k) ? xe[k] : r;
+  return r;
+}
+
+template <int MT, int CPT, int R, bool VERIFY>
+__global__ void __launch_bounds__(512) gemv_kernel(GemvArgs a) {
+  const int T = blockDim.x;
+  const int t = threadIdx.x;
+  const int lane = t & 31, warp = t >> 5, nwarps = T >> 5;
+  const int C = a.K >> 5;                       // 32-element chunks per row
+  const long long rowq = a.K >> 1;              // bytes of q per row
+  const long long rows = a.K >> 4;              // bytes of sf per row
+
+  // X slice -> registers, zero outside [0, C) and beyond M; then each row's shift from its
+  // amax (every CTA holds whole rows) and the conversion to f16x2
   extern __shared__ float red[];                // [2][nwarps][R][MT]
+  uint32_t xr[MT][CPT][16];
+  int xe[MT];
+  load_x_rows<MT, CPT>(a, t, T, C, xr);
+  row_shifts<MT>(xr, red, lane, warp, nwarps, xe, [] { __syncthreads(); });
+  convert_x_rows<MT, CPT>(xr, xe);
   const float ts = *a.ts;
   const int ngroups = (int)((a.N + R - 1) / R);
 
@@ -152,7 +206,7 @@ __global__ void __launch_bounds__(512) gemv_kernel(GemvArgs a) {
         if (n < a.N && mm < a.M) {
           float s = 0.f;
           for (int w = 0; w < nwarps; ++w) s += red[((buf * nwarps + w) * R + r) * MT + m];
-          const float y = s * ts;
+          const float y = mul_pow2(s * ts, pick<MT>(xe, m));
           if (a.y_bf16)
             reinterpret_cast<uint16_t*>(a.Y)[(long long)mm * a.N + n] = f32_to_bf16_rn(y);
           else
@@ -161,13 +215,14 @@ __global__ void __launch_bounds__(512) gemv_kernel(GemvArgs a) {
       }
     } else {
       if (t < MT) {
+        const int et = pick<MT>(xe, t);
 #pragma unroll
         for (int r = 0; r < R; ++r) {
           const long long n = (long long)g * R + r;
           if (n < a.N) {
             float s = 0.f;
             for (int w = 0; w < nwarps; ++w) s += red[((buf * nwarps + w) * R + r) * MT + t];
-            const float y = s * ts;
+            const float y = mul_pow2(s * ts, et);
             if (argmax_better(y, (int)n, bestv, besti)) { bestv = y; besti = (int)n; }
           }
         }
@@ -246,27 +301,10 @@ __global__ void __launch_bounds__(544, 1) gemv_staged_kernel(GemvArgs a, int sta
 
   // ---------------- compute threads
   uint32_t xr[MT][CPT][16];
-#pragma unroll
-  for (int m = 0; m < MT; ++m)
-#pragma unroll
-    for (int j = 0; j < CPT; ++j) {
-      const int c = t + j * T;
-      const int mm = a.m0 + m;
-      if (c < C && mm < a.M) {
-        const uint4* src = reinterpret_cast<const uint4*>(a.X + (long long)mm * a.K + (long long)c * 32);
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          uint4 b = src[v];
-          xr[m][j][4 * v + 0] = bf16x2_to_f16x2_sat(b.x);
-          xr[m][j][4 * v + 1] = bf16x2_to_f16x2_sat(b.y);
-          xr[m][j][4 * v + 2] = bf16x2_to_f16x2_sat(b.z);
-          xr[m][j][4 * v + 3] = bf16x2_to_f16x2_sat(b.w);
-        }
-      } else {
-#pragma unroll
-        for (int v = 0; v < 16; ++v) xr[m][j][v] = 0u;
-      }
-    }
+  int xe[MT];
+  load_x_rows<MT, CPT>(a, t, T, C, xr);
+  row_shifts<MT>(xr, red, lane, warp, nwarps, xe, [T] { named_bar(1, T); });
+  convert_x_rows<MT, CPT>(xr, xe);
   const float ts = *a.ts;
   float bestv = -INFINITY;
   int besti = INT_MAX;
@@ -327,7 +365,7 @@ __global__ void __launch_bounds__(544, 1) gemv_staged_kernel(GemvArgs a, int sta
         if (n < a.N && mm < a.M) {
           float sum = 0.f;
           for (int w = 0; w < nwarps; ++w) sum += red[((buf * nwarps + w) * RG + r) * MT + m];
-          const float y = sum * ts;
+          const float y = mul_pow2(sum * ts, pick<MT>(xe, m));
           if (a.y_bf16)
             reinterpret_cast<uint16_t*>(a.Y)[(long long)mm * a.N + n] = f32_to_bf16_rn(y);
           else
@@ -335,13 +373,14 @@ __global__ void __launch_bounds__(544, 1) gemv_staged_kernel(GemvArgs a, int sta
         }
       }
     } else if (t < MT) {
+      const int et = pick<MT>(xe, t);
 #pragma unroll
       for (int r = 0; r < RG; ++r) {
         const long long n = (long long)g * RG + r;
         if (n < a.N) {
           float sum = 0.f;
           for (int w = 0; w < nwarps; ++w) sum += red[((buf * nwarps + w) * RG + r) * MT + t];
-          const float y = sum * ts;
+          const float y = mul_pow2(sum * ts, et);
           if (argmax_better(y, (int)n, bestv, besti)) { bestv = y; besti = (int)n; }
         }
       }

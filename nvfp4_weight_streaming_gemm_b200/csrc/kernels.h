@@ -33,6 +33,10 @@ GemvPlan gemv_plan(long long M, long long N, long long K, bool regs_only);
 bool gemv_supported(long long K);
 int launch_gemv(const GemvArgs& a, bool verify, bool regs_only, cudaStream_t s);
 
+// xe[m] = the power-of-two shift of activation row m (bf16 [M, K], K even) that the f16
+// kernels apply before converting it (row_shift_of_amax in common.cuh).
+int launch_row_shifts(const uint16_t* X, long long M, long long K, int* xe, cudaStream_t s);
+
 int launch_pack(const float* W, long long N, long long K, uint8_t* q, uint8_t* sf, float* ts,
                 const float* ts_in, cudaStream_t s);
 

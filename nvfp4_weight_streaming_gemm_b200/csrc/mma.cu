@@ -21,9 +21,11 @@
 //                 E4M3 block scale in f16 (exact). It writes the f16 A operand
 //                 straight into TMEM with tcgen05.st, so A never takes a round
 //                 trip through shared memory. The same threads convert the
-//                 chunk's X rows from bf16 to f16 in place, saturating at 65504.
-//   warps 12-15   Epilogue warpgroup: tcgen05.ld of the accumulators, times ts,
-//                 then Y (or, in verify mode, the per-tile argmax).
+//                 chunk's X rows from bf16 to f16 in place, each row shifted by
+//                 its power of two xe[m] (x_shift_kernel, launched first), so the
+//                 conversion is exact and never saturates.
+//   warps 12-15   Epilogue warpgroup: tcgen05.ld of the accumulators, times ts
+//                 and 2^xe[m], then Y (or, in verify mode, the per-tile argmax).
 //
 // Scheduling. The units are (128-row tile, 256-wide K-chunk) pairs. They are
 // split into equal contiguous ranges, one per CTA (stream-K), so every SM streams
@@ -78,6 +80,7 @@ struct Params {
   // workspace
   unsigned int* counters;  // [tiles], zero between calls
   float* partials;         // [2 * grid][M][128]
+  const int* xe;           // [M] power-of-two shift of each X row (x_shift_kernel)
   // verify mode
   int verify;
   float* part_val;         // [tiles][M]
@@ -213,6 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* s_last = reinterpret_cast<int*>(s_tmem + 2);
   float* s_val = reinterpret_cast<float*>(s_tmem + 4);                  // [4][kMaxNpad]
   int* s_idx = reinterpret_cast<int*>(s_val + 4 * kMaxNpad);            // [4][kMaxNpad]
+  int* s_xe = s_idx + 4 * kMaxNpad;                                     // [kMaxNpad] row shifts
 
   auto bar_full = [&](int s) { return smem_u32(bars + s); };
   auto bar_empty = [&](int s) { return smem_u32(bars + S + s); };
@@ -240,6 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     *s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  for (int m = threadIdx.x; m < kMaxNpad; m += kThreads) s_xe[m] = m < p.M ? p.xe[m] : 0;
   if (warp == 1) {   // whole warp allocates all 512 TMEM columns (one CTA per SM)
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(s_tmem)),
                  "r"(512));
@@ -343,8 +348,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int a = w / (p.M * 8), rem = w - a * (p.M * 8);
           uint4* ptr = reinterpret_cast<uint4*>(xs + a * npad * 128 + (rem >> 3) * 128 + (rem & 7) * 16);
           uint4 v = *ptr;
-          v.x = bf16x2_to_f16x2_sat(v.x); v.y = bf16x2_to_f16x2_sat(v.y);
-          v.z = bf16x2_to_f16x2_sat(v.z); v.w = bf16x2_to_f16x2_sat(v.w);
+          const int e = s_xe[rem >> 3];
+          v.x = bf16x2_to_f16x2_shifted(v.x, e); v.y = bf16x2_to_f16x2_shifted(v.y, e);
+          v.z = bf16x2_to_f16x2_shifted(v.z, e); v.w = bf16x2_to_f16x2_shifted(v.w, e);
           *ptr = v;
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -409,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (complete) {
           float y[16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) y[j] = __uint_as_float(v[j]) * ts;
+          for (int j = 0; j < 16; ++j) y[j] = mul_pow2(__uint_as_float(v[j]) * ts, s_xe[m0 + j]);
           if (p.verify) tile_argmax(p, row, m0, y, s_val, s_idx, q, lane);
           else write_y(p, row, m0, y);
         } else {
@@ -471,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < 16; ++j) y[j] += v[j];
           }
 #pragma unroll
-          for (int j = 0; j < 16; ++j) y[j] *= ts;
+          for (int j = 0; j < 16; ++j) y[j] = mul_pow2(y[j] * ts, s_xe[m0 + j]);
           if (p.verify) tile_argmax(p, row, m0, y, s_val, s_idx, q, lane);
           else write_y(p, row, m0, y);
         }
@@ -565,10 +571,15 @@ static MmaPlan plan_of(long long M, long long N, long long K) {
 
 static size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
+// GEMM workspace: ticket counters [tiles] | partials [2 * grid][M][128] | row shifts [M].
+static size_t xe_offset(const MmaPlan& pl, long long M) {
+  return align256((size_t)pl.tiles * 4) + align256((size_t)2 * pl.grid * M * kTileRows * 4);
+}
+
 size_t mma_gemm_workspace_bytes(long long M, long long N, long long K) {
   if (!mma_supported(M, K)) return 0;
   MmaPlan pl = plan_of(M, N, K);
-  return align256((size_t)pl.tiles * 4) + align256((size_t)2 * pl.grid * M * kTileRows * 4);
+  return xe_offset(pl, M) + align256((size_t)M * 4);
 }
 
 size_t mma_gemm_counter_bytes(long long M, long long N, long long K) {
@@ -611,6 +622,8 @@ static int launch_mma(const uint16_t* X, const uint8_t* q, const uint8_t* sf, co
   char* ws = static_cast<char*>(workspace);
   p.counters = reinterpret_cast<unsigned int*>(ws);
   p.partials = reinterpret_cast<float*>(ws + align256((size_t)pl.tiles * 4));
+  int* xe = reinterpret_cast<int*>(ws + xe_offset(pl, M));
+  p.xe = xe;
   p.verify = verify ? 1 : 0;
   if (verify) {
     char* v = ws + mma_gemm_workspace_bytes(M, N, K);
@@ -630,6 +643,7 @@ static int launch_mma(const uint16_t* X, const uint8_t* q, const uint8_t* sf, co
       return check_launch("cudaFuncSetAttribute(mma_kernel)");
     attr_set[dev].store(true, std::memory_order_release);
   }
+  if (int e = launch_row_shifts(X, M, K, xe, s)) return e;
   mma_kernel<<<pl.grid, kThreads, pl.smem, s>>>(tq, tsf, tx, p);
   return check_launch("mma_kernel");
 }

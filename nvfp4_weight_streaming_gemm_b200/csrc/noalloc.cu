@@ -65,6 +65,7 @@ using namespace nvfp4ws;
 extern "C" int nvfp4_gemm_skinny_noalloc(const void* X, const uint8_t* q, const uint8_t* sf,
                                          const float* tensor_scale, int64_t M, int64_t N, int64_t K, void* Y,
                                          int y_dtype, nvfp4ws_stream_t stream) {
+  clear_error();
   if (!X || !q || !sf || !tensor_scale || !Y)
     return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_gemm_skinny_noalloc: null pointer");
   if (M < 1 || N < 1 || K < 1)
@@ -88,8 +89,11 @@ extern "C" int nvfp4_gemm_skinny_noalloc(const void* X, const uint8_t* q, const 
   if (int e = scratch_address(&scratch)) return e;
   cudaStream_t s = (cudaStream_t)stream;
   // The leading ticket counters must start at zero.
-  if (cudaMemsetAsync(scratch, 0, mma_gemm_counter_bytes(M, N, K), s) != cudaSuccess)
-    return check_launch("nvfp4_gemm_skinny_noalloc: counter clear");
+  // (check_launch also counts the memset node, as nvfp4ws_kernel_launches documents.)
+  const cudaError_t me = cudaMemsetAsync(scratch, 0, mma_gemm_counter_bytes(M, N, K), s);
+  if (int e = check_launch("nvfp4_gemm_skinny_noalloc: counter clear")) return e;
+  if (me != cudaSuccess)
+    return set_error(NVFP4WS_ERR_CUDA, "nvfp4_gemm_skinny_noalloc: counter clear: %s", cudaGetErrorString(me));
   return launch_mma_gemm(static_cast<const uint16_t*>(X), q, sf, tensor_scale, M, N, K, Y, y_dtype, scratch,
                          kNoAllocScratchBytes, s);
 }

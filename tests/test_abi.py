@@ -146,3 +146,52 @@ def test_fp8_rejects_on_the_host(lib):
     assert v(FAKE, FAKE, FAKE, 17, 100, 128, None, FAKE, 1 << 30, None) == 1                 # no rule
     spec = L.VerifySpec(None, 1, 16, FAKE, FAKE, None, None, None)
     assert v(FAKE, FAKE, FAKE, 17, 100, 128, ctypes.byref(spec), FAKE, 1 << 30, None) == 1   # drafts missing
+
+
+class _OldGemmProblem(ctypes.Structure):
+    """nvfp4_gemm_problem as it was before struct_size (ABI versions up to 102)."""
+    _fields_ = [("X", ctypes.c_void_p), ("q", ctypes.c_void_p), ("sf", ctypes.c_void_p),
+                ("tensor_scale", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("Y", ctypes.c_void_p), ("y_dtype", ctypes.c_int32)]
+
+
+class _OldVerifySpec(ctypes.Structure):
+    """nvfp4_verify_spec of ABI version 100: no struct_size, no parents, no accept_node."""
+    _fields_ = [("drafts", ctypes.c_void_p), ("B", ctypes.c_int32), ("D", ctypes.c_int32),
+                ("argmax", ctypes.c_void_p), ("accept_len", ctypes.c_void_p), ("max_logit", ctypes.c_void_p)]
+
+
+def test_structs_carry_their_size(lib):
+    from nvfp4_weight_streaming_gemm_b200 import _lib as L
+    assert lib.nvfp4ws_version() >= 200
+    assert L.GemmProblem(FAKE, FAKE, FAKE, FAKE, 128, 256, FAKE, 0).struct_size == ctypes.sizeof(L.GemmProblem)
+    assert L.VerifySpec(FAKE, 1, 16).struct_size == ctypes.sizeof(L.VerifySpec)
+
+
+def test_pass_refuses_a_struct_of_another_size(lib):
+    """A caller built against another header version is refused on the host with
+    INVALID_ARG, before any member past struct_size is read."""
+    from nvfp4_weight_streaming_gemm_b200 import _lib as L
+    arr = (L.GemmProblem * 2)()
+    for i in range(2):
+        arr[i] = L.GemmProblem(FAKE, FAKE, FAKE, FAKE, 128, 256, FAKE, 0)
+    arr[1].struct_size = ctypes.sizeof(L.GemmProblem) - 8
+    st = L.PassState()
+    assert lib.nvfp4_pass_workspace_bytes(arr, 2, 17, 0) == 0
+    assert lib.nvfp4_pass_init(ctypes.byref(st), arr, 2, 17, None, FAKE, 1 << 30) == 1
+    assert b"problem 1: struct_size" in lib.nvfp4ws_last_error()
+    # an array of the old layout: its first member is a pointer, never the struct size
+    old = (_OldGemmProblem * 1)()
+    old[0] = _OldGemmProblem(FAKE, FAKE, FAKE, FAKE, 128, 256, FAKE, 0)
+    old_ptr = ctypes.cast(old, ctypes.POINTER(L.GemmProblem))
+    assert lib.nvfp4_pass_init(ctypes.byref(st), old_ptr, 1, 17, None, FAKE, 1 << 30) == 1
+    assert b"struct_size" in lib.nvfp4ws_last_error()
+    # a short verify struct (the one that once had its missing members read as pointers)
+    arr1 = (L.GemmProblem * 1)()
+    arr1[0] = L.GemmProblem(FAKE, FAKE, FAKE, FAKE, 128, 256, None, 0)
+    short = _OldVerifySpec(FAKE, 1, 16, FAKE, FAKE, None)
+    vs_ptr = ctypes.cast(ctypes.pointer(short), ctypes.POINTER(L.VerifySpec))
+    assert lib.nvfp4_pass_init(ctypes.byref(st), arr1, 1, 17, vs_ptr, FAKE, 1 << 30) == 1
+    assert b"verify struct_size" in lib.nvfp4ws_last_error()
+    assert lib.fp8_lmhead_verify(FAKE, FAKE, FAKE, 17, 100, 128, vs_ptr, FAKE, 1 << 30, None) == 1
+    assert b"struct_size" in lib.nvfp4ws_last_error()

@@ -151,13 +151,58 @@ def test_gemm_bf16_output(nv):
 
 
 def test_gemm_extreme_activations(nv):
-    """bf16 activations outside f16's normal range: tiny values lose only < 2^-25 absolute."""
+    """bf16 activations below f16's normal range inside a row of ordinary values."""
     W, x = S.random_case(41, 2, 64, 256)
     xf = G.bf16_bits_to_float64(x)
     xf[0, ::7] *= 1e-6                       # below 2^-14: f16 subnormal range
     x2 = S.f32_to_bf16_bits(xf.astype(np.float32))
     Y, y_ref = run_gemm(nv, W, x2)
     assert_rowwise(Y.cpu().numpy(), y_ref)
+
+
+def _extreme_rows(seed, M, K):
+    """bf16 rows far outside f16's range: large (|x| up to ~4e6, far above 65504), all tiny
+    (~1e-30), one 1e30 outlier among N(0, 1) values, N(0, 1) with every 7th value scaled
+    by 1e-6, and all zero; repeated to M rows."""
+    rng = np.random.default_rng(seed)
+    base = rng.standard_normal((M, K))
+    kinds = [lambda r: r * 2.0 ** 20, lambda r: r * 1e-30, None, None, lambda r: r * 0.0]
+    for m in range(M):
+        k = kinds[m % len(kinds)]
+        if k is not None:
+            base[m] = k(base[m])
+        elif m % len(kinds) == 2:
+            base[m, rng.integers(0, K)] = 1e30
+        else:
+            base[m, ::7] *= 1e-6
+    return S.f32_to_bf16_bits(base.astype(np.float32))
+
+
+@pytest.mark.parametrize("path,M,N,K", [("gemv", 1, 700, 5120), ("gemv", 5, 300, 1024), ("gemv_regs", 5, 300, 96),
+                                        ("mma_f16", 5, 300, 1024), ("mma_f16", 100, 513, 768), ("mma", 10, 400, 512),
+                                        ("auto", 1, 1000, 17408)])
+def test_gemm_activation_range(nv, path, M, N, K):
+    """Activations the f16 paths used to saturate (above 65504) or round away (below
+    2^-14): each row is shifted by a power of two before the f16 conversion, so every row
+    meets the GEMM bar, the zero row gives exactly zero, and the result is finite."""
+    W, _ = S.random_case(4242 + M + K, 1, N, K)
+    x = _extreme_rows(17 + M, M, K)
+    Y, y_ref = run_gemm(nv, W, x, path=path)
+    y = Y.cpu().numpy()
+    assert np.isfinite(y).all()
+    assert_rowwise(y, y_ref)
+
+
+def test_verify_activation_range(nv):
+    """The fused verify on the GEMV and f16 paths (one row, D = 0) with activations far above
+    65504: the argmax follows the oracle. (A row of ~1e-30 values is checked too; its logits
+    are all within the tie band, so only the band check bites there.)"""
+    N, K = 3000, 1024
+    W, _ = S.random_case(99, 1, N, K, w_std=0.05)
+    rows = _extreme_rows(5, 5, K)
+    for x in (rows[0:1], rows[1:2]):
+        run_verify(nv, W, x, np.array([0]), 0, path="gemv")
+        run_verify(nv, W, x, np.array([0]), 0, path="mma_f16")
 
 
 @pytest.mark.parametrize("name", S.LAYER_ORDER)

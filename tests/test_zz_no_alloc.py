@@ -5,7 +5,9 @@ pooling allocator, or a plugin interface with no scratch buffer.
 nvfp4_gemm_skinny_noalloc takes its scratch from a built-in device array instead
 of a caller workspace. This test calls it through the C ABI twice in a row. Both
 results must match nvfp4_gemm_skinny (which gets a workspace) within the
-tolerance used by the other GEMM tests, and must also match the CPU oracle. It
+tolerance used by the other GEMM tests, and must also match the CPU oracle. Around
+the second call neither torch's allocator nor the device's free memory may change.
+One row of X lies far above f16's range (the f16 path shifts it into range). It
 sits in a file of its own, collected last, so that a run which stops at the first
 failure has already run every other test. It passes alone in a fresh process too.
 """
@@ -34,6 +36,10 @@ def test_noalloc_matches_workspace_entry_point(M, N, K):
     build.build()
     lib = nv.lib()
     W, x = S.random_case(900 + M + N, M, N, K)
+    if M > 1:                                            # one row far above f16's range (|x| up to ~4e6)
+        xf = G.bf16_bits_to_float64(x)
+        xf[M // 2] *= 2.0 ** 20
+        x = S.f32_to_bf16_bits(xf.astype(np.float32))
     q, sf, ts = nv.pack(torch.from_numpy(W).cuda())
     X = torch.from_numpy(x.view(np.int16).copy()).view(torch.bfloat16).cuda()
     stream = torch.cuda.current_stream().cuda_stream
@@ -45,14 +51,20 @@ def test_noalloc_matches_workspace_entry_point(M, N, K):
                                y_ws.data_ptr(), 0, ws.data_ptr(), ws_bytes, stream)
     assert st == 0, lib.nvfp4ws_last_error()
 
-    outs = []
-    for _ in range(2):                                   # two calls in a row share the built-in scratch
-        y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    outs = [torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda") for _ in range(2)]
+    torch.cuda.synchronize()
+    for i, y in enumerate(outs):                         # two calls in a row share the built-in scratch
+        if i == 1:                                       # the first call has looked up the scratch address
+            torch.cuda.synchronize()
+            alloc0, free0 = torch.cuda.memory_allocated(), torch.cuda.mem_get_info()[0]
         st = lib.nvfp4_gemm_skinny_noalloc(X.data_ptr(), q.data_ptr(), sf.data_ptr(), ts.data_ptr(), M, N, K,
                                            y.data_ptr(), 0, stream)
         assert st == 0, lib.nvfp4ws_last_error()
-        outs.append(y)
+        assert lib.nvfp4ws_last_error() == b""
     torch.cuda.synchronize()
+    # the call allocated nothing: neither through torch nor from the device
+    assert torch.cuda.memory_allocated() == alloc0
+    assert torch.cuda.mem_get_info()[0] == free0
     nv.check()
 
     ref_ws = y_ws.cpu().numpy().astype(np.float64)
