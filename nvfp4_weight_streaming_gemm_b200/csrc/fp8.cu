@@ -378,6 +378,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
     long long tile_it = u_begin / kbs;
     int kb_it = (int)(u_begin % kbs);
+    // Block scales, four units ahead: a unit's index is its scale's index (tile-major, K/128
+    // blocks per tile), and the L2 round trip would otherwise sit on every unit's path.
+    auto scale_of = [&](long long u) { return u < u_end ? __ldg(p.scales + u) : 0.0f; };
+    float sc_next[4] = {scale_of(u_begin), scale_of(u_begin + 1), scale_of(u_begin + 2), scale_of(u_begin + 3)};
     for (int i = 0; i < nunits; ++i) {
       const long long u = u_begin + i;
       const long long tile = tile_it;
@@ -386,7 +390,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool seg_last = (i == nunits - 1) || (kb == kbs - 1);
       if (++kb_it == kbs) { kb_it = 0; ++tile_it; }
       const int b = i % NP, k = i / NP;
-      const float sc = __ldg(p.scales + tile * kbs + kb);
+      const float sc = sc_next[0];
+      sc_next[0] = sc_next[1];
+      sc_next[1] = sc_next[2];
+      sc_next[2] = sc_next[3];
+      sc_next[3] = scale_of(u + 4);
       // Every thread reaches the barrier, so a give-up seen by any of them ends the loop for all.
       mbar_wait(bar_pfull(b), (uint32_t)k & 1u, s_abort, p.err);
       named_bar(1, 128);
