@@ -10,18 +10,20 @@
 // Exactness. An E4M3 value has at most 4 significant bits and lies in [2^-9, 448], so it is
 // exact in f16, as is the activation for |x| in [2^-14, 65504] (bf16 -> f16, nearest,
 // saturating). Every product is then exact in the fp32 accumulator. The block scale is an
-// arbitrary fp32 and would round if folded into either f16 operand, so a unit of work is one
-// 128 x 128 block: the tensor core sums the block's 128 products per (row, token) into a fresh
-// TMEM buffer P, and the epilogue promotes it into a running sum R = s * P, then R += s * P,
-// in fp32 (R also lives in TMEM).
+// arbitrary fp32 and would round if folded into either f16 operand, so the tensor core sums
+// each 128 x 128 block's 128 products per (row, token) into a fresh TMEM buffer P, and the
+// epilogue promotes it into a running sum R = s * P, then R += s * P, in fp32 (R also lives
+// in TMEM). A unit of work is BPU = 1 or 2 such blocks of one 128-row tile: two while TMEM
+// leaves room for two rotating P sets (npad <= 48), which halves the per-unit hand-offs per
+// weight byte.
 //
 // Roles per CTA (one persistent CTA per SM, 16 warps):
-//   warp 0        TMA producer: the 16 KB code tile (128 rows x 128 B, 128-byte swizzle) and
-//                 the unit's bf16 X slice (two 64-wide swizzled atoms) into a ring of stages.
+//   warp 0        TMA producer: the unit's 16 KB code tiles (128 rows x 128 B, 128-byte
+//                 swizzle) and its bf16 X slice (2*BPU 64-wide swizzled atoms) into a ring.
 //                 No multicast.
 //   warp 1        TMEM allocator and the single MMA-issuing thread: 8 x kind::f16 (K = 16)
-//                 per unit, A from TMEM, B from shared memory, into one of np rotating P
-//                 buffers.
+//                 per block, A from TMEM, B from shared memory, each block into its own P of
+//                 one of np rotating P sets.
 //   warps 4-7,    two dequantisation warpgroups taking alternate units. Each thread owns one
 //   warps 8-11    weight row (its TMEM lane): E4M3 pairs -> f16 pairs (cvt.rn.f16x2.e4m3x2)
 //                 written into TMEM as the A operand. The same threads convert the unit's X
@@ -29,10 +31,10 @@
 //   warps 12-15   promotion and epilogue: at the end of a tile's K range, Y (or the tile's
 //                 per-token argmax in verify mode, or a split-K partial).
 //
-// TMEM columns (512, one CTA per SM): [0, 64) and [64, 128) the two A buffers (64 f16 pairs
-// per row), [128, 128 + npad) R, then np P buffers of npad columns.
+// TMEM columns (512, one CTA per SM): two A buffers of 64*BPU columns (64 f16 pairs per row
+// and block), then R (npad columns), then np P sets of BPU*npad columns.
 //
-// Scheduling is stream-K: the (tile, K-block) units are cut into equal contiguous ranges, one
+// Scheduling is stream-K: the (tile, K-range) units are cut into equal contiguous ranges, one
 // per CTA. A tile whose K range spans several CTAs is finished by the last to arrive: each
 // publishes its fp32 partial, takes a ticket, and the holder of the last ticket sums the
 // partials in K order, so results are deterministic and no CTA waits for another. Every
@@ -56,11 +58,10 @@ namespace fp8k {
 
 constexpr int kThreads = 512;
 constexpr int kTileRows = 128;
-constexpr int kKB = kFp8Block;                       // K elements per unit = one scale block
-constexpr uint32_t kWBytes = kTileRows * kKB;        // 16 KB of codes per unit
+constexpr int kKB = kFp8Block;                       // K elements of one scale block
+constexpr uint32_t kWBytes = kTileRows * kKB;        // 16 KB of codes per block
 constexpr int kMaxNpad = 128;
-constexpr int kACols = kKB / 2;                      // f16 pairs per row = TMEM columns per A buffer
-constexpr uint32_t kRCol = 2 * kACols;               // running sums after the two A buffers
+constexpr int kACols = kKB / 2;                      // f16 pairs per row and block = TMEM columns
 constexpr int kMaxP = 4;
 constexpr int kMaxStages = 8;
 constexpr size_t kTailBytes = 8192;
@@ -68,10 +69,10 @@ constexpr size_t kTailBytes = 8192;
 struct Params {
   float* Y;                // fp32 or bf16 (y_bf16)
   int y_bf16;
-  const float* scales;     // [tiles][kbs]
+  const float* scales;     // [tiles][K / 128]
   int M, npad, np;
   long long N, K;
-  int tiles, kbs;
+  int tiles, kus;          // units per tile: K / (128 * BPU)
   long long units;
   int grid;
   int stages;
@@ -211,8 +212,15 @@ __device__ __forceinline__ void tile_argmax_out(const Params& p, int tile, int e
 
 // ---------------------------------------------------------------- the kernel
 
+// BPU scale blocks (128 K each) per unit. Two blocks per unit halve the per-unit fixed costs
+// (barrier hand-offs, the epilogue's TMEM round trips) per weight byte; the sums are the same
+// fma sequence either way, so the result does not depend on BPU.
+template <int BPU>
 __global__ void __launch_bounds__(kThreads, 1)
     fp8_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x, const Params p) {
+  constexpr uint32_t kUW = BPU * kWBytes;           // code bytes per unit
+  constexpr int kUACols = BPU * kACols;             // TMEM columns of one A buffer
+  constexpr uint32_t kR = 2 * kUACols;              // running sums after the two A buffers
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int S = p.stages, NP = p.np;
@@ -238,8 +246,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const long long U = p.units;
   const long long u_begin = unit_begin(c, U, p.grid), u_end = unit_begin(c + 1, U, p.grid);
   const int nunits = (int)(u_end - u_begin);
-  const int npad = p.npad, kbs = p.kbs;
-  const uint32_t pcol0 = kRCol + (uint32_t)npad;   // first P buffer
+  const int npad = p.npad, kus = p.kus;
+  const uint32_t pcol0 = kR + (uint32_t)npad;      // first P buffer; buffer b, block h at + (b*BPU + h)*npad
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) { mbar_init(bar_full(s), 1); mbar_init(bar_empty(s), 1); }
@@ -263,22 +271,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       const uint64_t pol_w = policy_evict_first(), pol_x = policy_evict_last();
-      const uint32_t tx = kWBytes + (uint32_t)npad * 256u;
+      const uint32_t tx = kUW + (uint32_t)(BPU * npad) * 256u;
       int issued = 0;
-      long long tile = u_begin / kbs;
-      int kb = (int)(u_begin % kbs);
+      long long tile = u_begin / kus;
+      int ku = (int)(u_begin % kus);
       int s = 0;
       uint32_t ph = 0;
       for (int i = 0; i < nunits; ++i) {
         if (!mbar_wait(bar_empty(s), ph ^ 1u, s_abort, p.err)) break;
         uint8_t* st = smem + (size_t)s * p.stage_bytes;
+        const int k0 = ku * BPU * kKB;                 // first K element of the unit
         mbar_arrive_expect_tx(bar_full(s), tx);
-        tma_load_2d(smem_u32(st), &tm_w, kb * kKB, (int)(tile * kTileRows), bar_full(s), pol_w);
 #pragma unroll
-        for (int a = 0; a < 2; ++a)
-          tma_load_2d(smem_u32(st + kWBytes + a * npad * 128), &tm_x, kb * kKB + a * 64, 0, bar_full(s), pol_x);
+        for (int h = 0; h < BPU; ++h)
+          tma_load_2d(smem_u32(st + h * kWBytes), &tm_w, k0 + h * kKB, (int)(tile * kTileRows), bar_full(s), pol_w);
+#pragma unroll
+        for (int a = 0; a < 2 * BPU; ++a)
+          tma_load_2d(smem_u32(st + kUW + a * npad * 128), &tm_x, k0 + a * 64, 0, bar_full(s), pol_x);
         issued = i + 1;
-        if (++kb == kbs) { kb = 0; ++tile; }
+        if (++ku == kus) { ku = 0; ++tile; }
         if (++s == S) { s = 0; ph ^= 1u; }
       }
       if (*s_abort) {       // drain: wait (bounded) for every copy this thread issued
@@ -302,17 +313,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mbar_wait(bar_afull(g), (uint32_t)(i >> 1) & 1u, s_abort, p.err);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t xbase = smem_u32(smem + (size_t)s * p.stage_bytes + kWBytes);
-        const uint32_t d_tmem = tmem + pcol0 + (uint32_t)(b * npad);
-        const uint32_t a_tmem = tmem + (uint32_t)(g * kACols);
+        const uint32_t xbase = smem_u32(smem + (size_t)s * p.stage_bytes + kUW);
 #pragma unroll
-        for (int kk = 0; kk < kKB / 16; ++kk) {
-          const uint64_t bdesc = sw128_desc(xbase + (kk >> 2) * npad * 128 + (kk & 3) * 32);
-          tc_mma_f16_ts(d_tmem, a_tmem + kk * 8, bdesc, idesc, kk == 0 ? 0u : 1u);
+        for (int h = 0; h < BPU; ++h) {            // each block into its own P: its scale comes later
+          const uint32_t d_tmem = tmem + pcol0 + (uint32_t)((b * BPU + h) * npad);
+          const uint32_t a_tmem = tmem + (uint32_t)(g * kUACols + h * kACols);
+#pragma unroll
+          for (int kk = 0; kk < kKB / 16; ++kk) {
+            const uint64_t bdesc = sw128_desc(xbase + (2 * h + (kk >> 2)) * npad * 128 + (kk & 3) * 32);
+            tc_mma_f16_ts(d_tmem, a_tmem + kk * 8, bdesc, idesc, kk == 0 ? 0u : 1u);
+          }
         }
         tc_commit(bar_empty(s));       // stage reusable once these MMAs retire
         tc_commit(bar_aempty(g));      // A buffer reusable
-        tc_commit(bar_pfull(b));       // the block's sums are ready for promotion
+        tc_commit(bar_pfull(b));       // the blocks' sums are ready for promotion
         if (++s == S) { s = 0; ph ^= 1u; }
       }
       tc_commit(bar_drain);            // completes when every MMA issued above has retired
@@ -338,8 +352,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint8_t* st = smem + (size_t)s * p.stage_bytes;
       // X slice: bf16 -> f16 in place (rows < M; TMA zero-filled the rest)
       {
-        uint8_t* xs = st + kWBytes;
-        const int words = 2 * p.M * 8;               // 16-byte words: 2 atoms x M rows x 8
+        uint8_t* xs = st + kUW;
+        const int words = 2 * BPU * p.M * 8;         // 16-byte words: 2*BPU atoms x M rows x 8
         for (int w = tg; w < words; w += 128) {
           const int a = w / (p.M * 8), rem = w - a * (p.M * 8);
           uint4* ptr = reinterpret_cast<uint4*>(xs + a * npad * 128 + (rem >> 3) * 128 + (rem & 7) * 16);
@@ -350,21 +364,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       }
-      // weight row r: 128 codes in eight swizzled 16-byte chunks -> 64 f16 pairs in TMEM
-      const uint8_t* row = st + r * 128;
-      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(g * kACols);
+      // weight row r of each block: 128 codes in eight swizzled 16-byte chunks -> 64 f16 pairs
+      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(g * kUACols);
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t out[32];
+      for (int h = 0; h < BPU; ++h) {
+        const uint8_t* row = st + h * kWBytes + r * 128;
 #pragma unroll
-        for (int j2 = 0; j2 < 4; ++j2) {
-          const int j = half * 4 + j2;                // logical chunk: elements 16j .. 16j+15
-          const uint4 w = *reinterpret_cast<const uint4*>(row + ((j ^ (r & 7)) << 4));
-          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+        for (int half = 0; half < 2; ++half) {
+          uint32_t out[32];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) out[j2 * 8 + e] = e4m3x2_to_f16x2(ww[e >> 1] >> ((e & 1) * 16));
+          for (int j2 = 0; j2 < 4; ++j2) {
+            const int j = half * 4 + j2;              // logical chunk: elements 16j .. 16j+15
+            const uint4 w = *reinterpret_cast<const uint4*>(row + ((j ^ (r & 7)) << 4));
+            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) out[j2 * 8 + e] = e4m3x2_to_f16x2(ww[e >> 1] >> ((e & 1) * 16));
+          }
+          tc_st_x32(taddr + (uint32_t)(h * kACols + half * 32), out);
         }
-        tc_st_x32(taddr + half * 32, out);
       }
       tc_wait_st();
       tc_fence_before();
@@ -376,50 +393,63 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int rowl = q * 32 + lane;
     const int et = threadIdx.x - 12 * 32;            // 0..127
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
-    long long tile_it = u_begin / kbs;
-    int kb_it = (int)(u_begin % kbs);
-    // Block scales, four units ahead: a unit's index is its scale's index (tile-major, K/128
-    // blocks per tile), and the L2 round trip would otherwise sit on every unit's path.
-    auto scale_of = [&](long long u) { return u < u_end ? __ldg(p.scales + u) : 0.0f; };
-    float sc_next[4] = {scale_of(u_begin), scale_of(u_begin + 1), scale_of(u_begin + 2), scale_of(u_begin + 3)};
+    long long tile_it = u_begin / kus;
+    int ku_it = (int)(u_begin % kus);
+    // Block scales, four units ahead: block h of unit u has scale index BPU*u + h (tile-major,
+    // K/128 blocks per tile), and the L2 round trip would otherwise sit on every unit's path.
+    auto scale_of = [&](long long u, int h) { return u < u_end ? __ldg(p.scales + BPU * u + h) : 0.0f; };
+    float scn[4][BPU];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int h = 0; h < BPU; ++h) scn[a][h] = scale_of(u_begin + a, h);
     for (int i = 0; i < nunits; ++i) {
       const long long u = u_begin + i;
       const long long tile = tile_it;
-      const int kb = kb_it;
-      const bool seg_first = (i == 0) || (kb == 0);
-      const bool seg_last = (i == nunits - 1) || (kb == kbs - 1);
-      if (++kb_it == kbs) { kb_it = 0; ++tile_it; }
+      const int ku = ku_it;
+      const bool seg_first = (i == 0) || (ku == 0);
+      const bool seg_last = (i == nunits - 1) || (ku == kus - 1);
+      if (++ku_it == kus) { ku_it = 0; ++tile_it; }
       const int b = i % NP, k = i / NP;
-      const float sc = sc_next[0];
-      sc_next[0] = sc_next[1];
-      sc_next[1] = sc_next[2];
-      sc_next[2] = sc_next[3];
-      sc_next[3] = scale_of(u + 4);
+      float sc[BPU];
+#pragma unroll
+      for (int h = 0; h < BPU; ++h) {
+        sc[h] = scn[0][h];
+        scn[0][h] = scn[1][h];
+        scn[1][h] = scn[2][h];
+        scn[2][h] = scn[3][h];
+        scn[3][h] = scale_of(u + 4, h);
+      }
       // Every thread reaches the barrier, so a give-up seen by any of them ends the loop for all.
       mbar_wait(bar_pfull(b), (uint32_t)k & 1u, s_abort, p.err);
       named_bar(1, 128);
       if (ld_shared_volatile(s_abort)) break;
       tc_fence_after();
       const long long n = tile * kTileRows + rowl;
-      const long long tile_u0 = tile * kbs, tile_u1 = tile_u0 + kbs;
+      const long long tile_u0 = tile * kus, tile_u1 = tile_u0 + kus;
       const long long seg_u0 = u_begin > tile_u0 ? u_begin : tile_u0;
       const bool complete = (seg_u0 == tile_u0) && (u + 1 == tile_u1);
       const int slot = (seg_u0 == u_begin) ? 2 * c : 2 * c + 1;
-      const uint32_t pcol = pcol0 + (uint32_t)(b * npad);
+      const uint32_t pcol = pcol0 + (uint32_t)(b * BPU * npad);
       for (int m0 = 0; m0 < p.M; m0 += 16) {
-        uint32_t pv[16], rv[16];
-        tc_ld_x16(lane_base + pcol + m0, pv);
-        if (!seg_first) tc_ld_x16(lane_base + kRCol + m0, rv);
+        uint32_t pv[BPU][16], rv[16];
+#pragma unroll
+        for (int h = 0; h < BPU; ++h) tc_ld_x16(lane_base + pcol + (uint32_t)(h * npad + m0), pv[h]);
+        if (!seg_first) tc_ld_x16(lane_base + kR + m0, rv);
         tc_wait_ld();
         float y[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          y[j] = seg_first ? sc * __uint_as_float(pv[j]) : fmaf(sc, __uint_as_float(pv[j]), __uint_as_float(rv[j]));
+        for (int j = 0; j < 16; ++j) {
+          float acc = seg_first ? sc[0] * __uint_as_float(pv[0][j]) : fmaf(sc[0], __uint_as_float(pv[0][j]), __uint_as_float(rv[j]));
+#pragma unroll
+          for (int h = 1; h < BPU; ++h) acc = fmaf(sc[h], __uint_as_float(pv[h][j]), acc);
+          y[j] = acc;
+        }
         if (!seg_last) {
           uint32_t o[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(y[j]);
-          tc_st_x16(lane_base + kRCol + m0, o);
+          tc_st_x16(lane_base + kR + m0, o);
         } else if (complete) {
           if (p.verify) warp_argmax(p, n, m0, y, s_val, s_idx, q, lane);
           else write_y(p, n, m0, y);
@@ -532,7 +562,7 @@ bool fp8_supported(long long M, long long K) {
 }
 
 struct Fp8Plan {
-  int npad, np, tiles, kbs, grid, stages;
+  int npad, bpu, np, tiles, kus, grid, stages;
   long long units;
   uint32_t stage_bytes;
   size_t smem;
@@ -541,13 +571,17 @@ struct Fp8Plan {
 static Fp8Plan fp8_plan(long long M, long long N, long long K) {
   Fp8Plan pl{};
   pl.npad = (int)std::max<long long>(16, (M + 15) / 16 * 16);
-  pl.np = std::min(kMaxP, (int)((512 - kRCol - pl.npad) / pl.npad));
+  // TMEM: two A buffers (64 columns per block each), R (npad), np rotating P sets (bpu * npad
+  // each). Two blocks per unit while that leaves at least two P sets.
+  const long long kbs = K / kKB;
+  pl.bpu = (kbs % 2 == 0 && (512 - 2 * 2 * kACols - pl.npad) / (2 * pl.npad) >= 2) ? 2 : 1;
+  pl.np = std::min(kMaxP, (512 - 2 * pl.bpu * kACols - pl.npad) / (pl.bpu * pl.npad));
   pl.tiles = (int)((N + kTileRows - 1) / kTileRows);
-  pl.kbs = (int)(K / kKB);
-  pl.units = (long long)pl.tiles * pl.kbs;
+  pl.kus = (int)(kbs / pl.bpu);
+  pl.units = (long long)pl.tiles * pl.kus;
   const int sms = std::max(1, device_sm_count());
   pl.grid = (int)std::min<long long>(sms, pl.units);
-  pl.stage_bytes = kWBytes + (uint32_t)pl.npad * 256u;
+  pl.stage_bytes = (uint32_t)pl.bpu * (kWBytes + (uint32_t)pl.npad * 256u);
   const size_t budget = 227 * 1024 - 1024 - kTailBytes;
   pl.stages = (int)std::min<size_t>(kMaxStages, budget / pl.stage_bytes);
   pl.smem = 1024 + (size_t)pl.stages * pl.stage_bytes + kTailBytes;
@@ -586,7 +620,7 @@ static int launch_fp8(const uint16_t* X, const uint8_t* q, const float* scales, 
   p.N = N;
   p.K = K;
   p.tiles = pl.tiles;
-  p.kbs = pl.kbs;
+  p.kus = pl.kus;
   p.units = pl.units;
   p.grid = pl.grid;
   p.stages = pl.stages;
@@ -609,11 +643,13 @@ static int launch_fp8(const uint16_t* X, const uint8_t* q, const float* scales, 
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev].load(std::memory_order_acquire)) {
-    if (cudaFuncSetAttribute(fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
+    if (cudaFuncSetAttribute(fp8_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess ||
+        cudaFuncSetAttribute(fp8_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
       return check_launch("cudaFuncSetAttribute(fp8_kernel)");
     attr_set[dev].store(true, std::memory_order_release);
   }
-  fp8_kernel<<<pl.grid, kThreads, pl.smem, s>>>(tw, tx, p);
+  if (pl.bpu == 2) fp8_kernel<2><<<pl.grid, kThreads, pl.smem, s>>>(tw, tx, p);
+  else fp8_kernel<1><<<pl.grid, kThreads, pl.smem, s>>>(tw, tx, p);
   return check_launch("fp8_kernel");
 }
 

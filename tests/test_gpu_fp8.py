@@ -62,7 +62,8 @@ def test_fp8_pack_bit_exact(nv, N, K):
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 1000, 256), (17, 3000, 1024), (68, 777, 768), (128, 4096, 5120),
-                                   (5, 130, 128), (17, 640, 5120), (17, 128, 16384)])
+                                   (5, 130, 128), (17, 640, 5120), (17, 128, 16384), (40, 1000, 1024),
+                                   (49, 333, 512)])
 def test_fp8_gemm(nv, M, N, K):
     W, x = S.block_varied_case(1000 + M + N, M, N, K)
     q, s, codes_ref, scales_ref = packed(nv, W)
