@@ -27,6 +27,11 @@ class VerifySpec(ctypes.Structure):
                 ("max_logit", c_p), ("parents", c_p), ("accept_node", c_p)]
 
 
+class Fp8Problem(ctypes.Structure):
+    """fp8_gemm_problem: one GEMM of an FP8 weight pass."""
+    _fields_ = [("X", c_p), ("q", c_p), ("scales", c_p), ("N", c_i64), ("K", c_i64), ("Y", c_p), ("y_dtype", c_i32)]
+
+
 class PassState(ctypes.Structure):
     """nvfp4_pass: caller-owned host state of an initialised pass."""
     _fields_ = [("opaque", ctypes.c_uint64 * 32)]
@@ -68,6 +73,10 @@ SIGNATURES = {
     "fp8_lmhead_verify_workspace_bytes": (c_sz, [c_i64, c_i64, c_i64]),
     "fp8_lmhead_verify": (ctypes.c_int, [c_p, c_p, c_p, c_i64, c_i64, c_i64, ctypes.POINTER(VerifySpec), c_p, c_sz,
                                          c_p]),
+    "fp8_pass_workspace_bytes": (c_sz, [ctypes.POINTER(Fp8Problem), c_i32, c_i64, c_i32]),
+    "fp8_pass_init": (ctypes.c_int, [ctypes.POINTER(PassState), ctypes.POINTER(Fp8Problem), c_i32, c_i64,
+                                     ctypes.POINTER(VerifySpec), c_p, c_sz]),
+    "fp8_pass_run": (ctypes.c_int, [ctypes.POINTER(PassState), c_p]),
 }
 
 _lib = None
