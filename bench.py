@@ -669,6 +669,90 @@ def run_fp8(args):
                 "steps": args.steps, "warmup": args.warmup, "cpu_baseline": cpu}), flush=True)
 
 
+def run_mixed(args):
+    """The pages' precision map for the 27B step: per layer the gate+up and down projections
+    in NVFP4 and the qkv projection in FP8 (E4M3, 128x128 fp32 block scales), then an FP8
+    lm_head with the fused verify. One NVFP4 pass (128 GEMMs) and one FP8 pass (64 GEMMs and
+    the head), captured together in one CUDA graph and timed by CUDA events. One JSON line per
+    M with the weight GB/s against the HBM roofline."""
+    import torch
+    import nvfp4_weight_streaming_gemm_b200 as nv
+    from nvfp4_weight_streaming_gemm_b200 import build as nvbuild
+    nvbuild.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    nv4, f8 = [], []
+    for layer in range(args.layers):
+        for j, name in enumerate(S.LAYER_ORDER):
+            K, N = S.LAYER_SHAPES[name]
+            g = torch.Generator(device=dev)
+            g.manual_seed(1000 * layer + j)
+            W = torch.randn(N, K, generator=g, device=dev, dtype=torch.float32).mul_(S.W_STD)
+            if name == "qkv":
+                f8.append((K, N) + nv.fp8_pack(W))
+            else:
+                nv4.append((K, N) + nv.pack(W))
+            del W
+    g = torch.Generator(device=dev)
+    g.manual_seed(S.LMHEAD_W_SEED)
+    W = torch.randn(S.VOCAB, S.LMHEAD_K, generator=g, device=dev, dtype=torch.float32).mul_(S.W_STD)
+    qh, sh = nv.fp8_pack(W)
+    del W
+    torch.cuda.synchronize()
+    wbytes = (sum(weight_bytes(N, K) for (K, N, _, _, _) in nv4) +
+              sum(N * K + sc.numel() * 4 for (K, N, _, sc) in f8) + S.VOCAB * S.LMHEAD_K + sh.numel() * 4)
+    hbm, hbm_kind = measured_peaks()
+    st = torch.cuda.current_stream()
+    for M in [int(m) for m in args.ms.split(",")]:
+        B = max(1, M // (S.DRAFT_LEN + 1))
+        D = M // B - 1
+        if B * (D + 1) != M:
+            raise SystemExit(f"--mixed: M={M} is not B*(D+1)")
+        gx = torch.Generator(device=dev)
+        gx.manual_seed(11 + M)
+        p4 = nv.WeightPass([(torch.randn(M, K, generator=gx, device=dev).to(torch.bfloat16), q, sf, ts,
+                             torch.empty((M, N), dtype=torch.bfloat16, device=dev)) for (K, N, q, sf, ts) in nv4], M)
+        drafts = torch.zeros((B, D), dtype=torch.int32, device=dev)
+        t = torch.empty(M, dtype=torch.int32, device=dev)
+        L = torch.empty(B, dtype=torch.int32, device=dev)
+        probs8 = [(torch.randn(M, K, generator=gx, device=dev).to(torch.bfloat16), q, sc,
+                   torch.empty((M, N), dtype=torch.bfloat16, device=dev)) for (K, N, q, sc) in f8]
+        probs8.append((torch.randn(M, S.LMHEAD_K, generator=gx, device=dev).to(torch.bfloat16), qh, sh, None))
+        p8 = nv.Fp8Pass(probs8, M, verify=(drafts, t, L, None))
+        s = torch.cuda.Stream()
+        s.wait_stream(st)
+        with torch.cuda.stream(s):
+            p4.run(s)
+            p8.run(s)
+        st.wait_stream(s)
+        torch.cuda.synchronize()
+        nv.check()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            p4.run()
+            p8.run()
+        for _ in range(args.warmup):
+            graph.replay()
+        torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+        ev[0].record(st)
+        for k in range(args.steps):
+            graph.replay()
+            ev[k + 1].record(st)
+        torch.cuda.synchronize()
+        nv.check()
+        per = np.array([ev[k].elapsed_time(ev[k + 1]) for k in range(args.steps)])
+        ms = ev[0].elapsed_time(ev[-1]) / args.steps
+        gbs = wbytes / (ms * 1e-3) / 1e9
+        print(json.dumps({
+            "metric": "27B step with the pages' precision map (NVFP4 MLP, FP8 qkv and lm_head verify)", "M": M,
+            "layers": args.layers, "ms_per_step": ms, "ms_min": float(per.min()), "weight_bytes": wbytes,
+            "weight_gbs": gbs, "hbm_frac": gbs / hbm, "hbm_peak_kind": hbm_kind, "y_dtype": "bf16",
+            "steps": args.steps, "warmup": args.warmup}), flush=True)
+        del graph, p4, p8, probs8
+        torch.cuda.synchronize()
+
+
 def run_reference(args, rank, world):
     """The CPU oracle timed as it stands: each step dequantises and multiplies one qkv
     matrix (5120->10240) in float64 at M=17. That is a bounded sample of the pass, in
@@ -720,6 +804,8 @@ def main():
     ap.add_argument("--binv", action="store_true", help="batch-invariant passes (same row bits for every M)")
     ap.add_argument("--w4a4", action="store_true",
                     help="time W4A4 passes (NVFP4 activations) over the stack at the --ms values, e.g. 128,256")
+    ap.add_argument("--mixed", action="store_true",
+                    help="the 27B step with NVFP4 MLP weights and an FP8 qkv projection and lm_head")
     ap.add_argument("--fp8", action="store_true",
                     help="the FP8 (E4M3, 128x128 block-scaled) output head: verify and GEMM per M")
     ap.add_argument("--sweep", action="store_true", help="time one matrix shape per M and path (no pass)")
@@ -738,6 +824,8 @@ def main():
         run_w4a4(args)
     elif args.fp8:
         run_fp8(args)
+    elif args.mixed:
+        run_mixed(args)
     elif args.impl == "reference":
         run_reference(args, rank, world)
     else:

@@ -415,6 +415,59 @@ int fp8_lmhead_verify(const void* X, const uint8_t* q, const float* scales, int6
                       nvfp4ws_stream_t stream);
 
 /*
+ * FP8 weight passes -- a list of independent FP8 GEMMs that share M, run by ONE persistent
+ * launch, optionally ending with the fused verify over an FP8 lm_head.
+ *
+ * Passages: "TandemLLM", "How it works" (one decode step reads every weight once) and "The
+ * parts" (the FP8 attention projections and head beside the 4-bit weights). As for NVFP4
+ * passes, the units of all the problems (128-row tile x 128- or 256-wide K range) form one
+ * sequence split evenly across the SMs. Each problem computes what fp8_gemm_skinny computes.
+ * The problems run concurrently in no particular order: no problem's X may be another
+ * problem's Y. With `verify` non-NULL the LAST problem is the lm_head: its Y is ignored and
+ * the pass ends with the argmax and accept rule of fp8_lmhead_verify. An NVFP4 pass and an
+ * FP8 pass can be enqueued back to back (or captured in one CUDA graph) to stream a model
+ * whose matrices use both formats.
+ *
+ * fp8_pass_workspace_bytes -- device workspace for this list (verify_last != 0 when the last
+ *   problem is the verify problem); 0 when the list is invalid.
+ * fp8_pass_init -- validates the list, lays out the workspace and writes the problems'
+ *   descriptors into it with a SYNCHRONOUS copy (call it at set-up, outside stream capture).
+ *   The workspace must be zero-filled before the first run; every run leaves it reusable.
+ *   The pointers given are baked into the pass.
+ * fp8_pass_run -- enqueues the pass on `stream` (2 kernels with verify, else 1). It can be
+ *   captured in a CUDA graph.
+ *
+ * Arguments
+ *   problems[i]   X: bf16 [M, K], device, 16-byte aligned.  q, scales: as written by fp8_pack.
+ *                 N >= 1.  K a positive multiple of 128.  Y: [M, N] fp32 or bf16 per y_dtype,
+ *                 16-byte aligned (ignored for the verify problem).
+ *   count         >= 1.
+ *   M             1 <= M <= 128.
+ *   verify        NULL, or the verify rule and buffers (nvfp4_verify_spec): M must equal
+ *                 B * (D + 1); parents NULL for the chain rule.
+ *   pass          caller-owned host state, filled by fp8_pass_init (an nvfp4_pass handle;
+ *                 nvfp4_pass_run refuses it).
+ * Returns NVFP4WS_OK, or INVALID_ARG / UNSUPPORTED / MISALIGNED / WORKSPACE / CUDA.
+ */
+typedef struct fp8_gemm_problem {
+  uint32_t struct_size;    /* = NVFP4WS_FP8_PROBLEM_SIZE (see nvfp4_gemm_problem) */
+  const void* X;
+  const uint8_t* q;
+  const float* scales;
+  int64_t N;
+  int64_t K;
+  void* Y;
+  int32_t y_dtype;
+} fp8_gemm_problem;
+
+#define NVFP4WS_FP8_PROBLEM_SIZE ((uint32_t)sizeof(fp8_gemm_problem))
+
+size_t fp8_pass_workspace_bytes(const fp8_gemm_problem* problems, int32_t count, int64_t M, int32_t verify_last);
+int fp8_pass_init(nvfp4_pass* pass, const fp8_gemm_problem* problems, int32_t count, int64_t M,
+                  const nvfp4_verify_spec* verify, void* workspace, size_t workspace_bytes);
+int fp8_pass_run(const nvfp4_pass* pass, nvfp4ws_stream_t stream);
+
+/*
  * nvfp4_gemm_skinny_noalloc -- the tensor-core GEMM of nvfp4_gemm_skinny for callers
  * that cannot allocate device memory and so cannot pass a workspace. Examples are a
  * host that fixes its device-memory plan at start-up and forbids later allocation,

@@ -332,3 +332,65 @@ class WeightPass:
 
     def run(self, stream=None):
         _check(lib().nvfp4_pass_run(ctypes.byref(self.state), _stream(stream)), "nvfp4_pass_run")
+
+
+class Fp8Pass:
+    """A list of independent FP8 GEMMs sharing M, run by one persistent launch (``fp8_pass_*``).
+
+    ``problems`` is a list of ``(X, q, scales, Y)``: X bf16 [M, K], the weight from
+    :func:`fp8_pack`, and Y fp32 or bf16 [M, N]. ``verify`` is as for :class:`WeightPass`:
+    ``(drafts, argmax, accept_len, max_logit[, parents, accept_node])``, and makes the last
+    problem the lm_head (its Y may be None). Every tensor is referenced by address: keep
+    them alive and refill X in place between runs.
+    """
+
+    def __init__(self, problems, M: int, verify=None, workspace: torch.Tensor | None = None):
+        L = _lib
+        n = len(problems)
+        self._keep = []
+        arr = (L.Fp8Problem * n)()
+        for i, (X, q, scales, Y) in enumerate(problems):
+            _need_cuda(X, "X", torch.bfloat16)
+            _need_cuda(q, "q", torch.uint8)
+            _need_cuda(scales, "scales", torch.float32)
+            if X.shape[0] != M:
+                raise ValueError(f"problem {i}: X has {X.shape[0]} rows, expected M={M}")
+            K = X.shape[1]
+            N = q.shape[0]
+            if q.shape[1] != K or scales.shape != ((N + 127) // 128, (K + 127) // 128):
+                raise ValueError(f"problem {i}: q / scales shapes do not match X")
+            yd = 0
+            if Y is not None:
+                _need_cuda(Y, "Y")
+                if Y.shape != (M, N):
+                    raise ValueError(f"problem {i}: Y must be [{M}, {N}]")
+                yd = {torch.float32: 0, torch.bfloat16: 1}[Y.dtype]
+            arr[i] = L.Fp8Problem(_ptr(X), _ptr(q), _ptr(scales), N, K, _ptr(Y), yd)
+            self._keep.extend([X, q, scales, Y])
+        vs = None
+        if verify is not None:
+            drafts, amax, acc, vmax = verify[:4]
+            parents, node = (tuple(verify[4:]) + (None, None))[:2]
+            _need_cuda(drafts, "drafts", torch.int32)
+            B, D = drafts.shape
+            if parents is not None:
+                _need_cuda(parents, "parents", torch.int32)
+                if parents.shape != (B, D):
+                    raise ValueError("parents must have the shape of drafts")
+            vs = L.VerifySpec(_ptr(drafts) if drafts.numel() else None, B, D, _ptr(amax), _ptr(acc), _ptr(vmax),
+                              _ptr(parents) if parents is not None and parents.numel() else None, _ptr(node))
+            self._keep.extend([drafts, amax, acc, vmax, parents, node])
+        nbytes = int(lib().fp8_pass_workspace_bytes(arr, n, M, 1 if verify is not None else 0))
+        if nbytes == 0:
+            raise NVFP4WSError(1, "fp8_pass_workspace_bytes")
+        dev = problems[0][0].device
+        self.workspace = _workspace(nbytes, dev, workspace)
+        self.workspace_bytes = nbytes
+        self.state = L.PassState()
+        _check(lib().fp8_pass_init(ctypes.byref(self.state), arr, n, M, ctypes.byref(vs) if vs is not None else None,
+                                   _ptr(self.workspace), nbytes), "fp8_pass_init")
+        self.M = M
+        self.count = n
+
+    def run(self, stream=None):
+        _check(lib().fp8_pass_run(ctypes.byref(self.state), _stream(stream)), "fp8_pass_run")

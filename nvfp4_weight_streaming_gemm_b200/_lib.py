@@ -35,6 +35,15 @@ class VerifySpec(ctypes.Structure):
         super().__init__(ctypes.sizeof(VerifySpec), *args, **kw)
 
 
+class Fp8Problem(ctypes.Structure):
+    """fp8_gemm_problem: one GEMM of an FP8 weight pass. ``struct_size`` is filled in by the constructor."""
+    _fields_ = [("struct_size", ctypes.c_uint32), ("X", c_p), ("q", c_p), ("scales", c_p), ("N", c_i64),
+                ("K", c_i64), ("Y", c_p), ("y_dtype", c_i32)]
+
+    def __init__(self, *args, **kw):
+        super().__init__(ctypes.sizeof(Fp8Problem), *args, **kw)
+
+
 class PassState(ctypes.Structure):
     """nvfp4_pass: caller-owned host state of an initialised pass."""
     _fields_ = [("opaque", ctypes.c_uint64 * 32)]
@@ -76,6 +85,10 @@ SIGNATURES = {
     "fp8_lmhead_verify_workspace_bytes": (c_sz, [c_i64, c_i64, c_i64]),
     "fp8_lmhead_verify": (ctypes.c_int, [c_p, c_p, c_p, c_i64, c_i64, c_i64, ctypes.POINTER(VerifySpec), c_p, c_sz,
                                          c_p]),
+    "fp8_pass_workspace_bytes": (c_sz, [ctypes.POINTER(Fp8Problem), c_i32, c_i64, c_i32]),
+    "fp8_pass_init": (ctypes.c_int, [ctypes.POINTER(PassState), ctypes.POINTER(Fp8Problem), c_i32, c_i64,
+                                     ctypes.POINTER(VerifySpec), c_p, c_sz]),
+    "fp8_pass_run": (ctypes.c_int, [ctypes.POINTER(PassState), c_p]),
 }
 
 _lib = None

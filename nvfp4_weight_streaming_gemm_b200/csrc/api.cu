@@ -498,6 +498,79 @@ int fp8_lmhead_verify(const void* X, const uint8_t* q, const float* scales, int6
   return launch_fp8_verify(static_cast<const uint16_t*>(X), q, scales, M, N, K, v, workspace, (cudaStream_t)stream);
 }
 
+static int fp8_host_problems(const fp8_gemm_problem* problems, int32_t count, int64_t M, int verify_last,
+                             std::vector<Fp8HostProblem>* out, const char* who) {
+  if (!problems || count < 1) return set_error(NVFP4WS_ERR_INVALID_ARG, "%s: need count >= 1 problems", who);
+  for (int32_t i = 0; i < count; ++i)
+    if (problems[i].struct_size != NVFP4WS_FP8_PROBLEM_SIZE)
+      return set_error(NVFP4WS_ERR_INVALID_ARG, "%s: problem %d: struct_size %u, this library expects %u (rebuild "
+                       "against this nvfp4ws.h)", who, i, problems[i].struct_size, NVFP4WS_FP8_PROBLEM_SIZE);
+  out->clear();
+  for (int32_t i = 0; i < count; ++i) {
+    const fp8_gemm_problem& p = problems[i];
+    const bool v = verify_last && i == count - 1;
+    if (!p.X || !p.q || !p.scales) return set_error(NVFP4WS_ERR_INVALID_ARG, "%s: problem %d: null input", who, i);
+    if (p.N < 1 || p.N > (int64_t)0x7fffffff)
+      return set_error(NVFP4WS_ERR_INVALID_ARG, "%s: problem %d: N=%lld out of range", who, i, (long long)p.N);
+    if (!fp8_supported(M, p.K))
+      return set_error(NVFP4WS_ERR_UNSUPPORTED, "%s: problem %d: needs 1 <= M <= 128 and K a positive multiple of 128 "
+                       "(M=%lld K=%lld)", who, i, (long long)M, (long long)p.K);
+    if (!aligned16(p.X) || !aligned16(p.q))
+      return set_error(NVFP4WS_ERR_MISALIGNED, "%s: problem %d: X and q must be 16-byte aligned", who, i);
+    if ((uintptr_t)p.scales & 3u)
+      return set_error(NVFP4WS_ERR_MISALIGNED, "%s: problem %d: scales must be 4-byte aligned", who, i);
+    if (!v) {
+      if (!p.Y) return set_error(NVFP4WS_ERR_INVALID_ARG, "%s: problem %d: Y is null", who, i);
+      if (!aligned16(p.Y)) return set_error(NVFP4WS_ERR_MISALIGNED, "%s: problem %d: Y must be 16-byte aligned", who, i);
+      if (p.y_dtype != NVFP4WS_Y_F32 && p.y_dtype != NVFP4WS_Y_BF16)
+        return set_error(NVFP4WS_ERR_INVALID_ARG, "%s: problem %d: bad y_dtype %d", who, i, p.y_dtype);
+    }
+    out->push_back(Fp8HostProblem{static_cast<const uint16_t*>(p.X), p.q, p.scales, p.N, p.K, v ? nullptr : p.Y,
+                                  (!v && p.y_dtype == NVFP4WS_Y_BF16) ? 1 : 0, v ? 1 : 0});
+  }
+  return NVFP4WS_OK;
+}
+
+size_t fp8_pass_workspace_bytes(const fp8_gemm_problem* problems, int32_t count, int64_t M, int32_t verify_last) {
+  std::vector<Fp8HostProblem> hp;
+  if (fp8_host_problems(problems, count, M, verify_last, &hp, "fp8_pass_workspace_bytes") != NVFP4WS_OK) return 0;
+  return fp8_pass_workspace_bytes_int(hp.data(), count, M);
+}
+
+int fp8_pass_init(nvfp4_pass* pass, const fp8_gemm_problem* problems, int32_t count, int64_t M,
+                  const nvfp4_verify_spec* verify, void* workspace, size_t workspace_bytes) {
+  g_last_error[0] = 0;
+  static_assert(sizeof(nvfp4_pass) >= kFp8PassStateBytes, "nvfp4_pass is too small for the FP8 pass state");
+  if (!pass) return set_error(NVFP4WS_ERR_INVALID_ARG, "fp8_pass_init: pass is null");
+  std::memset(pass, 0, sizeof(nvfp4_pass));
+  if (verify)
+    if (int e = check_verify_size(verify, "fp8_pass_init")) return e;
+  std::vector<Fp8HostProblem> hp;
+  if (int e = fp8_host_problems(problems, count, M, verify != nullptr, &hp, "fp8_pass_init")) return e;
+  VerifyRule vs{};
+  if (verify) {
+    if (verify->B < 1 || verify->D < 0)
+      return set_error(NVFP4WS_ERR_INVALID_ARG, "fp8_pass_init: verify needs B >= 1 and D >= 0");
+    if ((int64_t)verify->B * (verify->D + 1) != M)
+      return set_error(NVFP4WS_ERR_INVALID_ARG, "fp8_pass_init: M=%lld must equal B*(D+1)=%lld", (long long)M,
+                       (long long)verify->B * (verify->D + 1));
+    if (verify->D > 0 && !verify->drafts) return set_error(NVFP4WS_ERR_INVALID_ARG, "fp8_pass_init: drafts is null");
+    if (!verify->argmax || !verify->accept_len)
+      return set_error(NVFP4WS_ERR_INVALID_ARG, "fp8_pass_init: null verify output pointer");
+    vs = VerifyRule{verify->drafts, verify->D > 0 ? verify->parents : nullptr, verify->B, verify->D, verify->argmax,
+                    verify->accept_len, verify->accept_node, verify->max_logit};
+  }
+  if (!workspace) return set_error(NVFP4WS_ERR_WORKSPACE, "fp8_pass_init: workspace is null");
+  if (!aligned16(workspace)) return set_error(NVFP4WS_ERR_MISALIGNED, "fp8_pass_init: workspace must be 16-byte aligned");
+  return fp8_pass_init_int(pass->opaque, hp.data(), count, M, verify ? &vs : nullptr, workspace, workspace_bytes);
+}
+
+int fp8_pass_run(const nvfp4_pass* pass, nvfp4ws_stream_t stream) {
+  g_last_error[0] = 0;
+  if (!pass) return set_error(NVFP4WS_ERR_INVALID_ARG, "fp8_pass_run: pass is null");
+  return fp8_pass_run_int(pass->opaque, (cudaStream_t)stream);
+}
+
 int nvfp4ws_check(nvfp4ws_stream_t stream) {
   g_last_error[0] = 0;
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);

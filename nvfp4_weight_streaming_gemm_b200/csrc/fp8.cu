@@ -1,4 +1,5 @@
-// FP8 (E4M3) block-scaled weight GEMM and fused verify on the tcgen05 tensor cores (sm_100a).
+// FP8 (E4M3) block-scaled weight GEMMs and fused verify on the tcgen05 tensor cores (sm_100a):
+// one GEMM, or a whole list of them (an FP8 weight pass) in one persistent launch.
 //
 //   Y[m, n] = sum_kb s[n / 128, kb] * sum_{k in block kb} x16[m, k] * e4m3(code[n, k])
 //
@@ -8,36 +9,43 @@
 // name no block shape; 128 x 128 is the reading taken here.
 //
 // Exactness. An E4M3 value has at most 4 significant bits and lies in [2^-9, 448], so it is
-// exact in f16, as is the activation for |x| in [2^-14, 65504] (bf16 -> f16, nearest,
-// saturating). Every product is then exact in the fp32 accumulator. The block scale is an
-// arbitrary fp32 and would round if folded into either f16 operand, so a unit of work is one
-// 128 x 128 block: the tensor core sums the block's 128 products per (row, token) into a fresh
-// TMEM buffer P, and the epilogue promotes it into a running sum R = s * P, then R += s * P,
-// in fp32 (R also lives in TMEM).
+// exact in f16. Each activation row is multiplied by a power of two 2^-e (e from the row's
+// amax, computed by fp8_x_shift_kernel first) so that its amax lies in [2^14, 2^15): the
+// bf16 -> f16 conversion is then exact for every value above 2^-25 of the amax and never
+// saturates, and the output is multiplied by 2^e. Every product is exact in the fp32
+// accumulator. The block scale is an
+// arbitrary fp32 and would round if folded into either f16 operand, so the tensor core sums
+// each 128 x 128 block's 128 products per (row, token) into a fresh TMEM buffer P, and the
+// epilogue promotes it into a running sum R = s * P, then R += s * P, in fp32 (R also lives
+// in TMEM). A unit of work is BPU = 1 or 2 such blocks of one 128-row tile: two while TMEM
+// leaves room for two rotating P sets (npad <= 48) and every problem's K is a multiple of 256,
+// which halves the per-unit hand-offs per weight byte.
 //
 // Roles per CTA (one persistent CTA per SM, 16 warps):
-//   warp 0        TMA producer: the 16 KB code tile (128 rows x 128 B, 128-byte swizzle) and
-//                 the unit's bf16 X slice (two 64-wide swizzled atoms) into a ring of stages.
+//   warp 0        TMA producer: the unit's 16 KB code tiles (128 rows x 128 B, 128-byte
+//                 swizzle) and its bf16 X slice (2*BPU 64-wide swizzled atoms) into a ring.
 //                 No multicast.
 //   warp 1        TMEM allocator and the single MMA-issuing thread: 8 x kind::f16 (K = 16)
-//                 per unit, A from TMEM, B from shared memory, into one of np rotating P
-//                 buffers.
+//                 per block, A from TMEM, B from shared memory, each block into its own P of
+//                 one of np rotating P sets.
 //   warps 4-7,    two dequantisation warpgroups taking alternate units. Each thread owns one
 //   warps 8-11    weight row (its TMEM lane): E4M3 pairs -> f16 pairs (cvt.rn.f16x2.e4m3x2)
 //                 written into TMEM as the A operand. The same threads convert the unit's X
 //                 rows from bf16 to f16 in place.
 //   warps 12-15   promotion and epilogue: at the end of a tile's K range, Y (or the tile's
-//                 per-token argmax in verify mode, or a split-K partial).
+//                 per-token argmax for the verify problem, or a split-K partial).
 //
-// TMEM columns (512, one CTA per SM): [0, 64) and [64, 128) the two A buffers (64 f16 pairs
-// per row), [128, 128 + npad) R, then np P buffers of npad columns.
+// TMEM columns (512, one CTA per SM): two A buffers of 64*BPU columns (64 f16 pairs per row
+// and block), then R (npad columns), then np P sets of BPU*npad columns.
 //
-// Scheduling is stream-K: the (tile, K-block) units are cut into equal contiguous ranges, one
-// per CTA. A tile whose K range spans several CTAs is finished by the last to arrive: each
-// publishes its fp32 partial, takes a ticket, and the holder of the last ticket sums the
-// partials in K order, so results are deterministic and no CTA waits for another. Every
-// mbarrier wait is bounded; on expiry the thread records kDevErrWaitTimeout and the CTA
-// winds down (drains its copies and MMAs, frees its TMEM).
+// Scheduling is stream-K over the concatenated (problem, tile, K-range) units of all the
+// launch's problems: they are cut into equal contiguous ranges, one per CTA, so every SM
+// streams the same number of bytes however the list's shapes fall. A tile whose K range spans
+// several CTAs is finished by the last to arrive: each publishes its fp32 partial, takes a
+// ticket, and the holder of the last ticket sums the partials in K order, so results are
+// deterministic and no CTA waits for another. Every mbarrier wait is bounded; on expiry the
+// thread records kDevErrWaitTimeout and the CTA winds down (drains its copies and MMAs, frees
+// its TMEM).
 #include "common.cuh"
 #include "fp8.h"
 #include "kernels.h"
@@ -50,37 +58,51 @@
 #include <atomic>
 #include <climits>
 #include <cmath>
+#include <cstring>
+#include <vector>
 
 namespace nvfp4ws {
 namespace fp8k {
 
 constexpr int kThreads = 512;
 constexpr int kTileRows = 128;
-constexpr int kKB = kFp8Block;                       // K elements per unit = one scale block
-constexpr uint32_t kWBytes = kTileRows * kKB;        // 16 KB of codes per unit
+constexpr int kKB = kFp8Block;                       // K elements of one scale block
+constexpr uint32_t kWBytes = kTileRows * kKB;        // 16 KB of codes per block
 constexpr int kMaxNpad = 128;
-constexpr int kACols = kKB / 2;                      // f16 pairs per row = TMEM columns per A buffer
-constexpr uint32_t kRCol = 2 * kACols;               // running sums after the two A buffers
+constexpr int kACols = kKB / 2;                      // f16 pairs per row and block = TMEM columns
 constexpr int kMaxP = 4;
 constexpr int kMaxStages = 8;
 constexpr size_t kTailBytes = 8192;
 
+// One GEMM of a launch. A pass keeps an array of these in device memory; TMA reads the tensor
+// maps from there.
+struct alignas(64) Problem {
+  CUtensorMap tm_w;        // codes [N, K] u8, box 128 B x 128 rows, 128-byte swizzle
+  CUtensorMap tm_x;        // X [M, K] bf16, box 64 x npad, 128-byte swizzle
+  const float* scales;     // [tiles][K / 128]
+  void* Y;                 // [M, N] fp32 or bf16 (unused by the verify problem)
+  float* part_val;         // verify problem: per-tile row maxima [tiles][M]
+  int* part_idx;           //                 and their indices
+  long long N;
+  long long unit0;         // first unit of this problem in the launch's numbering
+  int tile0;               // first ticket counter of this problem
+  int kus;                 // units per tile: K / (128 * BPU)
+  int tiles, y_bf16, verify;
+  const uint16_t* X;       // [M, K] bf16 (read by the row-shift kernel)
+  long long K;
+  int* xe;                 // [M] power-of-two shift of each X row (fp8_x_shift_kernel)
+};
+
 struct Params {
-  float* Y;                // fp32 or bf16 (y_bf16)
-  int y_bf16;
-  const float* scales;     // [tiles][kbs]
+  const Problem* probs;    // device array of a pass, or nullptr: the single problem passed by value
+  int nprob;
   int M, npad, np;
-  long long N, K;
-  int tiles, kbs;
   long long units;
   int grid;
   int stages;
   uint32_t stage_bytes;
-  unsigned int* counters;  // [tiles], zero between calls
+  unsigned int* counters;  // [tiles of all problems], zero between calls
   float* partials;         // [2 * grid][M][128]
-  int verify;
-  float* part_val;         // [tiles][M]
-  int* part_idx;
   unsigned int* err;
 };
 
@@ -160,30 +182,54 @@ __device__ __forceinline__ int cta_of_unit(long long u, long long U, int G) {
   return c;
 }
 
+// Position of a unit: its problem, the tile within that problem and the unit within the tile.
+struct Cursor {
+  int pi;
+  long long tile;
+  int ku;
+  __device__ __forceinline__ void init(const Problem* probs, int nprob, long long u) {
+    pi = 0;
+    while (pi + 1 < nprob && probs[pi + 1].unit0 <= u) ++pi;
+    const Problem& pr = probs[pi];
+    const long long r = u - pr.unit0;
+    tile = r / pr.kus;
+    ku = (int)(r - tile * pr.kus);
+  }
+  // Steps to the next unit. Past the launch's last unit pi equals nprob; do not read it then.
+  __device__ __forceinline__ void next(const Problem* probs) {
+    const Problem& pr = probs[pi];
+    if (++ku == pr.kus) {
+      ku = 0;
+      if (++tile == pr.tiles) { tile = 0; ++pi; }
+    }
+  }
+};
+
 // ---------------------------------------------------------------- epilogue pieces
 
-// Writes y for tokens [m0, m0+16) of weight row n.
-__device__ __forceinline__ void write_y(const Params& p, long long n, int m0, const float (&y)[16]) {
-  if (n >= p.N) return;
+// Writes y for tokens [m0, m0+16) of weight row n of problem pr.
+__device__ __forceinline__ void write_y(const Params& p, const Problem& pr, long long n, int m0,
+                                        const float (&y)[16]) {
+  if (n >= pr.N) return;
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
     const int m = m0 + j;
     if (m < p.M) {
-      if (p.y_bf16)
-        reinterpret_cast<uint16_t*>(p.Y)[(long long)m * p.N + n] = f32_to_bf16_rn(y[j]);
+      if (pr.y_bf16)
+        reinterpret_cast<uint16_t*>(pr.Y)[(long long)m * pr.N + n] = f32_to_bf16_rn(y[j]);
       else
-        p.Y[(long long)m * p.N + n] = y[j];
+        reinterpret_cast<float*>(pr.Y)[(long long)m * pr.N + n] = y[j];
     }
   }
 }
 
 // Per-token argmax over the 32 rows of this warp; lane 0 stages the warp's winner.
-__device__ __forceinline__ void warp_argmax(const Params& p, long long n, int m0, const float (&y)[16], float* s_val,
-                                            int* s_idx, int q, int lane) {
+__device__ __forceinline__ void warp_argmax(const Problem& pr, long long n, int m0, const float (&y)[16],
+                                            float* s_val, int* s_idx, int q, int lane) {
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
-    float v = (n < p.N) ? y[j] : -INFINITY;
-    int i = (n < p.N) ? (int)n : INT_MAX;
+    float v = (n < pr.N) ? y[j] : -INFINITY;
+    int i = (n < pr.N) ? (int)n : INT_MAX;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       const float ov = __shfl_xor_sync(0xffffffffu, v, o);
@@ -195,8 +241,8 @@ __device__ __forceinline__ void warp_argmax(const Params& p, long long n, int m0
 }
 
 // Combines the 4 warps' staged winners into the tile's partial (one thread per token).
-__device__ __forceinline__ void tile_argmax_out(const Params& p, int tile, int et, const float* s_val,
-                                                const int* s_idx) {
+__device__ __forceinline__ void tile_argmax_out(const Params& p, const Problem& pr, long long tile, int et,
+                                                const float* s_val, const int* s_idx) {
   if (et >= p.M) return;
   float bv = s_val[et];
   int bi = s_idx[et];
@@ -205,14 +251,21 @@ __device__ __forceinline__ void tile_argmax_out(const Params& p, int tile, int e
       bv = s_val[w * kMaxNpad + et];
       bi = s_idx[w * kMaxNpad + et];
     }
-  p.part_val[(long long)tile * p.M + et] = bv;
-  p.part_idx[(long long)tile * p.M + et] = bi;
+  pr.part_val[tile * p.M + et] = bv;
+  pr.part_idx[tile * p.M + et] = bi;
 }
 
 // ---------------------------------------------------------------- the kernel
 
+// BPU scale blocks (128 K each) per unit. Two blocks per unit halve the per-unit fixed costs
+// (barrier hand-offs, the epilogue's TMEM round trips) per weight byte; the sums are the same
+// fma sequence either way, so the result does not depend on BPU.
+template <int BPU>
 __global__ void __launch_bounds__(kThreads, 1)
-    fp8_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x, const Params p) {
+    fp8_kernel(const __grid_constant__ Problem single, const Params p) {
+  constexpr uint32_t kUW = BPU * kWBytes;           // code bytes per unit
+  constexpr int kUACols = BPU * kACols;             // TMEM columns of one A buffer
+  constexpr uint32_t kR = 2 * kUACols;              // running sums after the two A buffers
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int S = p.stages, NP = p.np;
@@ -224,6 +277,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* s_last = reinterpret_cast<int*>(s_tmem + 2);
   float* s_val = reinterpret_cast<float*>(s_tmem + 4);                  // [4][kMaxNpad]
   int* s_idx = reinterpret_cast<int*>(s_val + 4 * kMaxNpad);            // [4][kMaxNpad]
+  // row shifts of the problem each stage holds, written by the producer before its arrive
+  const int** s_stage_xe = reinterpret_cast<const int**>(s_idx + 4 * kMaxNpad);   // [kMaxStages]
 
   auto bar_full = [&](int s) { return smem_u32(bars + s); };
   auto bar_empty = [&](int s) { return smem_u32(bars + S + s); };
@@ -238,8 +293,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const long long U = p.units;
   const long long u_begin = unit_begin(c, U, p.grid), u_end = unit_begin(c + 1, U, p.grid);
   const int nunits = (int)(u_end - u_begin);
-  const int npad = p.npad, kbs = p.kbs;
-  const uint32_t pcol0 = kRCol + (uint32_t)npad;   // first P buffer
+  const int npad = p.npad;
+  const Problem* probs = p.probs ? p.probs : &single;
+  const uint32_t pcol0 = kR + (uint32_t)npad;      // first P buffer; buffer b, block h at + (b*BPU + h)*npad
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) { mbar_init(bar_full(s), 1); mbar_init(bar_empty(s), 1); }
@@ -263,22 +319,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       const uint64_t pol_w = policy_evict_first(), pol_x = policy_evict_last();
-      const uint32_t tx = kWBytes + (uint32_t)npad * 256u;
+      const uint32_t tx = kUW + (uint32_t)(BPU * npad) * 256u;
       int issued = 0;
-      long long tile = u_begin / kbs;
-      int kb = (int)(u_begin % kbs);
+      Cursor cur;
+      cur.init(probs, p.nprob, u_begin);
       int s = 0;
       uint32_t ph = 0;
       for (int i = 0; i < nunits; ++i) {
         if (!mbar_wait(bar_empty(s), ph ^ 1u, s_abort, p.err)) break;
         uint8_t* st = smem + (size_t)s * p.stage_bytes;
+        const Problem& pr = probs[cur.pi];
+        const int k0 = cur.ku * BPU * kKB;             // first K element of the unit
+        s_stage_xe[s] = pr.xe;                         // published by the arrive below
         mbar_arrive_expect_tx(bar_full(s), tx);
-        tma_load_2d(smem_u32(st), &tm_w, kb * kKB, (int)(tile * kTileRows), bar_full(s), pol_w);
 #pragma unroll
-        for (int a = 0; a < 2; ++a)
-          tma_load_2d(smem_u32(st + kWBytes + a * npad * 128), &tm_x, kb * kKB + a * 64, 0, bar_full(s), pol_x);
+        for (int h = 0; h < BPU; ++h)
+          tma_load_2d(smem_u32(st + h * kWBytes), &pr.tm_w, k0 + h * kKB, (int)(cur.tile * kTileRows), bar_full(s),
+                      pol_w);
+#pragma unroll
+        for (int a = 0; a < 2 * BPU; ++a)
+          tma_load_2d(smem_u32(st + kUW + a * npad * 128), &pr.tm_x, k0 + a * 64, 0, bar_full(s), pol_x);
         issued = i + 1;
-        if (++kb == kbs) { kb = 0; ++tile; }
+        cur.next(probs);
         if (++s == S) { s = 0; ph ^= 1u; }
       }
       if (*s_abort) {       // drain: wait (bounded) for every copy this thread issued
@@ -302,17 +364,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mbar_wait(bar_afull(g), (uint32_t)(i >> 1) & 1u, s_abort, p.err);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t xbase = smem_u32(smem + (size_t)s * p.stage_bytes + kWBytes);
-        const uint32_t d_tmem = tmem + pcol0 + (uint32_t)(b * npad);
-        const uint32_t a_tmem = tmem + (uint32_t)(g * kACols);
+        const uint32_t xbase = smem_u32(smem + (size_t)s * p.stage_bytes + kUW);
 #pragma unroll
-        for (int kk = 0; kk < kKB / 16; ++kk) {
-          const uint64_t bdesc = sw128_desc(xbase + (kk >> 2) * npad * 128 + (kk & 3) * 32);
-          tc_mma_f16_ts(d_tmem, a_tmem + kk * 8, bdesc, idesc, kk == 0 ? 0u : 1u);
+        for (int h = 0; h < BPU; ++h) {            // each block into its own P: its scale comes later
+          const uint32_t d_tmem = tmem + pcol0 + (uint32_t)((b * BPU + h) * npad);
+          const uint32_t a_tmem = tmem + (uint32_t)(g * kUACols + h * kACols);
+#pragma unroll
+          for (int kk = 0; kk < kKB / 16; ++kk) {
+            const uint64_t bdesc = sw128_desc(xbase + (2 * h + (kk >> 2)) * npad * 128 + (kk & 3) * 32);
+            tc_mma_f16_ts(d_tmem, a_tmem + kk * 8, bdesc, idesc, kk == 0 ? 0u : 1u);
+          }
         }
         tc_commit(bar_empty(s));       // stage reusable once these MMAs retire
         tc_commit(bar_aempty(g));      // A buffer reusable
-        tc_commit(bar_pfull(b));       // the block's sums are ready for promotion
+        tc_commit(bar_pfull(b));       // the blocks' sums are ready for promotion
         if (++s == S) { s = 0; ph ^= 1u; }
       }
       tc_commit(bar_drain);            // completes when every MMA issued above has retired
@@ -336,35 +401,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(bar_aempty(g), ((uint32_t)(i >> 1) & 1u) ^ 1u, s_abort, p.err)) break;
       tc_fence_after();
       uint8_t* st = smem + (size_t)s * p.stage_bytes;
-      // X slice: bf16 -> f16 in place (rows < M; TMA zero-filled the rest)
+      // X slice: bf16 -> f16 in place, each row shifted by its power of two (rows < M; TMA
+      // zero-filled the rest)
       {
-        uint8_t* xs = st + kWBytes;
-        const int words = 2 * p.M * 8;               // 16-byte words: 2 atoms x M rows x 8
+        uint8_t* xs = st + kUW;
+        const int* xe = s_stage_xe[s];
+        const int words = 2 * BPU * p.M * 8;         // 16-byte words: 2*BPU atoms x M rows x 8
         for (int w = tg; w < words; w += 128) {
           const int a = w / (p.M * 8), rem = w - a * (p.M * 8);
           uint4* ptr = reinterpret_cast<uint4*>(xs + a * npad * 128 + (rem >> 3) * 128 + (rem & 7) * 16);
           uint4 v = *ptr;
-          v.x = bf16x2_to_f16x2_sat(v.x); v.y = bf16x2_to_f16x2_sat(v.y);
-          v.z = bf16x2_to_f16x2_sat(v.z); v.w = bf16x2_to_f16x2_sat(v.w);
+          const int e = __ldg(xe + (rem >> 3));
+          v.x = bf16x2_to_f16x2_shifted(v.x, e); v.y = bf16x2_to_f16x2_shifted(v.y, e);
+          v.z = bf16x2_to_f16x2_shifted(v.z, e); v.w = bf16x2_to_f16x2_shifted(v.w, e);
           *ptr = v;
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       }
-      // weight row r: 128 codes in eight swizzled 16-byte chunks -> 64 f16 pairs in TMEM
-      const uint8_t* row = st + r * 128;
-      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(g * kACols);
+      // weight row r of each block: 128 codes in eight swizzled 16-byte chunks -> 64 f16 pairs
+      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(g * kUACols);
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t out[32];
+      for (int h = 0; h < BPU; ++h) {
+        const uint8_t* row = st + h * kWBytes + r * 128;
 #pragma unroll
-        for (int j2 = 0; j2 < 4; ++j2) {
-          const int j = half * 4 + j2;                // logical chunk: elements 16j .. 16j+15
-          const uint4 w = *reinterpret_cast<const uint4*>(row + ((j ^ (r & 7)) << 4));
-          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+        for (int half = 0; half < 2; ++half) {
+          uint32_t out[32];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) out[j2 * 8 + e] = e4m3x2_to_f16x2(ww[e >> 1] >> ((e & 1) * 16));
+          for (int j2 = 0; j2 < 4; ++j2) {
+            const int j = half * 4 + j2;              // logical chunk: elements 16j .. 16j+15
+            const uint4 w = *reinterpret_cast<const uint4*>(row + ((j ^ (r & 7)) << 4));
+            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) out[j2 * 8 + e] = e4m3x2_to_f16x2(ww[e >> 1] >> ((e & 1) * 16));
+          }
+          tc_st_x32(taddr + (uint32_t)(h * kACols + half * 32), out);
         }
-        tc_st_x32(taddr + half * 32, out);
       }
       tc_wait_st();
       tc_fence_before();
@@ -376,45 +447,82 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int rowl = q * 32 + lane;
     const int et = threadIdx.x - 12 * 32;            // 0..127
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
-    long long tile_it = u_begin / kbs;
-    int kb_it = (int)(u_begin % kbs);
+    // Block scales, four units ahead: the L2 round trip would otherwise sit on every unit's
+    // path. Block h of unit (tile, ku) has scale [tile][ku * BPU + h].
+    Cursor ahead;
+    ahead.init(probs, p.nprob, u_begin);
+    int ia = 0;                                      // unit of this CTA's range that `ahead` is at
+    auto load_ahead = [&](float (&dst)[BPU]) {
+      if (ia < nunits) {
+        const Problem& pa = probs[ahead.pi];
+        const float* sp = pa.scales + (ahead.tile * pa.kus + ahead.ku) * BPU;
+#pragma unroll
+        for (int h = 0; h < BPU; ++h) dst[h] = __ldg(sp + h);
+        ahead.next(probs);
+      } else {
+#pragma unroll
+        for (int h = 0; h < BPU; ++h) dst[h] = 0.0f;
+      }
+      ++ia;
+    };
+    float scn[4][BPU];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) load_ahead(scn[a]);
+    Cursor cur;
+    cur.init(probs, p.nprob, u_begin);
     for (int i = 0; i < nunits; ++i) {
       const long long u = u_begin + i;
-      const long long tile = tile_it;
-      const int kb = kb_it;
-      const bool seg_first = (i == 0) || (kb == 0);
-      const bool seg_last = (i == nunits - 1) || (kb == kbs - 1);
-      if (++kb_it == kbs) { kb_it = 0; ++tile_it; }
+      const Problem& pr = probs[cur.pi];
+      const long long tile = cur.tile;
+      const int ku = cur.ku, kus = pr.kus;
+      cur.next(probs);
+      const bool seg_first = (i == 0) || (ku == 0);
+      const bool seg_last = (i == nunits - 1) || (ku == kus - 1);
       const int b = i % NP, k = i / NP;
-      const float sc = __ldg(p.scales + tile * kbs + kb);
+      float sc[BPU];
+#pragma unroll
+      for (int h = 0; h < BPU; ++h) {
+        sc[h] = scn[0][h];
+        scn[0][h] = scn[1][h];
+        scn[1][h] = scn[2][h];
+        scn[2][h] = scn[3][h];
+      }
+      load_ahead(scn[3]);
       // Every thread reaches the barrier, so a give-up seen by any of them ends the loop for all.
       mbar_wait(bar_pfull(b), (uint32_t)k & 1u, s_abort, p.err);
       named_bar(1, 128);
       if (ld_shared_volatile(s_abort)) break;
       tc_fence_after();
       const long long n = tile * kTileRows + rowl;
-      const long long tile_u0 = tile * kbs, tile_u1 = tile_u0 + kbs;
+      const long long tile_u0 = pr.unit0 + tile * kus, tile_u1 = tile_u0 + kus;
       const long long seg_u0 = u_begin > tile_u0 ? u_begin : tile_u0;
       const bool complete = (seg_u0 == tile_u0) && (u + 1 == tile_u1);
       const int slot = (seg_u0 == u_begin) ? 2 * c : 2 * c + 1;
-      const uint32_t pcol = pcol0 + (uint32_t)(b * npad);
+      const uint32_t pcol = pcol0 + (uint32_t)(b * BPU * npad);
       for (int m0 = 0; m0 < p.M; m0 += 16) {
-        uint32_t pv[16], rv[16];
-        tc_ld_x16(lane_base + pcol + m0, pv);
-        if (!seg_first) tc_ld_x16(lane_base + kRCol + m0, rv);
+        uint32_t pv[BPU][16], rv[16];
+#pragma unroll
+        for (int h = 0; h < BPU; ++h) tc_ld_x16(lane_base + pcol + (uint32_t)(h * npad + m0), pv[h]);
+        if (!seg_first) tc_ld_x16(lane_base + kR + m0, rv);
         tc_wait_ld();
         float y[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          y[j] = seg_first ? sc * __uint_as_float(pv[j]) : fmaf(sc, __uint_as_float(pv[j]), __uint_as_float(rv[j]));
+        for (int j = 0; j < 16; ++j) {
+          float acc = seg_first ? sc[0] * __uint_as_float(pv[0][j]) : fmaf(sc[0], __uint_as_float(pv[0][j]), __uint_as_float(rv[j]));
+#pragma unroll
+          for (int h = 1; h < BPU; ++h) acc = fmaf(sc[h], __uint_as_float(pv[h][j]), acc);
+          y[j] = acc;
+        }
         if (!seg_last) {
           uint32_t o[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(y[j]);
-          tc_st_x16(lane_base + kRCol + m0, o);
+          tc_st_x16(lane_base + kR + m0, o);
         } else if (complete) {
-          if (p.verify) warp_argmax(p, n, m0, y, s_val, s_idx, q, lane);
-          else write_y(p, n, m0, y);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) y[j] = mul_pow2(y[j], m0 + j < p.M ? __ldg(pr.xe + m0 + j) : 0);
+          if (pr.verify) warp_argmax(pr, n, m0, y, s_val, s_idx, q, lane);
+          else write_y(p, pr, n, m0, y);
         } else {
           float* dst = p.partials + ((long long)slot * p.M) * kTileRows;
 #pragma unroll
@@ -427,9 +535,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(bar_pempty(b));
       if (!seg_last) continue;
       if (complete) {
-        if (p.verify) {
+        if (pr.verify) {
           named_bar(1, 128);
-          tile_argmax_out(p, (int)tile, et, s_val, s_idx);
+          tile_argmax_out(p, pr, tile, et, s_val, s_idx);
           named_bar(1, 128);
         }
         continue;
@@ -442,7 +550,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int expected = 0;
         for (int cc = c0; cc <= c1; ++cc)
           if (unit_begin(cc + 1, U, p.grid) > unit_begin(cc, U, p.grid)) ++expected;
-        const unsigned int prev = atomicAdd(p.counters + tile, 1u);
+        const unsigned int prev = atomicAdd(p.counters + pr.tile0 + tile, 1u);
         *s_last = (prev + 1 == (unsigned int)expected) ? 1 : 0;
       }
       named_bar(1, 128);
@@ -465,14 +573,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 16; ++j) y[j] += v[j];
           }
-          if (p.verify) warp_argmax(p, n, m0, y, s_val, s_idx, q, lane);
-          else write_y(p, n, m0, y);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) y[j] = mul_pow2(y[j], m0 + j < p.M ? __ldg(pr.xe + m0 + j) : 0);
+          if (pr.verify) warp_argmax(pr, n, m0, y, s_val, s_idx, q, lane);
+          else write_y(p, pr, n, m0, y);
         }
-        if (p.verify) {
+        if (pr.verify) {
           named_bar(1, 128);
-          tile_argmax_out(p, (int)tile, et, s_val, s_idx);
+          tile_argmax_out(p, pr, tile, et, s_val, s_idx);
         }
-        if (et == 0) p.counters[tile] = 0u;          // ready for the next call
+        if (et == 0) p.counters[pr.tile0 + tile] = 0u;   // ready for the next call
       }
       named_bar(1, 128);
     }
@@ -483,6 +593,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+  }
+}
+
+
+// Row shifts of every problem's X (one CTA per (problem, row)): xe[m] from the row's amax,
+// as row_shift_of_amax defines it. The GEMM converts x * 2^-xe[m] to f16 and multiplies its
+// output by 2^xe[m].
+constexpr int kShiftThreads = 256;
+
+__global__ void __launch_bounds__(kShiftThreads)
+    fp8_x_shift_kernel(const __grid_constant__ Problem single, const Problem* probs, int M) {
+  const Problem& pr = probs ? probs[blockIdx.x / M] : single;
+  const int m = blockIdx.x % M, t = threadIdx.x;
+  const uint32_t* row = reinterpret_cast<const uint32_t*>(pr.X + (long long)m * pr.K);   // bf16 pairs
+  float v = 0.f;
+  for (long long i = t; i < pr.K / 2; i += kShiftThreads) v = fmaxf(v, bf16x2_absmax(__ldg(row + i)));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  __shared__ float s_red[kShiftThreads / 32];
+  if ((t & 31) == 0) s_red[t >> 5] = v;
+  __syncthreads();
+  if (t == 0) {
+    float a = 0.f;
+    for (int w = 0; w < kShiftThreads / 32; ++w) a = fmaxf(a, s_red[w]);
+    pr.xe[m] = row_shift_of_amax(a);
   }
 }
 
@@ -523,104 +658,208 @@ bool fp8_supported(long long M, long long K) {
   return M >= 1 && M <= kMaxNpad && K >= kKB && K % kKB == 0 && K / kKB <= (1ll << 24);
 }
 
+static size_t al256_fp8(size_t v) { return (v + 255) / 256 * 256; }
+
+// The launch shape and the workspace layout of a list of GEMMs sharing M.
 struct Fp8Plan {
-  int npad, np, tiles, kbs, grid, stages;
+  int npad, bpu, np, grid, stages;
+  int tiles, vtiles;       // tiles of all problems; of the verify problem (0 without one)
   long long units;
   uint32_t stage_bytes;
   size_t smem;
+  size_t off_partials, off_verify, off_xe, off_desc, bytes;
 };
 
-static Fp8Plan fp8_plan(long long M, long long N, long long K) {
+static Fp8Plan fp8_plan(long long M, const Fp8HostProblem* hp, int n, bool with_desc) {
   Fp8Plan pl{};
   pl.npad = (int)std::max<long long>(16, (M + 15) / 16 * 16);
-  pl.np = std::min(kMaxP, (int)((512 - kRCol - pl.npad) / pl.npad));
-  pl.tiles = (int)((N + kTileRows - 1) / kTileRows);
-  pl.kbs = (int)(K / kKB);
-  pl.units = (long long)pl.tiles * pl.kbs;
+  // TMEM: two A buffers (64 columns per block each), R (npad), np rotating P sets (bpu * npad
+  // each). Two blocks per unit while that leaves at least two P sets and every K allows it.
+  bool even = true;
+  for (int i = 0; i < n; ++i) even = even && ((hp[i].K / kKB) % 2 == 0);
+  pl.bpu = (even && (512 - 2 * 2 * kACols - pl.npad) / (2 * pl.npad) >= 2) ? 2 : 1;
+  pl.np = std::min(kMaxP, (512 - 2 * pl.bpu * kACols - pl.npad) / (pl.bpu * pl.npad));
+  for (int i = 0; i < n; ++i) {
+    const int tiles = (int)((hp[i].N + kTileRows - 1) / kTileRows);
+    pl.units += (long long)tiles * (hp[i].K / kKB / pl.bpu);
+    pl.tiles += tiles;
+    if (hp[i].verify) pl.vtiles = tiles;
+  }
   const int sms = std::max(1, device_sm_count());
   pl.grid = (int)std::min<long long>(sms, pl.units);
-  pl.stage_bytes = kWBytes + (uint32_t)pl.npad * 256u;
+  pl.stage_bytes = (uint32_t)pl.bpu * (kWBytes + (uint32_t)pl.npad * 256u);
   const size_t budget = 227 * 1024 - 1024 - kTailBytes;
   pl.stages = (int)std::min<size_t>(kMaxStages, budget / pl.stage_bytes);
   pl.smem = 1024 + (size_t)pl.stages * pl.stage_bytes + kTailBytes;
+  pl.off_partials = al256_fp8((size_t)pl.tiles * 4);
+  pl.off_verify = pl.off_partials + al256_fp8((size_t)2 * pl.grid * M * kTileRows * 4);
+  pl.off_xe = pl.off_verify + (pl.vtiles ? 2 * al256_fp8((size_t)pl.vtiles * M * 4) : 0);
+  pl.off_desc = pl.off_xe + al256_fp8((size_t)n * M * 4);                 // row shifts [n][M]
+  pl.bytes = pl.off_desc + (with_desc ? al256_fp8((size_t)n * sizeof(Problem)) : 0);
   return pl;
 }
 
-static size_t al256_fp8(size_t v) { return (v + 255) / 256 * 256; }
-
-size_t fp8_gemm_workspace_bytes_int(long long M, long long N, long long K) {
-  if (!fp8_supported(M, K) || N < 1) return 0;
-  const Fp8Plan pl = fp8_plan(M, N, K);
-  return al256_fp8((size_t)pl.tiles * 4) + al256_fp8((size_t)2 * pl.grid * M * kTileRows * 4);
-}
-
-size_t fp8_verify_workspace_bytes_int(long long M, long long N, long long K) {
-  if (!fp8_supported(M, K) || N < 1) return 0;
-  const Fp8Plan pl = fp8_plan(M, N, K);
-  return fp8_gemm_workspace_bytes_int(M, N, K) + 2 * al256_fp8((size_t)pl.tiles * M * 4);
-}
-
-static int launch_fp8(const uint16_t* X, const uint8_t* q, const float* scales, long long M, long long N,
-                      long long K, void* Y, int y_dtype, void* workspace, bool verify, float** pv_out, int** pi_out,
-                      int* nparts_out, cudaStream_t s) {
-  const Fp8Plan pl = fp8_plan(M, N, K);
-  alignas(64) CUtensorMap tw, tx;
-  if (!make_map_fp8(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, K, N, K, kKB, kTileRows) ||
-      !make_map_fp8(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, pl.npad))
+static int fill_problem(Problem* P, const Fp8HostProblem& h, long long M, const Fp8Plan& pl, long long unit0,
+                        int tile0, char* ws, int index) {
+  memset(P, 0, sizeof(*P));
+  if (!make_map_fp8(&P->tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, h.q, h.K, h.N, h.K, kKB, kTileRows) ||
+      !make_map_fp8(&P->tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h.X, h.K, M, h.K * 2, 64, pl.npad))
     return set_error(NVFP4WS_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  P->scales = h.scales;
+  P->Y = h.Y;
+  P->N = h.N;
+  P->unit0 = unit0;
+  P->tile0 = tile0;
+  P->kus = (int)(h.K / kKB / pl.bpu);
+  P->tiles = (int)((h.N + kTileRows - 1) / kTileRows);
+  P->y_bf16 = h.y_bf16;
+  P->verify = h.verify;
+  P->X = h.X;
+  P->K = h.K;
+  P->xe = reinterpret_cast<int*>(ws + pl.off_xe) + (size_t)index * M;
+  if (h.verify) {
+    P->part_val = reinterpret_cast<float*>(ws + pl.off_verify);
+    P->part_idx = reinterpret_cast<int*>(ws + pl.off_verify + al256_fp8((size_t)pl.vtiles * M * 4));
+  }
+  return NVFP4WS_OK;
+}
+
+static int launch_kernel(const Problem& single, const Problem* probs_dev, int nprob, long long M, const Fp8Plan& pl,
+                         char* ws, cudaStream_t s) {
   Params p{};
-  p.Y = static_cast<float*>(Y);
-  p.y_bf16 = (y_dtype == NVFP4WS_Y_BF16);
-  p.scales = scales;
+  p.probs = probs_dev;
+  p.nprob = nprob;
   p.M = (int)M;
   p.npad = pl.npad;
   p.np = pl.np;
-  p.N = N;
-  p.K = K;
-  p.tiles = pl.tiles;
-  p.kbs = pl.kbs;
   p.units = pl.units;
   p.grid = pl.grid;
   p.stages = pl.stages;
   p.stage_bytes = pl.stage_bytes;
-  char* ws = static_cast<char*>(workspace);
   p.counters = reinterpret_cast<unsigned int*>(ws);
-  p.partials = reinterpret_cast<float*>(ws + al256_fp8((size_t)pl.tiles * 4));
-  p.verify = verify ? 1 : 0;
-  if (verify) {
-    char* v = ws + fp8_gemm_workspace_bytes_int(M, N, K);
-    p.part_val = reinterpret_cast<float*>(v);
-    p.part_idx = reinterpret_cast<int*>(v + al256_fp8((size_t)pl.tiles * M * 4));
-    *pv_out = p.part_val;
-    *pi_out = p.part_idx;
-    *nparts_out = pl.tiles;
-  }
+  p.partials = reinterpret_cast<float*>(ws + pl.off_partials);
   p.err = device_error_word();
   if (!p.err) return set_error(NVFP4WS_ERR_CUDA, "cannot resolve the device error word");
   static std::atomic<bool> attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev].load(std::memory_order_acquire)) {
-    if (cudaFuncSetAttribute(fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
+    if (cudaFuncSetAttribute(fp8_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess ||
+        cudaFuncSetAttribute(fp8_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
       return check_launch("cudaFuncSetAttribute(fp8_kernel)");
     attr_set[dev].store(true, std::memory_order_release);
   }
-  fp8_kernel<<<pl.grid, kThreads, pl.smem, s>>>(tw, tx, p);
+  fp8_x_shift_kernel<<<(unsigned)(M * nprob), kShiftThreads, 0, s>>>(single, probs_dev, (int)M);
+  if (int e = check_launch("fp8_x_shift_kernel")) return e;
+  if (pl.bpu == 2) fp8_kernel<2><<<pl.grid, kThreads, pl.smem, s>>>(single, p);
+  else fp8_kernel<1><<<pl.grid, kThreads, pl.smem, s>>>(single, p);
   return check_launch("fp8_kernel");
+}
+
+// ---------------------------------------------------------------------------- one GEMM
+
+static Fp8HostProblem one(const uint16_t* X, const uint8_t* q, const float* scales, long long N, long long K, void* Y,
+                          int y_dtype, bool verify) {
+  return Fp8HostProblem{X, q, scales, N, K, Y, y_dtype == NVFP4WS_Y_BF16 ? 1 : 0, verify ? 1 : 0};
+}
+
+size_t fp8_gemm_workspace_bytes_int(long long M, long long N, long long K) {
+  if (!fp8_supported(M, K) || N < 1) return 0;
+  const Fp8HostProblem h = one(nullptr, nullptr, nullptr, N, K, nullptr, 0, false);
+  return fp8_plan(M, &h, 1, false).bytes;
+}
+
+size_t fp8_verify_workspace_bytes_int(long long M, long long N, long long K) {
+  if (!fp8_supported(M, K) || N < 1) return 0;
+  const Fp8HostProblem h = one(nullptr, nullptr, nullptr, N, K, nullptr, 0, true);
+  return fp8_plan(M, &h, 1, false).bytes;
+}
+
+static int launch_one(const Fp8HostProblem& h, long long M, void* workspace, cudaStream_t s, Fp8Plan* out) {
+  const Fp8Plan pl = fp8_plan(M, &h, 1, false);
+  char* ws = static_cast<char*>(workspace);
+  alignas(64) Problem P;
+  if (int e = fill_problem(&P, h, M, pl, 0, 0, ws, 0)) return e;
+  *out = pl;
+  return launch_kernel(P, nullptr, 1, M, pl, ws, s);
 }
 
 int launch_fp8_gemm(const uint16_t* X, const uint8_t* q, const float* scales, long long M, long long N, long long K,
                     void* Y, int y_dtype, void* workspace, cudaStream_t s) {
-  return launch_fp8(X, q, scales, M, N, K, Y, y_dtype, workspace, false, nullptr, nullptr, nullptr, s);
+  Fp8Plan pl;
+  return launch_one(one(X, q, scales, N, K, Y, y_dtype, false), M, workspace, s, &pl);
 }
 
 int launch_fp8_verify(const uint16_t* X, const uint8_t* q, const float* scales, long long M, long long N,
                       long long K, const VerifyRule& v, void* workspace, cudaStream_t s) {
-  float* pv = nullptr;
-  int* pi = nullptr;
-  int nparts = 0;
-  if (int e = launch_fp8(X, q, scales, M, N, K, nullptr, 0, workspace, true, &pv, &pi, &nparts, s)) return e;
-  return launch_verify_stage2(pv, pi, nparts, (int)M, v, s);
+  Fp8Plan pl;
+  if (int e = launch_one(one(X, q, scales, N, K, nullptr, 0, true), M, workspace, s, &pl)) return e;
+  char* ws = static_cast<char*>(workspace);
+  return launch_verify_stage2(reinterpret_cast<const float*>(ws + pl.off_verify),
+                              reinterpret_cast<const int*>(ws + pl.off_verify + al256_fp8((size_t)pl.vtiles * M * 4)),
+                              pl.vtiles, (int)M, v, s);
+}
+
+// ---------------------------------------------------------------------------- FP8 weight passes
+
+struct Fp8PassState {
+  uint32_t magic;
+  int nprob, has_verify;
+  long long M;
+  const Problem* probs;    // device copy, in the workspace
+  char* ws;
+  Fp8Plan pl;
+  VerifyRule vr;
+};
+static_assert(sizeof(Fp8PassState) <= kFp8PassStateBytes, "pass state does not fit the caller's handle");
+constexpr uint32_t kFp8PassMagic = 0x46503850u;
+
+size_t fp8_pass_workspace_bytes_int(const Fp8HostProblem* hp, int n, long long M) {
+  return fp8_plan(M, hp, n, true).bytes;
+}
+
+int fp8_pass_init_int(void* state, const Fp8HostProblem* hp, int n, long long M, const VerifyRule* vr,
+                      void* workspace, size_t workspace_bytes) {
+  const Fp8Plan pl = fp8_plan(M, hp, n, true);
+  if (workspace_bytes < pl.bytes)
+    return set_error(NVFP4WS_ERR_WORKSPACE, "fp8_pass_init: workspace needs %zu bytes", pl.bytes);
+  char* ws = static_cast<char*>(workspace);
+  std::vector<Problem> P(n);
+  long long unit0 = 0;
+  int tile0 = 0;
+  for (int i = 0; i < n; ++i) {
+    if (int e = fill_problem(&P[i], hp[i], M, pl, unit0, tile0, ws, i)) return e;
+    unit0 += (long long)P[i].tiles * P[i].kus;
+    tile0 += P[i].tiles;
+  }
+  Problem* dev = reinterpret_cast<Problem*>(ws + pl.off_desc);
+  if (cudaMemcpy(dev, P.data(), (size_t)n * sizeof(Problem), cudaMemcpyHostToDevice) != cudaSuccess)
+    return check_launch("fp8_pass_init: descriptor copy");
+  Fp8PassState st{};
+  st.magic = kFp8PassMagic;
+  st.nprob = n;
+  st.has_verify = vr != nullptr;
+  st.M = M;
+  st.probs = dev;
+  st.ws = ws;
+  st.pl = pl;
+  if (vr) st.vr = *vr;
+  memcpy(state, &st, sizeof(st));
+  return NVFP4WS_OK;
+}
+
+int fp8_pass_run_int(const void* state, cudaStream_t s) {
+  Fp8PassState st;
+  memcpy(&st, state, sizeof(st));
+  if (st.magic != kFp8PassMagic) return set_error(NVFP4WS_ERR_INVALID_ARG, "fp8_pass_run: pass is not initialised");
+  alignas(64) Problem unused;
+  memset(&unused, 0, sizeof(unused));
+  if (int e = launch_kernel(unused, st.probs, st.nprob, st.M, st.pl, st.ws, s)) return e;
+  if (!st.has_verify) return NVFP4WS_OK;
+  return launch_verify_stage2(reinterpret_cast<const float*>(st.ws + st.pl.off_verify),
+                              reinterpret_cast<const int*>(st.ws + st.pl.off_verify +
+                                                           al256_fp8((size_t)st.pl.vtiles * st.M * 4)),
+                              st.pl.vtiles, (int)st.M, st.vr, s);
 }
 
 }  // namespace nvfp4ws

@@ -21,6 +21,22 @@ int launch_fp8_gemm(const uint16_t* X, const uint8_t* q, const float* scales, lo
 int launch_fp8_verify(const uint16_t* X, const uint8_t* q, const float* scales, long long M, long long N,
                       long long K, const VerifyRule& v, void* workspace, cudaStream_t s);
 
+// One GEMM of an FP8 weight pass, as the host sees it. verify: the pass's lm_head (last).
+struct Fp8HostProblem {
+  const uint16_t* X;
+  const uint8_t* q;
+  const float* scales;
+  long long N, K;
+  void* Y;
+  int y_bf16, verify;
+};
+// Host state of an initialised FP8 pass lives in a caller-owned buffer of this many bytes.
+constexpr size_t kFp8PassStateBytes = 256;
+size_t fp8_pass_workspace_bytes_int(const Fp8HostProblem* hp, int n, long long M);
+int fp8_pass_init_int(void* state, const Fp8HostProblem* hp, int n, long long M, const VerifyRule* vr,
+                      void* workspace, size_t workspace_bytes);
+int fp8_pass_run_int(const void* state, cudaStream_t s);
+
 // fp32 W [N, K] -> E4M3 codes [N, K] and fp32 scales [ceil(N/128), ceil(K/128)].
 int launch_fp8_pack(const float* W, long long N, long long K, uint8_t* q, float* scales, cudaStream_t s);
 

@@ -195,3 +195,25 @@ def test_pass_refuses_a_struct_of_another_size(lib):
     assert b"verify struct_size" in lib.nvfp4ws_last_error()
     assert lib.fp8_lmhead_verify(FAKE, FAKE, FAKE, 17, 100, 128, vs_ptr, FAKE, 1 << 30, None) == 1
     assert b"struct_size" in lib.nvfp4ws_last_error()
+
+
+def test_fp8_pass_rejects_on_the_host(lib):
+    from nvfp4_weight_streaming_gemm_b200 import _lib as L
+    arr = (L.Fp8Problem * 2)()
+    arr[0] = L.Fp8Problem(FAKE, FAKE, FAKE, 128, 256, FAKE, 0)
+    arr[1] = L.Fp8Problem(FAKE, FAKE, FAKE, 128, 192, FAKE, 0)              # K % 128
+    assert lib.fp8_pass_workspace_bytes(arr, 2, 17, 0) == 0
+    assert lib.fp8_pass_workspace_bytes(arr, 1, 17, 0) > 0
+    assert lib.fp8_pass_workspace_bytes(arr, 1, 129, 0) == 0                  # M > 128
+    st = L.PassState()
+    assert lib.fp8_pass_init(ctypes.byref(st), arr, 2, 17, None, FAKE, 1 << 30) == 2
+    arr[1] = L.Fp8Problem(FAKE, FAKE, FAKE, 128, 256, None, 0)              # Y missing, not a verify problem
+    assert lib.fp8_pass_init(ctypes.byref(st), arr, 2, 17, None, FAKE, 1 << 30) == 1
+    spec = L.VerifySpec(FAKE, 2, 16, FAKE, FAKE, None, None, None)          # M != B*(D+1)
+    assert lib.fp8_pass_init(ctypes.byref(st), arr, 2, 17, ctypes.byref(spec), FAKE, 1 << 30) == 1
+    arr[0].struct_size = 8                                                   # another header's struct
+    assert lib.fp8_pass_workspace_bytes(arr, 1, 17, 0) == 0
+    assert lib.fp8_pass_init(ctypes.byref(st), arr, 1, 17, None, FAKE, 1 << 30) == 1
+    assert b"struct_size" in lib.nvfp4ws_last_error()
+    assert lib.fp8_pass_run(None, None) == 1
+    assert lib.fp8_pass_run(ctypes.byref(L.PassState()), None) == 1       # never initialised

@@ -62,7 +62,8 @@ def test_fp8_pack_bit_exact(nv, N, K):
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 1000, 256), (17, 3000, 1024), (68, 777, 768), (128, 4096, 5120),
-                                   (5, 130, 128), (17, 640, 5120), (17, 128, 16384)])
+                                   (5, 130, 128), (17, 640, 5120), (17, 128, 16384), (40, 1000, 1024),
+                                   (49, 333, 512)])
 def test_fp8_gemm(nv, M, N, K):
     W, x = S.block_varied_case(1000 + M + N, M, N, K)
     q, s, codes_ref, scales_ref = packed(nv, W)
@@ -120,3 +121,55 @@ def test_fp8_verify_tree(nv):
     assert V.comparable_tree_sequences(gap, parents, D).all()  # no near tie for this seed (oracle-checked)
     assert np.array_equal(t.cpu().numpy(), t_ref)
     assert np.array_equal(L.cpu().numpy(), L_ref) and np.array_equal(node.cpu().numpy(), node_ref)
+
+
+@pytest.mark.parametrize("M,shapes", [
+    (17, [(3000, 1024), (640, 5120), (1500, 2560), (77, 512)]),    # every K a multiple of 256: two blocks per unit
+    (17, [(700, 384), (300, 1280), (129, 128)]),                   # odd block counts: one block per unit
+    (68, [(1000, 1024), (200, 2048), (64, 256)]),                  # npad 80: one block per unit
+])
+def test_fp8_pass(nv, M, shapes):
+    probs, refs = [], []
+    for i, (N, K) in enumerate(shapes):
+        W, x = S.block_varied_case(1400 + 10 * M + i, M, N, K)
+        q, s, codes_ref, scales_ref = packed(nv, W)
+        Y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+        probs.append((to_dev_bf16(x), q, s, Y))
+        refs.append(P.gemm_fp8_ref(x, codes_ref, scales_ref))
+    p = nv.Fp8Pass(probs, M)
+    p.run()
+    nv.check()
+    first = [Y.clone() for (_, _, _, Y) in probs]
+    for (_, _, _, Y), y_ref in zip(probs, refs):
+        assert rowwise_err(Y.cpu().numpy(), y_ref) <= TOL
+    p.run()                                                     # tickets were reset: the same bits again
+    nv.check()
+    for (_, _, _, Y), Y1 in zip(probs, first):
+        assert torch.equal(Y, Y1)
+
+
+def test_fp8_pass_with_verify_tail(nv):
+    """Two FP8 GEMMs and the FP8 head of the chain-verify test in one launch, ending in the verify."""
+    B, D, N, K = 1, 16, 20077, 2048
+    M = B * (D + 1)
+    Wh, xh = S.random_case(1200, M, N, K, w_std=0.2)
+    qh, sh, ch_ref, sch_ref = packed(nv, Wh)
+    t_ref = V.argmax_fast(P.gemm_fp8_ref(xh, ch_ref, sch_ref))
+    drafts = S.drafts_with_prefix(t_ref, np.array([9]), D, N)
+    probs, refs = [], []
+    for i, (Ng, Kg) in enumerate([(900, 1024), (333, 2048)]):
+        W, x = S.block_varied_case(1500 + i, M, Ng, Kg)
+        q, s, codes_ref, scales_ref = packed(nv, W)
+        Y = torch.empty((M, Ng), dtype=torch.float32, device="cuda")
+        probs.append((to_dev_bf16(x), q, s, Y))
+        refs.append(P.gemm_fp8_ref(x, codes_ref, scales_ref))
+    probs.append((to_dev_bf16(xh), qh, sh, None))
+    t = torch.empty(M, dtype=torch.int32, device="cuda")
+    L = torch.empty(B, dtype=torch.int32, device="cuda")
+    p = nv.Fp8Pass(probs, M, verify=(torch.from_numpy(drafts).cuda(), t, L, None))
+    p.run()
+    nv.check()
+    for (_, _, _, Y), y_ref in zip(probs[:2], refs):
+        assert rowwise_err(Y.cpu().numpy(), y_ref) <= TOL
+    assert np.array_equal(t.cpu().numpy(), t_ref)              # no near tie for this seed (the chain test checks it)
+    assert L.cpu().numpy().tolist() == [9]
