@@ -163,12 +163,13 @@ int nvfp4_gemm_skinny_path(const void* X, const uint8_t* q, const uint8_t* sf, c
  *
  * Passages: "Qwen3.8 on DGX Spark (GB10)", introduction (NVFP4 on the block-scaled
  * tensor cores) and "TandemLLM", "The parts" (4-bit projections). The pages give no
- * activation recipe; this library applies the weights' two-level NVFP4 scheme to each
- * row of X, with the row's amax in place of the tensor's, every decision in fp32:
+ * activation recipe; this library applies the weights' two-level NVFP4 scheme (the rule of
+ * nvfp4_pack) to each row of X, with the row's amax in place of the tensor's:
  *   g[m]   = fp32(amax_k |x[m,k]| / 2688)
- *   S      = E4M3_rne_satfinite(fp32(amax_block * fp32(1 / fp32(6 g[m]))))   per 16 elements
- *   c      = E2M1_rne_satfinite(fp32(x / fp32(S g[m])))                     (0 where S g = 0)
- *   Y[m,n] = sum_k (e2m1(c)·S·g[m])[m,k] · dequant(W)[n,k], accumulated in fp32.
+ *   S      = E4M3_rne_satfinite(amax_block / (6 g[m]))        per 16 elements
+ *   c      = E2M1_rne_satfinite(x / (S g[m]))                 (+0 where S g = 0; sign kept)
+ *   Y[m,n] = sum_k (e2m1(c)·S·g[m])[m,k] · dequant(W)[n,k], accumulated in fp32,
+ * with both quotients exact and rounded once.
  * This is not the exact bf16 product nvfp4_gemm_skinny computes: each activation
  * carries up to half an E2M1 step of quantisation error.
  *

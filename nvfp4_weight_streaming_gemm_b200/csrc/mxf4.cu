@@ -19,7 +19,7 @@
 // absolute. The terms are extra B rows (token m, term t -> row m*T + t). The
 // epilogue folds them: y[m] = ts * sum_t g_t acc[m*T+t]. With T = 1 (the W4A4
 // product) the single term is the NVFP4 quantisation of the row, its code taken
-// from a correctly rounded fp32 quotient.
+// and scale taken from the exact quotients, rounded once (the weights' rule).
 //
 // Kernels.
 //   x_prep_kernel   one CTA per (activation row, problem): the T-term decomposition,
@@ -178,10 +178,74 @@ __device__ __forceinline__ float rcp_approx(float x) {
   return y;
 }
 
+// v narrowed to fp32 by rounding to odd: the result rounded to nearest (ties to even) in any
+// format with at most 22 significant bits equals the single rounding of v itself, when v is
+// the correctly rounded double of a quotient of an 8-bit by a <= 28-bit number (such a
+// quotient is either exact in fp32 or at least 2^-52 away from every fp32 value, so the
+// double rounding loses no sticky bit).
+__device__ __forceinline__ float to_f32_odd(double v) {
+  float r = __double2float_rz(v);
+  if ((double)r != v) r = __uint_as_float(__float_as_uint(r) | 1u);
+  return r;
+}
+
+// |q| within a relative 2^-20 of a point where E2M1 rounding changes (0.25, 0.75, 1.25,
+// 1.75, 2.5, 3.5, 5): an fp32 quotient with a few ulps of error may decide such a q wrongly.
+__device__ __forceinline__ bool near_e2m1_midpoint(float q) {
+  const float a = fabsf(q), t = a * 0x1p-20f;
+  return (fabsf(a - 0.25f) <= t) | (fabsf(a - 0.75f) <= t) | (fabsf(a - 1.25f) <= t) | (fabsf(a - 1.75f) <= t) |
+         (fabsf(a - 2.5f) <= t) | (fabsf(a - 3.5f) <= t) | (fabsf(a - 5.0f) <= t);
+}
+
+// One NVFP4 term of block b (the W4A4 activations): the weights' two-level rule with the
+// row scale g in place of the tensor scale, both quotients exact and rounded once:
+//   S = E4M3_rne_satfinite(amax_block / (6 g)),  c = E2M1_rne_satfinite(x / (S g)).
+// 6 g and S g are exact in double. The scale takes a correctly rounded double quotient; the
+// codes take an fp32 quotient and, within 2^-20 of a rounding point, the exact one.
+__device__ __forceinline__ void quantise_block_single(const float (&r)[16], int b, int m, float g0, const Geom& g,
+                                                      uint8_t* img) {
+  const int kc = b >> 4, bi = b & 15;
+  uint8_t* base = img + (size_t)kc * g.img_stride;
+  uint32_t sbits = 0, lo = 0, hi = 0;
+  if (g0 > 0.f) {
+    const double g64 = (double)g0;
+    uint16_t s2;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
+        : "=h"(s2) : "f"(0.0f), "f"(to_f32_odd(__ddiv_rn((double)block_amax16(r), 6.0 * g64))));
+    sbits = s2 & 0xFFu;
+    const double den = (double)f16lo_to_f32(e4m3x2_to_f16x2(sbits)) * g64;
+    if (den > 0.0) {
+      const bool fast = den >= 0x1p-100;
+      const float inv = fast ? __frcp_rn((float)den) : 0.f;
+      float q[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        q[i] = r[i] * inv;
+        if (!fast || near_e2m1_midpoint(q[i])) q[i] = to_f32_odd(__ddiv_rn((double)r[i], den));
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        uint16_t c2;
+        asm("{ .reg .b8 b; cvt.rn.satfinite.e2m1x2.f32 b, %1, %2; cvt.u16.u8 %0, b; }"
+            : "=h"(c2) : "f"(q[2 * i + 1]), "f"(q[2 * i]));
+        if (i < 4) lo |= (uint32_t)(c2 & 0xFF) << (8 * i);
+        else hi |= (uint32_t)(c2 & 0xFF) << (8 * (i - 4));
+      }
+    }
+  }
+  const uint32_t off = (uint32_t)m * 128u + ((uint32_t)((bi >> 1) ^ (m & 7)) << 4) + ((uint32_t)(bi & 1) << 3);
+  *reinterpret_cast<uint2*>(base + off) = make_uint2(lo, hi);
+  base[g.img_xs_off + (uint32_t)m * 16u + (uint32_t)bi] = (uint8_t)sbits;
+}
+
 // The T terms of block b (16 values in r) into the chunk images; gt0 = g_0, inv6 = 1/(6 g_t).
 template <int T>
 __device__ __forceinline__ void quantise_block(float (&r)[16], int b, int m, float gt0, const float (&inv6)[T],
                                                const Geom& g, uint8_t* img) {
+  if constexpr (T == 1) {
+    quantise_block_single(r, b, m, gt0, g, img);
+    return;
+  }
   const int kc = b >> 4, bi = b & 15;           // K-chunk and block within it
   uint8_t* base = img + (size_t)kc * g.img_stride;
   float gt = gt0;
@@ -198,10 +262,9 @@ __device__ __forceinline__ void quantise_block(float (&r)[16], int b, int m, flo
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           uint16_t c2;
-          // One term (W4A4): the code is the rounding of the correctly rounded fp32 quotient,
-          // a decision a reader can redo exactly. Several terms: the residual corrects it.
-          const float q1 = T == 1 ? __fdiv_rn(r[2 * i + 1], den) : r[2 * i + 1] * inv;
-          const float q0 = T == 1 ? __fdiv_rn(r[2 * i], den) : r[2 * i] * inv;
+          // Approximate codes are fine here: each residual is exact and the next term corrects it.
+          const float q1 = r[2 * i + 1] * inv;
+          const float q0 = r[2 * i] * inv;
           asm("{ .reg .b8 b; cvt.rn.satfinite.e2m1x2.f32 b, %1, %2; cvt.u16.u8 %0, b; }"
               : "=h"(c2) : "f"(q1), "f"(q0));
           const uint32_t h = e2m1x2_to_f16x2(c2);

@@ -15,8 +15,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from .nvfp4 import (E2M1_VALUES, E4M3_VALUES, GROUP, TENSOR_SCALE_DIVISOR, dequantize_nvfp4, e2m1_encode,
-                    e4m3_encode)
+from .nvfp4 import E2M1_VALUES, E4M3_VALUES, GROUP, dequantize_nvfp4, quantize_codes
 
 
 def bf16_bits_to_float64(bits: np.ndarray) -> np.ndarray:
@@ -55,15 +54,15 @@ def quantize_x_rows(x_bits: np.ndarray):
     The pages run prefill on the block-scaled tensor cores with both operands in
     4 bits ("Qwen3.8 on DGX Spark (GB10)", introduction: NVFP4 on block-scaled tensor
     cores; "TandemLLM", "The parts"). They give no activation recipe. Reading: the
-    weights' two-level NVFP4 scheme applied to each row, with the row's amax in place
-    of the tensor's. Every decision is taken in fp32, as the kernel takes it (IEEE
-    round-to-nearest; numpy float32 arithmetic is the same):
+    weights' two-level NVFP4 scheme (``oracle.nvfp4.quantize_codes``) applied to each
+    row on its own, the row's amax taking the place of the tensor's:
 
         g   = fp32(amax|x_row| / 2688)
-        inv = fp32(1 / fp32(6 * g))
-        S   = E4M3_rne_satfinite(fp32(amax_block * inv))
-        den = fp32(S * g)
-        c   = E2M1_rne_satfinite(fp32(x / den))     (0 where den = 0)
+        S   = E4M3_rne_satfinite(amax_block / (6 g))
+        c   = E2M1_rne_satfinite(x / (S g))            (+0 where S g = 0)
+
+    with both quotients formed exactly (float64, in which 6 g and S g are exact) and
+    rounded once, as for the weights.
 
     Returns ``(codes uint8 [M, K], sf uint8 [M, K/16], g float32 [M])``.
     """
@@ -71,21 +70,12 @@ def quantize_x_rows(x_bits: np.ndarray):
     if x.ndim != 2 or x.shape[1] % GROUP:
         raise ValueError("X must be [M, K] with K a multiple of 16")
     M, K = x.shape
-    amax = np.max(np.abs(x), axis=1)
-    g = (amax / np.float32(TENSOR_SCALE_DIVISOR)).astype(np.float32)
-    with np.errstate(divide="ignore"):
-        inv = np.where(g > 0, np.float32(1.0) / (np.float32(6.0) * g), np.float32(0.0)).astype(np.float32)
-    blocks = x.reshape(M, K // GROUP, GROUP)
-    a = (np.max(np.abs(blocks), axis=2) * inv[:, None]).astype(np.float32)
-    sf = e4m3_encode(a.astype(np.float64))
-    S = E4M3_VALUES[sf].astype(np.float32)
-    den = (S * g[:, None]).astype(np.float32)
-    with np.errstate(divide="ignore", invalid="ignore"):
-        r = np.where(den[:, :, None] > 0, blocks / np.where(den > 0, den, np.float32(1.0))[:, :, None],
-                     np.float32(0.0)).astype(np.float32)
-    codes = e2m1_encode(r.astype(np.float64))
-    codes = np.where(den[:, :, None] > 0, codes, np.uint8(0)).astype(np.uint8)
-    return codes.reshape(M, K), sf.astype(np.uint8), g
+    codes = np.zeros((M, K), dtype=np.uint8)
+    sf = np.zeros((M, K // GROUP), dtype=np.uint8)
+    g = np.zeros(M, dtype=np.float32)
+    for m in range(M):                                       # each row is its own "tensor"
+        codes[m:m + 1], sf[m:m + 1], g[m] = quantize_codes(x[m:m + 1])
+    return codes, sf, g
 
 
 def dequantize_x_rows(codes: np.ndarray, sf: np.ndarray, g: np.ndarray) -> np.ndarray:

@@ -15,8 +15,10 @@ the same shapes stand in for them:
 * stack       64 layers of the three layer shapes (192 matrices, 11.51 GB
               NVFP4), with M=17 (verify) or M=68 (4 sequences x 17).
 * lm_head     K=5120, N=248320, or the first 65,536 rows as the sliced draft
-              vocabulary. W seed 7, X seed 107, prefix lengths L* ~ U{0..16}
-              from seed 207.
+              vocabulary. W is drawn in chunks of 4,096 rows, chunk c from its own
+              generator default_rng([7, c]), so any chunk can be drawn alone (the
+              full-vocabulary oracle draws them in parallel). X seed 107, prefix
+              lengths L* ~ U{0..16} from seed 207.
 * sweep       M in {1, 2, 4, 8, 17, 34, 68, 128} on the gate+up shape.
 """
 
@@ -100,16 +102,43 @@ def block_varied_case(seed: int, M: int, N: int, K: int, block: int = 128, sprea
     return W, normal_x_bits(rng, M, K)
 
 
+LMHEAD_CHUNK = 4096
+
+
+def lmhead_weight_chunk(c: int, N: int = VOCAB, K: int = LMHEAD_K) -> np.ndarray:
+    """Rows [4096 c, min(N, 4096 (c + 1))) of the lm_head weight: fp32 ~ N(0, 0.02^2) from
+    ``default_rng([7, c])``."""
+    n0 = c * LMHEAD_CHUNK
+    rows = min(N, n0 + LMHEAD_CHUNK) - n0
+    return (np.random.default_rng([LMHEAD_W_SEED, c]).standard_normal((rows, K)) * W_STD).astype(np.float32)
+
+
+def lmhead_weight(N: int = VOCAB, K: int = LMHEAD_K) -> np.ndarray:
+    """The lm_head weight fp32 [N, K], chunk by chunk (see lmhead_weight_chunk)."""
+    W = np.empty((N, K), dtype=np.float32)
+    for c in range(-(-N // LMHEAD_CHUNK)):
+        n0 = c * LMHEAD_CHUNK
+        W[n0: n0 + LMHEAD_CHUNK] = lmhead_weight_chunk(c, N, K)
+    return W
+
+
+def lmhead_x(B: int = 1, D: int = DRAFT_LEN, K: int = LMHEAD_K) -> np.ndarray:
+    """lm_head hidden states bf16 [B*(D+1), K]; the rows of B sequences start with those of B' < B."""
+    return normal_x_bits(np.random.default_rng(LMHEAD_X_SEED), B * (D + 1), K)
+
+
+def lmhead_lstar(B: int = 1, D: int = DRAFT_LEN) -> np.ndarray:
+    """Prefix lengths L* ~ U{0..D}, int64 [B]."""
+    return np.random.default_rng(LMHEAD_L_SEED).integers(0, D + 1, size=B)
+
+
 def lmhead_inputs(N: int = VOCAB, B: int = 1, D: int = DRAFT_LEN, K: int = LMHEAD_K):
     """lm_head weight, hidden states and prefix lengths.
 
     Returns ``(W fp32 [N, K], x_bits [B*(D+1), K], Lstar int64 [B])``. With N=65536
-    this is the sliced draft vocabulary: the first 65,536 rows of the full draw.
+    this is the sliced draft vocabulary: the first 65,536 rows of the full weight.
     """
-    W = normal_weight(np.random.default_rng(LMHEAD_W_SEED), N, K)
-    x = normal_x_bits(np.random.default_rng(LMHEAD_X_SEED), B * (D + 1), K)
-    Lstar = np.random.default_rng(LMHEAD_L_SEED).integers(0, D + 1, size=B)
-    return W, x, Lstar
+    return lmhead_weight(N, K), lmhead_x(B, D, K), lmhead_lstar(B, D)
 
 
 def drafts_with_prefix(t: np.ndarray, Lstar: np.ndarray, D: int, vocab: int, seed: int = 208) -> np.ndarray:

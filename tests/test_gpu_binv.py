@@ -70,4 +70,6 @@ def test_pass_rows_identical_for_every_m(nv):
         W, x = weights[i][0], xs[i][:17]
         q, sf, ts = F.quantize_nvfp4(W)
         y_ref = G.gemm_ref(x, q, sf, ts)
-        assert (np.abs(ys[i] - y_ref).max(axis=1) <= 2e-3 * np.abs(y_ref).max(axis=1)).all()
+        err, scale = np.abs(ys[i] - y_ref).max(axis=1), np.abs(y_ref).max(axis=1)
+        assert (err <= 2e-3 * scale).all()
+        assert (err <= 1e-4 * scale).all()              # the five residual activation terms

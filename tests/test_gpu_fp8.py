@@ -73,6 +73,26 @@ def test_fp8_gemm(nv, M, N, K):
     assert rowwise_err(Y.cpu().numpy(), y_ref) <= TOL
 
 
+@pytest.mark.parametrize("M,N,K", [(5, 700, 1024), (68, 300, 512)])
+def test_fp8_gemm_activation_range(nv, M, N, K):
+    """Activation rows far above f16's range (|x| up to ~4e6), of ~1e-30 values, and of
+    zeros: each row is shifted by a power of two before the f16 conversion, so every row
+    meets the bar and the zero row gives exact zeros."""
+    W, x = S.block_varied_case(3000 + M, M, N, K)
+    xf = (np.asarray(x, np.uint32) << 16).view(np.float32).astype(np.float64)
+    for m in range(M):
+        xf[m] *= (2.0 ** 20, 1e-30, 1.0, 0.0)[m % 4]
+    x = S.f32_to_bf16_bits(xf.astype(np.float32))
+    q, s, codes_ref, scales_ref = packed(nv, W)
+    Y = nv.fp8_gemm(to_dev_bf16(x), q, s)
+    nv.check()
+    y_ref = P.gemm_fp8_ref(x, codes_ref, scales_ref)
+    y = Y.cpu().numpy().astype(np.float64)
+    assert np.isfinite(y).all()
+    err = np.abs(y - y_ref).max(axis=1)
+    assert (err <= TOL * np.abs(y_ref).max(axis=1)).all()
+
+
 def test_fp8_gemm_bf16_and_repeat(nv):
     M, N, K = 17, 2500, 2048
     W, x = S.block_varied_case(1100, M, N, K)

@@ -21,6 +21,7 @@ from oracle import verify as V
 
 pytestmark = pytest.mark.gpu
 REL_TOL = 2e-3
+TERMS_TOL = 1e-4          # the block-scaled path's five residual activation terms (~1e-5 measured)
 
 
 @pytest.fixture(scope="module")
@@ -277,31 +278,6 @@ def test_verify_lmhead_slice_m68(nv):
     run_verify(nv, W, x, Lstar, S.DRAFT_LEN)
 
 
-def test_verify_full_vocab_sampled(nv):
-    """Full 248,320-row vocabulary at M = 17: sampled property checks (the full
-    oracle argmax is too slow here). The GPU's winning logit must equal the
-    oracle's logit at that index. No sampled row may beat it by more than the tie
-    band. The accept lengths must follow from the GPU's argmax."""
-    W, x, Lstar = S.lmhead_inputs(N=S.VOCAB, B=1)
-    N, K = W.shape
-    D = S.DRAFT_LEN
-    drafts = np.random.default_rng(9).integers(0, N, size=(1, D)).astype(np.int32)
-    q, sf, ts = nv.pack(torch.from_numpy(W).cuda())
-    t, L, vmax = nv.verify(to_dev_bf16(x), q, sf, ts, torch.from_numpy(drafts).cuda())
-    torch.cuda.synchronize()
-    t, L, vmax = t.cpu().numpy(), L.cpu().numpy(), vmax.cpu().numpy()
-    ts_ref = F.tensor_scale(W)
-    rows = np.unique(np.concatenate([t, np.random.default_rng(10).choice(N, 3000, replace=False)]))
-    qs, sfs, _ = F.quantize_nvfp4(W[rows], ts_ref)
-    y_s = G.gemm_ref(x, qs, sfs, ts_ref)                  # oracle logits of the sampled rows, all tokens
-    col = {int(r): i for i, r in enumerate(rows)}
-    for m in range(len(t)):
-        y_t = y_s[m, col[int(t[m])]]
-        assert abs(vmax[m] - y_t) <= 1e-4 * max(1.0, abs(y_t))
-        assert (y_s[m] <= y_t + V.NEAR_TIE).all()
-    assert np.array_equal(L, V.accept_ref(t, drafts, D))
-
-
 def test_verify_workspace_too_small(nv):
     W, x = S.random_case(5, 2, 500, 64)
     q, sf, ts = nv.pack(torch.from_numpy(W).cuda())
@@ -336,7 +312,9 @@ def test_gemm_mma(nv, M, N, K, path):
     """mma: block-scaled kind::mxf4nvf4 where M*5 <= 352, else f16; mma_f16: the exact f16 kernel."""
     W, x = S.random_case(M * 31 + N + K, M, N, K)
     Y, y_ref = run_gemm(nv, W, x, path=path)
-    assert_rowwise(Y.cpu().numpy(), y_ref)
+    worst = assert_rowwise(Y.cpu().numpy(), y_ref)
+    if path == "mma" and M * 5 <= 352:                 # block-scaled: five residual activation terms
+        assert worst <= TERMS_TOL, f"{worst:.2e} of max|y|"
 
 
 @pytest.mark.parametrize("path", ["mma", "mma_f16"])
@@ -362,7 +340,9 @@ def test_gemm_layer_shapes_mma(nv, name, M, path):
     """The M=17 and M=68 launch configurations of the bench at the 27B layer shapes."""
     W, x = S.layer(name, M=M)
     Y, y_ref = run_gemm(nv, W, x, path=path)
-    assert_rowwise(Y.cpu().numpy(), y_ref)
+    worst = assert_rowwise(Y.cpu().numpy(), y_ref)
+    if path == "mma":                                  # block-scaled: five residual activation terms
+        assert worst <= TERMS_TOL, f"{worst:.2e} of max|y|"
 
 
 @pytest.mark.parametrize("path", ["mma", "mma_f16"])

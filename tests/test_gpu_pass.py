@@ -5,11 +5,13 @@ A pass splits the concatenated (problem, tile, K-chunk) units of the whole list
 evenly across the SMs. So besides ragged shapes these cases cover: a list with
 fewer units than SMs (one unit per CTA, so nearly every tile is split), CTA ranges
 that cross several problems, tiles split three or more ways, mixed K, M up to the
-two-B-tile layout (M=68), a verify problem at the end, run-to-run determinism, and
-the full-size layer shapes on sampled outputs.
+two-B-tile layout (M=68), a verify problem at the end and run-to-run determinism. The
+full-size layer shapes and the whole vocabulary are in test_gpu_full_vocab.
 
-Bars as in the other parity tests: GEMM rows within 2e-3 of max|y_ref|; argmax and
-accept lengths bit-exact away from near ties (top-2 gap < 1e-3).
+Bars as in the other parity tests: GEMM rows within 2e-3 of max|y_ref| (the task's bar)
+and within 1e-4 (what the five residual activation terms of the block-scaled path are
+claimed to reach, ~1e-5); argmax and accept lengths bit-exact away from near ties
+(top-2 gap < 1e-3).
 """
 
 import numpy as np
@@ -23,6 +25,7 @@ from oracle import verify as V
 
 pytestmark = pytest.mark.gpu
 REL_TOL = 2e-3
+TERMS_TOL = 1e-4
 
 
 @pytest.fixture(scope="module")
@@ -37,11 +40,12 @@ def to_dev_bf16(x_bits: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(x_bits.view(np.int16).copy()).view(torch.bfloat16).cuda()
 
 
-def assert_rowwise(y: np.ndarray, y_ref: np.ndarray, rel=REL_TOL):
+def assert_rowwise(y: np.ndarray, y_ref: np.ndarray, rel=REL_TOL, terms=TERMS_TOL):
     err = np.abs(y.astype(np.float64) - y_ref).max(axis=1)
     scale = np.abs(y_ref).max(axis=1)
     worst = (err / np.maximum(scale, 1e-300)).max()
     assert (err <= rel * scale).all(), f"rowwise error {worst:.3e} > {rel}"
+    assert (err <= terms * scale).all(), f"rowwise error {worst:.3e} > {terms} (five-term accuracy)"
 
 
 def make_problems(nv, shapes, M, seed, y_dtype=torch.float32):
@@ -166,49 +170,3 @@ def test_pass_with_verify_tail(nv, B, D):
     ymax = y_ref[np.arange(M), t]
     assert (np.abs(vmax - ymax) <= REL_TOL * np.abs(y_ref).max(axis=1)).all()
     assert (y_ref.max(axis=1) - ymax <= V.NEAR_TIE).all()
-
-
-def test_pass_layer_shapes_sampled(nv):
-    """The 27B layer shapes at M=17 in one pass with the full 248,320-row lm_head as
-    its verify tail: sampled outputs against the oracle, computed element by element
-    from the oracle's quantisation of the sampled weight rows."""
-    M, D = 17, S.DRAFT_LEN
-    probs, sampled = [], []
-    rng = np.random.default_rng(2024)
-    for name in S.LAYER_ORDER:
-        W, x = S.layer(name, M=M)
-        q, sf, ts = nv.pack(torch.from_numpy(W).cuda())
-        Y = torch.full((M, W.shape[0]), float("nan"), dtype=torch.float32, device="cuda")
-        probs.append((to_dev_bf16(x), q, sf, ts, Y))
-        rows = rng.choice(W.shape[0], 256, replace=False)
-        sampled.append((W[rows].copy(), rows, x, F.tensor_scale(W)))
-        del W
-    Wl, xl, _ = S.lmhead_inputs(N=S.VOCAB, B=1)
-    ql, sfl, tsl = nv.pack(torch.from_numpy(Wl).cuda())
-    drafts = np.random.default_rng(11).integers(0, S.VOCAB, size=(1, D)).astype(np.int32)
-    probs.append((to_dev_bf16(xl), ql, sfl, tsl, None))
-    t = torch.empty(M, dtype=torch.int32, device="cuda")
-    L = torch.empty(1, dtype=torch.int32, device="cuda")
-    vmax = torch.empty(M, dtype=torch.float32, device="cuda")
-    p = nv.WeightPass(probs, M, verify=(torch.from_numpy(drafts).cuda(), t, L, vmax))
-    p.run()
-    torch.cuda.synchronize()
-    nv.check()
-    for (_, _, _, _, Y), (Wr, rows, x, ts_ref) in zip(probs, sampled):
-        q_r, sf_r, _ = F.quantize_nvfp4(Wr, ts_ref)
-        y_s = G.gemm_ref(x, q_r, sf_r, ts_ref)             # oracle at the sampled rows, all tokens
-        y_full = Y.cpu().numpy()
-        assert np.isfinite(y_full).all()
-        scale = np.abs(y_s).max(axis=1)                    # the sampled rows' magnitude stands in for max|y|
-        assert (np.abs(y_full[:, rows] - y_s).max(axis=1) <= REL_TOL * scale).all()
-    t, L, vmax = t.cpu().numpy(), L.cpu().numpy(), vmax.cpu().numpy()
-    rows = np.unique(np.concatenate([t, np.random.default_rng(12).choice(S.VOCAB, 3000, replace=False)]))
-    ts_l = F.tensor_scale(Wl)
-    q_r, sf_r, _ = F.quantize_nvfp4(Wl[rows], ts_l)
-    y_s = G.gemm_ref(xl, q_r, sf_r, ts_l)
-    col = {int(r): i for i, r in enumerate(rows)}
-    for m in range(M):
-        y_t = y_s[m, col[int(t[m])]]
-        assert abs(vmax[m] - y_t) <= 1e-4 * max(1.0, abs(y_t))
-        assert (y_s[m] <= y_t + V.NEAR_TIE).all()
-    assert np.array_equal(L, V.accept_ref(t, drafts, D))

@@ -228,22 +228,72 @@ def test_w4a4_baseline_passes():
 
 def test_w4a4_fp8_style_row_scale_caught(monkeypatch):
     """g = amax/448 (an FP8 rule) in place of amax/2688."""
-    from oracle import gemm as G
-    monkeypatch.setattr(G, "TENSOR_SCALE_DIVISOR", 448.0)
+    monkeypatch.setattr(F, "TENSOR_SCALE_DIVISOR", 448.0)
     assert not _w4a4_pins_pass()
 
 
 def test_w4a4_dropped_sign_caught(monkeypatch):
-    from oracle import gemm as G
-    orig = G.e2m1_encode
-    monkeypatch.setattr(G, "e2m1_encode", lambda r: orig(np.abs(np.asarray(r, np.float64))))
+    orig = F.e2m1_encode
+    monkeypatch.setattr(F, "e2m1_encode", lambda r: orig(np.abs(np.asarray(r, np.float64))))
     assert not _w4a4_pins_pass()
 
 
 def test_w4a4_ties_away_from_zero_caught(monkeypatch):
+    orig = F.e2m1_encode
+    monkeypatch.setattr(F, "e2m1_encode", lambda r: orig(np.asarray(r, np.float64) * (1.0 + 2.0 ** -30)))
+    assert not _w4a4_pins_pass()
+
+
+def _fp32_activation_quantiser(recip_scale: bool, fp32_codes: bool):
+    """A planted mistake: the activation rows quantised with fp32 steps instead of exact
+    quotients: the block scale as amax_block * fp32(1 / fp32(6 g)) and/or the code from
+    fp32(x / fp32(S g))."""
     from oracle import gemm as G
-    orig = G.e2m1_encode
-    monkeypatch.setattr(G, "e2m1_encode", lambda r: orig(np.asarray(r, np.float64) * (1.0 + 2.0 ** -30)))
+
+    def q(x_bits):
+        x = G.bf16_bits_to_float64(x_bits).astype(np.float32)
+        M, K = x.shape
+        amax = np.max(np.abs(x), axis=1)
+        g = (amax / np.float32(2688.0)).astype(np.float32)
+        blocks = x.reshape(M, K // 16, 16)
+        bmax = np.max(np.abs(blocks), axis=2)
+        with np.errstate(divide="ignore", invalid="ignore"):
+            if recip_scale:
+                inv = np.where(g > 0, np.float32(1.0) / (np.float32(6.0) * g), np.float32(0.0)).astype(np.float32)
+                a = (bmax * inv[:, None]).astype(np.float64)
+            else:
+                a = np.where(g[:, None] > 0, bmax.astype(np.float64) / (6.0 * g[:, None].astype(np.float64)), 0.0)
+            sf = F.e4m3_encode(a)
+            Sv = F.E4M3_VALUES[sf]
+            if fp32_codes:
+                den = (Sv.astype(np.float32) * g[:, None]).astype(np.float32)
+                r = np.where(den[:, :, None] > 0, blocks / np.where(den > 0, den, 1)[:, :, None], 0).astype(np.float32)
+            else:
+                den = Sv * g[:, None].astype(np.float64)
+                r = np.where(den[:, :, None] > 0, blocks / np.where(den > 0, den, 1)[:, :, None], 0.0)
+        codes = np.where(Sv[:, :, None] > 0, F.e2m1_encode(np.asarray(r, np.float64)), 0).astype(np.uint8)
+        return codes.reshape(M, K), sf.astype(np.uint8), g
+    return q
+
+
+def test_w4a4_plain_form_of_the_planted_quantiser_passes(monkeypatch):
+    """The planting helper with exact quotients is the oracle's rule: the pins pass with it."""
+    from oracle import gemm as G
+    monkeypatch.setattr(G, "quantize_x_rows", _fp32_activation_quantiser(False, False))
+    assert _w4a4_pins_pass()
+
+
+def test_w4a4_reciprocal_block_scale_caught(monkeypatch):
+    """S from amax_block * fp32(1 / fp32(6 g)) instead of the exact quotient (golden row 5)."""
+    from oracle import gemm as G
+    monkeypatch.setattr(G, "quantize_x_rows", _fp32_activation_quantiser(True, False))
+    assert not _w4a4_pins_pass()
+
+
+def test_w4a4_fp32_code_quotient_caught(monkeypatch):
+    """Codes from fp32(x / fp32(S g)) instead of the exact quotient (golden row 4)."""
+    from oracle import gemm as G
+    monkeypatch.setattr(G, "quantize_x_rows", _fp32_activation_quantiser(False, True))
     assert not _w4a4_pins_pass()
 
 

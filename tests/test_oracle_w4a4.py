@@ -3,6 +3,7 @@ product with NVFP4 weights. CPU only."""
 
 import json
 import os
+from fractions import Fraction
 
 import numpy as np
 import pytest
@@ -30,36 +31,45 @@ def test_hand_worked_rows():
     assert codes.tolist() == g["codes"]
 
 
-def _near_midpoint(v: np.ndarray, grid: np.ndarray, ulps: float = 4.0) -> np.ndarray:
-    """True where |v| lies within ``ulps`` fp32 ulps of a midpoint between two grid values."""
-    mids = (grid[1:] + grid[:-1]) / 2.0
-    a = np.abs(v)
-    d = np.min(np.abs(a[..., None] - mids), axis=-1)
-    return d <= ulps * np.spacing(np.float32(1.0)) * np.maximum(a, 1e-30)
+def _nearest_even(q, values, codes):
+    """The value of ``values`` nearest to the exact rational q >= 0, ties to the even code,
+    saturating at the largest (a brute-force search over the whole value set)."""
+    best = None
+    for v, c in zip(values, codes):
+        d = abs(Fraction(v) - q)
+        if best is None or d < best[0] or (d == best[0] and c % 2 == 0):
+            best = (d, v, c)
+    return best[2]
 
 
-def test_agrees_with_the_float64_weight_quantiser_except_at_boundaries():
-    """Per row, the fp32 decisions agree with the weight quantiser's float64 ones except where
-    the float64 value sits within a few fp32 ulps of a rounding midpoint (bf16 inputs hit
-    exact midpoints often), or in a block whose scale already differs."""
-    _, x = S.random_case(5, 64, 16, 4096)
+def test_rows_against_exact_fractions():
+    """Brute force in exact rational arithmetic: g is the fp32 rounding of amax/2688; S is
+    the E4M3 value nearest to amax_block/(6 g) and each code the E2M1 value nearest to
+    x/(S g), found by search over the whole value sets with ties to the even code. Random
+    rows, plus rows built around E4M3 and E2M1 midpoints."""
+    e4 = [(float(F.E4M3_VALUES[c]), c) for c in range(0x7F)]
+    e2 = [(float(F.E2M1_VALUES[c]), c) for c in range(8)]
+    _, x = S.random_case(5, 6, 16, 64)
+    xf = G.bf16_bits_to_float64(x)
+    xf[1, 16:32] *= 1e-4                                    # one block far below the row amax
+    xf[2, :] = np.round(xf[2, :] * 8) / 8                   # many exact halves and quarters: ties
+    x = S.f32_to_bf16_bits(xf.astype(np.float32))
+    xf = G.bf16_bits_to_float64(x)
     codes, sf, g = G.quantize_x_rows(x)
-    xf = G.bf16_bits_to_float64(x).astype(np.float32)
-    e4m3_pos = np.unique(np.abs(F.E4M3_VALUES[np.isfinite(F.E4M3_VALUES)]))
-    e2m1_pos = np.unique(np.abs(F.E2M1_VALUES))
-    n_diff = 0
     for m in range(x.shape[0]):
-        c64, s64, ts = F.quantize_codes(xf[m:m + 1], tensor_scale_in=g[m])
-        assert np.float32(ts) == g[m]
-        blocks = xf[m].astype(np.float64).reshape(-1, 16)
-        a64 = np.abs(blocks).max(axis=1) / (6.0 * float(g[m]))
-        bad_s = s64[0] != sf[m]
-        assert _near_midpoint(a64[bad_s], e4m3_pos).all()
-        r64 = blocks / (F.E4M3_VALUES[s64[0]][:, None] * float(g[m]))
-        bad_c = (c64[0] != codes[m]).reshape(-1, 16) & ~bad_s[:, None]
-        assert _near_midpoint(r64[bad_c], e2m1_pos).all()
-        n_diff += int(bad_c.sum())
-    assert n_diff <= 0.001 * codes.size
+        amax = float(np.max(np.abs(xf[m])))
+        g_ref = np.float32(np.float32(amax) / np.float32(2688.0))   # fp32 quotient, correctly rounded
+        assert g[m] == g_ref
+        gq = Fraction(float(g_ref))
+        for b in range(x.shape[1] // 16):
+            blk = xf[m, 16 * b: 16 * b + 16]
+            s_code = _nearest_even(Fraction(float(np.max(np.abs(blk)))) / (6 * gq), *zip(*e4)) if gq else 0
+            assert sf[m, b] == s_code, (m, b)
+            den = Fraction(float(F.E4M3_VALUES[s_code])) * gq
+            for k in range(16):
+                want = 0 if den == 0 else _nearest_even(abs(Fraction(float(blk[k]))) / den, *zip(*e2)) | \
+                    (8 if np.signbit(blk[k]) else 0)
+                assert codes[m, 16 * b + k] == want, (m, b, k)
 
 
 def test_dequantised_rows_within_half_a_step():

@@ -86,3 +86,16 @@ def test_block_varied_case_scales_whole_blocks_by_powers_of_two():
             r = np.unique(ratio[i:i + 128, j:j + 128])
             assert r.size == 1 and r[0] == 2.0 ** e[i // 128, j // 128]
     assert np.array_equal(x, S.normal_x_bits(rng, 2, 384))
+
+
+def test_lmhead_weight_is_chunk_seeded():
+    """Chunk c of the lm_head weight comes from default_rng([7, c]) alone, so a slice is the
+    first rows of the full weight and any chunk can be drawn by itself."""
+    K = 32
+    W = S.lmhead_weight(N=3 * S.LMHEAD_CHUNK + 5, K=K)
+    ref1 = (np.random.default_rng([S.LMHEAD_W_SEED, 1]).standard_normal((S.LMHEAD_CHUNK, K)) * S.W_STD)
+    assert np.array_equal(W[S.LMHEAD_CHUNK: 2 * S.LMHEAD_CHUNK], ref1.astype(np.float32))
+    assert np.array_equal(W[3 * S.LMHEAD_CHUNK:], S.lmhead_weight_chunk(3, N=3 * S.LMHEAD_CHUNK + 5, K=K))
+    assert np.array_equal(S.lmhead_weight(N=S.LMHEAD_CHUNK + 7, K=K), W[:S.LMHEAD_CHUNK + 7])
+    x4, x1 = S.lmhead_x(B=4, K=K), S.lmhead_x(B=1, K=K)
+    assert x4.shape == (68, K) and np.array_equal(x4[:17], x1)
