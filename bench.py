@@ -226,6 +226,7 @@ class Pass:
             verify = verify + (self.parents, self.node)
         self.binv = binv
         self.wp = nv.WeightPass(problems, M, verify=verify, batch_invariant=binv)
+        self.problems, self.verify_bufs = problems, verify
         if chain:
             wsb = max(nv.gemm_workspace_bytes(M, N, K) for (_, K, N, _, _, _) in stack)
             self.gws = torch.zeros(max(wsb, 16), dtype=torch.uint8, device=dev)
@@ -295,20 +296,218 @@ class Pass:
         per = np.array([ev[k].elapsed_time(ev[k + 1]) for k in range(steps)])
         return ev[0].elapsed_time(ev[-1]), per
 
+    def add_second_input_buffer(self):
+        """A second device copy of every X with its own weight pass and graph (same weights, Y
+        and verify outputs), so that the end-to-end leg can copy step k+1's inputs in while
+        step k's pass runs."""
+        torch, M = self.torch, self.M
+        self.x_all2 = torch.empty_like(self.x_all)
+        xs2, off = [], 0
+        for x in self.xs:
+            xs2.append(self.x_all2[off: off + x.numel()])
+            off += x.numel()
+        probs2 = [(xs2[i].view(M, X.shape[1]), q, sf, ts, Y) for i, (X, q, sf, ts, Y) in enumerate(self.problems)]
+        self.wp2 = self.nv.WeightPass(probs2, M, verify=self.verify_bufs, batch_invariant=self.binv)
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self.wp2.run()
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        self.g_pass2 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.g_pass2):
+            self.wp2.run()
+        torch.cuda.synchronize()
+
     def run_e2e(self, steps: int, x_host, out_host):
-        """Host buffers: copy every input in (pinned -> device) and the verify result out, each step."""
+        """Through the public API with host buffers, every step: the step's inputs copied in
+        from pinned host memory, the pass, and the verify result (argmax and accept lengths)
+        copied out. Two device input buffers alternate: step k+1's copy runs on its own
+        stream while step k's pass runs, and a buffer is refilled only after the pass that
+        read it has finished. Returns the device time of the whole sequence (ms)."""
         torch = self.torch
         st = torch.cuda.current_stream()
+        cp = torch.cuda.Stream()
+        bufs, graphs = (self.x_all, self.x_all2), (self.g_pass, self.g_pass2)
+        ev = lambda: torch.cuda.Event()                                        # noqa: E731
+        copied, used = [ev() for _ in range(steps)], [ev() for _ in range(steps)]
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(st)
-        for _ in range(steps):
-            self.x_all.copy_(x_host, non_blocking=True)
-            self.g_pass.replay()
-            out_host[0][: self.M].copy_(self.argmax, non_blocking=True)
-            out_host[1][: self.B].copy_(self.accept, non_blocking=True)
+        cp.wait_stream(st)
+        for k in range(min(2, steps)):                                         # fill both buffers
+            with torch.cuda.stream(cp):
+                bufs[k % 2].copy_(x_host[k % len(x_host)], non_blocking=True)
+                copied[k].record(cp)
+        for k in range(steps):
+            st.wait_event(copied[k])
+            graphs[k % 2].replay()
+            used[k].record(st)
+            out_host[0][k % len(out_host[0])][: self.M].copy_(self.argmax, non_blocking=True)
+            out_host[1][k % len(out_host[1])][: self.B].copy_(self.accept, non_blocking=True)
+            if k + 2 < steps:                                                  # refill this buffer
+                cp.wait_event(used[k])
+                with torch.cuda.stream(cp):
+                    bufs[k % 2].copy_(x_host[(k + 2) % len(x_host)], non_blocking=True)
+                    copied[k + 2].record(cp)
         e1.record(st)
         torch.cuda.synchronize()
         return e0.elapsed_time(e1)
+
+
+def time_calls(torch, calls, reps: int) -> float:
+    """Mean device time (us) of one call in a stream of ``calls`` repeated ``reps`` times:
+    the calls are captured once into a CUDA graph, which is replayed after two warm-up
+    replays, with CUDA events on the launching stream around the timed replays."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):                       # first calls outside capture (one-time set-up)
+        for c in calls:
+            c()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for c in calls:
+            c()
+    for _ in range(2):
+        g.replay()
+    st = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(st)
+    for _ in range(reps):
+        g.replay()
+    e1.record(st)
+    torch.cuda.synchronize()
+    del g
+    return 1e3 * e0.elapsed_time(e1) / (reps * len(calls))
+
+
+def _entry(us: float, wbytes: int, alg_bytes: int, peak: float, **kw) -> dict:
+    d = {"us": round(us, 3), "weight_gbs": round(wbytes / us / 1e3, 1),
+         "pct_of_8tbs": round(100.0 * wbytes / (us * 1e-6) / 8e12, 2),
+         "alg_gbs": round(alg_bytes / us / 1e3, 1), "hbm_frac": round(alg_bytes / us / 1e3 / peak, 4)}
+    d.update(kw)
+    return d
+
+
+def run_extras(nv, torch, dev, stack, lm, peak: float, reps: int) -> dict:
+    """The measurement configurations beside the full pass, each a stream of single library
+    calls timed as a CUDA graph, rotating through distinct weight copies so every call
+    reads its weights from HBM:
+      single_m1   one GEMM at M=1 (nvfp4_gemm_skinny, the GEMV path) at each 27B layer
+                  shape, over the stack's 64 copies of that shape;
+      verify      the standalone fused verify (lmhead_verify_argmax_accept) at N=248,320
+                  and at the 65,536-row slice (four disjoint slices in turn), M=17 and 68;
+      m_sweep     one GEMM (nvfp4_gemm_skinny, default path) on gate+up 5120->34816 at
+                  M in {1, 2, 4, 8, 17, 34, 68, 128}, over the 64 copies.
+    Per entry: us per call, weight GB/s, % of 8 TB/s and the algorithmic bytes (weights,
+    activations, outputs) over the measured HBM peak."""
+    out = {}
+    g = torch.Generator(device=dev)
+    g.manual_seed(4242)
+    by_shape = {n: [(q, sf, ts) for (nm, _, _, q, sf, ts) in stack if nm == n] for n in S.LAYER_ORDER}
+
+    single = {}
+    for name in S.LAYER_ORDER:
+        K, N = S.LAYER_SHAPES[name]
+        X = torch.randn(1, K, generator=g, device=dev).to(torch.bfloat16)
+        Y = torch.empty(1, N, device=dev)
+        ws = torch.zeros(max(16, nv.gemm_workspace_bytes(1, N, K)), dtype=torch.uint8, device=dev)
+        calls = [lambda q=q, sf=sf, ts=ts: nv.gemm(X, q, sf, ts, out=Y, workspace=ws) for (q, sf, ts) in by_shape[name]]
+        wb = weight_bytes(N, K)
+        single[name] = _entry(time_calls(torch, calls, reps), wb, wb + K * 2 + N * 4, peak, N=N, K=K,
+                              copies=len(calls), path="gemv")
+    out["single_m1"] = single
+
+    ql, sfl, tsl = lm
+    verify = {}
+    for N in (S.VOCAB, S.VOCAB_SLICE):
+        heads = [(ql[i:i + N], sfl[i:i + N]) for i in range(0, S.VOCAB - N + 1, N)][:4]
+        for M in (17, 68):
+            B = M // (S.DRAFT_LEN + 1)
+            X = torch.randn(M, S.LMHEAD_K, generator=g, device=dev).to(torch.bfloat16)
+            drafts = torch.randint(0, N, (B, S.DRAFT_LEN), generator=g, device=dev, dtype=torch.int32)
+            o = (torch.empty(M, dtype=torch.int32, device=dev), torch.empty(B, dtype=torch.int32, device=dev),
+                 torch.empty(M, dtype=torch.float32, device=dev))
+            ws = torch.zeros(nv.verify_workspace_bytes(M, N, S.LMHEAD_K), dtype=torch.uint8, device=dev)
+            calls = [lambda q=q, sf=sf: nv.verify(X, q, sf, tsl, drafts, workspace=ws, out=o) for (q, sf) in heads]
+            wb = weight_bytes(N, S.LMHEAD_K)
+            verify[f"N{N}_M{M}"] = _entry(time_calls(torch, calls, reps * 4), wb, wb + M * S.LMHEAD_K * 2, peak,
+                                          N=N, M=M, B=B, copies=len(heads))
+    out["verify"] = verify
+
+    K, N = S.LAYER_SHAPES["gate_up"]
+    sweep = {}
+    for M in S.SWEEP_M:
+        X = torch.randn(M, K, generator=g, device=dev).to(torch.bfloat16)
+        Y = torch.empty(M, N, device=dev)
+        ws = torch.zeros(max(16, nv.gemm_workspace_bytes(M, N, K)), dtype=torch.uint8, device=dev)
+        calls = [lambda q=q, sf=sf, ts=ts: nv.gemm(X, q, sf, ts, out=Y, workspace=ws) for (q, sf, ts) in by_shape["gate_up"]]
+        wb = weight_bytes(N, K)
+        sweep[str(M)] = _entry(time_calls(torch, calls, reps), wb, wb + M * K * 2 + M * N * 4, peak,
+                               copies=len(calls))
+    out["m_sweep_gate_up"] = sweep
+    return out
+
+
+def run_fp8_extras(nv, torch, dev, peak: float, layers: int, reps: int) -> dict:
+    """FP8 weights (E4M3, one fp32 scale per 128 x 128 block) in the pages' precision map: the
+    64 qkv projections (5120->10240) and the 248,320-row output head, packed on the GPU from
+    seeded N(0, 0.02) weights (4.63 GB, 37 times L2).
+      pass_M{17,68}     one FP8 weight pass over the 64 qkv GEMMs with the head as its verify
+                        tail (fp8_pass_run), timed as a CUDA graph;
+      head_verify_M*    the head's fused verify alone (fp8_lmhead_verify);
+      head_gemm_M1      the head as a plain M=1 GEMM (fp8_gemm_skinny).
+    Per entry: us per call, weight GB/s, % of 8 TB/s and algorithmic bytes over the measured
+    HBM peak."""
+    K, N = S.LAYER_SHAPES["qkv"]
+    qkv = []
+    for layer in range(layers):
+        g = torch.Generator(device=dev)
+        g.manual_seed(7000 + layer)
+        W = torch.randn(N, K, generator=g, device=dev).mul_(S.W_STD)
+        qkv.append(nv.fp8_pack(W))
+        del W
+    g = torch.Generator(device=dev)
+    g.manual_seed(S.LMHEAD_W_SEED)
+    W = torch.randn(S.VOCAB, S.LMHEAD_K, generator=g, device=dev).mul_(S.W_STD)
+    qh, sh = nv.fp8_pack(W)
+    del W
+    torch.cuda.synchronize()
+    head_bytes = S.VOCAB * S.LMHEAD_K + sh.numel() * 4
+    qkv_bytes = sum(N * K + sc.numel() * 4 for (_, sc) in qkv)
+    out = {}
+    gx = torch.Generator(device=dev)
+    gx.manual_seed(77)
+    for M in (17, 68):
+        B = M // (S.DRAFT_LEN + 1)
+        drafts = torch.zeros((B, S.DRAFT_LEN), dtype=torch.int32, device=dev)
+        t = torch.empty(M, dtype=torch.int32, device=dev)
+        L = torch.empty(B, dtype=torch.int32, device=dev)
+        Xh = torch.randn(M, S.LMHEAD_K, generator=gx, device=dev).to(torch.bfloat16)
+        probs = [(torch.randn(M, K, generator=gx, device=dev).to(torch.bfloat16), q, sc,
+                  torch.empty((M, N), dtype=torch.bfloat16, device=dev)) for (q, sc) in qkv]
+        probs.append((Xh, qh, sh, None))
+        p8 = nv.Fp8Pass(probs, M, verify=(drafts, t, L, None))
+        wb = qkv_bytes + head_bytes
+        alg = wb + M * (K * 2 * layers + S.LMHEAD_K * 2) + M * N * 2 * layers
+        out[f"pass_M{M}"] = _entry(time_calls(torch, [p8.run], max(3, reps // 2)), wb, alg, peak, M=M,
+                                   problems=len(probs))
+        del p8, probs
+        ws = torch.zeros(int(nv.lib().fp8_lmhead_verify_workspace_bytes(M, S.VOCAB, S.LMHEAD_K)), dtype=torch.uint8,
+                         device=dev)
+        out[f"head_verify_M{M}"] = _entry(
+            time_calls(torch, [lambda: nv.fp8_verify(Xh, qh, sh, drafts, workspace=ws)], reps * 4), head_bytes,
+            head_bytes + M * S.LMHEAD_K * 2, peak, M=M)
+    X1 = torch.randn(1, S.LMHEAD_K, generator=gx, device=dev).to(torch.bfloat16)
+    Y1 = torch.empty(1, S.VOCAB, device=dev)
+    ws = torch.zeros(int(nv.lib().fp8_gemm_workspace_bytes(1, S.VOCAB, S.LMHEAD_K)), dtype=torch.uint8, device=dev)
+    out["head_gemm_M1"] = _entry(time_calls(torch, [lambda: nv.fp8_gemm(X1, qh, sh, out=Y1, workspace=ws)], reps * 4),
+                                 head_bytes, head_bytes + S.LMHEAD_K * 2 + S.VOCAB * 4, peak, M=1)
+    del qkv, qh, sh
+    torch.cuda.synchronize()
+    return {"fp8": out}
 
 
 def cpu_baseline(seconds: float = 12.0):
@@ -435,14 +634,29 @@ def run_ours(args, rank, world, local_rank):
             res["chained_weight_gbs"] = job_gbs(world, wbytes, chain_ms)
         results[M] = res
 
-    # end to end through the public API with host buffers (headline M)
+    # single calls and the standalone verify (the other measurement configurations)
+    extras, clocks_extras = None, None
+    if not args.no_extras:
+        if dist:
+            dist.barrier()
+        sampler = ClockSampler(local_rank) if rank == 0 else None
+        if sampler:
+            sampler.start()
+        extras = run_extras(nv, torch, dev, stack, lm, peak, reps=max(3, args.steps // 4))
+        extras.update(run_fp8_extras(nv, torch, dev, peak, args.layers, reps=max(3, args.steps // 4)))
+        if sampler:
+            clocks_extras = sampler.stop()
+
+    # end to end through the public API with host buffers (headline M): two host input sets
+    # (distinct values each step), two device input buffers, the result read back each step
     p = passes[head]
-    x_host = torch.empty(p.x_all.numel(), dtype=torch.bfloat16, pin_memory=True)
-    x_host.copy_(p.x_all.cpu())
-    out_host = (torch.empty(p.M, dtype=torch.int32, pin_memory=True),
-                torch.empty(p.B, dtype=torch.int32, pin_memory=True))
-    for _ in range(args.warmup):
-        p.run_e2e(1, x_host, out_host)
+    p.add_second_input_buffer()
+    x_host = [torch.empty(p.x_all.numel(), dtype=torch.bfloat16, pin_memory=True) for _ in range(2)]
+    x_host[0].copy_(p.x_all.cpu())
+    x_host[1].copy_(x_host[0].flip(0))
+    out_host = ([torch.empty(p.M, dtype=torch.int32, pin_memory=True) for _ in range(2)],
+                [torch.empty(p.B, dtype=torch.int32, pin_memory=True) for _ in range(2)])
+    p.run_e2e(max(2, args.warmup), x_host, out_host)
     if dist:
         dist.barrier()
     e2e_ms = max_over_ranks(dist, torch, p.run_e2e(args.steps, x_host, out_host), dev) / args.steps
@@ -485,10 +699,17 @@ def run_ours(args, rank, world, local_rank):
                      "traffic": args.traffic if args.traffic is not None else measured_traffic(head, args.layers),
                      "algorithmic_bytes_per_launch": pass_alg_bytes(head, args.layers)},
         "e2e": {"value": job_gbs(world, wbytes, e2e_ms), "unit": "GB/s", "ms_per_step": e2e_ms,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "what": "every X of the pass copied in from pinned host memory each step (double-buffered: the "
+                        "next step's copy runs under the current pass); the verify result read back each step: "
+                        "argmax [M] and accept_len [B] int32 (the GEMM outputs stay on the device for the next "
+                        "layer)"},
         "gpu_launches": r["launches_per_pass"] * args.steps,
         "clocks": clocks,
     }
+    if extras is not None:
+        line.update(extras)
+        line["clocks_extras"] = clocks_extras
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     print(json.dumps(line), flush=True)
@@ -793,6 +1014,8 @@ def main():
     ap.add_argument("--ms", default="17,1,68", help="comma list of M; the first 17 (else the first) is the headline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-chain", action="store_true", help="skip the chained per-GEMM comparison")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the single-call, standalone-verify and M-sweep entries of the default line")
     ap.add_argument("--layers", type=int, default=S.N_LAYERS,
                     help="layers in the stack (the default is the 27B model's; fewer only for small profiling cases)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
