@@ -845,7 +845,7 @@ def run_fp8(args):
     nvbuild.build()
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    N, K = S.VOCAB, S.LMHEAD_K
+    N, K = args.fp8_rows, S.LMHEAD_K
     g = torch.Generator(device=dev)
     g.manual_seed(S.LMHEAD_W_SEED)
     W = torch.randn(N, K, generator=g, device=dev) * S.W_STD
@@ -1031,6 +1031,8 @@ def main():
                     help="the 27B step with NVFP4 MLP weights and an FP8 qkv projection and lm_head")
     ap.add_argument("--fp8", action="store_true",
                     help="the FP8 (E4M3, 128x128 block-scaled) output head: verify and GEMM per M")
+    ap.add_argument("--fp8-rows", type=int, default=S.VOCAB,
+                    help="rows of the FP8 head for --fp8 (fewer only for small profiling cases)")
     ap.add_argument("--sweep", action="store_true", help="time one matrix shape per M and path (no pass)")
     ap.add_argument("--shape", default="gate_up", help="sweep shape: gate_up, down, qkv or lm_head")
     ap.add_argument("--paths", default="auto,gemv,mma")
