@@ -656,15 +656,16 @@ def run_fp8(args):
             B = M // (S.DRAFT_LEN + 1)
             drafts = torch.zeros((B, S.DRAFT_LEN), dtype=torch.int32, device=dev)
             wsv = torch.zeros(int(nv.lib().fp8_lmhead_verify_workspace_bytes(M, N, K)), dtype=torch.uint8, device=dev)
-            calls.append(("verify", lambda: nv.fp8_verify(X, q, sc, drafts, workspace=wsv)))
+            calls.append(("verify", lambda: nv.fp8_verify(X, q, sc, drafts, workspace=wsv, path=args.fp8_path)))
         Y = torch.empty((M, N), dtype=torch.float32, device=dev)
         wsg = torch.zeros(int(nv.lib().fp8_gemm_workspace_bytes(M, N, K)), dtype=torch.uint8, device=dev)
-        calls.append(("gemm", lambda: nv.fp8_gemm(X, q, sc, out=Y, workspace=wsg)))
+        calls.append(("gemm", lambda: nv.fp8_gemm(X, q, sc, out=Y, workspace=wsg, path=args.fp8_path)))
         for name, fn in calls:
             ms, ms_min = timed(fn)
             gbs = wbytes / (ms * 1e-3) / 1e9
             print(json.dumps({
                 "metric": f"FP8 lm_head {name} (E4M3, 128x128 fp32 block scales)", "M": M, "N": N, "K": K,
+                "fp8_path": args.fp8_path,
                 "ms": ms, "ms_min": ms_min, "weight_gbs": gbs, "hbm_frac": gbs / hbm, "hbm_peak_kind": hbm_kind,
                 "steps": args.steps, "warmup": args.warmup, "cpu_baseline": cpu}), flush=True)
 
@@ -808,6 +809,8 @@ def main():
                     help="the 27B step with NVFP4 MLP weights and an FP8 qkv projection and lm_head")
     ap.add_argument("--fp8", action="store_true",
                     help="the FP8 (E4M3, 128x128 block-scaled) output head: verify and GEMM per M")
+    ap.add_argument("--fp8-path", choices=["f16", "terms"], default="f16",
+                    help="FP8 kernel: codes dequantised to f16, or straight into the FP8 tensor cores")
     ap.add_argument("--sweep", action="store_true", help="time one matrix shape per M and path (no pass)")
     ap.add_argument("--shape", default="gate_up", help="sweep shape: gate_up, down, qkv or lm_head")
     ap.add_argument("--paths", default="auto,gemv,mma")
