@@ -201,3 +201,22 @@ def test_fp8_terms_path_extreme_rows(nv):
     assert (Y[2] == 0).all()
     rows = [m for m in range(M) if m != 2]
     assert rowwise_err(Y[rows], y_ref[rows]) <= TOL_TERMS
+
+
+@pytest.mark.parametrize("path", ["f16", "terms"])
+def test_fp8_accumulation_keeps_small_products(nv, path):
+    """One 128-wide block whose sum needs ~19 significant bits: 448 * 1 plus 127 products of
+    2^-10. fp32 accumulation keeps every small product; an accumulator of ~14 bits would drop
+    them (an error of ~3e-4 of the result). This measures the tensor core's accumulation width."""
+    M, N, K = 1, 128, 128
+    W = np.ones((N, K), dtype=np.float32)
+    W[:, 0] = 448.0                                            # block scale exactly 1, codes 448 and 1
+    x = np.full((M, K), 2.0 ** -10, dtype=np.float32)
+    x[0, 0] = 1.0
+    xb = S.f32_to_bf16_bits(x)
+    q, s, codes_ref, scales_ref = packed(nv, W)
+    assert float(scales_ref[0, 0]) == 1.0
+    Y = nv.fp8_gemm(to_dev_bf16(xb), q, s, path=path).cpu().numpy()
+    nv.check()
+    y_ref = 448.0 + 127 * 2.0 ** -10
+    assert np.abs(Y.astype(np.float64) - y_ref).max() <= 1e-6 * y_ref
