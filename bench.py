@@ -457,8 +457,9 @@ def run_fp8_extras(nv, torch, dev, peak: float, layers: int, reps: int) -> dict:
     seeded N(0, 0.02) weights (4.63 GB, 37 times L2).
       pass_M{17,68}     one FP8 weight pass over the 64 qkv GEMMs with the head as its verify
                         tail (fp8_pass_run), timed as a CUDA graph;
-      head_verify_M*    the head's fused verify alone (fp8_lmhead_verify);
-      head_gemm_M1      the head as a plain M=1 GEMM (fp8_gemm_skinny).
+      head_verify_M*    the head's fused verify alone (fp8_lmhead_verify_path), on the f16
+                        kernel and (suffix _terms) on the E4M3-term kernel;
+      head_gemm_M1*     the head as a plain M=1 GEMM (fp8_gemm_skinny_path), both kernels.
     Per entry: us per call, weight GB/s, % of 8 TB/s and algorithmic bytes over the measured
     HBM peak."""
     K, N = S.LAYER_SHAPES["qkv"]
@@ -497,14 +498,17 @@ def run_fp8_extras(nv, torch, dev, peak: float, layers: int, reps: int) -> dict:
         del p8, probs
         ws = torch.zeros(int(nv.lib().fp8_lmhead_verify_workspace_bytes(M, S.VOCAB, S.LMHEAD_K)), dtype=torch.uint8,
                          device=dev)
-        out[f"head_verify_M{M}"] = _entry(
-            time_calls(torch, [lambda: nv.fp8_verify(Xh, qh, sh, drafts, workspace=ws)], reps * 4), head_bytes,
-            head_bytes + M * S.LMHEAD_K * 2, peak, M=M)
+        for path, tag in (("f16", ""), ("terms", "_terms")):
+            out[f"head_verify_M{M}{tag}"] = _entry(
+                time_calls(torch, [lambda path=path: nv.fp8_verify(Xh, qh, sh, drafts, workspace=ws, path=path)],
+                           reps * 4), head_bytes, head_bytes + M * S.LMHEAD_K * 2, peak, M=M, kernel=path)
     X1 = torch.randn(1, S.LMHEAD_K, generator=gx, device=dev).to(torch.bfloat16)
     Y1 = torch.empty(1, S.VOCAB, device=dev)
     ws = torch.zeros(int(nv.lib().fp8_gemm_workspace_bytes(1, S.VOCAB, S.LMHEAD_K)), dtype=torch.uint8, device=dev)
-    out["head_gemm_M1"] = _entry(time_calls(torch, [lambda: nv.fp8_gemm(X1, qh, sh, out=Y1, workspace=ws)], reps * 4),
-                                 head_bytes, head_bytes + S.LMHEAD_K * 2 + S.VOCAB * 4, peak, M=1)
+    for path, tag in (("f16", ""), ("terms", "_terms")):
+        out[f"head_gemm_M1{tag}"] = _entry(
+            time_calls(torch, [lambda path=path: nv.fp8_gemm(X1, qh, sh, out=Y1, workspace=ws, path=path)], reps * 4),
+            head_bytes, head_bytes + S.LMHEAD_K * 2 + S.VOCAB * 4, peak, M=1, kernel=path)
     del qkv, qh, sh
     torch.cuda.synchronize()
     return {"fp8": out}
@@ -877,15 +881,16 @@ def run_fp8(args):
             B = M // (S.DRAFT_LEN + 1)
             drafts = torch.zeros((B, S.DRAFT_LEN), dtype=torch.int32, device=dev)
             wsv = torch.zeros(int(nv.lib().fp8_lmhead_verify_workspace_bytes(M, N, K)), dtype=torch.uint8, device=dev)
-            calls.append(("verify", lambda: nv.fp8_verify(X, q, sc, drafts, workspace=wsv)))
+            calls.append(("verify", lambda: nv.fp8_verify(X, q, sc, drafts, workspace=wsv, path=args.fp8_path)))
         Y = torch.empty((M, N), dtype=torch.float32, device=dev)
         wsg = torch.zeros(int(nv.lib().fp8_gemm_workspace_bytes(M, N, K)), dtype=torch.uint8, device=dev)
-        calls.append(("gemm", lambda: nv.fp8_gemm(X, q, sc, out=Y, workspace=wsg)))
+        calls.append(("gemm", lambda: nv.fp8_gemm(X, q, sc, out=Y, workspace=wsg, path=args.fp8_path)))
         for name, fn in calls:
             ms, ms_min = timed(fn)
             gbs = wbytes / (ms * 1e-3) / 1e9
             print(json.dumps({
                 "metric": f"FP8 lm_head {name} (E4M3, 128x128 fp32 block scales)", "M": M, "N": N, "K": K,
+                "fp8_path": args.fp8_path,
                 "ms": ms, "ms_min": ms_min, "weight_gbs": gbs, "hbm_frac": gbs / hbm, "hbm_peak_kind": hbm_kind,
                 "steps": args.steps, "warmup": args.warmup, "cpu_baseline": cpu}), flush=True)
 
@@ -1033,6 +1038,8 @@ def main():
                     help="the FP8 (E4M3, 128x128 block-scaled) output head: verify and GEMM per M")
     ap.add_argument("--fp8-rows", type=int, default=S.VOCAB,
                     help="rows of the FP8 head for --fp8 (fewer only for small profiling cases)")
+    ap.add_argument("--fp8-path", choices=["f16", "terms"], default="f16",
+                    help="FP8 kernel: codes dequantised to f16, or straight into the FP8 tensor cores")
     ap.add_argument("--sweep", action="store_true", help="time one matrix shape per M and path (no pass)")
     ap.add_argument("--shape", default="gate_up", help="sweep shape: gate_up, down, qkv or lm_head")
     ap.add_argument("--paths", default="auto,gemv,mma")

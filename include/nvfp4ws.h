@@ -407,13 +407,28 @@ int nvfp4_pass_run(const nvfp4_pass* pass, nvfp4ws_stream_t stream);
  *   verify->B * (verify->D + 1). Workspace: fp8_lmhead_verify_workspace_bytes(M, N, K).
  */
 int fp8_pack(const float* W, int64_t N, int64_t K, uint8_t* q, float* scales, nvfp4ws_stream_t stream);
+
+/* FP8 kernel of fp8_gemm_skinny_path / fp8_lmhead_verify_path. DEQUANT_F16 (the default of the
+ * calls without _path): the codes are converted to f16 (exact) for tcgen05 kind::f16, and every
+ * product is exact. E4M3_TERMS: the codes go straight into kind::f8f6f4, and each row of X is
+ * written as two residual E4M3 terms under one power-of-two scale g = 2^(e-8), amax|x| in
+ * [2^(e-1), 2^e): exact except for elements whose low bits fall below E4M3's subnormal step in
+ * the second term (absolute error below 2^-14 g per element). */
+#define NVFP4WS_FP8_DEQUANT_F16 0
+#define NVFP4WS_FP8_E4M3_TERMS 1
 size_t fp8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 int fp8_gemm_skinny(const void* X, const uint8_t* q, const float* scales, int64_t M, int64_t N, int64_t K,
                     void* Y, int y_dtype, void* workspace, size_t workspace_bytes, nvfp4ws_stream_t stream);
+int fp8_gemm_skinny_path(const void* X, const uint8_t* q, const float* scales, int64_t M, int64_t N, int64_t K,
+                         void* Y, int y_dtype, void* workspace, size_t workspace_bytes, int path,
+                         nvfp4ws_stream_t stream);
 size_t fp8_lmhead_verify_workspace_bytes(int64_t M, int64_t N, int64_t K);
 int fp8_lmhead_verify(const void* X, const uint8_t* q, const float* scales, int64_t M, int64_t N, int64_t K,
                       const nvfp4_verify_spec* verify, void* workspace, size_t workspace_bytes,
                       nvfp4ws_stream_t stream);
+int fp8_lmhead_verify_path(const void* X, const uint8_t* q, const float* scales, int64_t M, int64_t N, int64_t K,
+                           const nvfp4_verify_spec* verify, void* workspace, size_t workspace_bytes, int path,
+                           nvfp4ws_stream_t stream);
 
 /*
  * FP8 weight passes -- a list of independent FP8 GEMMs that share M, run by ONE persistent

@@ -26,6 +26,7 @@ from . import _lib
 PATHS = {"auto": 0, "gemv": 1, "mma": 2, "gemv_regs": 3, "mma_f16": 4}
 PASS_BATCH_INVARIANT = 1
 PASS_W4A4 = 2
+FP8_PATHS = {"f16": 0, "terms": 1}
 STATUS_OK = 0
 
 
@@ -212,8 +213,11 @@ def fp8_pack(W: torch.Tensor, stream=None, out=None):
 
 
 def fp8_gemm(X: torch.Tensor, q: torch.Tensor, scales: torch.Tensor, out: torch.Tensor | None = None,
-             y_dtype: torch.dtype = torch.float32, workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """Y[M, N] = X[M, K] . dequant(W)^T for FP8 block-scaled W (``fp8_gemm_skinny``); X bf16."""
+             y_dtype: torch.dtype = torch.float32, workspace: torch.Tensor | None = None, path: str = "f16",
+             stream=None) -> torch.Tensor:
+    """Y[M, N] = X[M, K] . dequant(W)^T for FP8 block-scaled W (``fp8_gemm_skinny_path``); X bf16.
+    ``path``: "f16" (codes dequantised exactly to f16) or "terms" (codes straight into the FP8
+    tensor cores, X as two residual E4M3 terms)."""
     _need_cuda(X, "X", torch.bfloat16)
     _need_cuda(q, "q", torch.uint8)
     _need_cuda(scales, "scales", torch.float32)
@@ -225,14 +229,14 @@ def fp8_gemm(X: torch.Tensor, q: torch.Tensor, scales: torch.Tensor, out: torch.
     yd = {torch.float32: 0, torch.bfloat16: 1}[Y.dtype]
     ws = _workspace(int(lib().fp8_gemm_workspace_bytes(M, N, K)), X.device, workspace)
     nbytes = 0 if ws is None else ws.numel()
-    _check(lib().fp8_gemm_skinny(_ptr(X), _ptr(q), _ptr(scales), M, N, K, _ptr(Y), yd, _ptr(ws), nbytes,
-                                 _stream(stream)), "fp8_gemm_skinny")
+    _check(lib().fp8_gemm_skinny_path(_ptr(X), _ptr(q), _ptr(scales), M, N, K, _ptr(Y), yd, _ptr(ws), nbytes,
+                                      FP8_PATHS[path], _stream(stream)), "fp8_gemm_skinny")
     return Y
 
 
 def fp8_verify(X: torch.Tensor, q: torch.Tensor, scales: torch.Tensor, drafts: torch.Tensor,
                parents: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
-               with_max_logit: bool = True, stream=None):
+               with_max_logit: bool = True, path: str = "f16", stream=None):
     """Fused greedy verify over an FP8 lm_head (``fp8_lmhead_verify``): the chain rule, or the
     tree rule when ``parents`` is given.
 
@@ -255,8 +259,8 @@ def fp8_verify(X: torch.Tensor, q: torch.Tensor, scales: torch.Tensor, drafts: t
                            _ptr(parents) if parents is not None and parents.numel() else None, _ptr(node))
     ws = _workspace(int(lib().fp8_lmhead_verify_workspace_bytes(M, N, K)), X.device, workspace)
     nbytes = 0 if ws is None else ws.numel()
-    _check(lib().fp8_lmhead_verify(_ptr(X), _ptr(q), _ptr(scales), M, N, K, ctypes.byref(spec), _ptr(ws), nbytes,
-                                   _stream(stream)), "fp8_lmhead_verify")
+    _check(lib().fp8_lmhead_verify_path(_ptr(X), _ptr(q), _ptr(scales), M, N, K, ctypes.byref(spec), _ptr(ws),
+                                        nbytes, FP8_PATHS[path], _stream(stream)), "fp8_lmhead_verify")
     return amax, acc, node, vmax
 
 

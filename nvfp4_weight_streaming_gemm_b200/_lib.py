@@ -82,6 +82,10 @@ SIGNATURES = {
     "fp8_pack": (ctypes.c_int, [c_p, c_i64, c_i64, c_p, c_p, c_p]),
     "fp8_gemm_workspace_bytes": (c_sz, [c_i64, c_i64, c_i64]),
     "fp8_gemm_skinny": (ctypes.c_int, [c_p, c_p, c_p, c_i64, c_i64, c_i64, c_p, ctypes.c_int, c_p, c_sz, c_p]),
+    "fp8_gemm_skinny_path": (ctypes.c_int, [c_p, c_p, c_p, c_i64, c_i64, c_i64, c_p, ctypes.c_int, c_p, c_sz,
+                                            ctypes.c_int, c_p]),
+    "fp8_lmhead_verify_path": (ctypes.c_int, [c_p, c_p, c_p, c_i64, c_i64, c_i64, ctypes.POINTER(VerifySpec), c_p,
+                                              c_sz, ctypes.c_int, c_p]),
     "fp8_lmhead_verify_workspace_bytes": (c_sz, [c_i64, c_i64, c_i64]),
     "fp8_lmhead_verify": (ctypes.c_int, [c_p, c_p, c_p, c_i64, c_i64, c_i64, ctypes.POINTER(VerifySpec), c_p, c_sz,
                                          c_p]),

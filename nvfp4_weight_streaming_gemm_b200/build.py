@@ -15,7 +15,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libnvfp4ws.so")
-SOURCES = ["api.cu", "pack.cu", "gemv.cu", "verify.cu", "mma.cu", "mxf4.cu", "noalloc.cu", "fp8.cu", "xshift.cu"]
+SOURCES = ["api.cu", "pack.cu", "gemv.cu", "verify.cu", "mma.cu", "mxf4.cu", "noalloc.cu", "fp8.cu", "fp8q.cu",
+           "xshift.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -440,10 +440,13 @@ int fp8_pack(const float* W, int64_t N, int64_t K, uint8_t* q, float* scales, nv
   return launch_fp8_pack(W, N, K, q, scales, (cudaStream_t)stream);
 }
 
-size_t fp8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) { return fp8_gemm_workspace_bytes_int(M, N, K); }
+// Enough for either FP8 kernel, so a forced path works with the same buffer.
+size_t fp8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  return std::max(fp8_gemm_workspace_bytes_int(M, N, K), fp8q_workspace_bytes_int(M, N, K, false));
+}
 
 size_t fp8_lmhead_verify_workspace_bytes(int64_t M, int64_t N, int64_t K) {
-  return fp8_verify_workspace_bytes_int(M, N, K);
+  return std::max(fp8_verify_workspace_bytes_int(M, N, K), fp8q_workspace_bytes_int(M, N, K, true));
 }
 
 static int validate_fp8(const void* X, const uint8_t* q, const float* scales, int64_t M, int64_t N, int64_t K,
@@ -462,24 +465,45 @@ static int validate_fp8(const void* X, const uint8_t* q, const float* scales, in
   return NVFP4WS_OK;
 }
 
-int fp8_gemm_skinny(const void* X, const uint8_t* q, const float* scales, int64_t M, int64_t N, int64_t K, void* Y,
-                    int y_dtype, void* workspace, size_t workspace_bytes, nvfp4ws_stream_t stream) {
+int fp8_gemm_skinny_path(const void* X, const uint8_t* q, const float* scales, int64_t M, int64_t N, int64_t K,
+                         void* Y, int y_dtype, void* workspace, size_t workspace_bytes, int path,
+                         nvfp4ws_stream_t stream) {
   g_last_error[0] = 0;
   if (!Y) return set_error(NVFP4WS_ERR_INVALID_ARG, "fp8_gemm_skinny: Y is null");
   if (y_dtype != NVFP4WS_Y_F32 && y_dtype != NVFP4WS_Y_BF16)
     return set_error(NVFP4WS_ERR_INVALID_ARG, "fp8_gemm_skinny: bad y_dtype %d", y_dtype);
-  if (int e = validate_fp8(X, q, scales, M, N, K, workspace, workspace_bytes, fp8_gemm_workspace_bytes_int(M, N, K),
+  if (path != NVFP4WS_FP8_DEQUANT_F16 && path != NVFP4WS_FP8_E4M3_TERMS)
+    return set_error(NVFP4WS_ERR_INVALID_ARG, "fp8_gemm_skinny: bad path %d", path);
+  if (int e = validate_fp8(X, q, scales, M, N, K, workspace, workspace_bytes, fp8_gemm_workspace_bytes(M, N, K),
                            "fp8_gemm_skinny"))
     return e;
   if (!aligned16(Y)) return set_error(NVFP4WS_ERR_MISALIGNED, "fp8_gemm_skinny: Y must be 16-byte aligned");
+  if (path == NVFP4WS_FP8_E4M3_TERMS)
+    return launch_fp8q_gemm(static_cast<const uint16_t*>(X), q, scales, M, N, K, Y, y_dtype, workspace,
+                            (cudaStream_t)stream);
   return launch_fp8_gemm(static_cast<const uint16_t*>(X), q, scales, M, N, K, Y, y_dtype, workspace,
                          (cudaStream_t)stream);
+}
+
+int fp8_gemm_skinny(const void* X, const uint8_t* q, const float* scales, int64_t M, int64_t N, int64_t K, void* Y,
+                    int y_dtype, void* workspace, size_t workspace_bytes, nvfp4ws_stream_t stream) {
+  return fp8_gemm_skinny_path(X, q, scales, M, N, K, Y, y_dtype, workspace, workspace_bytes,
+                              NVFP4WS_FP8_DEQUANT_F16, stream);
 }
 
 int fp8_lmhead_verify(const void* X, const uint8_t* q, const float* scales, int64_t M, int64_t N, int64_t K,
                       const nvfp4_verify_spec* verify, void* workspace, size_t workspace_bytes,
                       nvfp4ws_stream_t stream) {
+  return fp8_lmhead_verify_path(X, q, scales, M, N, K, verify, workspace, workspace_bytes, NVFP4WS_FP8_DEQUANT_F16,
+                                stream);
+}
+
+int fp8_lmhead_verify_path(const void* X, const uint8_t* q, const float* scales, int64_t M, int64_t N, int64_t K,
+                           const nvfp4_verify_spec* verify, void* workspace, size_t workspace_bytes, int path,
+                           nvfp4ws_stream_t stream) {
   g_last_error[0] = 0;
+  if (path != NVFP4WS_FP8_DEQUANT_F16 && path != NVFP4WS_FP8_E4M3_TERMS)
+    return set_error(NVFP4WS_ERR_INVALID_ARG, "fp8_lmhead_verify: bad path %d", path);
   if (!verify) return set_error(NVFP4WS_ERR_INVALID_ARG, "fp8_lmhead_verify: verify is null");
   if (int e = check_verify_size(verify, "fp8_lmhead_verify")) return e;
   const int32_t B = verify->B, D = verify->D;
@@ -490,11 +514,13 @@ int fp8_lmhead_verify(const void* X, const uint8_t* q, const float* scales, int6
   if (D > 0 && !verify->drafts) return set_error(NVFP4WS_ERR_INVALID_ARG, "fp8_lmhead_verify: drafts is null");
   if (!verify->argmax || !verify->accept_len)
     return set_error(NVFP4WS_ERR_INVALID_ARG, "fp8_lmhead_verify: null output pointer");
-  if (int e = validate_fp8(X, q, scales, M, N, K, workspace, workspace_bytes, fp8_verify_workspace_bytes_int(M, N, K),
-                           "fp8_lmhead_verify"))
+  if (int e = validate_fp8(X, q, scales, M, N, K, workspace, workspace_bytes,
+                           fp8_lmhead_verify_workspace_bytes(M, N, K), "fp8_lmhead_verify"))
     return e;
   const VerifyRule v{verify->drafts, D > 0 ? verify->parents : nullptr, B, D, verify->argmax, verify->accept_len,
                      verify->accept_node, verify->max_logit};
+  if (path == NVFP4WS_FP8_E4M3_TERMS)
+    return launch_fp8q_verify(static_cast<const uint16_t*>(X), q, scales, M, N, K, v, workspace, (cudaStream_t)stream);
   return launch_fp8_verify(static_cast<const uint16_t*>(X), q, scales, M, N, K, v, workspace, (cudaStream_t)stream);
 }
 

@@ -37,6 +37,15 @@ int fp8_pass_init_int(void* state, const Fp8HostProblem* hp, int n, long long M,
                       void* workspace, size_t workspace_bytes);
 int fp8_pass_run_int(const void* state, cudaStream_t s);
 
+// The E4M3-term kernel (fp8q.cu): the codes straight into kind::f8f6f4, the activations as two
+// residual E4M3 terms with a power-of-two row scale. Same limits as fp8_supported.
+bool fp8q_supported(long long M, long long K);
+size_t fp8q_workspace_bytes_int(long long M, long long N, long long K, bool verify);
+int launch_fp8q_gemm(const uint16_t* X, const uint8_t* q, const float* scales, long long M, long long N, long long K,
+                     void* Y, int y_dtype, void* workspace, cudaStream_t s);
+int launch_fp8q_verify(const uint16_t* X, const uint8_t* q, const float* scales, long long M, long long N,
+                       long long K, const VerifyRule& v, void* workspace, cudaStream_t s);
+
 // fp32 W [N, K] -> E4M3 codes [N, K] and fp32 scales [ceil(N/128), ceil(K/128)].
 int launch_fp8_pack(const float* W, long long N, long long K, uint8_t* q, float* scales, cudaStream_t s);
 

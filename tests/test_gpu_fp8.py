@@ -21,10 +21,16 @@ import torch
 
 import synthetic as S
 from oracle import fp8 as P
+from oracle import gemm as G
 from oracle import verify as V
 
 pytestmark = pytest.mark.gpu
 TOL = 1e-5
+# The E4M3-term path: the activation terms are exact for these inputs up to E4M3's subnormal
+# step (2^-14 g per element); the bar leaves room for the FP8 tensor core's accumulation inside
+# a 128-wide block, whose precision is what this test measures.
+TOL_TERMS = 2e-4
+TOLS = {"f16": TOL, "terms": TOL_TERMS}
 
 
 @pytest.fixture(scope="module")
@@ -61,16 +67,17 @@ def test_fp8_pack_bit_exact(nv, N, K):
     packed(nv, W)
 
 
+@pytest.mark.parametrize("path", ["f16", "terms"])
 @pytest.mark.parametrize("M,N,K", [(1, 1000, 256), (17, 3000, 1024), (68, 777, 768), (128, 4096, 5120),
                                    (5, 130, 128), (17, 640, 5120), (17, 128, 16384), (40, 1000, 1024),
                                    (49, 333, 512)])
-def test_fp8_gemm(nv, M, N, K):
+def test_fp8_gemm(nv, M, N, K, path):
     W, x = S.block_varied_case(1000 + M + N, M, N, K)
     q, s, codes_ref, scales_ref = packed(nv, W)
-    Y = nv.fp8_gemm(to_dev_bf16(x), q, s)
+    Y = nv.fp8_gemm(to_dev_bf16(x), q, s, path=path)
     nv.check()
     y_ref = P.gemm_fp8_ref(x, codes_ref, scales_ref)
-    assert rowwise_err(Y.cpu().numpy(), y_ref) <= TOL
+    assert rowwise_err(Y.cpu().numpy(), y_ref) <= TOLS[path]
 
 
 @pytest.mark.parametrize("M,N,K", [(5, 700, 1024), (68, 300, 512)])
@@ -106,7 +113,8 @@ def test_fp8_gemm_bf16_and_repeat(nv):
     assert torch.equal(Yb, Y1.to(torch.bfloat16))
 
 
-def test_fp8_verify_chain(nv):
+@pytest.mark.parametrize("path", ["f16", "terms"])
+def test_fp8_verify_chain(nv, path):
     B, D, N, K = 1, 16, 20077, 2048
     W, x = S.random_case(1200, B * (D + 1), N, K, w_std=0.2)
     q, s, codes_ref, scales_ref = packed(nv, W)
@@ -114,7 +122,7 @@ def test_fp8_verify_chain(nv):
     t_ref = V.argmax_fast(y_ref)
     Lstar = np.array([9])
     drafts = S.drafts_with_prefix(t_ref, Lstar, D, N)
-    t, L, _, vmax = nv.fp8_verify(to_dev_bf16(x), q, s, torch.from_numpy(drafts).cuda())
+    t, L, _, vmax = nv.fp8_verify(to_dev_bf16(x), q, s, torch.from_numpy(drafts).cuda(), path=path)
     nv.check()
     t, L = t.cpu().numpy(), L.cpu().numpy()
     gap = V.top2_gap(y_ref)
@@ -122,7 +130,7 @@ def test_fp8_verify_chain(nv):
     assert rows.all()                                          # no near tie for this seed (oracle-checked)
     assert np.array_equal(t, t_ref)
     assert L.tolist() == V.accept_ref(t_ref, drafts, D).tolist() == [9]
-    np.testing.assert_allclose(vmax.cpu().numpy(), y_ref.max(axis=1), rtol=TOL, atol=0)
+    np.testing.assert_allclose(vmax.cpu().numpy(), y_ref.max(axis=1), rtol=TOLS[path], atol=0)
 
 
 def test_fp8_verify_tree(nv):
@@ -193,3 +201,42 @@ def test_fp8_pass_with_verify_tail(nv):
         assert rowwise_err(Y.cpu().numpy(), y_ref) <= TOL
     assert np.array_equal(t.cpu().numpy(), t_ref)              # no near tie for this seed (the chain test checks it)
     assert L.cpu().numpy().tolist() == [9]
+
+
+def test_fp8_terms_path_extreme_rows(nv):
+    """Rows with 100x outliers and rows of tiny values: the row's power-of-two scale follows the
+    row maximum, so the second term still carries each element's low bits."""
+    M, N, K = 17, 1000, 2048
+    W, x = S.block_varied_case(1600, M, N, K)
+    xf = G.bf16_bits_to_float64(x).copy()
+    rng = np.random.default_rng(1601)
+    xf[0, rng.integers(0, K, 20)] *= 100.0                      # outliers
+    xf[1] *= 2.0 ** -30                                          # a row of tiny values
+    xf[2] = 0.0                                                  # an all-zero row
+    x = S.f32_to_bf16_bits(xf.astype(np.float32))
+    q, s, codes_ref, scales_ref = packed(nv, W)
+    Y = nv.fp8_gemm(to_dev_bf16(x), q, s, path="terms").cpu().numpy()
+    nv.check()
+    y_ref = P.gemm_fp8_ref(x, codes_ref, scales_ref)
+    assert (Y[2] == 0).all()
+    rows = [m for m in range(M) if m != 2]
+    assert rowwise_err(Y[rows], y_ref[rows]) <= TOL_TERMS
+
+
+@pytest.mark.parametrize("path", ["f16", "terms"])
+def test_fp8_accumulation_keeps_small_products(nv, path):
+    """One 128-wide block whose sum needs ~19 significant bits: 448 * 1 plus 127 products of
+    2^-10. fp32 accumulation keeps every small product; an accumulator of ~14 bits would drop
+    them (an error of ~3e-4 of the result). This measures the tensor core's accumulation width."""
+    M, N, K = 1, 128, 128
+    W = np.ones((N, K), dtype=np.float32)
+    W[:, 0] = 448.0                                            # block scale exactly 1, codes 448 and 1
+    x = np.full((M, K), 2.0 ** -10, dtype=np.float32)
+    x[0, 0] = 1.0
+    xb = S.f32_to_bf16_bits(x)
+    q, s, codes_ref, scales_ref = packed(nv, W)
+    assert float(scales_ref[0, 0]) == 1.0
+    Y = nv.fp8_gemm(to_dev_bf16(xb), q, s, path=path).cpu().numpy()
+    nv.check()
+    y_ref = 448.0 + 127 * 2.0 ** -10
+    assert np.abs(Y.astype(np.float64) - y_ref).max() <= 1e-6 * y_ref
