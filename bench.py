@@ -395,8 +395,9 @@ def run_extras(nv, torch, dev, stack, lm, peak: float, reps: int) -> dict:
     """The measurement configurations beside the full pass, each a stream of single library
     calls timed as a CUDA graph, rotating through distinct weight copies so every call
     reads its weights from HBM:
-      single_m1   one GEMM at M=1 (nvfp4_gemm_skinny, the GEMV path) at each 27B layer
-                  shape, over the stack's 64 copies of that shape;
+      single_m1   one GEMM at M=1 (nvfp4_gemm_skinny, default path: the block-scaled tensor
+                  cores) at each 27B layer shape, over the stack's 64 copies of that shape;
+      single_m1_gemv  the same on the CUDA-core GEMV (register-prefetch variant);
       verify      the standalone fused verify (lmhead_verify_argmax_accept) at N=248,320
                   and at the 65,536-row slice (four disjoint slices in turn), M=17 and 68;
       m_sweep     one GEMM (nvfp4_gemm_skinny, default path) on gate+up 5120->34816 at
@@ -408,17 +409,19 @@ def run_extras(nv, torch, dev, stack, lm, peak: float, reps: int) -> dict:
     g.manual_seed(4242)
     by_shape = {n: [(q, sf, ts) for (nm, _, _, q, sf, ts) in stack if nm == n] for n in S.LAYER_ORDER}
 
-    single = {}
-    for name in S.LAYER_ORDER:
-        K, N = S.LAYER_SHAPES[name]
-        X = torch.randn(1, K, generator=g, device=dev).to(torch.bfloat16)
-        Y = torch.empty(1, N, device=dev)
-        ws = torch.zeros(max(16, nv.gemm_workspace_bytes(1, N, K)), dtype=torch.uint8, device=dev)
-        calls = [lambda q=q, sf=sf, ts=ts: nv.gemm(X, q, sf, ts, out=Y, workspace=ws) for (q, sf, ts) in by_shape[name]]
-        wb = weight_bytes(N, K)
-        single[name] = _entry(time_calls(torch, calls, reps), wb, wb + K * 2 + N * 4, peak, N=N, K=K,
-                              copies=len(calls), path="gemv")
-    out["single_m1"] = single
+    for key, path in (("single_m1", "auto"), ("single_m1_gemv", "gemv_regs")):
+        single = {}
+        for name in S.LAYER_ORDER:
+            K, N = S.LAYER_SHAPES[name]
+            X = torch.randn(1, K, generator=g, device=dev).to(torch.bfloat16)
+            Y = torch.empty(1, N, device=dev)
+            ws = torch.zeros(max(16, nv.gemm_workspace_bytes(1, N, K)), dtype=torch.uint8, device=dev)
+            calls = [lambda q=q, sf=sf, ts=ts: nv.gemm(X, q, sf, ts, out=Y, workspace=ws, path=path)
+                     for (q, sf, ts) in by_shape[name]]
+            wb = weight_bytes(N, K)
+            single[name] = _entry(time_calls(torch, calls, reps), wb, wb + K * 2 + N * 4, peak, N=N, K=K,
+                                  copies=len(calls), path=path)
+        out[key] = single
 
     ql, sfl, tsl = lm
     verify = {}

@@ -75,7 +75,11 @@ enum { KPATH_GEMV = 1, KPATH_MXF4 = 2, KPATH_GEMV_REGS = 3, KPATH_MMA_F16 = 4, K
 static int resolve_path(int path, int64_t M, int64_t K) {
   switch (path) {
     case NVFP4WS_PATH_AUTO:
-      if (M >= mma_min_m() && mxf4_supported(M, K)) return KPATH_MXF4;
+      // The block-scaled tensor-core kernel whenever it applies, M = 1 included: on B200 a
+      // CUDA-core GEMV spends ~3.4 instructions per weight element on dequantisation and
+      // products, more than an SM can issue at HBM rate (measured: 1.5 of 4 per cycle, 0.3-0.5
+      // of HBM), while kind::mxf4nvf4 takes the packed weights with no per-element work.
+      if (mxf4_supported(M, K)) return KPATH_MXF4;
       if (M >= mma_min_m() && mma_supported(M, K)) return KPATH_MMA_F16;
       return KPATH_GEMV;
     case NVFP4WS_PATH_GEMV: return KPATH_GEMV;

@@ -394,282 +394,6 @@ __global__ void __launch_bounds__(544, 1) gemv_staged_kernel(GemvArgs a, int sta
 }
 
 // ---------------------------------------------------------------------------
-// One activation row (M = 1, K % 256 == 0): row teams.
-//
-// The kernels above spread one weight row over the whole CTA, so every row ends in a
-// CTA-wide reduction and barrier. Here a team of P warps owns whole rows: P = ceil(K / 4096),
-// so each lane holds at most four 32-element chunks of x (64 registers) for the whole kernel:
-// P = 2 at K = 5120, 5 at K = 17408. Lane l of team warp p takes the chunks
-// c = 32 p + l + 32 P j (j < J, c < K/32). A row needs one warp-shuffle reduction per warp and
-// a sum of P partials in warp order. Each team works on kRowRPT rows of a stage together, so
-// a warp has independent conversions and FMAs in flight while others wait on their inputs.
-// A producer warp stages R = (NW / P) * kRowRPT whole rows per stage (NW = 10 consumer warps,
-// or the largest multiple of P below it) with two bulk copies (nibbles, scales) into a ring
-// of up to 14 stages (about 200 KB in flight per SM at the 27B shapes). The kernel is a
-// programmatic dependent: its weight loads start while the previous kernel of the stream
-// drains, and X is read only after that kernel has finished.
-// ---------------------------------------------------------------------------
-
-constexpr int kRowMaxJ = 4;                     // chunks per lane: x takes 16 J registers
-constexpr int kRowWarpsMax = 10;                // consumer warps
-constexpr int kRowMaxStages = 14;
-constexpr int kRowRPT = 2;                      // rows per team per stage, worked on together
-
-struct RowPlan {
-  int P, J, NW, R, stages, grid;
-  unsigned int stage_bytes;
-  long long ngroups;
-  size_t smem;
-};
-
-// bar.red.or: a barrier whose threads all leave with the OR of their predicates, so that a
-// give-up seen by one warp of a team ends the loop for every warp of it.
-__device__ __forceinline__ bool named_bar_or(int id, int n, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{ .reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, %2, %3, p;\n\t"
-      "selp.u32 %0, 1, 0, q; }"
-      : "=r"(r)
-      : "r"((uint32_t)pred), "r"(id), "r"(n)
-      : "memory");
-  return r != 0;
-}
-
-template <int J>
-__global__ void __launch_bounds__((kRowWarpsMax + 1) * 32, 1) gemv_row_kernel(GemvArgs a, RowPlan pl) {
-  asm volatile("griddepcontrol.launch_dependents;");
-  extern __shared__ __align__(128) uint8_t smem[];
-  const int S = pl.stages, P = pl.P, NW = pl.NW, R = pl.R, T = NW / P;   // R = T * kRowRPT
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int C = (int)(a.K >> 5);
-  const long long rowq = a.K >> 1, rows = a.K >> 4;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)S * pl.stage_bytes);
-  volatile int* s_abort = reinterpret_cast<volatile int*>(bars + 2 * S);
-  float* s_red = reinterpret_cast<float*>(bars + 2 * S + 2);          // [2][kRowRPT][kRowWarpsMax]
-  float* s_bv = s_red + 2 * kRowRPT * kRowWarpsMax;                    // [kRowWarpsMax] team bests
-  int* s_bi = reinterpret_cast<int*>(s_bv + kRowWarpsMax);
-  auto bar_full = [&](int s) { return smem_u32(bars + s); };
-  auto bar_empty = [&](int s) { return smem_u32(bars + S + s); };
-  const long long G = gridDim.x;
-  const long long g0 = (long long)blockIdx.x * pl.ngroups / G, g1 = ((long long)blockIdx.x + 1) * pl.ngroups / G;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) { mbar_init(bar_full(s), 1); mbar_init(bar_empty(s), NW); }
-    *s_abort = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  __syncthreads();
-
-  if (warp == NW) {
-    // ---------------- producer: R whole rows per stage, two bulk copies
-    if (lane == 0) {
-      const uint64_t pol = policy_evict_first();
-      int i = 0;
-      for (long long g = g0; g < g1; ++g, ++i) {
-        const int s = i % S;
-        if (!mbar_wait(bar_empty(s), ((uint32_t)(i / S) & 1u) ^ 1u, s_abort, a.err)) break;
-        const long long n0 = g * R;
-        const long long nr = (a.N - n0 < R) ? (a.N - n0) : R;
-        uint8_t* st = smem + (size_t)s * pl.stage_bytes;
-        mbar_arrive_expect_tx(bar_full(s), (uint32_t)(nr * rowq + nr * rows));
-        bulk_load(smem_u32(st), a.q + n0 * rowq, (uint32_t)(nr * rowq), bar_full(s), pol);
-        bulk_load(smem_u32(st + R * rowq), a.sf + n0 * rows, (uint32_t)(nr * rows), bar_full(s), pol);
-      }
-      if (*s_abort) {                            // drain the copies still in flight (bounded)
-        for (int k = (i > S ? i - S : 0); k < i; ++k) {
-          const unsigned long long t0 = globaltimer();
-          while (!mbar_try_wait(bar_full(k % S), (uint32_t)(k / S) & 1u) && globaltimer() - t0 < kWaitLimitNs) {}
-        }
-      }
-    }
-    return;    // the producer takes no part in the consumers' named barriers
-  }
-
-  // ---------------- consumers
-  asm volatile("griddepcontrol.wait;" ::: "memory");   // X may come from the previous kernel
-  const int team = warp / P, p = warp - team * P;
-  uint32_t xr[J][16];
-  float lmax = 0.f;
-#pragma unroll
-  for (int j = 0; j < J; ++j) {
-    const int c = 32 * p + lane + 32 * P * j;
-    if (c < C) {
-      const uint4* src = reinterpret_cast<const uint4*>(a.X + (long long)c * 32);
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        const uint4 b = src[v];
-        xr[j][4 * v + 0] = b.x; xr[j][4 * v + 1] = b.y; xr[j][4 * v + 2] = b.z; xr[j][4 * v + 3] = b.w;
-      }
-    } else {
-#pragma unroll
-      for (int v = 0; v < 16; ++v) xr[j][v] = 0u;
-    }
-#pragma unroll
-    for (int v = 0; v < 16; ++v) lmax = fmaxf(lmax, bf16x2_absmax(xr[j][v]));
-  }
-  // the row's shift: every team covers all of K, so the amax over one team's warps is the row's
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
-  if (lane == 0) s_red[warp] = lmax;
-  named_bar(1, NW * 32);
-  float amax = 0.f;
-  for (int w = 0; w < P; ++w) amax = fmaxf(amax, s_red[team * P + w]);
-  const int xe = row_shift_of_amax(amax);
-  named_bar(1, NW * 32);                         // s_red is reused below
-#pragma unroll
-  for (int j = 0; j < J; ++j)
-#pragma unroll
-    for (int v = 0; v < 16; ++v) xr[j][v] = bf16x2_to_f16x2_shifted(xr[j][v], xe);
-
-  const float ts = *a.ts;
-  float bestv = -INFINITY;
-  int besti = INT_MAX;
-  int i = 0;
-  for (long long g = g0; g < g1; ++g, ++i) {
-    const int s = i % S;
-    bool ok = mbar_wait(bar_full(s), (uint32_t)(i / S) & 1u, s_abort, a.err);
-    if (P > 1) ok = !named_bar_or(2 + team, P * 32, !ok);
-    if (!ok) break;
-    const uint8_t* st = smem + (size_t)s * pl.stage_bytes;
-    // the team's kRowRPT rows of this stage (row rr * T + team): independent work in flight
-    float acc[kRowRPT];
-#pragma unroll
-    for (int rr = 0; rr < kRowRPT; ++rr) {
-      const int r = rr * T + team;
-      acc[rr] = 0.f;
-      if (g * R + r < a.N) {
-        const uint8_t* qrow = st + (size_t)r * rowq;
-        const uint8_t* srow = st + (size_t)R * rowq + (size_t)r * rows;
-#pragma unroll
-        for (int j = 0; j < J; ++j) {
-          const int c = 32 * p + lane + 32 * P * j;
-          if (c < C) {
-            const uint4 w4 = *reinterpret_cast<const uint4*>(qrow + (long long)c * 16);
-            const uint32_t s2 = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(srow + (long long)c * 2));
-            const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
-            float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) dot2_f16_f32(p0, p1, e2m1x2_to_f16x2(w[e >> 2] >> (8 * (e & 3))), xr[j][e]);
-#pragma unroll
-            for (int e = 8; e < 16; ++e) dot2_f16_f32(p2, p3, e2m1x2_to_f16x2(w[e >> 2] >> (8 * (e & 3))), xr[j][e]);
-            acc[rr] = fmaf(f16lo_to_f32(s2), p0 + p1, acc[rr]);
-            acc[rr] = fmaf(f16hi_to_f32(s2), p2 + p3, acc[rr]);
-          }
-        }
-      }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(bar_empty(s));   // this warp is done reading the stage
-#pragma unroll
-    for (int rr = 0; rr < kRowRPT; ++rr)
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc[rr] += __shfl_xor_sync(0xffffffffu, acc[rr], o);
-    if (P > 1) {                                 // the team's partials in warp order
-      float* red = s_red + (i & 1) * kRowRPT * kRowWarpsMax;
-      if (lane == 0) {
-#pragma unroll
-        for (int rr = 0; rr < kRowRPT; ++rr) red[rr * kRowWarpsMax + warp] = acc[rr];
-      }
-      named_bar(2 + team, P * 32);
-      if (p == 0) {
-#pragma unroll
-        for (int rr = 0; rr < kRowRPT; ++rr) {
-          acc[rr] = 0.f;
-          for (int w = 0; w < P; ++w) acc[rr] += red[rr * kRowWarpsMax + team * P + w];
-        }
-      }
-    }
-    if (p == 0 && lane == 0) {
-#pragma unroll
-      for (int rr = 0; rr < kRowRPT; ++rr) {
-        const long long n = g * R + rr * T + team;
-        if (n < a.N) {
-          const float y = mul_pow2(acc[rr] * ts, xe);
-          if (a.verify) {
-            if (argmax_better(y, (int)n, bestv, besti)) { bestv = y; besti = (int)n; }
-          } else if (a.y_bf16) {
-            reinterpret_cast<uint16_t*>(a.Y)[n] = f32_to_bf16_rn(y);
-          } else {
-            reinterpret_cast<float*>(a.Y)[n] = y;
-          }
-        }
-      }
-    }
-  }
-  if (a.verify) {                                // the CTA's best row: teams in order
-    if (p == 0 && lane == 0) { s_bv[team] = bestv; s_bi[team] = besti; }
-    named_bar(1, NW * 32);
-    if (threadIdx.x == 0) {
-      float bv = s_bv[0];
-      int bi = s_bi[0];
-      for (int t = 1; t < T; ++t)
-        if (argmax_better(s_bv[t], s_bi[t], bv, bi)) { bv = s_bv[t]; bi = s_bi[t]; }
-      a.part_val[blockIdx.x] = bv;
-      a.part_idx[blockIdx.x] = bi;
-    }
-  }
-}
-
-// The row-team plan for one activation row, or P = 0 when the shape does not suit it.
-static RowPlan row_plan(long long M, long long N, long long K) {
-  RowPlan p{};
-  if (M != 1 || K % 256 != 0 || K < 256) return p;
-  const int C = (int)(K / 32);
-  const int P = (C + 32 * kRowMaxJ - 1) / (32 * kRowMaxJ);
-  if (P > kRowWarpsMax / 2) return p;            // at least two rows per stage
-  p.P = P;
-  p.J = (C + 32 * P - 1) / (32 * P);
-  p.NW = P * (kRowWarpsMax / P);
-  p.R = (p.NW / P) * kRowRPT;
-  p.stage_bytes = (unsigned int)(((long long)p.R * (K / 2 + K / 16) + 127) / 128 * 128);
-  const size_t tail = 2 * kRowMaxStages * 8 + 16 + (2 * kRowRPT + 2) * kRowWarpsMax * 4 + 128;
-  p.stages = (int)std::min<size_t>(kRowMaxStages, (size_t)(220 * 1024 - tail) / p.stage_bytes);
-  if (p.stages < 2) { p.P = 0; return p; }
-  p.smem = (size_t)p.stages * p.stage_bytes + tail;
-  p.ngroups = (N + p.R - 1) / p.R;
-  p.grid = (int)std::max<long long>(1, std::min<long long>(p.ngroups, std::max(1, device_sm_count())));
-  return p;
-}
-
-template <int J>
-static int launch_row_j(const GemvArgs& a, const RowPlan& p, cudaStream_t s) {
-  static std::atomic<bool> attr[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr[dev].load(std::memory_order_acquire)) {
-    if (cudaFuncSetAttribute(gemv_row_kernel<J>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
-        cudaSuccess)
-      return check_launch("cudaFuncSetAttribute(gemv_row_kernel)");
-    attr[dev].store(true, std::memory_order_release);
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)p.grid);
-  cfg.blockDim = dim3((unsigned)((p.NW + 1) * 32));
-  cfg.dynamicSmemBytes = p.smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr1[1];
-  attr1[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr1[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr1;
-  cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_row_kernel<J>, a, p);
-  if (e != cudaSuccess) return set_error(NVFP4WS_ERR_CUDA, "gemv_row_kernel launch: %s", cudaGetErrorString(e));
-  return check_launch("gemv_row_kernel");
-}
-
-static int launch_row(const GemvArgs& a, const RowPlan& p, cudaStream_t s) {
-  static_assert(kRowMaxJ == 4, "one instance per J");
-  switch (p.J) {
-    case 1: return launch_row_j<1>(a, p, s);
-    case 2: return launch_row_j<2>(a, p, s);
-    case 3: return launch_row_j<3>(a, p, s);
-    default: return launch_row_j<4>(a, p, s);
-  }
-}
-
-// ---------------------------------------------------------------------------
 // Host side: pick (MT, CPT, R, T) and the grid
 // ---------------------------------------------------------------------------
 
@@ -708,15 +432,6 @@ static int launch_staged(const GemvArgs& a, const GemvPlan& p, cudaStream_t s) {
 
 GemvPlan gemv_plan(long long M, long long N, long long K, bool regs_only) {
   GemvPlan p{};
-  if (!regs_only) {                              // one activation row: the row-team kernel
-    const RowPlan r = row_plan(M, N, K);
-    if (r.P > 0) {
-      p.row = 1;
-      p.mt = 1;
-      p.grid = r.grid;
-      return p;
-    }
-  }
   const int C = (int)(K / 32);
   p.cpt = C <= 512 ? 1 : (C <= 1024 ? 2 : 4);
   int per = (C + p.cpt - 1) / p.cpt;
@@ -753,13 +468,6 @@ bool gemv_supported(long long K) { return K % 32 == 0 && K / 32 <= 2048; }
 
 int launch_gemv(const GemvArgs& base, bool verify, bool regs_only, cudaStream_t s) {
   const GemvPlan p = gemv_plan(base.M, base.N, base.K, regs_only);
-  if (p.row) {
-    GemvArgs a = base;
-    a.m0 = 0;
-    a.verify = verify ? 1 : 0;
-    a.err = device_error_word();
-    return launch_row(a, row_plan(base.M, base.N, base.K), s);
-  }
   for (long long m0 = 0; m0 < base.M;) {
     GemvArgs a = base;
     a.m0 = (int)m0;

@@ -24,7 +24,6 @@ struct GemvArgs {
 struct GemvPlan {
   int mt, cpt, rows, threads, grid;
   int staged;               // 1: bulk-copy-staged kernel (threads includes the producer warp)
-  int row;                  // 1: the row-team kernel for one activation row (grid is its grid)
   int stages;
   unsigned int stage_bytes;
   size_t smem;

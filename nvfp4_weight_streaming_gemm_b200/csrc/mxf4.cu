@@ -22,7 +22,8 @@
 // and scale taken from the exact quotients, rounded once (the weights' rule).
 //
 // Kernels.
-//   x_prep_kernel   one CTA per (activation row, problem): the T-term decomposition,
+//   x_prep_kernel   one CTA per (activation row, problem; a single GEMM splits each row over
+//                   several CTAs along K): the T-term decomposition,
 //                   written as per-K-chunk images that are byte-for-byte the shared
 //                   memory operand (128-byte-swizzled code rows, then 16 scale bytes
 //                   per row). The GEMM fetches each with ONE contiguous bulk copy:
@@ -284,16 +285,21 @@ __device__ __forceinline__ void quantise_block(float (&r)[16], int b, int m, flo
   }
 }
 
+// slices: CTAs per activation row. Each takes the row's amax over all of K, then writes the
+// terms of its share of the row's blocks. One slice serves a pass (thousands of rows run at
+// once); a single GEMM splits each row so that the prep's latency, which the GEMM waits for,
+// does not grow with K.
 template <int T>
 __global__ void __launch_bounds__(kPrepThreads, 6) x_prep_kernel(const __grid_constant__ Problem single,
-                                                                  const Problem* probs, const Geom g) {
+                                                                  const Problem* probs, const Geom g, int slices) {
   asm volatile("griddepcontrol.launch_dependents;");
   // X may come from the previous kernel of the stream, and the previous GEMM may still
   // read this workspace: nothing is read or written before that kernel has finished.
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const int m = blockIdx.x % g.M;
-  const Problem* pr = probs ? probs + blockIdx.x / g.M : &single;
+  const int row_cta = blockIdx.x / slices, sl = blockIdx.x - row_cta * slices;
+  const int m = row_cta % g.M;
+  const Problem* pr = probs ? probs + row_cta / g.M : &single;
   const int nblk = pr->K / 16;
   const uint16_t* X = pr->X + (long long)m * pr->K;
   uint8_t* img = pr->ximg;
@@ -318,10 +324,11 @@ __global__ void __launch_bounds__(kPrepThreads, 6) x_prep_kernel(const __grid_co
 #pragma unroll
     for (int term = 0; term < T; ++term, gt *= 0.25f) {
       inv6[term] = gt > 0.f ? 1.0f / (6.0f * gt) : 0.f;
-      if (t == 0) pr->xg[m * T + term] = gt;
+      if (t == 0 && sl == 0) pr->xg[m * T + term] = gt;
     }
   }
-  for (int b = t; b < nblk; b += kPrepThreads) {
+  const int b1 = (int)((long long)(sl + 1) * nblk / slices);
+  for (int b = (int)((long long)sl * nblk / slices) + t; b < b1; b += kPrepThreads) {
     float r[16];
     load_block16(X, b, r);
     quantise_block<T>(r, b, m, g0, inv6, g, img);
@@ -985,8 +992,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       named_bar(1, 128);
       if (et == 0 && seg <= 2) MX_CTA(10 + 4 * (seg - 1));
       if (*s_last) {
-        // Sum the contributors' partials in CTA order (deterministic), two contributors'
-        // loads in flight at a time, 16 tokens per pass.
+        // Sum the contributors' partials in CTA order (deterministic), 16 tokens per pass. The
+        // loads of four contributors are issued together: a tile split across many CTAs (the
+        // down projection's 40 tiles over 148 CTAs) then costs a quarter of the dependent L2
+        // round trips, which set the tail of a single GEMM.
         for (int tj = 0; tj < g.tpu; ++tj) {
           const int tile = group * g.tpu + tj;
           const long long n = (long long)tile * kTileRows + rowl;
@@ -994,25 +1003,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             float acc[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) acc[j] = 0.f;
-            for (int cc = c0; cc <= c1; cc += 2) {
-              const bool two = cc + 1 <= c1;
-              const int sl0 = (w0 + unit_begin((uint32_t)cc, Uw, G) >= tile_u0) ? 2 * cc : 2 * cc + 1;
-              const int sl1 = two ? ((w0 + unit_begin((uint32_t)cc + 1u, Uw, G) >= tile_u0) ? 2 * cc + 2 : 2 * cc + 3) : sl0;
-              const float4* src0 =
-                  reinterpret_cast<const float4*>(wave_part + ((long long)(sl0 * g.tpu + tj) * kTileRows + rowl) * Mp + mc);
-              const float4* src1 =
-                  reinterpret_cast<const float4*>(wave_part + ((long long)(sl1 * g.tpu + tj) * kTileRows + rowl) * Mp + mc);
-              float4 v0[4], v1[4];
+            for (int cc = c0; cc <= c1; cc += 4) {
+              float4 v[4][4];
 #pragma unroll
-              for (int b = 0; b < 4; ++b) {
-                v0[b] = (mc + 4 * b < Mp) ? __ldcg(src0 + b) : make_float4(0.f, 0.f, 0.f, 0.f);
-                v1[b] = (two && mc + 4 * b < Mp) ? __ldcg(src1 + b) : make_float4(0.f, 0.f, 0.f, 0.f);
+              for (int k = 0; k < 4; ++k) {
+                const int cx = cc + k;
+                const bool on = cx <= c1;
+                const int sl = on ? ((w0 + unit_begin((uint32_t)cx, Uw, G) >= tile_u0) ? 2 * cx : 2 * cx + 1) : 0;
+                const float4* src =
+                    reinterpret_cast<const float4*>(wave_part + ((long long)(sl * g.tpu + tj) * kTileRows + rowl) * Mp + mc);
+#pragma unroll
+                for (int b = 0; b < 4; ++b)
+                  v[k][b] = (on && mc + 4 * b < Mp) ? __ldcg(src + b) : make_float4(0.f, 0.f, 0.f, 0.f);
               }
 #pragma unroll
-              for (int b = 0; b < 4; ++b) {
-                acc[4 * b] += v0[b].x; acc[4 * b + 1] += v0[b].y; acc[4 * b + 2] += v0[b].z; acc[4 * b + 3] += v0[b].w;
-                if (two) {
-                  acc[4 * b] += v1[b].x; acc[4 * b + 1] += v1[b].y; acc[4 * b + 2] += v1[b].z; acc[4 * b + 3] += v1[b].w;
+              for (int k = 0; k < 4; ++k) {
+                if (cc + k <= c1) {
+#pragma unroll
+                  for (int b = 0; b < 4; ++b) {
+                    acc[4 * b] += v[k][b].x; acc[4 * b + 1] += v[k][b].y;
+                    acc[4 * b + 2] += v[k][b].z; acc[4 * b + 3] += v[k][b].w;
+                  }
                 }
               }
             }
@@ -1293,6 +1304,11 @@ struct PassTables {           // device wave tables of a pass (all null for one 
   int nwave;
 };
 
+// CTAs per activation row in the prep of one GEMM: about 2048 elements each.
+static int prep_slices(int nprob, long long K) {
+  return nprob == 1 ? (int)std::max<long long>(1, std::min<long long>(16, K / 2048)) : 1;
+}
+
 static int launch_pass(const Problem& single, const Problem* probs_dev, const PassTables& tb, int nprob,
                        const MxPlan& pl, int grid, unsigned long long units, size_t off_part, long long max_k,
                        char* ws, cudaStream_t s) {
@@ -1303,8 +1319,9 @@ static int launch_pass(const Problem& single, const Problem* probs_dev, const Pa
   // 1) activation decomposition (programmatic dependent launch: it may start while the
   //    previous kernel of the stream finishes, and waits for it before any access)
   {
+    const int slices = prep_slices(nprob, max_k);
     cudaLaunchConfig_t pc = {};
-    pc.gridDim = dim3((unsigned)(pl.g.M * nprob));
+    pc.gridDim = dim3((unsigned)(pl.g.M * nprob * slices));
     pc.blockDim = dim3(kPrepThreads);
     pc.stream = s;
     cudaLaunchAttribute pa[1];
@@ -1313,8 +1330,8 @@ static int launch_pass(const Problem& single, const Problem* probs_dev, const Pa
     pc.attrs = pa;
     pc.numAttrs = 1;
     const Geom g = pl.g;
-    cudaError_t pe = g.T == 1 ? cudaLaunchKernelEx(&pc, x_prep_kernel<1>, single, probs_dev, g)
-                              : cudaLaunchKernelEx(&pc, x_prep_kernel<kMxf4Terms>, single, probs_dev, g);
+    cudaError_t pe = g.T == 1 ? cudaLaunchKernelEx(&pc, x_prep_kernel<1>, single, probs_dev, g, slices)
+                              : cudaLaunchKernelEx(&pc, x_prep_kernel<kMxf4Terms>, single, probs_dev, g, slices);
     if (pe != cudaSuccess) return set_error(NVFP4WS_ERR_CUDA, "x_prep_kernel launch: %s", cudaGetErrorString(pe));
     if (int e = check_launch("x_prep_kernel")) return e;
   }

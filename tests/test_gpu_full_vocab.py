@@ -89,7 +89,7 @@ def check_verify(orc, x, M, Dd, drafts, t, L, vmax):
 
 @pytest.mark.parametrize("M,B,Dd", CASES)
 def test_verify_full_vocab_exact(nv, head, M, B, Dd):
-    """lmhead_verify_argmax_accept on the whole head (M=1: the GEMV; 17, 68: block-scaled)."""
+    """lmhead_verify_argmax_accept on the whole head (the default path: block-scaled)."""
     x, orc, (q, sf, ts) = head
     drafts, _ = drafts_for(orc, M, B, Dd)
     t, L, vmax = nv.verify(to_dev_bf16(x[:M]), q, sf, ts, torch.from_numpy(drafts).cuda())
@@ -98,14 +98,14 @@ def test_verify_full_vocab_exact(nv, head, M, B, Dd):
     assert frac > 0.9
 
 
-@pytest.mark.parametrize("path", ["mma_f16", "gemv"])
-def test_verify_full_vocab_other_paths(nv, head, path):
-    """The same head at M = 17 on the f16 tensor-core kernel and on the GEMV."""
+@pytest.mark.parametrize("path,M,B,Dd", [("mma_f16", 17, 1, D), ("gemv", 17, 1, D), ("gemv", 1, 1, 0)])
+def test_verify_full_vocab_other_paths(nv, head, path, M, B, Dd):
+    """The same head on the f16 tensor-core kernel and on the CUDA-core GEMV."""
     x, orc, (q, sf, ts) = head
-    drafts, _ = drafts_for(orc, 17, 1, D)
-    t, L, vmax = nv.verify(to_dev_bf16(x[:17]), q, sf, ts, torch.from_numpy(drafts).cuda(), path=path)
+    drafts, _ = drafts_for(orc, M, B, Dd)
+    t, L, vmax = nv.verify(to_dev_bf16(x[:M]), q, sf, ts, torch.from_numpy(drafts).cuda(), path=path)
     nv.check()
-    check_verify(orc, x, 17, D, drafts, t.cpu().numpy(), L.cpu().numpy(), vmax.cpu().numpy())
+    check_verify(orc, x, M, Dd, drafts, t.cpu().numpy(), L.cpu().numpy(), vmax.cpu().numpy())
 
 
 @pytest.fixture(scope="module")

@@ -206,12 +206,16 @@ def test_verify_activation_range(nv):
         run_verify(nv, W, x, np.array([0]), 0, path="mma_f16")
 
 
+@pytest.mark.parametrize("path", ["auto", "gemv", "gemv_regs"])
 @pytest.mark.parametrize("name", S.LAYER_ORDER)
-def test_gemm_layer_shapes_m1(nv, name):
-    """The M=1 decode configuration at the 27B layer shapes (the launch the bench times)."""
+def test_gemm_layer_shapes_m1(nv, name, path):
+    """The M=1 decode configuration at the 27B layer shapes, on the default path (the
+    block-scaled tensor cores) and on both CUDA-core GEMVs."""
     W, x = S.layer(name, M=1)
-    Y, y_ref = run_gemm(nv, W, x)
-    assert_rowwise(Y.cpu().numpy(), y_ref)
+    Y, y_ref = run_gemm(nv, W, x, path=path)
+    worst = assert_rowwise(Y.cpu().numpy(), y_ref)
+    if path == "auto":
+        assert worst <= TERMS_TOL, f"{worst:.2e} of max|y|"
 
 
 # ------------------------------------------------------------------ verify
