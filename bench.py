@@ -458,8 +458,9 @@ def run_fp8_extras(nv, torch, dev, peak: float, layers: int, reps: int) -> dict:
     """FP8 weights (E4M3, one fp32 scale per 128 x 128 block) in the pages' precision map: the
     64 qkv projections (5120->10240) and the 248,320-row output head, packed on the GPU from
     seeded N(0, 0.02) weights (4.63 GB, 37 times L2).
-      pass_M{17,68}     one FP8 weight pass over the 64 qkv GEMMs with the head as its verify
-                        tail (fp8_pass_run), timed as a CUDA graph;
+      pass_M{17,68}*    one FP8 weight pass over the 64 qkv GEMMs with the head as its verify
+                        tail (fp8_pass_run), timed as a CUDA graph, on the f16 kernel and
+                        (suffix _terms) on the E4M3-term kernel;
       head_verify_M*    the head's fused verify alone (fp8_lmhead_verify_path), on the f16
                         kernel and (suffix _terms) on the E4M3-term kernel;
       head_gemm_M1*     the head as a plain M=1 GEMM (fp8_gemm_skinny_path), both kernels.
@@ -493,12 +494,14 @@ def run_fp8_extras(nv, torch, dev, peak: float, layers: int, reps: int) -> dict:
         probs = [(torch.randn(M, K, generator=gx, device=dev).to(torch.bfloat16), q, sc,
                   torch.empty((M, N), dtype=torch.bfloat16, device=dev)) for (q, sc) in qkv]
         probs.append((Xh, qh, sh, None))
-        p8 = nv.Fp8Pass(probs, M, verify=(drafts, t, L, None))
         wb = qkv_bytes + head_bytes
         alg = wb + M * (K * 2 * layers + S.LMHEAD_K * 2) + M * N * 2 * layers
-        out[f"pass_M{M}"] = _entry(time_calls(torch, [p8.run], max(3, reps // 2)), wb, alg, peak, M=M,
-                                   problems=len(probs))
-        del p8, probs
+        for path, tag in (("f16", ""), ("terms", "_terms")):
+            p8 = nv.Fp8Pass(probs, M, verify=(drafts, t, L, None), path=path)
+            out[f"pass_M{M}{tag}"] = _entry(time_calls(torch, [p8.run], max(3, reps // 2)), wb, alg, peak, M=M,
+                                            problems=len(probs), kernel=path)
+            del p8
+        del probs
         ws = torch.zeros(int(nv.lib().fp8_lmhead_verify_workspace_bytes(M, S.VOCAB, S.LMHEAD_K)), dtype=torch.uint8,
                          device=dev)
         for path, tag in (("f16", ""), ("terms", "_terms")):
@@ -947,7 +950,7 @@ def run_mixed(args):
         probs8 = [(torch.randn(M, K, generator=gx, device=dev).to(torch.bfloat16), q, sc,
                    torch.empty((M, N), dtype=torch.bfloat16, device=dev)) for (K, N, q, sc) in f8]
         probs8.append((torch.randn(M, S.LMHEAD_K, generator=gx, device=dev).to(torch.bfloat16), qh, sh, None))
-        p8 = nv.Fp8Pass(probs8, M, verify=(drafts, t, L, None))
+        p8 = nv.Fp8Pass(probs8, M, verify=(drafts, t, L, None), path=args.fp8_path)
         s = torch.cuda.Stream()
         s.wait_stream(st)
         with torch.cuda.stream(s):
@@ -975,7 +978,8 @@ def run_mixed(args):
         gbs = wbytes / (ms * 1e-3) / 1e9
         print(json.dumps({
             "metric": "27B step with the pages' precision map (NVFP4 MLP, FP8 qkv and lm_head verify)", "M": M,
-            "layers": args.layers, "ms_per_step": ms, "ms_min": float(per.min()), "weight_bytes": wbytes,
+            "layers": args.layers, "fp8_kernel": args.fp8_path, "ms_per_step": ms, "ms_min": float(per.min()),
+            "weight_bytes": wbytes,
             "weight_gbs": gbs, "hbm_frac": gbs / hbm, "hbm_peak_kind": hbm_kind, "y_dtype": "bf16",
             "steps": args.steps, "warmup": args.warmup}), flush=True)
         del graph, p4, p8, probs8

@@ -484,6 +484,15 @@ int fp8_pass_init(nvfp4_pass* pass, const fp8_gemm_problem* problems, int32_t co
                   const nvfp4_verify_spec* verify, void* workspace, size_t workspace_bytes);
 int fp8_pass_run(const nvfp4_pass* pass, nvfp4ws_stream_t stream);
 
+/* As fp8_pass_workspace_bytes / fp8_pass_init, with the FP8 kernel chosen by `path`
+ * (NVFP4WS_FP8_DEQUANT_F16, the default of the calls above, or NVFP4WS_FP8_E4M3_TERMS with the
+ * arithmetic fp8_gemm_skinny_path describes for it). Pass the same path to both; fp8_pass_run
+ * runs whichever kernel the pass was initialised with. */
+size_t fp8_pass_workspace_bytes_path(const fp8_gemm_problem* problems, int32_t count, int64_t M, int32_t verify_last,
+                                     int path);
+int fp8_pass_init_path(nvfp4_pass* pass, const fp8_gemm_problem* problems, int32_t count, int64_t M,
+                       const nvfp4_verify_spec* verify, int path, void* workspace, size_t workspace_bytes);
+
 /*
  * nvfp4_gemm_skinny_noalloc -- the tensor-core GEMM of nvfp4_gemm_skinny for callers
  * that cannot allocate device memory and so cannot pass a workspace. Examples are a

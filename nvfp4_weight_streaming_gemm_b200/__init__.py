@@ -344,11 +344,13 @@ class Fp8Pass:
     ``problems`` is a list of ``(X, q, scales, Y)``: X bf16 [M, K], the weight from
     :func:`fp8_pack`, and Y fp32 or bf16 [M, N]. ``verify`` is as for :class:`WeightPass`:
     ``(drafts, argmax, accept_len, max_logit[, parents, accept_node])``, and makes the last
-    problem the lm_head (its Y may be None). Every tensor is referenced by address: keep
+    problem the lm_head (its Y may be None). ``path`` picks the FP8 kernel: "f16" (codes
+    dequantised exactly to f16) or "terms" (codes straight into the FP8 tensor cores, X as two
+    residual E4M3 terms; ``fp8_pass_init_path``). Every tensor is referenced by address: keep
     them alive and refill X in place between runs.
     """
 
-    def __init__(self, problems, M: int, verify=None, workspace: torch.Tensor | None = None):
+    def __init__(self, problems, M: int, verify=None, workspace: torch.Tensor | None = None, path: str = "f16"):
         L = _lib
         n = len(problems)
         self._keep = []
@@ -384,15 +386,17 @@ class Fp8Pass:
             vs = L.VerifySpec(_ptr(drafts) if drafts.numel() else None, B, D, _ptr(amax), _ptr(acc), _ptr(vmax),
                               _ptr(parents) if parents is not None and parents.numel() else None, _ptr(node))
             self._keep.extend([drafts, amax, acc, vmax, parents, node])
-        nbytes = int(lib().fp8_pass_workspace_bytes(arr, n, M, 1 if verify is not None else 0))
+        kp = FP8_PATHS[path]
+        nbytes = int(lib().fp8_pass_workspace_bytes_path(arr, n, M, 1 if verify is not None else 0, kp))
         if nbytes == 0:
             raise NVFP4WSError(1, "fp8_pass_workspace_bytes")
         dev = problems[0][0].device
         self.workspace = _workspace(nbytes, dev, workspace)
         self.workspace_bytes = nbytes
         self.state = L.PassState()
-        _check(lib().fp8_pass_init(ctypes.byref(self.state), arr, n, M, ctypes.byref(vs) if vs is not None else None,
-                                   _ptr(self.workspace), nbytes), "fp8_pass_init")
+        _check(lib().fp8_pass_init_path(ctypes.byref(self.state), arr, n, M,
+                                        ctypes.byref(vs) if vs is not None else None, kp, _ptr(self.workspace),
+                                        nbytes), "fp8_pass_init")
         self.M = M
         self.count = n
 

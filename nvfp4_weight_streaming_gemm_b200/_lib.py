@@ -90,6 +90,9 @@ SIGNATURES = {
     "fp8_lmhead_verify": (ctypes.c_int, [c_p, c_p, c_p, c_i64, c_i64, c_i64, ctypes.POINTER(VerifySpec), c_p, c_sz,
                                          c_p]),
     "fp8_pass_workspace_bytes": (c_sz, [ctypes.POINTER(Fp8Problem), c_i32, c_i64, c_i32]),
+    "fp8_pass_workspace_bytes_path": (c_sz, [ctypes.POINTER(Fp8Problem), c_i32, c_i64, c_i32, ctypes.c_int]),
+    "fp8_pass_init_path": (ctypes.c_int, [ctypes.POINTER(PassState), ctypes.POINTER(Fp8Problem), c_i32, c_i64,
+                                          ctypes.POINTER(VerifySpec), ctypes.c_int, c_p, c_sz]),
     "fp8_pass_init": (ctypes.c_int, [ctypes.POINTER(PassState), ctypes.POINTER(Fp8Problem), c_i32, c_i64,
                                      ctypes.POINTER(VerifySpec), c_p, c_sz]),
     "fp8_pass_run": (ctypes.c_int, [ctypes.POINTER(PassState), c_p]),

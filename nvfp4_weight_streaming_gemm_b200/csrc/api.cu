@@ -561,18 +561,27 @@ static int fp8_host_problems(const fp8_gemm_problem* problems, int32_t count, in
   return NVFP4WS_OK;
 }
 
-size_t fp8_pass_workspace_bytes(const fp8_gemm_problem* problems, int32_t count, int64_t M, int32_t verify_last) {
+size_t fp8_pass_workspace_bytes_path(const fp8_gemm_problem* problems, int32_t count, int64_t M, int32_t verify_last,
+                                     int path) {
   std::vector<Fp8HostProblem> hp;
+  if (path != NVFP4WS_FP8_DEQUANT_F16 && path != NVFP4WS_FP8_E4M3_TERMS) return 0;
   if (fp8_host_problems(problems, count, M, verify_last, &hp, "fp8_pass_workspace_bytes") != NVFP4WS_OK) return 0;
-  return fp8_pass_workspace_bytes_int(hp.data(), count, M);
+  return path == NVFP4WS_FP8_E4M3_TERMS ? fp8q_pass_workspace_bytes_int(hp.data(), count, M)
+                                        : fp8_pass_workspace_bytes_int(hp.data(), count, M);
 }
 
-int fp8_pass_init(nvfp4_pass* pass, const fp8_gemm_problem* problems, int32_t count, int64_t M,
-                  const nvfp4_verify_spec* verify, void* workspace, size_t workspace_bytes) {
+size_t fp8_pass_workspace_bytes(const fp8_gemm_problem* problems, int32_t count, int64_t M, int32_t verify_last) {
+  return fp8_pass_workspace_bytes_path(problems, count, M, verify_last, NVFP4WS_FP8_DEQUANT_F16);
+}
+
+int fp8_pass_init_path(nvfp4_pass* pass, const fp8_gemm_problem* problems, int32_t count, int64_t M,
+                       const nvfp4_verify_spec* verify, int path, void* workspace, size_t workspace_bytes) {
   g_last_error[0] = 0;
   static_assert(sizeof(nvfp4_pass) >= kFp8PassStateBytes, "nvfp4_pass is too small for the FP8 pass state");
   if (!pass) return set_error(NVFP4WS_ERR_INVALID_ARG, "fp8_pass_init: pass is null");
   std::memset(pass, 0, sizeof(nvfp4_pass));
+  if (path != NVFP4WS_FP8_DEQUANT_F16 && path != NVFP4WS_FP8_E4M3_TERMS)
+    return set_error(NVFP4WS_ERR_INVALID_ARG, "fp8_pass_init: bad path %d", path);
   if (verify)
     if (int e = check_verify_size(verify, "fp8_pass_init")) return e;
   std::vector<Fp8HostProblem> hp;
@@ -592,12 +601,20 @@ int fp8_pass_init(nvfp4_pass* pass, const fp8_gemm_problem* problems, int32_t co
   }
   if (!workspace) return set_error(NVFP4WS_ERR_WORKSPACE, "fp8_pass_init: workspace is null");
   if (!aligned16(workspace)) return set_error(NVFP4WS_ERR_MISALIGNED, "fp8_pass_init: workspace must be 16-byte aligned");
+  if (path == NVFP4WS_FP8_E4M3_TERMS)
+    return fp8q_pass_init_int(pass->opaque, hp.data(), count, M, verify ? &vs : nullptr, workspace, workspace_bytes);
   return fp8_pass_init_int(pass->opaque, hp.data(), count, M, verify ? &vs : nullptr, workspace, workspace_bytes);
+}
+
+int fp8_pass_init(nvfp4_pass* pass, const fp8_gemm_problem* problems, int32_t count, int64_t M,
+                  const nvfp4_verify_spec* verify, void* workspace, size_t workspace_bytes) {
+  return fp8_pass_init_path(pass, problems, count, M, verify, NVFP4WS_FP8_DEQUANT_F16, workspace, workspace_bytes);
 }
 
 int fp8_pass_run(const nvfp4_pass* pass, nvfp4ws_stream_t stream) {
   g_last_error[0] = 0;
   if (!pass) return set_error(NVFP4WS_ERR_INVALID_ARG, "fp8_pass_run: pass is null");
+  if (fp8q_pass_owns(pass->opaque)) return fp8q_pass_run_int(pass->opaque, (cudaStream_t)stream);
   return fp8_pass_run_int(pass->opaque, (cudaStream_t)stream);
 }
 

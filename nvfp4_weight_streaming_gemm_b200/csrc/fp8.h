@@ -45,6 +45,12 @@ int launch_fp8q_gemm(const uint16_t* X, const uint8_t* q, const float* scales, l
                      void* Y, int y_dtype, void* workspace, cudaStream_t s);
 int launch_fp8q_verify(const uint16_t* X, const uint8_t* q, const float* scales, long long M, long long N,
                        long long K, const VerifyRule& v, void* workspace, cudaStream_t s);
+// FP8 weight passes on the E4M3-term kernel (state in the same caller-owned handle).
+size_t fp8q_pass_workspace_bytes_int(const Fp8HostProblem* hp, int n, long long M);
+int fp8q_pass_init_int(void* state, const Fp8HostProblem* hp, int n, long long M, const VerifyRule* vr,
+                       void* workspace, size_t workspace_bytes);
+int fp8q_pass_run_int(const void* state, cudaStream_t s);
+bool fp8q_pass_owns(const void* state);
 
 // fp32 W [N, K] -> E4M3 codes [N, K] and fp32 scales [ceil(N/128), ceil(K/128)].
 int launch_fp8_pack(const float* W, long long N, long long K, uint8_t* q, float* scales, cudaStream_t s);

@@ -16,6 +16,8 @@
 // the epilogue folds them with exact power-of-two weights before the block scale, and applies
 // g at the end.
 //
+// One GEMM, or a whole list of them (an FP8 weight pass) in one persistent launch, as fp8.cu.
+//
 // Roles per CTA (one persistent CTA per SM, 8 warps):
 //   warp 0        TMA producer: the unit's 16 KB code tiles (2-D, 128-byte swizzle) and the
 //                 matching term images (one contiguous bulk copy each; the prep kernel wrote
@@ -37,6 +39,7 @@
 #include <climits>
 #include <cmath>
 #include <cstring>
+#include <vector>
 
 namespace nvfp4ws {
 namespace fp8q {
@@ -52,26 +55,59 @@ constexpr int kMaxStages = 8;
 constexpr size_t kTailBytes = 8192;
 constexpr int kPrepThreads = 256;
 
-struct Params {
-  float* Y;                // fp32 or bf16 (y_bf16)
-  int y_bf16;
+// One GEMM of a launch. A pass keeps an array of these in device memory; TMA reads the tensor
+// map from there.
+struct alignas(64) Problem {
+  CUtensorMap tm_w;        // codes [N, K] u8, box 128 B x 128 rows, 128-byte swizzle
+  const uint16_t* X;       // [M, K] bf16 (read by the prep kernel)
   const float* scales;     // [tiles][K / 128]
-  const uint8_t* img;      // [K / 128][npadB][128] term images (shared-memory operand layout)
-  const float* gx;         // [M] per-row power-of-two scales
+  uint8_t* img;            // [K / 128][npadB][128] term images (shared-memory operand layout)
+  float* gx;               // [M] per-row power-of-two scales
+  void* Y;                 // [M, N] fp32 or bf16 (unused by the verify problem)
+  float* part_val;         // verify problem: per-tile row maxima [tiles][M]
+  int* part_idx;           //                 and their indices
+  long long N, K;
+  long long unit0;         // first unit of this problem in the launch's numbering
+  int tile0;               // first ticket counter of this problem
+  int kus;                 // units per tile: K / (128 * BPU)
+  int tiles, y_bf16, verify;
+};
+
+struct Params {
+  const Problem* probs;    // device array of a pass, or nullptr: the single problem passed by value
+  int nprob;
   uint32_t img_bytes;      // one block's image: npadB * 128
   int M, npad, npadB, np;
-  long long N, K;
-  int tiles, kus;
   long long units;
   int grid;
   int stages;
   uint32_t stage_bytes;
-  unsigned int* counters;  // [tiles], zero between calls
+  unsigned int* counters;  // [tiles of all problems], zero between calls
   float* partials;         // [2 * grid][M][128]
-  int verify;
-  float* part_val;         // [tiles][M]
-  int* part_idx;
   unsigned int* err;
+};
+
+// Position of a unit: its problem, the tile within that problem and the unit within the tile.
+struct Cursor {
+  int pi;
+  long long tile;
+  int ku;
+  __device__ __forceinline__ void init(const Problem* probs, int nprob, long long u) {
+    pi = 0;
+    while (pi + 1 < nprob && probs[pi + 1].unit0 <= u) ++pi;
+    const Problem& pr = probs[pi];
+    const long long r = u - pr.unit0;
+    tile = r / pr.kus;
+    ku = (int)(r - tile * pr.kus);
+  }
+  // Steps to the next unit. Past the launch's last unit pi equals nprob; do not read it then.
+  __device__ __forceinline__ void next(const Problem* probs) {
+    const Problem& pr = probs[pi];
+    if (++ku == pr.kus) {
+      ku = 0;
+      if (++tile == pr.tiles) { tile = 0; ++pi; }
+    }
+  }
 };
 
 // ---------------------------------------------------------------- activation terms
@@ -83,13 +119,17 @@ __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float first, float second) {
   return r;
 }
 
-// One CTA per row m: g[m], then the kT terms of every element into the block images. Image of
-// block kb: npadB rows of 128 B, row m*kT + t, 16-byte chunk j of a row stored at chunk j ^ (row % 8)
-// (the 128-byte swizzle the MMA's descriptor names).
-__global__ void __launch_bounds__(kPrepThreads) fp8q_prep_kernel(const uint16_t* __restrict__ X, long long K,
-                                                                   uint8_t* __restrict__ img, uint32_t img_bytes,
-                                                                   float* __restrict__ gx) {
-  const int m = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+// One CTA per (problem, row m): g[m], then the kT terms of every element into the block images.
+// Image of block kb: npadB rows of 128 B, row m*kT + t, 16-byte chunk j of a row stored at chunk
+// j ^ (row % 8) (the 128-byte swizzle the MMA's descriptor names).
+__global__ void __launch_bounds__(kPrepThreads) fp8q_prep_kernel(const __grid_constant__ Problem single,
+                                                                   const Problem* probs, int M, uint32_t img_bytes) {
+  const Problem& pr = probs ? probs[blockIdx.x / M] : single;
+  const uint16_t* X = pr.X;
+  const long long K = pr.K;
+  uint8_t* img = pr.img;
+  float* gx = pr.gx;
+  const int m = blockIdx.x % M, t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const uint16_t* xr = X + (long long)m * K;
   const long long nchunk = K / 16;
   __shared__ float s_red[kPrepThreads / 32];
@@ -214,26 +254,27 @@ __device__ __forceinline__ int cta_of_unit(long long u, long long U, int G) {
 
 // ---------------------------------------------------------------- epilogue pieces
 
-__device__ __forceinline__ void write_y(const Params& p, long long n, int m0, const float (&y)[16]) {
-  if (n >= p.N) return;
+__device__ __forceinline__ void write_y(const Params& p, const Problem& pr, long long n, int m0,
+                                        const float (&y)[16]) {
+  if (n >= pr.N) return;
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
     const int m = m0 + j;
     if (m < p.M) {
-      if (p.y_bf16)
-        reinterpret_cast<uint16_t*>(p.Y)[(long long)m * p.N + n] = f32_to_bf16_rn(y[j]);
+      if (pr.y_bf16)
+        reinterpret_cast<uint16_t*>(pr.Y)[(long long)m * pr.N + n] = f32_to_bf16_rn(y[j]);
       else
-        p.Y[(long long)m * p.N + n] = y[j];
+        reinterpret_cast<float*>(pr.Y)[(long long)m * pr.N + n] = y[j];
     }
   }
 }
 
-__device__ __forceinline__ void warp_argmax(const Params& p, long long n, int m0, const float (&y)[16], float* s_val,
-                                            int* s_idx, int q, int lane) {
+__device__ __forceinline__ void warp_argmax(const Problem& pr, long long n, int m0, const float (&y)[16],
+                                            float* s_val, int* s_idx, int q, int lane) {
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
-    float v = (n < p.N) ? y[j] : -INFINITY;
-    int i = (n < p.N) ? (int)n : INT_MAX;
+    float v = (n < pr.N) ? y[j] : -INFINITY;
+    int i = (n < pr.N) ? (int)n : INT_MAX;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       const float ov = __shfl_xor_sync(0xffffffffu, v, o);
@@ -244,8 +285,8 @@ __device__ __forceinline__ void warp_argmax(const Params& p, long long n, int m0
   }
 }
 
-__device__ __forceinline__ void tile_argmax_out(const Params& p, long long tile, int et, const float* s_val,
-                                                const int* s_idx) {
+__device__ __forceinline__ void tile_argmax_out(const Params& p, const Problem& pr, long long tile, int et,
+                                                const float* s_val, const int* s_idx) {
   if (et >= p.M) return;
   float bv = s_val[et];
   int bi = s_idx[et];
@@ -254,15 +295,15 @@ __device__ __forceinline__ void tile_argmax_out(const Params& p, long long tile,
       bv = s_val[w * kMaxM + et];
       bi = s_idx[w * kMaxM + et];
     }
-  p.part_val[tile * p.M + et] = bv;
-  p.part_idx[tile * p.M + et] = bi;
+  pr.part_val[tile * p.M + et] = bv;
+  pr.part_idx[tile * p.M + et] = bi;
 }
 
 // ---------------------------------------------------------------- the GEMM kernel
 
 template <int BPU>
 __global__ void __launch_bounds__(kThreads, 1)
-    fp8q_kernel(const __grid_constant__ CUtensorMap tm_w, const Params p) {
+    fp8q_kernel(const __grid_constant__ Problem single, const Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int S = p.stages, NP = p.np;
@@ -285,7 +326,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const long long U = p.units;
   const long long u_begin = unit_begin(c, U, p.grid), u_end = unit_begin(c + 1, U, p.grid);
   const int nunits = (int)(u_end - u_begin);
-  const int npadB = p.npadB, kus = p.kus;
+  const int npadB = p.npadB;
+  const Problem* probs = p.probs ? p.probs : &single;
   const uint32_t img_bytes = p.img_bytes;
   const uint32_t kR = 0;                           // running sums: columns [0, npad)
   const uint32_t pcol0 = (uint32_t)p.npad;         // P set b, block h at pcol0 + (b*BPU + h)*npadB
@@ -313,23 +355,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t pol_w = policy_evict_first(), pol_x = policy_evict_last();
       const uint32_t tx = (uint32_t)BPU * (kWBytes + img_bytes);
       int issued = 0;
-      long long tile = u_begin / kus;
-      int ku = (int)(u_begin % kus);
+      Cursor cur;
+      cur.init(probs, p.nprob, u_begin);
       int s = 0;
       uint32_t ph = 0;
       for (int i = 0; i < nunits; ++i) {
         if (!mbar_wait(bar_empty(s), ph ^ 1u, s_abort, p.err)) break;
         uint8_t* st = smem + (size_t)s * p.stage_bytes;
         mbar_arrive_expect_tx(bar_full(s), tx);
+        const Problem& pr = probs[cur.pi];
 #pragma unroll
         for (int h = 0; h < BPU; ++h) {
-          const int kb = ku * BPU + h;
-          tma_load_2d(smem_u32(st + h * kWBytes), &tm_w, kb * kKB, (int)(tile * kTileRows), bar_full(s), pol_w);
-          bulk_load(smem_u32(st + BPU * kWBytes + h * img_bytes), p.img + (size_t)kb * img_bytes, img_bytes,
+          const int kb = cur.ku * BPU + h;
+          tma_load_2d(smem_u32(st + h * kWBytes), &pr.tm_w, kb * kKB, (int)(cur.tile * kTileRows), bar_full(s),
+                      pol_w);
+          bulk_load(smem_u32(st + BPU * kWBytes + h * img_bytes), pr.img + (size_t)kb * img_bytes, img_bytes,
                     bar_full(s), pol_x);
         }
         issued = i + 1;
-        if (++ku == kus) { ku = 0; ++tile; }
+        cur.next(probs);
         if (++s == S) { s = 0; ph ^= 1u; }
       }
       if (*s_abort) {       // drain: wait (bounded) for every copy this thread issued
@@ -375,22 +419,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int rowl = q * 32 + lane;
     const int et = threadIdx.x - 4 * 32;             // 0..127
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
-    long long tile_it = u_begin / kus;
-    int ku_it = (int)(u_begin % kus);
-    // Block scales, four units ahead: block h of unit u has scale index BPU*u + h.
-    auto scale_of = [&](long long u, int h) { return u < u_end ? __ldg(p.scales + BPU * u + h) : 0.0f; };
+    // Block scales, four units ahead: block h of unit (tile, ku) has scale [tile][ku * BPU + h]
+    // of its problem; the L2 round trip is then off every unit's path.
+    Cursor ahead;
+    ahead.init(probs, p.nprob, u_begin);
+    int ia = 0;                                      // unit of this CTA's range that `ahead` is at
+    auto load_ahead = [&](float (&dst)[BPU]) {
+      if (ia < nunits) {
+        const Problem& pa = probs[ahead.pi];
+        const float* sp = pa.scales + (ahead.tile * pa.kus + ahead.ku) * BPU;
+#pragma unroll
+        for (int h = 0; h < BPU; ++h) dst[h] = __ldg(sp + h);
+        ahead.next(probs);
+      } else {
+#pragma unroll
+        for (int h = 0; h < BPU; ++h) dst[h] = 0.0f;
+      }
+      ++ia;
+    };
     float scn[4][BPU];
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int h = 0; h < BPU; ++h) scn[a][h] = scale_of(u_begin + a, h);
+    for (int a = 0; a < 4; ++a) load_ahead(scn[a]);
+    Cursor cur;
+    cur.init(probs, p.nprob, u_begin);
     for (int i = 0; i < nunits; ++i) {
       const long long u = u_begin + i;
-      const long long tile = tile_it;
-      const int ku = ku_it;
+      const Problem& pr = probs[cur.pi];
+      const long long tile = cur.tile;
+      const int ku = cur.ku, kus = pr.kus;
+      if (i + 1 < nunits) cur.next(probs);
       const bool seg_first = (i == 0) || (ku == 0);
       const bool seg_last = (i == nunits - 1) || (ku == kus - 1);
-      if (++ku_it == kus) { ku_it = 0; ++tile_it; }
       const int b = i % NP, k = i / NP;
       float sc[BPU];
 #pragma unroll
@@ -399,15 +458,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         scn[0][h] = scn[1][h];
         scn[1][h] = scn[2][h];
         scn[2][h] = scn[3][h];
-        scn[3][h] = scale_of(u + 4, h);
       }
+      load_ahead(scn[3]);
       // Every thread reaches the barrier, so a give-up seen by any of them ends the loop for all.
       mbar_wait(bar_pfull(b), (uint32_t)k & 1u, s_abort, p.err);
       named_bar(1, 128);
       if (ld_shared_volatile(s_abort)) break;
       tc_fence_after();
       const long long n = tile * kTileRows + rowl;
-      const long long tile_u0 = tile * kus, tile_u1 = tile_u0 + kus;
+      const long long tile_u0 = pr.unit0 + tile * kus, tile_u1 = tile_u0 + kus;
       const long long seg_u0 = u_begin > tile_u0 ? u_begin : tile_u0;
       const bool complete = (seg_u0 == tile_u0) && (u + 1 == tile_u1);
       const int slot = (seg_u0 == u_begin) ? 2 * c : 2 * c + 1;
@@ -441,10 +500,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_st_x16(lane_base + kR + m0, o);
         } else {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) y[j] *= (m0 + j < p.M) ? __ldg(p.gx + m0 + j) : 0.0f;   // exact: 2^e
+          for (int j = 0; j < 16; ++j) y[j] *= (m0 + j < p.M) ? __ldg(pr.gx + m0 + j) : 0.0f;   // exact: 2^e
           if (complete) {
-            if (p.verify) warp_argmax(p, n, m0, y, s_val, s_idx, q, lane);
-            else write_y(p, n, m0, y);
+            if (pr.verify) warp_argmax(pr, n, m0, y, s_val, s_idx, q, lane);
+            else write_y(p, pr, n, m0, y);
           } else {
             float* dst = p.partials + ((long long)slot * p.M) * kTileRows;
 #pragma unroll
@@ -458,9 +517,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(bar_pempty(b));
       if (!seg_last) continue;
       if (complete) {
-        if (p.verify) {
+        if (pr.verify) {
           named_bar(1, 128);
-          tile_argmax_out(p, tile, et, s_val, s_idx);
+          tile_argmax_out(p, pr, tile, et, s_val, s_idx);
           named_bar(1, 128);
         }
         continue;
@@ -473,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int expected = 0;
         for (int cc = c0; cc <= c1; ++cc)
           if (unit_begin(cc + 1, U, p.grid) > unit_begin(cc, U, p.grid)) ++expected;
-        const unsigned int prev = atomicAdd(p.counters + tile, 1u);
+        const unsigned int prev = atomicAdd(p.counters + pr.tile0 + tile, 1u);
         *s_last = (prev + 1 == (unsigned int)expected) ? 1 : 0;
       }
       named_bar(1, 128);
@@ -496,14 +555,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 16; ++j) y[j] += v[j];
           }
-          if (p.verify) warp_argmax(p, n, m0, y, s_val, s_idx, q, lane);
-          else write_y(p, n, m0, y);
+          if (pr.verify) warp_argmax(pr, n, m0, y, s_val, s_idx, q, lane);
+          else write_y(p, pr, n, m0, y);
         }
-        if (p.verify) {
+        if (pr.verify) {
           named_bar(1, 128);
-          tile_argmax_out(p, tile, et, s_val, s_idx);
+          tile_argmax_out(p, pr, tile, et, s_val, s_idx);
         }
-        if (et == 0) p.counters[tile] = 0u;          // ready for the next call
+        if (et == 0) p.counters[pr.tile0 + tile] = 0u;   // ready for the next call
       }
       named_bar(1, 128);
     }
@@ -541,27 +600,37 @@ bool fp8q_supported(long long M, long long K) {
 
 static size_t al256_q(size_t v) { return (v + 255) / 256 * 256; }
 
+// The launch shape and the workspace layout of a list of FP8 GEMMs sharing M.
 struct QPlan {
-  int npad, npadB, bpu, np, tiles, kus, grid, stages;
+  int npad, npadB, bpu, np, grid, stages;
+  int tiles, vtiles;       // tiles of all problems; of the verify problem (0 without one)
   long long units;
   uint32_t img_bytes, stage_bytes;
   size_t smem;
-  size_t off_partials, off_verify, off_img, off_gx, bytes;
+  size_t off_partials, off_verify, off_img, off_gx, off_desc, bytes;
+  std::vector<size_t> img_off;   // per problem, from off_img
 };
 
-static QPlan q_plan(long long M, long long N, long long K, bool verify) {
+static QPlan q_plan(long long M, const Fp8HostProblem* hp, int n, bool with_desc) {
   QPlan pl{};
   pl.npad = (int)std::max<long long>(16, (M + 15) / 16 * 16);
   pl.npadB = kT * pl.npad;                          // the epilogue reads 16 tokens' terms at a time
   pl.img_bytes = (uint32_t)pl.npadB * 128u;
-  const long long kbs = K / kKB;
+  bool even = true;
+  for (int i = 0; i < n; ++i) even = even && ((hp[i].K / kKB) % 2 == 0);
   // TMEM: R (npad), then np P sets of bpu * npadB columns.
   const int room = 512 - pl.npad;
-  pl.bpu = (kbs % 2 == 0 && room / (2 * pl.npadB) >= 2) ? 2 : 1;
+  pl.bpu = (even && room / (2 * pl.npadB) >= 2) ? 2 : 1;
   pl.np = std::max(1, std::min(kMaxP, room / (pl.bpu * pl.npadB)));
-  pl.tiles = (int)((N + kTileRows - 1) / kTileRows);
-  pl.kus = (int)(kbs / pl.bpu);
-  pl.units = (long long)pl.tiles * pl.kus;
+  size_t img = 0;
+  for (int i = 0; i < n; ++i) {
+    const int tiles = (int)((hp[i].N + kTileRows - 1) / kTileRows);
+    pl.units += (long long)tiles * (hp[i].K / kKB / pl.bpu);
+    pl.tiles += tiles;
+    if (hp[i].verify) pl.vtiles = tiles;
+    pl.img_off.push_back(img);
+    img += (size_t)(hp[i].K / kKB) * pl.img_bytes;   // multiples of 1024: npadB is a multiple of 16
+  }
   const int sms = std::max(1, device_sm_count());
   pl.grid = (int)std::min<long long>(sms, pl.units);
   pl.stage_bytes = (uint32_t)pl.bpu * (kWBytes + pl.img_bytes);
@@ -570,66 +639,68 @@ static QPlan q_plan(long long M, long long N, long long K, bool verify) {
   pl.smem = 1024 + (size_t)pl.stages * pl.stage_bytes + kTailBytes;
   pl.off_partials = al256_q((size_t)pl.tiles * 4);
   pl.off_verify = pl.off_partials + al256_q((size_t)2 * pl.grid * M * kTileRows * 4);
-  pl.off_img = pl.off_verify + (verify ? 2 * al256_q((size_t)pl.tiles * M * 4) : 0);
+  pl.off_img = pl.off_verify + (pl.vtiles ? 2 * al256_q((size_t)pl.vtiles * M * 4) : 0);
   pl.off_img = (pl.off_img + 1023) / 1024 * 1024;
-  pl.off_gx = pl.off_img + (size_t)kbs * pl.img_bytes;
-  pl.bytes = pl.off_gx + al256_q((size_t)M * 4);
+  pl.off_gx = pl.off_img + img;
+  pl.off_desc = pl.off_gx + al256_q((size_t)n * M * 4);
+  pl.bytes = pl.off_desc + (with_desc ? al256_q((size_t)n * sizeof(Problem)) : 0);
   return pl;
 }
 
-size_t fp8q_workspace_bytes_int(long long M, long long N, long long K, bool verify) {
-  if (!fp8q_supported(M, K) || N < 1) return 0;
-  return q_plan(M, N, K, verify).bytes;
-}
-
-static int launch_q(const uint16_t* X, const uint8_t* q, const float* scales, long long M, long long N, long long K,
-                    void* Y, int y_dtype, void* workspace, bool verify, QPlan* out, cudaStream_t s) {
-  const QPlan pl = q_plan(M, N, K, verify);
-  if (pl.stages < 2) return set_error(NVFP4WS_ERR_UNSUPPORTED, "fp8 term path: stage does not fit shared memory");
+static int fill_problem(Problem* P, const Fp8HostProblem& h, long long M, const QPlan& pl, long long unit0, int tile0,
+                        char* ws, int index) {
+  memset(static_cast<void*>(P), 0, sizeof(*P));
   auto fn = encode_fn_fp8q();
   if (!fn) return set_error(NVFP4WS_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-  alignas(64) CUtensorMap tw;
-  {
-    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)N};
-    cuuint64_t strides[1] = {(cuuint64_t)K};
-    cuuint32_t box[2] = {kKB, kTileRows};
-    cuuint32_t estr[2] = {1, 1};
-    if (fn(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(q), dims, strides, box, estr,
-           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return set_error(NVFP4WS_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  cuuint64_t dims[2] = {(cuuint64_t)h.K, (cuuint64_t)h.N};
+  cuuint64_t strides[1] = {(cuuint64_t)h.K};
+  cuuint32_t box[2] = {kKB, kTileRows};
+  cuuint32_t estr[2] = {1, 1};
+  if (fn(&P->tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(h.q), dims, strides, box, estr,
+         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return set_error(NVFP4WS_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  P->X = h.X;
+  P->scales = h.scales;
+  P->img = reinterpret_cast<uint8_t*>(ws + pl.off_img + pl.img_off[index]);
+  P->gx = reinterpret_cast<float*>(ws + pl.off_gx) + (size_t)index * M;
+  P->Y = h.Y;
+  P->N = h.N;
+  P->K = h.K;
+  P->unit0 = unit0;
+  P->tile0 = tile0;
+  P->kus = (int)(h.K / kKB / pl.bpu);
+  P->tiles = (int)((h.N + kTileRows - 1) / kTileRows);
+  P->y_bf16 = h.y_bf16;
+  P->verify = h.verify;
+  if (h.verify) {
+    P->part_val = reinterpret_cast<float*>(ws + pl.off_verify);
+    P->part_idx = reinterpret_cast<int*>(ws + pl.off_verify + al256_q((size_t)pl.vtiles * M * 4));
   }
-  char* ws = static_cast<char*>(workspace);
-  uint8_t* img = reinterpret_cast<uint8_t*>(ws + pl.off_img);
-  float* gx = reinterpret_cast<float*>(ws + pl.off_gx);
-  fp8q_prep_kernel<<<(unsigned)M, kPrepThreads, 0, s>>>(X, K, img, pl.img_bytes, gx);
+  return NVFP4WS_OK;
+}
+
+// Enqueue the term prep (one CTA per problem and row) and the GEMM. `single` is used when
+// `probs_dev` is null (one problem).
+static int launch_kernels(const Problem& single, const Problem* probs_dev, int nprob, long long M, const QPlan& pl,
+                          char* ws, cudaStream_t s) {
+  if (pl.stages < 2) return set_error(NVFP4WS_ERR_UNSUPPORTED, "fp8 term path: stage does not fit shared memory");
+  fp8q_prep_kernel<<<(unsigned)(M * nprob), kPrepThreads, 0, s>>>(single, probs_dev, (int)M, pl.img_bytes);
   if (int e = check_launch("fp8q_prep_kernel")) return e;
   Params p{};
-  p.Y = static_cast<float*>(Y);
-  p.y_bf16 = (y_dtype == NVFP4WS_Y_BF16);
-  p.scales = scales;
-  p.img = img;
-  p.gx = gx;
+  p.probs = probs_dev;
+  p.nprob = nprob;
   p.img_bytes = pl.img_bytes;
   p.M = (int)M;
   p.npad = pl.npad;
   p.npadB = pl.npadB;
   p.np = pl.np;
-  p.N = N;
-  p.K = K;
-  p.tiles = pl.tiles;
-  p.kus = pl.kus;
   p.units = pl.units;
   p.grid = pl.grid;
   p.stages = pl.stages;
   p.stage_bytes = pl.stage_bytes;
   p.counters = reinterpret_cast<unsigned int*>(ws);
   p.partials = reinterpret_cast<float*>(ws + pl.off_partials);
-  p.verify = verify ? 1 : 0;
-  if (verify) {
-    p.part_val = reinterpret_cast<float*>(ws + pl.off_verify);
-    p.part_idx = reinterpret_cast<int*>(ws + pl.off_verify + al256_q((size_t)pl.tiles * M * 4));
-  }
   p.err = device_error_word();
   if (!p.err) return set_error(NVFP4WS_ERR_CUDA, "cannot resolve the device error word");
   static std::atomic<bool> attr_set[64] = {};
@@ -641,26 +712,129 @@ static int launch_q(const uint16_t* X, const uint8_t* q, const float* scales, lo
       return check_launch("cudaFuncSetAttribute(fp8q_kernel)");
     attr_set[dev].store(true, std::memory_order_release);
   }
-  if (pl.bpu == 2) fp8q_kernel<2><<<pl.grid, kThreads, pl.smem, s>>>(tw, p);
-  else fp8q_kernel<1><<<pl.grid, kThreads, pl.smem, s>>>(tw, p);
-  *out = pl;
+  if (pl.bpu == 2) fp8q_kernel<2><<<pl.grid, kThreads, pl.smem, s>>>(single, p);
+  else fp8q_kernel<1><<<pl.grid, kThreads, pl.smem, s>>>(single, p);
   return check_launch("fp8q_kernel");
+}
+
+// ---------------------------------------------------------------------------- one GEMM
+
+static Fp8HostProblem one_q(const uint16_t* X, const uint8_t* q, const float* scales, long long N, long long K,
+                            void* Y, int y_dtype, bool verify) {
+  return Fp8HostProblem{X, q, scales, N, K, Y, y_dtype == NVFP4WS_Y_BF16 ? 1 : 0, verify ? 1 : 0};
+}
+
+size_t fp8q_workspace_bytes_int(long long M, long long N, long long K, bool verify) {
+  if (!fp8q_supported(M, K) || N < 1) return 0;
+  const Fp8HostProblem h = one_q(nullptr, nullptr, nullptr, N, K, nullptr, 0, verify);
+  return q_plan(M, &h, 1, false).bytes;
+}
+
+static int launch_one_q(const Fp8HostProblem& h, long long M, void* workspace, cudaStream_t s, QPlan* out) {
+  const QPlan pl = q_plan(M, &h, 1, false);
+  char* ws = static_cast<char*>(workspace);
+  alignas(64) Problem P;
+  if (int e = fill_problem(&P, h, M, pl, 0, 0, ws, 0)) return e;
+  *out = pl;
+  return launch_kernels(P, nullptr, 1, M, pl, ws, s);
 }
 
 int launch_fp8q_gemm(const uint16_t* X, const uint8_t* q, const float* scales, long long M, long long N, long long K,
                      void* Y, int y_dtype, void* workspace, cudaStream_t s) {
   QPlan pl;
-  return launch_q(X, q, scales, M, N, K, Y, y_dtype, workspace, false, &pl, s);
+  return launch_one_q(one_q(X, q, scales, N, K, Y, y_dtype, false), M, workspace, s, &pl);
 }
 
 int launch_fp8q_verify(const uint16_t* X, const uint8_t* q, const float* scales, long long M, long long N,
                        long long K, const VerifyRule& v, void* workspace, cudaStream_t s) {
   QPlan pl;
-  if (int e = launch_q(X, q, scales, M, N, K, nullptr, 0, workspace, true, &pl, s)) return e;
+  if (int e = launch_one_q(one_q(X, q, scales, N, K, nullptr, 0, true), M, workspace, s, &pl)) return e;
   char* ws = static_cast<char*>(workspace);
   return launch_verify_stage2(reinterpret_cast<const float*>(ws + pl.off_verify),
-                              reinterpret_cast<const int*>(ws + pl.off_verify + al256_q((size_t)pl.tiles * M * 4)),
-                              pl.tiles, (int)M, v, s);
+                              reinterpret_cast<const int*>(ws + pl.off_verify + al256_q((size_t)pl.vtiles * M * 4)),
+                              pl.vtiles, (int)M, v, s);
+}
+
+// ---------------------------------------------------------------------------- FP8 weight passes
+
+// Host state of an initialised pass on this kernel: plain data in the caller's nvfp4_pass.
+struct QPassState {
+  uint32_t magic;
+  int nprob, has_verify, vtiles;
+  long long M;
+  const Problem* probs;    // device copy, in the workspace
+  char* ws;
+  int npad, npadB, bpu, np, grid, stages;
+  long long units;
+  uint32_t img_bytes, stage_bytes;
+  size_t smem, off_partials, off_verify;
+  VerifyRule vr;
+};
+static_assert(sizeof(QPassState) <= kFp8PassStateBytes, "pass state does not fit the caller's handle");
+constexpr uint32_t kQPassMagic = 0x46503851u;
+
+bool fp8q_pass_owns(const void* state) {
+  uint32_t m;
+  memcpy(&m, state, sizeof(m));
+  return m == kQPassMagic;
+}
+
+size_t fp8q_pass_workspace_bytes_int(const Fp8HostProblem* hp, int n, long long M) {
+  return q_plan(M, hp, n, true).bytes;
+}
+
+int fp8q_pass_init_int(void* state, const Fp8HostProblem* hp, int n, long long M, const VerifyRule* vr,
+                       void* workspace, size_t workspace_bytes) {
+  const QPlan pl = q_plan(M, hp, n, true);
+  if (workspace_bytes < pl.bytes)
+    return set_error(NVFP4WS_ERR_WORKSPACE, "fp8_pass_init: workspace needs %zu bytes", pl.bytes);
+  if (pl.stages < 2) return set_error(NVFP4WS_ERR_UNSUPPORTED, "fp8 term path: stage does not fit shared memory");
+  char* ws = static_cast<char*>(workspace);
+  std::vector<Problem> P(n);
+  long long unit0 = 0;
+  int tile0 = 0;
+  for (int i = 0; i < n; ++i) {
+    if (int e = fill_problem(&P[i], hp[i], M, pl, unit0, tile0, ws, i)) return e;
+    unit0 += (long long)P[i].tiles * P[i].kus;
+    tile0 += P[i].tiles;
+  }
+  Problem* dev = reinterpret_cast<Problem*>(ws + pl.off_desc);
+  if (cudaMemcpy(dev, P.data(), (size_t)n * sizeof(Problem), cudaMemcpyHostToDevice) != cudaSuccess)
+    return check_launch("fp8_pass_init: descriptor copy");
+  QPassState st{};
+  st.magic = kQPassMagic;
+  st.nprob = n;
+  st.has_verify = vr != nullptr;
+  st.vtiles = pl.vtiles;
+  st.M = M;
+  st.probs = dev;
+  st.ws = ws;
+  st.npad = pl.npad; st.npadB = pl.npadB; st.bpu = pl.bpu; st.np = pl.np; st.grid = pl.grid; st.stages = pl.stages;
+  st.units = pl.units;
+  st.img_bytes = pl.img_bytes; st.stage_bytes = pl.stage_bytes;
+  st.smem = pl.smem; st.off_partials = pl.off_partials; st.off_verify = pl.off_verify;
+  if (vr) st.vr = *vr;
+  memcpy(state, &st, sizeof(st));
+  return NVFP4WS_OK;
+}
+
+int fp8q_pass_run_int(const void* state, cudaStream_t s) {
+  QPassState st;
+  memcpy(&st, state, sizeof(st));
+  if (st.magic != kQPassMagic) return set_error(NVFP4WS_ERR_INVALID_ARG, "fp8_pass_run: pass is not initialised");
+  QPlan pl{};
+  pl.npad = st.npad; pl.npadB = st.npadB; pl.bpu = st.bpu; pl.np = st.np; pl.grid = st.grid; pl.stages = st.stages;
+  pl.units = st.units;
+  pl.img_bytes = st.img_bytes; pl.stage_bytes = st.stage_bytes;
+  pl.smem = st.smem; pl.off_partials = st.off_partials; pl.off_verify = st.off_verify;
+  alignas(64) Problem unused;
+  memset(static_cast<void*>(&unused), 0, sizeof(unused));
+  if (int e = launch_kernels(unused, st.probs, st.nprob, st.M, pl, st.ws, s)) return e;
+  if (!st.has_verify) return NVFP4WS_OK;
+  return launch_verify_stage2(reinterpret_cast<const float*>(st.ws + st.off_verify),
+                              reinterpret_cast<const int*>(st.ws + st.off_verify +
+                                                           al256_q((size_t)st.vtiles * st.M * 4)),
+                              st.vtiles, (int)st.M, st.vr, s);
 }
 
 }  // namespace nvfp4ws
