@@ -88,9 +88,11 @@ def pass_kernel_source_hash() -> str:
 
 
 def measured_traffic(M: int, layers: int):
-    """DRAM bytes (read + write) of one pass_kernel launch at this M from the stored ncu
-    capture, or None when there is none for this workload or the kernel sources changed
-    since it was taken."""
+    """DRAM bytes (read + write) of one full-size pass_kernel launch at this M, from the stored
+    ncu capture, or None when there is none for this M or the kernel sources changed since it
+    was taken. The capture is of a reduced stack (its "layers"); its bytes are scaled to the
+    64-layer pass by the ratio of the algorithmic bytes, which assumes the excess over them
+    is the same fraction at both sizes."""
     if not os.path.exists(TRAFFIC_PROFILE) or layers != S.N_LAYERS:
         return None
     with open(TRAFFIC_PROFILE) as f:
@@ -98,7 +100,10 @@ def measured_traffic(M: int, layers: int):
     if prof.get("source_sha256") != pass_kernel_source_hash():
         return None
     v = prof.get("per_m", {}).get(str(M))
-    return None if v is None else float(v["dram_read_bytes"] + v["dram_write_bytes"])
+    if v is None:
+        return None
+    cap_layers = int(prof.get("layers", S.N_LAYERS))
+    return float(v["dram_read_bytes"] + v["dram_write_bytes"]) * pass_alg_bytes(M, layers) / pass_alg_bytes(M, cap_layers)
 
 
 def measured_peaks():
