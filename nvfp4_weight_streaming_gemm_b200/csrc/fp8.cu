@@ -488,10 +488,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         scn[2][h] = scn[3][h];
       }
       load_ahead(scn[3]);
-      // Every thread reaches the barrier, so a give-up seen by any of them ends the loop for all.
-      mbar_wait(bar_pfull(b), (uint32_t)k & 1u, s_abort, p.err);
-      named_bar(1, 128);
-      if (ld_shared_volatile(s_abort)) break;
+      // Every thread reaches the barrier and leaves with the same decision, so a give-up seen by
+      // any of them ends the loop for all.
+      const bool got = mbar_wait(bar_pfull(b), (uint32_t)k & 1u, s_abort, p.err);
+      if (named_bar_any(1, 128, !got || ld_shared_volatile(s_abort) != 0)) break;
       tc_fence_after();
       const long long n = tile * kTileRows + rowl;
       const long long tile_u0 = pr.unit0 + tile * kus, tile_u1 = tile_u0 + kus;

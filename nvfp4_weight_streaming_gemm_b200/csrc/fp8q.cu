@@ -24,7 +24,9 @@
 //                 them in the shared-memory operand layout). No multicast.
 //   warp 1        TMEM allocator and MMA issuer: 4 x kind::f8f6f4 (K = 32) per block, each
 //                 block into its own P of one of np rotating P sets.
-//   warps 4-7     promotion and epilogue, as in fp8.cu.
+//   warps 4-11    promotion and epilogue, as in fp8.cu: two warpgroups, each lane quarter's rows
+//                 served by two warps that take alternate groups of 16 tokens (the promotion's
+//                 TMEM round trips grow with M).
 // Scheduling, split tiles and bounded waits are those of fp8.cu.
 #include "common.cuh"
 #include "fp8.h"
@@ -44,7 +46,8 @@
 namespace nvfp4ws {
 namespace fp8q {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
+constexpr int kEpiThreads = 256;                     // warps 4-11
 constexpr int kTileRows = 128;
 constexpr int kKB = kFp8Block;                       // K elements of one scale block
 constexpr uint32_t kWBytes = kTileRows * kKB;        // 16 KB of codes per block
@@ -334,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) { mbar_init(bar_full(s), 1); mbar_init(bar_empty(s), 1); }
-    for (int b = 0; b < kMaxP; ++b) { mbar_init(bar_pfull(b), 1); mbar_init(bar_pempty(b), 128); }
+    for (int b = 0; b < kMaxP; ++b) { mbar_init(bar_pfull(b), 1); mbar_init(bar_pempty(b), kEpiThreads); }
     mbar_init(bar_drain, 1);
     *s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -416,8 +419,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= 4) {
     // ------------------------------------------------------------ promotion and epilogue warpgroup
     const int q = warp & 3;
+    const int half = (warp - 4) >> 2;                // token groups m0 / 16 of this parity
     const int rowl = q * 32 + lane;
-    const int et = threadIdx.x - 4 * 32;             // 0..127
+    const int et = threadIdx.x - 4 * 32;             // 0..255
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
     // Block scales, four units ahead: block h of unit (tile, ku) has scale [tile][ku * BPU + h]
     // of its problem; the L2 round trip is then off every unit's path.
@@ -460,10 +464,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         scn[2][h] = scn[3][h];
       }
       load_ahead(scn[3]);
-      // Every thread reaches the barrier, so a give-up seen by any of them ends the loop for all.
-      mbar_wait(bar_pfull(b), (uint32_t)k & 1u, s_abort, p.err);
-      named_bar(1, 128);
-      if (ld_shared_volatile(s_abort)) break;
+      // Every thread reaches the barrier and leaves with the same decision, so a give-up seen by
+      // any of them ends the loop for all.
+      const bool got = mbar_wait(bar_pfull(b), (uint32_t)k & 1u, s_abort, p.err);
+      if (named_bar_any(1, kEpiThreads, !got || ld_shared_volatile(s_abort) != 0)) break;
       tc_fence_after();
       const long long n = tile * kTileRows + rowl;
       const long long tile_u0 = pr.unit0 + tile * kus, tile_u1 = tile_u0 + kus;
@@ -471,7 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool complete = (seg_u0 == tile_u0) && (u + 1 == tile_u1);
       const int slot = (seg_u0 == u_begin) ? 2 * c : 2 * c + 1;
       const uint32_t pcol = pcol0 + (uint32_t)(b * BPU * npadB);
-      for (int m0 = 0; m0 < p.M; m0 += 16) {
+      for (int m0 = 16 * half; m0 < p.M; m0 += 32) {
         // tokens m0 .. m0+15: their 2 x 16 term columns of each block, and the running sums
         float y[16];
         uint32_t rv[16];
@@ -518,15 +522,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!seg_last) continue;
       if (complete) {
         if (pr.verify) {
-          named_bar(1, 128);
+          named_bar(1, kEpiThreads);
           tile_argmax_out(p, pr, tile, et, s_val, s_idx);
-          named_bar(1, 128);
+          named_bar(1, kEpiThreads);
         }
         continue;
       }
       // split tile: publish the partial, take a ticket; the last arrival finishes the tile
       __threadfence();
-      named_bar(1, 128);
+      named_bar(1, kEpiThreads);
       if (et == 0) {
         const int c0 = cta_of_unit(tile_u0, U, p.grid), c1 = cta_of_unit(tile_u1 - 1, U, p.grid);
         int expected = 0;
@@ -535,11 +539,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const unsigned int prev = atomicAdd(p.counters + pr.tile0 + tile, 1u);
         *s_last = (prev + 1 == (unsigned int)expected) ? 1 : 0;
       }
-      named_bar(1, 128);
+      named_bar(1, kEpiThreads);
       if (*s_last) {
         __threadfence();
         const int c0 = cta_of_unit(tile_u0, U, p.grid), c1 = cta_of_unit(tile_u1 - 1, U, p.grid);
-        for (int m0 = 0; m0 < p.M; m0 += 16) {
+        for (int m0 = 16 * half; m0 < p.M; m0 += 32) {
           float y[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) y[j] = 0.0f;
@@ -559,12 +563,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           else write_y(p, pr, n, m0, y);
         }
         if (pr.verify) {
-          named_bar(1, 128);
+          named_bar(1, kEpiThreads);
           tile_argmax_out(p, pr, tile, et, s_val, s_idx);
         }
         if (et == 0) p.counters[pr.tile0 + tile] = 0u;   // ready for the next call
       }
-      named_bar(1, 128);
+      named_bar(1, kEpiThreads);
     }
   }
 
