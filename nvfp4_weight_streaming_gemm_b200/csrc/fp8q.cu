@@ -91,25 +91,43 @@ struct Params {
 };
 
 // Position of a unit: its problem, the tile within that problem and the unit within the tile.
+// The problem's unit and tile counts are kept in registers and read again only when the walk
+// enters the next problem.
 struct Cursor {
   int pi;
   long long tile;
-  int ku;
+  int ku, kus, tiles;
   __device__ __forceinline__ void init(const Problem* probs, int nprob, long long u) {
     pi = 0;
     while (pi + 1 < nprob && probs[pi + 1].unit0 <= u) ++pi;
     const Problem& pr = probs[pi];
+    kus = pr.kus;
+    tiles = pr.tiles;
     const long long r = u - pr.unit0;
-    tile = r / pr.kus;
-    ku = (int)(r - tile * pr.kus);
+    tile = r / kus;
+    ku = (int)(r - tile * kus);
   }
-  // Steps to the next unit. Past the launch's last unit pi equals nprob; do not read it then.
-  __device__ __forceinline__ void next(const Problem* probs) {
-    const Problem& pr = probs[pi];
-    if (++ku == pr.kus) {
-      ku = 0;
-      if (++tile == pr.tiles) { tile = 0; ++pi; }
-    }
+  // Steps to the next unit. Past the launch's last unit pi equals nprob and nothing is read.
+  __device__ __forceinline__ void next(const Problem* probs, int nprob) {
+    if (++ku < kus) return;
+    ku = 0;
+    if (++tile < tiles) return;
+    tile = 0;
+    if (++pi < nprob) { kus = probs[pi].kus; tiles = probs[pi].tiles; }
+  }
+};
+
+// What the epilogue needs of the problem it is in, in registers (read once per problem).
+struct ProbView {
+  long long N, unit0;
+  int tile0, y_bf16, verify;
+  const float* gx;
+  void* Y;
+  float* part_val;
+  int* part_idx;
+  __device__ __forceinline__ void load(const Problem& pr) {
+    N = pr.N; unit0 = pr.unit0; tile0 = pr.tile0; y_bf16 = pr.y_bf16; verify = pr.verify;
+    gx = pr.gx; Y = pr.Y; part_val = pr.part_val; part_idx = pr.part_idx;
   }
 };
 
@@ -257,7 +275,7 @@ __device__ __forceinline__ int cta_of_unit(long long u, long long U, int G) {
 
 // ---------------------------------------------------------------- epilogue pieces
 
-__device__ __forceinline__ void write_y(const Params& p, const Problem& pr, long long n, int m0,
+__device__ __forceinline__ void write_y(const Params& p, const ProbView& pr, long long n, int m0,
                                         const float (&y)[16]) {
   if (n >= pr.N) return;
 #pragma unroll
@@ -272,7 +290,7 @@ __device__ __forceinline__ void write_y(const Params& p, const Problem& pr, long
   }
 }
 
-__device__ __forceinline__ void warp_argmax(const Problem& pr, long long n, int m0, const float (&y)[16],
+__device__ __forceinline__ void warp_argmax(const ProbView& pr, long long n, int m0, const float (&y)[16],
                                             float* s_val, int* s_idx, int q, int lane) {
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
@@ -288,7 +306,7 @@ __device__ __forceinline__ void warp_argmax(const Problem& pr, long long n, int 
   }
 }
 
-__device__ __forceinline__ void tile_argmax_out(const Params& p, const Problem& pr, long long tile, int et,
+__device__ __forceinline__ void tile_argmax_out(const Params& p, const ProbView& pr, long long tile, int et,
                                                 const float* s_val, const int* s_idx) {
   if (et >= p.M) return;
   float bv = s_val[et];
@@ -376,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     bar_full(s), pol_x);
         }
         issued = i + 1;
-        cur.next(probs);
+        cur.next(probs, p.nprob);
         if (++s == S) { s = 0; ph ^= 1u; }
       }
       if (*s_abort) {       // drain: wait (bounded) for every copy this thread issued
@@ -427,14 +445,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     // of its problem; the L2 round trip is then off every unit's path.
     Cursor ahead;
     ahead.init(probs, p.nprob, u_begin);
+    int ahead_pi = ahead.pi;
+    const float* ahead_scales = probs[ahead_pi].scales;
     int ia = 0;                                      // unit of this CTA's range that `ahead` is at
     auto load_ahead = [&](float (&dst)[BPU]) {
       if (ia < nunits) {
-        const Problem& pa = probs[ahead.pi];
-        const float* sp = pa.scales + (ahead.tile * pa.kus + ahead.ku) * BPU;
+        if (ahead.pi != ahead_pi) { ahead_pi = ahead.pi; ahead_scales = probs[ahead_pi].scales; }
+        const float* sp = ahead_scales + (ahead.tile * ahead.kus + ahead.ku) * BPU;
 #pragma unroll
         for (int h = 0; h < BPU; ++h) dst[h] = __ldg(sp + h);
-        ahead.next(probs);
+        ahead.next(probs, p.nprob);
       } else {
 #pragma unroll
         for (int h = 0; h < BPU; ++h) dst[h] = 0.0f;
@@ -446,12 +466,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int a = 0; a < 4; ++a) load_ahead(scn[a]);
     Cursor cur;
     cur.init(probs, p.nprob, u_begin);
+    ProbView pr;
+    int view_pi = cur.pi;
+    pr.load(probs[view_pi]);
     for (int i = 0; i < nunits; ++i) {
       const long long u = u_begin + i;
-      const Problem& pr = probs[cur.pi];
+      if (cur.pi != view_pi) { view_pi = cur.pi; pr.load(probs[view_pi]); }
       const long long tile = cur.tile;
-      const int ku = cur.ku, kus = pr.kus;
-      if (i + 1 < nunits) cur.next(probs);
+      const int ku = cur.ku, kus = cur.kus;
+      if (i + 1 < nunits) cur.next(probs, p.nprob);
       const bool seg_first = (i == 0) || (ku == 0);
       const bool seg_last = (i == nunits - 1) || (ku == kus - 1);
       const int b = i % NP, k = i / NP;
