@@ -476,13 +476,15 @@ struct Walk {
   }
 };
 
-// Most tokens a kernel instance serves. Five terms: the row is folded in registers; two
-// B tiles hold M*T <= 352 rows (M <= 70), one B tile M*T <= 256 (M <= 51), and a tile
-// pair needs a double-buffered accumulator, which leaves N <= 104 per tile (M <= 20).
-// One term (W4A4): the row is streamed from TMEM, so only the B rows bound M (352).
+// Most tokens a kernel instance serves, rounded up to 8 (the fold takes 8 tokens at a
+// time). Several terms: the row is folded in registers; two B tiles hold M*T <= 352 rows
+// (T = 5: M <= 70), one B tile M*T <= 256, and a tile pair needs a double-buffered
+// accumulator, which leaves N <= 104 per tile (T = 5: M <= 20). One term (W4A4): the row
+// is streamed from TMEM, so only the B rows bound M (352).
 __host__ __device__ constexpr int pass_max_tokens(int nbt, int tpu, int terms) {
-  return terms == 1 ? kMaxB : (tpu == 2 ? 24 : (nbt == 2 ? 72 : 56));
+  return terms == 1 ? kMaxB : ((tpu == 2 ? 104 : nbt == 2 ? kMaxB : 256) / terms + 7) / 8 * 8;
 }
+
 
 // T: activation terms (kMxf4Terms residual terms, or 1 for NVFP4 activations).
 template <int NBT, int KU, int TPU, int T>
@@ -858,17 +860,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         named_bar(1, 128);
       };
       // Fold the T terms of each token: y[m] = sum_t g_t acc[m*T + t] with g_t = g_0 / 4^t,
-      // i.e. g_0 * (acc_0 + (acc_1 + (acc_2 + (acc_3 + acc_4/4)/4)/4)/4) (the multiplications
-      // by 1/4 are exact; the prep kernel's g_t are the same sequence unless it underflows).
+      // i.e. g_0 * (acc_0 + (acc_1 + (... + acc_{T-1}/4)/4)/4) (the multiplications by 1/4
+      // are exact; the prep kernel's g_t are the same sequence unless it underflows).
       // Accumulator column j holds B row j, so token m's terms are columns m*T .. m*T+T-1.
-      // Tokens are taken 8 at a time: five TMEM loads of 8 columns are issued back to back
-      // and waited for once. The folded row (at most MT tokens) stays in registers, so the
+      // Tokens are taken 8 at a time: T TMEM loads of 8 columns are issued back to back and
+      // waited for once. The folded row (at most MT tokens) stays in registers, so the
       // accumulator is handed back to the MMA thread before any global store: with one
       // accumulator buffer (M=68) the stores of a tile then overlap the next tile's MMAs
       // (measured: holding the buffer through the stores stalled the MMA thread ~15 us per
       // tile under full HBM load).
-      if constexpr (T == kMxf4Terms) {
-        static_assert(kMxf4Terms == 5, "the fold below is written for 5 terms");
+      if constexpr (T > 1) {
         const int nb16 = (g.nb + 15) & ~15;                 // columns that exist in the accumulator
         float yr[TPU][MT];
 #pragma unroll
@@ -877,11 +878,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int mc = 0; mc < MT; mc += 8) {
             if (mc < M) {
-              const int col0 = mc * kMxf4Terms;               // multiple of 40
+              const int col0 = mc * T;                        // multiple of 8T
               const int n8 = (nb16 - col0) >> 3;              // >= 1: loads stay inside the accumulator
-              uint32_t v[40];
+              uint32_t v[8 * T];
 #pragma unroll
-              for (int k = 0; k < 5; ++k)
+              for (int k = 0; k < T; ++k)
                 if (k < n8) tc_ld_x8(taddr + (uint32_t)(col0 + 8 * k), v + 8 * k);
               const float4 ga = reinterpret_cast<const float4*>(s_g0 + mc)[0];
               const float4 gb = reinterpret_cast<const float4*>(s_g0 + mc)[1];
@@ -889,11 +890,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               tc_wait_ld();
 #pragma unroll
               for (int j = 0; j < 8; ++j) {
-                float a = __uint_as_float(v[j * kMxf4Terms + 4]);
-                a = fmaf(a, 0.25f, __uint_as_float(v[j * kMxf4Terms + 3]));
-                a = fmaf(a, 0.25f, __uint_as_float(v[j * kMxf4Terms + 2]));
-                a = fmaf(a, 0.25f, __uint_as_float(v[j * kMxf4Terms + 1]));
-                a = fmaf(a, 0.25f, __uint_as_float(v[j * kMxf4Terms + 0]));
+                float a = __uint_as_float(v[j * T + T - 1]);
+#pragma unroll
+                for (int t = T - 2; t >= 0; --t) a = fmaf(a, 0.25f, __uint_as_float(v[j * T + t]));
                 yr[tj][mc + j] = (mc + j < M) ? a * g0[j] : 0.f;   // columns past the tokens are never loaded
               }
             } else {
@@ -937,7 +936,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Up to 352 tokens do not fit in registers: the row is scaled and stored 16 tokens
         // at a time while the accumulator is held, and handed back after the last load.
         // (The host runs no verify problem here: its candidates are kept for <= 72 rows.)
-        static_assert(T == 1, "one or kMxf4Terms activation terms");
+        static_assert(T == 1, "one term or several");
         for (int tj = 0; tj < TPU; ++tj) {
           const uint32_t taddr = taddr0 + (uint32_t)(tj * NBT * g.nb_tile);
           const int tile = group * TPU + tj;
