@@ -79,7 +79,7 @@ const char* nvfp4ws_status_string(int status);
 const char* nvfp4ws_last_error(void);
 
 /* Library version as major*10000 + minor*100 + patch. 200 added struct_size to
- * nvfp4_gemm_problem and nvfp4_verify_spec. */
+ * nvfp4_gemm_problem and nvfp4_verify_spec. 201 added NVFP4WS_PASS_FOUR_TERMS. */
 int nvfp4ws_version(void);
 
 /* Largest M (rows of X) accepted by the GEMM and verify entry points. */
@@ -287,7 +287,8 @@ int lmhead_verify_argmax_accept_path(const void* X, const uint8_t* q, const uint
  *   leaves the part that needs it zero again. The pointers given (X, W, Y, verify
  *   buffers, workspace) are baked into the pass: later runs read and write the
  *   same buffers, so refill X in place between runs.
- * nvfp4_pass_run -- enqueues the pass on `stream` (3 kernels with verify, else 2).
+ * nvfp4_pass_run -- enqueues the pass on `stream` (3 kernels with verify, else 2; a
+ *   NVFP4WS_PASS_FOUR_TERMS pass with a verify after GEMMs: 5).
  *   It can be captured in a CUDA graph.
  *
  * Arguments
@@ -296,7 +297,8 @@ int lmhead_verify_argmax_accept_path(const void* X, const uint8_t* q, const uint
  *                 32768.  Y: [M, N] fp32 or bf16 per y_dtype (ignored for the verify
  *                 problem).
  *   count         >= 1.
- *   M             1 <= M <= 70 (the block-scaled path's limit).
+ *   M             1 <= M <= 70 (the block-scaled path's limit: M times the 5 activation
+ *                 terms fits 352 B rows; 88 for a NVFP4WS_PASS_FOUR_TERMS pass without verify).
  *   verify        NULL, or the verify buffers: M must equal B * (D + 1); drafts int32
  *                 [B, D] (may be NULL when D == 0); argmax int32 [M]; accept_len int32
  *                 [B]; max_logit fp32 [M] or NULL; parents int32 [B, D] for a tree
@@ -358,13 +360,23 @@ int nvfp4_pass_init(nvfp4_pass* pass, const nvfp4_gemm_problem* problems, int32_
  * bandwidth at small M, where the default plan uses larger units.
  *
  * nvfp4_pass_workspace_bytes_ex / nvfp4_pass_init_ex -- as the calls above, with
- *   `flags`, an OR of NVFP4WS_PASS_BATCH_INVARIANT and NVFP4WS_PASS_W4A4 (other bits
- *   are INVALID_ARG, and the workspace query returns 0). Pass the same flags to both.
+ *   `flags`, an OR of NVFP4WS_PASS_BATCH_INVARIANT, NVFP4WS_PASS_W4A4 and
+ *   NVFP4WS_PASS_FOUR_TERMS (other bits, or W4A4 with FOUR_TERMS, are INVALID_ARG, and
+ *   the workspace query returns 0). Pass the same flags to both.
  */
 #define NVFP4WS_PASS_BATCH_INVARIANT 1u
 /* A W4A4 pass: every problem as nvfp4_gemm_w4a4 computes it (M up to NVFP4WS_MAX_M, no
  * verify problem). */
 #define NVFP4WS_PASS_W4A4 2u
+/* The GEMMs of the pass write X as 4 residual NVFP4 terms instead of 5: their error against
+ * the exact product is ~1e-4 of a row's max|y| instead of ~1e-5 (a float64 model of the terms
+ * leaves 7e-5 to 1e-4 on the 27B layer shapes), and the tensor core, the image copies and the
+ * scale copies do a fifth less work per weight byte. Where a row has few outputs (N of a few
+ * columns) the per-row bar of 2e-3 of max|y| can then be missed on an output near zero. A
+ * verify problem keeps 5 terms (its argmax compares logits that may lie 1e-3 apart) and runs as
+ * a second persistent launch after the GEMMs' launch, whose weight loads may start while the
+ * GEMMs' last tiles finish. M up to 88 without a verify. */
+#define NVFP4WS_PASS_FOUR_TERMS 4u
 size_t nvfp4_pass_workspace_bytes_ex(const nvfp4_gemm_problem* problems, int32_t count, int64_t M,
                                      int32_t verify_last, uint32_t flags);
 int nvfp4_pass_init_ex(nvfp4_pass* pass, const nvfp4_gemm_problem* problems, int32_t count, int64_t M,

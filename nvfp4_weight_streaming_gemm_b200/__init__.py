@@ -26,6 +26,7 @@ from . import _lib
 PATHS = {"auto": 0, "gemv": 1, "mma": 2, "gemv_regs": 3, "mma_f16": 4}
 PASS_BATCH_INVARIANT = 1
 PASS_W4A4 = 2
+PASS_FOUR_TERMS = 4
 FP8_PATHS = {"f16": 0, "terms": 1}
 STATUS_OK = 0
 
@@ -278,13 +279,15 @@ class WeightPass:
     argmax over its rows and the accept lengths. ``verify`` may add ``(parents,
     accept_node)`` for a tree verify (``accept_node`` may be None). With
     ``batch_invariant`` every row gets the same bits for any M; with ``w4a4`` every
-    problem is the W4A4 product of :func:`gemm_w4a4` (no verify; ``nvfp4_pass_init_ex``).
+    problem is the W4A4 product of :func:`gemm_w4a4` (no verify; ``nvfp4_pass_init_ex``);
+    with ``four_terms`` the GEMMs take 4 residual activation terms instead of 5 (~1e-4 of
+    max|y| instead of ~1e-5; the verify keeps 5 and runs as a second launch).
     Every tensor is referenced by address: keep them alive and refill X in place
     between runs.
     """
 
     def __init__(self, problems, M: int, verify=None, workspace: torch.Tensor | None = None,
-                 batch_invariant: bool = False, w4a4: bool = False):
+                 batch_invariant: bool = False, w4a4: bool = False, four_terms: bool = False):
         L = _lib
         n = len(problems)
         self._keep = []
@@ -320,7 +323,8 @@ class WeightPass:
             vs = L.VerifySpec(_ptr(drafts) if drafts.numel() else None, B, D, _ptr(amax), _ptr(acc), _ptr(vmax),
                               _ptr(parents) if parents is not None and parents.numel() else None, _ptr(node))
             self._keep.extend([drafts, amax, acc, vmax, parents, node])
-        flags = (PASS_BATCH_INVARIANT if batch_invariant else 0) | (PASS_W4A4 if w4a4 else 0)
+        flags = ((PASS_BATCH_INVARIANT if batch_invariant else 0) | (PASS_W4A4 if w4a4 else 0)
+                 | (PASS_FOUR_TERMS if four_terms else 0))
         nbytes = int(lib().nvfp4_pass_workspace_bytes_ex(arr, n, M, 1 if verify is not None else 0, flags))
         if nbytes == 0:
             raise NVFP4WSError(1, "nvfp4_pass_workspace_bytes")

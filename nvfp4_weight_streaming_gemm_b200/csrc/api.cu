@@ -72,20 +72,21 @@ static int validate_gemm(const void* X, const uint8_t* q, const uint8_t* sf, con
 // shape allows it, else the f16 tensor-core kernel.
 enum { KPATH_GEMV = 1, KPATH_MXF4 = 2, KPATH_GEMV_REGS = 3, KPATH_MMA_F16 = 4, KPATH_NONE = 0 };
 
-static int resolve_path(int path, int64_t M, int64_t K) {
+// terms: activation terms of the block-scaled kernel for this call (a GEMM's or the verify's).
+static int resolve_path(int path, int64_t M, int64_t K, int terms = kGemmTerms) {
   switch (path) {
     case NVFP4WS_PATH_AUTO:
       // The block-scaled tensor-core kernel whenever it applies, M = 1 included: on B200 a
       // CUDA-core GEMV spends ~3.4 instructions per weight element on dequantisation and
       // products, more than an SM can issue at HBM rate (measured: 1.5 of 4 per cycle, 0.3-0.5
       // of HBM), while kind::mxf4nvf4 takes the packed weights with no per-element work.
-      if (mxf4_supported(M, K)) return KPATH_MXF4;
+      if (mxf4_supported(M, K, terms)) return KPATH_MXF4;
       if (M >= mma_min_m() && mma_supported(M, K)) return KPATH_MMA_F16;
       return KPATH_GEMV;
     case NVFP4WS_PATH_GEMV: return KPATH_GEMV;
     case NVFP4WS_PATH_GEMV_REGS: return KPATH_GEMV_REGS;
     case NVFP4WS_PATH_MMA:
-      if (mxf4_supported(M, K)) return KPATH_MXF4;
+      if (mxf4_supported(M, K, terms)) return KPATH_MXF4;
       return mma_supported(M, K) ? KPATH_MMA_F16 : KPATH_NONE;
     case NVFP4WS_PATH_MMA_F16: return mma_supported(M, K) ? KPATH_MMA_F16 : KPATH_NONE;
     default: return KPATH_NONE;
@@ -120,7 +121,7 @@ const char* nvfp4ws_status_string(int status) {
 
 const char* nvfp4ws_last_error(void) { return g_last_error; }
 
-int nvfp4ws_version(void) { return 200; }
+int nvfp4ws_version(void) { return 201; }
 
 int nvfp4ws_sm_count(void) { return device_sm_count(); }
 
@@ -233,7 +234,7 @@ size_t lmhead_verify_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   if (M < 1 || N < 1 || K < 32) return 0;
   size_t w = gemv_verify_workspace(M, N, K);
   size_t m = mma_supported(M, K) ? mma_verify_workspace_bytes(M, N, K) : 0;
-  size_t x = mxf4_supported(M, K) ? mxf4_workspace_bytes(M, N, K) : 0;
+  size_t x = mxf4_supported(M, K, kVerifyTerms) ? mxf4_workspace_bytes(M, N, K, kVerifyTerms) : 0;
   if (m > w) w = m;
   return x > w ? x : w;
 }
@@ -256,12 +257,12 @@ static int verify_impl(const void* X, const uint8_t* q, const uint8_t* sf, const
   if (!argmax || !accept_len) return set_error(NVFP4WS_ERR_INVALID_ARG, "lmhead_verify: null output pointer");
   if (path < NVFP4WS_PATH_AUTO || path > NVFP4WS_PATH_MMA_F16)
     return set_error(NVFP4WS_ERR_INVALID_ARG, "lmhead_verify: bad path %d", path);
-  const int kp = resolve_path(path, M, K);
+  const int kp = resolve_path(path, M, K, kVerifyTerms);
   if (kp == KPATH_NONE)
     return set_error(NVFP4WS_ERR_UNSUPPORTED, "lmhead_verify: the tensor-core paths need K %% 256 == 0 and "
                      "M <= 128 (M=%lld K=%lld)", (long long)M, (long long)K);
   if (kp == KPATH_MXF4) {
-    size_t need = mxf4_workspace_bytes(M, N, K);
+    size_t need = mxf4_workspace_bytes(M, N, K, kVerifyTerms);
     if (workspace == nullptr || workspace_bytes < need)
       return set_error(NVFP4WS_ERR_WORKSPACE, "lmhead_verify: workspace needs %zu bytes", need);
     if (!aligned16(workspace)) return set_error(NVFP4WS_ERR_MISALIGNED, "lmhead_verify: workspace must be 16-byte aligned");
@@ -342,10 +343,11 @@ static int check_verify_size(const nvfp4_verify_spec* v, const char* who) {
 }
 
 static int to_host_problems(const nvfp4_gemm_problem* problems, int32_t count, int64_t M, int verify_last,
-                            std::vector<MxHostProblem>* out, const char* who, int terms = kMxf4Terms) {
+                            std::vector<MxHostProblem>* out, const char* who, int terms) {
   if (!problems || count < 1) return set_error(NVFP4WS_ERR_INVALID_ARG, "%s: need count >= 1 problems", who);
   if (int e = check_problem_sizes(problems, count, who)) return e;
-  const int max_m = std::min(352 / terms, NVFP4WS_MAX_M);
+  // a verify problem takes more activation terms than the GEMMs, so fewer tokens fit
+  const int max_m = std::min(352 / (verify_last ? std::max(terms, kVerifyTerms) : terms), NVFP4WS_MAX_M);
   if (M < 1 || M > max_m || !mxf4_supported(M, 256, terms))
     return set_error(NVFP4WS_ERR_UNSUPPORTED, "%s: M=%lld outside 1..%d", who, (long long)M, max_m);
   out->clear();
@@ -369,13 +371,19 @@ static int to_host_problems(const nvfp4_gemm_problem* problems, int32_t count, i
   return NVFP4WS_OK;
 }
 
-static constexpr uint32_t kPassFlags = NVFP4WS_PASS_BATCH_INVARIANT | NVFP4WS_PASS_W4A4;
-static int pass_terms(uint32_t flags) { return (flags & NVFP4WS_PASS_W4A4) ? 1 : kMxf4Terms; }
+static constexpr uint32_t kPassFlags = NVFP4WS_PASS_BATCH_INVARIANT | NVFP4WS_PASS_W4A4 | NVFP4WS_PASS_FOUR_TERMS;
+static int pass_terms(uint32_t flags) {
+  return (flags & NVFP4WS_PASS_W4A4) ? 1 : (flags & NVFP4WS_PASS_FOUR_TERMS) ? kGemmTermsFast : kGemmTerms;
+}
+static bool pass_flags_ok(uint32_t flags) {
+  return (flags & ~kPassFlags) == 0 && (flags & (NVFP4WS_PASS_W4A4 | NVFP4WS_PASS_FOUR_TERMS)) !=
+                                           (NVFP4WS_PASS_W4A4 | NVFP4WS_PASS_FOUR_TERMS);
+}
 
 size_t nvfp4_pass_workspace_bytes_ex(const nvfp4_gemm_problem* problems, int32_t count, int64_t M,
                                      int32_t verify_last, uint32_t flags) {
   std::vector<MxHostProblem> hp;
-  if ((flags & ~kPassFlags) != 0 || ((flags & NVFP4WS_PASS_W4A4) && verify_last)) return 0;
+  if (!pass_flags_ok(flags) || ((flags & NVFP4WS_PASS_W4A4) && verify_last)) return 0;
   if (to_host_problems(problems, count, M, verify_last, &hp, "nvfp4_pass_workspace_bytes", pass_terms(flags)) !=
       NVFP4WS_OK)
     return 0;
@@ -395,8 +403,8 @@ int nvfp4_pass_init(nvfp4_pass* pass, const nvfp4_gemm_problem* problems, int32_
 int nvfp4_pass_init_ex(nvfp4_pass* pass, const nvfp4_gemm_problem* problems, int32_t count, int64_t M,
                        const nvfp4_verify_spec* verify, uint32_t flags, void* workspace, size_t workspace_bytes) {
   g_last_error[0] = 0;
-  if ((flags & ~kPassFlags) != 0)
-    return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_pass_init: unknown flags 0x%x", flags);
+  if (!pass_flags_ok(flags))
+    return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_pass_init: unknown flags or W4A4 with four terms (0x%x)", flags);
   if ((flags & NVFP4WS_PASS_W4A4) && verify)
     return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_pass_init: a W4A4 pass runs no verify");
   static_assert(sizeof(nvfp4_pass) >= kMxPassStateBytes, "nvfp4_pass is too small for the pass state");

@@ -20,14 +20,18 @@ int launch_mma_gemm(const uint16_t* X, const uint8_t* q, const uint8_t* sf, cons
 int launch_mma_verify(const uint16_t* X, const uint8_t* q, const uint8_t* sf, const float* ts, long long M,
                       long long N, long long K, const VerifyRule& v, void* workspace, cudaStream_t s);
 
-// Block-scaled (kind::mxf4nvf4) path: activations as kMxf4Terms residual NVFP4 terms, or
-// (terms = 1) as one NVFP4 quantisation per row: the W4A4 product.
-constexpr int kMxf4Terms = 5;
-bool mxf4_supported(long long M, long long K, int terms = kMxf4Terms);
-size_t mxf4_workspace_bytes(long long M, long long N, long long K, int terms = kMxf4Terms);
+// Block-scaled (kind::mxf4nvf4) path: activations as residual NVFP4 terms, kGemmTerms of them
+// for a GEMM and kVerifyTerms for the verify; kGemmTermsFast for the GEMMs of a pass that asks
+// for them (NVFP4WS_PASS_FOUR_TERMS); or (terms = 1) one NVFP4 quantisation per row: the W4A4
+// product.
+constexpr int kGemmTerms = 5;
+constexpr int kVerifyTerms = 5;
+constexpr int kGemmTermsFast = 4;
+bool mxf4_supported(long long M, long long K, int terms = kGemmTerms);
+size_t mxf4_workspace_bytes(long long M, long long N, long long K, int terms = kGemmTerms);
 int launch_mxf4_gemm(const uint16_t* X, const uint8_t* q, const uint8_t* sf, const float* ts, long long M,
                      long long N, long long K, void* Y, int y_dtype, void* workspace, cudaStream_t s,
-                     int terms = kMxf4Terms);
+                     int terms = kGemmTerms);
 int launch_mxf4_verify(const uint16_t* X, const uint8_t* q, const uint8_t* sf, const float* ts, long long M,
                        long long N, long long K, const VerifyRule& v, void* workspace, cudaStream_t s);
 
@@ -43,8 +47,9 @@ struct MxHostProblem {
 };
 // Host state of an initialised pass lives in a caller-owned buffer of this many bytes.
 constexpr size_t kMxPassStateBytes = 256;
-// binv: a batch-invariant pass (one unit shape for every M). terms: activation terms
-// (kMxf4Terms, or 1 for a W4A4 pass, which runs no verify).
+// binv: a batch-invariant pass (one unit shape for every M). terms: activation terms of the
+// GEMMs (kGemmTerms, kGemmTermsFast, or 1 for a W4A4 pass, which runs no verify); a verify
+// problem, which must be the last, always takes kVerifyTerms.
 size_t mxf4_pass_workspace_bytes(const MxHostProblem* hp, int n, long long M, bool binv, int terms);
 int mxf4_pass_init(void* state, const MxHostProblem* hp, int n, long long M, const VerifyRule* vs, bool binv,
                    int terms, void* workspace, size_t workspace_bytes);

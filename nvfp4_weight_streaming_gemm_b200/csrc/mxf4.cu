@@ -486,7 +486,7 @@ __host__ __device__ constexpr int pass_max_tokens(int nbt, int tpu, int terms) {
 }
 
 
-// T: activation terms (kMxf4Terms residual terms, or 1 for NVFP4 activations).
+// T: activation terms (kGemmTerms or kVerifyTerms residual terms, or 1 for NVFP4 activations).
 template <int NBT, int KU, int TPU, int T>
 __global__ void __launch_bounds__(kThreads, 1)
     pass_kernel(const __grid_constant__ Problem single, const PassParams p) {
@@ -1091,7 +1091,7 @@ struct MxPlan {
   size_t smem;
 };
 
-static MxPlan mx_plan_ku(long long M, int ku, int tpu, int terms = kMxf4Terms) {
+static MxPlan mx_plan_ku(long long M, int ku, int tpu, int terms) {
   MxPlan pl{};
   Geom& g = pl.g;
   g.M = (int)M;
@@ -1132,7 +1132,7 @@ static MxPlan mx_plan_ku(long long M, int ku, int tpu, int terms = kMxf4Terms) {
 // of 3). Either needs one B tile and a double-buffered accumulator.
 // Batch-invariant passes (binv) use one unit shape for every M, so that a row's units,
 // split points and summation order do not depend on how many rows share the pass.
-static MxPlan mx_plan(long long M, bool k512, bool binv = false, int terms = kMxf4Terms) {
+static MxPlan mx_plan(long long M, bool k512, bool binv, int terms) {
   auto ok = [](const MxPlan& x, int min_stages) {
     return x.g.nbt == 1 && x.acc_bufs == 2 && x.stages >= min_stages;
   };
@@ -1185,8 +1185,7 @@ static bool all_k512(const MxHostProblem* hp, int n) {
 }
 
 // with_desc: a pass keeps its descriptors and wave tables in the workspace.
-static WsLayout mx_layout(const MxHostProblem* hp, int n, long long M, bool with_desc, bool binv = false,
-                          int terms = kMxf4Terms) {
+static WsLayout mx_layout(const MxHostProblem* hp, int n, long long M, bool with_desc, bool binv, int terms) {
   const MxPlan pl = mx_plan(M, all_k512(hp, n), binv, terms);
   // waves are cut by image bytes; a batch-invariant pass cuts them as the largest M would
   const uint32_t wave_img_stride =
@@ -1275,8 +1274,9 @@ static const void* pass_instance_t(const Geom& g) {
                                                                                           : pass_fn<1, 1, 1, T>();
 }
 static const void* pass_instance(const Geom& g) {
-  static_assert(kMxf4Terms == 5, "pass kernel instances are built for 5 terms and 1");
-  return g.T == 1 ? pass_instance_t<1>(g) : pass_instance_t<5>(g);
+  static_assert(kGemmTerms == 5 && kVerifyTerms == 5 && kGemmTermsFast == 4,
+                "pass kernel instances are built for 1, 4 and 5 terms");
+  return g.T == 1 ? pass_instance_t<1>(g) : g.T == 4 ? pass_instance_t<4>(g) : pass_instance_t<5>(g);
 }
 
 static int ensure_attrs() {
@@ -1286,6 +1286,7 @@ static int ensure_attrs() {
     return set_error(NVFP4WS_ERR_CUDA, "cannot get the current device");
   if (!attr_set[dev]) {
     const void* fns[] = {pass_fn<1, 1, 1, 5>(), pass_fn<1, 2, 1, 5>(), pass_fn<1, 1, 2, 5>(), pass_fn<2, 1, 1, 5>(),
+                         pass_fn<1, 1, 1, 4>(), pass_fn<1, 2, 1, 4>(), pass_fn<1, 1, 2, 4>(), pass_fn<2, 1, 1, 4>(),
                          pass_fn<1, 1, 1, 1>(), pass_fn<1, 2, 1, 1>(), pass_fn<1, 1, 2, 1>(), pass_fn<2, 1, 1, 1>()};
     for (const void* f : fns)
       if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
@@ -1308,34 +1309,37 @@ static int prep_slices(int nprob, long long K) {
   return nprob == 1 ? (int)std::max<long long>(1, std::min<long long>(16, K / 2048)) : 1;
 }
 
-static int launch_pass(const Problem& single, const Problem* probs_dev, const PassTables& tb, int nprob,
-                       const MxPlan& pl, int grid, unsigned long long units, size_t off_part, long long max_k,
-                       char* ws, cudaStream_t s) {
+// 1) Activation decomposition of the launch's problems (a programmatic dependent launch: it
+//    may start while the previous kernel of the stream finishes, and waits for it before any
+//    access).
+static int launch_prep(const Problem& single, const Problem* probs_dev, int nprob, const MxPlan& pl, long long max_k,
+                       cudaStream_t s) {
+  if (int e = ensure_attrs()) return e;
+  const int slices = prep_slices(nprob, max_k);
+  cudaLaunchConfig_t pc = {};
+  pc.gridDim = dim3((unsigned)(pl.g.M * nprob * slices));
+  pc.blockDim = dim3(kPrepThreads);
+  pc.stream = s;
+  cudaLaunchAttribute pa[1];
+  pa[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pa[0].val.programmaticStreamSerializationAllowed = 1;
+  pc.attrs = pa;
+  pc.numAttrs = 1;
+  const Geom g = pl.g;
+  cudaError_t pe = g.T == 1   ? cudaLaunchKernelEx(&pc, x_prep_kernel<1>, single, probs_dev, g, slices)
+                   : g.T == 4 ? cudaLaunchKernelEx(&pc, x_prep_kernel<4>, single, probs_dev, g, slices)
+                              : cudaLaunchKernelEx(&pc, x_prep_kernel<5>, single, probs_dev, g, slices);
+  if (pe != cudaSuccess) return set_error(NVFP4WS_ERR_CUDA, "x_prep_kernel launch: %s", cudaGetErrorString(pe));
+  return check_launch("x_prep_kernel");
+}
+
+// 2) The GEMM, a programmatic dependent of the kernel before it (its prep kernel, or another
+//    prep kernel that waited for that one).
+static int launch_main(const Problem& single, const Problem* probs_dev, const PassTables& tb, int nprob,
+                       const MxPlan& pl, int grid, unsigned long long units, size_t off_part, char* ws, cudaStream_t s) {
   if (units * (unsigned long long)grid >= (1ull << 32))
     return set_error(NVFP4WS_ERR_UNSUPPORTED, "block-scaled path: too many units for the stream-K partition");
   if (int e = ensure_attrs()) return e;
-
-  // 1) activation decomposition (programmatic dependent launch: it may start while the
-  //    previous kernel of the stream finishes, and waits for it before any access)
-  {
-    const int slices = prep_slices(nprob, max_k);
-    cudaLaunchConfig_t pc = {};
-    pc.gridDim = dim3((unsigned)(pl.g.M * nprob * slices));
-    pc.blockDim = dim3(kPrepThreads);
-    pc.stream = s;
-    cudaLaunchAttribute pa[1];
-    pa[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    pa[0].val.programmaticStreamSerializationAllowed = 1;
-    pc.attrs = pa;
-    pc.numAttrs = 1;
-    const Geom g = pl.g;
-    cudaError_t pe = g.T == 1 ? cudaLaunchKernelEx(&pc, x_prep_kernel<1>, single, probs_dev, g, slices)
-                              : cudaLaunchKernelEx(&pc, x_prep_kernel<kMxf4Terms>, single, probs_dev, g, slices);
-    if (pe != cudaSuccess) return set_error(NVFP4WS_ERR_CUDA, "x_prep_kernel launch: %s", cudaGetErrorString(pe));
-    if (int e = check_launch("x_prep_kernel")) return e;
-  }
-
-  // 2) the GEMM, a programmatic dependent of the prep kernel
   PassParams p{};
   p.g = pl.g;
   p.probs = probs_dev;
@@ -1382,13 +1386,14 @@ size_t mxf4_workspace_bytes(long long M, long long N, long long K, int terms) {
 }
 
 static int launch_single(const MxHostProblem& h, long long M, void* workspace, cudaStream_t s, Problem* out,
-                         int terms = kMxf4Terms) {
+                         int terms) {
   const MxPlan pl = mx_plan(M, all_k512(&h, 1), false, terms);
   const WsLayout L = mx_layout(&h, 1, M, false, false, terms);
   char* ws = static_cast<char*>(workspace);
   if (int e = fill_problem(out, h, L, 0, 0, ws, pl.g.ku, pl.g.tpu)) return e;
   const PassTables none{nullptr, nullptr, nullptr, 1};
-  return launch_pass(*out, nullptr, none, 1, pl, L.grid, L.units, L.off_part, h.K, ws, s);
+  if (int e = launch_prep(*out, nullptr, 1, pl, h.K, s)) return e;
+  return launch_main(*out, nullptr, none, 1, pl, L.grid, L.units, L.off_part, ws, s);
 }
 
 int launch_mxf4_gemm(const uint16_t* X, const uint8_t* q, const uint8_t* sf, const float* ts, long long M,
@@ -1402,54 +1407,86 @@ int launch_mxf4_verify(const uint16_t* X, const uint8_t* q, const uint8_t* sf, c
                        long long N, long long K, const VerifyRule& v, void* workspace, cudaStream_t s) {
   MxHostProblem h{X, q, sf, ts, N, K, nullptr, 0, 1};
   Problem P;
-  if (int e = launch_single(h, M, workspace, s, &P)) return e;
+  if (int e = launch_single(h, M, workspace, s, &P, kVerifyTerms)) return e;
   return launch_verify_stage2(P.part_val, P.part_idx, P.tiles, (int)M, v, s);
 }
 
 // ------------------------------------------------------------------ multi-problem passes
 
+// A pass runs as one persistent launch, or as two when it ends in a verify and its GEMMs take
+// fewer activation terms than the verify (NVFP4WS_PASS_FOUR_TERMS): the GEMMs' launch, then
+// the verify's. Each launch has its own plan (term count, unit shape, stages) and its own
+// region of the workspace.
+struct PassPart {
+  int first, count, terms;
+};
+
+static int pass_parts(const MxHostProblem* hp, int n, int terms, PassPart (&parts)[2]) {
+  const bool verify = hp[n - 1].verify != 0;
+  if (!verify || terms == kVerifyTerms) {
+    parts[0] = PassPart{0, n, verify ? kVerifyTerms : terms};
+    return 1;
+  }
+  if (n == 1) {
+    parts[0] = PassPart{0, 1, kVerifyTerms};
+    return 1;
+  }
+  parts[0] = PassPart{0, n - 1, terms};
+  parts[1] = PassPart{n - 1, 1, kVerifyTerms};
+  return 2;
+}
+
+// One launch of a pass. Device addresses are offsets into the pass workspace, so two launches
+// fit the caller's fixed-size handle.
+struct MxLaunch {
+  unsigned long long base;     // this launch's region of the workspace
+  uint32_t off_part, off_desc, off_wave, off_cta, off_cunits;   // within the region
+  int32_t nprob, grid, nwave, max_k, terms, k512;
+  uint32_t units;
+};
+
 // Host state of a pass: plain data in caller-owned memory (no allocation).
 struct MxPassState {
   uint32_t magic;
-  int nprob, grid, verify, vtiles, k512, binv, terms;
-  long long M, max_k;
-  unsigned long long units;
-  size_t off_part;
+  int32_t nlaunch, verify, vtiles, binv;
+  long long M;
   char* ws;
-  Problem* probs_dev;
-  PassTables tb;
+  MxLaunch L[2];
   float* pv;
   int* pi;
   VerifyRule vs;
 };
 static_assert(sizeof(MxPassState) <= kMxPassStateBytes, "pass state does not fit the caller's handle");
-constexpr uint32_t kPassMagic = 0x4e565053u;
+constexpr uint32_t kPassMagic = 0x4e565054u;
 
 size_t mxf4_pass_workspace_bytes(const MxHostProblem* hp, int n, long long M, bool binv, int terms) {
-  return mx_layout(hp, n, M, true, binv, terms).total;
+  PassPart parts[2];
+  const int np = pass_parts(hp, n, terms, parts);
+  size_t total = 0;
+  for (int k = 0; k < np; ++k)
+    total = al256(total) + mx_layout(hp + parts[k].first, parts[k].count, M, true, binv, parts[k].terms).total;
+  return total;
 }
 
-int mxf4_pass_init(void* state, const MxHostProblem* hp, int n, long long M, const VerifyRule* vs, bool binv,
-                   int terms, void* workspace, size_t workspace_bytes) {
-  MxPassState* P = static_cast<MxPassState*>(state);
-  std::memset(static_cast<void*>(P), 0, sizeof(MxPassState));
+// Problem descriptors and wave tables of one launch, uploaded into its workspace region.
+static int init_launch(MxLaunch* out, const MxHostProblem* hp, int n, long long M, bool binv, int terms, char* ws,
+                       unsigned long long base, Problem* last) {
   const WsLayout L = mx_layout(hp, n, M, true, binv, terms);
   const MxPlan plan = mx_plan(M, all_k512(hp, n), binv, terms);
   const int ku = plan.g.ku, tpu = plan.g.tpu;
-  if (workspace_bytes < L.total)
-    return set_error(NVFP4WS_ERR_WORKSPACE, "nvfp4_pass_init: workspace %zu bytes < required %zu", workspace_bytes,
-                     L.total);
-  char* ws = static_cast<char*>(workspace);
+  char* reg = ws + base;
   std::vector<Problem> host(n);
   std::vector<unsigned long long> first(n);
   unsigned long long unit0 = 0;
   long long max_k = 0;
   for (int i = 0; i < n; ++i) {
     first[i] = unit0;
-    if (int e = fill_problem(&host[i], hp[i], L, i, unit0, ws, ku, tpu)) return e;
+    if (int e = fill_problem(&host[i], hp[i], L, i, unit0, reg, ku, tpu)) return e;
     unit0 += (unsigned long long)host[i].groups * (unsigned long long)host[i].kch;
     max_k = std::max(max_k, hp[i].K);
   }
+  if (unit0 * (unsigned long long)L.grid >= (1ull << 32))
+    return set_error(NVFP4WS_ERR_UNSUPPORTED, "nvfp4_pass_init: too many units for the stream-K partition");
   // wave tables: wave starts, each CTA's first problem in each wave, each CTA's unit count
   std::vector<uint32_t> wave_u0(L.nwave + 1);
   std::vector<int> cta_prob((size_t)L.nwave * L.grid), cta_units(L.grid, 0);
@@ -1470,46 +1507,94 @@ int mxf4_pass_init(void* state, const MxHostProblem* hp, int n, long long M, con
     }
   }
   wave_u0[L.nwave] = (uint32_t)unit0;
-  Problem* probs_dev = reinterpret_cast<Problem*>(ws + L.off_desc);
-  uint32_t* wave_dev = reinterpret_cast<uint32_t*>(ws + L.off_wave);
-  int* cta_dev = reinterpret_cast<int*>(ws + L.off_cta);
-  int* cunits_dev = reinterpret_cast<int*>(ws + L.off_cunits);
-  if (cudaMemcpy(probs_dev, host.data(), sizeof(Problem) * (size_t)n, cudaMemcpyHostToDevice) != cudaSuccess ||
-      cudaMemcpy(wave_dev, wave_u0.data(), sizeof(uint32_t) * wave_u0.size(), cudaMemcpyHostToDevice) != cudaSuccess ||
-      cudaMemcpy(cta_dev, cta_prob.data(), sizeof(int) * cta_prob.size(), cudaMemcpyHostToDevice) != cudaSuccess ||
-      cudaMemcpy(cunits_dev, cta_units.data(), sizeof(int) * cta_units.size(), cudaMemcpyHostToDevice) != cudaSuccess)
+  if (cudaMemcpy(reg + L.off_desc, host.data(), sizeof(Problem) * (size_t)n, cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(reg + L.off_wave, wave_u0.data(), sizeof(uint32_t) * wave_u0.size(), cudaMemcpyHostToDevice) !=
+          cudaSuccess ||
+      cudaMemcpy(reg + L.off_cta, cta_prob.data(), sizeof(int) * cta_prob.size(), cudaMemcpyHostToDevice) !=
+          cudaSuccess ||
+      cudaMemcpy(reg + L.off_cunits, cta_units.data(), sizeof(int) * cta_units.size(), cudaMemcpyHostToDevice) !=
+          cudaSuccess)
     return check_launch("nvfp4_pass_init: descriptor upload");
-  P->nprob = n;
-  P->k512 = all_k512(hp, n) ? 1 : 0;
+  out->base = base;
+  out->off_part = (uint32_t)L.off_part;
+  out->off_desc = (uint32_t)L.off_desc;
+  out->off_wave = (uint32_t)L.off_wave;
+  out->off_cta = (uint32_t)L.off_cta;
+  out->off_cunits = (uint32_t)L.off_cunits;
+  out->nprob = n;
+  out->grid = L.grid;
+  out->nwave = L.nwave;
+  out->max_k = (int32_t)max_k;
+  out->terms = terms;
+  out->k512 = all_k512(hp, n) ? 1 : 0;
+  out->units = (uint32_t)unit0;
+  *last = host[n - 1];
+  return NVFP4WS_OK;
+}
+
+int mxf4_pass_init(void* state, const MxHostProblem* hp, int n, long long M, const VerifyRule* vs, bool binv,
+                   int terms, void* workspace, size_t workspace_bytes) {
+  MxPassState* P = static_cast<MxPassState*>(state);
+  std::memset(static_cast<void*>(P), 0, sizeof(MxPassState));
+  const size_t need = mxf4_pass_workspace_bytes(hp, n, M, binv, terms);
+  if (workspace_bytes < need)
+    return set_error(NVFP4WS_ERR_WORKSPACE, "nvfp4_pass_init: workspace %zu bytes < required %zu", workspace_bytes,
+                     need);
+  char* ws = static_cast<char*>(workspace);
+  PassPart parts[2];
+  const int np = pass_parts(hp, n, terms, parts);
+  unsigned long long base = 0;
+  Problem last{};
+  for (int k = 0; k < np; ++k) {
+    base = al256(base);
+    const PassPart& pt = parts[k];
+    if (int e = init_launch(&P->L[k], hp + pt.first, pt.count, M, binv, pt.terms, ws, base, &last)) return e;
+    // layouts keep 32-bit offsets within a launch's region
+    const size_t bytes = mx_layout(hp + pt.first, pt.count, M, true, binv, pt.terms).total;
+    if (bytes >= (1ull << 32))
+      return set_error(NVFP4WS_ERR_UNSUPPORTED, "nvfp4_pass_init: a launch's workspace exceeds 4 GiB");
+    base += bytes;
+  }
+  P->nlaunch = np;
   P->binv = binv ? 1 : 0;
-  P->terms = terms;
-  P->grid = L.grid;
-  P->units = L.units;
-  P->off_part = L.off_part;
   P->M = M;
-  P->max_k = max_k;
   P->ws = ws;
-  P->probs_dev = probs_dev;
-  P->tb = PassTables{wave_dev, cta_dev, cunits_dev, L.nwave};
   P->verify = vs != nullptr;
   if (vs) {
     P->vs = *vs;
-    P->pv = host[n - 1].part_val;
-    P->pi = host[n - 1].part_idx;
-    P->vtiles = host[n - 1].tiles;
+    P->pv = last.part_val;
+    P->pi = last.part_idx;
+    P->vtiles = last.tiles;
   }
   P->magic = kPassMagic;
   return NVFP4WS_OK;
 }
 
+// Stream order: every launch's prep kernel, then every launch's GEMM kernel, then the verify's
+// stage 2. Each kernel is a programmatic dependent of the one before it and waits for it to
+// finish before reading what it wrote, so a later launch's weight loads may start while the
+// earlier launch's last tiles finish.
 int mxf4_pass_run(const void* state, cudaStream_t s) {
   const MxPassState* P = static_cast<const MxPassState*>(state);
   if (P->magic != kPassMagic) return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_pass_run: pass not initialised");
   static const Problem kNoProblem{};   // the kernels' by-value problem slot, unused by a pass
-  const MxPlan pl = mx_plan(P->M, P->k512 != 0, P->binv != 0, P->terms);
-  if (int e = launch_pass(kNoProblem, P->probs_dev, P->tb, P->nprob, pl, P->grid, P->units, P->off_part,
-                          P->max_k, P->ws, s))
-    return e;
+  for (int k = 0; k < P->nlaunch; ++k) {
+    const MxLaunch& L = P->L[k];
+    const MxPlan pl = mx_plan(P->M, L.k512 != 0, P->binv != 0, L.terms);
+    char* reg = P->ws + L.base;
+    if (int e = launch_prep(kNoProblem, reinterpret_cast<const Problem*>(reg + L.off_desc), L.nprob, pl, L.max_k, s))
+      return e;
+  }
+  for (int k = 0; k < P->nlaunch; ++k) {
+    const MxLaunch& L = P->L[k];
+    const MxPlan pl = mx_plan(P->M, L.k512 != 0, P->binv != 0, L.terms);
+    char* reg = P->ws + L.base;
+    const PassTables tb{reinterpret_cast<const uint32_t*>(reg + L.off_wave), reinterpret_cast<const int*>(reg + L.off_cta),
+                        reinterpret_cast<const int*>(reg + L.off_cunits), L.nwave};
+    if (int e = launch_main(kNoProblem, reinterpret_cast<const Problem*>(reg + L.off_desc), tb, L.nprob, pl, L.grid,
+                            L.units, L.off_part, reg, s))
+      return e;
+  }
   if (!P->verify) return NVFP4WS_OK;
   return launch_verify_stage2(P->pv, P->pi, P->vtiles, (int)P->M, P->vs, s);
 }

@@ -117,10 +117,16 @@ def test_pass_flags_are_checked_first(lib):
     from nvfp4_weight_streaming_gemm_b200 import _lib as L
     arr = (L.GemmProblem * 1)()
     arr[0] = L.GemmProblem(FAKE, FAKE, FAKE, FAKE, 128, 256, FAKE, 0)
-    assert lib.nvfp4_pass_workspace_bytes_ex(arr, 1, 17, 0, 4) == 0        # unknown flag
+    assert lib.nvfp4_pass_workspace_bytes_ex(arr, 1, 17, 0, 8) == 0        # unknown flag
     assert lib.nvfp4_pass_workspace_bytes_ex(arr, 1, 17, 1, 2) == 0        # W4A4 with a verify problem
+    assert lib.nvfp4_pass_workspace_bytes_ex(arr, 1, 17, 0, 6) == 0        # W4A4 with four terms
+    assert lib.nvfp4_pass_workspace_bytes_ex(arr, 1, 71, 0, 0) == 0        # 5 terms: M <= 70
+    assert lib.nvfp4_pass_workspace_bytes_ex(arr, 1, 89, 0, 4) == 0        # 4 terms: M <= 88
+    assert lib.nvfp4_pass_workspace_bytes_ex(arr, 1, 71, 1, 4) == 0        # the verify keeps 5 terms
     st = L.PassState()
     assert lib.nvfp4_pass_init_ex(ctypes.byref(st), arr, 1, 17, None, 8, FAKE, 1 << 20) == 1
+    assert b"flags" in lib.nvfp4ws_last_error()
+    assert lib.nvfp4_pass_init_ex(ctypes.byref(st), arr, 1, 17, None, 6, FAKE, 1 << 20) == 1
     assert b"flags" in lib.nvfp4ws_last_error()
 
 
