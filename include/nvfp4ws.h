@@ -59,8 +59,10 @@ typedef enum {
 /* Output element type of nvfp4_gemm_skinny. */
 typedef enum { NVFP4WS_Y_F32 = 0, NVFP4WS_Y_BF16 = 1 } nvfp4ws_ydtype;
 
-/* Kernel path of the GEMM. AUTO takes the block-scaled tensor-core kernel when K % 256 == 0 and
-   M <= 70, the f16 tensor-core kernel for larger M, and the GEMV otherwise. The others force a path. */
+/* Kernel path of the GEMM. AUTO takes the block-scaled tensor-core kernel when K % 256 == 0: in one
+   launch for M <= 70, and for larger M in ceil(M/70) equal slices of X's rows, one launch each
+   (nvfp4_gemm_skinny only; the verify takes the f16 tensor-core kernel for 70 < M <= 128). When
+   K % 256 != 0 it takes the GEMV. The others force a path. */
 typedef enum {
   NVFP4WS_PATH_AUTO = 0,
   NVFP4WS_PATH_GEMV = 1,          /* CUDA-core streaming GEMV: dequantises in registers; rows staged by
@@ -130,7 +132,7 @@ size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
  * (smaller ones round to f16 subnormals), and nothing saturates. Each product
  * x * (e2m1 * S) is then exact, sums are fp32, and the result is multiplied by ts and
  * by 2^e, in fp32.
- * Arithmetic of the block-scaled path (the default for 1 <= M <= 70 when K % 256 == 0):
+ * Arithmetic of the block-scaled path (the default when K % 256 == 0; M > 70 in row slices):
  * X is first written as 5 residual NVFP4 terms. Each is a per-row fp32 scale, an
  * E4M3 scale per 16 and E2M1 codes; each term quantises what the previous ones left.
  * The tensor core then multiplies the packed weights by those terms exactly, with

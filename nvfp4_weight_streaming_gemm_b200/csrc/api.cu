@@ -70,10 +70,22 @@ static int validate_gemm(const void* X, const uint8_t* q, const uint8_t* sf, con
 
 // Kernel actually used for a request: MMA means the block-scaled kernel when the
 // shape allows it, else the f16 tensor-core kernel.
-enum { KPATH_GEMV = 1, KPATH_MXF4 = 2, KPATH_GEMV_REGS = 3, KPATH_MMA_F16 = 4, KPATH_NONE = 0 };
+// MXF4_ROWS: the block-scaled kernel over consecutive slices of X's rows, one launch each.
+enum { KPATH_GEMV = 1, KPATH_MXF4 = 2, KPATH_GEMV_REGS = 3, KPATH_MMA_F16 = 4, KPATH_MXF4_ROWS = 5, KPATH_NONE = 0 };
+
+// Rows per launch when a GEMM's M exceeds what one block-scaled launch serves (M * 5 <= 352):
+// ceil(M / 70) slices of equal size. Each slice re-reads the weight, but at these M the f16
+// kernel is bound by its MMA issue rate (measured on the 27B gate+up shape: 204 us at M = 128
+// against 59 us at M = 68 on the block-scaled kernel), and past M = 128 only the GEMV is left.
+static int64_t mxf4_slice_rows(int64_t M) {
+  const int64_t cap = 352 / kGemmTerms;
+  const int64_t n = (M + cap - 1) / cap;
+  return (M + n - 1) / n;
+}
 
 // terms: activation terms of the block-scaled kernel for this call (a GEMM's or the verify's).
-static int resolve_path(int path, int64_t M, int64_t K, int terms = kGemmTerms) {
+// row_slices: AUTO may run the block-scaled kernel over slices of X's rows (GEMMs only).
+static int resolve_path(int path, int64_t M, int64_t K, int terms = kGemmTerms, bool row_slices = false) {
   switch (path) {
     case NVFP4WS_PATH_AUTO:
       // The block-scaled tensor-core kernel whenever it applies, M = 1 included: on B200 a
@@ -81,6 +93,7 @@ static int resolve_path(int path, int64_t M, int64_t K, int terms = kGemmTerms) 
       // products, more than an SM can issue at HBM rate (measured: 1.5 of 4 per cycle, 0.3-0.5
       // of HBM), while kind::mxf4nvf4 takes the packed weights with no per-element work.
       if (mxf4_supported(M, K, terms)) return KPATH_MXF4;
+      if (row_slices && mxf4_supported(mxf4_slice_rows(M), K, terms)) return KPATH_MXF4_ROWS;
       if (M >= mma_min_m() && mma_supported(M, K)) return KPATH_MMA_F16;
       return KPATH_GEMV;
     case NVFP4WS_PATH_GEMV: return KPATH_GEMV;
@@ -97,7 +110,9 @@ static int resolve_path(int path, int64_t M, int64_t K, int terms = kGemmTerms) 
 static size_t gemm_ws_any(int64_t M, int64_t N, int64_t K) {
   size_t a = mma_supported(M, K) ? mma_gemm_workspace_bytes(M, N, K) : 0;
   size_t b = mxf4_supported(M, K) ? mxf4_workspace_bytes(M, N, K) : 0;
-  return a > b ? a : b;
+  const int64_t mr = mxf4_slice_rows(M);
+  size_t c = (!mxf4_supported(M, K) && mxf4_supported(mr, K)) ? mxf4_workspace_bytes(mr, N, K) : 0;
+  return std::max(a, std::max(b, c));
 }
 
 }  // namespace nvfp4ws
@@ -156,11 +171,30 @@ int nvfp4_gemm_skinny_path(const void* X, const uint8_t* q, const uint8_t* sf, c
     return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_gemm_skinny: bad y_dtype %d", y_dtype);
   if (path < NVFP4WS_PATH_AUTO || path > NVFP4WS_PATH_MMA_F16)
     return set_error(NVFP4WS_ERR_INVALID_ARG, "nvfp4_gemm_skinny: bad path %d", path);
-  const int kp = resolve_path(path, M, K);
+  const int kp = resolve_path(path, M, K, kGemmTerms, true);
   cudaStream_t s = (cudaStream_t)stream;
   if (kp == KPATH_NONE)
     return set_error(NVFP4WS_ERR_UNSUPPORTED, "nvfp4_gemm_skinny: the tensor-core paths need K %% 256 == 0 and "
                      "M <= 128 (M=%lld K=%lld)", (long long)M, (long long)K);
+  if (kp == KPATH_MXF4_ROWS) {
+    // The slices run one after another on the stream and share the workspace: each launch's
+    // prep kernel waits for the previous GEMM to finish before it rewrites the images, and
+    // every launch leaves its tickets zero.
+    const int64_t mr = mxf4_slice_rows(M);
+    size_t need = mxf4_workspace_bytes(mr, N, K);
+    if (workspace == nullptr || workspace_bytes < need)
+      return set_error(NVFP4WS_ERR_WORKSPACE, "nvfp4_gemm_skinny: workspace needs %zu bytes", need);
+    if (!aligned16(workspace))
+      return set_error(NVFP4WS_ERR_MISALIGNED, "nvfp4_gemm_skinny: workspace must be 16-byte aligned");
+    const size_t ysz = y_dtype == NVFP4WS_Y_BF16 ? 2 : 4;
+    for (int64_t m0 = 0; m0 < M; m0 += mr) {
+      const int64_t m = std::min(mr, M - m0);
+      if (int e = launch_mxf4_gemm(static_cast<const uint16_t*>(X) + m0 * K, q, sf, tensor_scale, m, N, K,
+                                   static_cast<char*>(Y) + (size_t)(m0 * N) * ysz, y_dtype, workspace, s))
+        return e;
+    }
+    return NVFP4WS_OK;
+  }
   if (kp == KPATH_MXF4) {
     size_t need = mxf4_workspace_bytes(M, N, K);
     if (workspace == nullptr || workspace_bytes < need)

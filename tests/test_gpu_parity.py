@@ -321,6 +321,34 @@ def test_gemm_mma(nv, M, N, K, path):
         assert worst <= TERMS_TOL, f"{worst:.2e} of max|y|"
 
 
+@pytest.mark.parametrize("M", [71, 128, 200])
+def test_gemm_auto_row_slices(nv, M):
+    """AUTO past M = 70: the block-scaled kernel over ceil(M/70) equal slices of X's rows, one
+    launch each, sharing the workspace. A slice is the GEMM of its rows alone, so the result
+    equals the slices run as separate calls, bit for bit, and keeps the five-term accuracy."""
+    N, K = 1000, 1280
+    W, x = S.random_case(M * 7 + 5, M, N, K)
+    Wd = torch.from_numpy(W).cuda()
+    q, sf, ts = nv.pack(Wd)
+    X = to_dev_bf16(x)
+    ws = torch.zeros(nv.gemm_workspace_bytes(M, N, K), dtype=torch.uint8, device="cuda")
+    n0 = nv.lib().nvfp4ws_kernel_launches()
+    Y = nv.gemm(X, q, sf, ts, workspace=ws)
+    torch.cuda.synchronize()
+    nslice = -(-M // 70)
+    assert nv.lib().nvfp4ws_kernel_launches() - n0 == 2 * nslice          # prep + GEMM per slice
+    nv.check()
+    q_ref, sf_ref, ts_ref = F.quantize_nvfp4(W)
+    y_ref = G.gemm_ref(x, q_ref, sf_ref, ts_ref)
+    worst = assert_rowwise(Y.cpu().numpy(), y_ref)
+    assert worst <= TERMS_TOL, f"{worst:.2e} of max|y|"
+    mr = -(-M // nslice)
+    for m0 in range(0, M, mr):
+        Ys = nv.gemm(X[m0: m0 + mr], q, sf, ts, path="mma")
+        torch.cuda.synchronize()
+        assert torch.equal(Ys, Y[m0: m0 + mr])
+
+
 @pytest.mark.parametrize("path", ["mma", "mma_f16"])
 def test_gemm_mma_bf16_and_deterministic(nv, path):
     W, x = S.random_case(61, 17, 2000, 4096)
