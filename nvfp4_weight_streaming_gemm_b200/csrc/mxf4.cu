@@ -508,6 +508,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* s_idx = reinterpret_cast<int*>(s_val + 4 * 72);                 // [4][72]
   // g_0 of each token of the current problem, 16-byte aligned for float4 reads [kMaxB]
   float* s_g0 = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(s_idx + 4 * 72) + 15) & ~uintptr_t(15));
+  // the split tile group whose partials the whole CTA sums after the role loops (on = 0: none)
+  struct DeferredFixup {
+    int on, pi, group, c0, c1, wave;
+    uint32_t tile_u0, w0, Uw;
+  };
+  DeferredFixup* s_def = reinterpret_cast<DeferredFixup*>(s_g0 + kMaxB);
 
   auto bar_full = [&](int s) { return smem_u32(bars + s); };
   auto bar_empty = [&](int s) { return smem_u32(bars + S + s); };
@@ -531,6 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int b = 0; b < p.sf_bufs; ++b) mbar_init(bar_sffull(b), 128);
     mbar_init(bar_drain, 1);
     *s_abort = 0;
+    s_def->on = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
@@ -990,7 +997,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       named_bar(1, 128);
       if (et == 0 && seg <= 2) MX_CTA(10 + 4 * (seg - 1));
-      if (*s_last) {
+      // The CTA's final segment of a GEMM with tile-pair units: every warp is free once the
+      // role loops end, so the whole CTA sums the partials then (below), with a row's
+      // contributors 8 at a time in flight. (Measured on single GEMMs: M=17, tile pairs, a
+      // chained 27B pass 7.1 -> 6.7 ms; one tile per unit (M=1, M=68) slightly slower, so
+      // those keep the epilogue's own sum.)
+      const bool defer = TPU == 2 && *s_last && !verify && done >= nunits;
+      if (defer && et == 0) {
+        s_def->pi = pi; s_def->group = group; s_def->c0 = c0; s_def->c1 = c1; s_def->wave = wave;
+        s_def->tile_u0 = tile_u0; s_def->w0 = w0; s_def->Uw = Uw;
+        s_def->on = 1;
+        *ticket = 0u;                      // ready for the next launch
+      }
+      if (*s_last && !defer) {
         // Sum the contributors' partials in CTA order (deterministic), 16 tokens per pass. The
         // loads of four contributors are issued together: a tile split across many CTAs (the
         // down projection's 40 tiles over 148 CTAs) then costs a quarter of the dependent L2
@@ -1045,6 +1064,62 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+  }
+  if (s_def->on) {
+    // The deferred sum of a split tile group, by all warps: one work item per (tile, row,
+    // 8 tokens), its contributors' partials loaded 8 CTAs at a time and added in CTA order,
+    // as the epilogue's own sum does (the same bits). The epilogue thread that took the last
+    // ticket acquired the other CTAs' partials before the barrier above.
+    const DeferredFixup d = *s_def;
+    const Problem* pr = probs + d.pi;
+    const int M = g.M, Mp = (M + 3) & ~3, ng8 = (M + 7) >> 3;
+    const float* wave_part = p.partials + (long long)d.wave * 2 * G * g.tpu * kTileRows * Mp;
+    const float ts = *pr->ts;
+    const long long N = pr->N;
+    const int items = g.tpu * kTileRows * ng8;
+    for (int it = threadIdx.x; it < items; it += kThreads) {
+      const int row = it % kTileRows, rest = it / kTileRows, mg = rest % ng8, tj = rest / ng8;
+      const int mc = mg * 8;
+      float acc[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+      for (int cc = d.c0; cc <= d.c1; cc += 8) {
+        float4 v[8][2];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int cx = cc + k;
+          const bool on = cx <= d.c1;
+          const int sl =
+              on ? ((d.w0 + unit_begin((uint32_t)cx, d.Uw, G) >= d.tile_u0) ? 2 * cx : 2 * cx + 1) : 0;
+          const float4* src =
+              reinterpret_cast<const float4*>(wave_part + ((long long)(sl * g.tpu + tj) * kTileRows + row) * Mp + mc);
+#pragma unroll
+          for (int b = 0; b < 2; ++b)
+            v[k][b] = (on && mc + 4 * b < Mp) ? __ldcg(src + b) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          if (cc + k <= d.c1) {
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+              acc[4 * b] += v[k][b].x; acc[4 * b + 1] += v[k][b].y;
+              acc[4 * b + 2] += v[k][b].z; acc[4 * b + 3] += v[k][b].w;
+            }
+          }
+        }
+      }
+      const long long n = (long long)(d.group * g.tpu + tj) * kTileRows + row;
+      if (n < N) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int m = mc + j;
+          if (m < M) {
+            if (pr->y_bf16) reinterpret_cast<uint16_t*>(pr->Y)[(long long)m * N + n] = f32_to_bf16_rn(acc[j] * ts);
+            else static_cast<float*>(pr->Y)[(long long)m * N + n] = acc[j] * ts;
+          }
+        }
+      }
+    }
   }
   if (threadIdx.x == 0) MX_CTA(5);
 }
