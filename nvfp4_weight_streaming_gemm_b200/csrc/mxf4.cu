@@ -154,8 +154,12 @@ __device__ __forceinline__ float block_amax16(const float (&v)[16]) {
 }
 
 // One CTA per (activation row, problem). A first sweep over the row finds amax|x|
-// (one CTA reduction), a second re-reads it (from L2) and writes the T terms of each
-// 16-element block. Per-thread state is small, so several CTAs fit an SM and the many
+// (one CTA reduction; each thread has four blocks' loads in flight before it uses any),
+// a second re-reads it (from L2) and writes the T terms of each 16-element block. On the
+// path of a single GEMM the prep's latency is paid in full, so its registers are not
+// squeezed for occupancy (measured: 40 registers with spills and one round trip per block
+// made the prep 4-8 us after the previous kernel ended; 64 registers and the unrolled
+// sweep, 3-5 us). Per-thread state is small, so several CTAs fit an SM and the many
 // short rows of a pass are prepared at once. Repeated
 // multiplication by 0.25 is exact unless g underflows; the decomposition and the stored
 // g follow the same sequence. The code and scale choices only need to be consistent
@@ -290,7 +294,7 @@ __device__ __forceinline__ void quantise_block(float (&r)[16], int b, int m, flo
 // once); a single GEMM splits each row so that the prep's latency, which the GEMM waits for,
 // does not grow with K.
 template <int T>
-__global__ void __launch_bounds__(kPrepThreads, 6) x_prep_kernel(const __grid_constant__ Problem single,
+__global__ void __launch_bounds__(kPrepThreads, 4) x_prep_kernel(const __grid_constant__ Problem single,
                                                                   const Problem* probs, const Geom g, int slices) {
   asm volatile("griddepcontrol.launch_dependents;");
   // X may come from the previous kernel of the stream, and the previous GEMM may still
@@ -304,11 +308,25 @@ __global__ void __launch_bounds__(kPrepThreads, 6) x_prep_kernel(const __grid_co
   const uint16_t* X = pr->X + (long long)m * pr->K;
   uint8_t* img = pr->ximg;
   __shared__ float s_red[kPrepThreads / 32];
+  // amax over the row, four blocks' loads in flight per thread before any is used (a loop
+  // that uses each load before issuing the next costs one memory round trip per block)
   float amax = 0.f;
-  for (int b = t; b < nblk; b += kPrepThreads) {
-    float r[16];
-    load_block16(X, b, r);
-    amax = fmaxf(amax, block_amax16(r));
+  for (int b = t; b < nblk; b += 4 * kPrepThreads) {
+    uint4 u[4][2];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int bb = b + k * kPrepThreads;
+      const uint4* src = reinterpret_cast<const uint4*>(X + (long long)bb * 16);
+      u[k][0] = bb < nblk ? __ldg(src) : make_uint4(0u, 0u, 0u, 0u);
+      u[k][1] = bb < nblk ? __ldg(src + 1) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t w[8] = {u[k][0].x, u[k][0].y, u[k][0].z, u[k][0].w, u[k][1].x, u[k][1].y, u[k][1].z, u[k][1].w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        amax = fmaxf(amax, fmaxf(__uint_as_float((w[i] << 16) & 0x7FFFFFFFu), __uint_as_float(w[i] & 0x7FFF0000u)));
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
