@@ -93,6 +93,7 @@ constexpr int kMaxStages = 12;
 constexpr int kMaxB = 352;                         // B rows (tokens x terms) the TMEM budget allows
 constexpr size_t kTailBytes = 8192;
 constexpr int kMaxSfBufs = 8;
+constexpr int kFixupBatch = 12;                    // contributors whose partials a deferred sum loads at once
 
 // One GEMM of a launch. Lives in device memory (a pass) or in the kernel's parameter
 // space (a single GEMM); the tensor maps are read by TMA from wherever it lives.
@@ -1017,7 +1018,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (et == 0 && seg <= 2) MX_CTA(10 + 4 * (seg - 1));
       // The CTA's final segment of a GEMM with tile-pair units: every warp is free once the
       // role loops end, so the whole CTA sums the partials then (below), with a row's
-      // contributors 8 at a time in flight. (Measured on single GEMMs: M=17, tile pairs, a
+      // contributors 12 at a time in flight. (Measured on single GEMMs: M=17, tile pairs, a
       // chained 27B pass 7.1 -> 6.7 ms; one tile per unit (M=1, M=68) slightly slower, so
       // those keep the epilogue's own sum.)
       const bool defer = TPU == 2 && *s_last && !verify && done >= nunits;
@@ -1083,9 +1084,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
   }
-  if (s_def->on) {
+  if (TPU == 2 && s_def->on) {
     // The deferred sum of a split tile group, by all warps: one work item per (tile, row,
-    // 8 tokens), its contributors' partials loaded 8 CTAs at a time and added in CTA order,
+    // 8 tokens), its contributors' partials loaded 12 CTAs at a time and added in CTA order,
     // as the epilogue's own sum does (the same bits). The epilogue thread that took the last
     // ticket acquired the other CTAs' partials before the barrier above.
     const DeferredFixup d = *s_def;
@@ -1101,10 +1102,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       float acc[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-      for (int cc = d.c0; cc <= d.c1; cc += 8) {
-        float4 v[8][2];
+      for (int cc = d.c0; cc <= d.c1; cc += kFixupBatch) {
+        float4 v[kFixupBatch][2];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
+        for (int k = 0; k < kFixupBatch; ++k) {
           const int cx = cc + k;
           const bool on = cx <= d.c1;
           const int sl =
@@ -1116,7 +1117,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             v[k][b] = (on && mc + 4 * b < Mp) ? __ldcg(src + b) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
+        for (int k = 0; k < kFixupBatch; ++k) {
           if (cc + k <= d.c1) {
 #pragma unroll
             for (int b = 0; b < 2; ++b) {
