@@ -55,7 +55,7 @@ def _workers() -> int:
 
 
 def lmhead_oracle(x_bits: np.ndarray, N: int = S.VOCAB, K: int = S.LMHEAD_K) -> dict:
-    """The oracle's verdict on the seeded lm_head for the activation rows ``x_bits``.
+    """The oracle's result on the seeded lm_head for the activation rows ``x_bits``.
 
     Returns a dict with ``q`` uint8 [N, K/2], ``sf`` uint8 [N, K/16] and ``ts`` float32 (the
     oracle's packing of the weight), ``t`` int64 [M] (argmax, lowest index on ties),

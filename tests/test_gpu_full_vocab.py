@@ -53,7 +53,7 @@ def to_dev_bf16(x_bits: np.ndarray) -> torch.Tensor:
 @pytest.fixture(scope="module")
 def head(nv):
     """The 68 hidden rows (the first 17 are the one-sequence case, row 0 the M = 1 case),
-    the oracle's verdict over the whole head, and its packed bytes on the GPU."""
+    the oracle's argmax and logits over the whole head, and its packed bytes on the GPU."""
     x = S.lmhead_x(B=4)
     orc = FV.lmhead_oracle(x)
     dev = (torch.from_numpy(orc["q"]).cuda(), torch.from_numpy(orc["sf"]).cuda(),
