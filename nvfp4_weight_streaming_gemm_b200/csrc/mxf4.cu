@@ -47,11 +47,13 @@
 //                   from shared memory into TMEM in the layout the MMA reads (the 4
 //                   scales of row m0 + 32*j in column j of lane m0, replicated over the
 //                   four lane quarters), all of a chunk's shared loads first.
-//     warps 8-11    epilogue: tcgen05.ld of the accumulators; five terms are folded
-//                   into registers and the accumulator is released before any store,
-//                   one term is streamed 16 tokens at a time; then x ts and Y, the
-//                   per-tile argmax of a verify problem, or a split tile's partials,
-//                   which the last CTA to finish the tile sums in CTA order.
+//     warps 8-11    epilogue: tcgen05.ld of the accumulators; several terms (5, or 4 in
+//                   a pass that asks for them) are folded into registers and the
+//                   accumulator is released before any store, one term is streamed 16
+//                   tokens at a time; then x ts and Y, the per-tile argmax of a verify
+//                   problem, or a split tile's partials, which the last CTA to finish the
+//                   tile sums in CTA order (with tile-pair units, the CTA's final such sum
+//                   is done by all 12 warps once the role loops end).
 // Every wait is bounded (see sync.cuh); a timeout sets the device error word.
 #include "common.cuh"
 #include "kernels.h"
