@@ -1,0 +1,77 @@
+"""CPU: a float64 model of the block-scaled path's residual activation terms, which sets the
+GPU tests' accuracy bars for it (five terms: 1e-4 of a row's max|y|; four terms: 3e-4).
+
+The model follows the decomposition the kernels document (include/nvfp4ws.h, nvfp4_gemm_skinny):
+g_0 = amax|x| / 2688, g_t = g_0 / 4^t, r_0 = x, and per 16-element block and term
+S_t = E4M3(amax|r_t| / (6 g_t)), c_t = E2M1(r_t / (S_t g_t)), r_{t+1} = r_t - c_t S_t g_t, so that
+x = sum_t g_t S_t c_t + r_T. It is test infrastructure built on the oracle's format tables; it
+checks properties of the representation, not the kernels (the GPU tests compare those with the
+oracle's exact product).
+"""
+
+import numpy as np
+import pytest
+
+import synthetic as S
+from oracle import gemm as G
+from oracle import nvfp4 as F
+
+
+def decompose(x: np.ndarray, T: int):
+    """The T terms of each row of x (float64 [M, K]) and the residual left after them."""
+    M, K = x.shape
+    r = x.copy()
+    g0 = np.abs(r).max(axis=1) / 2688.0
+    g0 = np.where(g0 > 0, g0, 1.0)
+    terms, scales = [], []
+    for t in range(T):
+        g = g0 / 4.0 ** t
+        blk = r.reshape(M, K // 16, 16)
+        want = np.abs(blk).max(axis=2) / (6.0 * g[:, None])
+        Sb = F.E4M3_VALUES[F.e4m3_encode(want)]
+        den = (Sb * g[:, None])[:, :, None]
+        safe = np.where(den > 0, den, 1.0)
+        c = np.where(den > 0, F.E2M1_VALUES[F.e2m1_encode(blk / safe)], 0.0)
+        q = (c * den).reshape(M, K)
+        terms.append(q)
+        scales.append(want)
+        r = r - q
+    return terms, r, scales
+
+
+@pytest.fixture(scope="module")
+def case():
+    W, x_bits = S.random_case(4242, 17, 512, 5120)
+    q, sf, ts = F.quantize_nvfp4(W)
+    y = G.gemm_ref(x_bits, q, sf, ts)
+    return G.bf16_bits_to_float64(x_bits), F.dequantize_nvfp4(q, sf, ts), y
+
+
+@pytest.mark.parametrize("T", [4, 5])
+def test_terms_sum_back_and_scales_fit(case, T):
+    x, _, _ = case
+    terms, r, scales = decompose(x, T)
+    assert np.array_equal(sum(terms) + r, x) or np.abs(sum(terms) + r - x).max() <= 1e-12 * np.abs(x).max()
+    for want in scales:                                  # every block scale fits E4M3 unsaturated
+        assert want.max() <= 448.0 * (1 + 2 ** -20)
+    # each term leaves at most a fraction of the previous residual's block magnitude
+    resid = [np.abs(x - sum(terms[:t + 1])).max() for t in range(T)]
+    assert all(b <= 0.2 * a for a, b in zip(resid, resid[1:]))
+
+
+@pytest.mark.parametrize("T,bar", [(5, 1e-4), (4, 3e-4)])
+def test_gemm_error_inside_the_gpu_bars(case, T, bar):
+    x, Wd, y = case
+    terms, _, _ = decompose(x, T)
+    ya = sum(terms) @ Wd.T
+    rel = (np.abs(ya - y).max(axis=1) / np.abs(y).max(axis=1)).max()
+    assert rel <= bar / 3, f"{T} terms: {rel:.2e} of max|y| against a bar of {bar}"
+    assert rel <= 2e-3                                   # the task's per-row bar
+
+
+def test_three_terms_would_not_keep_the_margin(case):
+    """The reason for five (or, opt-in, four): three terms come within 2x of the task's bar."""
+    x, Wd, y = case
+    terms, _, _ = decompose(x, 3)
+    rel = (np.abs(sum(terms) @ Wd.T - y).max(axis=1) / np.abs(y).max(axis=1)).max()
+    assert rel > 2e-4
