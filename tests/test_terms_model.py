@@ -75,3 +75,26 @@ def test_three_terms_would_not_keep_the_margin(case):
     terms, _, _ = decompose(x, 3)
     rel = (np.abs(sum(terms) @ Wd.T - y).max(axis=1) / np.abs(y).max(axis=1)).max()
     assert rel > 2e-4
+
+
+def test_fp8_two_e4m3_terms_are_exact_above_the_subnormal_step():
+    """The FP8 term kernel's activations: per row g = 2^(e-8) with amax|x| in [2^(e-1), 2^e),
+    term 0 = E4M3(x/g), term 1 = E4M3(16 (x/g - term 0)). bf16's 8 significant bits fit two
+    4-bit E4M3 mantissas, so the pair is exact wherever |x/g| >= 2^-6, and below that the
+    residual stays under E4M3's subnormal step in term 1's units (2^-14 g). So the FP8 GPU
+    tests' 2e-4 bar measures the FP8 tensor core's accumulation, not the terms."""
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((64, 4096)).astype(np.float32)
+    x[1] *= 1e-3
+    x[1, 7] = 300.0                                      # an outlier over small values
+    x[2] *= 2.0 ** 20                                    # far above f16's range
+    xf = G.bf16_bits_to_float64(S.f32_to_bf16_bits(x))
+    e = np.floor(np.log2(np.abs(xf).max(axis=1))) + 1
+    g = 2.0 ** (e - 8)
+    u = xf / g[:, None]
+    assert np.abs(u).max() < 256.0
+    c0 = F.E4M3_VALUES[F.e4m3_encode(u)]
+    c1 = F.E4M3_VALUES[F.e4m3_encode(16.0 * (u - c0))]
+    res = np.abs(u - (c0 + c1 / 16.0))
+    assert (res[np.abs(u) >= 2.0 ** -6] == 0).all()
+    assert res.max() <= 2.0 ** -14
